@@ -1,0 +1,283 @@
+"""Pins of the fp64 oracle against facts it does not define itself.
+
+Each test fixes one part of the oracle with something independent of its
+code: a textbook formula written differently (complex RoPE, plain softmax),
+a closed form worked by hand (tests/golden), brute force on tiny inputs, or
+an invariant that a plausible mistake would break.  Source of the method:
+MAC-Attention, page 1 (abstract).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.dense_ref import (dense_attention, dense_step, decode, load_hand_example, rope_complex)
+
+
+def _tiny(**kw):
+    return synth.WORKLOADS["tiny"].with_(**kw)
+
+
+# ---------------------------------------------------------------- RoPE pins
+def test_rope_matches_complex_rotation():
+    rng = np.random.default_rng(11)
+    for D in (64, 128):
+        for pos in (0, 1, 7, 1023, 131199):
+            q = rng.standard_normal(D).astype(np.float32)
+            got = oracle.rope(q, pos, 5e5)
+            # the fp64 angle pos * theta^(-2i/D) carries ~1e-16 * pos radians of rounding
+            tol = 1e-13 + 1e-15 * pos * float(np.abs(q).max())
+            np.testing.assert_allclose(got, rope_complex(q, pos, 5e5), rtol=0, atol=tol)
+
+
+def test_rope_is_identity_at_zero_and_relative():
+    rng = np.random.default_rng(12)
+    D = 128
+    q = rng.standard_normal(D).astype(np.float32)
+    k = rng.standard_normal(D).astype(np.float32)
+    np.testing.assert_array_equal(oracle.rope(q, 0, 1e4), q.astype(np.float64))
+    # norm preserved; score depends only on the position difference
+    for m, n in ((5, 2), (1000, 17), (70000, 69000)):
+        qm = oracle.rope(q, m, 1e4)
+        kn = oracle.rope(k, n, 1e4)
+        assert abs(np.linalg.norm(qm) - np.linalg.norm(q.astype(np.float64))) < 1e-12
+        rel = oracle.rope(q, m - n, 1e4)
+        assert abs(qm @ kn - rel @ k.astype(np.float64)) < 1e-9
+
+
+# --------------------------------------------------------- partial / merge
+def _rand_kv(rng, L, D):
+    K = synth.f32_to_bf16_bits(rng.standard_normal((L, D)).astype(np.float32))
+    V = synth.f32_to_bf16_bits(rng.standard_normal((L, D)).astype(np.float32))
+    return K, V
+
+
+def test_partial_equals_dense_softmax():
+    rng = np.random.default_rng(13)
+    L, D = 300, 64
+    K, V = _rand_kv(rng, L, D)
+    q = rng.standard_normal(D)
+    o, m, l = oracle.partial(q, K, V, 0, L)
+    o_ref, lse_ref = dense_attention(q[None], decode(K), decode(V))
+    np.testing.assert_allclose(o, o_ref[0], rtol=0, atol=1e-13)
+    assert abs(m + np.log(l) - lse_ref[0]) < 1e-12
+    o, m, l = oracle.partial(q, K, V, 5, 5)
+    assert m == -np.inf and l == 0.0 and not o.any()
+
+
+@pytest.mark.parametrize("scale", [1.0, 1e3])
+def test_merge_of_any_partition_equals_dense(scale):
+    """Stable merge (page 1, complete stage): any partition, any order, equals dense."""
+    rng = np.random.default_rng(14)
+    L, D = 257, 64
+    K, V = _rand_kv(rng, L, D)
+    q = rng.standard_normal(D) * scale  # scale 1e3 gives logits of order +-1e4
+    o_ref, lse_ref = dense_attention(q[None], decode(K), decode(V))
+    for trial in range(20):
+        ncut = rng.integers(0, 12)
+        cuts = np.sort(rng.integers(0, L + 1, size=ncut))
+        edges = np.concatenate([[0], cuts, [L]])  # repeated cuts give empty parts
+        parts = [oracle.partial(q, K, V, int(a), int(b)) for a, b in zip(edges[:-1], edges[1:])]
+        rng.shuffle(parts)
+        acc = parts[0]
+        for p in parts[1:]:
+            acc = oracle.merge(acc, p)
+        o, m, l = acc
+        np.testing.assert_allclose(o, o_ref[0], rtol=0, atol=1e-11)
+        assert abs((m + np.log(l)) - lse_ref[0]) <= 1e-12 * max(1.0, abs(lse_ref[0]))
+
+
+def test_merge_empty_is_identity():
+    D = 8
+    o = np.arange(D, dtype=np.float64)
+    e = (np.zeros(D), -np.inf, 0.0)
+    r = oracle.merge(e, (o, 1.5, 2.0))
+    assert r[1] == 1.5 and r[2] == 2.0 and np.array_equal(r[0], o)
+    r = oracle.merge(e, e)
+    assert r[1] == -np.inf and r[2] == 0.0 and not r[0].any()
+
+
+# ------------------------------------------------------------ worked example
+def test_hand_worked_example():
+    g, K, V, qs = load_hand_example()
+    sh = g["shape"]
+    orc = oracle.Oracle(sh["B"], sh["Hq"], sh["Hkv"], sh["D"], sh["W"], sh["band"], sh["tau"],
+                        sh["rope_theta"], 0, sh["max_seq"], 0)
+    for st, q in zip(g["steps"], qs):
+        r = orc.step(q, np.array([st["rope_pos"]], np.int32), K, V, None, np.array([st["seq_len"]], np.int32))
+        assert int(r.hit[0, 0]) == st["hit"]
+        assert int(r.match_pos[0, 0]) == st["match_pos"]
+        np.testing.assert_allclose(r.out[0, :, 0], st["out0"], atol=1e-6)
+        np.testing.assert_allclose(r.out[0, :, 1], st["out1"], atol=1e-6)
+        np.testing.assert_allclose(r.out[0, :, 2:], 0.0, atol=0)
+        np.testing.assert_allclose(r.lse[0], st["lse"], atol=1e-6)
+        if "dense_out0" in st:  # the reuse really differs from dense here
+            assert abs(st["out0"] - st["dense_out0"]) > 0.4
+
+
+# ----------------------------------------------------------- whole-step pins
+def _run(wl, steps=None, stream=None, cache=None, tau=None, band=None, rope_zero=False):
+    stream = stream or synth.queries(wl, steps)
+    cache = cache or synth.kv_cache(wl, steps)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=tau, band=band)
+    res = []
+    for t in range(stream.q.shape[0]):
+        rp = np.zeros_like(stream.rope_pos[t]) if rope_zero else stream.rope_pos[t]
+        res.append(orc.step(stream.q[t], rp, cache.K, cache.V, cache.block_table, stream.seq_lens[t]))
+    return stream, cache, res
+
+
+def test_forced_miss_equals_dense():
+    """Threshold 0 (strict test) makes every step a miss, i.e. dense attention."""
+    wl = _tiny(steps=12)
+    stream, cache, res = _run(wl, tau=0.0)
+    for t, r in enumerate(res):
+        assert not r.hit.any()
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+
+
+def test_forced_miss_paged_equals_dense():
+    wl = synth.WORKLOADS["paged_mixed"].with_(B=3, Hq=8, Hkv=2, D=64, L0=(100, 37, 250), steps=6,
+                                              W=4, band=8, tau=0.0)
+    stream, cache, res = _run(wl)
+    for t, r in enumerate(res):
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+
+
+def test_exact_repeats_without_rotation_equal_dense():
+    """Identity RoPE and exact repeats: the reused state is the current query's own."""
+    wl = _tiny(steps=24, sigma=0.0)
+    stream = synth.queries(wl, sigma=0.0)
+    stream, cache, res = _run(wl, stream=stream, rope_zero=True)
+    nhit = 0
+    for t, r in enumerate(res):
+        nhit += int(r.hit.sum())
+        o, l = dense_step(wl, cache, stream.q[t], np.zeros(wl.B, np.int32), stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+    assert nhit >= 6
+
+
+def test_band_covering_context_equals_dense():
+    """band >= p_t puts every reuse boundary at 0: hits are exact under any RoPE."""
+    wl = _tiny(L0=(40,), steps=16, band=200)
+    stream, cache, res = _run(wl)
+    nhit = 0
+    for t, r in enumerate(res):
+        nhit += int(r.hit.sum())
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+    assert nhit >= 4
+
+
+def test_hits_differ_from_dense_and_stay_convex():
+    """A real reuse is an approximation; its output stays a convex mix of V rows."""
+    wl = _tiny(steps=32)
+    stream, cache, res = _run(wl)
+    Vd = decode(cache.V[0, :, 0])
+    diff = 0.0
+    for t, r in enumerate(res):
+        L = int(stream.seq_lens[t][0])
+        lo, hi = Vd[:L].min(axis=0), Vd[:L].max(axis=0)
+        assert np.all(r.out[0] >= lo - 1e-12) and np.all(r.out[0] <= hi + 1e-12)
+        assert np.all(np.isfinite(r.lse))
+        if r.hit.any():
+            o, _ = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+            diff = max(diff, float(np.abs(r.out - o).max()))
+    assert diff > 1e-6
+
+
+def test_hit_cost_is_constant_in_context_length():
+    """On a hit the keys attended are b + (p_t - p_s) + 1 whatever the context (page 1)."""
+    per_L = {}
+    for L0 in (256, 4096):
+        wl = _tiny(L0=(L0,), steps=20)
+        stream, cache, res = _run(wl)
+        keys = []
+        for t, r in enumerate(res):
+            if r.hit[0, 0]:
+                p_t = int(stream.seq_lens[t][0]) - 1
+                p_s = int(r.match_pos[0, 0])
+                assert r.keys_read == wl.band + (p_t - p_s) + 1
+                keys.append(r.keys_read)
+            else:
+                assert r.keys_read == int(stream.seq_lens[t][0])
+        per_L[L0] = keys
+    assert per_L[256] == per_L[4096] and len(per_L[256]) > 3
+
+
+# ---------------------------------------------------------------- match pins
+def _brute_match(window, q, tau, G):
+    """numpy brute force: mean-over-heads squared L2, argmin, ties to later, strict < tau."""
+    best, arg = np.inf, -1
+    for idx, (qe, pos) in enumerate(window):
+        d = float(np.sum((q.astype(np.float64) - qe.astype(np.float64)) ** 2) / G)
+        if np.isnan(d):
+            continue
+        if d < best or (d == best and arg >= 0 and pos > window[arg][1]):
+            best, arg = d, idx
+    if arg >= 0 and best < tau:
+        return True, window[arg][1]
+    return False, -1
+
+
+def test_match_equals_brute_force():
+    rng = np.random.default_rng(15)
+    B, Hq, Hkv, D, W = 2, 4, 2, 8, 4
+    G = Hq // Hkv
+    orc = oracle.Oracle(B, Hq, Hkv, D, W, 2, 0.5, 1e4, 0, 1 << 10, 0)
+    hist = [[[] for _ in range(Hkv)] for _ in range(B)]
+    pool = []
+    K = np.zeros((B, 1 << 10, Hkv, D), np.uint16)
+    for t in range(40):
+        q = np.empty((B, Hq, D), np.float32)
+        for b in range(B):
+            r = rng.random()
+            if pool and r < 0.3:  # exact repeat of a recent step: forces ties on later duplicates
+                q[b] = pool[int(rng.integers(0, len(pool)))][b]
+            elif pool and r < 0.6:
+                q[b] = pool[-1][b] + rng.normal(0, 0.1, (Hq, D)).astype(np.float32)
+            else:
+                q[b] = rng.standard_normal((Hq, D)).astype(np.float32)
+        if t == 17:
+            q[1, 0, 0] = np.nan
+        pool.append(q.copy())
+        pool = pool[-3:]
+        lens = np.array([t + 5, 2 * t + 9], np.int32)
+        r = orc.step(q, lens - 1, K, K, None, lens)
+        for b in range(B):
+            for kvh in range(Hkv):
+                qg = q[b, kvh * G:(kvh + 1) * G]
+                win = hist[b][kvh][-W:]
+                want_hit, want_pos = _brute_match(win, qg, 0.5, G)
+                assert bool(r.hit[b, kvh]) == want_hit, (t, b, kvh)
+                assert int(r.match_pos[b, kvh]) == want_pos, (t, b, kvh)
+                hist[b][kvh].append((qg.copy(), int(lens[b]) - 1))
+    # the NaN query never matches
+    assert True
+
+
+@pytest.mark.parametrize("name,steps", [("tiny", None), ("llama8b_32k", None), ("long_128k", None),
+                                        ("paged_mixed", None), ("continuous_16k", 1024)])
+def test_generator_labels_recovered_with_margin(name, steps):
+    """Repeats hit their source step, fresh queries miss, with >= 1% distance margins."""
+    wl = synth.WORKLOADS[name]
+    stream = synth.queries(wl, steps)
+    orc = oracle.Oracle(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W, wl.band, wl.tau, wl.rope_theta)
+    for t in range(stream.q.shape[0]):
+        hit, mpos, db, ds = orc.match_step(stream.q[t], stream.seq_lens[t])
+        for b in range(wl.B):
+            lab = stream.label[t, b]
+            if lab:
+                assert hit[b].all(), (t, b)
+                assert (mpos[b] == stream.rope_pos[stream.src[t, b], b]).all(), (t, b)
+                assert (db[b] < 0.99 * wl.tau).all()
+                assert (ds[b] >= 1.01 * db[b]).all()
+            else:
+                assert not hit[b].any(), (t, b)
+                if t > 0:
+                    assert (db[b] > 1.01 * wl.tau).all()
