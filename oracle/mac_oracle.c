@@ -235,7 +235,7 @@ int oracle_window(const ostate_t *s, int u, float *q, double *o, double *m, doub
  * [mean-dist] dist = (1/G) sum_h sum_i (q[h][i] - q_e[h][i])^2.
  * [window] only entries whose position precedes p_t are candidates.
  * [strict] returns the index of the smallest distance, ties to the larger
- * position; *best/*second receive the two smallest distances (+inf if absent). */
+ * position, then to the more recent entry; *best/*second receive the two smallest distances (+inf if absent). */
 static int match_unit(const ostate_t *s, int u, const float *qg, int p_t, double *best, double *second) {
     int G = s->G, D = s->c.D, W = s->c.W > 0 ? s->c.W : 1;
     int n = s->n[u];
@@ -253,7 +253,9 @@ static int match_unit(const ostate_t *s, int u, const float *qg, int p_t, double
             }
         double dist = acc / (double)G;
         if (isnan(dist)) continue;
-        if (dist < b1 || (dist == b1 && arg >= 0 && pos > s->wpos[(size_t)u * W + arg])) {
+        /* entries run oldest to newest, so on an exact tie of distance and
+         * position the later (more recent) entry wins */
+        if (dist < b1 || (dist == b1 && arg >= 0 && pos >= s->wpos[(size_t)u * W + arg])) {
             b2 = b1;
             b1 = dist;
             arg = e;

@@ -218,7 +218,7 @@ def _brute_match(window, q, tau, G):
         d = float(np.sum((q.astype(np.float64) - qe.astype(np.float64)) ** 2) / G)
         if np.isnan(d):
             continue
-        if d < best or (d == best and arg >= 0 and pos > window[arg][1]):
+        if d < best or (d == best and arg >= 0 and pos >= window[arg][1]):
             best, arg = d, idx
     if arg >= 0 and best < tau:
         return True, window[arg][1]
