@@ -1,0 +1,189 @@
+/*
+ * mac.h -- C ABI of the MAC-Attention decode step on NVIDIA B200 (sm_100a).
+ *
+ * MAC-Attention ("MAC-Attention: a Match-Amend-Complete Scheme for Fast and
+ * Accurate Attention Computation", page 1, abstract) speeds up long-context
+ * decoding by reusing attention already computed for a recent, similar query:
+ *   Match    -- the current pre-RoPE query is compared by L2 distance with a
+ *               short window of recent queries;
+ *   Amend    -- on a hit, the keys of a small band before the matched
+ *               query's position are recomputed with the current query;
+ *   Complete -- fresh attention over the KV tail is merged with the reused,
+ *               amended state by a numerically stable log-sum-exp merge.
+ * On a miss the step is ordinary split-KV decode attention over every key.
+ * On a hit the work does not grow with the context length.
+ *
+ * Conventions used by every entry point
+ *   - Group: each KV head serves G = num_q_heads / num_kv_heads query heads
+ *     (GQA, page 1 "composes with ... MQA/GQA"); this build requires G = 4.
+ *     One match decision is taken per (sequence, KV head) over its G heads.
+ *   - Distance: mean over the G heads of the squared L2 distance between the
+ *     pre-RoPE queries.  Hit iff the smallest distance over the window is
+ *     strictly below tau; ties go to the more recent entry; NaN never hits.
+ *     Only entries whose position precedes the current one are candidates.
+ *   - Window: the W most recent previous decode steps of the same sequence
+ *     (per KV head).  The first step after init or reset always misses.
+ *   - Cut: every step stores (pre-RoPE query, prefix state over keys
+ *     [0, c_t), position p_t) with c_t = max(0, p_t - band).  A hit on an
+ *     entry at position p_s reuses its prefix state over [0, c_s),
+ *     c_s = max(0, p_s - band), recomputes [c_s, c_t) (amend) and [c_t, p_t]
+ *     (complete) with the current query.  A miss computes [0, c_t) and
+ *     [c_t, p_t].
+ *   - RoPE: K in the cache is post-RoPE.  The library rotates q_pre to
+ *     rope_pos with rotate-half pairs (i, i + D/2), inv_freq_i =
+ *     rope_theta^(-2i/D), angles in fp64.  Scores are q.k / sqrt(D).
+ *   - Positions: step attends keys [0, seq_lens[b] - 1]; p_t = seq_lens[b]-1.
+ *     The step's own K/V row must already be in the cache (see
+ *     mac_append_kv).
+ *   - Memory: every tensor argument is caller-owned.  "device" pointers are
+ *     CUDA device memory of the device that was current at mac_init_state;
+ *     "host" pointers are host memory (pinned for overlap, pageable works).
+ *     The library owns only its MacState (ring buffers and scratch).
+ *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).
+ *     Device entry points only enqueue work and never synchronise; calls on
+ *     one MacState must be ordered on one stream.
+ *   - Errors: every int-returning function returns MAC_OK or a MAC_ERR_*
+ *     code; host-side validation failures enqueue nothing.  Faults found on
+ *     the device (bad sequence length, bad page id, a wait that timed out)
+ *     set bits of a device status word, write NaN to the affected unit's out
+ *     and lse and leave its window unchanged; mac_get_status reads them.
+ */
+#ifndef MAC_B200_H
+#define MAC_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    MAC_OK = 0,
+    MAC_ERR_ARG = 1,    /* NULL where a pointer is required, misaligned pointer, value out of range */
+    MAC_ERR_SHAPE = 2,  /* unsupported head_dim / group size / page size / window */
+    MAC_ERR_CUDA = 3,   /* a CUDA runtime or driver call failed */
+    MAC_ERR_OOM = 4,    /* device allocation failed */
+    MAC_ERR_DEVICE = 5  /* the device status word is non-zero (see mac_get_status) */
+};
+
+/* Bits of the device status word. */
+#define MAC_DEV_BAD_SEQ_LEN 1u /* seq_lens[b] < 1 or beyond the cache capacity */
+#define MAC_DEV_BAD_PAGE 2u    /* a block-table entry needed by the step is outside [0, num_pages) */
+#define MAC_DEV_TIMEOUT 4u     /* a bounded wait inside a kernel gave up; outputs of that launch are invalid */
+
+typedef struct MacConfig {
+    int batch;             /* B >= 1 */
+    int num_q_heads;       /* Hq */
+    int num_kv_heads;      /* Hkv; Hq / Hkv must be 4 */
+    int head_dim;          /* D: 64 or 128 */
+    int window;            /* W: entries kept per (sequence, KV head), 1..256 */
+    int band;              /* b >= 0: keys before the match position that are recomputed */
+    float tau;             /* match threshold on the mean squared L2 distance (strict <); 0 = never hit */
+    double rope_theta;     /* RoPE base (> 0) */
+    int page_size;         /* 0: contiguous K/V [B][max_seq][Hkv][D]; else tokens per page, a multiple of 16 */
+    int max_seq;           /* contiguous: rows per sequence in K/V (capacity); paged: unused */
+    int max_pages_per_seq; /* paged: row length of block_table; capacity = max_pages_per_seq * page_size */
+    int num_pages;         /* paged: pages P in the K/V pools [P][page_size][Hkv][D] */
+} MacConfig;
+
+typedef struct MacState MacState; /* opaque; owns device memory on the device current at init */
+
+/* Allocate the ring buffers (queries, (o, m, l) states, positions, step
+ * counters) and the scratch of one layer, on the current device.  Every
+ * sequence starts with an empty window.  *out receives the new state.
+ * Returns MAC_ERR_SHAPE for unsupported shapes, MAC_ERR_OOM / MAC_ERR_CUDA
+ * when allocation fails (nothing is leaked).  Synchronous. */
+int mac_init_state(const MacConfig *cfg, MacState **out);
+
+/* Release every device buffer of the state.  Waits for the device. */
+void mac_destroy(MacState *st);
+
+/* Empty the window of sequence b (all its KV heads): its next step misses.
+ * Enqueued on stream. */
+int mac_reset_seq(MacState *st, int b, void *stream);
+
+/* One MAC decode step of every sequence and KV head (page 1: match, then
+ * amend and complete on a hit, split-KV attention on a miss, stable merge).
+ *   q_pre       device fp32 [B][Hq][D], pre-RoPE queries, 16-byte aligned.
+ *   rope_pos    device int32 [B], position used to rotate the queries.
+ *   K, V        device bf16 bit patterns (uint16), 16-byte aligned:
+ *               contiguous [B][max_seq][Hkv][D] or paged [P][page_size][Hkv][D].
+ *   block_table device int32 [B][max_pages_per_seq] (paged), NULL if contiguous.
+ *   seq_lens    device int32 [B], keys visible at this step (p_t = seq_lens - 1).
+ *   out         device fp32 [B][Hq][D], attention output.
+ *   lse         device fp32 [B][Hq], natural-log log-sum-exp of the scores
+ *               the output combines (reused and fresh).
+ *   hit_mask    device uint8 [B][Hkv], 1 where the match hit; may be NULL.
+ *   match_pos   device int32 [B][Hkv], position of the matched entry or -1;
+ *               may be NULL.
+ * The window of every unit advances by one entry.  Enqueues two kernels. */
+int mac_decode_step(MacState *st, const float *q_pre, const int *rope_pos, const uint16_t *K,
+                    const uint16_t *V, const int *block_table, const int *seq_lens, float *out,
+                    float *lse, uint8_t *hit_mask, int *match_pos, void *stream);
+
+/* The two halves of mac_decode_step, for callers that time or overlap them.
+ * mac_match runs the match stage, rotates the queries, writes hit_mask /
+ * match_pos, records the step's query in the window and plans the key
+ * ranges; mac_attend runs amend, complete (or the miss path) and the merge
+ * using the plan of the preceding mac_match on the same state.  Arguments as
+ * in mac_decode_step; mac_match writes NaN to out/lse of invalid units. */
+int mac_match(MacState *st, const float *q_pre, const int *rope_pos, const int *block_table,
+              const int *seq_lens, float *out, float *lse, uint8_t *hit_mask, int *match_pos,
+              void *stream);
+int mac_attend(MacState *st, const uint16_t *K, const uint16_t *V, const int *block_table,
+               float *out, float *lse, void *stream);
+
+/* Write the step's own K/V rows into the cache at position seq_lens[b] - 1
+ * of every sequence (paged-KV manager composition, page 1).
+ *   K, V        device bf16 cache, layout as in mac_decode_step (written).
+ *   block_table device int32 (paged) or NULL.
+ *   seq_lens    device int32 [B].
+ *   k_new, v_new device bf16 [B][Hkv][D].
+ * Rows whose position or page id is invalid are skipped and flagged in the
+ * status word. */
+int mac_append_kv(MacState *st, uint16_t *K, uint16_t *V, const int *block_table,
+                  const int *seq_lens, const uint16_t *k_new, const uint16_t *v_new, void *stream);
+
+/* mac_append_kv (when k_new_h is not NULL) and mac_decode_step with the
+ * per-step inputs and outputs in HOST memory: copies q_pre_h, rope_pos_h,
+ * seq_lens_h and the new rows to library staging buffers, runs the step,
+ * copies out_h, lse_h, hit_h and match_pos_h back (any of the four may be
+ * NULL) and synchronises the stream before returning.  K, V, block_table
+ * stay device-resident (the cache is state, not a per-step input).  Returns
+ * MAC_ERR_DEVICE if the device status word is non-zero after the step. */
+int mac_decode_step_host(MacState *st, const float *q_pre_h, const int *rope_pos_h,
+                         const int *seq_lens_h, const uint16_t *k_new_h, const uint16_t *v_new_h,
+                         uint16_t *K, uint16_t *V, const int *block_table, float *out_h,
+                         float *lse_h, uint8_t *hit_h, int *match_pos_h, void *stream);
+
+/* Synchronise the device, copy the status word to *device_status (may be
+ * NULL) and clear it.  Returns MAC_ERR_DEVICE if it was non-zero. */
+int mac_get_status(MacState *st, int *device_status);
+
+/* Ring state export/import (checkpoint / resume).  The byte layout is:
+ * int32 header[8] = {magic 0x4D414331, B*Hkv, W+1, G, D, 0, 0, 0}, then
+ * fp32 q[U][W+1][G][D], fp32 o[U][W+1][G][D] (normalised output of each
+ * stored prefix state), fp32 m[U][W+1][G] (max score, natural-log units),
+ * fp32 l[U][W+1][G] (sum of exp(score - m)), int32 pos[U][W+1],
+ * int32 steps[U] (decode steps since reset; entry of step n sits in slot
+ * n mod (W+1)).  Both calls synchronise the device.  host_buf must hold
+ * mac_state_bytes(st) bytes. */
+size_t mac_state_bytes(const MacState *st);
+int mac_export_state(const MacState *st, void *host_buf, size_t bytes);
+int mac_import_state(MacState *st, const void *host_buf, size_t bytes);
+
+/* Tuning: minimum keys one CTA of the attention kernel takes (default 128).
+ * Smaller values spread short (hit) steps over more SMs. */
+int mac_set_min_keys_per_cta(MacState *st, int keys);
+
+/* Persistent grid size of the attention kernel (CTAs). */
+int mac_attend_grid(const MacState *st);
+
+/* Static description of a return code. */
+const char *mac_error_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MAC_B200_H */

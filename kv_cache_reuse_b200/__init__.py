@@ -1,0 +1,219 @@
+"""MAC-Attention decode step on B200: Python binding of libmac_b200.so.
+
+Argument marshalling only -- every stage of the step (match, RoPE, amend,
+complete, miss fallback, merge, ring update) runs in the library's CUDA
+kernels.  Tensors are torch tensors on the state's device (PyTorch is used for
+device memory and streams); the functions carry the names of the C ABI in
+include/mac.h and forward to it.  There is no CPU fallback: if the library is
+missing, importing the native module raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from typing import Optional
+
+from ._native import (MAC_DEV_BAD_PAGE, MAC_DEV_BAD_SEQ_LEN, MAC_DEV_TIMEOUT, MAC_ERR_ARG, MAC_ERR_CUDA,
+                      MAC_ERR_DEVICE, MAC_ERR_OOM, MAC_ERR_SHAPE, MAC_OK, LIB_PATH, MacConfig, MacError, check,
+                      load)
+
+__all__ = [
+    "MacConfig", "MacError", "MacState", "mac_init_state", "mac_destroy", "mac_reset_seq", "mac_decode_step",
+    "mac_match", "mac_attend", "mac_append_kv", "mac_decode_step_host", "mac_get_status", "mac_state_bytes",
+    "mac_export_state", "mac_import_state", "mac_set_min_keys_per_cta", "mac_attend_grid", "mac_error_string",
+    "MAC_OK", "MAC_ERR_ARG", "MAC_ERR_SHAPE", "MAC_ERR_CUDA", "MAC_ERR_OOM", "MAC_ERR_DEVICE",
+    "MAC_DEV_BAD_SEQ_LEN", "MAC_DEV_BAD_PAGE", "MAC_DEV_TIMEOUT", "LIB_PATH",
+]
+
+
+def _ptr(t) -> Optional[int]:
+    """Device (or host) address of a tensor / numpy array / int, None for None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        if not t.is_contiguous():
+            raise ValueError("tensor arguments must be contiguous")
+        return t.data_ptr()
+    if hasattr(t, "ctypes"):
+        return t.ctypes.data
+    raise TypeError("unsupported argument type %r" % type(t))
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class MacState:
+    """Owns one C MacState (ring buffers + scratch of one attention layer)."""
+
+    def __init__(self, batch, num_q_heads, num_kv_heads, head_dim, window, band, tau, rope_theta,
+                 page_size=0, max_seq=0, max_pages_per_seq=0, num_pages=0):
+        self.cfg = MacConfig(batch, num_q_heads, num_kv_heads, head_dim, window, band, float(tau),
+                             float(rope_theta), page_size, max_seq, max_pages_per_seq, num_pages)
+        self.lib = load()
+        h = C.c_void_p()
+        check("mac_init_state", self.lib.mac_init_state(C.byref(self.cfg), C.byref(h)))
+        self.handle = h
+
+    @classmethod
+    def for_workload(cls, wl, capacity=None, max_pages_per_seq=0, num_pages=0, tau=None, band=None, window=None):
+        """State sized for a synth.Workload (contiguous capacity or paged pool)."""
+        return cls(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W if window is None else window,
+                   wl.band if band is None else band, wl.tau if tau is None else tau, wl.rope_theta,
+                   wl.page_size, capacity or 0, max_pages_per_seq, num_pages)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            self.lib.mac_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # --- thin forwards -------------------------------------------------
+    def decode_step(self, q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
+                    stream=None):
+        return mac_decode_step(self, q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, hit_mask, match_pos,
+                               stream)
+
+    def match(self, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None, stream=None):
+        return mac_match(self, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream)
+
+    def attend(self, K, V, block_table, out, lse, stream=None):
+        return mac_attend(self, K, V, block_table, out, lse, stream)
+
+    def append_kv(self, K, V, block_table, seq_lens, k_new, v_new, stream=None):
+        return mac_append_kv(self, K, V, block_table, seq_lens, k_new, v_new, stream)
+
+    def reset_seq(self, b, stream=None):
+        return mac_reset_seq(self, b, stream)
+
+    def get_status(self) -> int:
+        return mac_get_status(self)
+
+    def export_state(self):
+        return mac_export_state(self)
+
+    def import_state(self, buf):
+        return mac_import_state(self, buf)
+
+
+def mac_init_state(cfg: MacConfig) -> C.c_void_p:
+    h = C.c_void_p()
+    check("mac_init_state", load().mac_init_state(C.byref(cfg), C.byref(h)))
+    return h
+
+
+def _h(st):
+    return st.handle if isinstance(st, MacState) else st
+
+
+def mac_destroy(st) -> None:
+    if isinstance(st, MacState):
+        st.close()
+    else:
+        load().mac_destroy(st)
+
+
+def mac_reset_seq(st, b: int, stream=None) -> None:
+    check("mac_reset_seq", load().mac_reset_seq(_h(st), int(b), _stream(stream)))
+
+
+def mac_decode_step(st, q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
+                    stream=None) -> None:
+    check("mac_decode_step", load().mac_decode_step(
+        _h(st), _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens), _ptr(out),
+        _ptr(lse), _ptr(hit_mask), _ptr(match_pos), _stream(stream)))
+
+
+def mac_match(st, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
+              stream=None) -> None:
+    check("mac_match", load().mac_match(
+        _h(st), _ptr(q_pre), _ptr(rope_pos), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
+        _ptr(hit_mask), _ptr(match_pos), _stream(stream)))
+
+
+def mac_attend(st, K, V, block_table, out, lse, stream=None) -> None:
+    check("mac_attend", load().mac_attend(_h(st), _ptr(K), _ptr(V), _ptr(block_table), _ptr(out), _ptr(lse),
+                                          _stream(stream)))
+
+
+def mac_append_kv(st, K, V, block_table, seq_lens, k_new, v_new, stream=None) -> None:
+    check("mac_append_kv", load().mac_append_kv(_h(st), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens),
+                                                _ptr(k_new), _ptr(v_new), _stream(stream)))
+
+
+def mac_decode_step_host(st, q_pre_h, rope_pos_h, seq_lens_h, k_new_h, v_new_h, K, V, block_table, out_h, lse_h,
+                         hit_h=None, match_pos_h=None, stream=None) -> int:
+    """Host-buffer step; returns MAC_OK or MAC_ERR_DEVICE (status word set)."""
+    rc = load().mac_decode_step_host(
+        _h(st), _ptr(q_pre_h), _ptr(rope_pos_h), _ptr(seq_lens_h), _ptr(k_new_h), _ptr(v_new_h), _ptr(K), _ptr(V),
+        _ptr(block_table), _ptr(out_h), _ptr(lse_h), _ptr(hit_h), _ptr(match_pos_h), _stream(stream))
+    if rc not in (MAC_OK, MAC_ERR_DEVICE):
+        check("mac_decode_step_host", rc)
+    return rc
+
+
+def mac_get_status(st) -> int:
+    v = C.c_int(0)
+    rc = load().mac_get_status(_h(st), C.byref(v))
+    if rc not in (MAC_OK, MAC_ERR_DEVICE):
+        check("mac_get_status", rc)
+    return v.value
+
+
+def mac_state_bytes(st) -> int:
+    return int(load().mac_state_bytes(_h(st)))
+
+
+def mac_export_state(st):
+    import numpy as np
+    buf = np.empty(mac_state_bytes(st), np.uint8)
+    check("mac_export_state", load().mac_export_state(_h(st), buf.ctypes.data, buf.nbytes))
+    return buf
+
+
+def mac_import_state(st, buf) -> None:
+    import numpy as np
+    buf = np.ascontiguousarray(buf, np.uint8)
+    check("mac_import_state", load().mac_import_state(_h(st), buf.ctypes.data, buf.nbytes))
+
+
+def mac_set_min_keys_per_cta(st, keys: int) -> None:
+    check("mac_set_min_keys_per_cta", load().mac_set_min_keys_per_cta(_h(st), int(keys)))
+
+
+def mac_attend_grid(st) -> int:
+    return int(load().mac_attend_grid(_h(st)))
+
+
+def mac_error_string(code: int) -> str:
+    return load().mac_error_string(int(code)).decode()
+
+
+def parse_state(buf, W: int, G: int, D: int):
+    """Split an exported state buffer into named numpy arrays (layout of include/mac.h)."""
+    import numpy as np
+    hdr = np.frombuffer(buf[:32].tobytes(), np.int32)
+    U, W1 = int(hdr[1]), int(hdr[2])
+    off = 32
+    out = {}
+    for name, n, dt, shape in (("q", U * W1 * G * D, np.float32, (U, W1, G, D)),
+                               ("o", U * W1 * G * D, np.float32, (U, W1, G, D)),
+                               ("m", U * W1 * G, np.float32, (U, W1, G)),
+                               ("l", U * W1 * G, np.float32, (U, W1, G)),
+                               ("pos", U * W1, np.int32, (U, W1)),
+                               ("steps", U, np.int32, (U,))):
+        nb = n * 4
+        out[name] = np.frombuffer(buf[off:off + nb].tobytes(), dt).reshape(shape)
+        off += nb
+    return out

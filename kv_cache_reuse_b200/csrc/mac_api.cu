@@ -1,0 +1,491 @@
+// mac_api.cu -- host side of the C ABI declared in include/mac.h: argument
+// checks, state and scratch allocation, TMA descriptors, kernel launches,
+// the KV append kernel, status and state export/import.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "mac_internal.cuh"
+
+#include "../../include/mac.h"
+
+using namespace mac;
+
+struct MacState {
+  MacConfig cfg;
+  int G, U, D, W, device, num_sms, grid, min_keys, capacity;
+  size_t max_parts;
+  // ring (library-owned state)
+  float* ring_q = nullptr;
+  float* ring_o = nullptr;
+  float* ring_m = nullptr;
+  float* ring_l = nullptr;
+  int* ring_pos = nullptr;
+  int* steps = nullptr;
+  // scratch
+  float* qrot = nullptr;
+  UnitPlan* plan = nullptr;
+  Segment* seg = nullptr;
+  PlanHeader* hdr = nullptr;
+  float* part = nullptr;
+  int* unit_cnt = nullptr;
+  int* done = nullptr;
+  unsigned* status = nullptr;
+  double* inv_freq = nullptr;
+  // staging for mac_decode_step_host
+  float* st_q = nullptr;
+  int* st_pos = nullptr;
+  int* st_lens = nullptr;
+  uint16_t* st_knew = nullptr;
+  uint16_t* st_vnew = nullptr;
+  float* st_out = nullptr;
+  float* st_lse = nullptr;
+  uint8_t* st_hit = nullptr;
+  int* st_mpos = nullptr;
+  // TMA descriptors of the last K/V pointers seen
+  const void* tm_k_ptr = nullptr;
+  const void* tm_v_ptr = nullptr;
+  CUtensorMap tmK, tmV;
+};
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename T>
+cudaError_t alloc(T** p, size_t count) {
+  return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T) + 16);
+}
+
+void free_all(MacState* s) {
+  void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot, s->plan,
+                  s->seg,    s->hdr,    s->part,   s->unit_cnt, s->done,   s->status, s->inv_freq,
+                  s->st_q,   s->st_pos, s->st_lens, s->st_knew, s->st_vnew, s->st_out, s->st_lse, s->st_hit,
+                  s->st_mpos};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+}
+
+int check_config(const MacConfig* c) {
+  if (!c) return MAC_ERR_ARG;
+  if (c->batch < 1 || c->num_kv_heads < 1 || c->num_q_heads < 1) return MAC_ERR_ARG;
+  if (c->num_q_heads % c->num_kv_heads != 0 || c->num_q_heads / c->num_kv_heads != kGroup) return MAC_ERR_SHAPE;
+  if (c->head_dim != 64 && c->head_dim != 128) return MAC_ERR_SHAPE;
+  if (c->window < 1 || c->window > kMaxWindow) return MAC_ERR_SHAPE;
+  if (c->band < 0) return MAC_ERR_ARG;
+  if (!(c->rope_theta > 0.0) || isnan(c->tau)) return MAC_ERR_ARG;
+  if (c->page_size == 0) {
+    if (c->max_seq < 1) return MAC_ERR_ARG;
+  } else {
+    if (c->page_size < 0 || c->page_size % kSubKeys != 0) return MAC_ERR_SHAPE;
+    if (c->max_pages_per_seq < 1 || c->num_pages < 1) return MAC_ERR_ARG;
+  }
+  return MAC_OK;
+}
+
+int encode_kv_map(MacState* s, CUtensorMap* map, const void* base) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MAC_ERR_CUDA;
+  const MacConfig& c = s->cfg;
+  const cuuint64_t D = (cuuint64_t)s->D, H = (cuuint64_t)c.num_kv_heads;
+  cuuint64_t dims[4], strides[3];
+  dims[0] = D;
+  dims[1] = H;
+  if (c.page_size == 0) {
+    dims[2] = (cuuint64_t)c.max_seq;
+    dims[3] = (cuuint64_t)c.batch;
+  } else {
+    dims[2] = (cuuint64_t)c.page_size;
+    dims[3] = (cuuint64_t)c.num_pages;
+  }
+  strides[0] = D * 2;
+  strides[1] = H * D * 2;
+  strides[2] = dims[2] * H * D * 2;
+  const cuuint32_t box[4] = {(cuuint32_t)D, 1u, (cuuint32_t)kSubKeys, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MAC_OK : MAC_ERR_CUDA;
+}
+
+__global__ void mac_append_kernel(const AppendParams p) {
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
+  const int pos = p.seq_lens[b] - 1;
+  if (pos < 0 || pos >= p.capacity) {
+    if (threadIdx.x == 0) atomicOr(p.status, MAC_DEV_BAD_SEQ_LEN);
+    return;
+  }
+  size_t row;
+  if (p.page_size > 0) {
+    const int pg = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
+    if (pg < 0 || pg >= p.num_pages) {
+      if (threadIdx.x == 0) atomicOr(p.status, MAC_DEV_BAD_PAGE);
+      return;
+    }
+    row = ((size_t)pg * p.page_size + (size_t)(pos % p.page_size)) * p.Hkv + kvh;
+  } else {
+    row = ((size_t)b * p.capacity + (size_t)pos) * p.Hkv + kvh;
+  }
+  const uint4* ks = reinterpret_cast<const uint4*>(p.k_new + (size_t)u * p.D);
+  const uint4* vs = reinterpret_cast<const uint4*>(p.v_new + (size_t)u * p.D);
+  uint4* kd = reinterpret_cast<uint4*>(p.K + row * p.D);
+  uint4* vd = reinterpret_cast<uint4*>(p.V + row * p.D);
+  for (int i = threadIdx.x; i < p.D / 8; i += blockDim.x) {
+    kd[i] = ks[i];
+    vd[i] = vs[i];
+  }
+}
+
+}  // namespace
+
+namespace mac {
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
+  mac_append_kernel<<<p.B * p.Hkv, 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+}  // namespace mac
+
+extern "C" {
+
+const char* mac_error_string(int code) {
+  switch (code) {
+    case MAC_OK: return "ok";
+    case MAC_ERR_ARG: return "invalid argument";
+    case MAC_ERR_SHAPE: return "unsupported shape";
+    case MAC_ERR_CUDA: return "CUDA call failed";
+    case MAC_ERR_OOM: return "device allocation failed";
+    case MAC_ERR_DEVICE: return "device-side fault flagged in the status word";
+    default: return "unknown error";
+  }
+}
+
+int mac_init_state(const MacConfig* cfg, MacState** out) {
+  if (!out) return MAC_ERR_ARG;
+  *out = nullptr;
+  int rc = check_config(cfg);
+  if (rc != MAC_OK) return rc;
+  MacState* s = new (std::nothrow) MacState();
+  if (!s) return MAC_ERR_OOM;
+  s->cfg = *cfg;
+  s->G = kGroup;
+  s->U = cfg->batch * cfg->num_kv_heads;
+  s->D = cfg->head_dim;
+  s->W = cfg->window;
+  s->min_keys = 128;
+  s->capacity = cfg->page_size == 0 ? cfg->max_seq : cfg->max_pages_per_seq * cfg->page_size;
+  if (cudaGetDevice(&s->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&s->num_sms, cudaDevAttrMultiProcessorCount, s->device) != cudaSuccess) {
+    delete s;
+    return MAC_ERR_CUDA;
+  }
+  s->grid = s->num_sms;  // one resident CTA per SM (shared-memory bound)
+  s->max_parts = (size_t)s->grid + 2 * (size_t)s->U;
+  const size_t U = s->U, W1 = s->W + 1, G = s->G, D = s->D, B = cfg->batch, Hq = cfg->num_q_heads;
+  const size_t Hkv = cfg->num_kv_heads;
+  cudaError_t e = cudaSuccess;
+  auto A = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+  };
+  A(alloc(&s->ring_q, U * W1 * G * D));
+  A(alloc(&s->ring_o, U * W1 * G * D));
+  A(alloc(&s->ring_m, U * W1 * G));
+  A(alloc(&s->ring_l, U * W1 * G));
+  A(alloc(&s->ring_pos, U * W1));
+  A(alloc(&s->steps, U));
+  A(alloc(&s->qrot, U * G * D));
+  A(alloc(&s->plan, U));
+  A(alloc(&s->seg, 2 * U));
+  A(alloc(&s->hdr, 1));
+  A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
+  A(alloc(&s->unit_cnt, U));
+  A(alloc(&s->done, 1));
+  A(alloc(&s->status, 1));
+  A(alloc(&s->inv_freq, D / 2));
+  A(alloc(&s->st_q, B * Hq * D));
+  A(alloc(&s->st_pos, B));
+  A(alloc(&s->st_lens, B));
+  A(alloc(&s->st_knew, B * Hkv * D));
+  A(alloc(&s->st_vnew, B * Hkv * D));
+  A(alloc(&s->st_out, B * Hq * D));
+  A(alloc(&s->st_lse, B * Hq));
+  A(alloc(&s->st_hit, U));
+  A(alloc(&s->st_mpos, U));
+  if (e != cudaSuccess) {
+    free_all(s);
+    delete s;
+    return e == cudaErrorMemoryAllocation ? MAC_ERR_OOM : MAC_ERR_CUDA;
+  }
+  A(cudaMemset(s->ring_q, 0, U * W1 * G * D * sizeof(float)));
+  A(cudaMemset(s->ring_o, 0, U * W1 * G * D * sizeof(float)));
+  A(cudaMemset(s->ring_m, 0, U * W1 * G * sizeof(float)));
+  A(cudaMemset(s->ring_l, 0, U * W1 * G * sizeof(float)));
+  A(cudaMemset(s->ring_pos, 0, U * W1 * sizeof(int)));
+  A(cudaMemset(s->steps, 0, U * sizeof(int)));
+  A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
+  A(cudaMemset(s->done, 0, sizeof(int)));
+  A(cudaMemset(s->status, 0, sizeof(unsigned)));
+  A(cudaMemset(s->hdr, 0, sizeof(PlanHeader)));
+  double* inv = (double*)malloc(sizeof(double) * (D / 2));
+  for (size_t i = 0; i < D / 2; ++i) inv[i] = pow(cfg->rope_theta, -2.0 * (double)i / (double)D);
+  A(cudaMemcpy(s->inv_freq, inv, sizeof(double) * (D / 2), cudaMemcpyHostToDevice));
+  free(inv);
+  A(attend_prepare((int)D));
+  A(cudaDeviceSynchronize());
+  if (e != cudaSuccess) {
+    free_all(s);
+    delete s;
+    return MAC_ERR_CUDA;
+  }
+  *out = s;
+  return MAC_OK;
+}
+
+void mac_destroy(MacState* s) {
+  if (!s) return;
+  cudaDeviceSynchronize();
+  free_all(s);
+  delete s;
+}
+
+int mac_reset_seq(MacState* s, int b, void* stream) {
+  if (!s || b < 0 || b >= s->cfg.batch) return MAC_ERR_ARG;
+  const int H = s->cfg.num_kv_heads;
+  cudaError_t e = cudaMemsetAsync(s->steps + (size_t)b * H, 0, sizeof(int) * H, (cudaStream_t)stream);
+  return e == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+}
+
+int mac_set_min_keys_per_cta(MacState* s, int keys) {
+  if (!s || keys < 1) return MAC_ERR_ARG;
+  s->min_keys = keys;
+  return MAC_OK;
+}
+
+int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
+
+int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
+              float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
+  if (!s || !q_pre || !rope_pos || !seq_lens || !out || !lse) return MAC_ERR_ARG;
+  if (!aligned16(q_pre)) return MAC_ERR_ARG;
+  if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
+  MatchParams p;
+  p.q_pre = q_pre;
+  p.rope_pos = rope_pos;
+  p.seq_lens = seq_lens;
+  p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
+  p.out = out;
+  p.lse = lse;
+  p.hit_mask = hit_mask;
+  p.match_pos = match_pos;
+  p.ring_q = s->ring_q;
+  p.ring_pos = s->ring_pos;
+  p.steps = s->steps;
+  p.inv_freq = s->inv_freq;
+  p.qrot = s->qrot;
+  p.plan = s->plan;
+  p.seg = s->seg;
+  p.hdr = s->hdr;
+  p.done = s->done;
+  p.status = s->status;
+  p.B = s->cfg.batch;
+  p.Hq = s->cfg.num_q_heads;
+  p.Hkv = s->cfg.num_kv_heads;
+  p.W = s->W;
+  p.band = s->cfg.band;
+  p.page_size = s->cfg.page_size;
+  p.max_pages = s->cfg.max_pages_per_seq;
+  p.num_pages = s->cfg.num_pages;
+  p.capacity = s->capacity;
+  p.tau = s->cfg.tau;
+  p.grid = s->grid;
+  p.min_keys = s->min_keys;
+  return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+}
+
+int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* block_table, float* out, float* lse,
+               void* stream) {
+  if (!s || !K || !V || !out || !lse) return MAC_ERR_ARG;
+  if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
+  if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
+  if (K != s->tm_k_ptr) {
+    int rc = encode_kv_map(s, &s->tmK, K);
+    if (rc != MAC_OK) return rc;
+    s->tm_k_ptr = K;
+  }
+  if (V != s->tm_v_ptr) {
+    int rc = encode_kv_map(s, &s->tmV, V);
+    if (rc != MAC_OK) return rc;
+    s->tm_v_ptr = V;
+  }
+  AttendParams p;
+  p.tmK = s->tmK;
+  p.tmV = s->tmV;
+  p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
+  p.qrot = s->qrot;
+  p.plan = s->plan;
+  p.seg = s->seg;
+  p.hdr = s->hdr;
+  p.part = s->part;
+  p.unit_cnt = s->unit_cnt;
+  p.ring_o = s->ring_o;
+  p.ring_m = s->ring_m;
+  p.ring_l = s->ring_l;
+  p.ring_pos = s->ring_pos;
+  p.out = out;
+  p.lse = lse;
+  p.status = s->status;
+  p.Hq = s->cfg.num_q_heads;
+  p.Hkv = s->cfg.num_kv_heads;
+  p.W = s->W;
+  p.page_size = s->cfg.page_size;
+  p.max_pages = s->cfg.max_pages_per_seq;
+  p.nseg = 2 * s->U;
+  return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+}
+
+int mac_decode_step(MacState* s, const float* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
+                    const int* block_table, const int* seq_lens, float* out, float* lse, uint8_t* hit_mask,
+                    int* match_pos, void* stream) {
+  if (!s || !K || !V) return MAC_ERR_ARG;
+  if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
+  int rc = mac_match(s, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream);
+  if (rc != MAC_OK) return rc;
+  return mac_attend(s, K, V, block_table, out, lse, stream);
+}
+
+int mac_append_kv(MacState* s, uint16_t* K, uint16_t* V, const int* block_table, const int* seq_lens,
+                  const uint16_t* k_new, const uint16_t* v_new, void* stream) {
+  if (!s || !K || !V || !seq_lens || !k_new || !v_new) return MAC_ERR_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(k_new) || !aligned16(v_new)) return MAC_ERR_ARG;
+  if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
+  AppendParams p;
+  p.K = K;
+  p.V = V;
+  p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
+  p.seq_lens = seq_lens;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.status = s->status;
+  p.B = s->cfg.batch;
+  p.Hkv = s->cfg.num_kv_heads;
+  p.D = s->D;
+  p.page_size = s->cfg.page_size;
+  p.max_pages = s->cfg.max_pages_per_seq;
+  p.num_pages = s->cfg.num_pages;
+  p.capacity = s->capacity;
+  return launch_append(p, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+}
+
+int mac_decode_step_host(MacState* s, const float* q_pre_h, const int* rope_pos_h, const int* seq_lens_h,
+                         const uint16_t* k_new_h, const uint16_t* v_new_h, uint16_t* K, uint16_t* V,
+                         const int* block_table, float* out_h, float* lse_h, uint8_t* hit_h, int* match_pos_h,
+                         void* stream) {
+  if (!s || !q_pre_h || !rope_pos_h || !seq_lens_h || !K || !V) return MAC_ERR_ARG;
+  if ((k_new_h == nullptr) != (v_new_h == nullptr)) return MAC_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t B = s->cfg.batch, Hq = s->cfg.num_q_heads, Hkv = s->cfg.num_kv_heads, D = s->D, U = s->U;
+  cudaError_t e = cudaSuccess;
+  auto A = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+  };
+  A(cudaMemcpyAsync(s->st_q, q_pre_h, B * Hq * D * sizeof(float), cudaMemcpyHostToDevice, st));
+  A(cudaMemcpyAsync(s->st_pos, rope_pos_h, B * sizeof(int), cudaMemcpyHostToDevice, st));
+  A(cudaMemcpyAsync(s->st_lens, seq_lens_h, B * sizeof(int), cudaMemcpyHostToDevice, st));
+  if (k_new_h) {
+    A(cudaMemcpyAsync(s->st_knew, k_new_h, B * Hkv * D * 2, cudaMemcpyHostToDevice, st));
+    A(cudaMemcpyAsync(s->st_vnew, v_new_h, B * Hkv * D * 2, cudaMemcpyHostToDevice, st));
+  }
+  if (e != cudaSuccess) return MAC_ERR_CUDA;
+  int rc;
+  if (k_new_h) {
+    rc = mac_append_kv(s, K, V, block_table, s->st_lens, s->st_knew, s->st_vnew, stream);
+    if (rc != MAC_OK) return rc;
+  }
+  rc = mac_decode_step(s, s->st_q, s->st_pos, K, V, block_table, s->st_lens, s->st_out, s->st_lse, s->st_hit,
+                       s->st_mpos, stream);
+  if (rc != MAC_OK) return rc;
+  if (out_h) A(cudaMemcpyAsync(out_h, s->st_out, B * Hq * D * sizeof(float), cudaMemcpyDeviceToHost, st));
+  if (lse_h) A(cudaMemcpyAsync(lse_h, s->st_lse, B * Hq * sizeof(float), cudaMemcpyDeviceToHost, st));
+  if (hit_h) A(cudaMemcpyAsync(hit_h, s->st_hit, U, cudaMemcpyDeviceToHost, st));
+  if (match_pos_h) A(cudaMemcpyAsync(match_pos_h, s->st_mpos, U * sizeof(int), cudaMemcpyDeviceToHost, st));
+  unsigned status = 0;
+  A(cudaMemcpyAsync(&status, s->status, sizeof(unsigned), cudaMemcpyDeviceToHost, st));
+  A(cudaStreamSynchronize(st));
+  if (e != cudaSuccess) return MAC_ERR_CUDA;
+  return status ? MAC_ERR_DEVICE : MAC_OK;
+}
+
+int mac_get_status(MacState* s, int* device_status) {
+  if (!s) return MAC_ERR_ARG;
+  unsigned v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MAC_ERR_CUDA;
+  if (cudaMemcpy(&v, s->status, sizeof(unsigned), cudaMemcpyDeviceToHost) != cudaSuccess) return MAC_ERR_CUDA;
+  if (cudaMemset(s->status, 0, sizeof(unsigned)) != cudaSuccess) return MAC_ERR_CUDA;
+  if (device_status) *device_status = (int)v;
+  return v ? MAC_ERR_DEVICE : MAC_OK;
+}
+
+size_t mac_state_bytes(const MacState* s) {
+  if (!s) return 0;
+  const size_t U = s->U, W1 = s->W + 1, G = s->G, D = s->D;
+  return 8 * sizeof(int) + 2 * U * W1 * G * D * sizeof(float) + 2 * U * W1 * G * sizeof(float) +
+         U * W1 * sizeof(int) + U * sizeof(int);
+}
+
+static int copy_state(MacState* s, void* host, size_t bytes, bool to_host) {
+  if (!s || !host || bytes < mac_state_bytes(s)) return MAC_ERR_ARG;
+  const size_t U = s->U, W1 = s->W + 1, G = s->G, D = s->D;
+  int hdr[8] = {0x4D414331, (int)U, (int)W1, (int)G, (int)D, 0, 0, 0};
+  unsigned char* h = static_cast<unsigned char*>(host);
+  if (to_host) {
+    memcpy(h, hdr, sizeof hdr);
+  } else {
+    if (memcmp(h, hdr, sizeof hdr) != 0) return MAC_ERR_SHAPE;
+  }
+  h += sizeof hdr;
+  struct Part {
+    void* dev;
+    size_t bytes;
+  } parts[] = {{s->ring_q, U * W1 * G * D * 4}, {s->ring_o, U * W1 * G * D * 4}, {s->ring_m, U * W1 * G * 4},
+               {s->ring_l, U * W1 * G * 4},     {s->ring_pos, U * W1 * 4},      {s->steps, U * 4}};
+  if (cudaDeviceSynchronize() != cudaSuccess) return MAC_ERR_CUDA;
+  for (const Part& p : parts) {
+    cudaError_t e = to_host ? cudaMemcpy(h, p.dev, p.bytes, cudaMemcpyDeviceToHost)
+                            : cudaMemcpy(p.dev, h, p.bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return MAC_ERR_CUDA;
+    h += p.bytes;
+  }
+  return MAC_OK;
+}
+
+int mac_export_state(const MacState* s, void* host_buf, size_t bytes) {
+  return copy_state(const_cast<MacState*>(s), host_buf, bytes, true);
+}
+
+int mac_import_state(MacState* s, const void* host_buf, size_t bytes) {
+  return copy_state(s, const_cast<void*>(host_buf), bytes, false);
+}
+
+}  // extern "C"

@@ -1,0 +1,663 @@
+// mac_attend.cu -- Amend, Complete, miss fallback and the stable merge.
+//
+// "MAC-Attention: a Match-Amend-Complete Scheme for Fast and Accurate
+// Attention Computation", page 1 (abstract): on a hit the amend stage
+// "rectifies the reused attention by recomputing a small band near the match
+// boundary" and the complete stage "fuses the rectified results with fresh
+// attention computed on the KV tail through a numerically stable merge"; on
+// a miss the step is split-KV decode attention over every key.  All three are
+// the same computation -- attention of the current query group over a key
+// range -- so one persistent kernel runs them over a flattened list of key
+// segments built by the match kernel:
+//   segment 2u   = [start, c_t)  -> folded into the unit's new prefix state
+//   segment 2u+1 = [c_t, p_t]    -> folded into the output only
+// The flattened keys are split evenly over the CTAs, so a mix of hits (a few
+// hundred keys) and misses (the whole context) keeps every SM equally busy.
+//
+// Per CTA: eight warps; warp w owns boxes w, w+8, w+16, ... of every piece,
+// where a box is 16 keys (it never crosses a page).  Each warp streams its
+// own boxes through its own ring of shared-memory slots with TMA
+// (cp.async.bulk.tensor, no multicast), keeping NST boxes in flight, so the
+// warps never wait on one another inside a piece.  Within a box a group of 8
+// lanes owns 4 keys and each lane owns D/8 dimensions of every head of the
+// GQA group (G = 4): q . k is a partial dot product per lane followed by a
+// reduce-scatter over the 8 lanes.  The work is HBM-bound (4 flop per byte
+// of K/V): the math stays on the FP32 pipes (packed f32x2 FMA), not on the
+// tensor cores, since a 4-row query tile is not a dense contraction.
+//
+// Softmax runs in exp2 units (the query is pre-scaled by log2(e)/sqrt(D)).
+// Every piece a CTA processes ends in a partial (o unnormalised, m, l).  The
+// CTA that delivers a unit's last partial (atomic counter, no waiting) merges
+// the reused ring state, the band and the tail partials, writes the new ring
+// entry, out and lse.
+//
+// Every wait is bounded (2 s on %globaltimer): on expiry the kernel sets
+// MAC_DEV_TIMEOUT in the status word and leaves without hanging the GPU.
+#include <math.h>
+#include <stdint.h>
+
+#include "mac_internal.cuh"
+
+#include "../../include/mac.h"
+
+namespace mac {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct StageMeta {
+  int unit, pidx;
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int NV = D / 64;  // 8-dim vectors per lane per row
+  static constexpr int NST = D == 128 ? 3 : 6;  // boxes in flight per warp
+  static constexpr int NQ = NST + 1;             // query buffers (pieces the issue cursor can be ahead)
+  static constexpr int GD = kGroup * D;
+  static constexpr int PF = kGroup * D + 2 * kGroup;  // floats of one partial
+  static constexpr int WB = (PF > 288 ? PF : 288);     // per-warp scratch floats
+};
+
+template <int D>
+struct __align__(128) AttnSmem {
+  uint16_t kv[kConsumerWarps][Cfg<D>::NST][2][kSubKeys * D];  // per warp: ring of (K box, V box)
+  float q[Cfg<D>::NQ][Cfg<D>::GD];                            // queries of the upcoming pieces
+  float wbuf[kConsumerWarps][Cfg<D>::WB];                     // weights exchange / piece combine
+  unsigned long long full[kConsumerWarps][Cfg<D>::NST];
+  unsigned long long qfull[Cfg<D>::NQ];
+  unsigned long long csync;
+  int abort_flag;
+  int last_flag;
+};
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* ptr) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait on phase `parity` of an mbarrier.  Returns false if the CTA
+// is aborting or the wait exceeded kWaitLimitNs (then it flags the abort).
+__device__ bool mbar_wait(unsigned long long* bar, uint32_t parity, volatile int* abort_flag,
+                          unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicOr(status, MAC_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, unsigned long long* bar, int c0,
+                                            int c1, int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ float sel(bool c, float a, float b) { return c ? a : b; }
+
+// ------------------------------------------------------------ consumer state
+template <int D>
+struct Acc {
+  float2 q[kGroup][Cfg<D>::NV][4];  // this lane's dims of every head, (even, odd) pairs
+  float2 o[kGroup][Cfg<D>::NV][4];  // unnormalised output accumulators
+  float m[kGroup];                  // running max (log2 units), same in all lanes of a group
+  float l[2];                       // running sum for heads 2*b0, 2*b0+1 over this lane's key
+};
+
+// One 16-key box for one warp.  Group g (lanes 8g..8g+7) takes keys 4g..4g+3
+// of the box; lane j of a group holds dims [64v + 8j, 64v + 8j + 8).
+template <int D, bool MASKED>
+__device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, const uint16_t* vbox, float* pbuf,
+                                            int key_box, int k0, int k1) {
+  constexpr int NV = Cfg<D>::NV;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 3, j = lane & 7;
+  const bool b2 = (j & 4) != 0, b1 = (j & 2) != 0, b0 = (j & 1) != 0;
+  const uint16_t* kg = kbox + (4 * g) * D + 8 * j;
+  const uint16_t* vg = vbox + (4 * g) * D + 8 * j;
+
+  // q . k partial sums over this lane's dims: acc[kk][h]
+  float s[16];
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    float2 acc[kGroup];
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) acc[h] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const uint4 kr = *reinterpret_cast<const uint4*>(kg + kk * D + 64 * v);
+      const uint32_t w4[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 kf = unpack_bf16x2(w4[e]);
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) acc[h] = __ffma2_rn(A.q[h][v][e], kf, acc[h]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) s[kk * 4 + h] = acc[h].x + acc[h].y;
+  }
+  // reduce-scatter over the 8 lanes: bit 2 picks the key pair, bit 1 the
+  // key, bit 0 the head pair.  Lane ends with the full scores of key
+  // kk = 2*b2 + b1 for heads 2*b0 and 2*b0 + 1.
+  float t8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float keep = sel(b2, s[i + 8], s[i]), send = sel(b2, s[i], s[i + 8]);
+    t8[i] = keep + __shfl_xor_sync(kFull, send, 4);
+  }
+  float t4[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = sel(b1, t8[i + 4], t8[i]), send = sel(b1, t8[i], t8[i + 4]);
+    t4[i] = keep + __shfl_xor_sync(kFull, send, 2);
+  }
+  float sc[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = sel(b0, t4[i + 2], t4[i]), send = sel(b0, t4[i], t4[i + 2]);
+    sc[i] = keep + __shfl_xor_sync(kFull, send, 1);
+  }
+  const int kkl = (b2 ? 2 : 0) + (b1 ? 1 : 0);
+  if (MASKED) {
+    const int key = key_box + 4 * g + kkl;
+    if (key < k0 || key >= k1) sc[0] = sc[1] = -INFINITY;
+  }
+  // block max per head over the group's 4 keys
+  float bm0 = fmaxf(sc[0], __shfl_xor_sync(kFull, sc[0], 4));
+  float bm1 = fmaxf(sc[1], __shfl_xor_sync(kFull, sc[1], 4));
+  bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, 2));
+  bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, 2));
+  const float om0 = __shfl_xor_sync(kFull, bm0, 1), om1 = __shfl_xor_sync(kFull, bm1, 1);
+  const float bmax[4] = {sel(b0, om0, bm0), sel(b0, om1, bm1), sel(b0, bm0, om0), sel(b0, bm1, om1)};
+  bool need = false;
+  float mnew[kGroup];
+#pragma unroll
+  for (int h = 0; h < kGroup; ++h) {
+    mnew[h] = fmaxf(A.m[h], bmax[h]);
+    need |= mnew[h] > A.m[h];
+  }
+  if (__any_sync(kFull, need)) {
+#pragma unroll
+    for (int h = 0; h < kGroup; ++h) {
+      const float mu = mnew[h] == -INFINITY ? 0.f : mnew[h];
+      const float a = ex2(A.m[h] - mu);
+      const float2 a2 = make_float2(a, a);
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) A.o[h][v][e] = __fmul2_rn(A.o[h][v][e], a2);
+      if (h == (b0 ? 2 : 0)) A.l[0] *= a;
+      if (h == (b0 ? 3 : 1)) A.l[1] *= a;
+      A.m[h] = mnew[h];
+    }
+  }
+  const float m0 = b0 ? A.m[2] : A.m[0], m1 = b0 ? A.m[3] : A.m[1];
+  const float p0 = ex2(sc[0] - (m0 == -INFINITY ? 0.f : m0));
+  const float p1 = ex2(sc[1] - (m1 == -INFINITY ? 0.f : m1));
+  A.l[0] += p0;
+  A.l[1] += p1;
+  // share the 16 weights of the group: float pairs (p, p) per (key, head)
+  float* pg = pbuf + g * 36;
+  *reinterpret_cast<float4*>(pg + kkl * 8 + 4 * (b0 ? 1 : 0)) = make_float4(p0, p0, p1, p1);
+  __syncwarp();
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const float4 pa = *reinterpret_cast<const float4*>(pg + kk * 8);
+    const float4 pc = *reinterpret_cast<const float4*>(pg + kk * 8 + 4);
+    const float2 pp[4] = {make_float2(pa.x, pa.y), make_float2(pa.z, pa.w), make_float2(pc.x, pc.y),
+                          make_float2(pc.z, pc.w)};
+    bool valid = true;
+    if (MASKED) {
+      const int key = key_box + 4 * g + kk;
+      valid = key >= k0 && key < k1;
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      uint4 vr = *reinterpret_cast<const uint4*>(vg + kk * D + 64 * v);
+      if (MASKED && !valid) vr = make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w4[4] = {vr.x, vr.y, vr.z, vr.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 vf = unpack_bf16x2(w4[e]);
+#pragma unroll
+        for (int h = 0; h < kGroup; ++h) A.o[h][v][e] = __ffma2_rn(pp[h], vf, A.o[h][v][e]);
+      }
+    }
+  }
+}
+
+// Bounded barrier of the 8 consumer warps (mbarrier with one arrival per warp).
+template <int D>
+__device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, unsigned* status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.csync);
+  const bool ok = mbar_wait(&sm.csync, phase, &sm.abort_flag, status);
+  phase ^= 1u;
+  __syncwarp();
+  return ok;
+}
+
+// Merge of unit u by the CTA holding its last partial (256 consumer threads).
+template <int D>
+__device__ void merge_unit(const AttendParams& p, int u) {
+  constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
+  const UnitPlan pl = p.plan[u];
+  const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
+  const int Wp1 = p.W + 1;
+  for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
+    const int h = idx / D, d = idx - h * D;
+    // new prefix state over [0, c_t): reused state (hit) + amend partials
+    float M = -INFINITY, rm = -INFINITY, rl = 0.f, ro = 0.f;
+    if (pl.hit) {
+      const size_t rs = (size_t)u * Wp1 + pl.src_slot;
+      rl = p.ring_l[rs * G + h];
+      rm = p.ring_m[rs * G + h] * kLog2e;
+      ro = p.ring_o[rs * GD + idx];
+      M = rm;
+    }
+    for (int i = 0; i < sA.npieces; ++i) M = fmaxf(M, __ldcg(p.part + (size_t)(sA.pbase + i) * PF + GD + h));
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f, O = 0.f;
+    if (pl.hit) {
+      const float a = ex2(rm - Mu);
+      L += rl * a;
+      O += ro * rl * a;
+    }
+    for (int i = 0; i < sA.npieces; ++i) {
+      const float* pp = p.part + (size_t)(sA.pbase + i) * PF;
+      const float a = ex2(__ldcg(pp + GD + h) - Mu);
+      L += __ldcg(pp + GD + G + h) * a;
+      O += __ldcg(pp + idx) * a;
+    }
+    const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
+    p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
+    if (d == 0) {
+      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
+      p.ring_l[ds * G + h] = L;
+    }
+    // output: new prefix state + tail partials
+    float M2 = M;
+    for (int i = 0; i < sB.npieces; ++i) M2 = fmaxf(M2, __ldcg(p.part + (size_t)(sB.pbase + i) * PF + GD + h));
+    const float M2u = M2 == -INFINITY ? 0.f : M2;
+    const float a0 = ex2(M - M2u);
+    float L2 = L * a0, O2 = O * a0;
+    for (int i = 0; i < sB.npieces; ++i) {
+      const float* pp = p.part + (size_t)(sB.pbase + i) * PF;
+      const float a = ex2(__ldcg(pp + GD + h) - M2u);
+      L2 += __ldcg(pp + GD + G + h) * a;
+      O2 += __ldcg(pp + idx) * a;
+    }
+    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    p.out[orow * D + d] = O2 / L2;
+    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+  }
+  if (threadIdx.x == 0) {
+    p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
+    p.unit_cnt[u] = 0;
+  }
+}
+
+// End of a piece: combine the 32 groups' states, write the partial, count it
+// and, if it was the unit's last, merge the unit.
+template <int D>
+__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, const StageMeta& m,
+                               uint32_t& sync_phase) {
+  constexpr int NV = Cfg<D>::NV, G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j = lane & 7;
+  const bool b0 = (j & 1) != 0;
+  __syncwarp();
+  // group sums of l for this lane's head pair, then all four heads
+  float l0 = A.l[0], l1 = A.l[1];
+  l0 += __shfl_xor_sync(kFull, l0, 4);
+  l1 += __shfl_xor_sync(kFull, l1, 4);
+  l0 += __shfl_xor_sync(kFull, l0, 2);
+  l1 += __shfl_xor_sync(kFull, l1, 2);
+  const float o0 = __shfl_xor_sync(kFull, l0, 1), o1 = __shfl_xor_sync(kFull, l1, 1);
+  float lg[4] = {sel(b0, o0, l0), sel(b0, o1, l1), sel(b0, l0, o0), sel(b0, l1, o1)};
+  // combine the warp's 4 groups
+#pragma unroll
+  for (int off = 8; off <= 16; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mo = __shfl_xor_sync(kFull, A.m[h], off);
+      const float M = fmaxf(A.m[h], mo);
+      const float Mu = M == -INFINITY ? 0.f : M;
+      const float a = ex2(A.m[h] - Mu), ao = ex2(mo - Mu);
+      lg[h] = lg[h] * a + __shfl_xor_sync(kFull, lg[h], off) * ao;
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = A.o[h][v][e];
+          const float2 y = make_float2(__shfl_xor_sync(kFull, x.x, off), __shfl_xor_sync(kFull, x.y, off));
+          A.o[h][v][e] = make_float2(x.x * a + y.x * ao, x.y * a + y.y * ao);
+        }
+      A.m[h] = M;
+    }
+  }
+  float* wb = sm.wbuf[warp];
+  if (lane < 8) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<float2*>(wb + h * D + 64 * v + 8 * j + 2 * e) = A.o[h][v][e];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      wb[GD + h] = A.m[h];
+      wb[GD + G + h] = lg[h];
+    }
+  }
+  if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  // combine the 8 warps and write the partial
+  float* dst = p.part + (size_t)m.pidx * PF;
+  for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
+    const int h = idx / D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wbuf[w][GD + h]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float acc = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float a = ex2(sm.wbuf[w][GD + h] - Mu);
+      acc += sm.wbuf[w][idx] * a;
+      L += sm.wbuf[w][GD + G + h] * a;
+    }
+    dst[idx] = acc;
+    if (idx - h * D == 0) {
+      dst[GD + h] = M;
+      dst[GD + G + h] = L;
+    }
+  }
+  __threadfence();
+  if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(p.unit_cnt + m.unit, 1);
+    sm.last_flag = (old == p.plan[m.unit].expected - 1);
+  }
+  if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  if (sm.last_flag) {
+    __threadfence();
+    merge_unit<D>(p, m.unit);
+  }
+  return true;
+}
+
+// The CTA's pieces, walked in order by every lane of every warp.
+struct Piece {
+  int unit, pidx, k0, k1, kb0, nbox;
+};
+struct Walker {
+  int s;
+  long long lo, hi;
+  __device__ __forceinline__ bool next(const AttendParams& p, int cta, Piece& pc) {
+    while (s < p.nseg) {
+      const Segment sg = p.seg[s];
+      if (sg.flat >= hi) {
+        s = p.nseg;
+        return false;
+      }
+      const int cur = s++;
+      if (sg.len == 0) continue;
+      const long long fa = lo > sg.flat ? lo : sg.flat;
+      const long long fe = hi < sg.flat + sg.len ? hi : sg.flat + sg.len;
+      pc.unit = cur >> 1;
+      pc.pidx = sg.pbase + (cta - sg.first_cta);
+      pc.k0 = sg.key0 + (int)(fa - sg.flat);
+      pc.k1 = sg.key0 + (int)(fe - sg.flat);
+      pc.kb0 = pc.k0 & ~(kSubKeys - 1);
+      pc.nbox = (((pc.k1 + kSubKeys - 1) & ~(kSubKeys - 1)) - pc.kb0) / kSubKeys;
+      return true;
+    }
+    return false;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
+  constexpr int NST = Cfg<D>::NST, NQ = Cfg<D>::NQ, NV = Cfg<D>::NV, G = kGroup, GD = Cfg<D>::GD;
+  constexpr uint32_t kBoxBytes = kSubKeys * D * 2;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int n_cta = p.hdr->n_cta;
+  const int cta = blockIdx.x;
+  if (cta >= n_cta) return;
+  if (tid == 0) {
+    for (int w = 0; w < kConsumerWarps; ++w)
+      for (int s = 0; s < NST; ++s) mbar_init(&sm.full[w][s], 1);
+    for (int s = 0; s < NQ; ++s) mbar_init(&sm.qfull[s], 1);
+    mbar_init(&sm.csync, kConsumerWarps);
+    sm.abort_flag = 0;
+    sm.last_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  const long long T = p.hdr->total;
+  const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
+  int first_seg = 0;
+  {
+    int a = 0, z = p.nseg - 1;  // last segment starting at or before lo
+    while (a < z) {
+      const int mid = (a + z + 1) >> 1;
+      if (p.seg[mid].flat <= lo) a = mid; else z = mid - 1;
+    }
+    first_seg = a;
+  }
+  const uint64_t pol = evict_first_policy();
+
+  // issue cursor: this warp's boxes w, w+8, ... of every piece, NST ahead
+  Walker wi{first_seg, lo, hi};
+  Piece ip;
+  bool ivalid = wi.next(p, cta, ip);
+  int ib = warp, ipn = 0, nissued = 0, nq_issued = 0;
+  auto issue_advance = [&]() {
+    while (ivalid && ib >= ip.nbox) {
+      ivalid = wi.next(p, cta, ip);
+      ib = warp;
+      ++ipn;
+    }
+  };
+  auto issue_box = [&](int st) {
+    if (lane == 0) {
+      if (warp == 0 && ib == 0) {  // first box of a piece: bring its query too
+        const int qs = ipn % NQ;
+        mbar_arrive_expect_tx(&sm.qfull[qs], GD * 4);
+        bulk_load(sm.q[qs], p.qrot + (size_t)ip.unit * GD, GD * 4, &sm.qfull[qs]);
+      }
+    }
+    if (warp == 0 && ib == 0) ++nq_issued;
+    if (lane == 0) {
+      const int key = ip.kb0 + ib * kSubKeys;
+      const int b = ip.unit / p.Hkv, kvh = ip.unit - b * p.Hkv;
+      int c2, c3;
+      if (p.page_size > 0) {
+        c3 = p.block_table[(size_t)b * p.max_pages + key / p.page_size];
+        c2 = key % p.page_size;
+      } else {
+        c2 = key;
+        c3 = b;
+      }
+      mbar_arrive_expect_tx(&sm.full[warp][st], 2 * kBoxBytes);
+      tma_load_4d(sm.kv[warp][st][0], &p.tmK, &sm.full[warp][st], 0, kvh, c2, c3, pol);
+      tma_load_4d(sm.kv[warp][st][1], &p.tmV, &sm.full[warp][st], 0, kvh, c2, c3, pol);
+    }
+    ++nissued;
+    ib += kConsumerWarps;
+    issue_advance();
+  };
+  issue_advance();
+  for (int k = 0; k < NST && ivalid; ++k) issue_box(k);
+
+  // consume cursor
+  Acc<D> A;
+  Walker wc{first_seg, lo, hi};
+  Piece cp;
+  int cpn = 0, cons = 0, par = 0;
+  uint32_t sync_phase = 0;
+  bool ok = true;
+  while (ok && wc.next(p, cta, cp)) {
+    const int qs = cpn % NQ;
+    if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
+    {
+      const float* qsm = sm.q[qs];
+      const int j = lane & 7;
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          const float4 x = *reinterpret_cast<const float4*>(qsm + h * D + 64 * v + 8 * j);
+          const float4 y = *reinterpret_cast<const float4*>(qsm + h * D + 64 * v + 8 * j + 4);
+          A.q[h][v][0] = make_float2(x.x, x.y);
+          A.q[h][v][1] = make_float2(x.z, x.w);
+          A.q[h][v][2] = make_float2(y.x, y.y);
+          A.q[h][v][3] = make_float2(y.z, y.w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) A.o[h][v][e] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+      for (int h = 0; h < G; ++h) A.m[h] = -INFINITY;
+      A.l[0] = A.l[1] = 0.f;
+    }
+    for (int bj = warp; bj < cp.nbox; bj += kConsumerWarps) {
+      const int st = cons % NST;
+      if (!mbar_wait(&sm.full[warp][st], (uint32_t)(cons / NST) & 1u, &sm.abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      const int key_box = cp.kb0 + bj * kSubKeys;
+      float* pbuf = sm.wbuf[warp] + par * 144;
+      if (key_box < cp.k0 || key_box + kSubKeys > cp.k1)
+        process_box<D, true>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cp.k0, cp.k1);
+      else
+        process_box<D, false>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cp.k0, cp.k1);
+      par ^= 1;
+      ++cons;
+      __syncwarp();
+      if (ivalid) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue_box(st);
+      }
+    }
+    if (!ok) break;
+    StageMeta m;
+    m.unit = cp.unit;
+    m.pidx = cp.pidx;
+    if (!finalize_piece<D>(p, sm, A, m, sync_phase)) break;
+    ++cpn;
+  }
+  if (nissued > cons || !ok) {
+    // aborting: let copies already issued land before the CTA leaves (bounded)
+    if (lane == 0) {
+      for (int k = cons; k < nissued; ++k) {
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(&sm.full[warp][k % NST], (uint32_t)(k / NST) & 1u) &&
+               globaltimer() - t0 < 100000000ull) {
+        }
+      }
+      if (warp == 0) {
+        for (int k = cpn; k < nq_issued; ++k) {
+          const unsigned long long t0 = globaltimer();
+          while (!mbar_try_wait(&sm.qfull[k % NQ], (uint32_t)(k / NQ) & 1u) && globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+
+size_t attend_smem_bytes(int D) {
+  return D == 128 ? sizeof(AttnSmem<128>) : sizeof(AttnSmem<64>);
+}
+
+cudaError_t attend_prepare(int D) {
+  if (D == 128)
+    return cudaFuncSetAttribute(mac_attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(AttnSmem<128>));
+  if (D == 64)
+    return cudaFuncSetAttribute(mac_attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(AttnSmem<64>));
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s) {
+  if (D == 128)
+    mac_attend_kernel<128><<<grid, kAttnThreads, sizeof(AttnSmem<128>), s>>>(p);
+  else if (D == 64)
+    mac_attend_kernel<64><<<grid, kAttnThreads, sizeof(AttnSmem<64>), s>>>(p);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+}  // namespace mac

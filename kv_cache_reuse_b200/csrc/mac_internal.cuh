@@ -1,0 +1,117 @@
+// mac_internal.cuh -- device-side data layout shared by the MAC kernels and
+// the host API of this library (not part of the public C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mac {
+
+constexpr int kGroup = 4;             // query heads per KV head handled by the kernels
+constexpr int kSubKeys = 16;          // keys per TMA box (one box never crosses a page)
+constexpr int kConsumerWarps = 8;     // attention warps that compute
+constexpr int kKeysPerStage = 128;    // keys in flight per round of boxes (kConsumerWarps * 16)
+constexpr int kAttnThreads = kConsumerWarps * 32;
+constexpr int kMatchThreads = 256;
+constexpr int kMaxWindow = 256;
+
+// Per (sequence, KV head) plan written by the match kernel.
+struct UnitPlan {
+  int start;     // first key attended with the current query (c_s on a hit, 0 on a miss)
+  int cut;       // c_t = max(0, p_t - band): end of the stored prefix state
+  int end;       // p_t + 1
+  int hit;       // 1 = reuse the state in ring slot src_slot
+  int src_slot;  // ring slot of the matched entry (hit only)
+  int dst_slot;  // ring slot receiving this step's entry
+  int bad;       // 1 = invalid inputs: no work, NaN outputs, window unchanged
+  int expected;  // partial results the unit's merge waits for
+};
+
+// Two key segments per unit: 2u = [start, cut) (into the new prefix state),
+// 2u+1 = [cut, end) (tail, into the output only).  The segments of all units
+// are laid end to end ("flattened") and split evenly over the CTAs.
+struct Segment {
+  long long flat;  // offset in the flattened key space
+  int len;         // keys
+  int key0;        // first key (absolute position in the sequence)
+  int first_cta;   // CTA holding key `flat`
+  int pbase;       // index of this segment's first partial result
+  int npieces;     // partial results (CTAs overlapping the segment)
+  int pad;
+};
+
+struct PlanHeader {
+  long long total;  // keys in the flattened space
+  int n_cta;        // CTAs with work (<= grid)
+  int pad;
+};
+
+// Layout of one partial result: o_acc [G][D] (unnormalised, relative to m),
+// then m [G] (log2 units), l [G].
+__host__ __device__ inline size_t partial_floats(int D) { return (size_t)kGroup * D + 2 * kGroup; }
+
+struct MatchParams {
+  const float* q_pre;      // [B][Hq][D]
+  const int* rope_pos;     // [B]
+  const int* seq_lens;     // [B]
+  const int* block_table;  // [B][max_pages] or null
+  float* out;              // [B][Hq][D] (NaN for bad units)
+  float* lse;              // [B][Hq]
+  uint8_t* hit_mask;       // [U] or null
+  int* match_pos;          // [U] or null
+  float* ring_q;           // [U][W+1][G][D]
+  const int* ring_pos;     // [U][W+1]
+  int* steps;              // [U]
+  const double* inv_freq;  // [D/2]
+  float* qrot;             // [U][G][D], RoPE'd and scaled by log2(e)/sqrt(D)
+  UnitPlan* plan;          // [U]
+  Segment* seg;            // [2U]
+  PlanHeader* hdr;
+  int* done;               // arrival counter of the match CTAs (reset by the last)
+  unsigned* status;
+  int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;
+  float tau;
+  int grid;       // CTAs of the attention kernel
+  int min_keys;   // minimum keys per attention CTA
+};
+
+struct AttendParams {
+  CUtensorMap tmK;  // 4D (D, Hkv, rows, seqs|pages), box (D, 1, 16, 1)
+  CUtensorMap tmV;
+  const int* block_table;
+  const float* qrot;
+  const UnitPlan* plan;
+  const Segment* seg;
+  const PlanHeader* hdr;
+  float* part;       // [max_parts][partial_floats]
+  int* unit_cnt;     // [U]
+  float* ring_o;     // [U][W+1][G][D]
+  float* ring_m;     // [U][W+1][G]
+  float* ring_l;     // [U][W+1][G]
+  int* ring_pos;     // [U][W+1]
+  float* out;        // [B][Hq][D]
+  float* lse;        // [B][Hq]
+  unsigned* status;
+  int Hq, Hkv, W, page_size, max_pages, nseg;
+};
+
+struct AppendParams {
+  uint16_t* K;
+  uint16_t* V;
+  const int* block_table;
+  const int* seq_lens;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  unsigned* status;
+  int B, Hkv, D, page_size, max_pages, num_pages, capacity;
+};
+
+// Launchers (defined in the .cu files).
+cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s);
+cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+cudaError_t attend_prepare(int D);
+size_t attend_smem_bytes(int D);
+
+}  // namespace mac

@@ -1,0 +1,308 @@
+// mac_match.cu -- Match stage of MAC-Attention and the step's work plan.
+//
+// "MAC-Attention: a Match-Amend-Complete Scheme for Fast and Accurate
+// Attention Computation", page 1 (abstract): the match stage "performs
+// pre-RoPE L2 matching over a short local window" of recent queries whose
+// attention results can be reused.  One CTA handles one (sequence, KV head)
+// unit:
+//   1. distance of the current pre-RoPE query group (G heads) to every
+//      window entry: mean over heads of the squared L2 distance, summed in
+//      fp32 as sum((a - b)^2) -- the expanded |a|^2 + |b|^2 - 2ab form would
+//      cancel catastrophically for near-repeats;
+//   2. argmin with ties to the more recent entry, hit iff the minimum is
+//      strictly below tau; NaN distances never win;
+//   3. key ranges: the reused prefix ends at c_s = max(0, p_s - band) (the
+//      amend band starts there), the stored prefix of this step ends at
+//      c_t = max(0, p_t - band), and the tail runs to p_t;
+//   4. RoPE of the query to rope_pos (fp64 angle), pre-scaled by
+//      log2(e)/sqrt(D) so the attention kernel works in exp2 units;
+//   5. the query enters the ring slot n mod (W+1) (W+1 slots: the slot
+//      written is never one the window can read this step).
+// The last CTA to finish lays every unit's two key segments end to end and
+// splits the total evenly over the attention kernel's CTAs (no CTA waits
+// for another: the last arrival does the work).
+#include <math.h>
+#include <stdint.h>
+
+#include "mac_internal.cuh"
+
+#include "../../include/mac.h"
+
+namespace mac {
+namespace {
+
+constexpr double kLog2e = 1.4426950408889634;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Exclusive scan of one value per thread over a block of kMatchThreads.
+__device__ long long block_exclusive_scan(long long v, long long* total, long long* sbuf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sbuf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = lane < kMatchThreads / 32 ? sbuf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      long long y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kMatchThreads / 32) sbuf[lane] = w;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  long long before = warp > 0 ? sbuf[warp - 1] : 0;
+  *total = sbuf[kMatchThreads / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// CTA holding flattened key x when T keys are split over N CTAs as
+// [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
+__device__ __forceinline__ int cta_of(long long x, long long T, int N) {
+  return (int)(((x + 1) * (long long)N + T - 1) / T) - 1;
+}
+
+__device__ void build_segments(const MatchParams& p, int U) {
+  __shared__ long long sbuf[kMatchThreads / 32];
+  const int tid = threadIdx.x;
+  const int nseg = 2 * U;
+  long long carry = 0;
+  for (int base = 0; base < nseg; base += kMatchThreads) {
+    const int s = base + tid;
+    int len = 0, key0 = 0;
+    if (s < nseg) {
+      const UnitPlan* pl = p.plan + (s >> 1);
+      const int bad = __ldcg(&pl->bad);
+      if (!bad) {
+        const int start = __ldcg(&pl->start), cut = __ldcg(&pl->cut), end = __ldcg(&pl->end);
+        len = (s & 1) ? end - cut : cut - start;
+        key0 = (s & 1) ? cut : start;
+      }
+    }
+    long long tot;
+    long long ex = block_exclusive_scan(len, &tot, sbuf);
+    if (s < nseg) {
+      p.seg[s].flat = carry + ex;
+      p.seg[s].len = len;
+      p.seg[s].key0 = key0;
+    }
+    carry += tot;
+  }
+  const long long T = carry;
+  int N = 0;
+  if (T > 0) {
+    long long want = (T + p.min_keys - 1) / p.min_keys;
+    N = (int)(want < (long long)p.grid ? want : (long long)p.grid);
+    if (N < 1) N = 1;
+  }
+  __syncthreads();
+  long long pcarry = 0;
+  for (int base = 0; base < nseg; base += kMatchThreads) {
+    const int s = base + tid;
+    int np = 0, first = 0;
+    if (s < nseg) {
+      const long long F = p.seg[s].flat;
+      const int len = p.seg[s].len;
+      if (len > 0) {
+        first = cta_of(F, T, N);
+        np = cta_of(F + len - 1, T, N) - first + 1;
+      }
+    }
+    long long tot;
+    long long ex = block_exclusive_scan(np, &tot, sbuf);
+    // units own segments (2u, 2u+1): adjacent threads of one warp
+    const int np_next = __shfl_down_sync(0xffffffffu, np, 1);
+    if (s < nseg) {
+      p.seg[s].first_cta = first;
+      p.seg[s].npieces = np;
+      p.seg[s].pbase = (int)(pcarry + ex);
+      if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
+    }
+    pcarry += tot;
+  }
+  if (tid == 0) {
+    p.hdr->total = T;
+    p.hdr->n_cta = N;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchParams p) {
+  constexpr int G = kGroup;
+  constexpr int GD = G * D;
+  __shared__ __align__(16) float sq[GD];
+  __shared__ float sdist[kMaxWindow];
+  __shared__ int spos[kMaxWindow];
+  __shared__ int sslot[kMaxWindow];
+  __shared__ int s_bad_page, s_last;
+  __shared__ UnitPlan s_plan;
+
+  const int u = blockIdx.x;
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int Wp1 = p.W + 1;
+
+  const float4* qsrc = reinterpret_cast<const float4*>(p.q_pre + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
+  for (int i = tid; i < GD / 4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = qsrc[i];
+  const int len = p.seq_lens[b];
+  const int p_t = len - 1;
+  const int n = p.steps[u];
+  const int occ = n < p.W ? n : p.W;
+  if (tid == 0) s_bad_page = 0;
+  __syncthreads();
+
+  // 1. distances to the window entries, newest first (age j = 0 is step n-1)
+  for (int j = warp; j < occ; j += kMatchThreads / 32) {
+    const int slot = (n - 1 - j) % Wp1;
+    const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
+    float acc = 0.f;
+    for (int i = lane; i < GD / 4; i += 32) {
+      const float4 r = rq[i];
+      const float4 q = reinterpret_cast<const float4*>(sq)[i];
+      const float dx = q.x - r.x, dy = q.y - r.y, dz = q.z - r.z, dw = q.w - r.w;
+      acc = fmaf(dx, dx, acc);
+      acc = fmaf(dy, dy, acc);
+      acc = fmaf(dz, dz, acc);
+      acc = fmaf(dw, dw, acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) {
+      sdist[j] = acc * (1.0f / G);
+      spos[j] = p.ring_pos[(size_t)u * Wp1 + slot];
+      sslot[j] = slot;
+    }
+  }
+  __syncthreads();
+
+  // 2. argmin: smaller distance, then larger position, then the newer entry
+  if (warp == 0) {
+    float bd = INFINITY;
+    int bp = 0, bj = -1;
+    for (int j = lane; j < occ; j += 32) {
+      const float d = sdist[j];
+      const int pos = spos[j];
+      if (pos < p_t && (d < bd || (d == bd && bj >= 0 && (pos > bp || (pos == bp && j < bj))))) {
+        bd = d;
+        bp = pos;
+        bj = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float od = __shfl_xor_sync(0xffffffffu, bd, o);
+      const int op = __shfl_xor_sync(0xffffffffu, bp, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      const bool take = oj >= 0 && (bj < 0 || od < bd || (od == bd && (op > bp || (op == bp && oj < bj))));
+      if (take) {
+        bd = od;
+        bp = op;
+        bj = oj;
+      }
+    }
+    if (lane == 0) {
+      const int hit = (bj >= 0) && (bd < p.tau);
+      UnitPlan pl;
+      pl.end = len;
+      pl.cut = p_t - p.band > 0 ? p_t - p.band : 0;
+      pl.hit = hit;
+      pl.src_slot = hit ? sslot[bj] : -1;
+      pl.start = hit ? (bp - p.band > 0 ? bp - p.band : 0) : 0;
+      pl.dst_slot = n % Wp1;
+      pl.bad = (len < 1 || len > p.capacity) ? 1 : 0;
+      pl.expected = 0;
+      s_plan = pl;
+      spos[0] = hit ? bp : -1;  // matched position (slot 0 of spos no longer needed)
+    }
+  }
+  __syncthreads();
+
+  // paged KV: every page the step reads must be a valid pool page
+  if (!s_plan.bad && p.page_size > 0) {
+    const int pg0 = s_plan.start / p.page_size, pg1 = (s_plan.end - 1) / p.page_size;
+    const int* row = p.block_table + (size_t)b * p.max_pages;
+    for (int i = pg0 + tid; i <= pg1; i += kMatchThreads) {
+      const int pg = row[i];
+      if (pg < 0 || pg >= p.num_pages) s_bad_page = 1;
+    }
+  }
+  __syncthreads();
+  const int bad = s_plan.bad | s_bad_page;
+
+  if (bad) {
+    const float qnan = __int_as_float(0x7fc00000);
+    for (int i = tid; i < GD; i += kMatchThreads) p.out[((size_t)b * p.Hq + (size_t)kvh * G) * D + i] = qnan;
+    if (tid < G) p.lse[(size_t)b * p.Hq + kvh * G + tid] = qnan;
+    if (tid == 0) {
+      atomicOr(p.status, s_plan.bad ? MAC_DEV_BAD_SEQ_LEN : MAC_DEV_BAD_PAGE);
+      if (p.hit_mask) p.hit_mask[u] = 0;
+      if (p.match_pos) p.match_pos[u] = -1;
+      UnitPlan pl = s_plan;
+      pl.bad = 1;
+      pl.hit = 0;
+      p.plan[u] = pl;
+    }
+  } else {
+    // 4. RoPE in fp64: pair i couples elements i and i + D/2
+    const double scale = kLog2e / sqrt((double)D);
+    const double pos = (double)p.rope_pos[b];
+    for (int i = tid; i < D / 2; i += kMatchThreads) {
+      double sn, cs;
+      sincos(pos * p.inv_freq[i], &sn, &cs);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const double x = sq[h * D + i], y = sq[h * D + i + D / 2];
+        float* dst = p.qrot + ((size_t)u * G + h) * D;
+        dst[i] = (float)((x * cs - y * sn) * scale);
+        dst[i + D / 2] = (float)((y * cs + x * sn) * scale);
+      }
+    }
+    // 5. this step's query enters the ring
+    float4* rdst = reinterpret_cast<float4*>(p.ring_q + ((size_t)u * Wp1 + s_plan.dst_slot) * GD);
+    for (int i = tid; i < GD / 4; i += kMatchThreads) rdst[i] = reinterpret_cast<const float4*>(sq)[i];
+    if (tid == 0) {
+      p.steps[u] = n + 1;
+      if (p.hit_mask) p.hit_mask[u] = (uint8_t)s_plan.hit;
+      if (p.match_pos) p.match_pos[u] = spos[0];
+      p.plan[u] = s_plan;
+    }
+  }
+
+  // last CTA to arrive builds the segment table for the attention kernel
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int ticket = atomicAdd(p.done, 1);
+    s_last = (ticket == (int)gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  build_segments(p, (int)gridDim.x);
+  if (tid == 0) *p.done = 0;
+}
+
+}  // namespace
+
+cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s) {
+  const int U = p.B * p.Hkv;
+  if (D == 128) {
+    mac_match_kernel<128><<<U, kMatchThreads, 0, s>>>(p);
+  } else if (D == 64) {
+    mac_match_kernel<64><<<U, kMatchThreads, 0, s>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mac

@@ -1,0 +1,52 @@
+"""The C ABI library builds for sm_100a, loads without a GPU and exports every
+entry point include/mac.h declares; the binding refuses to run without it."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "mac.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mac_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_reuse_b200 import build
+    build.build()
+    import kv_cache_reuse_b200 as mac
+    return mac.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_declares_every_symbol():
+    from kv_cache_reuse_b200._native import SIGNATURES
+    assert sorted(SIGNATURES) == _declared()
+
+
+def test_error_strings(lib):
+    import kv_cache_reuse_b200 as mac
+    assert mac.mac_error_string(mac.MAC_OK) == "ok"
+    assert "status" in mac.mac_error_string(mac.MAC_ERR_DEVICE)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from kv_cache_reuse_b200 import _native
+    with pytest.raises(ImportError):
+        _native._lib_backup = _native._lib
+        try:
+            _native._lib = None
+            _native.load(str(tmp_path / "nope.so"))
+        finally:
+            _native._lib = _native._lib_backup
+

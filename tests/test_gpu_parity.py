@@ -1,0 +1,252 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (libmac_b200.so).
+
+Bar (MAC-Attention, page 1, with this library's readings): hit/miss flags and
+matched positions bit-exact; out within 2e-3 max-abs; lse within 1e-3.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.dense_ref import load_hand_example
+from tests.gpu_harness import LSE_TOL, OUT_TOL, GpuRun, compare_stream, torch_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def test_hand_worked_example_on_gpu():
+    g, K, V, qs = load_hand_example()
+    sh = g["shape"]
+    wl = synth.Workload(name="hand", B=1, Hq=sh["Hq"], Hkv=sh["Hkv"], D=sh["D"], L0=(3,), steps=2, W=sh["W"],
+                        band=sh["band"], tau=sh["tau"], sigma=0.0, rope_theta=sh["rope_theta"], page_size=0,
+                        hit_model=("iid", 0.0), seed=0)
+    cache = synth.KVCache(K, V, None, sh["max_seq"], 0)
+    gpu = GpuRun(wl, cache)
+    for st, q in zip(g["steps"], qs):
+        out, lse, hit, mpos = gpu.step(q, np.array([st["rope_pos"]], np.int32), np.array([st["seq_len"]], np.int32))
+        assert int(hit[0, 0]) == st["hit"] and int(mpos[0, 0]) == st["match_pos"]
+        np.testing.assert_allclose(out[0, :, 0], st["out0"], atol=1e-5)
+        np.testing.assert_allclose(out[0, :, 1], st["out1"], atol=1e-5)
+        assert np.abs(out[0, :, 2:]).max() == 0.0
+        np.testing.assert_allclose(lse[0], st["lse"], atol=1e-5)
+
+
+def test_tiny_stream():
+    wl = synth.WORKLOADS["tiny"]
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl))
+    assert r["hits"] > 10
+
+
+def test_tiny_all_miss_equals_dense():
+    wl = synth.WORKLOADS["tiny"]
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=0.0)
+    assert r["hits"] == 0
+
+
+def test_llama8b_32k_stream():
+    wl = synth.WORKLOADS["llama8b_32k"]
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl))
+    assert r["hits"] > 100
+
+
+@pytest.mark.slow
+def test_long_128k_stream_full():
+    """The benchmark's workload at full size, every step, in the bench's launch configuration."""
+    wl = synth.WORKLOADS["long_128k"]
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl))
+    assert r["hits"] > 300
+
+
+@pytest.mark.slow
+def test_long_128k_all_miss_steps():
+    wl = synth.WORKLOADS["long_128k"]
+    compare_stream(wl, synth.queries(wl, 4), synth.kv_cache(wl, 4), tau=0.0)
+
+
+def test_paged_mixed_stream():
+    wl = synth.WORKLOADS["paged_mixed"]
+    steps = 24
+    compare_stream(wl, synth.queries(wl, steps), synth.kv_cache(wl, steps))
+
+
+def test_paged_equals_contiguous_bitwise():
+    """The same keys in contiguous and paged layouts give identical bits (chunking is by logical key)."""
+    wl = synth.WORKLOADS["paged_mixed"].with_(B=4, L0=(3000, 777, 4100, 1601), steps=16)
+    stream = synth.queries(wl)
+    paged = synth.kv_cache(wl)
+    cap = paged.max_seq
+    Kc = np.zeros((wl.B, cap, wl.Hkv, wl.D), np.uint16)
+    Vc = np.zeros_like(Kc)
+    ps = wl.page_size
+    for b in range(wl.B):
+        n = int(np.sum(paged.block_table[b] >= 0))
+        pages = paged.block_table[b, :n]
+        Kc[b, :n * ps] = paged.K[pages].reshape(n * ps, wl.Hkv, wl.D)
+        Vc[b, :n * ps] = paged.V[pages].reshape(n * ps, wl.Hkv, wl.D)
+    contig = synth.KVCache(Kc, Vc, None, cap, 0)
+    wc = wl.with_(page_size=0)
+    g1 = GpuRun(wl, paged)
+    g2 = GpuRun(wc, contig)
+    for t in range(wl.steps):
+        a = g1.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        b = g2.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        for x, y in zip(a, b):
+            np.testing.assert_array_equal(x, y)
+
+
+def test_continuous_append_stream():
+    """Paged cache filled one row per step through mac_append_kv, ring updated every step."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["continuous_16k"]
+    steps = 96
+    stream = synth.queries(wl, steps)
+    cache = synth.kv_cache(wl, steps)
+    torch, dev = torch_dev()
+    # device pool with every decode-step row poisoned (NaN) until appended
+    Kd = torch.from_numpy(cache.K.view(np.int16)).to(dev)
+    Vd = torch.from_numpy(cache.V.view(np.int16)).to(dev)
+    ps = wl.page_size
+    for b in range(wl.B):
+        for pos in range(wl.L0[b], wl.L0[b] + steps):
+            pg = int(cache.block_table[b, pos // ps])
+            Kd[pg, pos % ps] = 0x7FC0
+            Vd[pg, pos % ps] = 0x7FC0
+    gpu = GpuRun(wl, cache, K_dev=Kd, V_dev=Vd)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    knew = torch.empty((wl.B, wl.Hkv, wl.D), dtype=torch.int16, device=dev)
+    vnew = torch.empty_like(knew)
+    for t in range(steps):
+        kr, vr = synth.step_rows(cache, stream.seq_lens[t])
+        knew.copy_(torch.from_numpy(kr.view(np.int16)))
+        vnew.copy_(torch.from_numpy(vr.view(np.int16)))
+        gpu.lens.copy_(torch.from_numpy(stream.seq_lens[t]))
+        mac.mac_append_kv(gpu.st, Kd, Vd, gpu.bt, gpu.lens, knew, vnew)
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+        out, lse, hit, mpos = gpu.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_array_equal(hit, r.hit)
+        np.testing.assert_array_equal(mpos, r.match_pos)
+        assert np.abs(out - r.out).max() <= OUT_TOL
+        assert np.abs(lse - r.lse).max() <= LSE_TOL
+    assert gpu.st.get_status() == 0
+
+
+def test_ring_state_matches_oracle_window():
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(steps=40)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    r = compare_stream(wl, stream, cache)
+    gpu, orc = r["gpu"], r["oracle"]
+    st = mac.parse_state(gpu.st.export_state(), wl.W, wl.G, wl.D)
+    W1 = wl.W + 1
+    n = int(st["steps"][0])
+    assert n == wl.steps
+    q_o, o_o, m_o, l_o, pos_o = orc.window(0)
+    for age in range(wl.W):  # oracle window is oldest first
+        slot = (n - 1 - age) % W1
+        e = len(pos_o) - 1 - age
+        assert st["pos"][0, slot] == pos_o[e]
+        np.testing.assert_array_equal(st["q"][0, slot], q_o[e])
+        np.testing.assert_allclose(st["o"][0, slot], o_o[e], atol=OUT_TOL)
+        lse_g = st["m"][0, slot] + np.log(st["l"][0, slot])
+        np.testing.assert_allclose(lse_g, m_o[e] + np.log(l_o[e]), atol=LSE_TOL)
+
+
+def test_export_import_resumes_identically():
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(steps=30)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    a = GpuRun(wl, cache)
+    for t in range(15):
+        a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+    buf = a.st.export_state()
+    b = GpuRun(wl, cache)
+    b.st.import_state(buf)
+    for t in range(15, 30):
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        y = b.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        for u, v in zip(x, y):
+            np.testing.assert_array_equal(u, v)
+
+
+def test_host_entry_matches_device_entry():
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(steps=20)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    a = GpuRun(wl, cache)
+    b = GpuRun(wl, cache)
+    torch = a.torch
+    out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32).pin_memory()
+    lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+    hit_h = torch.empty((wl.B, wl.Hkv), dtype=torch.uint8).pin_memory()
+    mp_h = torch.empty((wl.B, wl.Hkv), dtype=torch.int32).pin_memory()
+    for t in range(wl.steps):
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        q_h = torch.from_numpy(stream.q[t]).pin_memory()
+        p_h = torch.from_numpy(stream.rope_pos[t]).pin_memory()
+        l_h = torch.from_numpy(stream.seq_lens[t]).pin_memory()
+        rc = mac.mac_decode_step_host(b.st, q_h, p_h, l_h, None, None, b.K, b.V, None, out_h, lse_h, hit_h, mp_h)
+        assert rc == mac.MAC_OK
+        for u, v in zip(x, (out_h.numpy(), lse_h.numpy(), hit_h.numpy(), mp_h.numpy())):
+            np.testing.assert_array_equal(u, v)
+
+
+@pytest.mark.parametrize("case", ["one_key", "band0", "window1", "ragged", "full_capacity", "band_covers", "d128_short"])
+def test_edge_cases(case):
+    base = synth.WORKLOADS["tiny"]
+    kw = {}
+    if case == "one_key":
+        kw = dict(L0=(0,), steps=12)  # first step sees a single key
+    elif case == "band0":
+        kw = dict(band=0, steps=32)
+    elif case == "window1":
+        kw = dict(W=1, steps=32)
+    elif case == "ragged":
+        kw = dict(L0=(1013,), steps=20)
+    elif case == "full_capacity":
+        kw = dict(L0=(500,), steps=12)
+    elif case == "band_covers":
+        kw = dict(L0=(40,), band=500, steps=24)
+    elif case == "d128_short":
+        base = synth.WORKLOADS["llama8b_32k"]
+        kw = dict(L0=(37,), steps=40, W=8)
+    wl = base.with_(**kw)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)  # capacity = L0 + steps exactly: the last step fills it
+    compare_stream(wl, stream, cache)
+
+
+def test_nan_query_misses_and_stays_local():
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, L0=(700, 900), steps=6)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    gpu = GpuRun(wl, cache)
+    for t in range(wl.steps):
+        q = stream.q[t].copy()
+        if t == 4:
+            q[1, 5, 3] = np.nan  # KV head 1 of sequence 1
+        out, lse, hit, mpos = gpu.step(q, stream.rope_pos[t], stream.seq_lens[t])
+        if t == 4:
+            assert hit[1, 1] == 0 and mpos[1, 1] == -1
+            assert np.isnan(out[1, 4:8]).all()
+            assert np.isfinite(out[0]).all() and np.isfinite(out[1, :4]).all() and np.isfinite(out[1, 8:]).all()
+    assert gpu.st.get_status() == 0
+
+
+def test_bad_page_and_seq_len_flagged():
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["paged_mixed"].with_(B=3, L0=(100, 200, 300), steps=3)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    bt = cache.block_table.copy()
+    bt[1, 2] = cache.num_pages + 5  # sequence 1 reads its page 2 at every step
+    bad = synth.KVCache(cache.K, cache.V, bt, cache.max_seq, cache.num_pages)
+    gpu = GpuRun(wl, bad)
+    out, lse, hit, mpos = gpu.step(stream.q[0], stream.rope_pos[0], stream.seq_lens[0])
+    assert np.isnan(out[1]).all() and np.isnan(lse[1]).all()
+    assert np.isfinite(out[0]).all() and np.isfinite(out[2]).all()
+    assert gpu.st.get_status() == mac.MAC_DEV_BAD_PAGE
+    lens = stream.seq_lens[1].copy()
+    lens[2] = bad.max_seq + 1
+    out, lse, hit, mpos = gpu.step(stream.q[1], stream.rope_pos[1], lens)
+    assert np.isnan(out[2]).all()
+    st = gpu.st.get_status()
+    assert st & mac.MAC_DEV_BAD_SEQ_LEN and st & mac.MAC_DEV_BAD_PAGE
+    assert gpu.st.get_status() == 0  # cleared by the read
