@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the MAC-Attention decode step on B200.
+
+A step is one mac_decode_step (match + amend/complete/miss + merge) over all
+B sequences of one attention layer, on the 128K-context workload
+(B=4, 32 query / 8 KV heads, D=128, bf16 contiguous KV, W=32, band=256, 90%
+of queries near-repeats of a recent one).  Inputs are seeded synthetic data of
+that shape (synth.WORKLOADS["long_128k"]).  L2 is flushed (256 MiB write)
+between timed steps.
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+batch of the workload (independent problems, no collective on the data path),
+so scaling is weak and value = all ranks' steps / max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MAC decode-attention steps/s at 128K ctx"
+UNIT = "steps/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("mac_attend.cu", "mac_internal.cuh"):
+        with open(os.path.join(ROOT, "kv_cache_reuse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "mac_attend_long_128k_traffic.txt")
+    try:
+        txt = open(p).read()
+    except OSError:
+        return None
+    m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+    b = re.search(r"dram_bytes_per_launch_scaled:\s*([0-9.eE+]+)", txt)
+    if not m or not b or m.group(1) != _kernel_hash():
+        return None
+    return float(b.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML during the timed region."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b],
+                "samples": len(self.samples)}
+
+
+def step_bytes(wl, hit, mpos, seq_lens, occ):
+    """Algorithmic HBM bytes of one step: (match kernel, attention kernel, K/V only).
+
+    Match: query G*D*4 per unit, window scan occ*G*D*4, ring-q write and rotated
+    query write G*D*4 each.  Attention: K+V of every key attended fresh
+    (2*D*2 per key), rotated query G*D*4, reused state G*(D+2)*4 on a hit, new
+    state G*(D+2)*4 + position, out and lse G*(D+1)*4.
+    """
+    G, D, band = wl.G, wl.D, wl.band
+    gd4 = G * D * 4
+    kv = att = mt = 0
+    for b in range(wl.B):
+        p_t = int(seq_lens[b]) - 1
+        for h in range(wl.Hkv):
+            start = max(0, int(mpos[b, h]) - band) if hit[b, h] else 0
+            keys = p_t + 1 - start
+            kv += keys * 2 * D * 2
+            att += gd4 + (G * (D + 2) * 4 if hit[b, h] else 0) + G * (D + 2) * 4 + 4 + G * (D + 1) * 4
+            mt += gd4 + occ * gd4 + 2 * gd4
+    return mt, att + kv, kv
+
+
+def run_mac(args, rank, world, local_rank):
+    import torch
+    import kv_cache_reuse_b200 as mac
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    base = synth.WORKLOADS[args.workload]
+    wl = base.with_(seed=base.seed + 1000 * rank)  # every rank: its own batch
+    T = max(base.steps, args.warmup + args.steps)
+    stream = synth.queries(wl, T)
+    cache = synth.kv_cache(wl, T)
+    K = torch.from_numpy(cache.K.view(np.int16)).to(dev)
+    V = torch.from_numpy(cache.V.view(np.int16)).to(dev)
+    bt = None if not cache.paged else torch.from_numpy(cache.block_table).to(dev)
+    kw = dict(max_pages_per_seq=cache.block_table.shape[1], num_pages=cache.num_pages) if cache.paged else \
+        dict(capacity=cache.max_seq)
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    q_all = torch.from_numpy(stream.q).to(dev)
+    pos_all = torch.from_numpy(stream.rope_pos).to(dev)
+    lens_all = torch.from_numpy(stream.seq_lens).to(dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    hit_all = torch.zeros((T, B, Hkv), dtype=torch.uint8, device=dev)
+    mpos_all = torch.zeros((T, B, Hkv), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    s = torch.cuda.current_stream(dev)
+    peak, peak_kind = _peaks()
+
+    def timed_run(tau, nwarm, nsteps):
+        st = mac.MacState.for_workload(wl, tau=tau, **kw)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+        for t in range(nwarm):
+            st.decode_step(q_all[t], pos_all[t], K, V, bt, lens_all[t], out, lse, hit_all[t], mpos_all[t], s)
+            flush.zero_()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        clocks = ClockSampler(local_rank)
+        with clocks:
+            for i in range(nsteps):
+                t = nwarm + i
+                e0, e1, e2 = ev[i]
+                e0.record(s)
+                mac.mac_match(st, q_all[t], pos_all[t], bt, lens_all[t], out, lse, hit_all[t], mpos_all[t], s)
+                e1.record(s)
+                mac.mac_attend(st, K, V, bt, out, lse, s)
+                e2.record(s)
+                flush.zero_()
+            torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        status = st.get_status()
+        st.close()
+        step_ms = [a.elapsed_time(c) for a, b_, c in ev]
+        att_ms = [b_.elapsed_time(c) for a, b_, c in ev]
+        match_ms = [a.elapsed_time(b_) for a, b_, c in ev]
+        hits = hit_all[nwarm:nwarm + nsteps].cpu().numpy()
+        mpos = mpos_all[nwarm:nwarm + nsteps].cpu().numpy()
+        mt_b = at_b = kv_b = dense_b = 0
+        for i in range(nsteps):
+            t = nwarm + i
+            occ = min(t, wl.W)
+            a, b_, c = step_bytes(wl, hits[i], mpos[i], stream.seq_lens[t], occ)
+            mt_b += a
+            at_b += b_
+            kv_b += c
+            dense_b += synth.dense_equiv_kv_bytes(wl, stream.seq_lens[t])
+        tot_ms = float(np.sum(step_ms))
+        return dict(total_ms=tot_ms, step_ms=step_ms, att_ms=float(np.sum(att_ms)), match_ms=float(np.sum(match_ms)),
+                    att_bytes=at_b, match_bytes=mt_b, kv_bytes=kv_b, dense_bytes=dense_b,
+                    hit_frac=float(hits.mean()), status=status, clocks=clocks.summary())
+
+    main = timed_run(wl.tau, args.warmup, args.steps)
+    allmiss = timed_run(0.0, 3, min(args.miss_steps, T - 3)) if args.miss_steps > 0 else None
+
+    # max over ranks of the timed duration
+    tot = main["total_ms"]
+    if world > 1:
+        tt = torch.tensor([tot], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        tot = float(tt.item())
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, stream, cache, K, V, bt, kw, dev, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(wl, stream, cache, args.cpu_seconds)
+
+    if rank != 0:
+        return None
+    K_ = args.steps
+    att_gbs = main["att_bytes"] / (main["att_ms"] * 1e-3) / 1e9
+    traffic = _profiled_traffic()
+    res = {
+        "metric": METRIC, "value": world * K_ / (tot * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K_,
+        "warmup": args.warmup, "ms_per_step": tot / K_, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.D,
+                   "context": int(wl.L0[0]), "window": wl.W, "band": wl.band, "tau": wl.tau,
+                   "hit_label_rate": wl.hit_model[1], "kv": "bf16 %s" % ("paged" if cache.paged else "contiguous"),
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas" if world > 1 else "1 GPU"},
+        "roofline": {"bound": "hbm", "kernel": "mac_attend_kernel", "achieved": att_gbs, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": att_gbs / peak,
+                     "traffic": traffic},
+        "hit_fraction": main["hit_frac"],
+        "match_kernel_gbs": main["match_bytes"] / (main["match_ms"] * 1e-3) / 1e9,
+        "step_gbs": (main["att_bytes"] + main["match_bytes"]) / (main["total_ms"] * 1e-3) / 1e9,
+        "effective_kv_gbs": main["dense_bytes"] / (main["total_ms"] * 1e-3) / 1e9,
+        "kv_bytes_per_step": main["kv_bytes"] / K_, "dense_kv_bytes_per_step": main["dense_bytes"] / K_,
+        "gpu_launches": 2 * K_ * world,
+        "clocks": main["clocks"],
+        "device_status": main["status"],
+    }
+    if allmiss:
+        n = len(allmiss["step_ms"])
+        a_gbs = allmiss["att_bytes"] / (allmiss["att_ms"] * 1e-3) / 1e9
+        res["all_miss"] = {"steps": n, "steps_per_s": n / (allmiss["total_ms"] * 1e-3),
+                           "ms_per_step": allmiss["total_ms"] / n, "attend_gbs": a_gbs, "attend_frac": a_gbs / peak,
+                           "speedup_of_mac": (world * K_ / (tot * 1e-3)) / (n / (allmiss["total_ms"] * 1e-3)),
+                           "clocks": allmiss["clocks"]}
+    if e2e:
+        res["e2e"] = e2e
+    if cpu:
+        res["cpu_baseline"] = cpu
+    return res
+
+
+def run_e2e(args, wl, stream, cache, K, V, bt, kw, dev, world):
+    """Same steps through mac_decode_step_host: pinned host inputs (query, positions,
+    the step's own K/V rows) copied in, out/lse/hit/match read back, every step."""
+    import torch
+    import kv_cache_reuse_b200 as mac
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    st = mac.MacState.for_workload(wl, **kw)
+    s = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    T = args.warmup + args.steps
+    q_h = [torch.from_numpy(stream.q[t]).pin_memory() for t in range(T)]
+    p_h = [torch.from_numpy(stream.rope_pos[t]).pin_memory() for t in range(T)]
+    l_h = [torch.from_numpy(stream.seq_lens[t]).pin_memory() for t in range(T)]
+    rows = [synth.step_rows(cache, stream.seq_lens[t]) for t in range(T)]
+    k_h = [torch.from_numpy(r[0].view(np.int16)).pin_memory() for r in rows]
+    v_h = [torch.from_numpy(r[1].view(np.int16)).pin_memory() for r in rows]
+    out_h = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    lse_h = torch.empty((B, Hq), dtype=torch.float32).pin_memory()
+    hit_h = torch.empty((B, Hkv), dtype=torch.uint8).pin_memory()
+    mp_h = torch.empty((B, Hkv), dtype=torch.int32).pin_memory()
+    tot = 0.0
+    for t in range(T):
+        flush.zero_()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        rc = mac.mac_decode_step_host(st, q_h[t], p_h[t], l_h[t], k_h[t], v_h[t], K, V, bt, out_h, lse_h, hit_h,
+                                      mp_h, s)
+        t1 = time.perf_counter()
+        if rc != mac.MAC_OK:
+            raise RuntimeError("device status %d in e2e step" % mac.mac_get_status(st))
+        if t >= args.warmup:
+            tot += t1 - t0
+    st.close()
+    if world > 1:
+        tt = torch.tensor([tot], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        tot = float(tt.item())
+    h2d = B * Hq * D * 4 + 2 * B * 4 + 2 * B * Hkv * D * 2
+    d2h = B * Hq * D * 4 + B * Hq * 4 + B * Hkv + B * Hkv * 4 + 4
+    return {"value": world * args.steps / tot, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "timer": "host wall clock around each mac_decode_step_host call (it synchronises)"}
+
+
+def run_cpu_baseline(wl, stream, cache, seconds):
+    """The fp64 oracle on the host cores, on the first steps of the same stream
+    (bounded to about `seconds` of CPU work)."""
+    import oracle
+    orc = oracle.Oracle.for_workload(wl, cache)
+    t0 = time.perf_counter()
+    n = nh = 0
+    while n < stream.q.shape[0]:
+        r = orc.step(stream.q[n], stream.rope_pos[n], cache.K, cache.V, cache.block_table, stream.seq_lens[n])
+        nh += int(r.hit.sum())
+        n += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "first %d decode steps of %s from an empty window (%d of %d unit decisions hit), %.1f s" % (
+                n, wl.name, nh, n * wl.B * wl.Hkv, dt)}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return None
+    import oracle
+    wl = synth.WORKLOADS[args.workload]
+    T = max(wl.steps, args.warmup + args.steps)
+    stream = synth.queries(wl, T)
+    cache = synth.kv_cache(wl, T)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    for t in range(args.warmup):
+        orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+    t0 = time.perf_counter()
+    n = 0
+    for t in range(args.warmup, args.warmup + args.steps):
+        orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+        n += 1
+        if time.perf_counter() - t0 > args.cpu_seconds * 6:
+            break
+    dt = time.perf_counter() - t0
+    v = n / dt
+    sample = "decode steps %d..%d of %s (fp64 oracle, every unit of every step)" % (args.warmup, args.warmup + n - 1,
+                                                                                    wl.name)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": n,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / n, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.D,
+                       "context": int(wl.L0[0]), "window": wl.W, "band": wl.band},
+            "cpu_baseline": {"value": v, "unit": UNIT, "kind": "oracle", "cores": oracle.num_threads(),
+                             "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=120)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="mac", choices=["mac", "reference"])
+    ap.add_argument("--workload", default="long_128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--miss-steps", type=int, default=16, help="timed steps of the all-miss run (0 = skip)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            import torch
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        res = run_mac(args, rank, world, local_rank)
+        if world > 1:
+            import torch
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()
