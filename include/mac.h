@@ -173,9 +173,14 @@ size_t mac_state_bytes(const MacState *st);
 int mac_export_state(const MacState *st, void *host_buf, size_t bytes);
 int mac_import_state(MacState *st, const void *host_buf, size_t bytes);
 
-/* Tuning: minimum keys one CTA of the attention kernel takes (default 128).
- * Smaller values spread short (hit) steps over more SMs. */
+/* Tuning of the work split of the attention kernel.  The key ranges of all
+ * units are laid end to end in a cost space where every non-empty range also
+ * weighs a fixed per-piece cost (in keys; default 1024) and the space is
+ * split evenly over min(grid, ceil(total / min_keys)) CTAs (min_keys default
+ * 128).  A larger piece cost spreads many short (hit) ranges over more CTAs
+ * when a batch also holds long (miss) ranges. */
 int mac_set_min_keys_per_cta(MacState *st, int keys);
+int mac_set_piece_cost(MacState *st, int keys);
 
 /* Persistent grid size of the attention kernel (CTAs). */
 int mac_attend_grid(const MacState *st);

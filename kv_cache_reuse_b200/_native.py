@@ -26,6 +26,7 @@ SIGNATURES = {
     "mac_export_state": (C.c_int, [_P, _P, C.c_size_t]),
     "mac_import_state": (C.c_int, [_P, _P, C.c_size_t]),
     "mac_set_min_keys_per_cta": (C.c_int, [_P, C.c_int]),
+    "mac_set_piece_cost": (C.c_int, [_P, C.c_int]),
     "mac_attend_grid": (C.c_int, [_P]),
     "mac_error_string": (C.c_char_p, [C.c_int]),
 }

@@ -18,7 +18,7 @@ using namespace mac;
 
 struct MacState {
   MacConfig cfg;
-  int G, U, D, W, device, num_sms, grid, min_keys, capacity;
+  int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, capacity;
   size_t max_parts;
   // ring (library-owned state)
   float* ring_q = nullptr;
@@ -195,6 +195,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   s->D = cfg->head_dim;
   s->W = cfg->window;
   s->min_keys = 128;
+  s->piece_cost = 1024;
   s->capacity = cfg->page_size == 0 ? cfg->max_seq : cfg->max_pages_per_seq * cfg->page_size;
   if (cudaGetDevice(&s->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&s->num_sms, cudaDevAttrMultiProcessorCount, s->device) != cudaSuccess) {
@@ -283,6 +284,12 @@ int mac_set_min_keys_per_cta(MacState* s, int keys) {
   return MAC_OK;
 }
 
+int mac_set_piece_cost(MacState* s, int keys) {
+  if (!s || keys < 0) return MAC_ERR_ARG;
+  s->piece_cost = keys;
+  return MAC_OK;
+}
+
 int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
 
 int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
@@ -321,6 +328,7 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.tau = s->cfg.tau;
   p.grid = s->grid;
   p.min_keys = s->min_keys;
+  p.piece_cost = s->piece_cost;
   return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 

@@ -314,6 +314,7 @@ __device__ void merge_unit(const AttendParams& p, int u) {
       ro = p.ring_o[rs * GD + idx];
       M = rm;
     }
+#pragma unroll 4
     for (int i = 0; i < sA.npieces; ++i) M = fmaxf(M, __ldcg(p.part + (size_t)(sA.pbase + i) * PF + GD + h));
     const float Mu = M == -INFINITY ? 0.f : M;
     float L = 0.f, O = 0.f;
@@ -322,6 +323,7 @@ __device__ void merge_unit(const AttendParams& p, int u) {
       L += rl * a;
       O += ro * rl * a;
     }
+#pragma unroll 4
     for (int i = 0; i < sA.npieces; ++i) {
       const float* pp = p.part + (size_t)(sA.pbase + i) * PF;
       const float a = ex2(__ldcg(pp + GD + h) - Mu);
@@ -336,10 +338,12 @@ __device__ void merge_unit(const AttendParams& p, int u) {
     }
     // output: new prefix state + tail partials
     float M2 = M;
+#pragma unroll 4
     for (int i = 0; i < sB.npieces; ++i) M2 = fmaxf(M2, __ldcg(p.part + (size_t)(sB.pbase + i) * PF + GD + h));
     const float M2u = M2 == -INFINITY ? 0.f : M2;
     const float a0 = ex2(M - M2u);
     float L2 = L * a0, O2 = O * a0;
+#pragma unroll 4
     for (int i = 0; i < sB.npieces; ++i) {
       const float* pp = p.part + (size_t)(sB.pbase + i) * PF;
       const float a = ex2(__ldcg(pp + GD + h) - M2u);
@@ -458,14 +462,15 @@ struct Walker {
   __device__ __forceinline__ bool next(const AttendParams& p, int cta, Piece& pc) {
     while (s < p.nseg) {
       const Segment sg = p.seg[s];
-      if (sg.flat >= hi) {
+      const int cur = s++;
+      if (sg.len == 0) continue;
+      if (sg.flat >= hi) {  // this and every later segment start past the range
         s = p.nseg;
         return false;
       }
-      const int cur = s++;
-      if (sg.len == 0) continue;
       const long long fa = lo > sg.flat ? lo : sg.flat;
       const long long fe = hi < sg.flat + sg.len ? hi : sg.flat + sg.len;
+      if (fa >= fe) continue;  // the range holds only this segment's padding, or ends before it
       pc.unit = cur >> 1;
       pc.pidx = sg.pbase + (cta - sg.first_cta);
       pc.k0 = sg.key0 + (int)(fa - sg.flat);
@@ -486,9 +491,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  const int n_cta = p.hdr->n_cta;
   const int cta = blockIdx.x;
-  if (cta >= n_cta) return;
   if (tid == 0) {
     for (int w = 0; w < kConsumerWarps; ++w)
       for (int s = 0; s < NST; ++s) mbar_init(&sm.full[w][s], 1);
@@ -499,6 +502,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // launched with programmatic stream serialization: everything above
+  // overlaps the match kernel; its results are visible after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int n_cta = p.hdr->n_cta;
+  if (cta >= n_cta) return;
 
   const long long T = p.hdr->total;
   const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
@@ -651,13 +659,27 @@ cudaError_t attend_prepare(int D) {
 }
 
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s) {
-  if (D == 128)
-    mac_attend_kernel<128><<<grid, kAttnThreads, sizeof(AttnSmem<128>), s>>>(p);
-  else if (D == 64)
-    mac_attend_kernel<64><<<grid, kAttnThreads, sizeof(AttnSmem<64>), s>>>(p);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  // Programmatic stream serialization: the kernel may be scheduled while the
+  // preceding match kernel drains; it calls griddepcontrol.wait before it
+  // reads anything that kernel wrote.
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) {
+    cfg.dynamicSmemBytes = sizeof(AttnSmem<128>);
+    return cudaLaunchKernelEx(&cfg, mac_attend_kernel<128>, p);
+  }
+  if (D == 64) {
+    cfg.dynamicSmemBytes = sizeof(AttnSmem<64>);
+    return cudaLaunchKernelEx(&cfg, mac_attend_kernel<64>, p);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace mac

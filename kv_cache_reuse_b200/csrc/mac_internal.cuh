@@ -30,19 +30,23 @@ struct UnitPlan {
 
 // Two key segments per unit: 2u = [start, cut) (into the new prefix state),
 // 2u+1 = [cut, end) (tail, into the output only).  The segments of all units
-// are laid end to end ("flattened") and split evenly over the CTAs.
+// are laid end to end ("flattened") in a cost space where a non-empty
+// segment weighs piece_cost + len (the fixed cost of a piece -- query load,
+// combine, merge -- expressed in keys), and that space is split evenly over
+// the CTAs.  A segment's keys occupy [flat, flat + len) of the space, after
+// its piece_cost of padding.
 struct Segment {
-  long long flat;  // offset in the flattened key space
+  long long flat;  // cost-space offset of the segment's first key
   int len;         // keys
   int key0;        // first key (absolute position in the sequence)
-  int first_cta;   // CTA holding key `flat`
+  int first_cta;   // CTA holding cost offset `flat`
   int pbase;       // index of this segment's first partial result
   int npieces;     // partial results (CTAs overlapping the segment)
   int pad;
 };
 
 struct PlanHeader {
-  long long total;  // keys in the flattened space
+  long long total;  // size of the flattened cost space
   int n_cta;        // CTAs with work (<= grid)
   int pad;
 };
@@ -73,7 +77,8 @@ struct MatchParams {
   int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;
   float tau;
   int grid;       // CTAs of the attention kernel
-  int min_keys;   // minimum keys per attention CTA
+  int min_keys;   // minimum cost-space units per attention CTA
+  int piece_cost; // fixed cost of one piece, in keys
 };
 
 struct AttendParams {

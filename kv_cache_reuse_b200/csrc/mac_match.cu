@@ -18,9 +18,12 @@
 //      log2(e)/sqrt(D) so the attention kernel works in exp2 units;
 //   5. the query enters the ring slot n mod (W+1) (W+1 slots: the slot
 //      written is never one the window can read this step).
-// The last CTA to finish lays every unit's two key segments end to end and
-// splits the total evenly over the attention kernel's CTAs (no CTA waits
-// for another: the last arrival does the work).
+// The last CTA to finish lays every unit's two key segments end to end in a
+// cost space (each non-empty segment weighs its keys plus a fixed per-piece
+// cost) and splits that space evenly over the attention kernel's CTAs, so a
+// batch mixing short hit ranges with whole-context misses is balanced by
+// time rather than by keys.  No CTA waits for another: the last arrival
+// does the work.
 #include <math.h>
 #include <stdint.h>
 
@@ -32,6 +35,9 @@ namespace mac {
 namespace {
 
 constexpr double kLog2e = 1.4426950408889634;
+constexpr double kInvTwoPi = 0.15915494309189535;
+constexpr double kTwoPiHi = 6.2831853069365025;    // 2*pi with the low 21 mantissa bits cleared
+constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -66,8 +72,8 @@ __device__ long long block_exclusive_scan(long long v, long long* total, long lo
   return before + x - v;
 }
 
-// CTA holding flattened key x when T keys are split over N CTAs as
-// [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
+// CTA holding cost-space offset x when the space [0, T) is split over N CTAs
+// as [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
 __device__ __forceinline__ int cta_of(long long x, long long T, int N) {
   return (int)(((x + 1) * (long long)N + T - 1) / T) - 1;
 }
@@ -80,6 +86,7 @@ __device__ void build_segments(const MatchParams& p, int U) {
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
     int len = 0, key0 = 0;
+    long long wlen = 0;
     if (s < nseg) {
       const UnitPlan* pl = p.plan + (s >> 1);
       const int bad = __ldcg(&pl->bad);
@@ -87,12 +94,13 @@ __device__ void build_segments(const MatchParams& p, int U) {
         const int start = __ldcg(&pl->start), cut = __ldcg(&pl->cut), end = __ldcg(&pl->end);
         len = (s & 1) ? end - cut : cut - start;
         key0 = (s & 1) ? cut : start;
+        wlen = len > 0 ? (long long)len + p.piece_cost : 0;
       }
     }
     long long tot;
-    long long ex = block_exclusive_scan(len, &tot, sbuf);
+    long long ex = block_exclusive_scan(wlen, &tot, sbuf);
     if (s < nseg) {
-      p.seg[s].flat = carry + ex;
+      p.seg[s].flat = carry + ex + (len > 0 ? p.piece_cost : 0);
       p.seg[s].len = len;
       p.seg[s].key0 = key0;
     }
@@ -147,6 +155,9 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   __shared__ int s_bad_page, s_last;
   __shared__ UnitPlan s_plan;
 
+  // the attention kernel (launched with programmatic stream serialization)
+  // may start its prologue now; it waits for this grid before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int u = blockIdx.x;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -161,25 +172,47 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   if (tid == 0) s_bad_page = 0;
   __syncthreads();
 
-  // 1. distances to the window entries, newest first (age j = 0 is step n-1)
-  for (int j = warp; j < occ; j += kMatchThreads / 32) {
-    const int slot = (n - 1 - j) % Wp1;
-    const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
-    float acc = 0.f;
-    for (int i = lane; i < GD / 4; i += 32) {
-      const float4 r = rq[i];
-      const float4 q = reinterpret_cast<const float4*>(sq)[i];
-      const float dx = q.x - r.x, dy = q.y - r.y, dz = q.z - r.z, dw = q.w - r.w;
-      acc = fmaf(dx, dx, acc);
-      acc = fmaf(dy, dy, acc);
-      acc = fmaf(dz, dz, acc);
-      acc = fmaf(dw, dw, acc);
-    }
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      sdist[j] = acc * (1.0f / G);
-      spos[j] = p.ring_pos[(size_t)u * Wp1 + slot];
-      sslot[j] = slot;
+  // 1. distances to the window entries, newest first (age j = 0 is step n-1).
+  // Warp w takes ages w, w+8, ...; each batch of 4 entries has all its loads
+  // in flight before any reduction.
+  {
+    constexpr int NW = kMatchThreads / 32;
+    constexpr int F4 = GD / 4 / 32;  // float4 per lane per entry
+    for (int j0 = warp; j0 < occ; j0 += 4 * NW) {
+      float4 r[4][F4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int j = j0 + k * NW;
+        if (j < occ) {
+          const int slot = (n - 1 - j) % Wp1;
+          const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
+#pragma unroll
+          for (int f = 0; f < F4; ++f) r[k][f] = rq[lane + 32 * f];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int j = j0 + k * NW;
+        if (j < occ) {
+          float acc = 0.f;
+#pragma unroll
+          for (int f = 0; f < F4; ++f) {
+            const float4 q = reinterpret_cast<const float4*>(sq)[lane + 32 * f];
+            const float dx = q.x - r[k][f].x, dy = q.y - r[k][f].y, dz = q.z - r[k][f].z, dw = q.w - r[k][f].w;
+            acc = fmaf(dx, dx, acc);
+            acc = fmaf(dy, dy, acc);
+            acc = fmaf(dz, dz, acc);
+            acc = fmaf(dw, dw, acc);
+          }
+          acc = warp_sum(acc);
+          if (lane == 0) {
+            const int slot = (n - 1 - j) % Wp1;
+            sdist[j] = acc * (1.0f / G);
+            spos[j] = p.ring_pos[(size_t)u * Wp1 + slot];
+            sslot[j] = slot;
+          }
+        }
+      }
     }
   }
   __syncthreads();
@@ -252,12 +285,22 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
       p.plan[u] = pl;
     }
   } else {
-    // 4. RoPE in fp64: pair i couples elements i and i + D/2
+    // 4. RoPE in fp64: pair i couples elements i and i + D/2.  The angle
+    // pos * inv_freq is reduced to [-pi, pi] with a two-constant Cody-Waite
+    // reduction (2*pi = C1 + C2, C1 carrying 32 significant bits so k*C1 is
+    // exact for |k| < 2^21), after which sincos runs on a small argument.
     const double scale = kLog2e / sqrt((double)D);
     const double pos = (double)p.rope_pos[b];
     for (int i = tid; i < D / 2; i += kMatchThreads) {
+      const double ang = pos * p.inv_freq[i];
+      const double k = rint(ang * kInvTwoPi);
+      double r = ang;
+      if (fabs(k) < 2097152.0) {
+        r = fma(-k, kTwoPiHi, ang);
+        r = fma(-k, kTwoPiLo, r);
+      }
       double sn, cs;
-      sincos(pos * p.inv_freq[i], &sn, &cs);
+      sincos(r, &sn, &cs);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const double x = sq[h * D + i], y = sq[h * D + i + D / 2];
