@@ -185,6 +185,41 @@ int mac_set_piece_cost(MacState *st, int keys);
 /* Persistent grid size of the attention kernel (CTAs). */
 int mac_attend_grid(const MacState *st);
 
+/* Dense split-KV decode attention with no allocation at all.  The paper has
+ * no counterpart: this is a convenience for callers that cannot call
+ * cudaMalloc -- inference-server plugins and embedded hosts that must take
+ * every byte of device memory from their host framework's pre-planned pool
+ * or a budget fixed at model load, and latency-critical paths that cannot
+ * afford an allocation's implicit device synchronisation.  It computes, for
+ * every sequence and KV head, attention of the RoPE'd query group over ALL
+ * keys [0, seq_lens[b] - 1] (the miss path of mac_decode_step: no window,
+ * no reuse, no MacState) with the same kernels, and keeps all their scratch
+ * (about 1 MiB) in one static device array inside the library.
+ *   q_pre, rope_pos, K, V, block_table, seq_lens, out, lse: as in
+ *       mac_decode_step (device pointers, caller-owned, 16-byte aligned
+ *       q_pre, K, V).
+ *   device_status: device uint32 receiving MAC_DEV_* bits (OR-ed in, not
+ *       cleared), or NULL to use a word inside the static scratch.
+ *   batch .. num_pages: shapes as in MacConfig.
+ * Limits: batch * num_kv_heads <= 64, head_dim 64 or 128, Hq/Hkv = 4;
+ * larger shapes return MAC_ERR_SHAPE before anything is enqueued.
+ * Nothing is allocated or freed; the static array exists on every device
+ * that loads the library until the process exits.  The first call on a
+ * device looks up the array's device address and sets kernel attributes
+ * (make that first call before any stream capture); a call whose
+ * rope_theta or head_dim differs from the previous call's uploads 512 bytes
+ * of inverse frequencies from host memory.  Every call shares the one array
+ * and finds it as the previous call left it; the call clears the counters
+ * that must start at zero.  Two calls whose kernels overlap on the GPU (on
+ * different streams, or on the same device from different threads without
+ * ordering) race on the array and produce garbage: order them. */
+int mac_dense_decode_static(const float *q_pre, const int *rope_pos, const uint16_t *K,
+                            const uint16_t *V, const int *block_table, const int *seq_lens,
+                            float *out, float *lse, unsigned *device_status, int batch,
+                            int num_q_heads, int num_kv_heads, int head_dim, double rope_theta,
+                            int page_size, int max_seq, int max_pages_per_seq, int num_pages,
+                            void *stream);
+
 /* Static description of a return code. */
 const char *mac_error_string(int code);
 

@@ -19,7 +19,7 @@ from ._native import (MAC_DEV_BAD_PAGE, MAC_DEV_BAD_SEQ_LEN, MAC_DEV_TIMEOUT, MA
 __all__ = [
     "MacConfig", "MacError", "MacState", "mac_init_state", "mac_destroy", "mac_reset_seq", "mac_decode_step",
     "mac_match", "mac_attend", "mac_append_kv", "mac_decode_step_host", "mac_get_status", "mac_state_bytes",
-    "mac_export_state", "mac_import_state", "mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_attend_grid", "mac_error_string",
+    "mac_export_state", "mac_import_state", "mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_attend_grid", "mac_error_string", "mac_dense_decode_static",
     "MAC_OK", "MAC_ERR_ARG", "MAC_ERR_SHAPE", "MAC_ERR_CUDA", "MAC_ERR_OOM", "MAC_ERR_DEVICE",
     "MAC_DEV_BAD_SEQ_LEN", "MAC_DEV_BAD_PAGE", "MAC_DEV_TIMEOUT", "LIB_PATH",
 ]
@@ -198,6 +198,17 @@ def mac_set_piece_cost(st, keys: int) -> None:
 
 def mac_attend_grid(st) -> int:
     return int(load().mac_attend_grid(_h(st)))
+
+
+def mac_dense_decode_static(q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, device_status, batch,
+                            num_q_heads, num_kv_heads, head_dim, rope_theta, page_size=0, max_seq=0,
+                            max_pages_per_seq=0, num_pages=0, stream=None) -> int:
+    """Dense decode attention whose scratch is the library's static device
+    array (no allocation); returns the C return code."""
+    return int(load().mac_dense_decode_static(
+        _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
+        _ptr(device_status), int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim), float(rope_theta),
+        int(page_size), int(max_seq), int(max_pages_per_seq), int(num_pages), _stream(stream)))
 
 
 def mac_error_string(code: int) -> str:

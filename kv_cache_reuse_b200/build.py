@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmac_b200.so")
-SOURCES = ["mac_api.cu", "mac_match.cu", "mac_attend.cu"]
+SOURCES = ["mac_api.cu", "mac_match.cu", "mac_attend.cu", "mac_noalloc.cu"]
 HEADERS = [os.path.join(CSRC, "mac_internal.cuh"), os.path.join(ROOT, "include", "mac.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2"]
