@@ -32,6 +32,7 @@ struct MacState {
   UnitPlan* plan = nullptr;
   Segment* seg = nullptr;
   PlanHeader* hdr = nullptr;
+  int* first_seg = nullptr;
   float* part = nullptr;
   int* unit_cnt = nullptr;
   int* done = nullptr;
@@ -80,7 +81,7 @@ cudaError_t alloc(T** p, size_t count) {
 
 void free_all(MacState* s) {
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot, s->plan,
-                  s->seg,    s->hdr,    s->part,   s->unit_cnt, s->done,   s->status, s->inv_freq,
+                  s->seg,    s->hdr, s->first_seg,    s->part,   s->unit_cnt, s->done,   s->status, s->inv_freq,
                   s->st_q,   s->st_pos, s->st_lens, s->st_knew, s->st_vnew, s->st_out, s->st_lse, s->st_hit,
                   s->st_mpos};
   for (void* p : ptrs)
@@ -220,6 +221,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->plan, U));
   A(alloc(&s->seg, 2 * U));
   A(alloc(&s->hdr, 1));
+  A(alloc(&s->first_seg, (size_t)s->grid));
   A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
   A(alloc(&s->unit_cnt, U));
   A(alloc(&s->done, 1));
@@ -314,6 +316,7 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.plan = s->plan;
   p.seg = s->seg;
   p.hdr = s->hdr;
+  p.first_seg = s->first_seg;
   p.done = s->done;
   p.status = s->status;
   p.B = s->cfg.batch;
@@ -355,6 +358,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.plan = s->plan;
   p.seg = s->seg;
   p.hdr = s->hdr;
+  p.first_seg = s->first_seg;
   p.part = s->part;
   p.unit_cnt = s->unit_cnt;
   p.ring_o = s->ring_o;

@@ -510,15 +510,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 
   const long long T = p.hdr->total;
   const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
-  int first_seg = 0;
-  {
-    int a = 0, z = p.nseg - 1;  // last segment starting at or before lo
-    while (a < z) {
-      const int mid = (a + z + 1) >> 1;
-      if (p.seg[mid].flat <= lo) a = mid; else z = mid - 1;
-    }
-    first_seg = a;
-  }
+  const int first_seg = p.first_seg[cta];
   const uint64_t pol = evict_first_policy();
 
   // issue cursor: this warp's boxes w, w+8, ... of every piece, NST ahead

@@ -72,6 +72,7 @@ struct MatchParams {
   UnitPlan* plan;          // [U]
   Segment* seg;            // [2U]
   PlanHeader* hdr;
+  int* first_seg;          // [grid] first segment of each attention CTA's range
   int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
   int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;
@@ -89,6 +90,7 @@ struct AttendParams {
   const UnitPlan* plan;
   const Segment* seg;
   const PlanHeader* hdr;
+  const int* first_seg;  // [grid]
   float* part;       // [max_parts][partial_floats]
   int* unit_cnt;     // [U]
   float* ring_o;     // [U][W+1][G][D]

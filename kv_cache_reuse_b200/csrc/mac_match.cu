@@ -135,6 +135,16 @@ __device__ void build_segments(const MatchParams& p, int U) {
       p.seg[s].npieces = np;
       p.seg[s].pbase = (int)(pcarry + ex);
       if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
+      // CTAs whose range starts inside this segment's cost extent
+      // [Fw, Fw + wlen) begin their walk here: lo_c = floor(c*T/N) lies in
+      // it iff ceil(Fw*N/T) <= c < ceil((Fw + wlen)*N/T)
+      const int len = p.seg[s].len;
+      if (len > 0 && N > 0) {
+        const long long Fw = p.seg[s].flat - p.piece_cost;
+        const long long Fe = p.seg[s].flat + len;
+        const long long ca = (Fw * N + T - 1) / T, cb = (Fe * N + T - 1) / T;
+        for (long long c = ca; c < cb && c < N; ++c) p.first_seg[c] = s;
+      }
     }
     pcarry += tot;
   }
@@ -163,36 +173,59 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Wp1 = p.W + 1;
 
+  // Every load below is independent of the others (no slot index waits for
+  // the step counter): ring slots are read whole and mapped to ages later.
+  constexpr int NW = kMatchThreads / 32;
+  constexpr int BS = 5;            // slots per warp per batch (8 warps x 5 >= W+1 for W <= 39)
+  constexpr int F4 = GD / 4 / 32;  // float4 per lane per slot
+  float4 r[BS][F4];
+  int rpos[BS];
+  auto load_batch = [&](int s0) {
+#pragma unroll
+    for (int k = 0; k < BS; ++k) {
+      const int slot = s0 + k * NW;
+      if (slot < Wp1) {
+        const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
+#pragma unroll
+        for (int f = 0; f < F4; ++f) r[k][f] = rq[lane + 32 * f];
+        rpos[k] = p.ring_pos[(size_t)u * Wp1 + slot];
+      }
+    }
+  };
+  load_batch(warp);
   const float4* qsrc = reinterpret_cast<const float4*>(p.q_pre + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
   for (int i = tid; i < GD / 4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = qsrc[i];
   const int len = p.seq_lens[b];
   const int p_t = len - 1;
   const int n = p.steps[u];
   const int occ = n < p.W ? n : p.W;
+  // RoPE angle of pair i = tid (D/2 <= 64 threads), reduced to [-pi, pi] with
+  // a two-constant Cody-Waite reduction (2*pi = C1 + C2, C1 carrying 32
+  // significant bits so k*C1 is exact for |k| < 2^21), then sincos in fp64.
+  double rot_sn = 0.0, rot_cs = 1.0;
+  if (tid < D / 2) {
+    const double ang = (double)p.rope_pos[b] * p.inv_freq[tid];
+    const double k = rint(ang * kInvTwoPi);
+    double rr = ang;
+    if (fabs(k) < 2097152.0) {
+      rr = fma(-k, kTwoPiHi, ang);
+      rr = fma(-k, kTwoPiLo, rr);
+    }
+    sincos(rr, &rot_sn, &rot_cs);
+  }
   if (tid == 0) s_bad_page = 0;
   __syncthreads();
 
-  // 1. distances to the window entries, newest first (age j = 0 is step n-1).
-  // Warp w takes ages w, w+8, ...; each batch of 4 entries has all its loads
-  // in flight before any reduction.
-  {
-    constexpr int NW = kMatchThreads / 32;
-    constexpr int F4 = GD / 4 / 32;  // float4 per lane per entry
-    for (int j0 = warp; j0 < occ; j0 += 4 * NW) {
-      float4 r[4][F4];
+  // 1. distances: mean over the G heads of sum((q - q_s)^2), for the slots
+  // holding the occ most recent entries (age j = 0 is step n - 1, in slot
+  // (n - 1) mod (W+1); the age of slot s is (n - 1 - s) mod (W+1)).
+  for (int s0 = warp; s0 < Wp1; s0 += BS * NW) {
+    if (s0 != warp) load_batch(s0);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int j = j0 + k * NW;
-        if (j < occ) {
-          const int slot = (n - 1 - j) % Wp1;
-          const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
-#pragma unroll
-          for (int f = 0; f < F4; ++f) r[k][f] = rq[lane + 32 * f];
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int j = j0 + k * NW;
+    for (int k = 0; k < BS; ++k) {
+      const int slot = s0 + k * NW;
+      if (slot < Wp1) {
+        const int j = (((n - 1 - slot) % Wp1) + Wp1) % Wp1;
         if (j < occ) {
           float acc = 0.f;
 #pragma unroll
@@ -206,9 +239,8 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
           }
           acc = warp_sum(acc);
           if (lane == 0) {
-            const int slot = (n - 1 - j) % Wp1;
             sdist[j] = acc * (1.0f / G);
-            spos[j] = p.ring_pos[(size_t)u * Wp1 + slot];
+            spos[j] = rpos[k];
             sslot[j] = slot;
           }
         }
@@ -285,22 +317,10 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
       p.plan[u] = pl;
     }
   } else {
-    // 4. RoPE in fp64: pair i couples elements i and i + D/2.  The angle
-    // pos * inv_freq is reduced to [-pi, pi] with a two-constant Cody-Waite
-    // reduction (2*pi = C1 + C2, C1 carrying 32 significant bits so k*C1 is
-    // exact for |k| < 2^21), after which sincos runs on a small argument.
+    // 4. rotate pair i = tid (i, i + D/2) by the angle computed above
     const double scale = kLog2e / sqrt((double)D);
-    const double pos = (double)p.rope_pos[b];
     for (int i = tid; i < D / 2; i += kMatchThreads) {
-      const double ang = pos * p.inv_freq[i];
-      const double k = rint(ang * kInvTwoPi);
-      double r = ang;
-      if (fabs(k) < 2097152.0) {
-        r = fma(-k, kTwoPiHi, ang);
-        r = fma(-k, kTwoPiLo, r);
-      }
-      double sn, cs;
-      sincos(r, &sn, &cs);
+      const double sn = rot_sn, cs = rot_cs;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const double x = sq[h * D + i], y = sq[h * D + i + D / 2];

@@ -41,7 +41,8 @@ constexpr size_t kOffQrot = 0;
 constexpr size_t kOffPlan = align256(kOffQrot + (size_t)kMaxUnits * kGroup * kMaxD * 4);
 constexpr size_t kOffSeg = align256(kOffPlan + kMaxUnits * sizeof(UnitPlan));
 constexpr size_t kOffHdr = align256(kOffSeg + 2 * kMaxUnits * sizeof(Segment));
-constexpr size_t kOffPart = align256(kOffHdr + sizeof(PlanHeader));
+constexpr size_t kOffFirst = align256(kOffHdr + sizeof(PlanHeader));
+constexpr size_t kOffPart = align256(kOffFirst + kMaxCtas * 4);
 constexpr size_t kOffCnt = align256(kOffPart + (size_t)(kMaxCtas + 2 * kMaxUnits) * kPartFloats * 4);
 // counters block, cleared on every call: unit_cnt[kMaxUnits], done, status, steps[kMaxUnits]
 constexpr size_t kCntBytes = (2 * kMaxUnits + 2) * 4;
@@ -171,6 +172,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.plan = reinterpret_cast<UnitPlan*>(base + kOffPlan);
   mp.seg = reinterpret_cast<Segment*>(base + kOffSeg);
   mp.hdr = reinterpret_cast<PlanHeader*>(base + kOffHdr);
+  mp.first_seg = reinterpret_cast<int*>(base + kOffFirst);
   mp.done = cnt + kMaxUnits;
   mp.status = status;
   mp.B = batch;
@@ -201,6 +203,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.plan = mp.plan;
   ap.seg = mp.seg;
   ap.hdr = mp.hdr;
+  ap.first_seg = mp.first_seg;
   ap.part = reinterpret_cast<float*>(base + kOffPart);
   ap.unit_cnt = cnt;
   ap.ring_o = reinterpret_cast<float*>(base + kOffRingO);
