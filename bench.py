@@ -146,6 +146,10 @@ def run_mac(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     base = synth.WORKLOADS[args.workload]
+    if args.batch:
+        base = base.with_(B=args.batch, L0=base.L0[:1] * args.batch)
+    if args.tau is not None:
+        base = base.with_(tau=args.tau)
     wl = base.with_(seed=base.seed + 1000 * rank)  # every rank: its own batch
     T = max(base.steps, args.warmup + args.steps)
     stream = synth.queries(wl, T)
@@ -403,6 +407,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling of smaller cases)")
+    ap.add_argument("--tau", type=float, default=None, help="override the match threshold (0 = every step misses)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
