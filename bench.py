@@ -55,15 +55,15 @@ def _kernel_hash() -> str:
 
 
 def _profiled_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source (else None)."""
+    """Ratio of DRAM bytes to algorithmic bytes of the attention kernel from the
+    committed ncu summary, if it was taken on the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "mac_attend_long_128k_traffic.txt")
     try:
         txt = open(p).read()
     except OSError:
         return None
     m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
-    b = re.search(r"dram_bytes_per_launch_scaled:\s*([0-9.eE+]+)", txt)
+    b = re.search(r"dram_traffic_over_algorithmic:\s*([0-9.eE+]+)", txt)
     if not m or not b or m.group(1) != _kernel_hash():
         return None
     return float(b.group(1))
@@ -262,7 +262,9 @@ def run_mac(args, rank, world, local_rank):
         return None
     K_ = args.steps
     att_gbs = kern["att_bytes"] / (kern["att_ms"] * 1e-3) / 1e9
-    traffic = _profiled_traffic()
+    ratio = _profiled_traffic()
+    # traffic per launch: the profiled DRAM/algorithmic ratio scaled to this run's launches
+    traffic = ratio * kern["att_bytes"] / K_ if ratio else None
     res = {
         "metric": METRIC, "value": world * K_ / (tot * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K_,
         "warmup": args.warmup, "ms_per_step": tot / K_, "higher_is_better": True, "scaling": "weak",
