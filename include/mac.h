@@ -182,6 +182,13 @@ int mac_import_state(MacState *st, const void *host_buf, size_t bytes);
 int mac_set_min_keys_per_cta(MacState *st, int keys);
 int mac_set_piece_cost(MacState *st, int keys);
 
+/* Tuning: a (sequence, KV head) whose fresh key range (amend band + tail on
+ * a hit, every key on a miss) holds at most `keys` keys (default 1024) is
+ * done end to end by one CTA, with no partial results; longer ranges are
+ * cut over several CTAs and merged by the last of them.  0 cuts every
+ * range. */
+int mac_set_whole_unit_keys(MacState *st, int keys);
+
 /* Persistent grid size of the attention kernel (CTAs). */
 int mac_attend_grid(const MacState *st);
 

@@ -18,7 +18,7 @@ using namespace mac;
 
 struct MacState {
   MacConfig cfg;
-  int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, capacity;
+  int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, unit_max, capacity;
   size_t max_parts;
   // ring (library-owned state)
   float* ring_q = nullptr;
@@ -197,6 +197,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   s->W = cfg->window;
   s->min_keys = 128;
   s->piece_cost = 1024;
+  s->unit_max = 1024;
   s->capacity = cfg->page_size == 0 ? cfg->max_seq : cfg->max_pages_per_seq * cfg->page_size;
   if (cudaGetDevice(&s->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&s->num_sms, cudaDevAttrMultiProcessorCount, s->device) != cudaSuccess) {
@@ -292,6 +293,12 @@ int mac_set_piece_cost(MacState* s, int keys) {
   return MAC_OK;
 }
 
+int mac_set_whole_unit_keys(MacState* s, int keys) {
+  if (!s || keys < 0) return MAC_ERR_ARG;
+  s->unit_max = keys;
+  return MAC_OK;
+}
+
 int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
 
 int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
@@ -332,6 +339,7 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.grid = s->grid;
   p.min_keys = s->min_keys;
   p.piece_cost = s->piece_cost;
+  p.unit_max = s->unit_max;
   return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 

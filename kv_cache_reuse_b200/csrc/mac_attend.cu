@@ -48,10 +48,6 @@ constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
-struct StageMeta {
-  int unit, pidx;
-};
-
 template <int D>
 struct Cfg {
   static constexpr int NV = D / 64;  // 8-dim vectors per lane per row
@@ -360,13 +356,13 @@ __device__ void merge_unit(const AttendParams& p, int u) {
   }
 }
 
-// End of a piece: combine the 32 groups' states, write the partial, count it
-// and, if it was the unit's last, merge the unit.
+// Combine the warp's 4 lane groups (each holds its own running max, sum and
+// output) and store the warp's state in its shared-memory slot:
+// o [G][D] unnormalised, then m [G] and l [G].
 template <int D>
-__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, const StageMeta& m,
-                               uint32_t& sync_phase) {
-  constexpr int NV = Cfg<D>::NV, G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ void warp_combine_store(Acc<D>& A, float* wb) {
+  constexpr int NV = Cfg<D>::NV, G = kGroup, GD = Cfg<D>::GD;
+  const int lane = threadIdx.x & 31;
   const int j = lane & 7;
   const bool b0 = (j & 1) != 0;
   __syncwarp();
@@ -378,7 +374,6 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
   l1 += __shfl_xor_sync(kFull, l1, 2);
   const float o0 = __shfl_xor_sync(kFull, l0, 1), o1 = __shfl_xor_sync(kFull, l1, 1);
   float lg[4] = {sel(b0, o0, l0), sel(b0, o1, l1), sel(b0, l0, o0), sel(b0, l1, o1)};
-  // combine the warp's 4 groups
 #pragma unroll
   for (int off = 8; off <= 16; off <<= 1) {
 #pragma unroll
@@ -399,7 +394,6 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
       A.m[h] = M;
     }
   }
-  float* wb = sm.wbuf[warp];
   if (lane < 8) {
 #pragma unroll
     for (int h = 0; h < G; ++h)
@@ -416,23 +410,40 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
       wb[GD + G + h] = lg[h];
     }
   }
+}
+
+// Merge the states of warps [w0, w1) for output element idx of head h:
+// returns (M, L, O) with O and L relative to 2^M.
+template <int D>
+__device__ __forceinline__ void combine_warps(const AttnSmem<D>& sm, int w0, int w1, int idx, int h, float& M,
+                                              float& L, float& O) {
+  constexpr int G = kGroup, GD = Cfg<D>::GD;
+  M = -INFINITY;
+  for (int w = w0; w < w1; ++w) M = fmaxf(M, sm.wbuf[w][GD + h]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  L = 0.f;
+  O = 0.f;
+  for (int w = w0; w < w1; ++w) {
+    const float a = ex2(sm.wbuf[w][GD + h] - Mu);
+    O += sm.wbuf[w][idx] * a;
+    L += sm.wbuf[w][GD + G + h] * a;
+  }
+}
+
+// End of a split piece: combine the 8 warps, write the partial, count it
+// and, if it was the unit's last, merge the unit.
+template <int D>
+__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int unit, int pidx,
+                               uint32_t& sync_phase) {
+  constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
+  warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  // combine the 8 warps and write the partial
-  float* dst = p.part + (size_t)m.pidx * PF;
+  float* dst = p.part + (size_t)pidx * PF;
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
     const int h = idx / D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wbuf[w][GD + h]);
-    const float Mu = M == -INFINITY ? 0.f : M;
-    float acc = 0.f, L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float a = ex2(sm.wbuf[w][GD + h] - Mu);
-      acc += sm.wbuf[w][idx] * a;
-      L += sm.wbuf[w][GD + G + h] * a;
-    }
-    dst[idx] = acc;
+    float M, L, O;
+    combine_warps<D>(sm, 0, kConsumerWarps, idx, h, M, L, O);
+    dst[idx] = O;
     if (idx - h * D == 0) {
       dst[GD + h] = M;
       dst[GD + G + h] = L;
@@ -441,21 +452,121 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
   __threadfence();
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (threadIdx.x == 0) {
-    const int old = atomicAdd(p.unit_cnt + m.unit, 1);
-    sm.last_flag = (old == p.plan[m.unit].expected - 1);
+    const int old = atomicAdd(p.unit_cnt + unit, 1);
+    sm.last_flag = (old == p.plan[unit].expected - 1);
   }
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
-    merge_unit<D>(p, m.unit);
+    merge_unit<D>(p, unit);
   }
   return true;
 }
 
-// The CTA's pieces, walked in order by every lane of every warp.
+// End of a whole-unit piece: warps [0, wA) hold the amend range [start, c_t),
+// warps [wA, 8) the tail [c_t, p_t].  New prefix state = reused ring state
+// (on a hit) + amend; output = new prefix + tail.  No partials, no counters.
+template <int D>
+__device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int u, int wA,
+                              uint32_t& sync_phase) {
+  constexpr int G = kGroup, GD = Cfg<D>::GD;
+  const UnitPlan pl = p.plan[u];
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
+  const int Wp1 = p.W + 1;
+  // the reused state is independent of the combine: fetch it first
+  constexpr int PER = (GD + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
+  float ro[PER], rm[PER], rl[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int idx = threadIdx.x + k * kConsumerWarps * 32;
+    ro[k] = 0.f;
+    rm[k] = -INFINITY;
+    rl[k] = 0.f;
+    if (pl.hit && idx < GD) {
+      const size_t rs = (size_t)u * Wp1 + pl.src_slot;
+      const int h = idx / D;
+      ro[k] = p.ring_o[rs * GD + idx];
+      rm[k] = p.ring_m[rs * G + h] * kLog2e;
+      rl[k] = p.ring_l[rs * G + h];
+    }
+  }
+  warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
+  if (!consumer_sync(sm, sync_phase, p.status)) return false;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int idx = threadIdx.x + k * kConsumerWarps * 32;
+    if (idx >= GD) break;
+    const int h = idx / D, d = idx - h * D;
+    float MA, LA, OA, MB, LB, OB;
+    combine_warps<D>(sm, 0, wA, idx, h, MA, LA, OA);
+    combine_warps<D>(sm, wA, kConsumerWarps, idx, h, MB, LB, OB);
+    // new prefix state S = reused (hit) + amend
+    float M = fmaxf(MA, pl.hit ? rm[k] : -INFINITY);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    const float aA = ex2(MA - Mu);
+    float L = LA * aA, O = OA * aA;
+    if (pl.hit) {
+      const float a = ex2(rm[k] - Mu);
+      L += rl[k] * a;
+      O += ro[k] * rl[k] * a;
+    }
+    const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
+    p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
+    if (d == 0) {
+      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
+      p.ring_l[ds * G + h] = L;
+    }
+    // output = S + tail
+    const float M2 = fmaxf(M, MB);
+    const float M2u = M2 == -INFINITY ? 0.f : M2;
+    const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
+    const float L2 = L * a0 + LB * aB, O2 = O * a0 + OB * aB;
+    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    p.out[orow * D + d] = O2 / L2;
+    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+  }
+  if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
+  // the warps' slots are reused by the next piece
+  return consumer_sync(sm, sync_phase, p.status);
+}
+
+// The CTA's pieces, walked in order by every lane of every warp.  A split
+// piece is part of one segment of a large unit; a whole-unit piece holds
+// both segments of a small unit: A = [a0, a1) (may be empty), B = [k0, k1).
 struct Piece {
-  int unit, pidx, k0, k1, kb0, nbox;
+  int unit, pidx, whole;
+  int k0, k1, kb0, nbox;      // split: its keys; whole unit: segment B
+  int a0, a1, akb0, anbox;    // whole unit: segment A
+  int wA;                     // whole unit: warps on segment A
 };
+// The boxes one warp takes from a piece: indices first, first + stride, ...
+struct WarpRange {
+  int kb0, k0, k1, nbox, first, stride;
+};
+__device__ __forceinline__ WarpRange warp_range(const Piece& pc, int warp) {
+  WarpRange r;
+  if (pc.whole && warp < pc.wA) {
+    r.kb0 = pc.akb0;
+    r.k0 = pc.a0;
+    r.k1 = pc.a1;
+    r.nbox = pc.anbox;
+    r.first = warp;
+    r.stride = pc.wA;
+  } else {
+    const int base = pc.whole ? pc.wA : 0;
+    r.kb0 = pc.kb0;
+    r.k0 = pc.k0;
+    r.k1 = pc.k1;
+    r.nbox = pc.nbox;
+    r.first = warp - base;
+    r.stride = kConsumerWarps - base;
+  }
+  return r;
+}
+__device__ __forceinline__ int box_count(int k0, int k1) {
+  const int kb0 = k0 & ~(kSubKeys - 1);
+  return k1 > k0 ? (((k1 + kSubKeys - 1) & ~(kSubKeys - 1)) - kb0) / kSubKeys : 0;
+}
 struct Walker {
   int s;
   long long lo, hi;
@@ -463,20 +574,45 @@ struct Walker {
     while (s < p.nseg) {
       const Segment sg = p.seg[s];
       const int cur = s++;
-      if (sg.len == 0) continue;
-      if (sg.flat >= hi) {  // this and every later segment start past the range
+      if (sg.kind < 0) continue;
+      if (sg.flat >= hi) {  // this and every later item start past the range
         s = p.nseg;
         return false;
+      }
+      pc.unit = cur >> 1;
+      if (sg.kind == kItemWhole) {
+        if (sg.first_cta != cta) continue;  // owned by the CTA whose range holds its start
+        const int start = sg.key0, cut = sg.pbase, end = sg.key0 + sg.len;
+        pc.whole = 1;
+        pc.pidx = -1;
+        pc.a0 = start;
+        pc.a1 = cut;
+        pc.akb0 = start & ~(kSubKeys - 1);
+        pc.anbox = box_count(start, cut);
+        pc.k0 = cut;
+        pc.k1 = end;
+        pc.kb0 = cut & ~(kSubKeys - 1);
+        pc.nbox = box_count(cut, end);
+        const int nA = pc.anbox, nB = pc.nbox;
+        int wA = 0;
+        if (nA > 0) {
+          wA = (kConsumerWarps * nA + (nA + nB) / 2) / (nA + nB);
+          wA = wA < 1 ? 1 : (wA > kConsumerWarps - 1 ? kConsumerWarps - 1 : wA);
+        }
+        pc.wA = wA;
+        return true;
       }
       const long long fa = lo > sg.flat ? lo : sg.flat;
       const long long fe = hi < sg.flat + sg.len ? hi : sg.flat + sg.len;
       if (fa >= fe) continue;  // the range holds only this segment's padding, or ends before it
-      pc.unit = cur >> 1;
+      pc.whole = 0;
+      pc.wA = 0;
+      pc.anbox = 0;
       pc.pidx = sg.pbase + (cta - sg.first_cta);
       pc.k0 = sg.key0 + (int)(fa - sg.flat);
       pc.k1 = sg.key0 + (int)(fe - sg.flat);
       pc.kb0 = pc.k0 & ~(kSubKeys - 1);
-      pc.nbox = (((pc.k1 + kSubKeys - 1) & ~(kSubKeys - 1)) - pc.kb0) / kSubKeys;
+      pc.nbox = box_count(pc.k0, pc.k1);
       return true;
     }
     return false;
@@ -513,29 +649,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   const int first_seg = p.first_seg[cta];
   const uint64_t pol = evict_first_policy();
 
-  // issue cursor: this warp's boxes w, w+8, ... of every piece, NST ahead
+  // issue cursor: this warp's boxes of every piece, NST ahead
   Walker wi{first_seg, lo, hi};
   Piece ip;
+  WarpRange ir;
   bool ivalid = wi.next(p, cta, ip);
-  int ib = warp, ipn = 0, nissued = 0, nq_issued = 0;
+  if (ivalid) ir = warp_range(ip, warp);
+  int ib = ivalid ? ir.first : 0, ipn = 0, nissued = 0, nq_issued = 0;
   auto issue_advance = [&]() {
-    while (ivalid && ib >= ip.nbox) {
+    while (ivalid && ib >= ir.nbox) {
       ivalid = wi.next(p, cta, ip);
-      ib = warp;
+      if (ivalid) {
+        ir = warp_range(ip, warp);
+        ib = ir.first;
+      }
       ++ipn;
     }
   };
   auto issue_box = [&](int st) {
+    // warp 0 always owns box 0 of its range in every piece: it brings the query
+    const bool qfirst = warp == 0 && ib == 0;
     if (lane == 0) {
-      if (warp == 0 && ib == 0) {  // first box of a piece: bring its query too
+      if (qfirst) {
         const int qs = ipn % NQ;
         mbar_arrive_expect_tx(&sm.qfull[qs], GD * 4);
         bulk_load(sm.q[qs], p.qrot + (size_t)ip.unit * GD, GD * 4, &sm.qfull[qs]);
       }
-    }
-    if (warp == 0 && ib == 0) ++nq_issued;
-    if (lane == 0) {
-      const int key = ip.kb0 + ib * kSubKeys;
+      const int key = ir.kb0 + ib * kSubKeys;
       const int b = ip.unit / p.Hkv, kvh = ip.unit - b * p.Hkv;
       int c2, c3;
       if (p.page_size > 0) {
@@ -549,8 +689,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       tma_load_4d(sm.kv[warp][st][0], &p.tmK, &sm.full[warp][st], 0, kvh, c2, c3, pol);
       tma_load_4d(sm.kv[warp][st][1], &p.tmV, &sm.full[warp][st], 0, kvh, c2, c3, pol);
     }
+    if (qfirst) ++nq_issued;
     ++nissued;
-    ib += kConsumerWarps;
+    ib += ir.stride;
     issue_advance();
   };
   issue_advance();
@@ -586,18 +727,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       for (int h = 0; h < G; ++h) A.m[h] = -INFINITY;
       A.l[0] = A.l[1] = 0.f;
     }
-    for (int bj = warp; bj < cp.nbox; bj += kConsumerWarps) {
+    const WarpRange cr = warp_range(cp, warp);
+    for (int bj = cr.first; bj < cr.nbox; bj += cr.stride) {
       const int st = cons % NST;
       if (!mbar_wait(&sm.full[warp][st], (uint32_t)(cons / NST) & 1u, &sm.abort_flag, p.status)) {
         ok = false;
         break;
       }
-      const int key_box = cp.kb0 + bj * kSubKeys;
+      const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * 144;
-      if (key_box < cp.k0 || key_box + kSubKeys > cp.k1)
-        process_box<D, true>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cp.k0, cp.k1);
+      if (key_box < cr.k0 || key_box + kSubKeys > cr.k1)
+        process_box<D, true>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1);
       else
-        process_box<D, false>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cp.k0, cp.k1);
+        process_box<D, false>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1);
       par ^= 1;
       ++cons;
       __syncwarp();
@@ -607,10 +749,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
     }
     if (!ok) break;
-    StageMeta m;
-    m.unit = cp.unit;
-    m.pidx = cp.pidx;
-    if (!finalize_piece<D>(p, sm, A, m, sync_phase)) break;
+    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, sync_phase)
+                              : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    if (!fin) break;
     ++cpn;
   }
   if (nissued > cons || !ok) {

@@ -28,21 +28,26 @@ struct UnitPlan {
   int expected;  // partial results the unit's merge waits for
 };
 
-// Two key segments per unit: 2u = [start, cut) (into the new prefix state),
-// 2u+1 = [cut, end) (tail, into the output only).  The segments of all units
-// are laid end to end ("flattened") in a cost space where a non-empty
-// segment weighs piece_cost + len (the fixed cost of a piece -- query load,
-// combine, merge -- expressed in keys), and that space is split evenly over
-// the CTAs.  A segment's keys occupy [flat, flat + len) of the space, after
-// its piece_cost of padding.
+// Work items, two slots per unit u.  A large unit (more than unit_max fresh
+// keys) has two split items: 2u = [start, cut) (into the new prefix state) and
+// 2u+1 = [cut, end) (tail, into the output only); each may be cut over several
+// CTAs, whose partial results the unit's last CTA merges.  A small unit is
+// one whole item in slot 2u, done end to end by one CTA, and slot 2u+1 is
+// empty.  The items of all units are laid end to end in a cost space where a
+// non-empty item weighs piece_cost + its keys (the fixed cost of a piece --
+// query load, combine, merge -- expressed in keys), and that space is split
+// evenly over the CTAs.  A split item's keys occupy [flat, flat + len) after
+// its piece_cost of padding; a whole item starts at flat and belongs to the
+// CTA whose range holds flat.
+enum { kItemEmpty = -1, kItemA = 0, kItemB = 1, kItemWhole = 2 };
 struct Segment {
-  long long flat;  // cost-space offset of the segment's first key
-  int len;         // keys
+  long long flat;  // split: cost offset of the first key; whole: cost offset of the item
+  int len;         // keys (whole: end - start)
   int key0;        // first key (absolute position in the sequence)
-  int first_cta;   // CTA holding cost offset `flat`
-  int pbase;       // index of this segment's first partial result
-  int npieces;     // partial results (CTAs overlapping the segment)
-  int pad;
+  int first_cta;   // split: CTA holding `flat`; whole: the owning CTA
+  int pbase;       // split: index of the first partial result; whole: the cut c_t
+  int npieces;     // split: partial results (CTAs overlapping the keys); whole: 0
+  int kind;        // kItem*
 };
 
 struct PlanHeader {
@@ -80,6 +85,7 @@ struct MatchParams {
   int grid;       // CTAs of the attention kernel
   int min_keys;   // minimum cost-space units per attention CTA
   int piece_cost; // fixed cost of one piece, in keys
+  int unit_max;   // units with at most this many fresh keys are whole items
 };
 
 struct AttendParams {

@@ -82,27 +82,42 @@ __device__ void build_segments(const MatchParams& p, int U) {
   __shared__ long long sbuf[kMatchThreads / 32];
   const int tid = threadIdx.x;
   const int nseg = 2 * U;
+  const long long cost = p.piece_cost;
+  // pass 1: item kinds, keys and cost-space offsets
   long long carry = 0;
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
-    int len = 0, key0 = 0;
+    int len = 0, key0 = 0, kind = kItemEmpty, cut = 0;
     long long wlen = 0;
     if (s < nseg) {
       const UnitPlan* pl = p.plan + (s >> 1);
       const int bad = __ldcg(&pl->bad);
       if (!bad) {
-        const int start = __ldcg(&pl->start), cut = __ldcg(&pl->cut), end = __ldcg(&pl->end);
-        len = (s & 1) ? end - cut : cut - start;
-        key0 = (s & 1) ? cut : start;
-        wlen = len > 0 ? (long long)len + p.piece_cost : 0;
+        const int start = __ldcg(&pl->start), c = __ldcg(&pl->cut), end = __ldcg(&pl->end);
+        if (end - start <= p.unit_max) {
+          if ((s & 1) == 0) {  // the whole unit in slot 2u
+            kind = kItemWhole;
+            len = end - start;
+            key0 = start;
+            cut = c;
+          }
+        } else {
+          len = (s & 1) ? end - c : c - start;
+          key0 = (s & 1) ? c : start;
+          kind = len > 0 ? ((s & 1) ? kItemB : kItemA) : kItemEmpty;
+        }
+        if (kind != kItemEmpty) wlen = (long long)len + cost;
       }
     }
     long long tot;
     long long ex = block_exclusive_scan(wlen, &tot, sbuf);
     if (s < nseg) {
-      p.seg[s].flat = carry + ex + (len > 0 ? p.piece_cost : 0);
-      p.seg[s].len = len;
+      const bool split = kind == kItemA || kind == kItemB;
+      p.seg[s].flat = carry + ex + (split ? cost : 0);
+      p.seg[s].len = kind == kItemEmpty ? 0 : len;
       p.seg[s].key0 = key0;
+      p.seg[s].kind = kind;
+      p.seg[s].pbase = cut;  // whole items keep their cut here; split items overwrite it below
     }
     carry += tot;
   }
@@ -114,34 +129,39 @@ __device__ void build_segments(const MatchParams& p, int U) {
     if (N < 1) N = 1;
   }
   __syncthreads();
+  // pass 2: owning / first CTA, partial slots, and each CTA's first item
   long long pcarry = 0;
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
-    int np = 0, first = 0;
+    int np = 0, first = 0, kind = kItemEmpty, len = 0;
+    long long F = 0;
     if (s < nseg) {
-      const long long F = p.seg[s].flat;
-      const int len = p.seg[s].len;
-      if (len > 0) {
+      F = p.seg[s].flat;
+      len = p.seg[s].len;
+      kind = p.seg[s].kind;
+      if (kind == kItemA || kind == kItemB) {
         first = cta_of(F, T, N);
         np = cta_of(F + len - 1, T, N) - first + 1;
+      } else if (kind == kItemWhole) {
+        first = cta_of(F, T, N);
       }
     }
     long long tot;
     long long ex = block_exclusive_scan(np, &tot, sbuf);
-    // units own segments (2u, 2u+1): adjacent threads of one warp
+    // units own items (2u, 2u+1): adjacent threads of one warp
     const int np_next = __shfl_down_sync(0xffffffffu, np, 1);
     if (s < nseg) {
       p.seg[s].first_cta = first;
       p.seg[s].npieces = np;
-      p.seg[s].pbase = (int)(pcarry + ex);
+      if (kind != kItemWhole) p.seg[s].pbase = (int)(pcarry + ex);
       if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
-      // CTAs whose range starts inside this segment's cost extent
-      // [Fw, Fw + wlen) begin their walk here: lo_c = floor(c*T/N) lies in
-      // it iff ceil(Fw*N/T) <= c < ceil((Fw + wlen)*N/T)
-      const int len = p.seg[s].len;
-      if (len > 0 && N > 0) {
-        const long long Fw = p.seg[s].flat - p.piece_cost;
-        const long long Fe = p.seg[s].flat + len;
+      // CTAs whose range starts inside this item's cost extent [Fw, Fe)
+      // begin their walk here: lo_c = floor(c*T/N) lies in it iff
+      // ceil(Fw*N/T) <= c < ceil(Fe*N/T)
+      if (kind != kItemEmpty && N > 0) {
+        const bool split = kind == kItemA || kind == kItemB;
+        const long long Fw = split ? F - cost : F;
+        const long long Fe = Fw + len + cost;
         const long long ca = (Fw * N + T - 1) / T, cb = (Fe * N + T - 1) / T;
         for (long long c = ca; c < cb && c < N; ++c) p.first_seg[c] = s;
       }

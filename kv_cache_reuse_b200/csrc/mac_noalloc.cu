@@ -188,6 +188,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.grid = grid;
   mp.min_keys = 128;
   mp.piece_cost = 1024;
+  mp.unit_max = 1024;
   if (launch_match(mp, head_dim, st) != cudaSuccess) return MAC_ERR_CUDA;
 
   // --- attention over every key, merge into out/lse (and the dummy ring)
