@@ -193,7 +193,7 @@ def mac_set_min_keys_per_cta(st, keys: int) -> None:
 
 
 def mac_set_piece_cost(st, keys: int) -> None:
-    check("mac_set_piece_cost", "mac_set_whole_unit_keys", load().mac_set_piece_cost(_h(st), int(keys)))
+    check("mac_set_piece_cost", load().mac_set_piece_cost(_h(st), int(keys)))
 
 
 def mac_set_whole_unit_keys(st, keys: int) -> None:

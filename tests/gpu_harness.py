@@ -19,7 +19,7 @@ def torch_dev():
 class GpuRun:
     """One MacState plus device copies of a workload's cache."""
 
-    def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None):
+    def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None, tune=None):
         import kv_cache_reuse_b200 as mac
         torch, dev = torch_dev()
         self.torch, self.dev, self.wl, self.cache = torch, dev, wl, cache
@@ -31,6 +31,8 @@ class GpuRun:
                                                 num_pages=cache.num_pages, tau=tau, band=band, window=window)
         else:
             self.st = mac.MacState.for_workload(wl, capacity=cache.max_seq, tau=tau, band=band, window=window)
+        for name, val in (tune or {}).items():  # work-split knobs: min_keys_per_cta, piece_cost, whole_unit_keys
+            getattr(mac, "mac_set_" + name)(self.st, val)
         B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
         f32, i32 = torch.float32, torch.int32
         self.q = torch.empty((B, Hq, D), dtype=f32, device=dev)
@@ -53,10 +55,10 @@ class GpuRun:
 
 
 def compare_stream(wl, stream, cache, steps=None, tau=None, band=None, window=None, gpu=None, orc=None,
-                   rope_zero=False):
+                   rope_zero=False, tune=None):
     """Run both sides over the stream; assert parity at every step.  Returns stats."""
     T = stream.q.shape[0] if steps is None else steps
-    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window)
+    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune)
     orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window)
     worst_o = worst_l = 0.0
     hits = 0

@@ -215,6 +215,18 @@ def test_edge_cases(case):
     compare_stream(wl, stream, cache)
 
 
+@pytest.mark.parametrize("tune", [
+    {"whole_unit_keys": 0},                                           # every range cut over CTAs
+    {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 16},  # many tiny pieces per unit
+    {"whole_unit_keys": 1 << 20},                                     # every unit done by one CTA
+    {"piece_cost": 1 << 16, "min_keys_per_cta": 1},                   # one piece per CTA at most
+])
+def test_work_split_settings_keep_parity(tune):
+    """How the keys are divided among CTAs changes only rounding, never decisions."""
+    wl = synth.WORKLOADS["paged_mixed"].with_(B=4, L0=(9000, 1500, 300, 4100), steps=12)
+    compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tune=tune)
+
+
 def test_nan_query_misses_and_stays_local():
     wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, L0=(700, 900), steps=6)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
