@@ -47,6 +47,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr int kItemCache = 64;  // work items of one CTA kept in shared memory
 
 template <int D>
 struct Cfg {
@@ -68,6 +69,7 @@ struct __align__(128) AttnSmem {
   unsigned long long csync;
   int abort_flag;
   int last_flag;
+  Segment items[kItemCache];  // the CTA's work items, from its first one on
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -291,14 +293,41 @@ __device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, 
   return ok;
 }
 
-// Merge of unit u by the CTA holding its last partial (256 consumer threads).
+// Merge of unit u by the CTA holding its last partial (256 threads).  Phase
+// 1 stages every partial's (m, l) in shared memory with one round of
+// independent loads; phase 2 weighs the partial outputs, all loads in flight.
 template <int D>
-__device__ void merge_unit(const AttendParams& p, int u) {
+__device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
+  constexpr int kCap = (kConsumerWarps * Cfg<D>::WB) / (2 * G);  // pieces whose (m, l) fit in wbuf
   const UnitPlan pl = p.plan[u];
   const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
+  const int nA = sA.npieces, n = sA.npieces + sB.npieces;
+  float* mm = &sm.wbuf[0][0];  // [piece][G] maxima, then [piece][G] sums
+  float* ll = mm + kCap * G;
+  const bool staged = n <= kCap;
+  if (staged) {
+    for (int t = threadIdx.x; t < n * G; t += kConsumerWarps * 32) {
+      const int i = t / G, h = t - i * G;
+      const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
+      const float* pp = p.part + (size_t)slot * PF;
+      mm[t] = __ldcg(pp + GD + h);
+      ll[t] = __ldcg(pp + GD + G + h);
+    }
+  }
+  if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  auto pm = [&](int i, int h) -> float {
+    if (staged) return mm[i * G + h];
+    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
+    return __ldcg(p.part + (size_t)slot * PF + GD + h);
+  };
+  auto pl_ = [&](int i, int h) -> float {
+    if (staged) return ll[i * G + h];
+    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
+    return __ldcg(p.part + (size_t)slot * PF + GD + G + h);
+  };
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
     const int h = idx / D, d = idx - h * D;
     // new prefix state over [0, c_t): reused state (hit) + amend partials
@@ -310,8 +339,7 @@ __device__ void merge_unit(const AttendParams& p, int u) {
       ro = p.ring_o[rs * GD + idx];
       M = rm;
     }
-#pragma unroll 4
-    for (int i = 0; i < sA.npieces; ++i) M = fmaxf(M, __ldcg(p.part + (size_t)(sA.pbase + i) * PF + GD + h));
+    for (int i = 0; i < nA; ++i) M = fmaxf(M, pm(i, h));
     const float Mu = M == -INFINITY ? 0.f : M;
     float L = 0.f, O = 0.f;
     if (pl.hit) {
@@ -319,12 +347,11 @@ __device__ void merge_unit(const AttendParams& p, int u) {
       L += rl * a;
       O += ro * rl * a;
     }
-#pragma unroll 4
-    for (int i = 0; i < sA.npieces; ++i) {
-      const float* pp = p.part + (size_t)(sA.pbase + i) * PF;
-      const float a = ex2(__ldcg(pp + GD + h) - Mu);
-      L += __ldcg(pp + GD + G + h) * a;
-      O += __ldcg(pp + idx) * a;
+#pragma unroll 8
+    for (int i = 0; i < nA; ++i) {
+      const float a = ex2(pm(i, h) - Mu);
+      L += pl_(i, h) * a;
+      O += __ldcg(p.part + (size_t)(sA.pbase + i) * PF + idx) * a;
     }
     const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
     p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
@@ -334,17 +361,15 @@ __device__ void merge_unit(const AttendParams& p, int u) {
     }
     // output: new prefix state + tail partials
     float M2 = M;
-#pragma unroll 4
-    for (int i = 0; i < sB.npieces; ++i) M2 = fmaxf(M2, __ldcg(p.part + (size_t)(sB.pbase + i) * PF + GD + h));
+    for (int i = nA; i < n; ++i) M2 = fmaxf(M2, pm(i, h));
     const float M2u = M2 == -INFINITY ? 0.f : M2;
     const float a0 = ex2(M - M2u);
     float L2 = L * a0, O2 = O * a0;
-#pragma unroll 4
-    for (int i = 0; i < sB.npieces; ++i) {
-      const float* pp = p.part + (size_t)(sB.pbase + i) * PF;
-      const float a = ex2(__ldcg(pp + GD + h) - M2u);
-      L2 += __ldcg(pp + GD + G + h) * a;
-      O2 += __ldcg(pp + idx) * a;
+#pragma unroll 8
+    for (int i = nA; i < n; ++i) {
+      const float a = ex2(pm(i, h) - M2u);
+      L2 += pl_(i, h) * a;
+      O2 += __ldcg(p.part + (size_t)(sB.pbase + (i - nA)) * PF + idx) * a;
     }
     const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
     p.out[orow * D + d] = O2 / L2;
@@ -354,6 +379,8 @@ __device__ void merge_unit(const AttendParams& p, int u) {
     p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
     p.unit_cnt[u] = 0;
   }
+  // wbuf is reused by the next piece
+  return consumer_sync(sm, sync_phase, p.status);
 }
 
 // Combine the warp's 4 lane groups (each holds its own running max, sum and
@@ -412,21 +439,37 @@ __device__ __forceinline__ void warp_combine_store(Acc<D>& A, float* wb) {
   }
 }
 
-// Merge the states of warps [w0, w1) for output element idx of head h:
-// returns (M, L, O) with O and L relative to 2^M.
+// Merge the warps' states for output element idx of head h: warps below wA
+// into (MA, LA, OA), the others into (MB, LB, OB); sums relative to 2^M.
 template <int D>
-__device__ __forceinline__ void combine_warps(const AttnSmem<D>& sm, int w0, int w1, int idx, int h, float& M,
-                                              float& L, float& O) {
+__device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, int idx, int h, float& MA, float& LA,
+                                               float& OA, float& MB, float& LB, float& OB) {
   constexpr int G = kGroup, GD = Cfg<D>::GD;
-  M = -INFINITY;
-  for (int w = w0; w < w1; ++w) M = fmaxf(M, sm.wbuf[w][GD + h]);
-  const float Mu = M == -INFINITY ? 0.f : M;
-  L = 0.f;
-  O = 0.f;
-  for (int w = w0; w < w1; ++w) {
-    const float a = ex2(sm.wbuf[w][GD + h] - Mu);
-    O += sm.wbuf[w][idx] * a;
-    L += sm.wbuf[w][GD + G + h] * a;
+  float m[kConsumerWarps], l[kConsumerWarps], o[kConsumerWarps];
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) {
+    m[w] = sm.wbuf[w][GD + h];
+    l[w] = sm.wbuf[w][GD + G + h];
+    o[w] = sm.wbuf[w][idx];
+  }
+  MA = MB = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) {
+    if (w < wA) MA = fmaxf(MA, m[w]);
+    else MB = fmaxf(MB, m[w]);
+  }
+  const float MAu = MA == -INFINITY ? 0.f : MA, MBu = MB == -INFINITY ? 0.f : MB;
+  LA = OA = LB = OB = 0.f;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) {
+    const float a = ex2(m[w] - (w < wA ? MAu : MBu));
+    if (w < wA) {
+      LA += l[w] * a;
+      OA += o[w] * a;
+    } else {
+      LB += l[w] * a;
+      OB += o[w] * a;
+    }
   }
 }
 
@@ -441,8 +484,8 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
   float* dst = p.part + (size_t)pidx * PF;
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
     const int h = idx / D;
-    float M, L, O;
-    combine_warps<D>(sm, 0, kConsumerWarps, idx, h, M, L, O);
+    float MA, LA, OA, M, L, O;
+    combine_warps2<D>(sm, 0, idx, h, MA, LA, OA, M, L, O);
     dst[idx] = O;
     if (idx - h * D == 0) {
       dst[GD + h] = M;
@@ -458,7 +501,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
-    merge_unit<D>(p, unit);
+    return merge_unit<D>(p, sm, unit, sync_phase);
   }
   return true;
 }
@@ -467,10 +510,9 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
 // warps [wA, 8) the tail [c_t, p_t].  New prefix state = reused ring state
 // (on a hit) + amend; output = new prefix + tail.  No partials, no counters.
 template <int D>
-__device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int u, int wA,
-                              uint32_t& sync_phase) {
+__device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int u, int wA, int hit,
+                              int src, int dst, int end, uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD;
-  const UnitPlan pl = p.plan[u];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
   // the reused state is independent of the combine: fetch it first
@@ -482,8 +524,8 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
     ro[k] = 0.f;
     rm[k] = -INFINITY;
     rl[k] = 0.f;
-    if (pl.hit && idx < GD) {
-      const size_t rs = (size_t)u * Wp1 + pl.src_slot;
+    if (hit && idx < GD) {
+      const size_t rs = (size_t)u * Wp1 + src;
       const int h = idx / D;
       ro[k] = p.ring_o[rs * GD + idx];
       rm[k] = p.ring_m[rs * G + h] * kLog2e;
@@ -498,19 +540,18 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
     if (idx >= GD) break;
     const int h = idx / D, d = idx - h * D;
     float MA, LA, OA, MB, LB, OB;
-    combine_warps<D>(sm, 0, wA, idx, h, MA, LA, OA);
-    combine_warps<D>(sm, wA, kConsumerWarps, idx, h, MB, LB, OB);
+    combine_warps2<D>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
     // new prefix state S = reused (hit) + amend
-    float M = fmaxf(MA, pl.hit ? rm[k] : -INFINITY);
+    float M = fmaxf(MA, hit ? rm[k] : -INFINITY);
     const float Mu = M == -INFINITY ? 0.f : M;
     const float aA = ex2(MA - Mu);
     float L = LA * aA, O = OA * aA;
-    if (pl.hit) {
+    if (hit) {
       const float a = ex2(rm[k] - Mu);
       L += rl[k] * a;
       O += ro[k] * rl[k] * a;
     }
-    const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
+    const size_t ds = (size_t)u * Wp1 + dst;
     p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
     if (d == 0) {
       p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
@@ -525,7 +566,7 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
     p.out[orow * D + d] = O2 / L2;
     if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
   }
-  if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
+  if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
   // the warps' slots are reused by the next piece
   return consumer_sync(sm, sync_phase, p.status);
 }
@@ -535,6 +576,7 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
 // both segments of a small unit: A = [a0, a1) (may be empty), B = [k0, k1).
 struct Piece {
   int unit, pidx, whole;
+  int hit, src, dst;          // whole unit: plan of the unit (end = k1)
   int k0, k1, kb0, nbox;      // split: its keys; whole unit: segment B
   int a0, a1, akb0, anbox;    // whole unit: segment A
   int wA;                     // whole unit: warps on segment A
@@ -570,9 +612,11 @@ __device__ __forceinline__ int box_count(int k0, int k1) {
 struct Walker {
   int s;
   long long lo, hi;
+  const Segment* cache;  // shared-memory copy of items [base, base + kItemCache)
+  int base;
   __device__ __forceinline__ bool next(const AttendParams& p, int cta, Piece& pc) {
     while (s < p.nseg) {
-      const Segment sg = p.seg[s];
+      const Segment sg = (s - base < kItemCache) ? cache[s - base] : p.seg[s];
       const int cur = s++;
       if (sg.kind < 0) continue;
       if (sg.flat >= hi) {  // this and every later item start past the range
@@ -585,6 +629,9 @@ struct Walker {
         const int start = sg.key0, cut = sg.pbase, end = sg.key0 + sg.len;
         pc.whole = 1;
         pc.pidx = -1;
+        pc.hit = sg.npieces & 1;
+        pc.src = (sg.npieces >> 1) & 0x7ff;
+        pc.dst = (sg.npieces >> 12) & 0x7ff;
         pc.a0 = start;
         pc.a1 = cut;
         pc.akb0 = start & ~(kSubKeys - 1);
@@ -641,16 +688,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   // launched with programmatic stream serialization: everything above
   // overlaps the match kernel; its results are visible after this wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // one round of loads: the split, then the CTA's items into shared memory
   const int n_cta = p.hdr->n_cta;
-  if (cta >= n_cta) return;
-
   const long long T = p.hdr->total;
-  const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
   const int first_seg = p.first_seg[cta];
+  if (cta >= n_cta) return;
+  const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
+  if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = p.seg[first_seg + tid];
+  __syncthreads();
   const uint64_t pol = evict_first_policy();
 
   // issue cursor: this warp's boxes of every piece, NST ahead
-  Walker wi{first_seg, lo, hi};
+  Walker wi{first_seg, lo, hi, sm.items, first_seg};
   Piece ip;
   WarpRange ir;
   bool ivalid = wi.next(p, cta, ip);
@@ -699,7 +748,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 
   // consume cursor
   Acc<D> A;
-  Walker wc{first_seg, lo, hi};
+  Walker wc{first_seg, lo, hi, sm.items, first_seg};
   Piece cp;
   int cpn = 0, cons = 0, par = 0;
   uint32_t sync_phase = 0;
@@ -749,7 +798,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
     }
     if (!ok) break;
-    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, sync_phase)
+    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.src, cp.dst, cp.k1, sync_phase)
                               : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (!fin) break;
     ++cpn;

@@ -46,7 +46,8 @@ struct Segment {
   int key0;        // first key (absolute position in the sequence)
   int first_cta;   // split: CTA holding `flat`; whole: the owning CTA
   int pbase;       // split: index of the first partial result; whole: the cut c_t
-  int npieces;     // split: partial results (CTAs overlapping the keys); whole: 0
+  int npieces;     // split: partial results (CTAs overlapping the keys);
+                   // whole: hit | reused slot << 1 | written slot << 12
   int kind;        // kItem*
 };
 

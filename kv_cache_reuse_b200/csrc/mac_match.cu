@@ -87,7 +87,7 @@ __device__ void build_segments(const MatchParams& p, int U) {
   long long carry = 0;
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
-    int len = 0, key0 = 0, kind = kItemEmpty, cut = 0;
+    int len = 0, key0 = 0, kind = kItemEmpty, cut = 0, packed = 0;
     long long wlen = 0;
     if (s < nseg) {
       const UnitPlan* pl = p.plan + (s >> 1);
@@ -100,6 +100,9 @@ __device__ void build_segments(const MatchParams& p, int U) {
             len = end - start;
             key0 = start;
             cut = c;
+            // the CTA doing it also needs hit, reused slot and written slot
+            const int hit = __ldcg(&pl->hit), src = __ldcg(&pl->src_slot), dst = __ldcg(&pl->dst_slot);
+            packed = (hit ? 1 : 0) | ((hit ? src : 0) << 1) | (dst << 12);
           }
         } else {
           len = (s & 1) ? end - c : c - start;
@@ -118,6 +121,7 @@ __device__ void build_segments(const MatchParams& p, int U) {
       p.seg[s].key0 = key0;
       p.seg[s].kind = kind;
       p.seg[s].pbase = cut;  // whole items keep their cut here; split items overwrite it below
+      if (kind == kItemWhole) p.seg[s].npieces = packed;
     }
     carry += tot;
   }
@@ -152,8 +156,10 @@ __device__ void build_segments(const MatchParams& p, int U) {
     const int np_next = __shfl_down_sync(0xffffffffu, np, 1);
     if (s < nseg) {
       p.seg[s].first_cta = first;
-      p.seg[s].npieces = np;
-      if (kind != kItemWhole) p.seg[s].pbase = (int)(pcarry + ex);
+      if (kind != kItemWhole) {
+        p.seg[s].npieces = np;
+        p.seg[s].pbase = (int)(pcarry + ex);
+      }
       if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
       // CTAs whose range starts inside this item's cost extent [Fw, Fe)
       // begin their walk here: lo_c = floor(c*T/N) lies in it iff
