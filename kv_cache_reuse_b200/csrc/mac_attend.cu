@@ -675,6 +675,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int cta = blockIdx.x;
+  if (tid == 32) {  // bring both TMA descriptors on chip while the match kernel runs
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmK)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmV)) : "memory");
+  }
   if (tid == 0) {
     for (int w = 0; w < kConsumerWarps; ++w)
       for (int s = 0; s < NST; ++s) mbar_init(&sm.full[w][s], 1);

@@ -85,6 +85,8 @@ __device__ void build_segments(const MatchParams& p, int U) {
   const long long cost = p.piece_cost;
   // pass 1: item kinds, keys and cost-space offsets
   long long carry = 0;
+  long long r_flat = 0;  // this thread's item, kept for pass 2 when nseg <= kMatchThreads
+  int r_len = 0, r_kind = kItemEmpty;
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
     int len = 0, key0 = 0, kind = kItemEmpty, cut = 0, packed = 0;
@@ -117,6 +119,9 @@ __device__ void build_segments(const MatchParams& p, int U) {
     if (s < nseg) {
       const bool split = kind == kItemA || kind == kItemB;
       p.seg[s].flat = carry + ex + (split ? cost : 0);
+      r_flat = carry + ex + (split ? cost : 0);
+      r_len = kind == kItemEmpty ? 0 : len;
+      r_kind = kind;
       p.seg[s].len = kind == kItemEmpty ? 0 : len;
       p.seg[s].key0 = key0;
       p.seg[s].kind = kind;
@@ -140,9 +145,15 @@ __device__ void build_segments(const MatchParams& p, int U) {
     int np = 0, first = 0, kind = kItemEmpty, len = 0;
     long long F = 0;
     if (s < nseg) {
-      F = p.seg[s].flat;
-      len = p.seg[s].len;
-      kind = p.seg[s].kind;
+      if (nseg <= kMatchThreads) {
+        F = r_flat;
+        len = r_len;
+        kind = r_kind;
+      } else {
+        F = p.seg[s].flat;
+        len = p.seg[s].len;
+        kind = p.seg[s].kind;
+      }
       if (kind == kItemA || kind == kItemB) {
         first = cta_of(F, T, N);
         np = cta_of(F + len - 1, T, N) - first + 1;
@@ -366,10 +377,11 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     }
   }
 
-  // last CTA to arrive builds the segment table for the attention kernel
-  __threadfence();
-  __syncthreads();
+  // last CTA to arrive builds the segment table for the attention kernel.
+  // Only the plan (written by thread 0) is read by that CTA; everything else
+  // goes to the attention kernel, which starts after this grid completes.
   if (tid == 0) {
+    __threadfence();
     const int ticket = atomicAdd(p.done, 1);
     s_last = (ticket == (int)gridDim.x - 1);
   }
