@@ -69,6 +69,7 @@ struct __align__(128) AttnSmem {
   unsigned long long csync;
   int abort_flag;
   int last_flag;
+  int warm_sink;              // keeps the instruction warm-up from being optimised away
   Segment items[kItemCache];  // the CTA's work items, from its first one on
 };
 
@@ -160,10 +161,13 @@ struct Acc {
 };
 
 // One 16-key box for one warp.  Group g (lanes 8g..8g+7) takes keys 4g..4g+3
-// of the box; lane j of a group holds dims [64v + 8j, 64v + 8j + 8).
-template <int D, bool MASKED>
-__device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, const uint16_t* vbox, float* pbuf,
-                                            int key_box, int k0, int k1) {
+// of the box; lane j of a group holds dims [64v + 8j, 64v + 8j + 8).  A box
+// at the edge of its range (masked) has rows outside [k0, k1): their scores
+// become -inf and their V rows are zeroed in shared memory (the rows may hold
+// anything, NaN included, and 0 * NaN would poison the sum).
+template <int D>
+__device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, uint16_t* vbox, float* pbuf,
+                                            int key_box, int k0, int k1, bool masked) {
   constexpr int NV = Cfg<D>::NV;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 3, j = lane & 7;
@@ -214,9 +218,15 @@ __device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, con
     sc[i] = keep + __shfl_xor_sync(kFull, send, 1);
   }
   const int kkl = (b2 ? 2 : 0) + (b1 ? 1 : 0);
-  if (MASKED) {
+  if (masked) {
     const int key = key_box + 4 * g + kkl;
     if (key < k0 || key >= k1) sc[0] = sc[1] = -INFINITY;
+    constexpr int VPR = D / 8;  // uint4 per row
+    for (int i = lane; i < kSubKeys * VPR; i += 32) {
+      const int row = i / VPR;
+      if (key_box + row < k0 || key_box + row >= k1)
+        reinterpret_cast<uint4*>(vbox)[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
   // block max per head over the group's 4 keys
   float bm0 = fmaxf(sc[0], __shfl_xor_sync(kFull, sc[0], 4));
@@ -262,15 +272,9 @@ __device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, con
     const float4 pc = *reinterpret_cast<const float4*>(pg + kk * 8 + 4);
     const float2 pp[4] = {make_float2(pa.x, pa.y), make_float2(pa.z, pa.w), make_float2(pc.x, pc.y),
                           make_float2(pc.z, pc.w)};
-    bool valid = true;
-    if (MASKED) {
-      const int key = key_box + 4 * g + kk;
-      valid = key >= k0 && key < k1;
-    }
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
-      uint4 vr = *reinterpret_cast<const uint4*>(vg + kk * D + 64 * v);
-      if (MASKED && !valid) vr = make_uint4(0u, 0u, 0u, 0u);
+      const uint4 vr = *reinterpret_cast<const uint4*>(vg + kk * D + 64 * v);
       const uint32_t w4[4] = {vr.x, vr.y, vr.z, vr.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -689,6 +693,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  // Instruction warm-up: while the match kernel still runs, execute the box
+  // and combine code once on this CTA's not-yet-used shared memory, so the
+  // real pass does not start on a cold instruction cache (the values are
+  // discarded; only a shared-memory sink keeps the code alive).
+  {
+    Acc<D> W;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      W.m[h] = -INFINITY;
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) W.q[h][v][e] = W.o[h][v][e] = make_float2(0.f, 0.f);
+    }
+    W.l[0] = W.l[1] = 0.f;
+    process_box<D>(W, sm.kv[warp][0][0], sm.kv[warp][0][1], sm.wbuf[warp], 0, 0, kSubKeys, true);
+    warp_combine_store<D>(W, sm.wbuf[warp]);
+    __syncwarp();
+    float MA, LA, OA, MB, LB, OB;
+    combine_warps2<D>(sm, 4, lane, 0, MA, LA, OA, MB, LB, OB);
+    if (lane == 0) sm.warm_sink = __float_as_int(LA + OA + LB + OB + MA + MB);
+  }
+  __syncthreads();
   // launched with programmatic stream serialization: everything above
   // overlaps the match kernel; its results are visible after this wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -789,10 +816,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
       const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * 144;
-      if (key_box < cr.k0 || key_box + kSubKeys > cr.k1)
-        process_box<D, true>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1);
-      else
-        process_box<D, false>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1);
+      process_box<D>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
+                     key_box < cr.k0 || key_box + kSubKeys > cr.k1);
       par ^= 1;
       ++cons;
       __syncwarp();
