@@ -123,10 +123,10 @@ int encode_kv_map(MacState* s, CUtensorMap* map, const void* base) {
   strides[0] = D * 2;
   strides[1] = H * D * 2;
   strides[2] = dims[2] * H * D * 2;
-  const cuuint32_t box[4] = {(cuuint32_t)D, 1u, (cuuint32_t)kSubKeys, 1u};
+  const cuuint32_t box[4] = {64u, 1u, (cuuint32_t)kSubKeys, 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MAC_OK : MAC_ERR_CUDA;
 }

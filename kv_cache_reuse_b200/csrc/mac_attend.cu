@@ -17,13 +17,23 @@
 // Per CTA: eight warps; warp w owns boxes w, w+8, w+16, ... of every piece,
 // where a box is 16 keys (it never crosses a page).  Each warp streams its
 // own boxes through its own ring of shared-memory slots with TMA
-// (cp.async.bulk.tensor, no multicast), keeping NST boxes in flight, so the
-// warps never wait on one another inside a piece.  Within a box a group of 8
-// lanes owns 4 keys and each lane owns D/8 dimensions of every head of the
-// GQA group (G = 4): q . k is a partial dot product per lane followed by a
-// reduce-scatter over the 8 lanes.  The work is HBM-bound (4 flop per byte
-// of K/V): the math stays on the FP32 pipes (packed f32x2 FMA), not on the
-// tensor cores, since a 4-row query tile is not a dense contraction.
+// (cp.async.bulk.tensor, 128-byte swizzle, no multicast), keeping NST boxes
+// in flight, so the warps never wait on one another inside a piece.
+//
+// A box is a small dense product on the tensor cores (mma.sync m16n8k16,
+// bf16 in, fp32 accumulate), keys on the M side:
+//   S^T[16 keys x 8] = K[16 x D] . Qx[D x 8]     (QK, D/16 k-steps)
+//   O^T[D x 8]      += V^T[D x 16] . Px[16 x 8]  (PV, D/16 row tiles)
+// The 8 columns are the 4 query heads of the GQA group twice: the fp32
+// query (and the fp32 softmax weights) split into a bf16 high part and a
+// bf16 residual, so every column carries data and the products keep ~16
+// mantissa bits; score = column h + column h+4.  This is not about tensor
+// throughput -- the work is HBM-bound (4 flop per byte of K/V) -- but about
+// instruction issue: a box costs ~100 warp instructions instead of ~700 on
+// the FP32 pipes, which keeps the miss path on the memory roofline and a
+// hit's few boxes short.  K fragments come from ldmatrix, V^T fragments from
+// ldmatrix.trans (the swizzle keeps both conflict-free); the weights reach
+// their B-fragment layout through 256 bytes of shared memory per warp.
 //
 // Softmax runs in exp2 units (the query is pre-scaled by log2(e)/sqrt(D)).
 // Every piece a CTA processes ends in a partial (o unnormalised, m, l).  The
@@ -35,6 +45,8 @@
 // MAC_DEV_TIMEOUT in the status word and leaves without hanging the GPU.
 #include <math.h>
 #include <stdint.h>
+
+#include <cuda_bf16.h>
 
 #include "mac_internal.cuh"
 
@@ -51,25 +63,26 @@ constexpr int kItemCache = 64;  // work items of one CTA kept in shared memory
 
 template <int D>
 struct Cfg {
-  static constexpr int NV = D / 64;  // 8-dim vectors per lane per row
-  static constexpr int NST = D == 128 ? 3 : 6;  // boxes in flight per warp
-  static constexpr int NQ = NST + 1;             // query buffers (pieces the issue cursor can be ahead)
+  static constexpr int KS = D / 16;               // k-steps of QK = row tiles of PV
+  static constexpr int HALVES = D / 64;           // 128-byte swizzled halves of a key row
+  static constexpr int NST = D == 128 ? 3 : 6;    // boxes in flight per warp
+  static constexpr int NQ = NST + 1;              // query buffers (pieces the issue cursor can be ahead)
   static constexpr int GD = kGroup * D;
   static constexpr int PF = kGroup * D + 2 * kGroup;  // floats of one partial
-  static constexpr int WB = (PF > 288 ? PF : 288);     // per-warp scratch floats
+  static constexpr int WB = (PF > 128 ? PF : 128);     // per-warp scratch floats
 };
 
 template <int D>
-struct __align__(128) AttnSmem {
-  uint16_t kv[kConsumerWarps][Cfg<D>::NST][2][kSubKeys * D];  // per warp: ring of (K box, V box)
-  float q[Cfg<D>::NQ][Cfg<D>::GD];                            // queries of the upcoming pieces
-  float wbuf[kConsumerWarps][Cfg<D>::WB];                     // weights exchange / piece combine
+struct __align__(1024) AttnSmem {
+  // per warp: ring of (K box, V box), each [HALVES][16 keys][64 dims] bf16, 128-byte swizzle
+  uint16_t kv[kConsumerWarps][Cfg<D>::NST][2][kSubKeys * D];
+  float q[Cfg<D>::NQ][Cfg<D>::GD];         // queries of the upcoming pieces
+  float wbuf[kConsumerWarps][Cfg<D>::WB];  // weights exchange / piece combine
   unsigned long long full[kConsumerWarps][Cfg<D>::NST];
   unsigned long long qfull[Cfg<D>::NQ];
   unsigned long long csync;
   int abort_flag;
   int last_flag;
-  int warm_sink;              // keeps the instruction warm-up from being optimised away
   Segment items[kItemCache];  // the CTA's work items, from its first one on
 };
 
@@ -146,143 +159,159 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
 }
-__device__ __forceinline__ float sel(bool c, float a, float b) { return c ? a : b; }
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D += A(16x16, row) . B(16x8, col), bf16 in, fp32 accumulate
+__device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Two fp32 values as bf16x2 (first in the low half), rounded to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// The bf16 residual pair of (a, b) after their bf16 rounding `hi`.
+__device__ __forceinline__ uint32_t pack_bf16_residual(float a, float b, uint32_t hi) {
+  return pack_bf16(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+// Byte offset of (key row, dim) in a box of [D/64][16][64] bf16 laid out by
+// TMA with the 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7).
+__device__ __forceinline__ uint32_t box_off(int row, int dim) {
+  return (uint32_t)((dim >> 6) * (kSubKeys * 128) + row * 128 + ((((dim >> 3) & 7) ^ (row & 7)) << 4) +
+                    (dim & 7) * 2);
+}
 
 // ------------------------------------------------------------ consumer state
+// Per warp, in mma fragment layout (lane = 4*gid + tig): the query columns
+// as B fragments, O^T as C fragments (dims 16*dt + gid and + 8, columns
+// 2*tig and 2*tig + 1), and the running max and sum of the two heads this
+// lane's columns belong to, hh = 2*(tig & 1) and hh + 1.
 template <int D>
 struct Acc {
-  float2 q[kGroup][Cfg<D>::NV][4];  // this lane's dims of every head, (even, odd) pairs
-  float2 o[kGroup][Cfg<D>::NV][4];  // unnormalised output accumulators
-  float m[kGroup];                  // running max (log2 units), same in all lanes of a group
-  float l[2];                       // running sum for heads 2*b0, 2*b0+1 over this lane's key
+  uint32_t qb[Cfg<D>::KS][2];
+  float o[Cfg<D>::KS][4];
+  float m[2];
+  float l[2];
 };
 
-// One 16-key box for one warp.  Group g (lanes 8g..8g+7) takes keys 4g..4g+3
-// of the box; lane j of a group holds dims [64v + 8j, 64v + 8j + 8).  A box
-// at the edge of its range (masked) has rows outside [k0, k1): their scores
-// become -inf and their V rows are zeroed in shared memory (the rows may hold
-// anything, NaN included, and 0 * NaN would poison the sum).
+// Load the query of a piece into B fragments: column n = gid is head
+// (gid & 3), its bf16 high part for gid < 4 and its bf16 residual otherwise.
+template <int D>
+__device__ __forceinline__ void load_query(Acc<D>& A, const float* qs) {
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+  const float* qh = qs + (gid & 3) * D + 2 * tig;
+#pragma unroll
+  for (int ks = 0; ks < Cfg<D>::KS; ++ks) {
+    const float2 x01 = *reinterpret_cast<const float2*>(qh + ks * 16);
+    const float2 x89 = *reinterpret_cast<const float2*>(qh + ks * 16 + 8);
+    const uint32_t h0 = pack_bf16(x01.x, x01.y), h1 = pack_bf16(x89.x, x89.y);
+    A.qb[ks][0] = gid < 4 ? h0 : pack_bf16_residual(x01.x, x01.y, h0);
+    A.qb[ks][1] = gid < 4 ? h1 : pack_bf16_residual(x89.x, x89.y, h1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) A.o[ks][i] = 0.f;
+  }
+  A.m[0] = A.m[1] = -INFINITY;
+  A.l[0] = A.l[1] = 0.f;
+}
+
+// One 16-key box for one warp.  A box at the edge of its range (masked) has
+// rows outside [k0, k1): their scores become -inf and their V rows are
+// zeroed in shared memory (the rows may hold anything, NaN included, and
+// 0 * NaN would poison the sum).
 template <int D>
 __device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, uint16_t* vbox, float* pbuf,
                                             int key_box, int k0, int k1, bool masked) {
-  constexpr int NV = Cfg<D>::NV;
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 3, j = lane & 7;
-  const bool b2 = (j & 4) != 0, b1 = (j & 2) != 0, b0 = (j & 1) != 0;
-  const uint16_t* kg = kbox + (4 * g) * D + 8 * j;
-  const uint16_t* vg = vbox + (4 * g) * D + 8 * j;
+  constexpr int KS = Cfg<D>::KS;
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+  const int mj = lane >> 3, mr = lane & 7;  // ldmatrix: matrix and row this lane addresses
+  const uint32_t kb = smem_u32(kbox), vb = smem_u32(vbox);
 
-  // q . k partial sums over this lane's dims: acc[kk][h]
-  float s[16];
+  // S^T = K . Qx, two accumulator chains
+  float s[4] = {0.f, 0.f, 0.f, 0.f}, t[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    float2 acc[kGroup];
-#pragma unroll
-    for (int h = 0; h < kGroup; ++h) acc[h] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const uint4 kr = *reinterpret_cast<const uint4*>(kg + kk * D + 64 * v);
-      const uint32_t w4[4] = {kr.x, kr.y, kr.z, kr.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 kf = unpack_bf16x2(w4[e]);
-#pragma unroll
-        for (int h = 0; h < kGroup; ++h) acc[h] = __ffma2_rn(A.q[h][v][e], kf, acc[h]);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < kGroup; ++h) s[kk * 4 + h] = acc[h].x + acc[h].y;
+  for (int ks = 0; ks < KS; ++ks) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4(kb + box_off(mr + ((mj & 1) << 3), ks * 16 + ((mj >> 1) << 3)), a0, a1, a2, a3);
+    mma16816((ks & 1) ? t : s, a0, a1, a2, a3, A.qb[ks][0], A.qb[ks][1]);
   }
-  // reduce-scatter over the 8 lanes: bit 2 picks the key pair, bit 1 the
-  // key, bit 0 the head pair.  Lane ends with the full scores of key
-  // kk = 2*b2 + b1 for heads 2*b0 and 2*b0 + 1.
-  float t8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float keep = sel(b2, s[i + 8], s[i]), send = sel(b2, s[i], s[i + 8]);
-    t8[i] = keep + __shfl_xor_sync(kFull, send, 4);
-  }
-  float t4[4];
+  // high + residual columns: lane tig and tig ^ 2 hold columns n and n + 4.
+  // sc = (key gid, head hh), (gid, hh + 1), (gid + 8, hh), (gid + 8, hh + 1)
+  float sc[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float keep = sel(b1, t8[i + 4], t8[i]), send = sel(b1, t8[i], t8[i + 4]);
-    t4[i] = keep + __shfl_xor_sync(kFull, send, 2);
+    sc[i] = s[i] + t[i];
+    sc[i] += __shfl_xor_sync(kFull, sc[i], 2);
   }
-  float sc[2];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float keep = sel(b0, t4[i + 2], t4[i]), send = sel(b0, t4[i], t4[i + 2]);
-    sc[i] = keep + __shfl_xor_sync(kFull, send, 1);
-  }
-  const int kkl = (b2 ? 2 : 0) + (b1 ? 1 : 0);
   if (masked) {
-    const int key = key_box + 4 * g + kkl;
-    if (key < k0 || key >= k1) sc[0] = sc[1] = -INFINITY;
-    constexpr int VPR = D / 8;  // uint4 per row
-    for (int i = lane; i < kSubKeys * VPR; i += 32) {
-      const int row = i / VPR;
-      if (key_box + row < k0 || key_box + row >= k1)
-        reinterpret_cast<uint4*>(vbox)[i] = make_uint4(0u, 0u, 0u, 0u);
+    const int ka = key_box + gid, kc = ka + 8;
+    if (ka < k0 || ka >= k1) sc[0] = sc[1] = -INFINITY;
+    if (kc < k0 || kc >= k1) sc[2] = sc[3] = -INFINITY;
+    // zero whole V rows (both halves) outside the range
+    for (int i = lane; i < Cfg<D>::HALVES * kSubKeys * 8; i += 32) {
+      const int row = (i >> 3) & (kSubKeys - 1);
+      if (key_box + row < k0 || key_box + row >= k1) reinterpret_cast<uint4*>(vbox)[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  // block max per head over the group's 4 keys
-  float bm0 = fmaxf(sc[0], __shfl_xor_sync(kFull, sc[0], 4));
-  float bm1 = fmaxf(sc[1], __shfl_xor_sync(kFull, sc[1], 4));
-  bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, 2));
-  bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, 2));
-  const float om0 = __shfl_xor_sync(kFull, bm0, 1), om1 = __shfl_xor_sync(kFull, bm1, 1);
-  const float bmax[4] = {sel(b0, om0, bm0), sel(b0, om1, bm1), sel(b0, bm0, om0), sel(b0, bm1, om1)};
-  bool need = false;
-  float mnew[kGroup];
+  // box max per head over its 16 keys (rows gid and gid + 8 of every lane)
+  float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
 #pragma unroll
-  for (int h = 0; h < kGroup; ++h) {
-    mnew[h] = fmaxf(A.m[h], bmax[h]);
-    need |= mnew[h] > A.m[h];
+  for (int off = 4; off <= 16; off <<= 1) {
+    bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, off));
+    bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, off));
   }
-  if (__any_sync(kFull, need)) {
+  const float mn0 = fmaxf(A.m[0], bm0), mn1 = fmaxf(A.m[1], bm1);
+  if (__any_sync(kFull, mn0 > A.m[0] || mn1 > A.m[1])) {
+    const float a0 = ex2(A.m[0] - (mn0 == -INFINITY ? 0.f : mn0));
+    const float a1 = ex2(A.m[1] - (mn1 == -INFINITY ? 0.f : mn1));
 #pragma unroll
-    for (int h = 0; h < kGroup; ++h) {
-      const float mu = mnew[h] == -INFINITY ? 0.f : mnew[h];
-      const float a = ex2(A.m[h] - mu);
-      const float2 a2 = make_float2(a, a);
-#pragma unroll
-      for (int v = 0; v < NV; ++v)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) A.o[h][v][e] = __fmul2_rn(A.o[h][v][e], a2);
-      if (h == (b0 ? 2 : 0)) A.l[0] *= a;
-      if (h == (b0 ? 3 : 1)) A.l[1] *= a;
-      A.m[h] = mnew[h];
+    for (int dt = 0; dt < KS; ++dt) {
+      A.o[dt][0] *= a0;
+      A.o[dt][1] *= a1;
+      A.o[dt][2] *= a0;
+      A.o[dt][3] *= a1;
     }
+    A.l[0] *= a0;
+    A.l[1] *= a1;
+    A.m[0] = mn0;
+    A.m[1] = mn1;
   }
-  const float m0 = b0 ? A.m[2] : A.m[0], m1 = b0 ? A.m[3] : A.m[1];
-  const float p0 = ex2(sc[0] - (m0 == -INFINITY ? 0.f : m0));
-  const float p1 = ex2(sc[1] - (m1 == -INFINITY ? 0.f : m1));
-  A.l[0] += p0;
-  A.l[1] += p1;
-  // share the 16 weights of the group: float pairs (p, p) per (key, head)
-  float* pg = pbuf + g * 36;
-  *reinterpret_cast<float4*>(pg + kkl * 8 + 4 * (b0 ? 1 : 0)) = make_float4(p0, p0, p1, p1);
+  const float mu0 = A.m[0] == -INFINITY ? 0.f : A.m[0], mu1 = A.m[1] == -INFINITY ? 0.f : A.m[1];
+  const float p0 = ex2(sc[0] - mu0), p1 = ex2(sc[1] - mu1), p2 = ex2(sc[2] - mu0), p3 = ex2(sc[3] - mu1);
+  A.l[0] += p0 + p2;
+  A.l[1] += p1 + p3;
+  // weights P[key][head] through shared memory into the B fragments of Px:
+  // b0 = keys 2*tig, 2*tig + 1; b1 = keys 2*tig + 8, + 9; column gid
+  const int hh = 2 * (tig & 1);
+  if (tig < 2) {
+    *reinterpret_cast<float2*>(pbuf + gid * 4 + hh) = make_float2(p0, p1);
+    *reinterpret_cast<float2*>(pbuf + (gid + 8) * 4 + hh) = make_float2(p2, p3);
+  }
   __syncwarp();
+  const int hc = gid & 3;
+  const float x0 = pbuf[(2 * tig) * 4 + hc], x1 = pbuf[(2 * tig + 1) * 4 + hc];
+  const float x2 = pbuf[(2 * tig + 8) * 4 + hc], x3 = pbuf[(2 * tig + 9) * 4 + hc];
+  const uint32_t h0 = pack_bf16(x0, x1), h1 = pack_bf16(x2, x3);
+  const uint32_t pb0 = gid < 4 ? h0 : pack_bf16_residual(x0, x1, h0);
+  const uint32_t pb1 = gid < 4 ? h1 : pack_bf16_residual(x2, x3, h1);
+  // O^T += V^T . Px, one row tile of 16 dims per mma
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const float4 pa = *reinterpret_cast<const float4*>(pg + kk * 8);
-    const float4 pc = *reinterpret_cast<const float4*>(pg + kk * 8 + 4);
-    const float2 pp[4] = {make_float2(pa.x, pa.y), make_float2(pa.z, pa.w), make_float2(pc.x, pc.y),
-                          make_float2(pc.z, pc.w)};
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const uint4 vr = *reinterpret_cast<const uint4*>(vg + kk * D + 64 * v);
-      const uint32_t w4[4] = {vr.x, vr.y, vr.z, vr.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 vf = unpack_bf16x2(w4[e]);
-#pragma unroll
-        for (int h = 0; h < kGroup; ++h) A.o[h][v][e] = __ffma2_rn(pp[h], vf, A.o[h][v][e]);
-      }
-    }
+  for (int dt = 0; dt < KS; ++dt) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4_t(vb + box_off(mr + ((mj >> 1) << 3), dt * 16 + ((mj & 1) << 3)), a0, a1, a2, a3);
+    mma16816(A.o[dt], a0, a1, a2, a3, pb0, pb1);
   }
 }
 
@@ -387,58 +416,39 @@ __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32
   return consumer_sync(sm, sync_phase, p.status);
 }
 
-// Combine the warp's 4 lane groups (each holds its own running max, sum and
-// output) and store the warp's state in its shared-memory slot:
-// o [G][D] unnormalised, then m [G] and l [G].
+// Store the warp's state in its shared-memory slot: o [G][D] unnormalised,
+// then m [G] and l [G].  Lanes tig and tig ^ 2 hold the high and residual
+// columns of the same heads; lanes of one tig hold different key rows.
 template <int D>
 __device__ __forceinline__ void warp_combine_store(Acc<D>& A, float* wb) {
-  constexpr int NV = Cfg<D>::NV, G = kGroup, GD = Cfg<D>::GD;
-  const int lane = threadIdx.x & 31;
-  const int j = lane & 7;
-  const bool b0 = (j & 1) != 0;
+  constexpr int G = kGroup, GD = Cfg<D>::GD, KS = Cfg<D>::KS;
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+  const int hh = 2 * (tig & 1);
   __syncwarp();
-  // group sums of l for this lane's head pair, then all four heads
   float l0 = A.l[0], l1 = A.l[1];
-  l0 += __shfl_xor_sync(kFull, l0, 4);
-  l1 += __shfl_xor_sync(kFull, l1, 4);
-  l0 += __shfl_xor_sync(kFull, l0, 2);
-  l1 += __shfl_xor_sync(kFull, l1, 2);
-  const float o0 = __shfl_xor_sync(kFull, l0, 1), o1 = __shfl_xor_sync(kFull, l1, 1);
-  float lg[4] = {sel(b0, o0, l0), sel(b0, o1, l1), sel(b0, l0, o0), sel(b0, l1, o1)};
 #pragma unroll
-  for (int off = 8; off <= 16; off <<= 1) {
+  for (int off = 4; off <= 16; off <<= 1) {
+    l0 += __shfl_xor_sync(kFull, l0, off);
+    l1 += __shfl_xor_sync(kFull, l1, off);
+  }
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mo = __shfl_xor_sync(kFull, A.m[h], off);
-      const float M = fmaxf(A.m[h], mo);
-      const float Mu = M == -INFINITY ? 0.f : M;
-      const float a = ex2(A.m[h] - Mu), ao = ex2(mo - Mu);
-      lg[h] = lg[h] * a + __shfl_xor_sync(kFull, lg[h], off) * ao;
+  for (int dt = 0; dt < KS; ++dt)
 #pragma unroll
-      for (int v = 0; v < NV; ++v)
+    for (int i = 0; i < 4; ++i) A.o[dt][i] += __shfl_xor_sync(kFull, A.o[dt][i], 2);
+  if (tig < 2) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 x = A.o[h][v][e];
-          const float2 y = make_float2(__shfl_xor_sync(kFull, x.x, off), __shfl_xor_sync(kFull, x.y, off));
-          A.o[h][v][e] = make_float2(x.x * a + y.x * ao, x.y * a + y.y * ao);
-        }
-      A.m[h] = M;
+    for (int dt = 0; dt < KS; ++dt) {
+      const int d0 = dt * 16 + gid;
+      wb[hh * D + d0] = A.o[dt][0];
+      wb[(hh + 1) * D + d0] = A.o[dt][1];
+      wb[hh * D + d0 + 8] = A.o[dt][2];
+      wb[(hh + 1) * D + d0 + 8] = A.o[dt][3];
     }
-  }
-  if (lane < 8) {
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int v = 0; v < NV; ++v)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<float2*>(wb + h * D + 64 * v + 8 * j + 2 * e) = A.o[h][v][e];
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      wb[GD + h] = A.m[h];
-      wb[GD + G + h] = lg[h];
+    if (gid == 0) {
+      wb[GD + hh] = A.m[0];
+      wb[GD + hh + 1] = A.m[1];
+      wb[GD + G + hh] = l0;
+      wb[GD + G + hh + 1] = l1;
     }
   }
 }
@@ -672,10 +682,11 @@ struct Walker {
 
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
-  constexpr int NST = Cfg<D>::NST, NQ = Cfg<D>::NQ, NV = Cfg<D>::NV, G = kGroup, GD = Cfg<D>::GD;
+  constexpr int NST = Cfg<D>::NST, NQ = Cfg<D>::NQ, GD = Cfg<D>::GD;
   constexpr uint32_t kBoxBytes = kSubKeys * D * 2;
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw);
+  // the swizzled TMA boxes need 1024-byte alignment of the shared window
+  AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int cta = blockIdx.x;
@@ -691,29 +702,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     sm.abort_flag = 0;
     sm.last_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
-  // Instruction warm-up: while the match kernel still runs, execute the box
-  // and combine code once on this CTA's not-yet-used shared memory, so the
-  // real pass does not start on a cold instruction cache (the values are
-  // discarded; only a shared-memory sink keeps the code alive).
-  {
-    Acc<D> W;
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      W.m[h] = -INFINITY;
-#pragma unroll
-      for (int v = 0; v < NV; ++v)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) W.q[h][v][e] = W.o[h][v][e] = make_float2(0.f, 0.f);
-    }
-    W.l[0] = W.l[1] = 0.f;
-    process_box<D>(W, sm.kv[warp][0][0], sm.kv[warp][0][1], sm.wbuf[warp], 0, 0, kSubKeys, true);
-    warp_combine_store<D>(W, sm.wbuf[warp]);
-    __syncwarp();
-    float MA, LA, OA, MB, LB, OB;
-    combine_warps2<D>(sm, 4, lane, 0, MA, LA, OA, MB, LB, OB);
-    if (lane == 0) sm.warm_sink = __float_as_int(LA + OA + LB + OB + MA + MB);
   }
   __syncthreads();
   // launched with programmatic stream serialization: everything above
@@ -766,8 +754,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
         c3 = b;
       }
       mbar_arrive_expect_tx(&sm.full[warp][st], 2 * kBoxBytes);
-      tma_load_4d(sm.kv[warp][st][0], &p.tmK, &sm.full[warp][st], 0, kvh, c2, c3, pol);
-      tma_load_4d(sm.kv[warp][st][1], &p.tmV, &sm.full[warp][st], 0, kvh, c2, c3, pol);
+#pragma unroll
+      for (int hf = 0; hf < Cfg<D>::HALVES; ++hf) {
+        tma_load_4d(sm.kv[warp][st][0] + hf * kSubKeys * 64, &p.tmK, &sm.full[warp][st], 64 * hf, kvh, c2, c3, pol);
+        tma_load_4d(sm.kv[warp][st][1] + hf * kSubKeys * 64, &p.tmV, &sm.full[warp][st], 64 * hf, kvh, c2, c3, pol);
+      }
     }
     if (qfirst) ++nq_issued;
     ++nissued;
@@ -787,26 +778,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   while (ok && wc.next(p, cta, cp)) {
     const int qs = cpn % NQ;
     if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
-    {
-      const float* qsm = sm.q[qs];
-      const int j = lane & 7;
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          const float4 x = *reinterpret_cast<const float4*>(qsm + h * D + 64 * v + 8 * j);
-          const float4 y = *reinterpret_cast<const float4*>(qsm + h * D + 64 * v + 8 * j + 4);
-          A.q[h][v][0] = make_float2(x.x, x.y);
-          A.q[h][v][1] = make_float2(x.z, x.w);
-          A.q[h][v][2] = make_float2(y.x, y.y);
-          A.q[h][v][3] = make_float2(y.z, y.w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) A.o[h][v][e] = make_float2(0.f, 0.f);
-        }
-#pragma unroll
-      for (int h = 0; h < G; ++h) A.m[h] = -INFINITY;
-      A.l[0] = A.l[1] = 0.f;
-    }
+    load_query<D>(A, sm.q[qs]);
     const WarpRange cr = warp_range(cp, warp);
     for (int bj = cr.first; bj < cr.nbox; bj += cr.stride) {
       const int st = cons % NST;
@@ -815,7 +787,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
         break;
       }
       const int key_box = cr.kb0 + bj * kSubKeys;
-      float* pbuf = sm.wbuf[warp] + par * 144;
+      float* pbuf = sm.wbuf[warp] + par * 64;
       process_box<D>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
                      key_box < cr.k0 || key_box + kSubKeys > cr.k1);
       par ^= 1;
@@ -856,16 +828,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 }  // namespace
 
 size_t attend_smem_bytes(int D) {
-  return D == 128 ? sizeof(AttnSmem<128>) : sizeof(AttnSmem<64>);
+  return (D == 128 ? sizeof(AttnSmem<128>) : sizeof(AttnSmem<64>)) + 1024;
 }
 
 cudaError_t attend_prepare(int D) {
   if (D == 128)
     return cudaFuncSetAttribute(mac_attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sizeof(AttnSmem<128>));
+                                (int)attend_smem_bytes(128));
   if (D == 64)
     return cudaFuncSetAttribute(mac_attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sizeof(AttnSmem<64>));
+                                (int)attend_smem_bytes(64));
   return cudaErrorInvalidValue;
 }
 
@@ -883,11 +855,11 @@ cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (D == 128) {
-    cfg.dynamicSmemBytes = sizeof(AttnSmem<128>);
+    cfg.dynamicSmemBytes = attend_smem_bytes(128);
     return cudaLaunchKernelEx(&cfg, mac_attend_kernel<128>, p);
   }
   if (D == 64) {
-    cfg.dynamicSmemBytes = sizeof(AttnSmem<64>);
+    cfg.dynamicSmemBytes = attend_smem_bytes(64);
     return cudaLaunchKernelEx(&cfg, mac_attend_kernel<64>, p);
   }
   return cudaErrorInvalidValue;
