@@ -779,6 +779,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     const int qs = cpn % NQ;
     if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
     load_query<D>(A, sm.q[qs]);
+    if (warp == 0 && cp.whole && cp.hit) {
+      // the merge at the end of the piece reads the reused ring state: start
+      // bringing it into L2 now (o: G*D floats, m and l: G floats each)
+      const size_t rs = (size_t)cp.unit * (p.W + 1) + cp.src;
+      const char* ro = reinterpret_cast<const char*>(p.ring_o + rs * GD);
+      if (lane < GD * 4 / 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(ro + lane * 128));
+      if (lane == 31) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ring_m + rs * kGroup));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ring_l + rs * kGroup));
+      }
+    }
     const WarpRange cr = warp_range(cp, warp);
     for (int bj = cr.first; bj < cr.nbox; bj += cr.stride) {
       const int st = cons % NST;
