@@ -81,9 +81,11 @@ struct __align__(1024) AttnSmem {
   unsigned long long full[kConsumerWarps][Cfg<D>::NST];
   unsigned long long qfull[Cfg<D>::NQ];
   unsigned long long csync;
+  unsigned long long rfull;          // reused ring state of the current whole-unit piece landed
   int abort_flag;
   int last_flag;
-  Segment items[kItemCache];  // the CTA's work items, from its first one on
+  Segment items[kItemCache];         // the CTA's work items, from its first one on
+  alignas(16) float ring[Cfg<D>::GD + 2 * kGroup];  // that ring state: o [G][D], m [G], l [G]
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -525,29 +527,15 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
 // (on a hit) + amend; output = new prefix + tail.  No partials, no counters.
 template <int D>
 __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int u, int wA, int hit,
-                              int src, int dst, int end, uint32_t& sync_phase) {
+                              int dst, int end, uint32_t ring_phase, uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
-  // the reused state is independent of the combine: fetch it first
   constexpr int PER = (GD + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
-  float ro[PER], rm[PER], rl[PER];
-#pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int idx = threadIdx.x + k * kConsumerWarps * 32;
-    ro[k] = 0.f;
-    rm[k] = -INFINITY;
-    rl[k] = 0.f;
-    if (hit && idx < GD) {
-      const size_t rs = (size_t)u * Wp1 + src;
-      const int h = idx / D;
-      ro[k] = p.ring_o[rs * GD + idx];
-      rm[k] = p.ring_m[rs * G + h] * kLog2e;
-      rl[k] = p.ring_l[rs * G + h];
-    }
-  }
   warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  // the reused state was copied on chip at the start of the piece
+  if (hit && !mbar_wait(&sm.rfull, ring_phase, &sm.abort_flag, p.status)) return false;
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
     const int idx = threadIdx.x + k * kConsumerWarps * 32;
@@ -556,14 +544,15 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
     float MA, LA, OA, MB, LB, OB;
     combine_warps2<D>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
     // new prefix state S = reused (hit) + amend
-    float M = fmaxf(MA, hit ? rm[k] : -INFINITY);
+    const float rm = hit ? sm.ring[GD + h] * kLog2e : -INFINITY;
+    float M = fmaxf(MA, rm);
     const float Mu = M == -INFINITY ? 0.f : M;
     const float aA = ex2(MA - Mu);
     float L = LA * aA, O = OA * aA;
     if (hit) {
-      const float a = ex2(rm[k] - Mu);
-      L += rl[k] * a;
-      O += ro[k] * rl[k] * a;
+      const float a = ex2(rm - Mu), rl = sm.ring[GD + kGroup + h];
+      L += rl * a;
+      O += sm.ring[idx] * rl * a;
     }
     const size_t ds = (size_t)u * Wp1 + dst;
     p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
@@ -699,6 +688,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       for (int s = 0; s < NST; ++s) mbar_init(&sm.full[w][s], 1);
     for (int s = 0; s < NQ; ++s) mbar_init(&sm.qfull[s], 1);
     mbar_init(&sm.csync, kConsumerWarps);
+    mbar_init(&sm.rfull, 1);
     sm.abort_flag = 0;
     sm.last_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -773,22 +763,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   Walker wc{first_seg, lo, hi, sm.items, first_seg};
   Piece cp;
   int cpn = 0, cons = 0, par = 0;
-  uint32_t sync_phase = 0;
+  uint32_t sync_phase = 0, ring_phase = 0;
+  bool ring_pending = false;  // a reused-state copy was issued and not yet waited for
   bool ok = true;
   while (ok && wc.next(p, cta, cp)) {
     const int qs = cpn % NQ;
     if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
     load_query<D>(A, sm.q[qs]);
-    if (warp == 0 && cp.whole && cp.hit) {
-      // the merge at the end of the piece reads the reused ring state: start
-      // bringing it into L2 now (o: G*D floats, m and l: G floats each)
+    const bool ring_copy = cp.whole && cp.hit;
+    ring_pending = ring_copy;
+    if (ring_copy && tid == 0) {
+      // the merge at the end of the piece reads the reused ring state: copy
+      // it on chip now (the previous piece's merge is done with the buffer)
       const size_t rs = (size_t)cp.unit * (p.W + 1) + cp.src;
-      const char* ro = reinterpret_cast<const char*>(p.ring_o + rs * GD);
-      if (lane < GD * 4 / 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(ro + lane * 128));
-      if (lane == 31) {
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ring_m + rs * kGroup));
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.ring_l + rs * kGroup));
-      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&sm.rfull, (GD + 2 * kGroup) * 4);
+      bulk_load(sm.ring, p.ring_o + rs * GD, GD * 4, &sm.rfull);
+      bulk_load(sm.ring + GD, p.ring_m + rs * kGroup, kGroup * 4, &sm.rfull);
+      bulk_load(sm.ring + GD + kGroup, p.ring_l + rs * kGroup, kGroup * 4, &sm.rfull);
     }
     const WarpRange cr = warp_range(cp, warp);
     for (int bj = cr.first; bj < cr.nbox; bj += cr.stride) {
@@ -810,8 +802,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
     }
     if (!ok) break;
-    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.src, cp.dst, cp.k1, sync_phase)
+    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, ring_phase, sync_phase)
                               : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    if (ring_copy) ring_phase ^= 1u;
+    ring_pending = false;
     if (!fin) break;
     ++cpn;
   }
@@ -825,6 +819,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
         }
       }
       if (warp == 0) {
+        // a reused-state copy of an unfinished hit piece may still be in flight
+        const unsigned long long tr = globaltimer();
+        while (ring_pending && !mbar_try_wait(&sm.rfull, ring_phase) && globaltimer() - tr < 100000000ull) {
+        }
         for (int k = cpn; k < nq_issued; ++k) {
           const unsigned long long t0 = globaltimer();
           while (!mbar_try_wait(&sm.qfull[k % NQ], (uint32_t)(k / NQ) & 1u) && globaltimer() - t0 < 100000000ull) {
