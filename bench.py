@@ -139,18 +139,34 @@ def step_bytes(wl, hit, mpos, seq_lens, occ):
     return mt, att + kv, kv
 
 
+def rank_workload(args, rank):
+    """The workload one rank runs: every rank takes its own batch (its own seed),
+    so ranks share no data and the job scales weakly with no collective."""
+    base = synth.WORKLOADS[args.workload]
+    if args.batch:
+        base = base.with_(B=args.batch, L0=base.L0[:1] * args.batch)
+    if args.tau is not None:
+        base = base.with_(tau=args.tau)
+    return base, base.with_(seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over the ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_mac(args, rank, world, local_rank):
     import torch
     import kv_cache_reuse_b200 as mac
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    base = synth.WORKLOADS[args.workload]
-    if args.batch:
-        base = base.with_(B=args.batch, L0=base.L0[:1] * args.batch)
-    if args.tau is not None:
-        base = base.with_(tau=args.tau)
-    wl = base.with_(seed=base.seed + 1000 * rank)  # every rank: its own batch
+    base, wl = rank_workload(args, rank)
     T = max(base.steps, args.warmup + args.steps)
     stream = synth.queries(wl, T)
     cache = synth.kv_cache(wl, T)
@@ -244,11 +260,7 @@ def run_mac(args, rank, world, local_rank):
     allmiss = timed_run(0.0, 3, min(args.miss_steps, T - 3), split=True) if args.miss_steps > 0 else None
 
     # max over ranks of the timed duration
-    tot = main["total_ms"]
-    if world > 1:
-        tt = torch.tensor([tot], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        tot = float(tt.item())
+    tot = max_over_ranks(main["total_ms"], world, dev)
 
     e2e = None
     if not args.no_e2e:
@@ -336,10 +348,7 @@ def run_e2e(args, wl, stream, cache, K, V, bt, kw, dev, world):
         if t >= args.warmup:
             tot += t1 - t0
     st.close()
-    if world > 1:
-        tt = torch.tensor([tot], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        tot = float(tt.item())
+    tot = max_over_ranks(tot, world, dev)
     h2d = B * Hq * D * 4 + 2 * B * 4 + 2 * B * Hkv * D * 2
     d2h = B * Hq * D * 4 + B * Hq * 4 + B * Hkv + B * Hkv * 4 + 4
     return {"value": world * args.steps / tot, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

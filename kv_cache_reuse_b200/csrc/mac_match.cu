@@ -74,8 +74,16 @@ __device__ long long block_exclusive_scan(long long v, long long* total, long lo
 
 // CTA holding cost-space offset x when the space [0, T) is split over N CTAs
 // as [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
-__device__ __forceinline__ int cta_of(long long x, long long T, int N) {
-  return (int)(((x + 1) * (long long)N + T - 1) / T) - 1;
+// ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit integer
+// division: an fp64 estimate (off by at most a few units) corrected exactly.
+__device__ __forceinline__ long long ceil_div(long long a, long long b, double rb) {
+  long long q = (long long)((double)a * rb);
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;  // q = floor(a / b)
+  return q + (q * b < a ? 1 : 0);
+}
+__device__ __forceinline__ int cta_of(long long x, long long T, int N, double rT) {
+  return (int)ceil_div((x + 1) * (long long)N, T, rT) - 1;
 }
 
 __device__ void build_segments(const MatchParams& p, int U) {
@@ -137,6 +145,7 @@ __device__ void build_segments(const MatchParams& p, int U) {
     N = (int)(want < (long long)p.grid ? want : (long long)p.grid);
     if (N < 1) N = 1;
   }
+  const double rT = T > 0 ? 1.0 / (double)T : 0.0;
   __syncthreads();
   // pass 2: owning / first CTA, partial slots, and each CTA's first item
   long long pcarry = 0;
@@ -155,10 +164,10 @@ __device__ void build_segments(const MatchParams& p, int U) {
         kind = p.seg[s].kind;
       }
       if (kind == kItemA || kind == kItemB) {
-        first = cta_of(F, T, N);
-        np = cta_of(F + len - 1, T, N) - first + 1;
+        first = cta_of(F, T, N, rT);
+        np = cta_of(F + len - 1, T, N, rT) - first + 1;
       } else if (kind == kItemWhole) {
-        first = cta_of(F, T, N);
+        first = cta_of(F, T, N, rT);
       }
     }
     long long tot;
@@ -179,7 +188,7 @@ __device__ void build_segments(const MatchParams& p, int U) {
         const bool split = kind == kItemA || kind == kItemB;
         const long long Fw = split ? F - cost : F;
         const long long Fe = Fw + len + cost;
-        const long long ca = (Fw * N + T - 1) / T, cb = (Fe * N + T - 1) / T;
+        const long long ca = ceil_div(Fw * N, T, rT), cb = ceil_div(Fe * N, T, rT);
         for (long long c = ca; c < cb && c < N; ++c) p.first_seg[c] = s;
       }
     }
