@@ -382,11 +382,19 @@ __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32
       L += rl * a;
       O += ro * rl * a;
     }
-#pragma unroll 8
-    for (int i = 0; i < nA; ++i) {
-      const float a = ex2(pm(i, h) - Mu);
-      L += pl_(i, h) * a;
-      O += __ldcg(p.part + (size_t)(sA.pbase + i) * PF + idx) * a;
+    for (int i0 = 0; i0 < nA; i0 += 16) {  // 16 partial outputs in flight at a time
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        v[k] = i0 + k < nA ? __ldcg(p.part + (size_t)(sA.pbase + i0 + k) * PF + idx) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (i0 + k < nA) {
+          const float a = ex2(pm(i0 + k, h) - Mu);
+          L += pl_(i0 + k, h) * a;
+          O += v[k] * a;
+        }
+      }
     }
     const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
     p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
@@ -400,11 +408,19 @@ __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32
     const float M2u = M2 == -INFINITY ? 0.f : M2;
     const float a0 = ex2(M - M2u);
     float L2 = L * a0, O2 = O * a0;
-#pragma unroll 8
-    for (int i = nA; i < n; ++i) {
-      const float a = ex2(pm(i, h) - M2u);
-      L2 += pl_(i, h) * a;
-      O2 += __ldcg(p.part + (size_t)(sB.pbase + (i - nA)) * PF + idx) * a;
+    for (int i0 = nA; i0 < n; i0 += 16) {
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        v[k] = i0 + k < n ? __ldcg(p.part + (size_t)(sB.pbase + (i0 + k - nA)) * PF + idx) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (i0 + k < n) {
+          const float a = ex2(pm(i0 + k, h) - M2u);
+          L2 += pl_(i0 + k, h) * a;
+          O2 += v[k] * a;
+        }
+      }
     }
     const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
     p.out[orow * D + d] = O2 / L2;
@@ -508,9 +524,11 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
       dst[GD + G + h] = L;
     }
   }
-  __threadfence();
+  // every thread's partial stores happen-before thread 0's fence through the
+  // barrier; the fence publishes them device-wide before the count
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (threadIdx.x == 0) {
+    __threadfence();
     const int old = atomicAdd(p.unit_cnt + unit, 1);
     sm.last_flag = (old == p.plan[unit].expected - 1);
   }
