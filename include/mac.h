@@ -151,7 +151,12 @@ int mac_append_kv(MacState *st, uint16_t *K, uint16_t *V, const int *block_table
  * copies out_h, lse_h, hit_h and match_pos_h back (any of the four may be
  * NULL) and synchronises the stream before returning.  K, V, block_table
  * stay device-resident (the cache is state, not a per-step input).  Returns
- * MAC_ERR_DEVICE if the device status word is non-zero after the step. */
+ * MAC_ERR_DEVICE if the device status word is non-zero after the step.
+ * The inputs go through one pinned host block and one copy each way; the
+ * copy-in, append, step and copy-out are recorded once as a CUDA graph per
+ * (K, V, block_table, append or not) and replayed on `stream` by later calls
+ * (the work-split setters drop the recording).  Not thread-safe on one
+ * state; do not call it while `stream` is being captured. */
 int mac_decode_step_host(MacState *st, const float *q_pre_h, const int *rope_pos_h,
                          const int *seq_lens_h, const uint16_t *k_new_h, const uint16_t *v_new_h,
                          uint16_t *K, uint16_t *V, const int *block_table, float *out_h,

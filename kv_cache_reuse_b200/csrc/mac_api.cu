@@ -38,16 +38,23 @@ struct MacState {
   int* done = nullptr;
   unsigned* status = nullptr;
   double* inv_freq = nullptr;
-  // staging for mac_decode_step_host
-  float* st_q = nullptr;
-  int* st_pos = nullptr;
-  int* st_lens = nullptr;
-  uint16_t* st_knew = nullptr;
-  uint16_t* st_vnew = nullptr;
-  float* st_out = nullptr;
-  float* st_lse = nullptr;
-  uint8_t* st_hit = nullptr;
-  int* st_mpos = nullptr;
+  // staging of mac_decode_step_host: one packed block each way, on the
+  // device and in pinned host memory; the state's status word is the last
+  // field of the output block, so one copy brings everything back
+  unsigned char* dev_in = nullptr;    // q | pos | lens | k_new | v_new
+  unsigned char* dev_out = nullptr;   // out | lse | hit | match_pos | status
+  unsigned char* host_in = nullptr;
+  unsigned char* host_out = nullptr;
+  size_t off_q = 0, off_pos = 0, off_lens = 0, off_knew = 0, off_vnew = 0, in_bytes = 0, in_bytes_noappend = 0;
+  size_t off_out = 0, off_lse = 0, off_hit = 0, off_mpos = 0, off_status = 0, out_bytes = 0;
+  // the host step as a CUDA graph (copy in, append, match, attend, copy out),
+  // captured for one set of cache pointers
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t gexec = nullptr;
+  const void* g_k = nullptr;
+  const void* g_v = nullptr;
+  const void* g_bt = nullptr;
+  int g_append = -1;
   // TMA descriptors of the last K/V pointers seen
   const void* tm_k_ptr = nullptr;
   const void* tm_v_ptr = nullptr;
@@ -79,14 +86,25 @@ cudaError_t alloc(T** p, size_t count) {
   return cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T) + 16);
 }
 
+void drop_graph(MacState* s) {
+  if (s->gexec) cudaGraphExecDestroy(s->gexec);
+  s->gexec = nullptr;
+  s->g_append = -1;
+}
+
 void free_all(MacState* s) {
-  void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot, s->plan,
-                  s->seg,    s->hdr, s->first_seg,    s->part,   s->unit_cnt, s->done,   s->status, s->inv_freq,
-                  s->st_q,   s->st_pos, s->st_lens, s->st_knew, s->st_vnew, s->st_out, s->st_lse, s->st_hit,
-                  s->st_mpos};
+  drop_graph(s);
+  void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,
+                  s->seg,    s->hdr,    s->first_seg, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
+                  s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  if (s->host_in) cudaFreeHost(s->host_in);
+  if (s->host_out) cudaFreeHost(s->host_out);
+  if (s->cap_stream) cudaStreamDestroy(s->cap_stream);
 }
+
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int check_config(const MacConfig* c) {
   if (!c) return MAC_ERR_ARG;
@@ -226,17 +244,26 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
   A(alloc(&s->unit_cnt, U));
   A(alloc(&s->done, 1));
-  A(alloc(&s->status, 1));
   A(alloc(&s->inv_freq, D / 2));
-  A(alloc(&s->st_q, B * Hq * D));
-  A(alloc(&s->st_pos, B));
-  A(alloc(&s->st_lens, B));
-  A(alloc(&s->st_knew, B * Hkv * D));
-  A(alloc(&s->st_vnew, B * Hkv * D));
-  A(alloc(&s->st_out, B * Hq * D));
-  A(alloc(&s->st_lse, B * Hq));
-  A(alloc(&s->st_hit, U));
-  A(alloc(&s->st_mpos, U));
+  s->off_q = 0;
+  s->off_pos = up256(s->off_q + B * Hq * D * sizeof(float));
+  s->off_lens = up256(s->off_pos + B * sizeof(int));
+  s->off_knew = up256(s->off_lens + B * sizeof(int));
+  s->in_bytes_noappend = s->off_knew;
+  s->off_vnew = up256(s->off_knew + B * Hkv * D * 2);
+  s->in_bytes = up256(s->off_vnew + B * Hkv * D * 2);
+  s->off_out = 0;
+  s->off_lse = up256(B * Hq * D * sizeof(float));
+  s->off_hit = up256(s->off_lse + B * Hq * sizeof(float));
+  s->off_mpos = up256(s->off_hit + U);
+  s->off_status = up256(s->off_mpos + U * sizeof(int));
+  s->out_bytes = s->off_status + 16;
+  A(alloc(&s->dev_in, s->in_bytes));
+  A(alloc(&s->dev_out, s->out_bytes));
+  A(cudaMallocHost(reinterpret_cast<void**>(&s->host_in), s->in_bytes));
+  A(cudaMallocHost(reinterpret_cast<void**>(&s->host_out), s->out_bytes));
+  A(cudaStreamCreateWithFlags(&s->cap_stream, cudaStreamNonBlocking));
+  if (e == cudaSuccess) s->status = reinterpret_cast<unsigned*>(s->dev_out + s->off_status);
   if (e != cudaSuccess) {
     free_all(s);
     delete s;
@@ -250,7 +277,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->steps, 0, U * sizeof(int)));
   A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
   A(cudaMemset(s->done, 0, sizeof(int)));
-  A(cudaMemset(s->status, 0, sizeof(unsigned)));
+  A(cudaMemset(s->dev_out, 0, s->out_bytes));
   A(cudaMemset(s->hdr, 0, sizeof(PlanHeader)));
   double* inv = (double*)malloc(sizeof(double) * (D / 2));
   for (size_t i = 0; i < D / 2; ++i) inv[i] = pow(cfg->rope_theta, -2.0 * (double)i / (double)D);
@@ -284,18 +311,21 @@ int mac_reset_seq(MacState* s, int b, void* stream) {
 int mac_set_min_keys_per_cta(MacState* s, int keys) {
   if (!s || keys < 1) return MAC_ERR_ARG;
   s->min_keys = keys;
+  drop_graph(s);
   return MAC_OK;
 }
 
 int mac_set_piece_cost(MacState* s, int keys) {
   if (!s || keys < 0) return MAC_ERR_ARG;
   s->piece_cost = keys;
+  drop_graph(s);
   return MAC_OK;
 }
 
 int mac_set_whole_unit_keys(MacState* s, int keys) {
   if (!s || keys < 0) return MAC_ERR_ARG;
   s->unit_max = keys;
+  drop_graph(s);
   return MAC_OK;
 }
 
@@ -418,42 +448,83 @@ int mac_append_kv(MacState* s, uint16_t* K, uint16_t* V, const int* block_table,
   return launch_append(p, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
+// Enqueue one host step on `st`: copy the packed inputs in, append the new
+// rows (optional), run the step, copy the packed outputs (and status) out.
+static int enqueue_host_step(MacState* s, uint16_t* K, uint16_t* V, const int* block_table, bool append,
+                             cudaStream_t st) {
+  unsigned char* di = s->dev_in;
+  unsigned char* dout = s->dev_out;
+  if (cudaMemcpyAsync(di, s->host_in, append ? s->in_bytes : s->in_bytes_noappend, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess)
+    return MAC_ERR_CUDA;
+  const int* lens = reinterpret_cast<const int*>(di + s->off_lens);
+  int rc;
+  if (append) {
+    rc = mac_append_kv(s, K, V, block_table, lens, reinterpret_cast<const uint16_t*>(di + s->off_knew),
+                       reinterpret_cast<const uint16_t*>(di + s->off_vnew), st);
+    if (rc != MAC_OK) return rc;
+  }
+  rc = mac_decode_step(s, reinterpret_cast<const float*>(di + s->off_q), reinterpret_cast<const int*>(di + s->off_pos),
+                       K, V, block_table, lens, reinterpret_cast<float*>(dout + s->off_out),
+                       reinterpret_cast<float*>(dout + s->off_lse), dout + s->off_hit,
+                       reinterpret_cast<int*>(dout + s->off_mpos), st);
+  if (rc != MAC_OK) return rc;
+  return cudaMemcpyAsync(s->host_out, dout, s->out_bytes, cudaMemcpyDeviceToHost, st) == cudaSuccess ? MAC_OK
+                                                                                                      : MAC_ERR_CUDA;
+}
+
 int mac_decode_step_host(MacState* s, const float* q_pre_h, const int* rope_pos_h, const int* seq_lens_h,
                          const uint16_t* k_new_h, const uint16_t* v_new_h, uint16_t* K, uint16_t* V,
                          const int* block_table, float* out_h, float* lse_h, uint8_t* hit_h, int* match_pos_h,
                          void* stream) {
   if (!s || !q_pre_h || !rope_pos_h || !seq_lens_h || !K || !V) return MAC_ERR_ARG;
   if ((k_new_h == nullptr) != (v_new_h == nullptr)) return MAC_ERR_ARG;
+  if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
+  if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   const size_t B = s->cfg.batch, Hq = s->cfg.num_q_heads, Hkv = s->cfg.num_kv_heads, D = s->D, U = s->U;
-  cudaError_t e = cudaSuccess;
-  auto A = [&](cudaError_t r) {
-    if (e == cudaSuccess) e = r;
-  };
-  A(cudaMemcpyAsync(s->st_q, q_pre_h, B * Hq * D * sizeof(float), cudaMemcpyHostToDevice, st));
-  A(cudaMemcpyAsync(s->st_pos, rope_pos_h, B * sizeof(int), cudaMemcpyHostToDevice, st));
-  A(cudaMemcpyAsync(s->st_lens, seq_lens_h, B * sizeof(int), cudaMemcpyHostToDevice, st));
-  if (k_new_h) {
-    A(cudaMemcpyAsync(s->st_knew, k_new_h, B * Hkv * D * 2, cudaMemcpyHostToDevice, st));
-    A(cudaMemcpyAsync(s->st_vnew, v_new_h, B * Hkv * D * 2, cudaMemcpyHostToDevice, st));
+  const bool append = k_new_h != nullptr;
+  // inputs into the pinned block (the graph copies the whole block in)
+  memcpy(s->host_in + s->off_q, q_pre_h, B * Hq * D * sizeof(float));
+  memcpy(s->host_in + s->off_pos, rope_pos_h, B * sizeof(int));
+  memcpy(s->host_in + s->off_lens, seq_lens_h, B * sizeof(int));
+  if (append) {
+    memcpy(s->host_in + s->off_knew, k_new_h, B * Hkv * D * 2);
+    memcpy(s->host_in + s->off_vnew, v_new_h, B * Hkv * D * 2);
   }
-  if (e != cudaSuccess) return MAC_ERR_CUDA;
-  int rc;
-  if (k_new_h) {
-    rc = mac_append_kv(s, K, V, block_table, s->st_lens, s->st_knew, s->st_vnew, stream);
+  const int* bt = s->cfg.page_size > 0 ? block_table : nullptr;
+  if (!s->gexec || s->g_k != K || s->g_v != V || s->g_bt != bt || s->g_append != (int)append) {
+    // (re)capture the step for these cache pointers
+    drop_graph(s);
+    cudaGraph_t graph = nullptr;
+    bool ok = cudaStreamBeginCapture(s->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    const int rc = ok ? enqueue_host_step(s, K, V, bt, append, s->cap_stream) : MAC_ERR_CUDA;
+    if (ok) ok = cudaStreamEndCapture(s->cap_stream, &graph) == cudaSuccess && rc == MAC_OK;
+    if (ok) ok = cudaGraphInstantiate(&s->gexec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+    if (!ok) {
+      drop_graph(s);
+      cudaGetLastError();
+    } else {
+      s->g_k = K;
+      s->g_v = V;
+      s->g_bt = bt;
+      s->g_append = (int)append;
+    }
+  }
+  if (s->gexec) {
+    if (cudaGraphLaunch(s->gexec, st) != cudaSuccess) return MAC_ERR_CUDA;
+  } else {
+    const int rc = enqueue_host_step(s, K, V, bt, append, st);  // no graph: the same work, launched directly
     if (rc != MAC_OK) return rc;
   }
-  rc = mac_decode_step(s, s->st_q, s->st_pos, K, V, block_table, s->st_lens, s->st_out, s->st_lse, s->st_hit,
-                       s->st_mpos, stream);
-  if (rc != MAC_OK) return rc;
-  if (out_h) A(cudaMemcpyAsync(out_h, s->st_out, B * Hq * D * sizeof(float), cudaMemcpyDeviceToHost, st));
-  if (lse_h) A(cudaMemcpyAsync(lse_h, s->st_lse, B * Hq * sizeof(float), cudaMemcpyDeviceToHost, st));
-  if (hit_h) A(cudaMemcpyAsync(hit_h, s->st_hit, U, cudaMemcpyDeviceToHost, st));
-  if (match_pos_h) A(cudaMemcpyAsync(match_pos_h, s->st_mpos, U * sizeof(int), cudaMemcpyDeviceToHost, st));
-  unsigned status = 0;
-  A(cudaMemcpyAsync(&status, s->status, sizeof(unsigned), cudaMemcpyDeviceToHost, st));
-  A(cudaStreamSynchronize(st));
-  if (e != cudaSuccess) return MAC_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MAC_ERR_CUDA;
+  if (out_h) memcpy(out_h, s->host_out + s->off_out, B * Hq * D * sizeof(float));
+  if (lse_h) memcpy(lse_h, s->host_out + s->off_lse, B * Hq * sizeof(float));
+  if (hit_h) memcpy(hit_h, s->host_out + s->off_hit, U);
+  if (match_pos_h) memcpy(match_pos_h, s->host_out + s->off_mpos, U * sizeof(int));
+  unsigned status;
+  memcpy(&status, s->host_out + s->off_status, sizeof status);
   return status ? MAC_ERR_DEVICE : MAC_OK;
 }
 

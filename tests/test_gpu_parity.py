@@ -190,6 +190,56 @@ def test_host_entry_matches_device_entry():
             np.testing.assert_array_equal(u, v)
 
 
+def test_host_entry_append_recapture():
+    """Host entry with appends on a paged pool, a swap of the cache buffers and a
+    work-split change mid-stream (each forces a new recording), against the device
+    entry on the same inputs, bit for bit."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["continuous_16k"].with_(L0=(3000, 1777, 4100, 2601), B=4)
+    steps = 30
+    stream = synth.queries(wl, steps)
+    cache = synth.kv_cache(wl, steps)
+    torch, dev = torch_dev()
+    pool = [torch.from_numpy(x.view(np.int16)).to(dev) for x in (cache.K, cache.V)]
+    a = GpuRun(wl, cache, K_dev=pool[0].clone(), V_dev=pool[1].clone())
+    b = GpuRun(wl, cache, K_dev=pool[0].clone(), V_dev=pool[1].clone())
+    Kb2, Vb2 = b.K.clone(), b.V.clone()
+    knew = torch.empty((wl.B, wl.Hkv, wl.D), dtype=torch.int16, device=dev)
+    vnew = torch.empty_like(knew)
+    out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32)
+    lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32)
+    hit_h = torch.empty((wl.B, wl.Hkv), dtype=torch.uint8)
+    mp_h = torch.empty((wl.B, wl.Hkv), dtype=torch.int32)
+    Kb, Vb = b.K, b.V
+    hits = 0
+    for t in range(steps):
+        kr, vr = synth.step_rows(cache, stream.seq_lens[t])
+        knew.copy_(torch.from_numpy(kr.view(np.int16)))
+        vnew.copy_(torch.from_numpy(vr.view(np.int16)))
+        a.lens.copy_(torch.from_numpy(stream.seq_lens[t]))
+        mac.mac_append_kv(a.st, a.K, a.V, a.bt, a.lens, knew, vnew)
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        if t == 10:  # move the cache to other buffers: the recording must follow
+            Kb2.copy_(Kb)
+            Vb2.copy_(Vb)
+            torch.cuda.synchronize()
+            Kb, Vb = Kb2, Vb2
+        if t == 20:  # a work-split change drops the recording
+            mac.mac_set_piece_cost(b.st, 512)
+            mac.mac_set_piece_cost(a.st, 512)
+        kh = torch.from_numpy(kr.view(np.int16).copy())
+        vh = torch.from_numpy(vr.view(np.int16).copy())
+        rc = mac.mac_decode_step_host(b.st, torch.from_numpy(stream.q[t]), torch.from_numpy(stream.rope_pos[t]),
+                                      torch.from_numpy(stream.seq_lens[t]), kh, vh, Kb, Vb, b.bt, out_h, lse_h,
+                                      hit_h, mp_h)
+        assert rc == mac.MAC_OK
+        for u, v in zip(x, (out_h.numpy(), lse_h.numpy(), hit_h.numpy(), mp_h.numpy())):
+            np.testing.assert_array_equal(u, v, err_msg="step %d" % t)
+        hits += int(x[2].sum())
+    assert hits > 0 and hits < steps * wl.B * wl.Hkv
+    assert a.st.get_status() == 0 and b.st.get_status() == 0
+
+
 @pytest.mark.parametrize("case", ["one_key", "band0", "window1", "ragged", "full_capacity", "band_covers", "d128_short"])
 def test_edge_cases(case):
     base = synth.WORKLOADS["tiny"]
