@@ -194,17 +194,6 @@ int mac_set_piece_cost(MacState *st, int keys);
  * range. */
 int mac_set_whole_unit_keys(MacState *st, int keys);
 
-/* Tuning: run-time balancing of the cut ranges.  The last `permille`/1000
- * of the keys of every cut range (default 250) are not assigned up front:
- * they form a pool of equal chunks (at least `chunk_keys` keys, a multiple
- * of 16; default 256; larger when the pools would exceed 8 chunks per CTA)
- * that CTAs take at run time once their assigned keys are done, so that CTAs
- * whose streaming multiprocessor draws less memory bandwidth take fewer
- * keys.  Results are the same up to the fp32 rounding of the merge order.
- * 0 turns the pools off.  Returns MAC_ERR_ARG for permille outside [0, 1000]
- * or chunk_keys < 16 or not a multiple of 16. */
-int mac_set_pool_share(MacState *st, int permille, int chunk_keys);
-
 /* Persistent grid size of the attention kernel (CTAs). */
 int mac_attend_grid(const MacState *st);
 

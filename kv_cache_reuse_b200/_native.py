@@ -28,7 +28,6 @@ SIGNATURES = {
     "mac_set_min_keys_per_cta": (C.c_int, [_P, C.c_int]),
     "mac_set_piece_cost": (C.c_int, [_P, C.c_int]),
     "mac_set_whole_unit_keys": (C.c_int, [_P, C.c_int]),
-    "mac_set_pool_share": (C.c_int, [_P, C.c_int, C.c_int]),
     "mac_attend_grid": (C.c_int, [_P]),
     "mac_error_string": (C.c_char_p, [C.c_int]),
     "mac_dense_decode_static": (C.c_int, [_P] * 9 + [C.c_int] * 4 + [C.c_double] + [C.c_int] * 4 + [_P]),

@@ -18,7 +18,7 @@ using namespace mac;
 
 struct MacState {
   MacConfig cfg;
-  int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, unit_max, pool_permille, pool_chunk, capacity;
+  int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, unit_max, capacity;
   size_t max_parts;
   // ring (library-owned state)
   float* ring_q = nullptr;
@@ -33,8 +33,6 @@ struct MacState {
   Segment* seg = nullptr;
   PlanHeader* hdr = nullptr;
   int* first_seg = nullptr;
-  PoolInfo* pool = nullptr;
-  int* pool_next = nullptr;  // pool_next [2U] then pool_slots [2U]
   float* part = nullptr;
   int* unit_cnt = nullptr;
   int* done = nullptr;
@@ -97,7 +95,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,
-                  s->seg,    s->hdr,    s->first_seg, s->pool, s->pool_next, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -218,8 +216,6 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   s->min_keys = 128;
   s->piece_cost = 1024;
   s->unit_max = 1024;
-  s->pool_permille = 250;
-  s->pool_chunk = kPoolChunkMin;
   s->capacity = cfg->page_size == 0 ? cfg->max_seq : cfg->max_pages_per_seq * cfg->page_size;
   if (cudaGetDevice(&s->device) != cudaSuccess ||
       cudaDeviceGetAttribute(&s->num_sms, cudaDevAttrMultiProcessorCount, s->device) != cudaSuccess) {
@@ -227,8 +223,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
     return MAC_ERR_CUDA;
   }
   s->grid = s->num_sms;  // one resident CTA per SM (shared-memory bound)
-  // static pieces (<= grid + 2U) and dynamic runs (<= the pool chunks, <= kPoolChunksPerCta x grid)
-  s->max_parts = (size_t)(1 + kPoolChunksPerCta) * s->grid + 2 * (size_t)s->U;
+  s->max_parts = (size_t)s->grid + 2 * (size_t)s->U;
   const size_t U = s->U, W1 = s->W + 1, G = s->G, D = s->D, B = cfg->batch, Hq = cfg->num_q_heads;
   const size_t Hkv = cfg->num_kv_heads;
   cudaError_t e = cudaSuccess;
@@ -246,8 +241,6 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->seg, 2 * U));
   A(alloc(&s->hdr, 1));
   A(alloc(&s->first_seg, (size_t)s->grid));
-  A(alloc(&s->pool, 2 * U));
-  A(alloc(&s->pool_next, 4 * U));
   A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
   A(alloc(&s->unit_cnt, U));
   A(alloc(&s->done, 1));
@@ -284,7 +277,6 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->steps, 0, U * sizeof(int)));
   A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
   A(cudaMemset(s->done, 0, sizeof(int)));
-  A(cudaMemset(s->pool_next, 0, 4 * U * sizeof(int)));
   A(cudaMemset(s->dev_out, 0, s->out_bytes));
   A(cudaMemset(s->hdr, 0, sizeof(PlanHeader)));
   double* inv = (double*)malloc(sizeof(double) * (D / 2));
@@ -337,14 +329,6 @@ int mac_set_whole_unit_keys(MacState* s, int keys) {
   return MAC_OK;
 }
 
-int mac_set_pool_share(MacState* s, int permille, int chunk_keys) {
-  if (!s || permille < 0 || permille > 1000 || chunk_keys < kSubKeys || chunk_keys % kSubKeys != 0) return MAC_ERR_ARG;
-  s->pool_permille = permille;
-  s->pool_chunk = chunk_keys;
-  drop_graph(s);
-  return MAC_OK;
-}
-
 int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
 
 int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
@@ -370,9 +354,6 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
-  p.pool = s->pool;
-  p.pool_next = s->pool_next;
-  p.pool_slots = s->pool_next + 2 * s->U;
   p.done = s->done;
   p.status = s->status;
   p.B = s->cfg.batch;
@@ -389,8 +370,6 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.min_keys = s->min_keys;
   p.piece_cost = s->piece_cost;
   p.unit_max = s->unit_max;
-  p.pool_permille = s->pool_permille;
-  p.pool_chunk = s->pool_chunk;
   return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
@@ -418,9 +397,6 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
-  p.pool = s->pool;
-  p.pool_next = s->pool_next;
-  p.pool_slots = s->pool_next + 2 * s->U;
   p.part = s->part;
   p.unit_cnt = s->unit_cnt;
   p.ring_o = s->ring_o;

@@ -72,12 +72,6 @@ struct Cfg {
   static constexpr int WB = (PF > 128 ? PF : 128);     // per-warp scratch floats
 };
 
-// A pool chunk taken at run time: keys [k0, k1) of item seg (seg < 0: none left).
-struct DynEntry {
-  int seg, k0, k1, sbase;
-};
-constexpr int kDynCap = 64;  // pool chunks one CTA may take
-
 template <int D>
 struct __align__(1024) AttnSmem {
   // per warp: ring of (K box, V box), each [HALVES][16 keys][64 dims] bf16, 128-byte swizzle
@@ -92,11 +86,6 @@ struct __align__(1024) AttnSmem {
   int last_flag;
   Segment items[kItemCache];         // the CTA's work items, from its first one on
   alignas(16) float ring[Cfg<D>::GD + 2 * kGroup];  // that ring state: o [G][D], m [G], l [G]
-  DynEntry dq[kDynCap];              // pool chunks taken by this CTA, in order
-  int dq_state[kDynCap];             // 0 free, 1 being taken, 2 ready
-  PoolInfo cur_info;                 // the pool the CTA takes chunks from
-  int cur_pool;
-  int slot_bcast;                    // partial slot of the run being finalized
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -339,124 +328,103 @@ __device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, 
   return ok;
 }
 
-// VEC consecutive floats of a partial or of the ring through L2 (they were
-// written by other CTAs of this launch or of an earlier one).
-template <int VEC>
-__device__ __forceinline__ void ld_vec(float (&v)[VEC], const float* src) {
-  if constexpr (VEC == 2) {
-    const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
-    v[0] = t.x;
-    v[1] = t.y;
-  } else {
-    v[0] = __ldcg(src);
-  }
-}
-
-// Last arriver of a split unit: merge its partials.  Segment A's partials
-// (with the reused state on a hit) give the new prefix state over [0, c_t),
-// stored in the ring; that state and segment B's partials give the output.
-// Each thread owns VEC consecutive output elements of one head; (m, l) of
-// every partial are staged in shared memory and the partial outputs are
-// fetched NB at a time, so the merge costs one round of loads per NB pieces.
+// Merge of unit u by the CTA holding its last partial (256 threads).  Phase
+// 1 stages every partial's (m, l) in shared memory with one round of
+// independent loads; phase 2 weighs the partial outputs, all loads in flight.
 template <int D>
 __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
-  constexpr int VEC = GD / (kConsumerWarps * 32);
-  static_assert(VEC * kConsumerWarps * 32 == GD && (VEC == 1 || VEC == 2), "merge layout");
-  constexpr int NB = 32 / VEC;  // partial outputs in flight per thread
   constexpr int kCap = (kConsumerWarps * Cfg<D>::WB) / (2 * G);  // pieces whose (m, l) fit in wbuf
   const UnitPlan pl = p.plan[u];
   const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
-  // static pieces, then one slot per dynamic run (final: every partial is counted)
-  const int nA = sA.npieces + __ldcg(p.pool_slots + 2 * u);
-  const int n = nA + sB.npieces + __ldcg(p.pool_slots + 2 * u + 1);
-  auto slot = [&](int i) { return i < nA ? sA.pbase + i : sB.pbase + (i - nA); };
+  const int nA = sA.npieces, n = sA.npieces + sB.npieces;
   float* mm = &sm.wbuf[0][0];  // [piece][G] maxima, then [piece][G] sums
   float* ll = mm + kCap * G;
   const bool staged = n <= kCap;
-  const int idx0 = threadIdx.x * VEC, h = idx0 / D, d0 = idx0 - h * D;
-
-  // one round of loads: the first NB partial outputs, the reused state, (m, l)
-  float v[NB][VEC];
-#pragma unroll
-  for (int k = 0; k < NB; ++k)
-    if (k < n) ld_vec<VEC>(v[k], p.part + (size_t)slot(k) * PF + idx0);
-  float ro[VEC], rm = -INFINITY, rl = 0.f;
-  if (pl.hit) {
-    const size_t rs = (size_t)u * Wp1 + pl.src_slot;
-    ld_vec<VEC>(ro, p.ring_o + rs * GD + idx0);
-    rl = __ldcg(p.ring_l + rs * G + h);
-    rm = __ldcg(p.ring_m + rs * G + h) * kLog2e;
-  }
   if (staged) {
     for (int t = threadIdx.x; t < n * G; t += kConsumerWarps * 32) {
-      const int i = t / G, hh = t - i * G;
-      const float* pp = p.part + (size_t)slot(i) * PF;
-      mm[t] = __ldcg(pp + GD + hh);
-      ll[t] = __ldcg(pp + GD + G + hh);
+      const int i = t / G, h = t - i * G;
+      const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
+      const float* pp = p.part + (size_t)slot * PF;
+      mm[t] = __ldcg(pp + GD + h);
+      ll[t] = __ldcg(pp + GD + G + h);
     }
   }
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  auto pm = [&](int i) -> float {
-    return staged ? mm[i * G + h] : __ldcg(p.part + (size_t)slot(i) * PF + GD + h);
+  auto pm = [&](int i, int h) -> float {
+    if (staged) return mm[i * G + h];
+    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
+    return __ldcg(p.part + (size_t)slot * PF + GD + h);
   };
-  auto pl_ = [&](int i) -> float {
-    return staged ? ll[i * G + h] : __ldcg(p.part + (size_t)slot(i) * PF + GD + G + h);
+  auto pl_ = [&](int i, int h) -> float {
+    if (staged) return ll[i * G + h];
+    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
+    return __ldcg(p.part + (size_t)slot * PF + GD + G + h);
   };
-  // maxima: M over the prefix (reused state + A), M2 over everything
-  float M = rm;
-  for (int i = 0; i < nA; ++i) M = fmaxf(M, pm(i));
-  float M2 = M;
-  for (int i = nA; i < n; ++i) M2 = fmaxf(M2, pm(i));
-  const float Mu = M == -INFINITY ? 0.f : M, M2u = M2 == -INFINITY ? 0.f : M2;
-  // sums: A relative to 2^M, B relative to 2^M2
-  float L = 0.f, LB = 0.f, O[VEC], OB[VEC];
-#pragma unroll
-  for (int j = 0; j < VEC; ++j) O[j] = OB[j] = 0.f;
-  if (pl.hit) {
-    const float a = ex2(rm - Mu);
-    L += rl * a;
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) O[j] += ro[j] * rl * a;
-  }
-  for (int i0 = 0; i0 < n; i0 += NB) {
-    if (i0 > 0) {
-#pragma unroll
-      for (int k = 0; k < NB; ++k)
-        if (i0 + k < n) ld_vec<VEC>(v[k], p.part + (size_t)slot(i0 + k) * PF + idx0);
+  for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
+    const int h = idx / D, d = idx - h * D;
+    // new prefix state over [0, c_t): reused state (hit) + amend partials
+    float M = -INFINITY, rm = -INFINITY, rl = 0.f, ro = 0.f;
+    if (pl.hit) {
+      const size_t rs = (size_t)u * Wp1 + pl.src_slot;
+      rl = p.ring_l[rs * G + h];
+      rm = p.ring_m[rs * G + h] * kLog2e;
+      ro = p.ring_o[rs * GD + idx];
+      M = rm;
     }
+    for (int i = 0; i < nA; ++i) M = fmaxf(M, pm(i, h));
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f, O = 0.f;
+    if (pl.hit) {
+      const float a = ex2(rm - Mu);
+      L += rl * a;
+      O += ro * rl * a;
+    }
+    for (int i0 = 0; i0 < nA; i0 += 16) {  // 16 partial outputs in flight at a time
+      float v[16];
 #pragma unroll
-    for (int k = 0; k < NB; ++k) {
-      const int i = i0 + k;
-      if (i < n) {
-        const bool inA = i < nA;
-        const float a = ex2(pm(i) - (inA ? Mu : M2u)), w = pl_(i) * a;
-        if (inA) {
-          L += w;
+      for (int k = 0; k < 16; ++k)
+        v[k] = i0 + k < nA ? __ldcg(p.part + (size_t)(sA.pbase + i0 + k) * PF + idx) : 0.f;
 #pragma unroll
-          for (int j = 0; j < VEC; ++j) O[j] += v[k][j] * a;
-        } else {
-          LB += w;
-#pragma unroll
-          for (int j = 0; j < VEC; ++j) OB[j] += v[k][j] * a;
+      for (int k = 0; k < 16; ++k) {
+        if (i0 + k < nA) {
+          const float a = ex2(pm(i0 + k, h) - Mu);
+          L += pl_(i0 + k, h) * a;
+          O += v[k] * a;
         }
       }
     }
-  }
-  const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
-  const float a0 = ex2(M - M2u), L2 = L * a0 + LB;
-  const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
+    p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
+    if (d == 0) {
+      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
+      p.ring_l[ds * G + h] = L;
+    }
+    // output: new prefix state + tail partials
+    float M2 = M;
+    for (int i = nA; i < n; ++i) M2 = fmaxf(M2, pm(i, h));
+    const float M2u = M2 == -INFINITY ? 0.f : M2;
+    const float a0 = ex2(M - M2u);
+    float L2 = L * a0, O2 = O * a0;
+    for (int i0 = nA; i0 < n; i0 += 16) {
+      float v[16];
 #pragma unroll
-  for (int j = 0; j < VEC; ++j) {
-    p.ring_o[ds * GD + idx0 + j] = L > 0.f ? O[j] / L : 0.f;
-    p.out[orow * D + d0 + j] = (O[j] * a0 + OB[j]) / L2;
-  }
-  if (d0 == 0) {
-    p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
-    p.ring_l[ds * G + h] = L;
-    p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+      for (int k = 0; k < 16; ++k)
+        v[k] = i0 + k < n ? __ldcg(p.part + (size_t)(sB.pbase + (i0 + k - nA)) * PF + idx) : 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        if (i0 + k < n) {
+          const float a = ex2(pm(i0 + k, h) - M2u);
+          L2 += pl_(i0 + k, h) * a;
+          O2 += v[k] * a;
+        }
+      }
+    }
+    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    p.out[orow * D + d] = O2 / L2;
+    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
   }
   if (threadIdx.x == 0) {
     p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
@@ -537,18 +505,15 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, in
   }
 }
 
-// End of a run (a static piece of a split item and/or pool chunks of the
-// same item, accumulated together): combine the 8 warps, write the partial
-// to `slot`, count the `cnt` pieces and chunks it covers and, if that
-// completes the unit, merge it.
+// End of a split piece: combine the 8 warps, write the partial, count it
+// and, if it was the unit's last, merge the unit.
 template <int D>
-__device__ bool finalize_run(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int unit, int slot, int cnt,
-                             uint32_t& sync_phase) {
+__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int unit, int pidx,
+                               uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
   warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
-  if (threadIdx.x == 0) sm.slot_bcast = slot;
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  float* dst = p.part + (size_t)sm.slot_bcast * PF;
+  float* dst = p.part + (size_t)pidx * PF;
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
     const int h = idx / D;
     float MA, LA, OA, M, L, O;
@@ -564,8 +529,8 @@ __device__ bool finalize_run(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, 
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (threadIdx.x == 0) {
     __threadfence();
-    const int old = atomicAdd(p.unit_cnt + unit, cnt);
-    sm.last_flag = (old + cnt == p.plan[unit].expected);
+    const int old = atomicAdd(p.unit_cnt + unit, 1);
+    sm.last_flag = (old == p.plan[unit].expected - 1);
   }
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
@@ -631,8 +596,7 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
 // piece is part of one segment of a large unit; a whole-unit piece holds
 // both segments of a small unit: A = [a0, a1) (may be empty), B = [k0, k1).
 struct Piece {
-  int unit, seg, pidx, whole, dyn;  // dyn: a pool chunk (pidx unused; partial slots from sbase)
-  int sbase;
+  int unit, pidx, whole;
   int hit, src, dst;          // whole unit: plan of the unit (end = k1)
   int k0, k1, kb0, nbox;      // split: its keys; whole unit: segment B
   int a0, a1, akb0, anbox;    // whole unit: segment A
@@ -681,8 +645,6 @@ struct Walker {
         return false;
       }
       pc.unit = cur >> 1;
-      pc.seg = cur;
-      pc.dyn = 0;
       if (sg.kind == kItemWhole) {
         if (sg.first_cta != cta) continue;  // owned by the CTA whose range holds its start
         const int start = sg.key0, cut = sg.pbase, end = sg.key0 + sg.len;
@@ -725,143 +687,6 @@ struct Walker {
   }
 };
 
-// Entry k of the CTA's queue of pool chunks, called by all lanes of a warp.
-// The first warp to ask takes the chunk: from the pool it is on (for k = 0:
-// the item of the CTA's last static piece), else from the pool with the most
-// chunks left; every other warp waits (bounded) for that entry.  Entries are
-// asked for in order by every cursor, so they are taken one at a time.
-template <int D>
-__device__ bool dyn_get(const AttendParams& p, AttnSmem<D>& sm, int k, int last_seg, int chunk, DynEntry& e) {
-  const int lane = threadIdx.x & 31;
-  int claim = 0;
-  if (lane == 0) claim = atomicCAS(&sm.dq_state[k], 0, 1) == 0;
-  claim = __shfl_sync(kFull, claim, 0);
-  if (claim) {
-    int s = k == 0 ? last_seg : sm.cur_pool;
-    PoolInfo inf{0, 0, 0, 0};
-    if (k > 0) {
-      inf = sm.cur_info;
-    } else if (s >= 0) {
-      inf = p.pool[s];
-    }
-    DynEntry r{-1, 0, 0, 0};
-    // every failed take means another CTA took a chunk: the chunks bound the tries
-    const int tries = kPoolChunksPerCta * (int)gridDim.x + 2;
-    for (int t = 0; t < tries; ++t) {
-      if (s >= 0 && inf.pn > 0) {
-        int g = 0;
-        if (lane == 0) g = atomicAdd(p.pool_next + s, 1);
-        g = __shfl_sync(kFull, g, 0);
-        if (g < inf.pn) {
-          r.seg = s;
-          r.k0 = inf.pk0 + g * chunk;
-          r.k1 = r.k0 + chunk < inf.pk1 ? r.k0 + chunk : inf.pk1;
-          r.sbase = inf.sbase;
-          break;
-        }
-      }
-      // that pool is empty: look for the one with the most chunks left
-      int best = -1, brem = 0;
-      for (int i = lane; i < p.nseg; i += 32) {
-        const int pn = p.pool[i].pn;
-        if (pn > 0) {
-          const int rem = pn - __ldcg(p.pool_next + i);
-          if (rem > brem) {
-            brem = rem;
-            best = i;
-          }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const int ob = __shfl_xor_sync(kFull, best, off), orem = __shfl_xor_sync(kFull, brem, off);
-        if (orem > brem || (orem == brem && orem > 0 && ob < best)) {
-          brem = orem;
-          best = ob;
-        }
-      }
-      if (best < 0) break;  // every pool is empty
-      s = best;
-      inf = p.pool[s];
-    }
-    if (lane == 0) {
-      sm.cur_pool = s;
-      sm.cur_info = inf;
-      sm.dq[k] = r;
-      __threadfence_block();
-      atomicExch(&sm.dq_state[k], 2);
-    }
-    __syncwarp();
-    e = r;
-    return true;
-  }
-  int ok = 1;
-  if (lane == 0) {
-    volatile int* st = &sm.dq_state[k];
-    const unsigned long long t0 = globaltimer();
-    while (*st != 2) {
-      if (sm.abort_flag) {
-        ok = 0;
-        break;
-      }
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        sm.abort_flag = 1;
-        atomicOr(p.status, MAC_DEV_TIMEOUT);
-        ok = 0;
-        break;
-      }
-    }
-    __threadfence_block();
-  }
-  ok = __shfl_sync(kFull, ok, 0);
-  __syncwarp();
-  if (!ok) return false;
-  const volatile int* q = reinterpret_cast<const volatile int*>(&sm.dq[k]);
-  e.seg = q[0];
-  e.k0 = q[1];
-  e.k1 = q[2];
-  e.sbase = q[3];
-  return true;
-}
-
-// The CTA's pieces in order: its static range (Walker), then pool chunks.
-struct Source {
-  Walker w;
-  int k;         // next queue entry, once the static range is done
-  int last_seg;  // item of the last static piece if it was a split one, else -1
-  bool in_dyn;
-  template <int D>
-  __device__ __forceinline__ bool next(const AttendParams& p, AttnSmem<D>& sm, int cta, int chunk, Piece& pc) {
-    if (!in_dyn) {
-      if (w.next(p, cta, pc)) {
-        last_seg = pc.whole ? -1 : pc.seg;
-        return true;
-      }
-      in_dyn = true;
-    }
-    if (k >= kDynCap) return false;
-    DynEntry e;
-    if (!dyn_get<D>(p, sm, k, last_seg, chunk, e) || e.seg < 0) {
-      k = kDynCap;
-      return false;
-    }
-    ++k;
-    pc.unit = e.seg >> 1;
-    pc.seg = e.seg;
-    pc.whole = 0;
-    pc.dyn = 1;
-    pc.sbase = e.sbase;
-    pc.pidx = -1;
-    pc.wA = 0;
-    pc.anbox = 0;
-    pc.k0 = e.k0;
-    pc.k1 = e.k1;
-    pc.kb0 = e.k0 & ~(kSubKeys - 1);
-    pc.nbox = box_count(e.k0, e.k1);
-    return true;
-  }
-};
-
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
   constexpr int NST = Cfg<D>::NST, NQ = Cfg<D>::NQ, GD = Cfg<D>::GD;
@@ -884,10 +709,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     mbar_init(&sm.rfull, 1);
     sm.abort_flag = 0;
     sm.last_flag = 0;
-    sm.cur_pool = -1;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < kDynCap) sm.dq_state[tid] = 0;
   __syncthreads();
   // launched with programmatic stream serialization: everything above
   // overlaps the match kernel; its results are visible after this wait
@@ -895,30 +718,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   // one round of loads: the split, then the CTA's items into shared memory
   const int n_cta = p.hdr->n_cta;
   const long long T = p.hdr->total;
-  const int chunk = p.hdr->chunk, pooled = p.hdr->pooled;
-  const int first_seg_c = p.first_seg[cta];
-  // CTAs past n_cta have no static range; they still take pool chunks, so
-  // every CTA of the grid drains the pools (no CTA can hold more than
-  // kDynCap chunks, and the pools never exceed kPoolChunksPerCta per CTA)
-  const bool has_static = cta < n_cta;
-  if (!has_static && pooled == 0) return;
-  const int first_seg = has_static ? first_seg_c : p.nseg;
-  const long long lo = has_static ? (long long)cta * T / n_cta : 0;
-  const long long hi = has_static ? (long long)(cta + 1) * T / n_cta : 0;
+  const int first_seg = p.first_seg[cta];
+  if (cta >= n_cta) return;
+  const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
   if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = p.seg[first_seg + tid];
   __syncthreads();
   const uint64_t pol = evict_first_policy();
 
   // issue cursor: this warp's boxes of every piece, NST ahead
-  Source si{Walker{first_seg, lo, hi, sm.items, first_seg}, 0, -1, false};
+  Walker wi{first_seg, lo, hi, sm.items, first_seg};
   Piece ip;
   WarpRange ir;
-  bool ivalid = si.next<D>(p, sm, cta, chunk, ip);
+  bool ivalid = wi.next(p, cta, ip);
   if (ivalid) ir = warp_range(ip, warp);
   int ib = ivalid ? ir.first : 0, ipn = 0, nissued = 0, nq_issued = 0;
   auto issue_advance = [&]() {
     while (ivalid && ib >= ir.nbox) {
-      ivalid = si.next<D>(p, sm, cta, chunk, ip);
+      ivalid = wi.next(p, cta, ip);
       if (ivalid) {
         ir = warp_range(ip, warp);
         ib = ir.first;
@@ -962,34 +778,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 
   // consume cursor
   Acc<D> A;
-  Source sc{Walker{first_seg, lo, hi, sm.items, first_seg}, 0, -1, false};
+  Walker wc{first_seg, lo, hi, sm.items, first_seg};
   Piece cp;
   int cpn = 0, cons = 0, par = 0;
   uint32_t sync_phase = 0, ring_phase = 0;
   bool ring_pending = false;  // a reused-state copy was issued and not yet waited for
   bool ok = true;
-  // the run being accumulated: item, unit, partial slot, pieces and chunks in it
-  bool run = false;
-  int run_seg = -1, run_unit = 0, run_slot = 0, run_cnt = 0;
-  while (ok) {
-    const bool have = sc.next<D>(p, sm, cta, chunk, cp);
-    if (run && !(have && cp.dyn && cp.seg == run_seg)) {
-      if (!finalize_run<D>(p, sm, A, run_unit, run_slot, run_cnt, sync_phase)) break;
-      run = false;
-    }
-    if (!have) break;
+  while (ok && wc.next(p, cta, cp)) {
     const int qs = cpn % NQ;
     if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
-    if (!run) load_query<D>(A, sm.q[qs]);  // a run goes on with the same query and state
-    if (!cp.whole && !run) {
-      run = true;
-      run_seg = cp.seg;
-      run_unit = cp.unit;
-      run_cnt = 0;
-      run_slot = cp.pidx;
-      // a dynamic run's slot: taken now, used by thread 0 at the run's end
-      if (cp.dyn && tid == 0) run_slot = cp.sbase + atomicAdd(p.pool_slots + cp.seg, 1);
-    }
+    load_query<D>(A, sm.q[qs]);
     const bool ring_copy = cp.whole && cp.hit;
     ring_pending = ring_copy;
     if (ring_copy && tid == 0) {
@@ -1022,14 +820,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
     }
     if (!ok) break;
-    if (cp.whole) {
-      const bool fin = finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, ring_phase, sync_phase);
-      if (ring_copy) ring_phase ^= 1u;
-      ring_pending = false;
-      if (!fin) break;
-    } else {
-      ++run_cnt;
-    }
+    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, ring_phase, sync_phase)
+                              : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    if (ring_copy) ring_phase ^= 1u;
+    ring_pending = false;
+    if (!fin) break;
     ++cpn;
   }
   if (nissued > cons || !ok) {
@@ -1058,10 +853,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 }
 
 }  // namespace
-
-// the largest dynamic shared-memory window of one CTA on sm_100 is 227 KiB
-static_assert(sizeof(AttnSmem<128>) + 1024 <= 227 * 1024 && sizeof(AttnSmem<64>) + 1024 <= 227 * 1024,
-              "attention kernel shared memory");
 
 size_t attend_smem_bytes(int D) {
   return (D == 128 ? sizeof(AttnSmem<128>) : sizeof(AttnSmem<64>)) + 1024;

@@ -25,9 +25,7 @@ struct UnitPlan {
   int src_slot;  // ring slot of the matched entry (hit only)
   int dst_slot;  // ring slot receiving this step's entry
   int bad;       // 1 = invalid inputs: no work, NaN outputs, window unchanged
-  int expected;  // static pieces + pool chunks of the unit's two items: the
-                 // count its merge waits for (each partial adds the pieces and
-                 // chunks it covers)
+  int expected;  // partial results the unit's merge waits for
 };
 
 // Work items, two slots per unit u.  A large unit (more than unit_max fresh
@@ -55,27 +53,9 @@ struct Segment {
 
 struct PlanHeader {
   long long total;  // size of the flattened cost space
-  int n_cta;        // CTAs with a static range (<= grid)
-  int chunk;        // keys per pool chunk
-  int pooled;       // pool chunks over all items (0: CTAs past n_cta have no work)
+  int n_cta;        // CTAs with work (<= grid)
   int pad;
 };
-
-// Dynamic tail of a split item.  The last pn * chunk keys of a large split
-// item, [pk0, pk1), are not in the cost space: they form a pool of chunks
-// that CTAs take at run time (an atomic counter per pool) once their static
-// range is done, so CTAs that stream faster take more of the keys.  A CTA
-// accumulates consecutive chunks of one item (and the static piece it ended
-// on, if the item is the same) into one partial result.  The partial results
-// of item s occupy slots [pbase, pbase + npieces + pool_slots[s]): the static
-// pieces first, then one slot per dynamic run from sbase = pbase + npieces.
-struct PoolInfo {
-  int pk0, pk1;  // pool keys
-  int pn;        // chunks (0 = no pool)
-  int sbase;     // first slot of the dynamic runs' partial results
-};
-constexpr int kPoolChunksPerCta = 8;  // pool chunks over all items <= this x grid
-constexpr int kPoolChunkMin = 256;    // default smallest chunk, in keys
 
 // Layout of one partial result: o_acc [G][D] (unnormalised, relative to m),
 // then m [G] (log2 units), l [G].
@@ -99,9 +79,6 @@ struct MatchParams {
   Segment* seg;            // [2U]
   PlanHeader* hdr;
   int* first_seg;          // [grid] first segment of each attention CTA's range
-  PoolInfo* pool;          // [2U]
-  int* pool_next;          // [2U] chunks taken (reset here every step)
-  int* pool_slots;         // [2U] dynamic-run partial slots taken (reset here every step)
   int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
   int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;
@@ -110,8 +87,6 @@ struct MatchParams {
   int min_keys;   // minimum cost-space units per attention CTA
   int piece_cost; // fixed cost of one piece, in keys
   int unit_max;   // units with at most this many fresh keys are whole items
-  int pool_permille;  // share of each split item's keys left to the pools
-  int pool_chunk;     // smallest pool chunk, in keys (a multiple of 16)
 };
 
 struct AttendParams {
@@ -123,9 +98,6 @@ struct AttendParams {
   const Segment* seg;
   const PlanHeader* hdr;
   const int* first_seg;  // [grid]
-  const PoolInfo* pool;  // [2U]
-  int* pool_next;        // [2U]
-  int* pool_slots;       // [2U]
   float* part;       // [max_parts][partial_floats]
   int* unit_cnt;     // [U]
   float* ring_o;     // [U][W+1][G][D]

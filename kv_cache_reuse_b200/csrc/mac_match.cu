@@ -72,50 +72,18 @@ __device__ long long block_exclusive_scan(long long v, long long* total, long lo
   return before + x - v;
 }
 
-// floor(a / b) and ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit
-// integer division: an fp64 estimate (off by at most a few units) corrected
-// exactly.
-__device__ __forceinline__ long long floor_div(long long a, long long b, double rb) {
-  long long q = (long long)((double)a * rb);
-  while (q > 0 && q * b > a) --q;
-  while ((q + 1) * b <= a) ++q;
-  return q;
-}
-__device__ __forceinline__ long long ceil_div(long long a, long long b, double rb) {
-  const long long q = floor_div(a, b, rb);
-  return q + (q * b < a ? 1 : 0);
-}
 // CTA holding cost-space offset x when the space [0, T) is split over N CTAs
 // as [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
+// ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit integer
+// division: an fp64 estimate (off by at most a few units) corrected exactly.
+__device__ __forceinline__ long long ceil_div(long long a, long long b, double rb) {
+  long long q = (long long)((double)a * rb);
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;  // q = floor(a / b)
+  return q + (q * b < a ? 1 : 0);
+}
 __device__ __forceinline__ int cta_of(long long x, long long T, int N, double rT) {
   return (int)ceil_div((x + 1) * (long long)N, T, rT) - 1;
-}
-
-// The work item in slot s of the segment table, from its unit's plan.
-struct ItemDesc {
-  int kind, len, key0, cut, packed;
-};
-__device__ __forceinline__ ItemDesc item_of(const MatchParams& p, int s) {
-  ItemDesc it{kItemEmpty, 0, 0, 0, 0};
-  const UnitPlan* pl = p.plan + (s >> 1);
-  if (__ldcg(&pl->bad)) return it;
-  const int start = __ldcg(&pl->start), c = __ldcg(&pl->cut), end = __ldcg(&pl->end);
-  if (end - start <= p.unit_max) {
-    if ((s & 1) == 0) {  // the whole unit in slot 2u
-      it.kind = kItemWhole;
-      it.len = end - start;
-      it.key0 = start;
-      it.cut = c;
-      // the CTA doing it also needs hit, reused slot and written slot
-      const int hit = __ldcg(&pl->hit), src = __ldcg(&pl->src_slot), dst = __ldcg(&pl->dst_slot);
-      it.packed = (hit ? 1 : 0) | ((hit ? src : 0) << 1) | (dst << 12);
-    }
-  } else {
-    it.len = (s & 1) ? end - c : c - start;
-    it.key0 = (s & 1) ? c : start;
-    it.kind = it.len > 0 ? ((s & 1) ? kItemB : kItemA) : kItemEmpty;
-  }
-  return it;
 }
 
 __device__ void build_segments(const MatchParams& p, int U) {
@@ -123,57 +91,50 @@ __device__ void build_segments(const MatchParams& p, int U) {
   const int tid = threadIdx.x;
   const int nseg = 2 * U;
   const long long cost = p.piece_cost;
-  const bool regs = nseg <= kMatchThreads;  // one item per thread, kept in registers between passes
-  // pass 0: keys of all split items, which fix the pool chunk size
-  ItemDesc r_it{kItemEmpty, 0, 0, 0, 0};
+  // pass 1: item kinds, keys and cost-space offsets
   long long carry = 0;
+  long long r_flat = 0;  // this thread's item, kept for pass 2 when nseg <= kMatchThreads
+  int r_len = 0, r_kind = kItemEmpty;
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
-    const ItemDesc it = s < nseg ? item_of(p, s) : ItemDesc{kItemEmpty, 0, 0, 0, 0};
-    if (regs) r_it = it;
-    long long tot;
-    block_exclusive_scan(it.kind == kItemA || it.kind == kItemB ? it.len : 0, &tot, sbuf);
-    carry += tot;
-  }
-  const long long pool_keys = floor_div(carry * p.pool_permille, 1000, 1e-3);
-  const long long budget = (long long)kPoolChunksPerCta * p.grid;
-  long long C = ceil_div(pool_keys, budget, 1.0 / (double)budget);
-  C = (C + kSubKeys - 1) & ~(long long)(kSubKeys - 1);
-  if (C < p.pool_chunk) C = p.pool_chunk;
-  const long long div_pn = 1000 * C;
-  const double rdiv_pn = 1.0 / (double)div_pn;
-  // pass 1: static keys (the pool tail cut off) and cost-space offsets
-  carry = 0;
-  long long pooled = 0;
-  long long r_flat = 0;
-  int r_slen = 0, r_pn = 0;
-  for (int base = 0; base < nseg; base += kMatchThreads) {
-    const int s = base + tid;
-    const ItemDesc it = regs ? r_it : (s < nseg ? item_of(p, s) : ItemDesc{kItemEmpty, 0, 0, 0, 0});
-    const bool split = it.kind == kItemA || it.kind == kItemB;
-    int pn = 0;
-    if (split && p.pool_permille > 0) {
-      pn = (int)floor_div((long long)it.len * p.pool_permille, div_pn, rdiv_pn);
-      if ((long long)pn * C >= it.len) pn = (int)((it.len - 1) / C);  // keep a static key
-    }
-    const int slen = it.len - (int)(pn * C);
-    const long long wlen = it.kind != kItemEmpty ? (long long)slen + cost : 0;
-    long long tot, ptot;
-    const long long ex = block_exclusive_scan(wlen, &tot, sbuf);
-    block_exclusive_scan(pn, &ptot, sbuf);
-    pooled += ptot;
+    int len = 0, key0 = 0, kind = kItemEmpty, cut = 0, packed = 0;
+    long long wlen = 0;
     if (s < nseg) {
-      const long long flat = carry + ex + (split ? cost : 0);
-      p.seg[s].flat = flat;
-      p.seg[s].len = it.kind == kItemEmpty ? 0 : slen;
-      p.seg[s].key0 = it.key0;
-      p.seg[s].kind = it.kind;
-      p.seg[s].pbase = it.cut;  // whole items keep their cut here; split items overwrite it below
-      if (it.kind == kItemWhole) p.seg[s].npieces = it.packed;
-      p.pool[s] = PoolInfo{it.key0 + slen, it.key0 + it.len, pn, 0};
-      r_flat = flat;
-      r_slen = it.kind == kItemEmpty ? 0 : slen;
-      r_pn = pn;
+      const UnitPlan* pl = p.plan + (s >> 1);
+      const int bad = __ldcg(&pl->bad);
+      if (!bad) {
+        const int start = __ldcg(&pl->start), c = __ldcg(&pl->cut), end = __ldcg(&pl->end);
+        if (end - start <= p.unit_max) {
+          if ((s & 1) == 0) {  // the whole unit in slot 2u
+            kind = kItemWhole;
+            len = end - start;
+            key0 = start;
+            cut = c;
+            // the CTA doing it also needs hit, reused slot and written slot
+            const int hit = __ldcg(&pl->hit), src = __ldcg(&pl->src_slot), dst = __ldcg(&pl->dst_slot);
+            packed = (hit ? 1 : 0) | ((hit ? src : 0) << 1) | (dst << 12);
+          }
+        } else {
+          len = (s & 1) ? end - c : c - start;
+          key0 = (s & 1) ? c : start;
+          kind = len > 0 ? ((s & 1) ? kItemB : kItemA) : kItemEmpty;
+        }
+        if (kind != kItemEmpty) wlen = (long long)len + cost;
+      }
+    }
+    long long tot;
+    long long ex = block_exclusive_scan(wlen, &tot, sbuf);
+    if (s < nseg) {
+      const bool split = kind == kItemA || kind == kItemB;
+      p.seg[s].flat = carry + ex + (split ? cost : 0);
+      r_flat = carry + ex + (split ? cost : 0);
+      r_len = kind == kItemEmpty ? 0 : len;
+      r_kind = kind;
+      p.seg[s].len = kind == kItemEmpty ? 0 : len;
+      p.seg[s].key0 = key0;
+      p.seg[s].kind = kind;
+      p.seg[s].pbase = cut;  // whole items keep their cut here; split items overwrite it below
+      if (kind == kItemWhole) p.seg[s].npieces = packed;
     }
     carry += tot;
   }
@@ -190,19 +151,17 @@ __device__ void build_segments(const MatchParams& p, int U) {
   long long pcarry = 0;
   for (int base = 0; base < nseg; base += kMatchThreads) {
     const int s = base + tid;
-    int np = 0, first = 0, kind = kItemEmpty, len = 0, pn = 0;
+    int np = 0, first = 0, kind = kItemEmpty, len = 0;
     long long F = 0;
     if (s < nseg) {
-      if (regs) {
+      if (nseg <= kMatchThreads) {
         F = r_flat;
-        len = r_slen;
-        kind = r_it.kind;
-        pn = r_pn;
-      } else {  // written by this thread in pass 1
+        len = r_len;
+        kind = r_kind;
+      } else {
         F = p.seg[s].flat;
         len = p.seg[s].len;
         kind = p.seg[s].kind;
-        pn = p.pool[s].pn;
       }
       if (kind == kItemA || kind == kItemB) {
         first = cta_of(F, T, N, rT);
@@ -211,24 +170,17 @@ __device__ void build_segments(const MatchParams& p, int U) {
         first = cta_of(F, T, N, rT);
       }
     }
-    // slots: one per static piece, and for the dynamic runs at most one per
-    // CTA of the grid (a CTA leaves a pool only once it is empty) and one per
-    // chunk
     long long tot;
-    const long long ex = block_exclusive_scan(np + (pn < p.grid ? pn : p.grid), &tot, sbuf);
+    long long ex = block_exclusive_scan(np, &tot, sbuf);
     // units own items (2u, 2u+1): adjacent threads of one warp
-    const int cnt = np + pn;
-    const int cnt_next = __shfl_down_sync(0xffffffffu, cnt, 1);
+    const int np_next = __shfl_down_sync(0xffffffffu, np, 1);
     if (s < nseg) {
       p.seg[s].first_cta = first;
       if (kind != kItemWhole) {
         p.seg[s].npieces = np;
         p.seg[s].pbase = (int)(pcarry + ex);
       }
-      p.pool[s].sbase = (int)(pcarry + ex) + np;
-      p.pool_next[s] = 0;
-      p.pool_slots[s] = 0;
-      if ((s & 1) == 0) p.plan[s >> 1].expected = cnt + cnt_next;
+      if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
       // CTAs whose range starts inside this item's cost extent [Fw, Fe)
       // begin their walk here: lo_c = floor(c*T/N) lies in it iff
       // ceil(Fw*N/T) <= c < ceil(Fe*N/T)
@@ -245,8 +197,6 @@ __device__ void build_segments(const MatchParams& p, int U) {
   if (tid == 0) {
     p.hdr->total = T;
     p.hdr->n_cta = N;
-    p.hdr->chunk = (int)C;
-    p.hdr->pooled = (int)pooled;
   }
 }
 

@@ -42,8 +42,7 @@ constexpr size_t kOffPlan = align256(kOffQrot + (size_t)kMaxUnits * kGroup * kMa
 constexpr size_t kOffSeg = align256(kOffPlan + kMaxUnits * sizeof(UnitPlan));
 constexpr size_t kOffHdr = align256(kOffSeg + 2 * kMaxUnits * sizeof(Segment));
 constexpr size_t kOffFirst = align256(kOffHdr + sizeof(PlanHeader));
-constexpr size_t kOffPool = align256(kOffFirst + kMaxCtas * 4);  // pool [2U], then pool_next, pool_slots [2U] each
-constexpr size_t kOffPart = align256(kOffPool + 2 * kMaxUnits * sizeof(PoolInfo) + 4 * kMaxUnits * 4);
+constexpr size_t kOffPart = align256(kOffFirst + kMaxCtas * 4);
 constexpr size_t kOffCnt = align256(kOffPart + (size_t)(kMaxCtas + 2 * kMaxUnits) * kPartFloats * 4);
 // counters block, cleared on every call: unit_cnt[kMaxUnits], done, status, steps[kMaxUnits]
 constexpr size_t kCntBytes = (2 * kMaxUnits + 2) * 4;
@@ -174,9 +173,6 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.seg = reinterpret_cast<Segment*>(base + kOffSeg);
   mp.hdr = reinterpret_cast<PlanHeader*>(base + kOffHdr);
   mp.first_seg = reinterpret_cast<int*>(base + kOffFirst);
-  mp.pool = reinterpret_cast<PoolInfo*>(base + kOffPool);
-  mp.pool_next = reinterpret_cast<int*>(base + kOffPool + 2 * kMaxUnits * sizeof(PoolInfo));
-  mp.pool_slots = mp.pool_next + 2 * kMaxUnits;
   mp.done = cnt + kMaxUnits;
   mp.status = status;
   mp.B = batch;
@@ -193,8 +189,6 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.min_keys = 128;
   mp.piece_cost = 1024;
   mp.unit_max = 1024;
-  mp.pool_permille = 0;  // no pools: the partial slots above hold the static pieces only
-  mp.pool_chunk = kPoolChunkMin;
   if (launch_match(mp, head_dim, st) != cudaSuccess) return MAC_ERR_CUDA;
 
   // --- attention over every key, merge into out/lse (and the dummy ring)
@@ -211,9 +205,6 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.seg = mp.seg;
   ap.hdr = mp.hdr;
   ap.first_seg = mp.first_seg;
-  ap.pool = mp.pool;
-  ap.pool_next = mp.pool_next;
-  ap.pool_slots = mp.pool_slots;
   ap.part = reinterpret_cast<float*>(base + kOffPart);
   ap.unit_cnt = cnt;
   ap.ring_o = reinterpret_cast<float*>(base + kOffRingO);

@@ -31,9 +31,8 @@ class GpuRun:
                                                 num_pages=cache.num_pages, tau=tau, band=band, window=window)
         else:
             self.st = mac.MacState.for_workload(wl, capacity=cache.max_seq, tau=tau, band=band, window=window)
-        for name, val in (tune or {}).items():  # work-split knobs: min_keys_per_cta, piece_cost, whole_unit_keys,
-            fn = getattr(mac, "mac_set_" + name)  # pool_share (permille, chunk_keys)
-            fn(self.st, *val) if isinstance(val, tuple) else fn(self.st, val)
+        for name, val in (tune or {}).items():  # work-split knobs: min_keys_per_cta, piece_cost, whole_unit_keys
+            getattr(mac, "mac_set_" + name)(self.st, val)
         B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
         f32, i32 = torch.float32, torch.int32
         self.q = torch.empty((B, Hq, D), dtype=f32, device=dev)

@@ -59,6 +59,3 @@ def test_tuning_setters_reject_bad_handles(lib):
         with pytest.raises(mac.MacError) as e:
             getattr(mac, name)(None, 4)
         assert e.value.code == mac.MAC_ERR_ARG
-    with pytest.raises(mac.MacError) as e:
-        mac.mac_set_pool_share(None, 250, 256)
-    assert e.value.code == mac.MAC_ERR_ARG

@@ -270,10 +270,6 @@ def test_edge_cases(case):
     {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 16},  # many tiny pieces per unit
     {"whole_unit_keys": 1 << 20},                                     # every unit done by one CTA
     {"piece_cost": 1 << 16, "min_keys_per_cta": 1},                   # one piece per CTA at most
-    {"pool_share": (0, 256)},                                         # no run-time balancing
-    {"pool_share": (1000, 16), "whole_unit_keys": 0},                 # nearly every key taken at run time
-    {"pool_share": (500, 64), "whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 16},
-    {"pool_share": (700, 16), "min_keys_per_cta": 1 << 24},           # one static CTA; the idle ones drain the pools
 ])
 def test_work_split_settings_keep_parity(tune):
     """How the keys are divided among CTAs changes only rounding, never decisions."""
