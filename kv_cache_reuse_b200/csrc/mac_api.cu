@@ -33,6 +33,9 @@ struct MacState {
   Segment* seg = nullptr;
   PlanHeader* hdr = nullptr;
   int* first_seg = nullptr;
+  float* rate = nullptr;        // learned streaming rate per SM (weighted split)
+  long long* bounds = nullptr;  // range starts of a weighted split
+  int* claim = nullptr;         // ranges taken by the attention CTAs
   float* part = nullptr;
   int* unit_cnt = nullptr;
   int* done = nullptr;
@@ -95,7 +98,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,
-                  s->seg,    s->hdr,    s->first_seg, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->rate, s->bounds, s->claim, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -241,6 +244,9 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->seg, 2 * U));
   A(alloc(&s->hdr, 1));
   A(alloc(&s->first_seg, (size_t)s->grid));
+  A(alloc(&s->rate, (size_t)s->grid));
+  A(alloc(&s->bounds, (size_t)s->grid + 1));
+  A(alloc(&s->claim, (size_t)s->grid));
   A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
   A(alloc(&s->unit_cnt, U));
   A(alloc(&s->done, 1));
@@ -277,6 +283,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->steps, 0, U * sizeof(int)));
   A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
   A(cudaMemset(s->done, 0, sizeof(int)));
+  A(cudaMemset(s->rate, 0, s->grid * sizeof(float)));
+  A(cudaMemset(s->claim, 0, s->grid * sizeof(int)));
   A(cudaMemset(s->dev_out, 0, s->out_bytes));
   A(cudaMemset(s->hdr, 0, sizeof(PlanHeader)));
   double* inv = (double*)malloc(sizeof(double) * (D / 2));
@@ -354,6 +362,9 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
+  p.rate = s->rate;
+  p.bounds = s->bounds;
+  p.claim = s->claim;
   p.done = s->done;
   p.status = s->status;
   p.B = s->cfg.batch;
@@ -397,6 +408,9 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
+  p.bounds = s->bounds;
+  p.claim = s->claim;
+  p.rate = s->rate;
   p.part = s->part;
   p.unit_cnt = s->unit_cnt;
   p.ring_o = s->ring_o;
@@ -412,6 +426,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.page_size = s->cfg.page_size;
   p.max_pages = s->cfg.max_pages_per_seq;
   p.nseg = 2 * s->U;
+  p.grid = s->grid;
   return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 

@@ -716,11 +716,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   // overlaps the match kernel; its results are visible after this wait
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // one round of loads: the split, then the CTA's items into shared memory
-  const int n_cta = p.hdr->n_cta;
+  unsigned smid;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+  const int n_cta = p.hdr->n_cta, weighted = p.hdr->weighted;
   const long long T = p.hdr->total;
-  const int first_seg = p.first_seg[cta];
-  if (cta >= n_cta) return;
-  const long long lo = (long long)cta * T / n_cta, hi = (long long)(cta + 1) * T / n_cta;
+  int first_seg = p.first_seg[cta];
+  // a weighted split: take the range of this SM (claimed in the same round
+  // of loads), else the first free one
+  int mine = 0;
+  if (tid == 0 && p.claim != nullptr && (int)smid < p.grid) mine = atomicCAS(p.claim + smid, 0, 1) == 0;
+  int slot = cta;
+  long long lo, hi;
+  if (weighted) {
+    if (tid == 0) {
+      int c = mine ? (int)smid : -1;
+      for (int k = 0; c < 0 && k < n_cta; ++k)
+        if (atomicCAS(p.claim + k, 0, 1) == 0) c = k;
+      sm.last_flag = c;
+    }
+    __syncthreads();
+    slot = sm.last_flag;
+    if (slot < 0) return;  // never: n_cta = grid ranges for grid CTAs
+    lo = p.bounds[slot];
+    hi = p.bounds[slot + 1];
+    first_seg = p.first_seg[slot];
+  } else {
+    if (cta >= n_cta) return;
+    lo = (long long)cta * T / n_cta;
+    hi = (long long)(cta + 1) * T / n_cta;
+  }
   if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = p.seg[first_seg + tid];
   __syncthreads();
   const uint64_t pol = evict_first_policy();
@@ -729,12 +753,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   Walker wi{first_seg, lo, hi, sm.items, first_seg};
   Piece ip;
   WarpRange ir;
-  bool ivalid = wi.next(p, cta, ip);
+  bool ivalid = wi.next(p, slot, ip);
   if (ivalid) ir = warp_range(ip, warp);
   int ib = ivalid ? ir.first : 0, ipn = 0, nissued = 0, nq_issued = 0;
   auto issue_advance = [&]() {
     while (ivalid && ib >= ir.nbox) {
-      ivalid = wi.next(p, cta, ip);
+      ivalid = wi.next(p, slot, ip);
       if (ivalid) {
         ir = warp_range(ip, warp);
         ib = ir.first;
@@ -784,7 +808,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   uint32_t sync_phase = 0, ring_phase = 0;
   bool ring_pending = false;  // a reused-state copy was issued and not yet waited for
   bool ok = true;
-  while (ok && wc.next(p, cta, cp)) {
+  unsigned long long t_first = 0, t_last = 0;  // thread 0: first and last box consumed
+  while (ok && wc.next(p, slot, cp)) {
     const int qs = cpn % NQ;
     if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
     load_query<D>(A, sm.q[qs]);
@@ -807,6 +832,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
         ok = false;
         break;
       }
+      if (tid == 0 && cons == 0) t_first = globaltimer();
       const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * 64;
       process_box<D>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
@@ -820,12 +846,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
     }
     if (!ok) break;
+    if (tid == 0) t_last = globaltimer();
     const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, ring_phase, sync_phase)
                               : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (ring_copy) ring_phase ^= 1u;
     ring_pending = false;
     if (!fin) break;
     ++cpn;
+  }
+  if (weighted && ok && tid == 0 && p.rate != nullptr && (int)smid < p.grid && t_last > t_first + 2000) {
+    // fold this SM's streaming rate (cost units per microsecond) into its record
+    const float r = (float)((double)(hi - lo) * 1000.0 / (double)(t_last - t_first));
+    const float old = p.rate[smid];
+    p.rate[smid] = old > 0.f ? 0.7f * old + 0.3f * r : r;
   }
   if (nissued > cons || !ok) {
     // aborting: let copies already issued land before the CTA leaves (bounded)

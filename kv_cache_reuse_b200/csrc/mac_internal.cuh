@@ -54,8 +54,16 @@ struct Segment {
 struct PlanHeader {
   long long total;  // size of the flattened cost space
   int n_cta;        // CTAs with work (<= grid)
-  int pad;
+  int weighted;     // 1: range c is [bounds[c], bounds[c+1]), sized by its SM's rate
 };
+
+// Weighted split.  HBM throughput differs between SMs, and the slow ones are
+// the same from step to step.  On steps with at least kWeightMinCost cost
+// units per CTA, range c of the split is sized in proportion to the learned
+// streaming rate of SM c, and the CTA running on SM c takes range c (a CTA
+// whose SM's range is already taken takes a free one).  At the end of such a
+// step every CTA folds its measured rate into rate[its SM].
+constexpr long long kWeightMinCost = 4096;
 
 // Layout of one partial result: o_acc [G][D] (unnormalised, relative to m),
 // then m [G] (log2 units), l [G].
@@ -79,6 +87,9 @@ struct MatchParams {
   Segment* seg;            // [2U]
   PlanHeader* hdr;
   int* first_seg;          // [grid] first segment of each attention CTA's range
+  const float* rate;       // [grid] learned rate per SM, or null (even split)
+  long long* bounds;       // [grid + 1] range starts of a weighted split
+  int* claim;              // [grid] ranges taken by the attention CTAs (reset here)
   int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
   int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;
@@ -98,6 +109,9 @@ struct AttendParams {
   const Segment* seg;
   const PlanHeader* hdr;
   const int* first_seg;  // [grid]
+  const long long* bounds;  // [grid + 1]
+  int* claim;        // [grid]
+  float* rate;       // [grid] or null
   float* part;       // [max_parts][partial_floats]
   int* unit_cnt;     // [U]
   float* ring_o;     // [U][W+1][G][D]
@@ -107,7 +121,7 @@ struct AttendParams {
   float* out;        // [B][Hq][D]
   float* lse;        // [B][Hq]
   unsigned* status;
-  int Hq, Hkv, W, page_size, max_pages, nseg;
+  int Hq, Hkv, W, page_size, max_pages, nseg, grid;
 };
 
 struct AppendParams {

@@ -72,6 +72,20 @@ __device__ long long block_exclusive_scan(long long v, long long* total, long lo
   return before + x - v;
 }
 
+// Sum of v over the block (every thread gets it).
+__device__ long long block_sum_ll(long long v, long long* sbuf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sbuf[warp] = v;
+  __syncthreads();
+  long long t = 0;
+#pragma unroll
+  for (int w = 0; w < kMatchThreads / 32; ++w) t += sbuf[w];
+  __syncthreads();
+  return t;
+}
+
 // CTA holding cost-space offset x when the space [0, T) is split over N CTAs
 // as [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
 // ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit integer
@@ -146,6 +160,52 @@ __device__ void build_segments(const MatchParams& p, int U) {
     if (N < 1) N = 1;
   }
   const double rT = T > 0 ? 1.0 / (double)T : 0.0;
+  // weighted split: range c in proportion to the learned rate of SM c
+  // (unknown rates count as the mean, all rates clamped to [1/2, 2] x mean)
+  __shared__ long long sbound[kMatchThreads + 1];
+  const bool weighted =
+      p.rate != nullptr && N == p.grid && p.grid <= kMatchThreads && T >= kWeightMinCost * (long long)p.grid;
+  if (weighted) {
+    const float r = tid < N ? p.rate[tid] : 0.f;
+    const long long packed = block_sum_ll(r > 0.f ? ((long long)1 << 40) + (long long)(r * 1048576.0f) : 0, sbuf);
+    const int known = (int)(packed >> 40);
+    const double mean = known > 0 ? (double)(packed & (((long long)1 << 40) - 1)) / (1048576.0 * known) : 1.0;
+    double w = r > 0.f ? (double)r : mean;
+    w = fmin(fmax(w, 0.5 * mean), 2.0 * mean);
+    // fixed point (units of mean / 2^20) so the scan is exact
+    const long long wi = tid < N ? (long long)(w / mean * 1048576.0) : 0;
+    long long wtot;
+    const long long wex = block_exclusive_scan(wi, &wtot, sbuf);
+    if (tid < N) sbound[tid] = (long long)((double)T * ((double)wex / (double)wtot));
+    if (tid == 0) {
+      sbound[0] = 0;
+      sbound[N] = T;
+    }
+    __syncthreads();
+    if (tid <= N) p.bounds[tid] = sbound[tid];
+  }
+  if (p.claim != nullptr)
+    for (int c = tid; c < p.grid; c += kMatchThreads) p.claim[c] = 0;
+  // CTA holding offset x: the largest c with start(c) <= x
+  auto owner = [&](long long x) -> int {
+    if (!weighted) return cta_of(x, T, N, rT);
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sbound[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  // first CTA whose range starts at or after x
+  auto first_from = [&](long long x) -> long long {
+    if (!weighted) return ceil_div(x * N, T, rT);
+    int lo = 0, hi = N;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sbound[mid] >= x) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+  };
   __syncthreads();
   // pass 2: owning / first CTA, partial slots, and each CTA's first item
   long long pcarry = 0;
@@ -164,10 +224,10 @@ __device__ void build_segments(const MatchParams& p, int U) {
         kind = p.seg[s].kind;
       }
       if (kind == kItemA || kind == kItemB) {
-        first = cta_of(F, T, N, rT);
-        np = cta_of(F + len - 1, T, N, rT) - first + 1;
+        first = owner(F);
+        np = owner(F + len - 1) - first + 1;
       } else if (kind == kItemWhole) {
-        first = cta_of(F, T, N, rT);
+        first = owner(F);
       }
     }
     long long tot;
@@ -182,13 +242,13 @@ __device__ void build_segments(const MatchParams& p, int U) {
       }
       if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
       // CTAs whose range starts inside this item's cost extent [Fw, Fe)
-      // begin their walk here: lo_c = floor(c*T/N) lies in it iff
-      // ceil(Fw*N/T) <= c < ceil(Fe*N/T)
+      // begin their walk here (even split: lo_c = floor(c*T/N) lies in it
+      // iff ceil(Fw*N/T) <= c < ceil(Fe*N/T))
       if (kind != kItemEmpty && N > 0) {
         const bool split = kind == kItemA || kind == kItemB;
         const long long Fw = split ? F - cost : F;
         const long long Fe = Fw + len + cost;
-        const long long ca = ceil_div(Fw * N, T, rT), cb = ceil_div(Fe * N, T, rT);
+        const long long ca = first_from(Fw), cb = first_from(Fe);
         for (long long c = ca; c < cb && c < N; ++c) p.first_seg[c] = s;
       }
     }
@@ -197,6 +257,7 @@ __device__ void build_segments(const MatchParams& p, int U) {
   if (tid == 0) {
     p.hdr->total = T;
     p.hdr->n_cta = N;
+    p.hdr->weighted = weighted ? 1 : 0;
   }
 }
 

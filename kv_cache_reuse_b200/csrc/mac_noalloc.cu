@@ -173,6 +173,9 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.seg = reinterpret_cast<Segment*>(base + kOffSeg);
   mp.hdr = reinterpret_cast<PlanHeader*>(base + kOffHdr);
   mp.first_seg = reinterpret_cast<int*>(base + kOffFirst);
+  mp.rate = nullptr;  // even split: no per-SM record
+  mp.bounds = nullptr;
+  mp.claim = nullptr;
   mp.done = cnt + kMaxUnits;
   mp.status = status;
   mp.B = batch;
@@ -205,6 +208,9 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.seg = mp.seg;
   ap.hdr = mp.hdr;
   ap.first_seg = mp.first_seg;
+  ap.bounds = nullptr;
+  ap.claim = nullptr;
+  ap.rate = nullptr;
   ap.part = reinterpret_cast<float*>(base + kOffPart);
   ap.unit_cnt = cnt;
   ap.ring_o = reinterpret_cast<float*>(base + kOffRingO);
@@ -220,5 +226,6 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.page_size = page_size;
   ap.max_pages = max_pages_per_seq;
   ap.nseg = 2 * U;
+  ap.grid = grid;
   return launch_attend(ap, head_dim, grid, st) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }

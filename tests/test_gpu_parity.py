@@ -265,6 +265,15 @@ def test_edge_cases(case):
     compare_stream(wl, stream, cache)
 
 
+def test_weighted_split_all_miss():
+    """Large all-miss steps take the rate-weighted split (ranges sized by each
+    SM's learned rate, taken by the CTA on that SM); results match the oracle
+    on the first step (even weights) and the later ones (learned weights)."""
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=4, L0=(32768, 30000, 31000, 29000), steps=5)
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=0.0)
+    assert r["hits"] == 0
+
+
 @pytest.mark.parametrize("tune", [
     {"whole_unit_keys": 0},                                           # every range cut over CTAs
     {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 16},  # many tiny pieces per unit
