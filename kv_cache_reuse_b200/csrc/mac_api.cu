@@ -35,6 +35,7 @@ struct MacState {
   int* first_seg = nullptr;
   float* rate = nullptr;        // learned streaming rate per SM (weighted split)
   long long* bounds = nullptr;  // range starts of a weighted split
+  double* cw = nullptr;         // cumulative range shares of the next weighted split
   int* claim = nullptr;         // ranges taken by the attention CTAs
   float* part = nullptr;
   int* unit_cnt = nullptr;
@@ -98,7 +99,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,
-                  s->seg,    s->hdr,    s->first_seg, s->rate, s->bounds, s->claim, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -246,6 +247,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->first_seg, (size_t)s->grid));
   A(alloc(&s->rate, (size_t)s->grid));
   A(alloc(&s->bounds, (size_t)s->grid + 1));
+  A(alloc(&s->cw, (size_t)s->grid + 1));
   A(alloc(&s->claim, (size_t)s->grid));
   A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
   A(alloc(&s->unit_cnt, U));
@@ -285,6 +287,12 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->done, 0, sizeof(int)));
   A(cudaMemset(s->rate, 0, s->grid * sizeof(float)));
   A(cudaMemset(s->claim, 0, s->grid * sizeof(int)));
+  {  // even shares until the first rates are measured
+    double* cw = (double*)malloc(sizeof(double) * (s->grid + 1));
+    for (int c = 0; c <= s->grid; ++c) cw[c] = (double)c / s->grid;
+    A(cudaMemcpy(s->cw, cw, sizeof(double) * (s->grid + 1), cudaMemcpyHostToDevice));
+    free(cw);
+  }
   A(cudaMemset(s->dev_out, 0, s->out_bytes));
   A(cudaMemset(s->hdr, 0, sizeof(PlanHeader)));
   double* inv = (double*)malloc(sizeof(double) * (D / 2));
@@ -362,7 +370,7 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
-  p.rate = s->rate;
+  p.cw = s->cw;
   p.bounds = s->bounds;
   p.claim = s->claim;
   p.done = s->done;
@@ -411,6 +419,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.bounds = s->bounds;
   p.claim = s->claim;
   p.rate = s->rate;
+  p.cw = s->cw;
   p.part = s->part;
   p.unit_cnt = s->unit_cnt;
   p.ring_o = s->ring_o;

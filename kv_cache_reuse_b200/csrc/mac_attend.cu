@@ -59,6 +59,7 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+constexpr int kRateMinBoxes = 256;  // a CTA's rate record needs this much streaming
 constexpr int kItemCache = 64;  // work items of one CTA kept in shared memory
 
 template <int D>
@@ -84,6 +85,7 @@ struct __align__(1024) AttnSmem {
   unsigned long long rfull;          // reused ring state of the current whole-unit piece landed
   int abort_flag;
   int last_flag;
+  int box_total;                     // boxes consumed by all warps (rate record)
   Segment items[kItemCache];         // the CTA's work items, from its first one on
   alignas(16) float ring[Cfg<D>::GD + 2 * kGroup];  // that ring state: o [G][D], m [G], l [G]
 };
@@ -687,6 +689,46 @@ struct Walker {
   }
 };
 
+// The cumulative range shares of the next weighted split from the SMs'
+// rate records, by all threads of one CTA: unknown rates count as the mean,
+// all are clamped to [1/2, 2] x mean, then scanned in fixed point (units of
+// mean / 2^20, so the scan is exact).  Rates of other SMs may still be
+// changing: any mix of old and new values is a valid split.
+__device__ __noinline__ void rate_shares(const AttendParams& p) {
+  __shared__ long long red[kConsumerWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, G = p.grid;
+  const float r = tid < G ? __ldcg(p.rate + tid) : 0.f;
+  long long v = r > 0.f ? ((long long)1 << 40) + (long long)(r * 1048576.0f) : 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  long long tot = 0;
+#pragma unroll
+  for (int w = 0; w < kConsumerWarps; ++w) tot += red[w];
+  __syncthreads();
+  const int known = (int)(tot >> 40);
+  const double mean = known > 0 ? (double)(tot & (((long long)1 << 40) - 1)) / (1048576.0 * known) : 1.0;
+  const double w = r > 0.f ? fmin(fmax((double)r, 0.5 * mean), 2.0 * mean) : mean;
+  const long long wi = tid < G ? (long long)(w / mean * 1048576.0) : 0;
+  long long x = wi;  // inclusive scan: lanes, then warps
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(kFull, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  long long before = 0, all = 0;
+#pragma unroll
+  for (int k = 0; k < kConsumerWarps; ++k) {
+    if (k < warp) before += red[k];
+    all += red[k];
+  }
+  if (tid < G) p.cw[tid] = (double)(before + x - wi) / (double)all;
+  if (tid == 0) p.cw[G] = 1.0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
   constexpr int NST = Cfg<D>::NST, NQ = Cfg<D>::NQ, GD = Cfg<D>::GD;
@@ -709,6 +751,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     mbar_init(&sm.rfull, 1);
     sm.abort_flag = 0;
     sm.last_flag = 0;
+    sm.box_total = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -854,11 +897,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     if (!fin) break;
     ++cpn;
   }
-  if (weighted && ok && tid == 0 && p.rate != nullptr && (int)smid < p.grid && t_last > t_first + 2000) {
-    // fold this SM's streaming rate (cost units per microsecond) into its record
-    const float r = (float)((double)(hi - lo) * 1000.0 / (double)(t_last - t_first));
-    const float old = p.rate[smid];
-    p.rate[smid] = old > 0.f ? 0.7f * old + 0.3f * r : r;
+  if (weighted && p.rate != nullptr) {
+    // fold this SM's streaming rate (boxes per microsecond) into its record;
+    // only CTAs that mostly streamed (at least kRateMinBoxes boxes) measure it
+    if (lane == 0) atomicAdd(&sm.box_total, cons);
+    __syncthreads();
+    const int boxes = sm.box_total;
+    if (ok && tid == 0 && (int)smid < p.grid && boxes >= kRateMinBoxes && t_last > t_first + 2000) {
+      const float r = (float)((double)boxes * 1000.0 / (double)(t_last - t_first));
+      const float old = p.rate[smid];
+      p.rate[smid] = old > 0.f ? 0.7f * old + 0.3f * r : r;
+    }
+    if (blockIdx.x == 0 && p.cw != nullptr && p.grid < kAttnThreads) rate_shares(p);
   }
   if (nissued > cons || !ok) {
     // aborting: let copies already issued land before the CTA leaves (bounded)

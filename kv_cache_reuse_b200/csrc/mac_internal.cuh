@@ -62,7 +62,9 @@ struct PlanHeader {
 // units per CTA, range c of the split is sized in proportion to the learned
 // streaming rate of SM c, and the CTA running on SM c takes range c (a CTA
 // whose SM's range is already taken takes a free one).  At the end of such a
-// step every CTA folds its measured rate into rate[its SM].
+// step every CTA folds its measured rate into rate[its SM], and CTA 0 turns
+// the rates into the cumulative shares cw[] that the next weighted step's
+// split uses (cw[c] = share of ranges 0..c-1, cw[grid] = 1).
 constexpr long long kWeightMinCost = 4096;
 
 // Layout of one partial result: o_acc [G][D] (unnormalised, relative to m),
@@ -87,7 +89,7 @@ struct MatchParams {
   Segment* seg;            // [2U]
   PlanHeader* hdr;
   int* first_seg;          // [grid] first segment of each attention CTA's range
-  const float* rate;       // [grid] learned rate per SM, or null (even split)
+  const double* cw;        // [grid + 1] cumulative range shares, or null (even split)
   long long* bounds;       // [grid + 1] range starts of a weighted split
   int* claim;              // [grid] ranges taken by the attention CTAs (reset here)
   int* done;               // arrival counter of the match CTAs (reset by the last)
@@ -111,7 +113,8 @@ struct AttendParams {
   const int* first_seg;  // [grid]
   const long long* bounds;  // [grid + 1]
   int* claim;        // [grid]
-  float* rate;       // [grid] or null
+  float* rate;       // [grid] learned rate per SM, or null
+  double* cw;        // [grid + 1] cumulative range shares (written by CTA 0)
   float* part;       // [max_parts][partial_floats]
   int* unit_cnt;     // [U]
   float* ring_o;     // [U][W+1][G][D]

@@ -72,20 +72,6 @@ __device__ long long block_exclusive_scan(long long v, long long* total, long lo
   return before + x - v;
 }
 
-// Sum of v over the block (every thread gets it).
-__device__ long long block_sum_ll(long long v, long long* sbuf) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (lane == 0) sbuf[warp] = v;
-  __syncthreads();
-  long long t = 0;
-#pragma unroll
-  for (int w = 0; w < kMatchThreads / 32; ++w) t += sbuf[w];
-  __syncthreads();
-  return t;
-}
-
 // CTA holding cost-space offset x when the space [0, T) is split over N CTAs
 // as [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
 // ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit integer
@@ -100,7 +86,7 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int N, double rT
   return (int)ceil_div((x + 1) * (long long)N, T, rT) - 1;
 }
 
-__device__ void build_segments(const MatchParams& p, int U) {
+__device__ void build_segments(const MatchParams& p, int U, double cw_c) {
   __shared__ long long sbuf[kMatchThreads / 32];
   const int tid = threadIdx.x;
   const int nseg = 2 * U;
@@ -160,51 +146,31 @@ __device__ void build_segments(const MatchParams& p, int U) {
     if (N < 1) N = 1;
   }
   const double rT = T > 0 ? 1.0 / (double)T : 0.0;
-  // weighted split: range c in proportion to the learned rate of SM c
-  // (unknown rates count as the mean, all rates clamped to [1/2, 2] x mean)
+  // weighted split: range c from the cumulative shares of the SMs' rates
   __shared__ long long sbound[kMatchThreads + 1];
   const bool weighted =
-      p.rate != nullptr && N == p.grid && p.grid <= kMatchThreads && T >= kWeightMinCost * (long long)p.grid;
+      p.cw != nullptr && N == p.grid && p.grid < kMatchThreads && T >= kWeightMinCost * (long long)p.grid;
   if (weighted) {
-    const float r = tid < N ? p.rate[tid] : 0.f;
-    const long long packed = block_sum_ll(r > 0.f ? ((long long)1 << 40) + (long long)(r * 1048576.0f) : 0, sbuf);
-    const int known = (int)(packed >> 40);
-    const double mean = known > 0 ? (double)(packed & (((long long)1 << 40) - 1)) / (1048576.0 * known) : 1.0;
-    double w = r > 0.f ? (double)r : mean;
-    w = fmin(fmax(w, 0.5 * mean), 2.0 * mean);
-    // fixed point (units of mean / 2^20) so the scan is exact
-    const long long wi = tid < N ? (long long)(w / mean * 1048576.0) : 0;
-    long long wtot;
-    const long long wex = block_exclusive_scan(wi, &wtot, sbuf);
-    if (tid < N) sbound[tid] = (long long)((double)T * ((double)wex / (double)wtot));
-    if (tid == 0) {
-      sbound[0] = 0;
-      sbound[N] = T;
-    }
+    if (tid <= N) sbound[tid] = tid == 0 ? 0 : (tid == N ? T : (long long)((double)T * cw_c));
     __syncthreads();
     if (tid <= N) p.bounds[tid] = sbound[tid];
   }
   if (p.claim != nullptr)
     for (int c = tid; c < p.grid; c += kMatchThreads) p.claim[c] = 0;
-  // CTA holding offset x: the largest c with start(c) <= x
+  // CTA holding offset x: the largest c with start(c) <= x (weighted: from
+  // the even split's guess, walked to the exact range; the weights are near 1)
   auto owner = [&](long long x) -> int {
     if (!weighted) return cta_of(x, T, N, rT);
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (sbound[mid] <= x) lo = mid; else hi = mid - 1;
-    }
-    return lo;
+    int c = (int)((double)x * N * rT);
+    c = c < 0 ? 0 : (c > N - 1 ? N - 1 : c);
+    while (c > 0 && sbound[c] > x) --c;
+    while (c < N - 1 && sbound[c + 1] <= x) ++c;
+    return c;
   };
   // first CTA whose range starts at or after x
   auto first_from = [&](long long x) -> long long {
     if (!weighted) return ceil_div(x * N, T, rT);
-    int lo = 0, hi = N;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (sbound[mid] >= x) hi = mid; else lo = mid + 1;
-    }
-    return lo;
+    return x <= 0 ? 0 : owner(x - 1) + 1;
   };
   __syncthreads();
   // pass 2: owning / first CTA, partial slots, and each CTA's first item
@@ -275,6 +241,9 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   // the attention kernel (launched with programmatic stream serialization)
   // may start its prologue now; it waits for this grid before reading
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the split's cumulative share of range tid, loaded now so the CTA that
+  // builds the split does not wait for it
+  const double cw_c = (p.cw != nullptr && (int)threadIdx.x <= p.grid) ? __ldcg(p.cw + threadIdx.x) : 0.0;
   const int u = blockIdx.x;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -458,7 +427,7 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  build_segments(p, (int)gridDim.x);
+  build_segments(p, (int)gridDim.x, cw_c);
   if (tid == 0) *p.done = 0;
 }
 

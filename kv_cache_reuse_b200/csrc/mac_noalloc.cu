@@ -173,7 +173,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.seg = reinterpret_cast<Segment*>(base + kOffSeg);
   mp.hdr = reinterpret_cast<PlanHeader*>(base + kOffHdr);
   mp.first_seg = reinterpret_cast<int*>(base + kOffFirst);
-  mp.rate = nullptr;  // even split: no per-SM record
+  mp.cw = nullptr;  // even split: no per-SM record
   mp.bounds = nullptr;
   mp.claim = nullptr;
   mp.done = cnt + kMaxUnits;
@@ -211,6 +211,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.bounds = nullptr;
   ap.claim = nullptr;
   ap.rate = nullptr;
+  ap.cw = nullptr;
   ap.part = reinterpret_cast<float*>(base + kOffPart);
   ap.unit_cnt = cnt;
   ap.ring_o = reinterpret_cast<float*>(base + kOffRingO);
