@@ -27,8 +27,10 @@
  *                 same sequence, per KV head; an entry is eligible only if its
  *                 position precedes the current one;
  *   [cut]         every step stores its prefix state over keys [0, c) with
- *                 c = max(0, p - b); on a hit the band [c_s, c_t) and the tail
- *                 [c_t, p_t] are recomputed with the current query;
+ *                 c = max(0, p - b) (cut_mode 0: the band is the b keys
+ *                 before p), or c = max(0, p + 1 - b) (cut_mode 1: the band
+ *                 ends at p itself); on a hit the band [c_s, c_t) and the
+ *                 tail [c_t, p_t] are recomputed with the current query;
  *   [rope]        keys in the cache are post-RoPE; the query is rotated here
  *                 with rotate-half pairs (i, i + D/2), inv_freq_i =
  *                 theta^(-2i/D), angle in fp64;
@@ -54,6 +56,7 @@ typedef struct {
     int page_size;         /* 0: contiguous K/V [B][max_seq][Hkv][D] */
     int max_seq;           /* rows per sequence (contiguous) */
     int max_pages_per_seq; /* block table row length (paged: K/V [P][page][Hkv][D]) */
+    int cut_mode;          /* [cut]: 0 or 1 */
 } ocfg_t;
 
 typedef struct {
@@ -190,7 +193,7 @@ void oracle_merge(const double *o1, double m1, double l1, const double *o2, doub
 
 ostate_t *oracle_create(const ocfg_t *cfg) {
     if (!cfg || cfg->Hkv <= 0 || cfg->Hq % cfg->Hkv != 0 || cfg->D <= 0 || (cfg->D & 1) || cfg->W < 0 ||
-        cfg->band < 0 || cfg->B <= 0)
+        cfg->band < 0 || cfg->B <= 0 || cfg->cut_mode < 0 || cfg->cut_mode > 1)
         return NULL;
     ostate_t *s = (ostate_t *)calloc(1, sizeof(ostate_t));
     s->c = *cfg;
@@ -326,8 +329,9 @@ int oracle_step(ostate_t *s, const float *q_pre, const int *rope_pos, const uint
         int p_s = is_hit ? s->wpos[(size_t)u * W + e] : -1;
 
         /* [cut] prefix boundaries. */
-        long c_t = p_t - c->band > 0 ? (long)(p_t - c->band) : 0;
-        long c_s = is_hit ? (p_s - c->band > 0 ? (long)(p_s - c->band) : 0) : 0;
+        const long shift = c->cut_mode;
+        long c_t = p_t - c->band + shift > 0 ? (long)(p_t - c->band + shift) : 0;
+        long c_s = is_hit ? (p_s - c->band + shift > 0 ? (long)(p_s - c->band + shift) : 0) : 0;
         long first_fresh = is_hit ? c_s : 0;
         total_keys += (long)p_t + 1 - first_fresh;
 

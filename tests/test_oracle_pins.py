@@ -116,10 +116,10 @@ def test_hand_worked_example():
 
 
 # ----------------------------------------------------------- whole-step pins
-def _run(wl, steps=None, stream=None, cache=None, tau=None, band=None, rope_zero=False):
+def _run(wl, steps=None, stream=None, cache=None, tau=None, band=None, rope_zero=False, cut_mode=0):
     stream = stream or synth.queries(wl, steps)
     cache = cache or synth.kv_cache(wl, steps)
-    orc = oracle.Oracle.for_workload(wl, cache, tau=tau, band=band)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, cut_mode=cut_mode)
     res = []
     for t in range(stream.q.shape[0]):
         rp = np.zeros_like(stream.rope_pos[t]) if rope_zero else stream.rope_pos[t]
@@ -127,10 +127,12 @@ def _run(wl, steps=None, stream=None, cache=None, tau=None, band=None, rope_zero
     return stream, cache, res
 
 
-def test_forced_miss_equals_dense():
-    """Threshold 0 (strict test) makes every step a miss, i.e. dense attention."""
+@pytest.mark.parametrize("cut_mode", [0, 1])
+def test_forced_miss_equals_dense(cut_mode):
+    """Threshold 0 (strict test) makes every step a miss, i.e. dense attention,
+    wherever the prefix/tail cut falls."""
     wl = _tiny(steps=12)
-    stream, cache, res = _run(wl, tau=0.0)
+    stream, cache, res = _run(wl, tau=0.0, cut_mode=cut_mode)
     for t, r in enumerate(res):
         assert not r.hit.any()
         o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
@@ -162,10 +164,11 @@ def test_exact_repeats_without_rotation_equal_dense():
     assert nhit >= 6
 
 
-def test_band_covering_context_equals_dense():
-    """band >= p_t puts every reuse boundary at 0: hits are exact under any RoPE."""
+@pytest.mark.parametrize("cut_mode", [0, 1])
+def test_band_covering_context_equals_dense(cut_mode):
+    """band >= p_t + 1 puts every reuse boundary at 0: hits are exact under any RoPE."""
     wl = _tiny(L0=(40,), steps=16, band=200)
-    stream, cache, res = _run(wl)
+    stream, cache, res = _run(wl, cut_mode=cut_mode)
     nhit = 0
     for t, r in enumerate(res):
         nhit += int(r.hit.sum())
@@ -191,23 +194,60 @@ def test_hits_differ_from_dense_and_stay_convex():
     assert diff > 1e-6
 
 
-def test_hit_cost_is_constant_in_context_length():
-    """On a hit the keys attended are b + (p_t - p_s) + 1 whatever the context (page 1)."""
+@pytest.mark.parametrize("cut_mode", [0, 1])
+def test_hit_cost_is_constant_in_context_length(cut_mode):
+    """On a hit the keys attended are b + (p_t - p_s) + 1 whatever the context (page 1);
+    one fewer when the band ends at the match position itself (cut_mode 1)."""
     per_L = {}
     for L0 in (256, 4096):
         wl = _tiny(L0=(L0,), steps=20)
-        stream, cache, res = _run(wl)
+        stream, cache, res = _run(wl, cut_mode=cut_mode)
         keys = []
         for t, r in enumerate(res):
             if r.hit[0, 0]:
                 p_t = int(stream.seq_lens[t][0]) - 1
                 p_s = int(r.match_pos[0, 0])
-                assert r.keys_read == wl.band + (p_t - p_s) + 1
+                assert r.keys_read == wl.band + (p_t - p_s) + 1 - cut_mode
                 keys.append(r.keys_read)
             else:
                 assert r.keys_read == int(stream.seq_lens[t][0])
         per_L[L0] = keys
     assert per_L[256] == per_L[4096] and len(per_L[256]) > 3
+
+
+@pytest.mark.parametrize("cut_mode", [0, 1])
+def test_stored_prefix_is_dense_attention_up_to_the_cut(cut_mode):
+    """After a miss the stored state is exact attention of the step's rotated
+    query over keys [0, c), c = max(0, p - b + cut_mode), written as a plain
+    softmax; an empty prefix is (o = 0, m = -inf)."""
+    wl = _tiny(L0=(20,), steps=10, band=24)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=0.0, cut_mode=cut_mode)
+    K, V = decode(cache.K[0, :, 0]), decode(cache.V[0, :, 0])
+    checked = empty = 0
+    for t in range(wl.steps):
+        orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        p = int(stream.seq_lens[t][0]) - 1
+        c = max(0, p - wl.band + cut_mode)
+        q, o, m, l, pos = orc.window(0)
+        assert int(pos[-1]) == p
+        if c == 0:
+            assert np.all(o[-1] == 0.0) and np.all(np.isneginf(m[-1]))
+            empty += 1
+            continue
+        qr = rope_complex(stream.q[t][0].astype(np.float64), int(stream.rope_pos[t][0]), wl.rope_theta)
+        o_ref, lse_ref = dense_attention(qr, K[:c], V[:c])
+        np.testing.assert_allclose(o[-1], o_ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(m[-1] + np.log(l[-1]), lse_ref, rtol=0, atol=1e-12)
+        checked += 1
+    assert checked >= 4 and empty >= 1
+
+
+def test_cut_mode_out_of_range_is_rejected():
+    wl = _tiny(steps=2)
+    with pytest.raises(ValueError):
+        oracle.Oracle.for_workload(wl, synth.kv_cache(wl), cut_mode=2)
 
 
 # ---------------------------------------------------------------- match pins
