@@ -85,6 +85,9 @@ typedef struct MacConfig {
     int max_seq;           /* contiguous: rows per sequence in K/V (capacity); paged: unused */
     int max_pages_per_seq; /* paged: row length of block_table; capacity = max_pages_per_seq * page_size */
     int num_pages;         /* paged: pages P in the K/V pools [P][page_size][Hkv][D] */
+    int cut_mode;          /* where a stored prefix ends, c = max(0, p - band + cut_mode):
+                            * 0 (default) the band is the b keys before the match position,
+                            * 1 it ends at the match position itself; other values MAC_ERR_ARG */
 } MacConfig;
 
 typedef struct MacState MacState; /* opaque; owns device memory on the device current at init */

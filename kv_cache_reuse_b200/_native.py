@@ -48,6 +48,7 @@ class MacConfig(C.Structure):
         ("max_seq", C.c_int),
         ("max_pages_per_seq", C.c_int),
         ("num_pages", C.c_int),
+        ("cut_mode", C.c_int),
     ]
 
 

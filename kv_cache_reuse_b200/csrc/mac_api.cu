@@ -116,7 +116,7 @@ int check_config(const MacConfig* c) {
   if (c->num_q_heads % c->num_kv_heads != 0 || c->num_q_heads / c->num_kv_heads != kGroup) return MAC_ERR_SHAPE;
   if (c->head_dim != 64 && c->head_dim != 128) return MAC_ERR_SHAPE;
   if (c->window < 1 || c->window > kMaxWindow) return MAC_ERR_SHAPE;
-  if (c->band < 0) return MAC_ERR_ARG;
+  if (c->band < 0 || c->cut_mode < 0 || c->cut_mode > 1) return MAC_ERR_ARG;
   if (!(c->rope_theta > 0.0) || isnan(c->tau)) return MAC_ERR_ARG;
   if (c->page_size == 0) {
     if (c->max_seq < 1) return MAC_ERR_ARG;
@@ -379,7 +379,7 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.Hq = s->cfg.num_q_heads;
   p.Hkv = s->cfg.num_kv_heads;
   p.W = s->W;
-  p.band = s->cfg.band;
+  p.band = s->cfg.band - s->cfg.cut_mode;  // c = max(0, p - band + cut_mode)
   p.page_size = s->cfg.page_size;
   p.max_pages = s->cfg.max_pages_per_seq;
   p.num_pages = s->cfg.num_pages;

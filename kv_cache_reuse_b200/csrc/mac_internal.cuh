@@ -94,7 +94,7 @@ struct MatchParams {
   int* claim;              // [grid] ranges taken by the attention CTAs (reset here)
   int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
-  int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;
+  int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
   float tau;
   int grid;       // CTAs of the attention kernel
   int min_keys;   // minimum cost-space units per attention CTA

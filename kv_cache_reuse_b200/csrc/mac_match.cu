@@ -13,7 +13,9 @@
 //      strictly below tau; NaN distances never win;
 //   3. key ranges: the reused prefix ends at c_s = max(0, p_s - band) (the
 //      amend band starts there), the stored prefix of this step ends at
-//      c_t = max(0, p_t - band), and the tail runs to p_t;
+//      c_t = max(0, p_t - band), and the tail runs to p_t (band here is the
+//      configured band minus the cut mode, so that with cut mode 1 the band
+//      ends at the position itself);
 //   4. RoPE of the query to rope_pos (fp64 angle), pre-scaled by
 //      log2(e)/sqrt(D) so the attention kernel works in exp2 units;
 //   5. the query enters the ring slot n mod (W+1) (W+1 slots: the slot

@@ -19,7 +19,7 @@ def torch_dev():
 class GpuRun:
     """One MacState plus device copies of a workload's cache."""
 
-    def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None, tune=None):
+    def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None, tune=None, cut_mode=0):
         import kv_cache_reuse_b200 as mac
         torch, dev = torch_dev()
         self.torch, self.dev, self.wl, self.cache = torch, dev, wl, cache
@@ -28,9 +28,11 @@ class GpuRun:
         self.bt = None if not cache.paged else torch.from_numpy(cache.block_table).to(dev)
         if cache.paged:
             self.st = mac.MacState.for_workload(wl, max_pages_per_seq=cache.block_table.shape[1],
-                                                num_pages=cache.num_pages, tau=tau, band=band, window=window)
+                                                num_pages=cache.num_pages, tau=tau, band=band, window=window,
+                                                cut_mode=cut_mode)
         else:
-            self.st = mac.MacState.for_workload(wl, capacity=cache.max_seq, tau=tau, band=band, window=window)
+            self.st = mac.MacState.for_workload(wl, capacity=cache.max_seq, tau=tau, band=band, window=window,
+                                                cut_mode=cut_mode)
         for name, val in (tune or {}).items():  # work-split knobs: min_keys_per_cta, piece_cost, whole_unit_keys
             getattr(mac, "mac_set_" + name)(self.st, val)
         B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
@@ -55,11 +57,11 @@ class GpuRun:
 
 
 def compare_stream(wl, stream, cache, steps=None, tau=None, band=None, window=None, gpu=None, orc=None,
-                   rope_zero=False, tune=None):
+                   rope_zero=False, tune=None, cut_mode=0):
     """Run both sides over the stream; assert parity at every step.  Returns stats."""
     T = stream.q.shape[0] if steps is None else steps
-    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune)
-    orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window)
+    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune, cut_mode=cut_mode)
+    orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window, cut_mode=cut_mode)
     worst_o = worst_l = 0.0
     hits = 0
     for t in range(T):

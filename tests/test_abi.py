@@ -59,3 +59,18 @@ def test_tuning_setters_reject_bad_handles(lib):
         with pytest.raises(mac.MacError) as e:
             getattr(mac, name)(None, 4)
         assert e.value.code == mac.MAC_ERR_ARG
+
+
+def test_init_rejects_bad_config_before_touching_the_device(lib):
+    """Configuration checks run on the host first: a bad cut mode, band or shape
+    is refused without a GPU."""
+    import kv_cache_reuse_b200 as mac
+    for kw, code in ((dict(cut_mode=2), mac.MAC_ERR_ARG), (dict(cut_mode=-1), mac.MAC_ERR_ARG),
+                     (dict(band=-1), mac.MAC_ERR_ARG), (dict(num_q_heads=24), mac.MAC_ERR_SHAPE),
+                     (dict(head_dim=96), mac.MAC_ERR_SHAPE)):
+        args = dict(batch=1, num_q_heads=32, num_kv_heads=8, head_dim=128, window=8, band=16, tau=0.1,
+                    rope_theta=1e4, max_seq=64)
+        args.update(kw)
+        with pytest.raises(mac.MacError) as e:
+            mac.MacState(**args)
+        assert e.value.code == code, kw

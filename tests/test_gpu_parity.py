@@ -274,6 +274,22 @@ def test_weighted_split_all_miss():
     assert r["hits"] == 0
 
 
+@pytest.mark.parametrize("case", ["tiny", "split", "band0", "llama_paged"])
+def test_cut_mode_band_ends_at_position(case):
+    """cut_mode 1: the stored prefix ends at max(0, p + 1 - band) on both sides."""
+    if case == "tiny":
+        wl, tune = synth.WORKLOADS["tiny"].with_(steps=40), None
+    elif case == "split":  # every range cut over CTAs and merged
+        wl, tune = synth.WORKLOADS["tiny"].with_(steps=40), {"whole_unit_keys": 0, "piece_cost": 0,
+                                                             "min_keys_per_cta": 64}
+    elif case == "band0":  # the prefix covers the current key: an empty tail
+        wl, tune = synth.WORKLOADS["tiny"].with_(steps=24, band=0), None
+    else:
+        wl, tune = synth.WORKLOADS["paged_mixed"].with_(B=3, L0=(3000, 900, 5000), steps=12), None
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tune=tune, cut_mode=1)
+    assert r["hits"] > 0
+
+
 @pytest.mark.parametrize("tune", [
     {"whole_unit_keys": 0},                                           # every range cut over CTAs
     {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 16},  # many tiny pieces per unit
