@@ -190,8 +190,10 @@ def run_mac(args, rank, world, local_rank):
     sptr = s.cuda_stream
     hsz = (B, Hkv)
 
+    qsrc = [q_all]  # the query stream the timed steps read (the hit-path run swaps it)
+
     def ptrs(t):
-        return (q_all[t].data_ptr(), pos_all[t].data_ptr(), lens_all[t].data_ptr(), hit_all[t].data_ptr(),
+        return (qsrc[0][t].data_ptr(), pos_all[t].data_ptr(), lens_all[t].data_ptr(), hit_all[t].data_ptr(),
                 mpos_all[t].data_ptr())
 
     def timed_run(tau, nwarm, nsteps, split):
@@ -258,6 +260,13 @@ def run_mac(args, rank, world, local_rank):
     main = timed_run(wl.tau, args.warmup, args.steps, split=False)
     kern = timed_run(wl.tau, args.warmup, args.steps, split=True)
     allmiss = timed_run(0.0, 3, min(args.miss_steps, T - 3), split=True) if args.miss_steps > 0 else None
+    hitrun = None
+    if args.hit_steps > 0:
+        # the hit path alone: the same shape with every labelled step a near-repeat
+        qh = synth.queries(wl.with_(hit_model=("iid", 1.0)), T).q
+        qsrc[0] = torch.from_numpy(qh).to(dev)
+        hitrun = timed_run(wl.tau, 3, min(args.hit_steps, T - 3), split=True)
+        qsrc[0] = q_all
 
     # max over ranks of the timed duration
     tot = max_over_ranks(main["total_ms"], world, dev)
@@ -308,6 +317,15 @@ def run_mac(args, rank, world, local_rank):
                            "ms_per_step": allmiss["total_ms"] / n, "attend_gbs": a_gbs, "attend_frac": a_gbs / peak,
                            "speedup_of_mac": (world * K_ / (tot * 1e-3)) / (n / (allmiss["total_ms"] * 1e-3)),
                            "clocks": allmiss["clocks"]}
+    if hitrun:
+        n = len(hitrun["step_ms"])
+        h_gbs = hitrun["att_bytes"] / (hitrun["att_ms"] * 1e-3) / 1e9
+        res["hit_path"] = {"steps": n, "hit_fraction": hitrun["hit_frac"],
+                           "steps_per_s": n / (hitrun["total_ms"] * 1e-3), "ms_per_step": hitrun["total_ms"] / n,
+                           "match_ms_per_step": hitrun["match_ms"] / n, "attend_ms_per_step": hitrun["att_ms"] / n,
+                           "attend_bytes_per_step": hitrun["att_bytes"] / n, "attend_gbs": h_gbs,
+                           "attend_frac": h_gbs / peak, "clocks": hitrun["clocks"],
+                           "note": "latency-bound: a few MB per launch"}
     if e2e:
         res["e2e"] = e2e
     if cpu:
@@ -417,6 +435,7 @@ def main():
     ap.add_argument("--impl", default="mac", choices=["mac", "reference"])
     ap.add_argument("--workload", default="long_128k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--miss-steps", type=int, default=16, help="timed steps of the all-miss run (0 = skip)")
+    ap.add_argument("--hit-steps", type=int, default=16, help="timed steps of the all-hit run (0 = skip)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
