@@ -51,6 +51,7 @@ def _load():
             lib.oracle_create.argtypes = [C.POINTER(_Cfg)]
             lib.oracle_free.argtypes = [P]
             lib.oracle_reset.argtypes = [P, C.c_int]
+            lib.oracle_set_tau.argtypes = [P, C.c_double]
             lib.oracle_window.restype = C.c_int
             lib.oracle_window.argtypes = [P, C.c_int, P, P, P, P, P]
             lib.oracle_rope.argtypes = [P, C.c_int, C.c_long, C.c_double, P]
@@ -184,6 +185,19 @@ class Oracle:
             raise ValueError("oracle_match_step rejected its inputs (rc=%d)" % rc)
         sh = (self.B, self.Hkv)
         return hit.reshape(sh), mpos.reshape(sh), db.reshape(sh), ds.reshape(sh)
+
+    def warm_start(self, q_pre, rope_pos, K, V, block_table, seq_lens) -> None:
+        """Seed every window from n prefill positions ([warm] in mac_oracle.c): each
+        sequence's window is emptied, then the n positions run as steps with
+        threshold 0.  q_pre [n][B][Hq][D], rope_pos and seq_lens [n][B]."""
+        for b in range(self.B):
+            self.reset(b)
+        self.lib.oracle_set_tau(self.h, 0.0)
+        try:
+            for j in range(len(q_pre)):
+                self.step(q_pre[j], rope_pos[j], K, V, block_table, seq_lens[j])
+        finally:
+            self.lib.oracle_set_tau(self.h, self.cfg.tau)
 
     def window(self, u: int):
         """(q, o, m, l, pos) of unit u's window, oldest first."""

@@ -34,7 +34,11 @@
  *   [rope]        keys in the cache are post-RoPE; the query is rotated here
  *                 with rotate-half pairs (i, i + D/2), inv_freq_i =
  *                 theta^(-2i/D), angle in fp64;
- *   [scale]       scores are q.k / sqrt(D), natural-log units.
+ *   [scale]       scores are q.k / sqrt(D), natural-log units;
+ *   [warm]        a window seeded from prefill holds, for each of the last n
+ *                 prefill positions, its pre-RoPE query and its prefix state
+ *                 over [0, c) with the query rotated at that position -- the
+ *                 state a decode step at that position would have stored.
  *
  * Arithmetic is fp64 throughout; inputs are fp32 queries and bf16 keys and
  * values, read exactly.
@@ -219,6 +223,12 @@ void oracle_free(ostate_t *s) {
 void oracle_reset(ostate_t *s, int b) {
     for (int kvh = 0; kvh < s->c.Hkv; ++kvh) s->n[b * s->c.Hkv + kvh] = 0;
 }
+
+/* Replace the match threshold.  A warm start from prefill runs its positions
+ * as steps with threshold 0: every one misses and stores (q, prefix state,
+ * position), i.e. the window is seeded with the prefill queries and their
+ * prefix states over [0, c) ([warm]). */
+void oracle_set_tau(ostate_t *s, double tau) { s->c.tau = tau; }
 
 /* Copy out the window of unit u = b * Hkv + kvh, oldest entry first. */
 int oracle_window(const ostate_t *s, int u, float *q, double *o, double *m, double *l, int *pos) {

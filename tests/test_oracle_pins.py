@@ -250,6 +250,55 @@ def test_cut_mode_out_of_range_is_rejected():
         oracle.Oracle.for_workload(wl, synth.kv_cache(wl), cut_mode=2)
 
 
+def test_warm_start_stores_prefill_queries_and_prefix_states():
+    """A window seeded from n prefill positions holds each position's own query,
+    its position, and exact attention of its rotated query over [0, c) (plain
+    softmax), oldest first; the window is emptied first."""
+    wl = _tiny(L0=(60,), steps=8, band=24)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    orc.step(stream.q[0], stream.rope_pos[0], cache.K, cache.V, None, stream.seq_lens[0])  # to be discarded
+    n = 5
+    orc.warm_start(stream.q[1:1 + n], stream.rope_pos[1:1 + n], cache.K, cache.V, None, stream.seq_lens[1:1 + n])
+    q, o, m, l, pos = orc.window(0)
+    assert len(pos) == n
+    K, V = decode(cache.K[0, :, 0]), decode(cache.V[0, :, 0])
+    for j in range(n):
+        t = 1 + j
+        p = int(stream.seq_lens[t][0]) - 1
+        assert int(pos[j]) == p
+        np.testing.assert_array_equal(q[j], stream.q[t][0])
+        c = max(0, p - wl.band)
+        qr = rope_complex(stream.q[t][0].astype(np.float64), int(stream.rope_pos[t][0]), wl.rope_theta)
+        o_ref, lse_ref = dense_attention(qr, K[:c], V[:c])
+        np.testing.assert_allclose(o[j], o_ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(m[j] + np.log(l[j]), lse_ref, rtol=0, atol=1e-12)
+
+
+def test_warm_start_lets_the_first_decode_step_hit():
+    """Without a seeded window the first decode step always misses; after a warm
+    start an exact repeat of a prefill query (identity RoPE) hits it, and the
+    output then equals dense attention."""
+    wl = _tiny(L0=(80,), steps=6, sigma=0.0)
+    stream = synth.queries(wl, sigma=0.0)
+    cache = synth.kv_cache(wl)
+    n = 4
+    zero = np.zeros((n, wl.B), np.int32)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    orc.warm_start(stream.q[:n], zero, cache.K, cache.V, None, stream.seq_lens[:n])
+    t = n
+    q = stream.q[1].copy()  # repeat of a seeded prefill query
+    r = orc.step(q, np.zeros(wl.B, np.int32), cache.K, cache.V, None, stream.seq_lens[t])
+    assert bool(r.hit[0, 0]) and int(r.match_pos[0, 0]) == int(stream.seq_lens[1][0]) - 1
+    o, lse = dense_step(wl, cache, q, np.zeros(wl.B, np.int32), stream.seq_lens[t])
+    np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r.lse, lse, rtol=0, atol=1e-12)
+    fresh = oracle.Oracle.for_workload(wl, cache)
+    r0 = fresh.step(q, np.zeros(wl.B, np.int32), cache.K, cache.V, None, stream.seq_lens[t])
+    assert not r0.hit.any()
+
+
 # ---------------------------------------------------------------- match pins
 def _brute_match(window, q, tau, G):
     """numpy brute force: mean-over-heads squared L2, argmin, ties to later, strict < tau."""
