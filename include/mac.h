@@ -148,6 +148,25 @@ int mac_attend(MacState *st, const uint16_t *K, const uint16_t *V, const int *bl
 int mac_append_kv(MacState *st, uint16_t *K, uint16_t *V, const int *block_table,
                   const int *seq_lens, const uint16_t *k_new, const uint16_t *v_new, void *stream);
 
+/* Seed every sequence's window from its last n prefill positions (0 <= n <=
+ * window), so that the first decode steps can already hit.  Each window is
+ * emptied, then position j (oldest first) is stored as a decode step at that
+ * position would store it: its pre-RoPE query and its prefix state over keys
+ * [0, c), c = max(0, p - band + cut_mode), computed here from the cache with
+ * the query rotated at rope_pos (the window of recent queries on the
+ * MAC-Attention page, filled before decoding instead of by the first W
+ * decode steps).  Cost: n dense passes over each prefix.
+ *   q_pre     device fp32 [n][B][Hq][D] pre-RoPE queries of the positions.
+ *   rope_pos  device int32 [n][B].
+ *   K, V, block_table  the cache, as in mac_decode_step; keys [0, p] of every
+ *             position must be in it.
+ *   seq_lens  device int32 [n][B]: p + 1 of each position.
+ * Enqueued on stream; uses the state's scratch (do not overlap with
+ * mac_decode_step_host on the same state).  MAC_ERR_ARG for n outside
+ * [0, window] or missing pointers. */
+int mac_warm_start(MacState *st, int n, const float *q_pre, const int *rope_pos, const uint16_t *K,
+                   const uint16_t *V, const int *block_table, const int *seq_lens, void *stream);
+
 /* mac_append_kv (when k_new_h is not NULL) and mac_decode_step with the
  * per-step inputs and outputs in HOST memory: copies q_pre_h, rope_pos_h,
  * seq_lens_h and the new rows to library staging buffers, runs the step,

@@ -19,7 +19,7 @@ from ._native import (MAC_DEV_BAD_PAGE, MAC_DEV_BAD_SEQ_LEN, MAC_DEV_TIMEOUT, MA
 __all__ = [
     "MacConfig", "MacError", "MacState", "mac_init_state", "mac_destroy", "mac_reset_seq", "mac_decode_step",
     "mac_match", "mac_attend", "mac_append_kv", "mac_decode_step_host", "mac_get_status", "mac_state_bytes",
-    "mac_export_state", "mac_import_state", "mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_set_whole_unit_keys", "mac_attend_grid", "mac_error_string", "mac_dense_decode_static",
+    "mac_export_state", "mac_import_state", "mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_set_whole_unit_keys", "mac_warm_start", "mac_attend_grid", "mac_error_string", "mac_dense_decode_static",
     "MAC_OK", "MAC_ERR_ARG", "MAC_ERR_SHAPE", "MAC_ERR_CUDA", "MAC_ERR_OOM", "MAC_ERR_DEVICE",
     "MAC_DEV_BAD_SEQ_LEN", "MAC_DEV_BAD_PAGE", "MAC_DEV_TIMEOUT", "LIB_PATH",
 ]
@@ -195,6 +195,11 @@ def mac_set_min_keys_per_cta(st, keys: int) -> None:
 
 def mac_set_piece_cost(st, keys: int) -> None:
     check("mac_set_piece_cost", load().mac_set_piece_cost(_h(st), int(keys)))
+
+
+def mac_warm_start(st, n: int, q_pre, rope_pos, K, V, block_table, seq_lens, stream=None) -> None:
+    check("mac_warm_start", load().mac_warm_start(_h(st), int(n), _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V),
+                                                 _ptr(block_table), _ptr(seq_lens), _stream(stream)))
 
 
 def mac_set_whole_unit_keys(st, keys: int) -> None:

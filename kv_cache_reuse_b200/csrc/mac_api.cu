@@ -347,8 +347,17 @@ int mac_set_whole_unit_keys(MacState* s, int keys) {
 
 int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
 
+static int match_impl(MacState* s, float tau, const float* q_pre, const int* rope_pos, const int* block_table,
+                      const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream);
+
 int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
               float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
+  if (!s) return MAC_ERR_ARG;
+  return match_impl(s, s->cfg.tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream);
+}
+
+static int match_impl(MacState* s, float tau, const float* q_pre, const int* rope_pos, const int* block_table,
+                      const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
   if (!s || !q_pre || !rope_pos || !seq_lens || !out || !lse) return MAC_ERR_ARG;
   if (!aligned16(q_pre)) return MAC_ERR_ARG;
   if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
@@ -384,7 +393,7 @@ int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* b
   p.max_pages = s->cfg.max_pages_per_seq;
   p.num_pages = s->cfg.num_pages;
   p.capacity = s->capacity;
-  p.tau = s->cfg.tau;
+  p.tau = tau;
   p.grid = s->grid;
   p.min_keys = s->min_keys;
   p.piece_cost = s->piece_cost;
@@ -470,6 +479,28 @@ int mac_append_kv(MacState* s, uint16_t* K, uint16_t* V, const int* block_table,
   p.num_pages = s->cfg.num_pages;
   p.capacity = s->capacity;
   return launch_append(p, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+}
+
+int mac_warm_start(MacState* s, int n, const float* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
+                   const int* block_table, const int* seq_lens, void* stream) {
+  if (!s || n < 0 || n > s->W) return MAC_ERR_ARG;
+  if (n > 0 && (!q_pre || !rope_pos || !seq_lens || !K || !V)) return MAC_ERR_ARG;
+  if (n > 0 && (!aligned16(q_pre) || !aligned16(K) || !aligned16(V))) return MAC_ERR_ARG;
+  if (s->cfg.page_size > 0 && n > 0 && !block_table) return MAC_ERR_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  // every window starts empty, then each position runs as a step with threshold 0
+  if (cudaMemsetAsync(s->steps, 0, (size_t)s->U * sizeof(int), st) != cudaSuccess) return MAC_ERR_CUDA;
+  const size_t B = s->cfg.batch, Hq = s->cfg.num_q_heads, D = s->D;
+  float* out = reinterpret_cast<float*>(s->dev_out + s->off_out);  // outputs of these steps are not kept
+  float* lse = reinterpret_cast<float*>(s->dev_out + s->off_lse);
+  for (int j = 0; j < n; ++j) {
+    int rc = match_impl(s, 0.f, q_pre + (size_t)j * B * Hq * D, rope_pos + (size_t)j * B, block_table,
+                        seq_lens + (size_t)j * B, out, lse, nullptr, nullptr, stream);
+    if (rc != MAC_OK) return rc;
+    rc = mac_attend(s, K, V, block_table, out, lse, stream);
+    if (rc != MAC_OK) return rc;
+  }
+  return MAC_OK;
 }
 
 // Enqueue one host step on `st`: copy the packed inputs in, append the new

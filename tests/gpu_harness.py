@@ -57,14 +57,14 @@ class GpuRun:
 
 
 def compare_stream(wl, stream, cache, steps=None, tau=None, band=None, window=None, gpu=None, orc=None,
-                   rope_zero=False, tune=None, cut_mode=0):
+                   rope_zero=False, tune=None, cut_mode=0, start=0):
     """Run both sides over the stream; assert parity at every step.  Returns stats."""
     T = stream.q.shape[0] if steps is None else steps
     gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune, cut_mode=cut_mode)
     orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window, cut_mode=cut_mode)
     worst_o = worst_l = 0.0
     hits = 0
-    for t in range(T):
+    for t in range(start, T):
         rp = np.zeros_like(stream.rope_pos[t]) if rope_zero else stream.rope_pos[t]
         r = orc.step(stream.q[t], rp, cache.K, cache.V, cache.block_table, stream.seq_lens[t])
         out, lse, hit, mpos = gpu.step(stream.q[t], rp, stream.seq_lens[t])

@@ -290,6 +290,40 @@ def test_cut_mode_band_ends_at_position(case):
     assert r["hits"] > 0
 
 
+@pytest.mark.parametrize("case", ["tiny", "paged"])
+def test_warm_start_from_prefill_then_decode(case):
+    """Windows seeded from the first n positions of the stream (as prefill
+    positions), then decoding: decisions bit-exact and outputs within tolerance
+    of the oracle doing the same, and the seeded ring equal to its window."""
+    import kv_cache_reuse_b200 as mac
+    if case == "tiny":
+        wl, n = synth.WORKLOADS["tiny"].with_(steps=40), 16
+    else:
+        wl, n = synth.WORKLOADS["paged_mixed"].with_(B=3, L0=(3000, 900, 5000), steps=20), 8
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    gpu = GpuRun(wl, cache)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    torch = gpu.torch
+    qn = torch.from_numpy(np.ascontiguousarray(stream.q[:n])).to(gpu.dev)
+    pn = torch.from_numpy(np.ascontiguousarray(stream.rope_pos[:n])).to(gpu.dev)
+    ln = torch.from_numpy(np.ascontiguousarray(stream.seq_lens[:n])).to(gpu.dev)
+    mac.mac_warm_start(gpu.st, n, qn, pn, gpu.K, gpu.V, gpu.bt, ln)
+    orc.warm_start(stream.q[:n], stream.rope_pos[:n], cache.K, cache.V, cache.block_table, stream.seq_lens[:n])
+    torch.cuda.synchronize()
+    st = mac.parse_state(gpu.st.export_state(), wl.W, wl.G, wl.D)
+    W1 = wl.W + 1
+    for u in range(wl.B * wl.Hkv):
+        assert int(st["steps"][u]) == n
+        q_o, o_o, m_o, l_o, pos_o = orc.window(u)
+        for j in range(n):
+            slot = j % W1
+            assert st["pos"][u, slot] == pos_o[j]
+            np.testing.assert_array_equal(st["q"][u, slot], q_o[j])
+            np.testing.assert_allclose(st["o"][u, slot], o_o[j], atol=OUT_TOL)
+    r = compare_stream(wl, stream, cache, gpu=gpu, orc=orc, start=n)
+    assert r["hits"] > 0
+
+
 @pytest.mark.parametrize("tune", [
     {"whole_unit_keys": 0},                                           # every range cut over CTAs
     {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 16},  # many tiny pieces per unit
