@@ -79,5 +79,5 @@ def test_init_rejects_bad_config_before_touching_the_device(lib):
 def test_warm_start_rejects_bad_arguments(lib):
     import kv_cache_reuse_b200 as mac
     with pytest.raises(mac.MacError) as e:
-        mac.mac_warm_start(None, 1, 16, 16, 16, 16, None, 16)
+        mac.mac_warm_start(None, 1, 16, 16, 16, 16, None, 16, stream=0)
     assert e.value.code == mac.MAC_ERR_ARG
