@@ -260,6 +260,26 @@ def run_mac(args, rank, world, local_rank):
     main = timed_run(wl.tau, args.warmup, args.steps, split=False)
     kern = timed_run(wl.tau, args.warmup, args.steps, split=True)
     allmiss = timed_run(0.0, 3, min(args.miss_steps, T - 3), split=True) if args.miss_steps > 0 else None
+    warm = None
+    if args.warm_start:
+        # seed the windows from the first W positions of the stream (as prefill
+        # positions): W threshold-0 steps over the whole prefix of every unit
+        n = min(wl.W, T)
+        st = mac.MacState.for_workload(wl, **kw)
+        args_w = (n, q_all[:n].contiguous(), pos_all[:n].contiguous(), K, V, bt, lens_all[:n].contiguous())
+        mac.mac_warm_start(st, *args_w, stream=s)  # warm-up
+        flush.zero_()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        mac.mac_warm_start(st, *args_w, stream=s)
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        wms = e0.elapsed_time(e1)
+        wbytes = sum(int(stream.seq_lens[j][b]) * 2 * wl.D * 2 * wl.Hkv for j in range(n) for b in range(wl.B))
+        warm = {"positions": n, "ms": wms, "kv_bytes": wbytes, "gbs": wbytes / (wms * 1e-3) / 1e9,
+                "frac": wbytes / (wms * 1e-3) / 1e9 / peak, "device_status": st.get_status()}
+        st.close()
     hitrun = None
     if args.hit_steps > 0:
         # the hit path alone: the same shape with every labelled step a near-repeat
@@ -326,6 +346,8 @@ def run_mac(args, rank, world, local_rank):
                            "attend_bytes_per_step": hitrun["att_bytes"] / n, "attend_gbs": h_gbs,
                            "attend_frac": h_gbs / peak, "clocks": hitrun["clocks"],
                            "note": "latency-bound: a few MB per launch"}
+    if warm:
+        res["warm_start"] = warm
     if e2e:
         res["e2e"] = e2e
     if cpu:
@@ -436,6 +458,7 @@ def main():
     ap.add_argument("--workload", default="long_128k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--miss-steps", type=int, default=16, help="timed steps of the all-miss run (0 = skip)")
     ap.add_argument("--hit-steps", type=int, default=16, help="timed steps of the all-hit run (0 = skip)")
+    ap.add_argument("--warm-start", action="store_true", help="also time seeding the windows from W positions")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
