@@ -30,10 +30,12 @@ struct MacState {
   // scratch
   float* qrot = nullptr;
   UnitPlan* plan = nullptr;
-  WorkItem* spill = nullptr;    // [grid][2U] each attention CTA's work items
+  Segment* seg = nullptr;
+  PlanHeader* hdr = nullptr;
+  int* first_seg = nullptr;
   float* rate = nullptr;        // learned streaming rate per SM (weighted split)
-  double* cw = nullptr;         // cumulative range shares of this step's weighted split
-  double* cw_next = nullptr;    // the same, for the next weighted step
+  long long* bounds = nullptr;  // range starts of a weighted split
+  double* cw = nullptr;         // cumulative range shares of the next weighted split
   int* claim = nullptr;         // ranges taken by the attention CTAs
   float* part = nullptr;
   int* unit_cnt = nullptr;
@@ -97,7 +99,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,
-                  s->spill,  s->rate,   s->cw,     s->cw_next, s->claim, s->part, s->unit_cnt, s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -240,13 +242,16 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->steps, U));
   A(alloc(&s->qrot, U * G * D));
   A(alloc(&s->plan, U));
-  A(alloc(&s->spill, (size_t)s->grid * 2 * U));
+  A(alloc(&s->seg, 2 * U));
+  A(alloc(&s->hdr, 1));
+  A(alloc(&s->first_seg, (size_t)s->grid));
   A(alloc(&s->rate, (size_t)s->grid));
+  A(alloc(&s->bounds, (size_t)s->grid + 1));
   A(alloc(&s->cw, (size_t)s->grid + 1));
-  A(alloc(&s->cw_next, (size_t)s->grid + 1));
   A(alloc(&s->claim, (size_t)s->grid));
   A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
   A(alloc(&s->unit_cnt, U));
+  A(alloc(&s->done, 1));
   A(alloc(&s->inv_freq, D / 2));
   s->off_q = 0;
   s->off_pos = up256(s->off_q + B * Hq * D * sizeof(float));
@@ -279,16 +284,17 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->ring_pos, 0, U * W1 * sizeof(int)));
   A(cudaMemset(s->steps, 0, U * sizeof(int)));
   A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
+  A(cudaMemset(s->done, 0, sizeof(int)));
   A(cudaMemset(s->rate, 0, s->grid * sizeof(float)));
   A(cudaMemset(s->claim, 0, s->grid * sizeof(int)));
   {  // even shares until the first rates are measured
     double* cw = (double*)malloc(sizeof(double) * (s->grid + 1));
     for (int c = 0; c <= s->grid; ++c) cw[c] = (double)c / s->grid;
     A(cudaMemcpy(s->cw, cw, sizeof(double) * (s->grid + 1), cudaMemcpyHostToDevice));
-    A(cudaMemcpy(s->cw_next, cw, sizeof(double) * (s->grid + 1), cudaMemcpyHostToDevice));
     free(cw);
   }
   A(cudaMemset(s->dev_out, 0, s->out_bytes));
+  A(cudaMemset(s->hdr, 0, sizeof(PlanHeader)));
   double* inv = (double*)malloc(sizeof(double) * (D / 2));
   for (size_t i = 0; i < D / 2; ++i) inv[i] = pow(cfg->rope_theta, -2.0 * (double)i / (double)D);
   A(cudaMemcpy(s->inv_freq, inv, sizeof(double) * (D / 2), cudaMemcpyHostToDevice));
@@ -370,9 +376,13 @@ static int match_impl(MacState* s, float tau, const float* q_pre, const int* rop
   p.inv_freq = s->inv_freq;
   p.qrot = s->qrot;
   p.plan = s->plan;
-  p.cw_next = s->cw_next;
+  p.seg = s->seg;
+  p.hdr = s->hdr;
+  p.first_seg = s->first_seg;
   p.cw = s->cw;
+  p.bounds = s->bounds;
   p.claim = s->claim;
+  p.done = s->done;
   p.status = s->status;
   p.B = s->cfg.batch;
   p.Hq = s->cfg.num_q_heads;
@@ -385,6 +395,9 @@ static int match_impl(MacState* s, float tau, const float* q_pre, const int* rop
   p.capacity = s->capacity;
   p.tau = tau;
   p.grid = s->grid;
+  p.min_keys = s->min_keys;
+  p.piece_cost = s->piece_cost;
+  p.unit_max = s->unit_max;
   return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
@@ -409,11 +422,13 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
   p.qrot = s->qrot;
   p.plan = s->plan;
-  p.cw = s->cw;
-  p.cw_next = s->cw_next;
+  p.seg = s->seg;
+  p.hdr = s->hdr;
+  p.first_seg = s->first_seg;
+  p.bounds = s->bounds;
   p.claim = s->claim;
   p.rate = s->rate;
-  p.spill = s->spill;
+  p.cw = s->cw;
   p.part = s->part;
   p.unit_cnt = s->unit_cnt;
   p.ring_o = s->ring_o;
@@ -430,9 +445,6 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.max_pages = s->cfg.max_pages_per_seq;
   p.nseg = 2 * s->U;
   p.grid = s->grid;
-  p.min_keys = s->min_keys;
-  p.piece_cost = s->piece_cost;
-  p.unit_max = s->unit_max;
   return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 

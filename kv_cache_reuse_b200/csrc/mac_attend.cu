@@ -86,10 +86,7 @@ struct __align__(1024) AttnSmem {
   int abort_flag;
   int last_flag;
   int box_total;                     // boxes consumed by all warps (rate record)
-  WorkItem items[kItemCache];        // the CTA's work items, from its first one on
-  long long sbound[kAttnThreads];    // range starts of a weighted split
-  long long sscan[kConsumerWarps];   // block scans of the split
-  int first_item;                    // the CTA's first work item
+  Segment items[kItemCache];         // the CTA's work items, from its first one on
   alignas(16) float ring[Cfg<D>::GD + 2 * kGroup];  // that ring state: o [G][D], m [G], l [G]
 };
 
@@ -337,21 +334,21 @@ __device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, 
 // 1 stages every partial's (m, l) in shared memory with one round of
 // independent loads; phase 2 weighs the partial outputs, all loads in flight.
 template <int D>
-__device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, int pbA, int nA, int pbB, int nB,
-                           uint32_t& sync_phase) {
+__device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
   constexpr int kCap = (kConsumerWarps * Cfg<D>::WB) / (2 * G);  // pieces whose (m, l) fit in wbuf
   const UnitPlan pl = p.plan[u];
+  const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
-  const int n = nA + nB;
+  const int nA = sA.npieces, n = sA.npieces + sB.npieces;
   float* mm = &sm.wbuf[0][0];  // [piece][G] maxima, then [piece][G] sums
   float* ll = mm + kCap * G;
   const bool staged = n <= kCap;
   if (staged) {
     for (int t = threadIdx.x; t < n * G; t += kConsumerWarps * 32) {
       const int i = t / G, h = t - i * G;
-      const int slot = i < nA ? pbA + i : pbB + (i - nA);
+      const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
       const float* pp = p.part + (size_t)slot * PF;
       mm[t] = __ldcg(pp + GD + h);
       ll[t] = __ldcg(pp + GD + G + h);
@@ -360,12 +357,12 @@ __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, int pb
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   auto pm = [&](int i, int h) -> float {
     if (staged) return mm[i * G + h];
-    const int slot = i < nA ? pbA + i : pbB + (i - nA);
+    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
     return __ldcg(p.part + (size_t)slot * PF + GD + h);
   };
   auto pl_ = [&](int i, int h) -> float {
     if (staged) return ll[i * G + h];
-    const int slot = i < nA ? pbA + i : pbB + (i - nA);
+    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
     return __ldcg(p.part + (size_t)slot * PF + GD + G + h);
   };
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
@@ -391,7 +388,7 @@ __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, int pb
       float v[16];
 #pragma unroll
       for (int k = 0; k < 16; ++k)
-        v[k] = i0 + k < nA ? __ldcg(p.part + (size_t)(pbA + i0 + k) * PF + idx) : 0.f;
+        v[k] = i0 + k < nA ? __ldcg(p.part + (size_t)(sA.pbase + i0 + k) * PF + idx) : 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         if (i0 + k < nA) {
@@ -417,7 +414,7 @@ __device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, int pb
       float v[16];
 #pragma unroll
       for (int k = 0; k < 16; ++k)
-        v[k] = i0 + k < n ? __ldcg(p.part + (size_t)(pbB + (i0 + k - nA)) * PF + idx) : 0.f;
+        v[k] = i0 + k < n ? __ldcg(p.part + (size_t)(sB.pbase + (i0 + k - nA)) * PF + idx) : 0.f;
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         if (i0 + k < n) {
@@ -510,24 +507,11 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, in
   }
 }
 
-// The CTA's pieces, walked in order by every lane of every warp.  A split
-// piece is part of one segment of a large unit; a whole-unit piece holds
-// both segments of a small unit: A = [a0, a1) (may be empty), B = [k0, k1).
-struct Piece {
-  int unit, pidx, whole;
-  int pbA, npA, pbB, npB;     // split: the unit's partial slots and counts (its merge)
-  int hit, src, dst;          // whole unit: plan of the unit (end = k1)
-  int k0, k1, kb0, nbox;      // split: its keys; whole unit: segment B
-  int a0, a1, akb0, anbox;    // whole unit: segment A
-  int wA;                     // whole unit: warps on segment A
-};
-
 // End of a split piece: combine the 8 warps, write the partial, count it
 // and, if it was the unit's last, merge the unit.
 template <int D>
-__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, const Piece& pc,
+__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int unit, int pidx,
                                uint32_t& sync_phase) {
-  const int unit = pc.unit, pidx = pc.pidx;
   constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
   warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
@@ -548,12 +532,12 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
   if (threadIdx.x == 0) {
     __threadfence();
     const int old = atomicAdd(p.unit_cnt + unit, 1);
-    sm.last_flag = (old == pc.npA + pc.npB - 1);
+    sm.last_flag = (old == p.plan[unit].expected - 1);
   }
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
-    return merge_unit<D>(p, sm, unit, pc.pbA, pc.npA, pc.pbB, pc.npB, sync_phase);
+    return merge_unit<D>(p, sm, unit, sync_phase);
   }
   return true;
 }
@@ -610,6 +594,16 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
   return consumer_sync(sm, sync_phase, p.status);
 }
 
+// The CTA's pieces, walked in order by every lane of every warp.  A split
+// piece is part of one segment of a large unit; a whole-unit piece holds
+// both segments of a small unit: A = [a0, a1) (may be empty), B = [k0, k1).
+struct Piece {
+  int unit, pidx, whole;
+  int hit, src, dst;          // whole unit: plan of the unit (end = k1)
+  int k0, k1, kb0, nbox;      // split: its keys; whole unit: segment B
+  int a0, a1, akb0, anbox;    // whole unit: segment A
+  int wA;                     // whole unit: warps on segment A
+};
 // The boxes one warp takes from a piece: indices first, first + stride, ...
 struct WarpRange {
   int kb0, k0, k1, nbox, first, stride;
@@ -641,12 +635,11 @@ __device__ __forceinline__ int box_count(int k0, int k1) {
 struct Walker {
   int s;
   long long lo, hi;
-  const WorkItem* cache;  // shared-memory copy of items [base, base + kItemCache)
+  const Segment* cache;  // shared-memory copy of items [base, base + kItemCache)
   int base;
-  const WorkItem* spill;  // this CTA's copy of every item (read beyond the cache)
   __device__ __forceinline__ bool next(const AttendParams& p, int cta, Piece& pc) {
     while (s < p.nseg) {
-      const WorkItem sg = (s - base < kItemCache) ? cache[s - base] : spill[s];
+      const Segment sg = (s - base < kItemCache) ? cache[s - base] : p.seg[s];
       const int cur = s++;
       if (sg.kind < 0) continue;
       if (sg.flat >= hi) {  // this and every later item start past the range
@@ -686,10 +679,6 @@ struct Walker {
       pc.wA = 0;
       pc.anbox = 0;
       pc.pidx = sg.pbase + (cta - sg.first_cta);
-      pc.pbA = sg.pbA;
-      pc.npA = sg.npA;
-      pc.pbB = sg.pbB;
-      pc.npB = sg.npB;
       pc.k0 = sg.key0 + (int)(fa - sg.flat);
       pc.k1 = sg.key0 + (int)(fe - sg.flat);
       pc.kb0 = pc.k0 & ~(kSubKeys - 1);
@@ -736,218 +725,8 @@ __device__ __noinline__ void rate_shares(const AttendParams& p) {
     if (k < warp) before += red[k];
     all += red[k];
   }
-  if (tid < G) p.cw_next[tid] = (double)(before + x - wi) / (double)all;
-  if (tid == 0) p.cw_next[G] = 1.0;
-}
-
-// ---------------------------------------------------------------- the split
-// Exclusive prefix sum of v over the block's 256 threads (every thread gets
-// the total); sbuf holds kConsumerWarps values.
-__device__ long long block_exclusive_scan(long long v, long long* total, long long* sbuf) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  long long x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sbuf[warp] = x;
-  __syncthreads();
-  long long before = 0, all = 0;
-#pragma unroll
-  for (int w = 0; w < kConsumerWarps; ++w) {
-    const long long t = sbuf[w];
-    before += w < warp ? t : 0;
-    all += t;
-  }
-  __syncthreads();
-  *total = all;
-  return before + x - v;
-}
-
-// floor(a / b) and ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit
-// integer division: an fp64 estimate (off by at most a few units) corrected
-// exactly.
-__device__ __forceinline__ long long floor_div(long long a, long long b, double rb) {
-  long long q = (long long)((double)a * rb);
-  while (q > 0 && q * b > a) --q;
-  while ((q + 1) * b <= a) ++q;
-  return q;
-}
-__device__ __forceinline__ long long ceil_div(long long a, long long b, double rb) {
-  const long long q = floor_div(a, b, rb);
-  return q + (q * b < a ? 1 : 0);
-}
-
-// The work item in slot s, from its unit's plan.
-struct ItemDesc {
-  int kind, len, key0, cut, packed;
-};
-__device__ __forceinline__ ItemDesc item_of(const AttendParams& p, int s) {
-  ItemDesc it{kItemEmpty, 0, 0, 0, 0};
-  const UnitPlan* pl = p.plan + (s >> 1);
-  if (pl->bad) return it;
-  const int start = pl->start, c = pl->cut, end = pl->end;
-  if (end - start <= p.unit_max) {
-    if ((s & 1) == 0) {  // the whole unit in slot 2u
-      it.kind = kItemWhole;
-      it.len = end - start;
-      it.key0 = start;
-      it.cut = c;
-      // the CTA doing it also needs hit, reused slot and written slot
-      const int hit = pl->hit;
-      it.packed = (hit ? 1 : 0) | ((hit ? pl->src_slot : 0) << 1) | (pl->dst_slot << 12);
-    }
-  } else {
-    it.len = (s & 1) ? end - c : c - start;
-    it.key0 = (s & 1) ? c : start;
-    it.kind = it.len > 0 ? ((s & 1) ? kItemB : kItemA) : kItemEmpty;
-  }
-  return it;
-}
-
-struct SplitOut {
-  long long lo, hi;  // the CTA's range of the cost space
-  int slot;          // its index among the ranges (-1: no range)
-  int first;         // its first work item
-  int weighted;
-};
-
-// Every CTA lays the units' items end to end in the cost space (each
-// non-empty item weighs piece_cost + its keys), splits the space over
-// n = min(grid, ceil(T / min_keys)) ranges -- evenly, or by the learned SM
-// shares cw[] on large steps -- and numbers the partial results, all from
-// the plans, so every CTA reaches the same split.  It keeps the items from
-// the one whose extent holds its range start on: the first kItemCache in
-// shared memory, all of them in its slice of p.spill.  Thread 0 of a CTA on
-// SM smid has claimed range smid (mine) before the call.  A dry call (made
-// while the match kernel still runs, on whatever plans memory holds) only
-// brings this code on chip: it claims nothing and writes no global memory.
-template <int D>
-__device__ __noinline__ SplitOut build_split(const AttendParams& p, AttnSmem<D>& sm, int mine, unsigned smid,
-                                             bool dry) {
-  const int tid = threadIdx.x;
-  const int nseg = p.nseg;
-  const long long cost = p.piece_cost;
-  const bool regs = nseg <= kAttnThreads;  // one item per thread, kept in registers
-  long long* sbuf = sm.sscan;
-  const double cw_c = (p.cw != nullptr && tid <= p.grid) ? __ldcg(p.cw + tid) : 0.0;
-  // pass 1: items and cost offsets
-  ItemDesc r_it{kItemEmpty, 0, 0, 0, 0};
-  long long r_flat = 0, carry = 0;
-  for (int base = 0; base < nseg; base += kAttnThreads) {
-    const int s = base + tid;
-    const ItemDesc it = s < nseg ? item_of(p, s) : ItemDesc{kItemEmpty, 0, 0, 0, 0};
-    const bool split = it.kind == kItemA || it.kind == kItemB;
-    long long tot;
-    const long long ex = block_exclusive_scan(it.kind != kItemEmpty ? (long long)it.len + cost : 0, &tot, sbuf);
-    if (regs) {
-      r_it = it;
-      r_flat = ex + (split ? cost : 0);
-    }
-    carry += tot;
-  }
-  const long long T = carry;
-  int N = 0;
-  if (T > 0) {
-    const long long want = (T + p.min_keys - 1) / p.min_keys;
-    N = (int)(want < (long long)p.grid ? want : (long long)p.grid);
-  }
-  if (dry && N < 1) N = 1;
-  const double rT = T > 0 ? 1.0 / (double)T : 0.0;
-  const bool weighted =
-      p.cw != nullptr && N == p.grid && p.grid < kAttnThreads && T >= kWeightMinCost * (long long)p.grid;
-  if (weighted && tid <= N) sm.sbound[tid] = tid == 0 ? 0 : (tid == N ? T : (long long)((double)T * cw_c));
-  if (tid == 0) {
-    int c = (int)blockIdx.x < N ? (int)blockIdx.x : (dry ? 0 : -1);
-    if (weighted && !dry) {  // this SM's range, else the first free one
-      c = mine ? (int)smid : -1;
-      for (int k = 0; c < 0 && k < N; ++k)
-        if (atomicCAS(p.claim + k, 0, 1) == 0) c = k;
-    }
-    sm.last_flag = c;
-    sm.first_item = nseg;
-  }
-  __syncthreads();
-  SplitOut out{0, 0, sm.last_flag, nseg, weighted ? 1 : 0};
-  if (out.slot < 0) return out;
-  const int slot = out.slot;
-  out.lo = weighted ? sm.sbound[slot] : (long long)slot * T / N;
-  out.hi = weighted ? sm.sbound[slot + 1] : (long long)(slot + 1) * T / N;
-  // range holding offset x: the largest c with start(c) <= x (weighted: from
-  // the even split's guess, walked to the exact range)
-  auto owner = [&](long long x) -> int {
-    if (!weighted) return (int)ceil_div((x + 1) * (long long)N, T, rT) - 1;
-    int c = (int)((double)x * N * rT);
-    c = c < 0 ? 0 : (c > N - 1 ? N - 1 : c);
-    while (c > 0 && sm.sbound[c] > x) --c;
-    while (c < N - 1 && sm.sbound[c + 1] <= x) ++c;
-    return c;
-  };
-  // pass 2: owners, partial slots, merge records, this CTA's items
-  WorkItem* spill = p.spill + (size_t)blockIdx.x * nseg;
-  WorkItem rec;
-  long long pcarry = 0, carry2 = 0;
-  for (int base = 0; base < nseg; base += kAttnThreads) {
-    const int s = base + tid;
-    ItemDesc it = r_it;
-    long long F = r_flat;
-    if (!regs) {  // recompute this chunk's items and offsets
-      it = s < nseg ? item_of(p, s) : ItemDesc{kItemEmpty, 0, 0, 0, 0};
-      const bool split = it.kind == kItemA || it.kind == kItemB;
-      long long tot;
-      const long long ex = block_exclusive_scan(it.kind != kItemEmpty ? (long long)it.len + cost : 0, &tot, sbuf);
-      F = carry2 + ex + (split ? cost : 0);
-      carry2 += tot;
-    }
-    const bool split = it.kind == kItemA || it.kind == kItemB;
-    int np = 0, first = 0;
-    if (s < nseg && N > 0) {
-      if (split) {
-        first = owner(F);
-        np = owner(F + it.len - 1) - first + 1;
-      } else if (it.kind == kItemWhole) {
-        first = owner(F);
-      }
-    }
-    long long tot;
-    const long long ex = block_exclusive_scan(np, &tot, sbuf);
-    const int pb = (int)(pcarry + ex);
-    // the unit's two items sit on adjacent lanes (2u, 2u + 1)
-    const int pb_o = __shfl_xor_sync(kFull, pb, 1), np_o = __shfl_xor_sync(kFull, np, 1);
-    rec.flat = F;
-    rec.len = it.kind == kItemEmpty ? 0 : it.len;
-    rec.key0 = it.key0;
-    rec.first_cta = first;
-    rec.pbase = it.kind == kItemWhole ? it.cut : pb;
-    rec.npieces = it.kind == kItemWhole ? it.packed : np;
-    rec.kind = it.kind;
-    const bool isA = (s & 1) == 0;
-    rec.pbA = isA ? pb : pb_o;
-    rec.npA = isA ? np : np_o;
-    rec.pbB = isA ? pb_o : pb;
-    rec.npB = isA ? np_o : np;
-    if (s < nseg && it.kind != kItemEmpty) {
-      const long long Fw = split ? F - cost : F, Fe = Fw + it.len + cost;
-      if (Fw <= out.lo && out.lo < Fe) sm.first_item = s;  // exactly one extent holds lo
-    }
-    if (!regs && s < nseg && !dry) spill[s] = rec;
-    pcarry += tot;
-  }
-  __syncthreads();
-  out.first = sm.first_item;
-  if (regs) {
-    const int s = tid, k = s - out.first;
-    if (s < nseg && k >= 0) {
-      if (k < kItemCache) sm.items[k] = rec;
-      else if (!dry) spill[s] = rec;
-    }
-  } else {
-    for (int k = tid; !dry && k < kItemCache && out.first + k < nseg; k += kAttnThreads)
-      sm.items[k] = spill[out.first + k];
-  }
-  __syncthreads();
-  return out;
+  if (tid < G) p.cw[tid] = (double)(before + x - wi) / (double)all;
+  if (tid == 0) p.cw[G] = 1.0;
 }
 
 template <int D>
@@ -959,6 +738,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  const int cta = blockIdx.x;
   if (tid == 32) {  // bring both TMA descriptors on chip while the match kernel runs
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmK)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmV)) : "memory");
@@ -976,25 +756,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   }
   __syncthreads();
   // launched with programmatic stream serialization: everything above
-  // overlaps the match kernel; its results are visible after this wait.
-  // Meanwhile a dry run of the split brings that code on chip.
+  // overlaps the match kernel; its results are visible after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // one round of loads: the split, then the CTA's items into shared memory
   unsigned smid;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-  build_split<D>(p, sm, 0, smid, true);
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // the split, computed here from the plans (the same on every CTA); thread
-  // 0 claims this SM's range first for a weighted split
+  const int n_cta = p.hdr->n_cta, weighted = p.hdr->weighted;
+  const long long T = p.hdr->total;
+  int first_seg = p.first_seg[cta];
+  // a weighted split: take the range of this SM (claimed in the same round
+  // of loads), else the first free one
   int mine = 0;
   if (tid == 0 && p.claim != nullptr && (int)smid < p.grid) mine = atomicCAS(p.claim + smid, 0, 1) == 0;
-  const SplitOut sp = build_split<D>(p, sm, mine, smid, false);
-  if (sp.slot < 0) return;
-  const int slot = sp.slot, first_seg = sp.first, weighted = sp.weighted;
-  const long long lo = sp.lo, hi = sp.hi;
-  const WorkItem* spill = p.spill + (size_t)blockIdx.x * p.nseg;
+  int slot = cta;
+  long long lo, hi;
+  if (weighted) {
+    if (tid == 0) {
+      int c = mine ? (int)smid : -1;
+      for (int k = 0; c < 0 && k < n_cta; ++k)
+        if (atomicCAS(p.claim + k, 0, 1) == 0) c = k;
+      sm.last_flag = c;
+    }
+    __syncthreads();
+    slot = sm.last_flag;
+    if (slot < 0) return;  // never: n_cta = grid ranges for grid CTAs
+    lo = p.bounds[slot];
+    hi = p.bounds[slot + 1];
+    first_seg = p.first_seg[slot];
+  } else {
+    if (cta >= n_cta) return;
+    lo = (long long)cta * T / n_cta;
+    hi = (long long)(cta + 1) * T / n_cta;
+  }
+  if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = p.seg[first_seg + tid];
+  __syncthreads();
   const uint64_t pol = evict_first_policy();
 
   // issue cursor: this warp's boxes of every piece, NST ahead
-  Walker wi{first_seg, lo, hi, sm.items, first_seg, spill};
+  Walker wi{first_seg, lo, hi, sm.items, first_seg};
   Piece ip;
   WarpRange ir;
   bool ivalid = wi.next(p, slot, ip);
@@ -1046,7 +845,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 
   // consume cursor
   Acc<D> A;
-  Walker wc{first_seg, lo, hi, sm.items, first_seg, spill};
+  Walker wc{first_seg, lo, hi, sm.items, first_seg};
   Piece cp;
   int cpn = 0, cons = 0, par = 0;
   uint32_t sync_phase = 0, ring_phase = 0;
@@ -1092,7 +891,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     if (!ok) break;
     if (tid == 0) t_last = globaltimer();
     const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, ring_phase, sync_phase)
-                              : finalize_piece<D>(p, sm, A, cp, sync_phase);
+                              : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (ring_copy) ring_phase ^= 1u;
     ring_pending = false;
     if (!fin) break;
@@ -1109,7 +908,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       const float old = p.rate[smid];
       p.rate[smid] = old > 0.f ? 0.7f * old + 0.3f * r : r;
     }
-    if (blockIdx.x == 0 && p.cw_next != nullptr && p.grid < kAttnThreads) rate_shares(p);
+    if (blockIdx.x == 0 && p.cw != nullptr && p.grid < kAttnThreads) rate_shares(p);
   }
   if (nissued > cons || !ok) {
     // aborting: let copies already issued land before the CTA leaves (bounded)

@@ -25,7 +25,7 @@ struct UnitPlan {
   int src_slot;  // ring slot of the matched entry (hit only)
   int dst_slot;  // ring slot receiving this step's entry
   int bad;       // 1 = invalid inputs: no work, NaN outputs, window unchanged
-  int pad;
+  int expected;  // partial results the unit's merge waits for
 };
 
 // Work items, two slots per unit u.  A large unit (more than unit_max fresh
@@ -36,21 +36,25 @@ struct UnitPlan {
 // empty.  The items of all units are laid end to end in a cost space where a
 // non-empty item weighs piece_cost + its keys (the fixed cost of a piece --
 // query load, combine, merge -- expressed in keys), and that space is split
-// over the CTAs.  A split item's keys occupy [flat, flat + len) after its
-// piece_cost of padding; a whole item starts at flat and belongs to the CTA
-// whose range holds flat.  Every attention CTA computes this split itself
-// from the units' plans (the same on all CTAs) and keeps its own items.
+// evenly over the CTAs.  A split item's keys occupy [flat, flat + len) after
+// its piece_cost of padding; a whole item starts at flat and belongs to the
+// CTA whose range holds flat.
 enum { kItemEmpty = -1, kItemA = 0, kItemB = 1, kItemWhole = 2 };
-struct WorkItem {
+struct Segment {
   long long flat;  // split: cost offset of the first key; whole: cost offset of the item
   int len;         // keys (whole: end - start)
   int key0;        // first key (absolute position in the sequence)
-  int first_cta;   // split: range holding `flat`; whole: the owning range
+  int first_cta;   // split: CTA holding `flat`; whole: the owning CTA
   int pbase;       // split: index of the first partial result; whole: the cut c_t
-  int npieces;     // split: partial results (ranges overlapping the keys);
+  int npieces;     // split: partial results (CTAs overlapping the keys);
                    // whole: hit | reused slot << 1 | written slot << 12
   int kind;        // kItem*
-  int pbA, npA, pbB, npB;  // split: partial slots and counts of the unit's two items (its merge)
+};
+
+struct PlanHeader {
+  long long total;  // size of the flattened cost space
+  int n_cta;        // CTAs with work (<= grid)
+  int weighted;     // 1: range c is [bounds[c], bounds[c+1]), sized by its SM's rate
 };
 
 // Weighted split.  HBM throughput differs between SMs, and the slow ones are
@@ -59,9 +63,8 @@ struct WorkItem {
 // streaming rate of SM c, and the CTA running on SM c takes range c (a CTA
 // whose SM's range is already taken takes a free one).  At the end of such a
 // step every CTA folds its measured rate into rate[its SM], and CTA 0 turns
-// the rates into the cumulative shares cw_next[] (cw[c] = share of ranges
-// 0..c-1, cw[grid] = 1); the next match kernel copies them to cw[], which the
-// next attention launch's split reads.
+// the rates into the cumulative shares cw[] that the next weighted step's
+// split uses (cw[c] = share of ranges 0..c-1, cw[grid] = 1).
 constexpr long long kWeightMinCost = 4096;
 
 // Layout of one partial result: o_acc [G][D] (unnormalised, relative to m),
@@ -83,13 +86,20 @@ struct MatchParams {
   const double* inv_freq;  // [D/2]
   float* qrot;             // [U][G][D], RoPE'd and scaled by log2(e)/sqrt(D)
   UnitPlan* plan;          // [U]
-  const double* cw_next;   // [grid + 1] shares written by the last attention launch, or null
-  double* cw;              // [grid + 1] shares of this step's split (copied here)
+  Segment* seg;            // [2U]
+  PlanHeader* hdr;
+  int* first_seg;          // [grid] first segment of each attention CTA's range
+  const double* cw;        // [grid + 1] cumulative range shares, or null (even split)
+  long long* bounds;       // [grid + 1] range starts of a weighted split
   int* claim;              // [grid] ranges taken by the attention CTAs (reset here)
+  int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
   int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
   float tau;
   int grid;       // CTAs of the attention kernel
+  int min_keys;   // minimum cost-space units per attention CTA
+  int piece_cost; // fixed cost of one piece, in keys
+  int unit_max;   // units with at most this many fresh keys are whole items
 };
 
 struct AttendParams {
@@ -98,11 +108,13 @@ struct AttendParams {
   const int* block_table;
   const float* qrot;
   const UnitPlan* plan;
-  const double* cw;  // [grid + 1] shares of a weighted split, or null (even split)
-  double* cw_next;   // [grid + 1] shares for the next weighted step (written by CTA 0)
+  const Segment* seg;
+  const PlanHeader* hdr;
+  const int* first_seg;  // [grid]
+  const long long* bounds;  // [grid + 1]
   int* claim;        // [grid]
   float* rate;       // [grid] learned rate per SM, or null
-  WorkItem* spill;   // [grid][2U] each CTA's items beyond its shared-memory copy
+  double* cw;        // [grid + 1] cumulative range shares (written by CTA 0)
   float* part;       // [max_parts][partial_floats]
   int* unit_cnt;     // [U]
   float* ring_o;     // [U][W+1][G][D]
@@ -113,9 +125,6 @@ struct AttendParams {
   float* lse;        // [B][Hq]
   unsigned* status;
   int Hq, Hkv, W, page_size, max_pages, nseg, grid;
-  int min_keys;    // minimum cost-space units per attention CTA
-  int piece_cost;  // fixed cost of one piece, in keys
-  int unit_max;    // units with at most this many fresh keys are whole items
 };
 
 struct AppendParams {

@@ -20,9 +20,12 @@
 //      log2(e)/sqrt(D) so the attention kernel works in exp2 units;
 //   5. the query enters the ring slot n mod (W+1) (W+1 slots: the slot
 //      written is never one the window can read this step).
-// The attention kernel turns the plans into work items itself (every CTA
-// computes the split from the plans).  CTA 0 also resets the attention
-// CTAs' range claims and fixes the shares of this step's weighted split.
+// The last CTA to finish lays every unit's two key segments end to end in a
+// cost space (each non-empty segment weighs its keys plus a fixed per-piece
+// cost) and splits that space evenly over the attention kernel's CTAs, so a
+// batch mixing short hit ranges with whole-context misses is balanced by
+// time rather than by keys.  No CTA waits for another: the last arrival
+// does the work.
 #include <math.h>
 #include <stdint.h>
 
@@ -45,6 +48,187 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Exclusive scan of one value per thread over a block of kMatchThreads.
+__device__ long long block_exclusive_scan(long long v, long long* total, long long* sbuf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sbuf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = lane < kMatchThreads / 32 ? sbuf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      long long y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kMatchThreads / 32) sbuf[lane] = w;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  long long before = warp > 0 ? sbuf[warp - 1] : 0;
+  *total = sbuf[kMatchThreads / 32 - 1];
+  __syncthreads();
+  return before + x - v;
+}
+
+// CTA holding cost-space offset x when the space [0, T) is split over N CTAs
+// as [c*T/N, (c+1)*T/N): the largest c with floor(c*T/N) <= x.
+// ceil(a / b) for 0 <= a < 2^62 and b > 0, without a 64-bit integer
+// division: an fp64 estimate (off by at most a few units) corrected exactly.
+__device__ __forceinline__ long long ceil_div(long long a, long long b, double rb) {
+  long long q = (long long)((double)a * rb);
+  while (q > 0 && q * b > a) --q;
+  while ((q + 1) * b <= a) ++q;  // q = floor(a / b)
+  return q + (q * b < a ? 1 : 0);
+}
+__device__ __forceinline__ int cta_of(long long x, long long T, int N, double rT) {
+  return (int)ceil_div((x + 1) * (long long)N, T, rT) - 1;
+}
+
+__device__ void build_segments(const MatchParams& p, int U, double cw_c) {
+  __shared__ long long sbuf[kMatchThreads / 32];
+  const int tid = threadIdx.x;
+  const int nseg = 2 * U;
+  const long long cost = p.piece_cost;
+  // pass 1: item kinds, keys and cost-space offsets
+  long long carry = 0;
+  long long r_flat = 0;  // this thread's item, kept for pass 2 when nseg <= kMatchThreads
+  int r_len = 0, r_kind = kItemEmpty;
+  for (int base = 0; base < nseg; base += kMatchThreads) {
+    const int s = base + tid;
+    int len = 0, key0 = 0, kind = kItemEmpty, cut = 0, packed = 0;
+    long long wlen = 0;
+    if (s < nseg) {
+      const UnitPlan* pl = p.plan + (s >> 1);
+      const int bad = __ldcg(&pl->bad);
+      if (!bad) {
+        const int start = __ldcg(&pl->start), c = __ldcg(&pl->cut), end = __ldcg(&pl->end);
+        if (end - start <= p.unit_max) {
+          if ((s & 1) == 0) {  // the whole unit in slot 2u
+            kind = kItemWhole;
+            len = end - start;
+            key0 = start;
+            cut = c;
+            // the CTA doing it also needs hit, reused slot and written slot
+            const int hit = __ldcg(&pl->hit), src = __ldcg(&pl->src_slot), dst = __ldcg(&pl->dst_slot);
+            packed = (hit ? 1 : 0) | ((hit ? src : 0) << 1) | (dst << 12);
+          }
+        } else {
+          len = (s & 1) ? end - c : c - start;
+          key0 = (s & 1) ? c : start;
+          kind = len > 0 ? ((s & 1) ? kItemB : kItemA) : kItemEmpty;
+        }
+        if (kind != kItemEmpty) wlen = (long long)len + cost;
+      }
+    }
+    long long tot;
+    long long ex = block_exclusive_scan(wlen, &tot, sbuf);
+    if (s < nseg) {
+      const bool split = kind == kItemA || kind == kItemB;
+      p.seg[s].flat = carry + ex + (split ? cost : 0);
+      r_flat = carry + ex + (split ? cost : 0);
+      r_len = kind == kItemEmpty ? 0 : len;
+      r_kind = kind;
+      p.seg[s].len = kind == kItemEmpty ? 0 : len;
+      p.seg[s].key0 = key0;
+      p.seg[s].kind = kind;
+      p.seg[s].pbase = cut;  // whole items keep their cut here; split items overwrite it below
+      if (kind == kItemWhole) p.seg[s].npieces = packed;
+    }
+    carry += tot;
+  }
+  const long long T = carry;
+  int N = 0;
+  if (T > 0) {
+    long long want = (T + p.min_keys - 1) / p.min_keys;
+    N = (int)(want < (long long)p.grid ? want : (long long)p.grid);
+    if (N < 1) N = 1;
+  }
+  const double rT = T > 0 ? 1.0 / (double)T : 0.0;
+  // weighted split: range c from the cumulative shares of the SMs' rates
+  __shared__ long long sbound[kMatchThreads + 1];
+  const bool weighted =
+      p.cw != nullptr && N == p.grid && p.grid < kMatchThreads && T >= kWeightMinCost * (long long)p.grid;
+  if (weighted) {
+    if (tid <= N) sbound[tid] = tid == 0 ? 0 : (tid == N ? T : (long long)((double)T * cw_c));
+    __syncthreads();
+    if (tid <= N) p.bounds[tid] = sbound[tid];
+  }
+  if (p.claim != nullptr)
+    for (int c = tid; c < p.grid; c += kMatchThreads) p.claim[c] = 0;
+  // CTA holding offset x: the largest c with start(c) <= x (weighted: from
+  // the even split's guess, walked to the exact range; the weights are near 1)
+  auto owner = [&](long long x) -> int {
+    if (!weighted) return cta_of(x, T, N, rT);
+    int c = (int)((double)x * N * rT);
+    c = c < 0 ? 0 : (c > N - 1 ? N - 1 : c);
+    while (c > 0 && sbound[c] > x) --c;
+    while (c < N - 1 && sbound[c + 1] <= x) ++c;
+    return c;
+  };
+  // first CTA whose range starts at or after x
+  auto first_from = [&](long long x) -> long long {
+    if (!weighted) return ceil_div(x * N, T, rT);
+    return x <= 0 ? 0 : owner(x - 1) + 1;
+  };
+  __syncthreads();
+  // pass 2: owning / first CTA, partial slots, and each CTA's first item
+  long long pcarry = 0;
+  for (int base = 0; base < nseg; base += kMatchThreads) {
+    const int s = base + tid;
+    int np = 0, first = 0, kind = kItemEmpty, len = 0;
+    long long F = 0;
+    if (s < nseg) {
+      if (nseg <= kMatchThreads) {
+        F = r_flat;
+        len = r_len;
+        kind = r_kind;
+      } else {
+        F = p.seg[s].flat;
+        len = p.seg[s].len;
+        kind = p.seg[s].kind;
+      }
+      if (kind == kItemA || kind == kItemB) {
+        first = owner(F);
+        np = owner(F + len - 1) - first + 1;
+      } else if (kind == kItemWhole) {
+        first = owner(F);
+      }
+    }
+    long long tot;
+    long long ex = block_exclusive_scan(np, &tot, sbuf);
+    // units own items (2u, 2u+1): adjacent threads of one warp
+    const int np_next = __shfl_down_sync(0xffffffffu, np, 1);
+    if (s < nseg) {
+      p.seg[s].first_cta = first;
+      if (kind != kItemWhole) {
+        p.seg[s].npieces = np;
+        p.seg[s].pbase = (int)(pcarry + ex);
+      }
+      if ((s & 1) == 0) p.plan[s >> 1].expected = np + np_next;
+      // CTAs whose range starts inside this item's cost extent [Fw, Fe)
+      // begin their walk here (even split: lo_c = floor(c*T/N) lies in it
+      // iff ceil(Fw*N/T) <= c < ceil(Fe*N/T))
+      if (kind != kItemEmpty && N > 0) {
+        const bool split = kind == kItemA || kind == kItemB;
+        const long long Fw = split ? F - cost : F;
+        const long long Fe = Fw + len + cost;
+        const long long ca = first_from(Fw), cb = first_from(Fe);
+        for (long long c = ca; c < cb && c < N; ++c) p.first_seg[c] = s;
+      }
+    }
+    pcarry += tot;
+  }
+  if (tid == 0) {
+    p.hdr->total = T;
+    p.hdr->n_cta = N;
+    p.hdr->weighted = weighted ? 1 : 0;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchParams p) {
   constexpr int G = kGroup;
@@ -53,21 +237,15 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   __shared__ float sdist[kMaxWindow];
   __shared__ int spos[kMaxWindow];
   __shared__ int sslot[kMaxWindow];
-  __shared__ int s_bad_page;
+  __shared__ int s_bad_page, s_last;
   __shared__ UnitPlan s_plan;
 
   // the attention kernel (launched with programmatic stream serialization)
   // may start its prologue now; it waits for this grid before reading
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (blockIdx.x == 0) {
-    // the attention launch that follows claims its ranges afresh, and splits
-    // by the shares the last attention launch left (its CTA 0 writes the next
-    // ones while this step's CTAs read these)
-    if (p.claim != nullptr)
-      for (int c = threadIdx.x; c < p.grid; c += kMatchThreads) p.claim[c] = 0;
-    if (p.cw_next != nullptr)
-      for (int c = threadIdx.x; c <= p.grid; c += kMatchThreads) p.cw[c] = __ldcg(p.cw_next + c);
-  }
+  // the split's cumulative share of range tid, loaded now so the CTA that
+  // builds the split does not wait for it
+  const double cw_c = (p.cw != nullptr && (int)threadIdx.x <= p.grid) ? __ldcg(p.cw + threadIdx.x) : 0.0;
   const int u = blockIdx.x;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -184,7 +362,7 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
       pl.start = hit ? (bp - p.band > 0 ? bp - p.band : 0) : 0;
       pl.dst_slot = n % Wp1;
       pl.bad = (len < 1 || len > p.capacity) ? 1 : 0;
-      pl.pad = 0;
+      pl.expected = 0;
       s_plan = pl;
       spos[0] = hit ? bp : -1;  // matched position (slot 0 of spos no longer needed)
     }
@@ -240,6 +418,19 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     }
   }
 
+  // last CTA to arrive builds the segment table for the attention kernel.
+  // Only the plan (written by thread 0) is read by that CTA; everything else
+  // goes to the attention kernel, which starts after this grid completes.
+  if (tid == 0) {
+    __threadfence();
+    const int ticket = atomicAdd(p.done, 1);
+    s_last = (ticket == (int)gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  build_segments(p, (int)gridDim.x, cw_c);
+  if (tid == 0) *p.done = 0;
 }
 
 }  // namespace

@@ -39,8 +39,10 @@ constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr size_t kPartFloats = (size_t)kGroup * kMaxD + 2 * kGroup;
 constexpr size_t kOffQrot = 0;
 constexpr size_t kOffPlan = align256(kOffQrot + (size_t)kMaxUnits * kGroup * kMaxD * 4);
-constexpr size_t kOffSpill = align256(kOffPlan + kMaxUnits * sizeof(UnitPlan));  // [CTA][2U] work items
-constexpr size_t kOffPart = align256(kOffSpill + (size_t)kMaxCtas * 2 * kMaxUnits * sizeof(WorkItem));
+constexpr size_t kOffSeg = align256(kOffPlan + kMaxUnits * sizeof(UnitPlan));
+constexpr size_t kOffHdr = align256(kOffSeg + 2 * kMaxUnits * sizeof(Segment));
+constexpr size_t kOffFirst = align256(kOffHdr + sizeof(PlanHeader));
+constexpr size_t kOffPart = align256(kOffFirst + kMaxCtas * 4);
 constexpr size_t kOffCnt = align256(kOffPart + (size_t)(kMaxCtas + 2 * kMaxUnits) * kPartFloats * 4);
 // counters block, cleared on every call: unit_cnt[kMaxUnits], done, status, steps[kMaxUnits]
 constexpr size_t kCntBytes = (2 * kMaxUnits + 2) * 4;
@@ -168,9 +170,13 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.inv_freq = reinterpret_cast<const double*>(base + kOffInv);
   mp.qrot = reinterpret_cast<float*>(base + kOffQrot);
   mp.plan = reinterpret_cast<UnitPlan*>(base + kOffPlan);
-  mp.cw_next = nullptr;  // even split: no per-SM record
-  mp.cw = nullptr;
+  mp.seg = reinterpret_cast<Segment*>(base + kOffSeg);
+  mp.hdr = reinterpret_cast<PlanHeader*>(base + kOffHdr);
+  mp.first_seg = reinterpret_cast<int*>(base + kOffFirst);
+  mp.cw = nullptr;  // even split: no per-SM record
+  mp.bounds = nullptr;
   mp.claim = nullptr;
+  mp.done = cnt + kMaxUnits;
   mp.status = status;
   mp.B = batch;
   mp.Hq = num_q_heads;
@@ -183,6 +189,9 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.capacity = page_size == 0 ? max_seq : max_pages_per_seq * page_size;
   mp.tau = 0.f;
   mp.grid = grid;
+  mp.min_keys = 128;
+  mp.piece_cost = 1024;
+  mp.unit_max = 1024;
   if (launch_match(mp, head_dim, st) != cudaSuccess) return MAC_ERR_CUDA;
 
   // --- attention over every key, merge into out/lse (and the dummy ring)
@@ -196,11 +205,13 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.block_table = page_size > 0 ? block_table : nullptr;
   ap.qrot = mp.qrot;
   ap.plan = mp.plan;
-  ap.cw = nullptr;
-  ap.cw_next = nullptr;
+  ap.seg = mp.seg;
+  ap.hdr = mp.hdr;
+  ap.first_seg = mp.first_seg;
+  ap.bounds = nullptr;
   ap.claim = nullptr;
   ap.rate = nullptr;
-  ap.spill = reinterpret_cast<WorkItem*>(base + kOffSpill);
+  ap.cw = nullptr;
   ap.part = reinterpret_cast<float*>(base + kOffPart);
   ap.unit_cnt = cnt;
   ap.ring_o = reinterpret_cast<float*>(base + kOffRingO);
@@ -217,8 +228,5 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.max_pages = max_pages_per_seq;
   ap.nseg = 2 * U;
   ap.grid = grid;
-  ap.min_keys = 128;
-  ap.piece_cost = 1024;
-  ap.unit_max = 1024;
   return launch_attend(ap, head_dim, grid, st) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
