@@ -47,10 +47,15 @@ def _peaks():
 
 
 def _kernel_hash() -> str:
+    """Hash of the attention kernel's source code (comments and blank space
+    removed, so that a comment edit does not orphan a profile)."""
     h = hashlib.sha256()
     for f in ("mac_attend.cu", "mac_internal.cuh"):
-        with open(os.path.join(ROOT, "kv_cache_reuse_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "kv_cache_reuse_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 
