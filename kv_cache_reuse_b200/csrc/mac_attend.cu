@@ -330,110 +330,133 @@ __device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, 
   return ok;
 }
 
-// Merge of unit u by the CTA holding its last partial (256 threads).  Phase
-// 1 stages every partial's (m, l) in shared memory with one round of
-// independent loads; phase 2 weighs the partial outputs, all loads in flight.
 template <int D>
-__device__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32_t& sync_phase) {
+__device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, int idx, int h, float& MA, float& LA,
+                                               float& OA, float& MB, float& LB, float& OB);
+
+// Fold one state (max m, sum l, outputs o relative to 2^m) into (M, L, O).
+template <int N>
+__device__ __forceinline__ void fold_state(float& M, float& L, float (&O)[N], float m, float l, const float* o) {
+  const float Mn = fmaxf(M, m);
+  const float Mu = Mn == -INFINITY ? 0.f : Mn;
+  const float a = ex2(M - Mu), c = ex2(m - Mu);
+  L = L * a + l * c;
+#pragma unroll
+  for (int j = 0; j < N; ++j) O[j] = O[j] * a + o[j] * c;
+  M = Mn;
+}
+
+// Last arriver of a split unit: merge its partials.  Segment A's partials
+// (with the reused state on a hit) give the new prefix state over [0, c_t),
+// stored in the ring; that state and segment B's partials give the output.
+// The 8 warps share the partials (warp w folds partials w, w + 8, ..., each
+// lane FPL consecutive floats of one head), with up to 48 partials' loads in
+// flight at once; the warps' states then meet in shared memory.
+template <int D>
+__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32_t& sync_phase) {
   constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
-  constexpr int kCap = (kConsumerWarps * Cfg<D>::WB) / (2 * G);  // pieces whose (m, l) fit in wbuf
+  constexpr int FPL = GD / 32, F4 = FPL / 4;  // floats and float4 of a partial per lane
+  constexpr int BP = 6;                       // partials per warp per round of loads
+  constexpr int VEC = GD / (kConsumerWarps * 32);
+  static_assert(VEC * kConsumerWarps * 32 == GD && F4 * 4 * 32 == GD, "merge layout");
   const UnitPlan pl = p.plan[u];
   const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
-  const int nA = sA.npieces, n = sA.npieces + sB.npieces;
-  float* mm = &sm.wbuf[0][0];  // [piece][G] maxima, then [piece][G] sums
-  float* ll = mm + kCap * G;
-  const bool staged = n <= kCap;
-  if (staged) {
-    for (int t = threadIdx.x; t < n * G; t += kConsumerWarps * 32) {
-      const int i = t / G, h = t - i * G;
-      const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
-      const float* pp = p.part + (size_t)slot * PF;
-      mm[t] = __ldcg(pp + GD + h);
-      ll[t] = __ldcg(pp + GD + G + h);
+  const int nA = sA.npieces, n = nA + sB.npieces;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f0 = lane * FPL, hl = f0 / D;
+
+  float MA = -INFINITY, LA = 0.f, OA[FPL], MB = -INFINITY, LB = 0.f, OB[FPL];
+#pragma unroll
+  for (int j = 0; j < FPL; ++j) OA[j] = OB[j] = 0.f;
+  if (warp == 0 && pl.hit) {  // the reused state joins set A (its o is normalised)
+    const size_t rs = (size_t)u * Wp1 + pl.src_slot;
+    const float rl = __ldcg(p.ring_l + rs * G + hl), rm = __ldcg(p.ring_m + rs * G + hl) * kLog2e;
+    float o[FPL];
+#pragma unroll
+    for (int f = 0; f < F4; ++f) {
+      const float4 t = __ldcg(reinterpret_cast<const float4*>(p.ring_o + rs * GD + f0) + f);
+      o[4 * f] = t.x * rl;
+      o[4 * f + 1] = t.y * rl;
+      o[4 * f + 2] = t.z * rl;
+      o[4 * f + 3] = t.w * rl;
+    }
+    fold_state<FPL>(MA, LA, OA, rm, rl, o);
+  }
+  for (int i0 = warp; i0 < n; i0 += kConsumerWarps * BP) {
+    float4 v[BP][F4];
+    float mv[BP], lv[BP];
+#pragma unroll
+    for (int k = 0; k < BP; ++k) {
+      const int i = i0 + k * kConsumerWarps;
+      if (i < n) {
+        const float* pp = p.part + (size_t)(i < nA ? sA.pbase + i : sB.pbase + (i - nA)) * PF;
+#pragma unroll
+        for (int f = 0; f < F4; ++f) v[k][f] = __ldcg(reinterpret_cast<const float4*>(pp + f0) + f);
+        mv[k] = __ldcg(pp + GD + hl);
+        lv[k] = __ldcg(pp + GD + G + hl);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < BP; ++k) {
+      const int i = i0 + k * kConsumerWarps;
+      if (i < n) {
+        const float* o = reinterpret_cast<const float*>(v[k]);
+        if (i < nA)
+          fold_state<FPL>(MA, LA, OA, mv[k], lv[k], o);
+        else
+          fold_state<FPL>(MB, LB, OB, mv[k], lv[k], o);
+      }
     }
   }
-  if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  auto pm = [&](int i, int h) -> float {
-    if (staged) return mm[i * G + h];
-    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
-    return __ldcg(p.part + (size_t)slot * PF + GD + h);
-  };
-  auto pl_ = [&](int i, int h) -> float {
-    if (staged) return ll[i * G + h];
-    const int slot = i < nA ? sA.pbase + i : sB.pbase + (i - nA);
-    return __ldcg(p.part + (size_t)slot * PF + GD + G + h);
-  };
-  for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
-    const int h = idx / D, d = idx - h * D;
-    // new prefix state over [0, c_t): reused state (hit) + amend partials
-    float M = -INFINITY, rm = -INFINITY, rl = 0.f, ro = 0.f;
-    if (pl.hit) {
-      const size_t rs = (size_t)u * Wp1 + pl.src_slot;
-      rl = p.ring_l[rs * G + h];
-      rm = p.ring_m[rs * G + h] * kLog2e;
-      ro = p.ring_o[rs * GD + idx];
-      M = rm;
-    }
-    for (int i = 0; i < nA; ++i) M = fmaxf(M, pm(i, h));
-    const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f, O = 0.f;
-    if (pl.hit) {
-      const float a = ex2(rm - Mu);
-      L += rl * a;
-      O += ro * rl * a;
-    }
-    for (int i0 = 0; i0 < nA; i0 += 16) {  // 16 partial outputs in flight at a time
-      float v[16];
+  // the warps' sets meet in shared memory: set A (prefix), then set B (tail)
+  float PM[VEC], PL[VEC], PO[VEC], QM[VEC], QL[VEC], QO[VEC];
+  float* wb = sm.wbuf[warp];
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        v[k] = i0 + k < nA ? __ldcg(p.part + (size_t)(sA.pbase + i0 + k) * PF + idx) : 0.f;
+  for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        if (i0 + k < nA) {
-          const float a = ex2(pm(i0 + k, h) - Mu);
-          L += pl_(i0 + k, h) * a;
-          O += v[k] * a;
-        }
+    for (int j = 0; j < FPL; ++j) wb[f0 + j] = pass == 0 ? OA[j] : OB[j];
+    if (f0 - hl * D == 0) {
+      wb[GD + hl] = pass == 0 ? MA : MB;
+      wb[GD + G + hl] = pass == 0 ? LA : LB;
+    }
+    if (!consumer_sync(sm, sync_phase, p.status)) return false;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) {
+      const int idx = threadIdx.x * VEC + j;
+      float m_, l_, o_, xm, xl, xo;
+      combine_warps2<D>(sm, kConsumerWarps, idx, idx / D, m_, l_, o_, xm, xl, xo);
+      if (pass == 0) {
+        PM[j] = m_, PL[j] = l_, PO[j] = o_;
+      } else {
+        QM[j] = m_, QL[j] = l_, QO[j] = o_;
       }
     }
-    const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
-    p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
-    if (d == 0) {
-      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
-      p.ring_l[ds * G + h] = L;
-    }
-    // output: new prefix state + tail partials
-    float M2 = M;
-    for (int i = nA; i < n; ++i) M2 = fmaxf(M2, pm(i, h));
+    if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  }
+  const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
+#pragma unroll
+  for (int j = 0; j < VEC; ++j) {
+    const int idx = threadIdx.x * VEC + j, h = idx / D, d = idx - h * D;
+    p.ring_o[ds * GD + idx] = PL[j] > 0.f ? PO[j] / PL[j] : 0.f;
+    const float M2 = fmaxf(PM[j], QM[j]);
     const float M2u = M2 == -INFINITY ? 0.f : M2;
-    const float a0 = ex2(M - M2u);
-    float L2 = L * a0, O2 = O * a0;
-    for (int i0 = nA; i0 < n; i0 += 16) {
-      float v[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k)
-        v[k] = i0 + k < n ? __ldcg(p.part + (size_t)(sB.pbase + (i0 + k - nA)) * PF + idx) : 0.f;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        if (i0 + k < n) {
-          const float a = ex2(pm(i0 + k, h) - M2u);
-          L2 += pl_(i0 + k, h) * a;
-          O2 += v[k] * a;
-        }
-      }
-    }
+    const float a0 = ex2(PM[j] - M2u), a1 = ex2(QM[j] - M2u);
+    const float L2 = PL[j] * a0 + QL[j] * a1;
     const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
-    p.out[orow * D + d] = O2 / L2;
-    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+    p.out[orow * D + d] = (PO[j] * a0 + QO[j] * a1) / L2;
+    if (d == 0) {
+      p.ring_m[ds * G + h] = PL[j] > 0.f ? PM[j] * kLn2 : -INFINITY;
+      p.ring_l[ds * G + h] = PL[j];
+      p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+    }
   }
   if (threadIdx.x == 0) {
     p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
     p.unit_cnt[u] = 0;
   }
-  // wbuf is reused by the next piece
-  return consumer_sync(sm, sync_phase, p.status);
+  return true;
 }
 
 // Store the warp's state in its shared-memory slot: o [G][D] unnormalised,

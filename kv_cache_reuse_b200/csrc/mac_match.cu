@@ -422,8 +422,10 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   // Only the plan (written by thread 0) is read by that CTA; everything else
   // goes to the attention kernel, which starts after this grid completes.
   if (tid == 0) {
-    __threadfence();
-    const int ticket = atomicAdd(p.done, 1);
+    // the ticket's release publishes this CTA's plan; its acquire (for the
+    // last CTA) orders the build's reads of the other plans
+    int ticket;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(p.done) : "memory");
     s_last = (ticket == (int)gridDim.x - 1);
   }
   __syncthreads();
