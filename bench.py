@@ -285,6 +285,7 @@ def run_mac(args, rank, world, local_rank):
         warm = {"positions": n, "ms": wms, "kv_bytes": wbytes, "gbs": wbytes / (wms * 1e-3) / 1e9,
                 "frac": wbytes / (wms * 1e-3) / 1e9 / peak, "device_status": st.get_status()}
         st.close()
+    layers = run_layers(args, wl, stream, cache, K, V, bt, kw, dev, peak) if args.layers > 0 else None
     hitrun = None
     if args.hit_steps > 0:
         # the hit path alone: the same shape with every labelled step a near-repeat
@@ -353,11 +354,83 @@ def run_mac(args, rank, world, local_rank):
                            "note": "latency-bound: a few MB per launch"}
     if warm:
         res["warm_start"] = warm
+    if layers:
+        res["layer_stack"] = layers
     if e2e:
         res["e2e"] = e2e
     if cpu:
         res["cpu_baseline"] = cpu
     return res
+
+
+def run_layers(args, wl, stream, cache, K, V, bt, kw, dev, peak):
+    """A stack of L independent layers per token -- each with its own state,
+    its own copy of the cache and its own query stream -- recorded once as
+    one CUDA graph over all layers and replayed per token (the inputs are
+    copied into the graph's fixed buffers first, inside the timed region;
+    L2 flushed between tokens)."""
+    import torch
+    import kv_cache_reuse_b200 as mac
+    L = args.layers
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    T = min(args.warmup + args.steps, stream.q.shape[0])
+    s = torch.cuda.current_stream(dev)
+    Ks = [K] + [K.clone() for _ in range(L - 1)]
+    Vs = [V] + [V.clone() for _ in range(L - 1)]
+    q_host = [stream.q[:T]] + [synth.queries(wl.with_(seed=wl.seed + 7919 * l), T).q for l in range(1, L)]
+    q_all = torch.from_numpy(np.ascontiguousarray(np.stack(q_host, axis=1))).to(dev)  # [T][L][B][Hq][D]
+    pos_all = torch.from_numpy(stream.rope_pos[:T]).to(dev)
+    lens_all = torch.from_numpy(stream.seq_lens[:T]).to(dev)
+    qb = torch.empty((L, B, Hq, D), dtype=torch.float32, device=dev)
+    posb = torch.empty(B, dtype=torch.int32, device=dev)
+    lensb = torch.empty(B, dtype=torch.int32, device=dev)
+    outs = torch.empty((L, B, Hq, D), dtype=torch.float32, device=dev)
+    lses = torch.empty((L, B, Hq), dtype=torch.float32, device=dev)
+    hitb = torch.zeros((L, B, Hkv), dtype=torch.uint8, device=dev)
+    mpb = torch.zeros((L, B, Hkv), dtype=torch.int32, device=dev)
+    hit_all = torch.zeros((T, L, B, Hkv), dtype=torch.uint8, device=dev)
+    mp_all = torch.zeros((T, L, B, Hkv), dtype=torch.int32, device=dev)
+    states = [mac.MacState.for_workload(wl, **kw) for _ in range(L)]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    cs = torch.cuda.Stream(dev)
+    cs.wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cs):
+        for l in range(L):
+            mac.mac_decode_step(states[l], qb[l], posb, Ks[l], Vs[l], bt, lensb, outs[l], lses[l], hitb[l], mpb[l])
+    torch.cuda.synchronize(dev)
+    ev = []
+    for t in range(T):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        qb.copy_(q_all[t])
+        posb.copy_(pos_all[t])
+        lensb.copy_(lens_all[t])
+        g.replay()
+        e1.record(s)
+        hit_all[t].copy_(hitb)
+        mp_all[t].copy_(mpb)
+        if t >= args.warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    ms = float(np.sum([a.elapsed_time(b) for a, b in ev]))
+    n = len(ev)
+    hits = hit_all.cpu().numpy()
+    mps = mp_all.cpu().numpy()
+    kv = 0
+    for t in range(args.warmup, T):
+        for l in range(L):
+            kv += step_bytes(wl, hits[t, l], mps[t, l], stream.seq_lens[t], min(t, wl.W))[2]
+    status = [st.get_status() for st in states]
+    for st in states:
+        st.close()
+    del g
+    return {"layers": L, "tokens": n, "tokens_per_s": n / (ms * 1e-3), "ms_per_token": ms / n,
+            "us_per_layer": ms * 1e3 / (n * L), "hit_fraction": float(hits[args.warmup:].mean()),
+            "kv_bytes_per_token": kv / n, "kv_gbs": kv / (ms * 1e-3) / 1e9, "kv_frac": kv / (ms * 1e-3) / 1e9 / peak,
+            "device_status": max(status),
+            "timing": "CUDA events around input copies + one graph replay per token; L2 flushed between tokens"}
 
 
 def run_e2e(args, wl, stream, cache, K, V, bt, kw, dev, world):
@@ -464,6 +537,8 @@ def main():
     ap.add_argument("--miss-steps", type=int, default=16, help="timed steps of the all-miss run (0 = skip)")
     ap.add_argument("--hit-steps", type=int, default=16, help="timed steps of the all-hit run (0 = skip)")
     ap.add_argument("--warm-start", action="store_true", help="also time seeding the windows from W positions")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="also time a stack of this many layers per token, one CUDA graph per token")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)

@@ -120,7 +120,10 @@ int mac_reset_seq(MacState *st, int b, void *stream);
  *   hit_mask    device uint8 [B][Hkv], 1 where the match hit; may be NULL.
  *   match_pos   device int32 [B][Hkv], position of the matched entry or -1;
  *               may be NULL.
- * The window of every unit advances by one entry.  Enqueues two kernels. */
+ * The window of every unit advances by one entry.  Enqueues two kernels and
+ * nothing else (no allocation, no host synchronisation), so the call can be
+ * recorded into a CUDA graph -- e.g. one graph per token over all layers'
+ * states -- and replayed; the recording holds the K/V addresses it saw. */
 int mac_decode_step(MacState *st, const float *q_pre, const int *rope_pos, const uint16_t *K,
                     const uint16_t *V, const int *block_table, const int *seq_lens, float *out,
                     float *lse, uint8_t *hit_mask, int *match_pos, void *stream);
