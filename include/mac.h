@@ -15,8 +15,10 @@
  *
  * Conventions used by every entry point
  *   - Group: each KV head serves G = num_q_heads / num_kv_heads query heads
- *     (GQA, page 1 "composes with ... MQA/GQA"); this build requires G = 4.
- *     One match decision is taken per (sequence, KV head) over its G heads.
+ *     (GQA, page 1 "composes with ... MQA/GQA"); G may be 1 (multi-head
+ *     attention) up to 8.  Larger groups (MQA with more than 8 query heads
+ *     per KV head) return MAC_ERR_SHAPE.  One match decision is taken per
+ *     (sequence, KV head) over its G heads.
  *   - Distance: mean over the G heads of the squared L2 distance between the
  *     pre-RoPE queries.  Hit iff the smallest distance over the window is
  *     strictly below tau; ties go to the more recent entry; NaN never hits.
@@ -75,7 +77,7 @@ enum {
 typedef struct MacConfig {
     int batch;             /* B >= 1 */
     int num_q_heads;       /* Hq */
-    int num_kv_heads;      /* Hkv; Hq / Hkv must be 4 */
+    int num_kv_heads;      /* Hkv; Hq must be a multiple of it, Hq / Hkv <= 8 */
     int head_dim;          /* D: 64 or 128 */
     int window;            /* W: entries kept per (sequence, KV head), 1..256 */
     int band;              /* b >= 0: keys before the match position that are recomputed */
@@ -231,15 +233,16 @@ int mac_attend_grid(const MacState *st);
  * every sequence and KV head, attention of the RoPE'd query group over ALL
  * keys [0, seq_lens[b] - 1] (the miss path of mac_decode_step: no window,
  * no reuse, no MacState) with the same kernels, and keeps all their scratch
- * (about 1 MiB) in one static device array inside the library.
+ * (about 2 MiB) in one static device array inside the library.
  *   q_pre, rope_pos, K, V, block_table, seq_lens, out, lse: as in
  *       mac_decode_step (device pointers, caller-owned, 16-byte aligned
  *       q_pre, K, V).
  *   device_status: device uint32 receiving MAC_DEV_* bits (OR-ed in, not
  *       cleared), or NULL to use a word inside the static scratch.
  *   batch .. num_pages: shapes as in MacConfig.
- * Limits: batch * num_kv_heads <= 64, head_dim 64 or 128, Hq/Hkv = 4;
- * larger shapes return MAC_ERR_SHAPE before anything is enqueued.
+ * Limits: batch * num_kv_heads <= 64, batch * num_q_heads <= 256, head_dim
+ * 64 or 128, Hq / Hkv an integer from 1 to 8; other shapes return
+ * MAC_ERR_SHAPE before anything is enqueued.
  * Nothing is allocated or freed; the static array exists on every device
  * that loads the library until the process exits.  The first call on a
  * device looks up the array's device address and sets kernel attributes

@@ -113,7 +113,7 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 int check_config(const MacConfig* c) {
   if (!c) return MAC_ERR_ARG;
   if (c->batch < 1 || c->num_kv_heads < 1 || c->num_q_heads < 1) return MAC_ERR_ARG;
-  if (c->num_q_heads % c->num_kv_heads != 0 || c->num_q_heads / c->num_kv_heads != kGroup) return MAC_ERR_SHAPE;
+  if (c->num_q_heads % c->num_kv_heads != 0 || c->num_q_heads / c->num_kv_heads > kMaxGroup) return MAC_ERR_SHAPE;
   if (c->head_dim != 64 && c->head_dim != 128) return MAC_ERR_SHAPE;
   if (c->window < 1 || c->window > kMaxWindow) return MAC_ERR_SHAPE;
   if (c->band < 0 || c->cut_mode < 0 || c->cut_mode > 1) return MAC_ERR_ARG;
@@ -213,7 +213,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   MacState* s = new (std::nothrow) MacState();
   if (!s) return MAC_ERR_OOM;
   s->cfg = *cfg;
-  s->G = kGroup;
+  s->G = cfg->num_q_heads / cfg->num_kv_heads;
   s->U = cfg->batch * cfg->num_kv_heads;
   s->D = cfg->head_dim;
   s->W = cfg->window;
@@ -249,7 +249,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->bounds, (size_t)s->grid + 1));
   A(alloc(&s->cw, (size_t)s->grid + 1));
   A(alloc(&s->claim, (size_t)s->grid));
-  A(alloc(&s->part, s->max_parts * partial_floats((int)D)));
+  A(alloc(&s->part, s->max_parts * partial_floats((int)G, (int)D)));
   A(alloc(&s->unit_cnt, U));
   A(alloc(&s->done, 1));
   A(alloc(&s->inv_freq, D / 2));
@@ -299,7 +299,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   for (size_t i = 0; i < D / 2; ++i) inv[i] = pow(cfg->rope_theta, -2.0 * (double)i / (double)D);
   A(cudaMemcpy(s->inv_freq, inv, sizeof(double) * (D / 2), cudaMemcpyHostToDevice));
   free(inv);
-  A(attend_prepare((int)D));
+  A(attend_prepare((int)D, (int)G));
   A(cudaDeviceSynchronize());
   if (e != cudaSuccess) {
     free_all(s);
@@ -387,6 +387,7 @@ static int match_impl(MacState* s, float tau, const float* q_pre, const int* rop
   p.B = s->cfg.batch;
   p.Hq = s->cfg.num_q_heads;
   p.Hkv = s->cfg.num_kv_heads;
+  p.G = s->G;
   p.W = s->W;
   p.band = s->cfg.band - s->cfg.cut_mode;  // c = max(0, p - band + cut_mode)
   p.page_size = s->cfg.page_size;
@@ -440,6 +441,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.status = s->status;
   p.Hq = s->cfg.num_q_heads;
   p.Hkv = s->cfg.num_kv_heads;
+  p.G = s->G;
   p.W = s->W;
   p.page_size = s->cfg.page_size;
   p.max_pages = s->cfg.max_pages_per_seq;

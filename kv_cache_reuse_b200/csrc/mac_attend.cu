@@ -24,16 +24,19 @@
 // bf16 in, fp32 accumulate), keys on the M side:
 //   S^T[16 keys x 8] = K[16 x D] . Qx[D x 8]     (QK, D/16 k-steps)
 //   O^T[D x 8]      += V^T[D x 16] . Px[16 x 8]  (PV, D/16 row tiles)
-// The 8 columns are the 4 query heads of the GQA group twice: the fp32
-// query (and the fp32 softmax weights) split into a bf16 high part and a
-// bf16 residual, so every column carries data and the products keep ~16
-// mantissa bits; score = column h + column h+4.  This is not about tensor
-// throughput -- the work is HBM-bound (4 flop per byte of K/V) -- but about
-// instruction issue: a box costs ~100 warp instructions instead of ~700 on
-// the FP32 pipes, which keeps the miss path on the memory roofline and a
-// hit's few boxes short.  K fragments come from ldmatrix, V^T fragments from
-// ldmatrix.trans (the swizzle keeps both conflict-free); the weights reach
-// their B-fragment layout through 256 bytes of shared memory per warp.
+// The fp32 query (and the fp32 softmax weights) is split into a bf16 high
+// part and a bf16 residual, so the products keep ~16 mantissa bits.  With up
+// to 4 query heads per KV head the 8 columns are the group twice (high parts,
+// then residuals; score = column h + column h+4; heads past the group are
+// zero columns); with 5 to 8 heads each head has one column and the high and
+// residual parts are two products into the same accumulator.  This is not
+// about tensor throughput -- the work is HBM-bound (G flop per byte of K/V
+// for G query heads) -- but about instruction issue: a box costs ~100 warp
+// instructions instead of ~700 on the FP32 pipes, which keeps the miss path
+// on the memory roofline and a hit's few boxes short.  K fragments come from
+// ldmatrix, V^T fragments from ldmatrix.trans (the swizzle keeps both
+// conflict-free); the weights reach their B-fragment layout through 64 bytes
+// per head of shared memory per warp.
 //
 // Softmax runs in exp2 units (the query is pre-scaled by log2(e)/sqrt(D)).
 // Every piece a CTA processes ends in a partial (o unnormalised, m, l).  The
@@ -62,32 +65,39 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 constexpr int kRateMinBoxes = 256;  // a CTA's rate record needs this much streaming
 constexpr int kItemCache = 64;  // work items of one CTA kept in shared memory
 
-template <int D>
+// GP: the query group padded to 4 or 8 heads.  GP = 4 puts each head in
+// two tile columns (bf16 high part, bf16 residual); GP = 8 gives each head
+// one column and runs the high and residual parts as two products into the
+// same accumulator.  The real group G = p.G <= GP sets the global layouts.
+template <int D, int GP>
 struct Cfg {
   static constexpr int KS = D / 16;               // k-steps of QK = row tiles of PV
   static constexpr int HALVES = D / 64;           // 128-byte swizzled halves of a key row
-  static constexpr int NST = D == 128 ? 3 : 6;    // boxes in flight per warp
+  static constexpr int NST = GP == 4 ? (D == 128 ? 3 : 6) : (D == 128 ? 2 : 4);  // boxes in flight per warp
   static constexpr int NQ = NST + 1;              // query buffers (pieces the issue cursor can be ahead)
-  static constexpr int GD = kGroup * D;
-  static constexpr int PF = kGroup * D + 2 * kGroup;  // floats of one partial
-  static constexpr int WB = (PF > 128 ? PF : 128);     // per-warp scratch floats
+  static constexpr int GD = GP * D;               // floats of a padded query group
+  static constexpr int SF = GP * D + 2 * GP;      // a warp's state: o [GP][D], m [GP], l [GP]
+  static constexpr int PB = kSubKeys * GP;        // floats of one weights exchange buffer
+  static constexpr int WB = SF > 2 * PB ? SF : 2 * PB;  // per-warp scratch floats
+  static constexpr int QW = GP == 4 ? 2 : 4;      // query B-fragment registers per k-step
 };
 
-template <int D>
+template <int D, int GP>
 struct __align__(1024) AttnSmem {
+  using C = Cfg<D, GP>;
   // per warp: ring of (K box, V box), each [HALVES][16 keys][64 dims] bf16, 128-byte swizzle
-  uint16_t kv[kConsumerWarps][Cfg<D>::NST][2][kSubKeys * D];
-  float q[Cfg<D>::NQ][Cfg<D>::GD];         // queries of the upcoming pieces
-  float wbuf[kConsumerWarps][Cfg<D>::WB];  // weights exchange / piece combine
-  unsigned long long full[kConsumerWarps][Cfg<D>::NST];
-  unsigned long long qfull[Cfg<D>::NQ];
+  uint16_t kv[kConsumerWarps][C::NST][2][kSubKeys * D];
+  float q[C::NQ][C::GD];              // queries of the upcoming pieces (heads >= G unused)
+  float wbuf[kConsumerWarps][C::WB];  // weights exchange / piece combine
+  unsigned long long full[kConsumerWarps][C::NST];
+  unsigned long long qfull[C::NQ];
   unsigned long long csync;
   unsigned long long rfull;          // reused ring state of the current whole-unit piece landed
   int abort_flag;
   int last_flag;
   int box_total;                     // boxes consumed by all warps (rate record)
   Segment items[kItemCache];         // the CTA's work items, from its first one on
-  alignas(16) float ring[Cfg<D>::GD + 2 * kGroup];  // that ring state: o [G][D], m [G], l [G]
+  alignas(16) float ring[C::SF];     // that ring state: o [G][D], then m at GD, l at GD + GP
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -198,32 +208,56 @@ __device__ __forceinline__ uint32_t box_off(int row, int dim) {
                     (dim & 7) * 2);
 }
 
+// The group size: GF when the kernel is built for one group size (4 or 8),
+// else the run-time value (padded to GP in registers and shared memory).
+template <int GF>
+__device__ __forceinline__ int group_of(const AttendParams& p) {
+  return GF > 0 ? GF : p.G;
+}
+// m and l of a ring entry are G-float runs at a multiple of G floats: bulk
+// copies need 16-byte runs, so only groups of 4 and 8 move them that way.
+template <int GF>
+constexpr bool kBulkML = GF > 0 && GF % 4 == 0;
+
 // ------------------------------------------------------------ consumer state
 // Per warp, in mma fragment layout (lane = 4*gid + tig): the query columns
 // as B fragments, O^T as C fragments (dims 16*dt + gid and + 8, columns
 // 2*tig and 2*tig + 1), and the running max and sum of the two heads this
-// lane's columns belong to, hh = 2*(tig & 1) and hh + 1.
-template <int D>
+// lane's columns belong to, hh and hh + 1 (GP = 4: hh = 2*(tig & 1);
+// GP = 8: hh = 2*tig).
+template <int D, int GP>
 struct Acc {
-  uint32_t qb[Cfg<D>::KS][2];
-  float o[Cfg<D>::KS][4];
+  uint32_t qb[Cfg<D, GP>::KS][Cfg<D, GP>::QW];
+  float o[Cfg<D, GP>::KS][4];
   float m[2];
   float l[2];
 };
 
-// Load the query of a piece into B fragments: column n = gid is head
-// (gid & 3), its bf16 high part for gid < 4 and its bf16 residual otherwise.
-template <int D>
-__device__ __forceinline__ void load_query(Acc<D>& A, const float* qs) {
+// Load the query of a piece into B fragments.  GP = 4: column n = gid is
+// head (gid & 3), its bf16 high part for gid < 4 and its bf16 residual
+// otherwise.  GP = 8: column n = gid is head gid; qb[ks][0..1] hold the high
+// parts, qb[ks][2..3] the residuals.  Heads >= G are zero columns.
+template <int D, int GP>
+__device__ __forceinline__ void load_query(Acc<D, GP>& A, const float* qs, int G) {
   const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-  const float* qh = qs + (gid & 3) * D + 2 * tig;
+  const int head = GP == 4 ? (gid & 3) : gid;
+  const bool live = head < G;
+  const float* qh = qs + head * D + 2 * tig;
 #pragma unroll
-  for (int ks = 0; ks < Cfg<D>::KS; ++ks) {
-    const float2 x01 = *reinterpret_cast<const float2*>(qh + ks * 16);
-    const float2 x89 = *reinterpret_cast<const float2*>(qh + ks * 16 + 8);
+  for (int ks = 0; ks < Cfg<D, GP>::KS; ++ks) {
+    const float2 z = make_float2(0.f, 0.f);
+    const float2 x01 = live ? *reinterpret_cast<const float2*>(qh + ks * 16) : z;
+    const float2 x89 = live ? *reinterpret_cast<const float2*>(qh + ks * 16 + 8) : z;
     const uint32_t h0 = pack_bf16(x01.x, x01.y), h1 = pack_bf16(x89.x, x89.y);
-    A.qb[ks][0] = gid < 4 ? h0 : pack_bf16_residual(x01.x, x01.y, h0);
-    A.qb[ks][1] = gid < 4 ? h1 : pack_bf16_residual(x89.x, x89.y, h1);
+    if constexpr (GP == 4) {
+      A.qb[ks][0] = gid < 4 ? h0 : pack_bf16_residual(x01.x, x01.y, h0);
+      A.qb[ks][1] = gid < 4 ? h1 : pack_bf16_residual(x89.x, x89.y, h1);
+    } else {
+      A.qb[ks][0] = h0;
+      A.qb[ks][1] = h1;
+      A.qb[ks][2] = pack_bf16_residual(x01.x, x01.y, h0);
+      A.qb[ks][3] = pack_bf16_residual(x89.x, x89.y, h1);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) A.o[ks][i] = 0.f;
   }
@@ -235,36 +269,42 @@ __device__ __forceinline__ void load_query(Acc<D>& A, const float* qs) {
 // rows outside [k0, k1): their scores become -inf and their V rows are
 // zeroed in shared memory (the rows may hold anything, NaN included, and
 // 0 * NaN would poison the sum).
-template <int D>
-__device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, uint16_t* vbox, float* pbuf,
+template <int D, int GP>
+__device__ __forceinline__ void process_box(Acc<D, GP>& A, const uint16_t* kbox, uint16_t* vbox, float* pbuf,
                                             int key_box, int k0, int k1, bool masked) {
-  constexpr int KS = Cfg<D>::KS;
+  constexpr int KS = Cfg<D, GP>::KS;
   const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
   const int mj = lane >> 3, mr = lane & 7;  // ldmatrix: matrix and row this lane addresses
   const uint32_t kb = smem_u32(kbox), vb = smem_u32(vbox);
 
-  // S^T = K . Qx, two accumulator chains
+  // S^T = K . Qx, two accumulator chains (GP = 4: alternate k-steps;
+  // GP = 8: high parts into s, residuals into t)
   float s[4] = {0.f, 0.f, 0.f, 0.f}, t[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     uint32_t a0, a1, a2, a3;
     ldsm_x4(kb + box_off(mr + ((mj & 1) << 3), ks * 16 + ((mj >> 1) << 3)), a0, a1, a2, a3);
-    mma16816((ks & 1) ? t : s, a0, a1, a2, a3, A.qb[ks][0], A.qb[ks][1]);
+    if constexpr (GP == 4) {
+      mma16816((ks & 1) ? t : s, a0, a1, a2, a3, A.qb[ks][0], A.qb[ks][1]);
+    } else {
+      mma16816(s, a0, a1, a2, a3, A.qb[ks][0], A.qb[ks][1]);
+      mma16816(t, a0, a1, a2, a3, A.qb[ks][2], A.qb[ks][3]);
+    }
   }
-  // high + residual columns: lane tig and tig ^ 2 hold columns n and n + 4.
-  // sc = (key gid, head hh), (gid, hh + 1), (gid + 8, hh), (gid + 8, hh + 1)
+  // sc = (key gid, head hh), (gid, hh + 1), (gid + 8, hh), (gid + 8, hh + 1);
+  // GP = 4: lanes tig and tig ^ 2 hold the high and residual columns
   float sc[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     sc[i] = s[i] + t[i];
-    sc[i] += __shfl_xor_sync(kFull, sc[i], 2);
+    if constexpr (GP == 4) sc[i] += __shfl_xor_sync(kFull, sc[i], 2);
   }
   if (masked) {
     const int ka = key_box + gid, kc = ka + 8;
     if (ka < k0 || ka >= k1) sc[0] = sc[1] = -INFINITY;
     if (kc < k0 || kc >= k1) sc[2] = sc[3] = -INFINITY;
     // zero whole V rows (both halves) outside the range
-    for (int i = lane; i < Cfg<D>::HALVES * kSubKeys * 8; i += 32) {
+    for (int i = lane; i < Cfg<D, GP>::HALVES * kSubKeys * 8; i += 32) {
       const int row = (i >> 3) & (kSubKeys - 1);
       if (key_box + row < k0 || key_box + row >= k1) reinterpret_cast<uint4*>(vbox)[i] = make_uint4(0u, 0u, 0u, 0u);
     }
@@ -296,32 +336,45 @@ __device__ __forceinline__ void process_box(Acc<D>& A, const uint16_t* kbox, uin
   const float p0 = ex2(sc[0] - mu0), p1 = ex2(sc[1] - mu1), p2 = ex2(sc[2] - mu0), p3 = ex2(sc[3] - mu1);
   A.l[0] += p0 + p2;
   A.l[1] += p1 + p3;
-  // weights P[key][head] through shared memory into the B fragments of Px:
-  // b0 = keys 2*tig, 2*tig + 1; b1 = keys 2*tig + 8, + 9; column gid
-  const int hh = 2 * (tig & 1);
-  if (tig < 2) {
-    *reinterpret_cast<float2*>(pbuf + gid * 4 + hh) = make_float2(p0, p1);
-    *reinterpret_cast<float2*>(pbuf + (gid + 8) * 4 + hh) = make_float2(p2, p3);
+  // weights P[key][head] ([16][GP] floats) through shared memory into the
+  // B fragments of Px: b0 = keys 2*tig, 2*tig + 1; b1 = keys 2*tig + 8, + 9;
+  // column gid
+  const int hh = GP == 4 ? 2 * (tig & 1) : 2 * tig;
+  if (GP == 8 || tig < 2) {
+    *reinterpret_cast<float2*>(pbuf + gid * GP + hh) = make_float2(p0, p1);
+    *reinterpret_cast<float2*>(pbuf + (gid + 8) * GP + hh) = make_float2(p2, p3);
   }
   __syncwarp();
-  const int hc = gid & 3;
-  const float x0 = pbuf[(2 * tig) * 4 + hc], x1 = pbuf[(2 * tig + 1) * 4 + hc];
-  const float x2 = pbuf[(2 * tig + 8) * 4 + hc], x3 = pbuf[(2 * tig + 9) * 4 + hc];
+  const int hc = GP == 4 ? (gid & 3) : gid;
+  const float x0 = pbuf[(2 * tig) * GP + hc], x1 = pbuf[(2 * tig + 1) * GP + hc];
+  const float x2 = pbuf[(2 * tig + 8) * GP + hc], x3 = pbuf[(2 * tig + 9) * GP + hc];
   const uint32_t h0 = pack_bf16(x0, x1), h1 = pack_bf16(x2, x3);
-  const uint32_t pb0 = gid < 4 ? h0 : pack_bf16_residual(x0, x1, h0);
-  const uint32_t pb1 = gid < 4 ? h1 : pack_bf16_residual(x2, x3, h1);
-  // O^T += V^T . Px, one row tile of 16 dims per mma
+  // O^T += V^T . Px, one row tile of 16 dims per mma (GP = 8: the high and
+  // the residual weights, two products into the same accumulator)
+  if constexpr (GP == 4) {
+    const uint32_t pb0 = gid < 4 ? h0 : pack_bf16_residual(x0, x1, h0);
+    const uint32_t pb1 = gid < 4 ? h1 : pack_bf16_residual(x2, x3, h1);
 #pragma unroll
-  for (int dt = 0; dt < KS; ++dt) {
-    uint32_t a0, a1, a2, a3;
-    ldsm_x4_t(vb + box_off(mr + ((mj >> 1) << 3), dt * 16 + ((mj & 1) << 3)), a0, a1, a2, a3);
-    mma16816(A.o[dt], a0, a1, a2, a3, pb0, pb1);
+    for (int dt = 0; dt < KS; ++dt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(vb + box_off(mr + ((mj >> 1) << 3), dt * 16 + ((mj & 1) << 3)), a0, a1, a2, a3);
+      mma16816(A.o[dt], a0, a1, a2, a3, pb0, pb1);
+    }
+  } else {
+    const uint32_t r0 = pack_bf16_residual(x0, x1, h0), r1 = pack_bf16_residual(x2, x3, h1);
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(vb + box_off(mr + ((mj >> 1) << 3), dt * 16 + ((mj & 1) << 3)), a0, a1, a2, a3);
+      mma16816(A.o[dt], a0, a1, a2, a3, h0, h1);
+      mma16816(A.o[dt], a0, a1, a2, a3, r0, r1);
+    }
   }
 }
 
 // Bounded barrier of the 8 consumer warps (mbarrier with one arrival per warp).
-template <int D>
-__device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, unsigned* status) {
+template <int D, int GP>
+__device__ __forceinline__ bool consumer_sync(AttnSmem<D, GP>& sm, uint32_t& phase, unsigned* status) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.csync);
   const bool ok = mbar_wait(&sm.csync, phase, &sm.abort_flag, status);
@@ -330,9 +383,9 @@ __device__ __forceinline__ bool consumer_sync(AttnSmem<D>& sm, uint32_t& phase, 
   return ok;
 }
 
-template <int D>
-__device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, int idx, int h, float& MA, float& LA,
-                                               float& OA, float& MB, float& LB, float& OB);
+template <int D, int GP, int NH>
+__device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA, int idx, int h, float& MA,
+                                               float& LA, float& OA, float& MB, float& LB, float& OB);
 
 // Fold one state (max m, sum l, outputs o relative to 2^m) into (M, L, O).
 template <int N>
@@ -349,107 +402,114 @@ __device__ __forceinline__ void fold_state(float& M, float& L, float (&O)[N], fl
 // Last arriver of a split unit: merge its partials.  Segment A's partials
 // (with the reused state on a hit) give the new prefix state over [0, c_t),
 // stored in the ring; that state and segment B's partials give the output.
-// The 8 warps share the partials (warp w folds partials w, w + 8, ..., each
-// lane FPL consecutive floats of one head), with up to 48 partials' loads in
-// flight at once; the warps' states then meet in shared memory.
-template <int D>
-__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, int u, uint32_t& sync_phase) {
-  constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
-  constexpr int FPL = GD / 32, F4 = FPL / 4;  // floats and float4 of a partial per lane
-  constexpr int BP = 6;                       // partials per warp per round of loads
-  constexpr int VEC = GD / (kConsumerWarps * 32);
-  static_assert(VEC * kConsumerWarps * 32 == GD && F4 * 4 * 32 == GD, "merge layout");
+// Four heads at a time: the 8 warps share the partials (warp w folds
+// partials w, w + 8, ..., each lane FPL consecutive floats of one head), with
+// up to 48 partials' loads in flight at once; the warps' states then meet in
+// shared memory.
+template <int D, int GP, int GF>
+__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
+  constexpr int QD = 4 * D;                    // floats of four heads
+  constexpr int FPL = QD / 32, F4 = FPL / 4;   // floats and float4 of those per lane
+  constexpr int BP = 6;                        // partials per warp per round of loads
+  constexpr int VEC = QD / (kConsumerWarps * 32);
+  static_assert(VEC * kConsumerWarps * 32 == QD && F4 * 4 * 32 == QD, "merge layout");
+  const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
   const UnitPlan pl = p.plan[u];
   const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
   const int nA = sA.npieces, n = nA + sB.npieces;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f0 = lane * FPL, hl = f0 / D;
-
-  float MA = -INFINITY, LA = 0.f, OA[FPL], MB = -INFINITY, LB = 0.f, OB[FPL];
-#pragma unroll
-  for (int j = 0; j < FPL; ++j) OA[j] = OB[j] = 0.f;
-  if (warp == 0 && pl.hit) {  // the reused state joins set A (its o is normalised)
-    const size_t rs = (size_t)u * Wp1 + pl.src_slot;
-    const float rl = __ldcg(p.ring_l + rs * G + hl), rm = __ldcg(p.ring_m + rs * G + hl) * kLog2e;
-    float o[FPL];
-#pragma unroll
-    for (int f = 0; f < F4; ++f) {
-      const float4 t = __ldcg(reinterpret_cast<const float4*>(p.ring_o + rs * GD + f0) + f);
-      o[4 * f] = t.x * rl;
-      o[4 * f + 1] = t.y * rl;
-      o[4 * f + 2] = t.z * rl;
-      o[4 * f + 3] = t.w * rl;
-    }
-    fold_state<FPL>(MA, LA, OA, rm, rl, o);
-  }
-  for (int i0 = warp; i0 < n; i0 += kConsumerWarps * BP) {
-    float4 v[BP][F4];
-    float mv[BP], lv[BP];
-#pragma unroll
-    for (int k = 0; k < BP; ++k) {
-      const int i = i0 + k * kConsumerWarps;
-      if (i < n) {
-        const float* pp = p.part + (size_t)(i < nA ? sA.pbase + i : sB.pbase + (i - nA)) * PF;
-#pragma unroll
-        for (int f = 0; f < F4; ++f) v[k][f] = __ldcg(reinterpret_cast<const float4*>(pp + f0) + f);
-        mv[k] = __ldcg(pp + GD + hl);
-        lv[k] = __ldcg(pp + GD + G + hl);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < BP; ++k) {
-      const int i = i0 + k * kConsumerWarps;
-      if (i < n) {
-        const float* o = reinterpret_cast<const float*>(v[k]);
-        if (i < nA)
-          fold_state<FPL>(MA, LA, OA, mv[k], lv[k], o);
-        else
-          fold_state<FPL>(MB, LB, OB, mv[k], lv[k], o);
-      }
-    }
-  }
-  // the warps' sets meet in shared memory: set A (prefix), then set B (tail)
-  float PM[VEC], PL[VEC], PO[VEC], QM[VEC], QL[VEC], QO[VEC];
+  const size_t rs = (size_t)u * Wp1 + pl.src_slot, ds = (size_t)u * Wp1 + pl.dst_slot;
   float* wb = sm.wbuf[warp];
+
+  for (int h0 = 0; h0 < G; h0 += 4) {
+    const int f0 = lane * FPL, hq = f0 / D, hl = h0 + hq;  // this lane's head
+    const bool live = hl < G;
+    const int fo = h0 * D + f0;                         // its first float in a partial's o
+    float MA = -INFINITY, LA = 0.f, OA[FPL], MB = -INFINITY, LB = 0.f, OB[FPL];
 #pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
+    for (int j = 0; j < FPL; ++j) OA[j] = OB[j] = 0.f;
+    if (warp == 0 && pl.hit && live) {  // the reused state joins set A (its o is normalised)
+      const float rl = __ldcg(p.ring_l + rs * G + hl), rm = __ldcg(p.ring_m + rs * G + hl) * kLog2e;
+      float o[FPL];
 #pragma unroll
-    for (int j = 0; j < FPL; ++j) wb[f0 + j] = pass == 0 ? OA[j] : OB[j];
-    if (f0 - hl * D == 0) {
-      wb[GD + hl] = pass == 0 ? MA : MB;
-      wb[GD + G + hl] = pass == 0 ? LA : LB;
+      for (int f = 0; f < F4; ++f) {
+        const float4 t = __ldcg(reinterpret_cast<const float4*>(p.ring_o + rs * GD + fo) + f);
+        o[4 * f] = t.x * rl;
+        o[4 * f + 1] = t.y * rl;
+        o[4 * f + 2] = t.z * rl;
+        o[4 * f + 3] = t.w * rl;
+      }
+      fold_state<FPL>(MA, LA, OA, rm, rl, o);
     }
-    if (!consumer_sync(sm, sync_phase, p.status)) return false;
+    for (int i0 = warp; i0 < n && live; i0 += kConsumerWarps * BP) {
+      float4 v[BP][F4];
+      float mv[BP], lv[BP];
+#pragma unroll
+      for (int k = 0; k < BP; ++k) {
+        const int i = i0 + k * kConsumerWarps;
+        if (i < n) {
+          const float* pp = p.part + (size_t)(i < nA ? sA.pbase + i : sB.pbase + (i - nA)) * PF;
+#pragma unroll
+          for (int f = 0; f < F4; ++f) v[k][f] = __ldcg(reinterpret_cast<const float4*>(pp + fo) + f);
+          mv[k] = __ldcg(pp + GD + hl);
+          lv[k] = __ldcg(pp + GD + G4 + hl);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < BP; ++k) {
+        const int i = i0 + k * kConsumerWarps;
+        if (i < n) {
+          const float* o = reinterpret_cast<const float*>(v[k]);
+          if (i < nA)
+            fold_state<FPL>(MA, LA, OA, mv[k], lv[k], o);
+          else
+            fold_state<FPL>(MB, LB, OB, mv[k], lv[k], o);
+        }
+      }
+    }
+    // the warps' sets meet in shared memory ([4][D], m [4], l [4]): set A
+    // (prefix), then set B (tail)
+    float PM[VEC], PL[VEC], PO[VEC], QM[VEC], QL[VEC], QO[VEC];
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+      for (int j = 0; j < FPL; ++j) wb[f0 + j] = pass == 0 ? OA[j] : OB[j];
+      if (f0 - hq * D == 0) {
+        wb[QD + hq] = pass == 0 ? MA : MB;
+        wb[QD + 4 + hq] = pass == 0 ? LA : LB;
+      }
+      if (!consumer_sync(sm, sync_phase, p.status)) return false;
+#pragma unroll
+      for (int j = 0; j < VEC; ++j) {
+        const int idx = threadIdx.x * VEC + j;
+        float m_, l_, o_, xm, xl, xo;
+        combine_warps2<D, GP, 4>(sm, kConsumerWarps, idx, idx / D, m_, l_, o_, xm, xl, xo);
+        if (pass == 0) {
+          PM[j] = m_, PL[j] = l_, PO[j] = o_;
+        } else {
+          QM[j] = m_, QL[j] = l_, QO[j] = o_;
+        }
+      }
+      if (!consumer_sync(sm, sync_phase, p.status)) return false;
+    }
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
-      const int idx = threadIdx.x * VEC + j;
-      float m_, l_, o_, xm, xl, xo;
-      combine_warps2<D>(sm, kConsumerWarps, idx, idx / D, m_, l_, o_, xm, xl, xo);
-      if (pass == 0) {
-        PM[j] = m_, PL[j] = l_, PO[j] = o_;
-      } else {
-        QM[j] = m_, QL[j] = l_, QO[j] = o_;
+      const int idx = threadIdx.x * VEC + j, h = h0 + idx / D, d = idx - (idx / D) * D;
+      if (h >= G) continue;
+      p.ring_o[ds * GD + (size_t)h * D + d] = PL[j] > 0.f ? PO[j] / PL[j] : 0.f;
+      const float M2 = fmaxf(PM[j], QM[j]);
+      const float M2u = M2 == -INFINITY ? 0.f : M2;
+      const float a0 = ex2(PM[j] - M2u), a1 = ex2(QM[j] - M2u);
+      const float L2 = PL[j] * a0 + QL[j] * a1;
+      const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+      p.out[orow * D + d] = (PO[j] * a0 + QO[j] * a1) / L2;
+      if (d == 0) {
+        p.ring_m[ds * G + h] = PL[j] > 0.f ? PM[j] * kLn2 : -INFINITY;
+        p.ring_l[ds * G + h] = PL[j];
+        p.lse[orow] = (M2 + log2f(L2)) * kLn2;
       }
-    }
-    if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  }
-  const size_t ds = (size_t)u * Wp1 + pl.dst_slot;
-#pragma unroll
-  for (int j = 0; j < VEC; ++j) {
-    const int idx = threadIdx.x * VEC + j, h = idx / D, d = idx - h * D;
-    p.ring_o[ds * GD + idx] = PL[j] > 0.f ? PO[j] / PL[j] : 0.f;
-    const float M2 = fmaxf(PM[j], QM[j]);
-    const float M2u = M2 == -INFINITY ? 0.f : M2;
-    const float a0 = ex2(PM[j] - M2u), a1 = ex2(QM[j] - M2u);
-    const float L2 = PL[j] * a0 + QL[j] * a1;
-    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
-    p.out[orow * D + d] = (PO[j] * a0 + QO[j] * a1) / L2;
-    if (d == 0) {
-      p.ring_m[ds * G + h] = PL[j] > 0.f ? PM[j] * kLn2 : -INFINITY;
-      p.ring_l[ds * G + h] = PL[j];
-      p.lse[orow] = (M2 + log2f(L2)) * kLn2;
     }
   }
   if (threadIdx.x == 0) {
@@ -459,14 +519,15 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D>& sm, 
   return true;
 }
 
-// Store the warp's state in its shared-memory slot: o [G][D] unnormalised,
-// then m [G] and l [G].  Lanes tig and tig ^ 2 hold the high and residual
-// columns of the same heads; lanes of one tig hold different key rows.
-template <int D>
-__device__ __forceinline__ void warp_combine_store(Acc<D>& A, float* wb) {
-  constexpr int G = kGroup, GD = Cfg<D>::GD, KS = Cfg<D>::KS;
+// Store the warp's state in its shared-memory slot: o [GP][D] unnormalised,
+// then m [GP] and l [GP].  GP = 4: lanes tig and tig ^ 2 hold the high and
+// residual columns of the same heads.  Lanes of one tig hold different key
+// rows for l.
+template <int D, int GP>
+__device__ __forceinline__ void warp_combine_store(Acc<D, GP>& A, float* wb) {
+  constexpr int GD = Cfg<D, GP>::GD, KS = Cfg<D, GP>::KS;
   const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
-  const int hh = 2 * (tig & 1);
+  const int hh = GP == 4 ? 2 * (tig & 1) : 2 * tig;
   __syncwarp();
   float l0 = A.l[0], l1 = A.l[1];
 #pragma unroll
@@ -474,11 +535,13 @@ __device__ __forceinline__ void warp_combine_store(Acc<D>& A, float* wb) {
     l0 += __shfl_xor_sync(kFull, l0, off);
     l1 += __shfl_xor_sync(kFull, l1, off);
   }
+  if constexpr (GP == 4) {
 #pragma unroll
-  for (int dt = 0; dt < KS; ++dt)
+    for (int dt = 0; dt < KS; ++dt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) A.o[dt][i] += __shfl_xor_sync(kFull, A.o[dt][i], 2);
-  if (tig < 2) {
+      for (int i = 0; i < 4; ++i) A.o[dt][i] += __shfl_xor_sync(kFull, A.o[dt][i], 2);
+  }
+  if (GP == 8 || tig < 2) {
 #pragma unroll
     for (int dt = 0; dt < KS; ++dt) {
       const int d0 = dt * 16 + gid;
@@ -490,23 +553,23 @@ __device__ __forceinline__ void warp_combine_store(Acc<D>& A, float* wb) {
     if (gid == 0) {
       wb[GD + hh] = A.m[0];
       wb[GD + hh + 1] = A.m[1];
-      wb[GD + G + hh] = l0;
-      wb[GD + G + hh + 1] = l1;
+      wb[GD + GP + hh] = l0;
+      wb[GD + GP + hh + 1] = l1;
     }
   }
 }
 
-// Merge the warps' states for output element idx of head h: warps below wA
-// into (MA, LA, OA), the others into (MB, LB, OB); sums relative to 2^M.
-template <int D>
-__device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, int idx, int h, float& MA, float& LA,
-                                               float& OA, float& MB, float& LB, float& OB) {
-  constexpr int G = kGroup, GD = Cfg<D>::GD;
+// Merge the warps' states for element idx of head h, from slots laid out as
+// o [NH][D], m [NH], l [NH]: warps below wA into (MA, LA, OA), the others
+// into (MB, LB, OB); sums relative to 2^M.
+template <int D, int GP, int NH>
+__device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA, int idx, int h, float& MA,
+                                               float& LA, float& OA, float& MB, float& LB, float& OB) {
   float m[kConsumerWarps], l[kConsumerWarps], o[kConsumerWarps];
 #pragma unroll
   for (int w = 0; w < kConsumerWarps; ++w) {
-    m[w] = sm.wbuf[w][GD + h];
-    l[w] = sm.wbuf[w][GD + G + h];
+    m[w] = sm.wbuf[w][NH * D + h];
+    l[w] = sm.wbuf[w][NH * D + NH + h];
     o[w] = sm.wbuf[w][idx];
   }
   MA = MB = -INFINITY;
@@ -532,21 +595,21 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D>& sm, int wA, in
 
 // End of a split piece: combine the 8 warps, write the partial, count it
 // and, if it was the unit's last, merge the unit.
-template <int D>
-__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int unit, int pidx,
+template <int D, int GP, int GF>
+__device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D, GP>& A, int unit, int pidx,
                                uint32_t& sync_phase) {
-  constexpr int G = kGroup, GD = Cfg<D>::GD, PF = Cfg<D>::PF;
-  warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
+  const int G = group_of<GF>(p), GD = G * D, G4 = group4(G);
+  warp_combine_store<D, GP>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  float* dst = p.part + (size_t)pidx * PF;
+  float* dst = p.part + (size_t)pidx * (GD + 2 * G4);
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
     const int h = idx / D;
     float MA, LA, OA, M, L, O;
-    combine_warps2<D>(sm, 0, idx, h, MA, LA, OA, M, L, O);
+    combine_warps2<D, GP, GP>(sm, 0, idx, h, MA, LA, OA, M, L, O);
     dst[idx] = O;
     if (idx - h * D == 0) {
       dst[GD + h] = M;
-      dst[GD + G + h] = L;
+      dst[GD + G4 + h] = L;
     }
   }
   // every thread's partial stores happen-before thread 0's fence through the
@@ -560,7 +623,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
-    return merge_unit<D>(p, sm, unit, sync_phase);
+    return merge_unit<D, GP, GF>(p, sm, unit, sync_phase);
   }
   return true;
 }
@@ -568,16 +631,21 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A
 // End of a whole-unit piece: warps [0, wA) hold the amend range [start, c_t),
 // warps [wA, 8) the tail [c_t, p_t].  New prefix state = reused ring state
 // (on a hit) + amend; output = new prefix + tail.  No partials, no counters.
-template <int D>
-__device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A, int u, int wA, int hit,
-                              int dst, int end, uint32_t ring_phase, uint32_t& sync_phase) {
-  constexpr int G = kGroup, GD = Cfg<D>::GD;
+// On a hit, the reused m and l come with o by bulk copy when GF is a multiple
+// of 4 (16-byte runs), else thread t < 2G brings m (t < G) or l in rml.
+template <int D, int GP, int GF>
+__device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D, GP>& A, int u, int wA, int hit,
+                              int dst, int end, float rml, uint32_t ring_phase, uint32_t& sync_phase) {
+  constexpr int GDP = Cfg<D, GP>::GD;
+  const int G = group_of<GF>(p), GD = G * D;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
-  constexpr int PER = (GD + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
-  warp_combine_store<D>(A, sm.wbuf[threadIdx.x >> 5]);
+  constexpr int PER = (GDP + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
+  warp_combine_store<D, GP>(A, sm.wbuf[threadIdx.x >> 5]);
+  if (!kBulkML<GF> && hit && (int)threadIdx.x < 2 * G)
+    sm.ring[GDP + ((int)threadIdx.x < G ? (int)threadIdx.x : GP + (int)threadIdx.x - G)] = rml;
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  // the reused state was copied on chip at the start of the piece
+  // the reused o was copied on chip at the start of the piece
   if (hit && !mbar_wait(&sm.rfull, ring_phase, &sm.abort_flag, p.status)) return false;
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
@@ -585,15 +653,15 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D>& sm, Acc<D>& A,
     if (idx >= GD) break;
     const int h = idx / D, d = idx - h * D;
     float MA, LA, OA, MB, LB, OB;
-    combine_warps2<D>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
+    combine_warps2<D, GP, GP>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
     // new prefix state S = reused (hit) + amend
-    const float rm = hit ? sm.ring[GD + h] * kLog2e : -INFINITY;
+    const float rm = hit ? sm.ring[GDP + h] * kLog2e : -INFINITY;
     float M = fmaxf(MA, rm);
     const float Mu = M == -INFINITY ? 0.f : M;
     const float aA = ex2(MA - Mu);
     float L = LA * aA, O = OA * aA;
     if (hit) {
-      const float a = ex2(rm - Mu), rl = sm.ring[GD + kGroup + h];
+      const float a = ex2(rm - Mu), rl = sm.ring[GDP + GP + h];
       L += rl * a;
       O += sm.ring[idx] * rl * a;
     }
@@ -752,14 +820,17 @@ __device__ __noinline__ void rate_shares(const AttendParams& p) {
   if (tid == 0) p.cw[G] = 1.0;
 }
 
-template <int D>
+template <int D, int GP, int GF>
 __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
-  constexpr int NST = Cfg<D>::NST, NQ = Cfg<D>::NQ, GD = Cfg<D>::GD;
+  using C = Cfg<D, GP>;
+  constexpr int NST = C::NST, NQ = C::NQ;
   constexpr uint32_t kBoxBytes = kSubKeys * D * 2;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // the swizzled TMA boxes need 1024-byte alignment of the shared window
-  AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  AttnSmem<D, GP>& sm =
+      *reinterpret_cast<AttnSmem<D, GP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = group_of<GF>(p), GD = G * D;  // real group: global layouts
 
   const int cta = blockIdx.x;
   if (tid == 32) {  // bring both TMA descriptors on chip while the match kernel runs
@@ -853,7 +924,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
       mbar_arrive_expect_tx(&sm.full[warp][st], 2 * kBoxBytes);
 #pragma unroll
-      for (int hf = 0; hf < Cfg<D>::HALVES; ++hf) {
+      for (int hf = 0; hf < C::HALVES; ++hf) {
         tma_load_4d(sm.kv[warp][st][0] + hf * kSubKeys * 64, &p.tmK, &sm.full[warp][st], 64 * hf, kvh, c2, c3, pol);
         tma_load_4d(sm.kv[warp][st][1] + hf * kSubKeys * 64, &p.tmV, &sm.full[warp][st], 64 * hf, kvh, c2, c3, pol);
       }
@@ -867,7 +938,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   for (int k = 0; k < NST && ivalid; ++k) issue_box(k);
 
   // consume cursor
-  Acc<D> A;
+  Acc<D, GP> A;
   Walker wc{first_seg, lo, hi, sm.items, first_seg};
   Piece cp;
   int cpn = 0, cons = 0, par = 0;
@@ -878,18 +949,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   while (ok && wc.next(p, slot, cp)) {
     const int qs = cpn % NQ;
     if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
-    load_query<D>(A, sm.q[qs]);
+    load_query<D, GP>(A, sm.q[qs], G);
     const bool ring_copy = cp.whole && cp.hit;
     ring_pending = ring_copy;
-    if (ring_copy && tid == 0) {
+    float rml = 0.f;  // m (thread t < G) or l (G <= t < 2G) of the reused state
+    if (ring_copy) {
       // the merge at the end of the piece reads the reused ring state: copy
-      // it on chip now (the previous piece's merge is done with the buffer)
+      // its o on chip now (the previous piece's merge is done with the
+      // buffer); m and l travel in registers
       const size_t rs = (size_t)cp.unit * (p.W + 1) + cp.src;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(&sm.rfull, (GD + 2 * kGroup) * 4);
-      bulk_load(sm.ring, p.ring_o + rs * GD, GD * 4, &sm.rfull);
-      bulk_load(sm.ring + GD, p.ring_m + rs * kGroup, kGroup * 4, &sm.rfull);
-      bulk_load(sm.ring + GD + kGroup, p.ring_l + rs * kGroup, kGroup * 4, &sm.rfull);
+      if (tid == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(&sm.rfull, (kBulkML<GF> ? GD + 2 * G : GD) * 4);
+        bulk_load(sm.ring, p.ring_o + rs * GD, GD * 4, &sm.rfull);
+        if constexpr (kBulkML<GF>) {
+          bulk_load(sm.ring + C::GD, p.ring_m + rs * G, G * 4, &sm.rfull);
+          bulk_load(sm.ring + C::GD + GP, p.ring_l + rs * G, G * 4, &sm.rfull);
+        }
+      }
+      if (!kBulkML<GF> && tid < 2 * G)
+        rml = __ldcg(tid < G ? p.ring_m + rs * G + tid : p.ring_l + rs * G + (tid - G));
     }
     const WarpRange cr = warp_range(cp, warp);
     for (int bj = cr.first; bj < cr.nbox; bj += cr.stride) {
@@ -900,8 +979,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
       if (tid == 0 && cons == 0) t_first = globaltimer();
       const int key_box = cr.kb0 + bj * kSubKeys;
-      float* pbuf = sm.wbuf[warp] + par * 64;
-      process_box<D>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
+      float* pbuf = sm.wbuf[warp] + par * C::PB;
+      process_box<D, GP>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
                      key_box < cr.k0 || key_box + kSubKeys > cr.k1);
       par ^= 1;
       ++cons;
@@ -913,8 +992,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     }
     if (!ok) break;
     if (tid == 0) t_last = globaltimer();
-    const bool fin = cp.whole ? finalize_unit<D>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, ring_phase, sync_phase)
-                              : finalize_piece<D>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    const bool fin = cp.whole ? finalize_unit<D, GP, GF>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, rml,
+                                                         ring_phase, sync_phase)
+                              : finalize_piece<D, GP, GF>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (ring_copy) ring_phase ^= 1u;
     ring_pending = false;
     if (!fin) break;
@@ -960,21 +1040,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
 
 }  // namespace
 
-size_t attend_smem_bytes(int D) {
-  return (D == 128 ? sizeof(AttnSmem<128>) : sizeof(AttnSmem<64>)) + 1024;
+size_t attend_smem_bytes(int D, int G) {
+  const bool g4 = group_pad(G) == 4;
+  if (D == 128) return (g4 ? sizeof(AttnSmem<128, 4>) : sizeof(AttnSmem<128, 8>)) + 1024;
+  return (g4 ? sizeof(AttnSmem<64, 4>) : sizeof(AttnSmem<64, 8>)) + 1024;
 }
 
-cudaError_t attend_prepare(int D) {
-  if (D == 128)
-    return cudaFuncSetAttribute(mac_attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)attend_smem_bytes(128));
-  if (D == 64)
-    return cudaFuncSetAttribute(mac_attend_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)attend_smem_bytes(64));
-  return cudaErrorInvalidValue;
+namespace {
+// Kernel variants: exact groups of 4 and 8 (compile-time G), and groups of
+// 1-3 and 5-7 padded to 4 and 8 (run-time G).
+template <int D, int GP, int GF>
+cudaError_t set_smem() {
+  return cudaFuncSetAttribute(mac_attend_kernel<D, GP, GF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)attend_smem_bytes(D, GP));
+}
+template <int D>
+cudaError_t set_smem_all() {
+  cudaError_t e = set_smem<D, 4, 4>();
+  if (e == cudaSuccess) e = set_smem<D, 4, 0>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 8>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 0>();
+  return e;
+}
+template <int D>
+cudaError_t launch_d(cudaLaunchConfig_t& cfg, const AttendParams& p) {
+  const int G = p.G;
+  cfg.dynamicSmemBytes = attend_smem_bytes(D, G);
+  if (G == 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 4>, p);
+  if (G == 8) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 8>, p);
+  if (G < 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 0>, p);
+  return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 0>, p);
+}
+}  // namespace
+
+cudaError_t attend_prepare(int D, int G) {
+  if ((D != 64 && D != 128) || G < 1 || G > kMaxGroup) return cudaErrorInvalidValue;
+  return D == 128 ? set_smem_all<128>() : set_smem_all<64>();
 }
 
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s) {
+  if ((D != 64 && D != 128) || p.G < 1 || p.G > kMaxGroup) return cudaErrorInvalidValue;
   // Programmatic stream serialization: the kernel may be scheduled while the
   // preceding match kernel drains; it calls griddepcontrol.wait before it
   // reads anything that kernel wrote.
@@ -987,15 +1092,7 @@ cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (D == 128) {
-    cfg.dynamicSmemBytes = attend_smem_bytes(128);
-    return cudaLaunchKernelEx(&cfg, mac_attend_kernel<128>, p);
-  }
-  if (D == 64) {
-    cfg.dynamicSmemBytes = attend_smem_bytes(64);
-    return cudaLaunchKernelEx(&cfg, mac_attend_kernel<64>, p);
-  }
-  return cudaErrorInvalidValue;
+  return D == 128 ? launch_d<128>(cfg, p) : launch_d<64>(cfg, p);
 }
 
 }  // namespace mac

@@ -8,7 +8,7 @@
 
 namespace mac {
 
-constexpr int kGroup = 4;             // query heads per KV head handled by the kernels
+constexpr int kMaxGroup = 8;          // query heads per KV head (G) the kernels handle: 1..8
 constexpr int kSubKeys = 16;          // keys per TMA box (one box never crosses a page)
 constexpr int kConsumerWarps = 8;     // attention warps that compute
 constexpr int kKeysPerStage = 128;    // keys in flight per round of boxes (kConsumerWarps * 16)
@@ -67,9 +67,14 @@ struct PlanHeader {
 // split uses (cw[c] = share of ranges 0..c-1, cw[grid] = 1).
 constexpr long long kWeightMinCost = 4096;
 
+// The kernels hold a query group padded to GP = 4 or 8 heads (the columns of
+// their tensor-core tiles); heads G..GP-1 are zero and never stored.
+__host__ __device__ inline int group_pad(int G) { return G <= 4 ? 4 : 8; }
+// G rounded up to a multiple of 4 (keeps every partial 16-byte aligned).
+__host__ __device__ inline int group4(int G) { return (G + 3) & ~3; }
 // Layout of one partial result: o_acc [G][D] (unnormalised, relative to m),
-// then m [G] (log2 units), l [G].
-__host__ __device__ inline size_t partial_floats(int D) { return (size_t)kGroup * D + 2 * kGroup; }
+// then m [G4] (log2 units) and l [G4], G4 = group4(G).
+__host__ __device__ inline size_t partial_floats(int G, int D) { return (size_t)G * D + 2 * (size_t)group4(G); }
 
 struct MatchParams {
   const float* q_pre;      // [B][Hq][D]
@@ -94,7 +99,7 @@ struct MatchParams {
   int* claim;              // [grid] ranges taken by the attention CTAs (reset here)
   int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
-  int B, Hq, Hkv, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
+  int B, Hq, Hkv, G, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
   float tau;
   int grid;       // CTAs of the attention kernel
   int min_keys;   // minimum cost-space units per attention CTA
@@ -115,7 +120,7 @@ struct AttendParams {
   int* claim;        // [grid]
   float* rate;       // [grid] learned rate per SM, or null
   double* cw;        // [grid + 1] cumulative range shares (written by CTA 0)
-  float* part;       // [max_parts][partial_floats]
+  float* part;       // [max_parts][partial_floats(G, D)]
   int* unit_cnt;     // [U]
   float* ring_o;     // [U][W+1][G][D]
   float* ring_m;     // [U][W+1][G]
@@ -124,7 +129,7 @@ struct AttendParams {
   float* out;        // [B][Hq][D]
   float* lse;        // [B][Hq]
   unsigned* status;
-  int Hq, Hkv, W, page_size, max_pages, nseg, grid;
+  int Hq, Hkv, G, W, page_size, max_pages, nseg, grid;
 };
 
 struct AppendParams {
@@ -142,7 +147,7 @@ struct AppendParams {
 cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s);
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
-cudaError_t attend_prepare(int D);
-size_t attend_smem_bytes(int D);
+cudaError_t attend_prepare(int D, int G);
+size_t attend_smem_bytes(int D, int G);
 
 }  // namespace mac

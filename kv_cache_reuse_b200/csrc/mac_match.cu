@@ -229,11 +229,14 @@ __device__ void build_segments(const MatchParams& p, int U, double cw_c) {
   }
 }
 
-template <int D>
+// GP: the query group padded to 4 or 8 heads (register and shared-memory
+// shapes); the real group G <= GP sets every global layout.  GF = G for the
+// variants built for one group size (4, 8), 0 for a run-time G (p.G).
+template <int D, int GP, int GF>
 __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchParams p) {
-  constexpr int G = kGroup;
-  constexpr int GD = G * D;
-  __shared__ __align__(16) float sq[GD];
+  const int G = GF > 0 ? GF : p.G;
+  const int GD = G * D;
+  __shared__ __align__(16) float sq[GP * D];
   __shared__ float sdist[kMaxWindow];
   __shared__ int spos[kMaxWindow];
   __shared__ int sslot[kMaxWindow];
@@ -254,8 +257,9 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   // Every load below is independent of the others (no slot index waits for
   // the step counter): ring slots are read whole and mapped to ages later.
   constexpr int NW = kMatchThreads / 32;
-  constexpr int BS = 5;            // slots per warp per batch (8 warps x 5 >= W+1 for W <= 39)
-  constexpr int F4 = GD / 4 / 32;  // float4 per lane per slot
+  constexpr int BS = GP == 4 ? 5 : 3;  // slots per warp per batch of loads (8 warps x 5 >= W+1 for W <= 39)
+  constexpr int F4 = GP * D / 4 / 32;  // float4 per lane per slot, at most
+  const int n4 = GD / 4;               // float4 of one slot
   float4 r[BS][F4];
   int rpos[BS];
   auto load_batch = [&](int s0) {
@@ -265,14 +269,15 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
       if (slot < Wp1) {
         const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
 #pragma unroll
-        for (int f = 0; f < F4; ++f) r[k][f] = rq[lane + 32 * f];
+        for (int f = 0; f < F4; ++f)
+          if (lane + 32 * f < n4) r[k][f] = rq[lane + 32 * f];
         rpos[k] = p.ring_pos[(size_t)u * Wp1 + slot];
       }
     }
   };
   load_batch(warp);
   const float4* qsrc = reinterpret_cast<const float4*>(p.q_pre + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
-  for (int i = tid; i < GD / 4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = qsrc[i];
+  for (int i = tid; i < n4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = qsrc[i];
   const int len = p.seq_lens[b];
   const int p_t = len - 1;
   const int n = p.steps[u];
@@ -308,6 +313,7 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
           float acc = 0.f;
 #pragma unroll
           for (int f = 0; f < F4; ++f) {
+            if (lane + 32 * f >= n4) break;
             const float4 q = reinterpret_cast<const float4*>(sq)[lane + 32 * f];
             const float dx = q.x - r[k][f].x, dy = q.y - r[k][f].y, dz = q.z - r[k][f].z, dw = q.w - r[k][f].w;
             acc = fmaf(dx, dx, acc);
@@ -317,7 +323,8 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
           }
           acc = warp_sum(acc);
           if (lane == 0) {
-            sdist[j] = acc * (1.0f / G);
+            // a power-of-two group divides exactly by its reciprocal
+            sdist[j] = (GF == 4 || GF == 8) ? acc * (1.0f / (GF > 0 ? GF : 1)) : __fdiv_rn(acc, (float)G);
             spos[j] = rpos[k];
             sslot[j] = slot;
           }
@@ -399,7 +406,6 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     const double scale = kLog2e / sqrt((double)D);
     for (int i = tid; i < D / 2; i += kMatchThreads) {
       const double sn = rot_sn, cs = rot_cs;
-#pragma unroll
       for (int h = 0; h < G; ++h) {
         const double x = sq[h * D + i], y = sq[h * D + i + D / 2];
         float* dst = p.qrot + ((size_t)u * G + h) * D;
@@ -409,7 +415,7 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     }
     // 5. this step's query enters the ring
     float4* rdst = reinterpret_cast<float4*>(p.ring_q + ((size_t)u * Wp1 + s_plan.dst_slot) * GD);
-    for (int i = tid; i < GD / 4; i += kMatchThreads) rdst[i] = reinterpret_cast<const float4*>(sq)[i];
+    for (int i = tid; i < n4; i += kMatchThreads) rdst[i] = reinterpret_cast<const float4*>(sq)[i];
     if (tid == 0) {
       p.steps[u] = n + 1;
       if (p.hit_mask) p.hit_mask[u] = (uint8_t)s_plan.hit;
@@ -435,17 +441,29 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   if (tid == 0) *p.done = 0;
 }
 
+template <int D>
+void launch_d(const MatchParams& p, int U, cudaStream_t s) {
+  if (p.G == 4)
+    mac_match_kernel<D, 4, 4><<<U, kMatchThreads, 0, s>>>(p);
+  else if (p.G == 8)
+    mac_match_kernel<D, 8, 8><<<U, kMatchThreads, 0, s>>>(p);
+  else if (p.G < 4)
+    mac_match_kernel<D, 4, 0><<<U, kMatchThreads, 0, s>>>(p);
+  else
+    mac_match_kernel<D, 8, 0><<<U, kMatchThreads, 0, s>>>(p);
+}
+
 }  // namespace
 
 cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s) {
   const int U = p.B * p.Hkv;
-  if (D == 128) {
-    mac_match_kernel<128><<<U, kMatchThreads, 0, s>>>(p);
-  } else if (D == 64) {
-    mac_match_kernel<64><<<U, kMatchThreads, 0, s>>>(p);
-  } else {
+  if (p.G < 1 || p.G > kMaxGroup) return cudaErrorInvalidValue;
+  if (D == 128)
+    launch_d<128>(p, U, s);
+  else if (D == 64)
+    launch_d<64>(p, U, s);
+  else
     return cudaErrorInvalidValue;
-  }
   return cudaGetLastError();
 }
 

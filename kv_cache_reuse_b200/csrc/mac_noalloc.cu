@@ -12,8 +12,9 @@
 // array below.  The caller passes the inputs and the outputs; nothing is
 // allocated, freed, or taken from an allocating library routine.
 //
-// Limits: batch * num_kv_heads <= kMaxUnits (64), head_dim 64 or 128, at most
-// kMaxCtas (160) CTAs of the attention kernel.  The array costs about 1 MiB
+// Limits: batch * num_kv_heads <= kMaxUnits (64), batch * num_q_heads <=
+// kMaxQRows (256), head_dim 64 or 128, groups of 1 to 8 query heads, at most
+// kMaxCtas (160) CTAs of the attention kernel.  The array costs about 2 MiB
 // on every GPU that loads the library, for the life of the process.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -31,14 +32,15 @@ using namespace mac;
 namespace {
 
 constexpr int kMaxUnits = 64;
+constexpr int kMaxQRows = 256;  // query heads over the batch (units x G)
 constexpr int kMaxD = 128;
 constexpr int kMaxCtas = 160;
 constexpr int kMaxDevices = 64;
 
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-constexpr size_t kPartFloats = (size_t)kGroup * kMaxD + 2 * kGroup;
+constexpr size_t kPartFloats = (size_t)kMaxGroup * kMaxD + 2 * kMaxGroup;  // partial_floats(G, D) at most
 constexpr size_t kOffQrot = 0;
-constexpr size_t kOffPlan = align256(kOffQrot + (size_t)kMaxUnits * kGroup * kMaxD * 4);
+constexpr size_t kOffPlan = align256(kOffQrot + (size_t)kMaxQRows * kMaxD * 4);
 constexpr size_t kOffSeg = align256(kOffPlan + kMaxUnits * sizeof(UnitPlan));
 constexpr size_t kOffHdr = align256(kOffSeg + 2 * kMaxUnits * sizeof(Segment));
 constexpr size_t kOffFirst = align256(kOffHdr + sizeof(PlanHeader));
@@ -48,10 +50,10 @@ constexpr size_t kOffCnt = align256(kOffPart + (size_t)(kMaxCtas + 2 * kMaxUnits
 constexpr size_t kCntBytes = (2 * kMaxUnits + 2) * 4;
 constexpr size_t kOffInv = align256(kOffCnt + kCntBytes);
 constexpr size_t kOffRingQ = align256(kOffInv + (kMaxD / 2) * 8);
-constexpr size_t kOffRingO = align256(kOffRingQ + (size_t)kMaxUnits * kGroup * kMaxD * 4);
-constexpr size_t kOffRingM = align256(kOffRingO + (size_t)kMaxUnits * kGroup * kMaxD * 4);
-constexpr size_t kOffRingL = align256(kOffRingM + kMaxUnits * kGroup * 4);
-constexpr size_t kOffRingPos = align256(kOffRingL + kMaxUnits * kGroup * 4);
+constexpr size_t kOffRingO = align256(kOffRingQ + (size_t)kMaxQRows * kMaxD * 4);
+constexpr size_t kOffRingM = align256(kOffRingO + (size_t)kMaxQRows * kMaxD * 4);
+constexpr size_t kOffRingL = align256(kOffRingM + kMaxQRows * 4);
+constexpr size_t kOffRingPos = align256(kOffRingL + kMaxQRows * 4);
 constexpr size_t kScratchBytes = align256(kOffRingPos + kMaxUnits * 4);
 
 // The scratch.  In host code this name is only a stand-in for the symbol;
@@ -105,9 +107,10 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   if (!q_pre || !rope_pos || !K || !V || !seq_lens || !out || !lse) return MAC_ERR_ARG;
   if (!aligned16(q_pre) || !aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
   if (batch < 1 || num_kv_heads < 1 || num_q_heads < 1 || !(rope_theta > 0.0)) return MAC_ERR_ARG;
-  if (num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads != kGroup) return MAC_ERR_SHAPE;
+  if (num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads > kMaxGroup) return MAC_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return MAC_ERR_SHAPE;
-  if ((long long)batch * num_kv_heads > kMaxUnits) return MAC_ERR_SHAPE;  // beyond the static scratch
+  // beyond the static scratch
+  if ((long long)batch * num_kv_heads > kMaxUnits || (long long)batch * num_q_heads > kMaxQRows) return MAC_ERR_SHAPE;
   if (page_size == 0) {
     if (max_seq < 1) return MAC_ERR_ARG;
   } else {
@@ -128,7 +131,8 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
       if (cudaGetSymbolAddress(&ptr, g_mac_static_scratch) != cudaSuccess || !ptr) return MAC_ERR_CUDA;
       int sms = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MAC_ERR_CUDA;
-      if (attend_prepare(64) != cudaSuccess || attend_prepare(128) != cudaSuccess) return MAC_ERR_CUDA;
+      for (int g : {4, 8})
+        if (attend_prepare(64, g) != cudaSuccess || attend_prepare(128, g) != cudaSuccess) return MAC_ERR_CUDA;
       ds->base = static_cast<unsigned char*>(ptr);
       ds->num_sms = sms;
       ds->inv_D = 0;
@@ -181,6 +185,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.B = batch;
   mp.Hq = num_q_heads;
   mp.Hkv = num_kv_heads;
+  mp.G = num_q_heads / num_kv_heads;
   mp.W = 0;
   mp.band = 1 << 30;
   mp.page_size = page_size;
@@ -223,6 +228,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.status = status;
   ap.Hq = num_q_heads;
   ap.Hkv = num_kv_heads;
+  ap.G = num_q_heads / num_kv_heads;
   ap.W = 0;
   ap.page_size = page_size;
   ap.max_pages = max_pages_per_seq;

@@ -66,7 +66,8 @@ def test_init_rejects_bad_config_before_touching_the_device(lib):
     is refused without a GPU."""
     import kv_cache_reuse_b200 as mac
     for kw, code in ((dict(cut_mode=2), mac.MAC_ERR_ARG), (dict(cut_mode=-1), mac.MAC_ERR_ARG),
-                     (dict(band=-1), mac.MAC_ERR_ARG), (dict(num_q_heads=24), mac.MAC_ERR_SHAPE),
+                     (dict(band=-1), mac.MAC_ERR_ARG), (dict(num_q_heads=20), mac.MAC_ERR_SHAPE),
+                     (dict(num_q_heads=72), mac.MAC_ERR_SHAPE),  # 9 query heads per KV head
                      (dict(head_dim=96), mac.MAC_ERR_SHAPE)):
         args = dict(batch=1, num_q_heads=32, num_kv_heads=8, head_dim=128, window=8, band=16, tau=0.1,
                     rope_theta=1e4, max_seq=64)

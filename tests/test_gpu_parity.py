@@ -274,6 +274,49 @@ def test_weighted_split_all_miss():
     assert r["hits"] == 0
 
 
+_SPLIT = {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 64}
+
+
+@pytest.mark.parametrize("case", ["g1_d64", "g1_d128_paged", "g2_split", "g3_paged", "g5_d64", "g6_split",
+                                  "g7_paged", "g8_d64", "g8_d128", "g8_split"])
+def test_group_sizes(case):
+    """Groups of 1 to 8 query heads per KV head (multi-head attention to
+    8-way GQA), whole and split units, contiguous and paged KV."""
+    tiny, llama, paged = synth.WORKLOADS["tiny"], synth.WORKLOADS["llama8b_32k"], synth.WORKLOADS["paged_mixed"]
+    tune = None
+    if case == "g1_d64":
+        wl = tiny.with_(Hq=2, Hkv=2, steps=40)
+    elif case == "g1_d128_paged":
+        wl = paged.with_(B=2, Hq=8, Hkv=8, L0=(3000, 700), steps=16)
+    elif case == "g2_split":
+        wl, tune = tiny.with_(Hq=4, Hkv=2, steps=40), _SPLIT
+    elif case == "g3_paged":
+        wl = paged.with_(B=3, Hq=12, Hkv=4, L0=(2500, 900, 4100), steps=16)
+    elif case == "g5_d64":
+        wl = tiny.with_(Hq=10, Hkv=2, steps=40)
+    elif case == "g6_split":
+        wl, tune = llama.with_(B=2, Hq=12, Hkv=2, L0=(5000, 3100), steps=16), _SPLIT
+    elif case == "g7_paged":  # 28 query heads over 4 KV heads
+        wl = paged.with_(B=3, Hq=28, Hkv=4, L0=(3000, 1200, 6000), steps=16)
+    elif case == "g8_d64":
+        wl = tiny.with_(Hq=8, Hkv=1, steps=40)
+    elif case == "g8_d128":  # 64 query heads over 8 KV heads
+        wl = llama.with_(B=2, Hq=64, Hkv=8, L0=(9000, 4000), steps=24)
+    else:
+        wl, tune = llama.with_(B=2, Hq=16, Hkv=2, L0=(6000, 2000), steps=16), _SPLIT
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tune=tune)
+    assert r["hits"] > 0
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (24, 8), (64, 8)])
+def test_group_sizes_all_miss_large(Hq, Hkv):
+    """Large all-miss steps (weighted split, many partials per unit) for
+    groups of 1, 3 and 8."""
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, Hq=Hq, Hkv=Hkv, L0=(32768, 20000), steps=3)
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=0.0)
+    assert r["hits"] == 0
+
+
 @pytest.mark.parametrize("case", ["tiny", "split", "band0", "llama_paged"])
 def test_cut_mode_band_ends_at_position(case):
     """cut_mode 1: the stored prefix ends at max(0, p + 1 - band) on both sides."""

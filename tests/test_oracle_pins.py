@@ -164,6 +164,34 @@ def test_exact_repeats_without_rotation_equal_dense():
     assert nhit >= 6
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (6, 2), (8, 1)])
+def test_group_sizes_forced_miss_equals_dense(Hq, Hkv):
+    """Groups of 1 (multi-head), 3 and 8 query heads per KV head: a forced
+    miss is dense attention of every query head over its KV head."""
+    wl = _tiny(steps=8, Hq=Hq, Hkv=Hkv)
+    stream, cache, res = _run(wl, tau=0.0)
+    for t, r in enumerate(res):
+        assert r.out.shape == (wl.B, Hq, wl.D) and r.hit.shape == (wl.B, Hkv)
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(3, 3), (10, 2), (8, 1)])
+def test_group_sizes_band_covering_hits_equal_dense(Hq, Hkv):
+    """With the band covering the context, hits reuse an empty prefix: the
+    stored and reused states of every head in the group must come out exact."""
+    wl = _tiny(L0=(40,), steps=16, band=200, Hq=Hq, Hkv=Hkv)
+    stream, cache, res = _run(wl)
+    nhit = 0
+    for t, r in enumerate(res):
+        nhit += int(r.hit.sum())
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+    assert nhit >= 4
+
+
 @pytest.mark.parametrize("cut_mode", [0, 1])
 def test_band_covering_context_equals_dense(cut_mode):
     """band >= p_t + 1 puts every reuse boundary at 0: hits are exact under any RoPE."""
@@ -314,9 +342,10 @@ def _brute_match(window, q, tau, G):
     return False, -1
 
 
-def test_match_equals_brute_force():
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (2, 2), (9, 3), (16, 2)])
+def test_match_equals_brute_force(Hq, Hkv):
     rng = np.random.default_rng(15)
-    B, Hq, Hkv, D, W = 2, 4, 2, 8, 4
+    B, D, W = 2, 8, 4
     G = Hq // Hkv
     orc = oracle.Oracle(B, Hq, Hkv, D, W, 2, 0.5, 1e4, 0, 1 << 10, 0)
     hist = [[[] for _ in range(Hkv)] for _ in range(B)]

@@ -25,6 +25,14 @@ def test_rejects_shapes_beyond_the_static_scratch():
     rc = mac.mac_dense_decode_static(16, 16, 16, 16, None, 16, 16, 16, None, 17, 16, 4, 128, 5e5,
                                      0, 1024, 0, 0, 0)
     assert rc == mac.MAC_ERR_SHAPE
+    # 4 sequences x 72 query heads = 288 query rows > 256
+    rc = mac.mac_dense_decode_static(16, 16, 16, 16, None, 16, 16, 16, None, 4, 72, 9, 128, 5e5,
+                                     0, 1024, 0, 0, 0)
+    assert rc == mac.MAC_ERR_SHAPE
+    # 9 query heads per KV head
+    rc = mac.mac_dense_decode_static(16, 16, 16, 16, None, 16, 16, 16, None, 1, 18, 2, 128, 5e5,
+                                     0, 1024, 0, 0, 0)
+    assert rc == mac.MAC_ERR_SHAPE
 
 
 @pytest.mark.gpu
