@@ -90,6 +90,12 @@ typedef struct MacConfig {
     int cut_mode;          /* where a stored prefix ends, c = max(0, p - band + cut_mode):
                             * 0 (default) the band is the b keys before the match position,
                             * 1 it ends at the match position itself; other values MAC_ERR_ARG */
+    int match_per_head;    /* 0 (default): one match decision per (sequence, KV head) over its G
+                            * query heads; 1: one decision per query head (its own squared L2
+                            * distance, nearest entry and reuse boundary), the KV head then reads
+                            * the union of its heads' key ranges once; hit_mask and match_pos
+                            * become [B][Hq].  Other values MAC_ERR_ARG.  (Page 1: the method
+                            * composes with MQA/GQA; the page does not fix the granularity.) */
 } MacConfig;
 
 typedef struct MacState MacState; /* opaque; owns device memory on the device current at init */
@@ -119,9 +125,10 @@ int mac_reset_seq(MacState *st, int b, void *stream);
  *   out         device fp32 [B][Hq][D], attention output.
  *   lse         device fp32 [B][Hq], natural-log log-sum-exp of the scores
  *               the output combines (reused and fresh).
- *   hit_mask    device uint8 [B][Hkv], 1 where the match hit; may be NULL.
- *   match_pos   device int32 [B][Hkv], position of the matched entry or -1;
- *               may be NULL.
+ *   hit_mask    device uint8 [B][Hkv] ([B][Hq] with match_per_head), 1 where
+ *               the match hit; may be NULL.
+ *   match_pos   device int32 [B][Hkv] ([B][Hq] with match_per_head), position
+ *               of the matched entry or -1; may be NULL.
  * The window of every unit advances by one entry.  Enqueues two kernels and
  * nothing else (no allocation, no host synchronisation), so the call can be
  * recorded into a CUDA graph -- e.g. one graph per token over all layers'

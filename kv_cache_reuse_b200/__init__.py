@@ -53,9 +53,10 @@ class MacState:
     """Owns one C MacState (ring buffers + scratch of one attention layer)."""
 
     def __init__(self, batch, num_q_heads, num_kv_heads, head_dim, window, band, tau, rope_theta,
-                 page_size=0, max_seq=0, max_pages_per_seq=0, num_pages=0, cut_mode=0):
+                 page_size=0, max_seq=0, max_pages_per_seq=0, num_pages=0, cut_mode=0, match_per_head=0):
         self.cfg = MacConfig(batch, num_q_heads, num_kv_heads, head_dim, window, band, float(tau),
-                             float(rope_theta), page_size, max_seq, max_pages_per_seq, num_pages, cut_mode)
+                             float(rope_theta), page_size, max_seq, max_pages_per_seq, num_pages, cut_mode,
+                             match_per_head)
         self.lib = load()
         h = C.c_void_p()
         check("mac_init_state", self.lib.mac_init_state(C.byref(self.cfg), C.byref(h)))
@@ -63,11 +64,11 @@ class MacState:
 
     @classmethod
     def for_workload(cls, wl, capacity=None, max_pages_per_seq=0, num_pages=0, tau=None, band=None, window=None,
-                     cut_mode=0):
+                     cut_mode=0, match_per_head=0):
         """State sized for a synth.Workload (contiguous capacity or paged pool)."""
         return cls(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W if window is None else window,
                    wl.band if band is None else band, wl.tau if tau is None else tau, wl.rope_theta,
-                   wl.page_size, capacity or 0, max_pages_per_seq, num_pages, cut_mode)
+                   wl.page_size, capacity or 0, max_pages_per_seq, num_pages, cut_mode, match_per_head)
 
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:

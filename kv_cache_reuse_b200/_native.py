@@ -50,6 +50,7 @@ class MacConfig(C.Structure):
         ("max_pages_per_seq", C.c_int),
         ("num_pages", C.c_int),
         ("cut_mode", C.c_int),
+        ("match_per_head", C.c_int),
     ]
 
 

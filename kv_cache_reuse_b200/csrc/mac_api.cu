@@ -19,6 +19,7 @@ using namespace mac;
 struct MacState {
   MacConfig cfg;
   int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, unit_max, capacity;
+  int ND;  // match decisions per unit: 1, or G with per-head matching
   size_t max_parts;
   // ring (library-owned state)
   float* ring_q = nullptr;
@@ -30,6 +31,7 @@ struct MacState {
   // scratch
   float* qrot = nullptr;
   UnitPlan* plan = nullptr;
+  HeadPlan* hplan = nullptr;  // per-head matching decisions
   Segment* seg = nullptr;
   PlanHeader* hdr = nullptr;
   int* first_seg = nullptr;
@@ -98,7 +100,7 @@ void drop_graph(MacState* s) {
 
 void free_all(MacState* s) {
   drop_graph(s);
-  void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,
+  void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,   s->hplan,
                   s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
@@ -117,6 +119,7 @@ int check_config(const MacConfig* c) {
   if (c->head_dim != 64 && c->head_dim != 128) return MAC_ERR_SHAPE;
   if (c->window < 1 || c->window > kMaxWindow) return MAC_ERR_SHAPE;
   if (c->band < 0 || c->cut_mode < 0 || c->cut_mode > 1) return MAC_ERR_ARG;
+  if (c->match_per_head < 0 || c->match_per_head > 1) return MAC_ERR_ARG;
   if (!(c->rope_theta > 0.0) || isnan(c->tau)) return MAC_ERR_ARG;
   if (c->page_size == 0) {
     if (c->max_seq < 1) return MAC_ERR_ARG;
@@ -214,6 +217,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   if (!s) return MAC_ERR_OOM;
   s->cfg = *cfg;
   s->G = cfg->num_q_heads / cfg->num_kv_heads;
+  s->ND = cfg->match_per_head ? s->G : 1;
   s->U = cfg->batch * cfg->num_kv_heads;
   s->D = cfg->head_dim;
   s->W = cfg->window;
@@ -242,6 +246,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->steps, U));
   A(alloc(&s->qrot, U * G * D));
   A(alloc(&s->plan, U));
+  A(alloc(&s->hplan, U));
   A(alloc(&s->seg, 2 * U));
   A(alloc(&s->hdr, 1));
   A(alloc(&s->first_seg, (size_t)s->grid));
@@ -263,8 +268,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   s->off_out = 0;
   s->off_lse = up256(B * Hq * D * sizeof(float));
   s->off_hit = up256(s->off_lse + B * Hq * sizeof(float));
-  s->off_mpos = up256(s->off_hit + U);
-  s->off_status = up256(s->off_mpos + U * sizeof(int));
+  s->off_mpos = up256(s->off_hit + U * s->ND);
+  s->off_status = up256(s->off_mpos + U * s->ND * sizeof(int));
   s->out_bytes = s->off_status + 16;
   A(alloc(&s->dev_in, s->in_bytes));
   A(alloc(&s->dev_out, s->out_bytes));
@@ -376,6 +381,7 @@ static int match_impl(MacState* s, float tau, const float* q_pre, const int* rop
   p.inv_freq = s->inv_freq;
   p.qrot = s->qrot;
   p.plan = s->plan;
+  p.hplan = s->hplan;
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
@@ -390,6 +396,7 @@ static int match_impl(MacState* s, float tau, const float* q_pre, const int* rop
   p.G = s->G;
   p.W = s->W;
   p.band = s->cfg.band - s->cfg.cut_mode;  // c = max(0, p - band + cut_mode)
+  p.per_head = s->cfg.match_per_head;
   p.page_size = s->cfg.page_size;
   p.max_pages = s->cfg.max_pages_per_seq;
   p.num_pages = s->cfg.num_pages;
@@ -423,6 +430,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
   p.qrot = s->qrot;
   p.plan = s->plan;
+  p.hplan = s->hplan;
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
@@ -447,6 +455,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.max_pages = s->cfg.max_pages_per_seq;
   p.nseg = 2 * s->U;
   p.grid = s->grid;
+  p.per_head = s->cfg.match_per_head;
   return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
@@ -578,8 +587,8 @@ int mac_decode_step_host(MacState* s, const float* q_pre_h, const int* rope_pos_
   if (cudaStreamSynchronize(st) != cudaSuccess) return MAC_ERR_CUDA;
   if (out_h) memcpy(out_h, s->host_out + s->off_out, B * Hq * D * sizeof(float));
   if (lse_h) memcpy(lse_h, s->host_out + s->off_lse, B * Hq * sizeof(float));
-  if (hit_h) memcpy(hit_h, s->host_out + s->off_hit, U);
-  if (match_pos_h) memcpy(match_pos_h, s->host_out + s->off_mpos, U * sizeof(int));
+  if (hit_h) memcpy(hit_h, s->host_out + s->off_hit, U * s->ND);
+  if (match_pos_h) memcpy(match_pos_h, s->host_out + s->off_mpos, U * s->ND * sizeof(int));
   unsigned status;
   memcpy(&status, s->host_out + s->off_status, sizeof status);
   return status ? MAC_ERR_DEVICE : MAC_OK;

@@ -46,6 +46,7 @@
 //
 // Every wait is bounded (2 s on %globaltimer): on expiry the kernel sets
 // MAC_DEV_TIMEOUT in the status word and leaves without hanging the GPU.
+#include <limits.h>
 #include <math.h>
 #include <stdint.h>
 
@@ -269,9 +270,13 @@ __device__ __forceinline__ void load_query(Acc<D, GP>& A, const float* qs, int G
 // rows outside [k0, k1): their scores become -inf and their V rows are
 // zeroed in shared memory (the rows may hold anything, NaN included, and
 // 0 * NaN would poison the sum).
-template <int D, int GP>
+//
+// PH (per-head matching): key rows below lo0 / lo1 are outside the ranges of
+// this lane's heads hh / hh + 1 (inside their reused states): their scores
+// become -inf for that head only (the rows are valid keys of the range).
+template <int D, int GP, bool PH>
 __device__ __forceinline__ void process_box(Acc<D, GP>& A, const uint16_t* kbox, uint16_t* vbox, float* pbuf,
-                                            int key_box, int k0, int k1, bool masked) {
+                                            int key_box, int k0, int k1, bool masked, int lo0, int lo1) {
   constexpr int KS = Cfg<D, GP>::KS;
   const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
   const int mj = lane >> 3, mr = lane & 7;  // ldmatrix: matrix and row this lane addresses
@@ -308,6 +313,13 @@ __device__ __forceinline__ void process_box(Acc<D, GP>& A, const uint16_t* kbox,
       const int row = (i >> 3) & (kSubKeys - 1);
       if (key_box + row < k0 || key_box + row >= k1) reinterpret_cast<uint4*>(vbox)[i] = make_uint4(0u, 0u, 0u, 0u);
     }
+  }
+  if constexpr (PH) {
+    const int ka = key_box + gid, kc = ka + 8;
+    if (ka < lo0) sc[0] = -INFINITY;
+    if (ka < lo1) sc[1] = -INFINITY;
+    if (kc < lo0) sc[2] = -INFINITY;
+    if (kc < lo1) sc[3] = -INFINITY;
   }
   // box max per head over its 16 keys (rows gid and gid + 8 of every lane)
   float bm0 = fmaxf(sc[0], sc[2]), bm1 = fmaxf(sc[1], sc[3]);
@@ -406,7 +418,7 @@ __device__ __forceinline__ void fold_state(float& M, float& L, float (&O)[N], fl
 // partials w, w + 8, ..., each lane FPL consecutive floats of one head), with
 // up to 48 partials' loads in flight at once; the warps' states then meet in
 // shared memory.
-template <int D, int GP, int GF>
+template <int D, int GP, int GF, bool PH>
 __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
   constexpr int QD = 4 * D;                    // floats of four heads
   constexpr int FPL = QD / 32, F4 = FPL / 4;   // floats and float4 of those per lane
@@ -414,13 +426,16 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
   constexpr int VEC = QD / (kConsumerWarps * 32);
   static_assert(VEC * kConsumerWarps * 32 == QD && F4 * 4 * 32 == QD, "merge layout");
   const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
-  const UnitPlan pl = p.plan[u];
+  const UnitPlan* const pp = p.plan + u;
+  const HeadPlan* const hp = p.hplan + u;
+  const int hit = pp->hit, hmask = PH ? hp->hmask : 0, src_slot = pp->src_slot, dst_slot = pp->dst_slot;
+  const int end = pp->end;
   const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
   const int nA = sA.npieces, n = nA + sB.npieces;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t rs = (size_t)u * Wp1 + pl.src_slot, ds = (size_t)u * Wp1 + pl.dst_slot;
+  const size_t ds = (size_t)u * Wp1 + dst_slot;
   float* wb = sm.wbuf[warp];
 
   for (int h0 = 0; h0 < G; h0 += 4) {
@@ -430,7 +445,9 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
     float MA = -INFINITY, LA = 0.f, OA[FPL], MB = -INFINITY, LB = 0.f, OB[FPL];
 #pragma unroll
     for (int j = 0; j < FPL; ++j) OA[j] = OB[j] = 0.f;
-    if (warp == 0 && pl.hit && live) {  // the reused state joins set A (its o is normalised)
+    const bool reuse = PH ? live && ((hmask >> hl) & 1) : hit && live;
+    if (warp == 0 && reuse) {  // the reused state joins set A (its o is normalised)
+      const size_t rs = (size_t)u * Wp1 + (PH ? hp->hsrc[hl] : src_slot);
       const float rl = __ldcg(p.ring_l + rs * G + hl), rm = __ldcg(p.ring_m + rs * G + hl) * kLog2e;
       float o[FPL];
 #pragma unroll
@@ -513,7 +530,7 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
     }
   }
   if (threadIdx.x == 0) {
-    p.ring_pos[(size_t)u * Wp1 + pl.dst_slot] = pl.end - 1;
+    p.ring_pos[(size_t)u * Wp1 + dst_slot] = end - 1;
     p.unit_cnt[u] = 0;
   }
   return true;
@@ -595,7 +612,7 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA
 
 // End of a split piece: combine the 8 warps, write the partial, count it
 // and, if it was the unit's last, merge the unit.
-template <int D, int GP, int GF>
+template <int D, int GP, int GF, bool PH>
 __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D, GP>& A, int unit, int pidx,
                                uint32_t& sync_phase) {
   const int G = group_of<GF>(p), GD = G * D, G4 = group4(G);
@@ -623,7 +640,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
-    return merge_unit<D, GP, GF>(p, sm, unit, sync_phase);
+    return merge_unit<D, GP, GF, PH>(p, sm, unit, sync_phase);
   }
   return true;
 }
@@ -633,16 +650,19 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D
 // (on a hit) + amend; output = new prefix + tail.  No partials, no counters.
 // On a hit, the reused m and l come with o by bulk copy when GF is a multiple
 // of 4 (16-byte runs), else thread t < 2G brings m (t < G) or l in rml.
+// hmask: heads with a reused state (any of them when hit is set; per-head
+// matching may leave some out).
 template <int D, int GP, int GF>
 __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D, GP>& A, int u, int wA, int hit,
-                              int dst, int end, float rml, uint32_t ring_phase, uint32_t& sync_phase) {
+                              int hmask, int dst, int end, float rml, uint32_t ring_phase, uint32_t& sync_phase) {
   constexpr int GDP = Cfg<D, GP>::GD;
   const int G = group_of<GF>(p), GD = G * D;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
   constexpr int PER = (GDP + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
   warp_combine_store<D, GP>(A, sm.wbuf[threadIdx.x >> 5]);
-  if (!kBulkML<GF> && hit && (int)threadIdx.x < 2 * G)
+  if (!kBulkML<GF> && hit && (int)threadIdx.x < 2 * G &&
+      ((hmask >> ((int)threadIdx.x < G ? (int)threadIdx.x : (int)threadIdx.x - G)) & 1))
     sm.ring[GDP + ((int)threadIdx.x < G ? (int)threadIdx.x : GP + (int)threadIdx.x - G)] = rml;
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   // the reused o was copied on chip at the start of the piece
@@ -655,12 +675,13 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D,
     float MA, LA, OA, MB, LB, OB;
     combine_warps2<D, GP, GP>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
     // new prefix state S = reused (hit) + amend
-    const float rm = hit ? sm.ring[GDP + h] * kLog2e : -INFINITY;
+    const bool hh = hit && ((hmask >> h) & 1);
+    const float rm = hh ? sm.ring[GDP + h] * kLog2e : -INFINITY;
     float M = fmaxf(MA, rm);
     const float Mu = M == -INFINITY ? 0.f : M;
     const float aA = ex2(MA - Mu);
     float L = LA * aA, O = OA * aA;
-    if (hit) {
+    if (hh) {
       const float a = ex2(rm - Mu), rl = sm.ring[GDP + GP + h];
       L += rl * a;
       O += sm.ring[idx] * rl * a;
@@ -689,7 +710,7 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D,
 // piece is part of one segment of a large unit; a whole-unit piece holds
 // both segments of a small unit: A = [a0, a1) (may be empty), B = [k0, k1).
 struct Piece {
-  int unit, pidx, whole;
+  int unit, pidx, whole, segA;  // segA: a split piece of segment A (the amend / prefix range)
   int hit, src, dst;          // whole unit: plan of the unit (end = k1)
   int k0, k1, kb0, nbox;      // split: its keys; whole unit: segment B
   int a0, a1, akb0, anbox;    // whole unit: segment A
@@ -742,6 +763,7 @@ struct Walker {
         if (sg.first_cta != cta) continue;  // owned by the CTA whose range holds its start
         const int start = sg.key0, cut = sg.pbase, end = sg.key0 + sg.len;
         pc.whole = 1;
+        pc.segA = 0;
         pc.pidx = -1;
         pc.hit = sg.npieces & 1;
         pc.src = (sg.npieces >> 1) & 0x7ff;
@@ -767,6 +789,7 @@ struct Walker {
       const long long fe = hi < sg.flat + sg.len ? hi : sg.flat + sg.len;
       if (fa >= fe) continue;  // the range holds only this segment's padding, or ends before it
       pc.whole = 0;
+      pc.segA = sg.kind == kItemA;
       pc.wA = 0;
       pc.anbox = 0;
       pc.pidx = sg.pbase + (cta - sg.first_cta);
@@ -820,7 +843,7 @@ __device__ __noinline__ void rate_shares(const AttendParams& p) {
   if (tid == 0) p.cw[G] = 1.0;
 }
 
-template <int D, int GP, int GF>
+template <int D, int GP, int GF, bool PH>
 __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
   using C = Cfg<D, GP>;
   constexpr int NST = C::NST, NQ = C::NQ;
@@ -953,7 +976,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     const bool ring_copy = cp.whole && cp.hit;
     ring_pending = ring_copy;
     float rml = 0.f;  // m (thread t < G) or l (G <= t < 2G) of the reused state
-    if (ring_copy) {
+    int hmask = ring_copy ? (1 << G) - 1 : 0;  // heads with a reused state
+    int lo0 = 0, lo1 = 0;                      // per-head matching: first keys of this lane's heads
+    if constexpr (PH) {
+      // each head starts its fresh keys at its own reuse boundary (amend range
+      // only; every head attends the whole tail)
+      const HeadPlan* pp = p.hplan + cp.unit;
+      if (ring_copy) hmask = pp->hmask;
+      const bool onA = cp.whole ? warp < cp.wA : cp.segA;
+      const int hh = GP == 4 ? 2 * ((lane & 3) & 1) : 2 * (lane & 3);
+      lo0 = onA && hh < G ? pp->hstart[hh] : INT_MIN;
+      lo1 = onA && hh + 1 < G ? pp->hstart[hh + 1] : INT_MIN;
+    }
+    if (PH && ring_copy) {
+      // per-head matching: each reusing head's state comes from its own slot
+      const size_t ub = (size_t)cp.unit * (p.W + 1);
+      if (warp == 0) {
+        if (lane == 0) mbar_arrive_expect_tx(&sm.rfull, __popc(hmask) * D * 4);
+        __syncwarp();
+        if (lane < G && ((hmask >> lane) & 1)) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          bulk_load(sm.ring + lane * D, p.ring_o + ((ub + p.hplan[cp.unit].hsrc[lane]) * G + lane) * D, D * 4,
+                    &sm.rfull);
+        }
+      }
+      if (tid < 2 * G) {
+        const int h = tid < G ? tid : tid - G;
+        if ((hmask >> h) & 1) {
+          const size_t e = (ub + p.hplan[cp.unit].hsrc[h]) * G + h;
+          rml = __ldcg(tid < G ? p.ring_m + e : p.ring_l + e);
+        }
+      }
+    } else if (ring_copy) {
       // the merge at the end of the piece reads the reused ring state: copy
       // its o on chip now (the previous piece's merge is done with the
       // buffer); m and l travel in registers
@@ -980,8 +1034,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       if (tid == 0 && cons == 0) t_first = globaltimer();
       const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * C::PB;
-      process_box<D, GP>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
-                     key_box < cr.k0 || key_box + kSubKeys > cr.k1);
+      process_box<D, GP, PH>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
+                             key_box < cr.k0 || key_box + kSubKeys > cr.k1, lo0, lo1);
       par ^= 1;
       ++cons;
       __syncwarp();
@@ -992,9 +1046,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     }
     if (!ok) break;
     if (tid == 0) t_last = globaltimer();
-    const bool fin = cp.whole ? finalize_unit<D, GP, GF>(p, sm, A, cp.unit, cp.wA, cp.hit, cp.dst, cp.k1, rml,
-                                                         ring_phase, sync_phase)
-                              : finalize_piece<D, GP, GF>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    const bool fin = cp.whole ? finalize_unit<D, GP, GF>(p, sm, A, cp.unit, cp.wA, cp.hit, hmask, cp.dst, cp.k1,
+                                                         rml, ring_phase, sync_phase)
+                              : finalize_piece<D, GP, GF, PH>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (ring_copy) ring_phase ^= 1u;
     ring_pending = false;
     if (!fin) break;
@@ -1047,29 +1101,36 @@ size_t attend_smem_bytes(int D, int G) {
 }
 
 namespace {
-// Kernel variants: exact groups of 4 and 8 (compile-time G), and groups of
-// 1-3 and 5-7 padded to 4 and 8 (run-time G).
-template <int D, int GP, int GF>
+// Kernel variants: exact groups of 4 and 8 (compile-time G), groups of 1-3
+// and 5-7 padded to 4 and 8 (run-time G), and per-head matching (run-time G).
+template <int D, int GP, int GF, bool PH>
 cudaError_t set_smem() {
-  return cudaFuncSetAttribute(mac_attend_kernel<D, GP, GF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(mac_attend_kernel<D, GP, GF, PH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)attend_smem_bytes(D, GP));
 }
 template <int D>
 cudaError_t set_smem_all() {
-  cudaError_t e = set_smem<D, 4, 4>();
-  if (e == cudaSuccess) e = set_smem<D, 4, 0>();
-  if (e == cudaSuccess) e = set_smem<D, 8, 8>();
-  if (e == cudaSuccess) e = set_smem<D, 8, 0>();
+  cudaError_t e = set_smem<D, 4, 4, false>();
+  if (e == cudaSuccess) e = set_smem<D, 4, 0, false>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 8, false>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 0, false>();
+  if (e == cudaSuccess) e = set_smem<D, 4, 0, true>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 0, true>();
   return e;
 }
+// Per-head matching runs the run-time-group variants with per-head bounds.
 template <int D>
 cudaError_t launch_d(cudaLaunchConfig_t& cfg, const AttendParams& p) {
   const int G = p.G;
   cfg.dynamicSmemBytes = attend_smem_bytes(D, G);
-  if (G == 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 4>, p);
-  if (G == 8) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 8>, p);
-  if (G < 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 0>, p);
-  return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 0>, p);
+  if (p.per_head) {
+    if (G <= 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 0, true>, p);
+    return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 0, true>, p);
+  }
+  if (G == 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 4, false>, p);
+  if (G == 8) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 8, false>, p);
+  if (G < 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 0, false>, p);
+  return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 0, false>, p);
 }
 }  // namespace
 

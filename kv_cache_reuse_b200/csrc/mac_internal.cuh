@@ -16,7 +16,10 @@ constexpr int kAttnThreads = kConsumerWarps * 32;
 constexpr int kMatchThreads = 256;
 constexpr int kMaxWindow = 256;
 
-// Per (sequence, KV head) plan written by the match kernel.
+// Per (sequence, KV head) plan written by the match kernel.  With per-head
+// matching start is the smallest first fresh key over the unit's heads, hit
+// says whether any head reuses a state, src_slot is the first reusing head's
+// slot, and the heads' own decisions are in HeadPlan.
 struct UnitPlan {
   int start;     // first key attended with the current query (c_s on a hit, 0 on a miss)
   int cut;       // c_t = max(0, p_t - band): end of the stored prefix state
@@ -26,6 +29,13 @@ struct UnitPlan {
   int dst_slot;  // ring slot receiving this step's entry
   int bad;       // 1 = invalid inputs: no work, NaN outputs, window unchanged
   int expected;  // partial results the unit's merge waits for
+};
+
+// Per-head matching: the decisions of a unit's query heads.
+struct HeadPlan {
+  int hmask;               // heads that reuse a state (bit h)
+  int hstart[kMaxGroup];   // first key head h attends freshly (its c_s on a hit, 0 on a miss)
+  int hsrc[kMaxGroup];     // ring slot of head h's reused state
 };
 
 // Work items, two slots per unit u.  A large unit (more than unit_max fresh
@@ -83,14 +93,15 @@ struct MatchParams {
   const int* block_table;  // [B][max_pages] or null
   float* out;              // [B][Hq][D] (NaN for bad units)
   float* lse;              // [B][Hq]
-  uint8_t* hit_mask;       // [U] or null
-  int* match_pos;          // [U] or null
+  uint8_t* hit_mask;       // [U] ([U][G] with per-head matching) or null
+  int* match_pos;          // [U] ([U][G] with per-head matching) or null
   float* ring_q;           // [U][W+1][G][D]
   const int* ring_pos;     // [U][W+1]
   int* steps;              // [U]
   const double* inv_freq;  // [D/2]
   float* qrot;             // [U][G][D], RoPE'd and scaled by log2(e)/sqrt(D)
   UnitPlan* plan;          // [U]
+  HeadPlan* hplan;         // [U], per-head matching only
   Segment* seg;            // [2U]
   PlanHeader* hdr;
   int* first_seg;          // [grid] first segment of each attention CTA's range
@@ -100,6 +111,7 @@ struct MatchParams {
   int* done;               // arrival counter of the match CTAs (reset by the last)
   unsigned* status;
   int B, Hq, Hkv, G, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
+  int per_head;   // 1: one match decision per query head
   float tau;
   int grid;       // CTAs of the attention kernel
   int min_keys;   // minimum cost-space units per attention CTA
@@ -113,6 +125,7 @@ struct AttendParams {
   const int* block_table;
   const float* qrot;
   const UnitPlan* plan;
+  const HeadPlan* hplan;  // [U], per-head matching only
   const Segment* seg;
   const PlanHeader* hdr;
   const int* first_seg;  // [grid]
@@ -130,6 +143,7 @@ struct AttendParams {
   float* lse;        // [B][Hq]
   unsigned* status;
   int Hq, Hkv, G, W, page_size, max_pages, nseg, grid;
+  int per_head;      // 1: heads of a unit reuse states on their own (plan hmask, hstart, hsrc)
 };
 
 struct AppendParams {

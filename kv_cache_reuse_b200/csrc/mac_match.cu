@@ -88,6 +88,8 @@ __device__ __forceinline__ int cta_of(long long x, long long T, int N, double rT
   return (int)ceil_div((x + 1) * (long long)N, T, rT) - 1;
 }
 
+static_assert(kMaxWindow + 1 <= 0x7ff, "ring slots must fit the 11-bit fields of a whole item");
+
 __device__ void build_segments(const MatchParams& p, int U, double cw_c) {
   __shared__ long long sbuf[kMatchThreads / 32];
   const int tid = threadIdx.x;
@@ -114,7 +116,8 @@ __device__ void build_segments(const MatchParams& p, int U, double cw_c) {
             cut = c;
             // the CTA doing it also needs hit, reused slot and written slot
             const int hit = __ldcg(&pl->hit), src = __ldcg(&pl->src_slot), dst = __ldcg(&pl->dst_slot);
-            packed = (hit ? 1 : 0) | ((hit ? src : 0) << 1) | (dst << 12);
+            // slots are below kMaxWindow + 1 <= 2^11: masked, neither field can spill into the other
+            packed = (hit ? 1 : 0) | ((hit && src >= 0 ? src & 0x7ff : 0) << 1) | ((dst & 0x7ff) << 12);
           }
         } else {
           len = (s & 1) ? end - c : c - start;
@@ -232,15 +235,17 @@ __device__ void build_segments(const MatchParams& p, int U, double cw_c) {
 // GP: the query group padded to 4 or 8 heads (register and shared-memory
 // shapes); the real group G <= GP sets every global layout.  GF = G for the
 // variants built for one group size (4, 8), 0 for a run-time G (p.G).
-template <int D, int GP, int GF>
+// PH: one decision per query head (per-head matching).
+template <int D, int GP, int GF, bool PH>
 __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchParams p) {
   const int G = GF > 0 ? GF : p.G;
   const int GD = G * D;
   __shared__ __align__(16) float sq[GP * D];
-  __shared__ float sdist[kMaxWindow];
+  __shared__ float sdist[PH ? GP : 1][kMaxWindow];  // [decision][age]: one row, or one per head (PH)
   __shared__ int spos[kMaxWindow];
   __shared__ int sslot[kMaxWindow];
   __shared__ int s_bad_page, s_last;
+  __shared__ int s_dhit[PH ? GP : 1], s_dpos[PH ? GP : 1], s_dslot[PH ? GP : 1];  // each decision's outcome
   __shared__ UnitPlan s_plan;
 
   // the attention kernel (launched with programmatic stream serialization)
@@ -309,7 +314,29 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
       const int slot = s0 + k * NW;
       if (slot < Wp1) {
         const int j = (((n - 1 - slot) % Wp1) + Wp1) % Wp1;
-        if (j < occ) {
+        if (PH && j < occ) {
+          // one distance per head: float4 i of a slot belongs to head i / (D/4)
+#pragma unroll
+          for (int f = 0; f < F4; ++f) {
+            const int i4 = lane + 32 * f;
+            float a = 0.f;
+            if (i4 < n4) {
+              const float4 q = reinterpret_cast<const float4*>(sq)[i4];
+              const float dx = q.x - r[k][f].x, dy = q.y - r[k][f].y, dz = q.z - r[k][f].z, dw = q.w - r[k][f].w;
+              a = fmaf(dx, dx, a);
+              a = fmaf(dy, dy, a);
+              a = fmaf(dz, dz, a);
+              a = fmaf(dw, dw, a);
+            }
+#pragma unroll
+            for (int o = D / 8; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);  // the head's D/4 lanes
+            if (i4 < n4 && i4 % (D / 4) == 0) sdist[PH ? i4 / (D / 4) : 0][j] = a;
+          }
+          if (lane == 0) {
+            spos[j] = rpos[k];
+            sslot[j] = slot;
+          }
+        } else if (j < occ) {
           float acc = 0.f;
 #pragma unroll
           for (int f = 0; f < F4; ++f) {
@@ -324,7 +351,7 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
           acc = warp_sum(acc);
           if (lane == 0) {
             // a power-of-two group divides exactly by its reciprocal
-            sdist[j] = (GF == 4 || GF == 8) ? acc * (1.0f / (GF > 0 ? GF : 1)) : __fdiv_rn(acc, (float)G);
+            sdist[0][j] = (GF == 4 || GF == 8) ? acc * (1.0f / (GF > 0 ? GF : 1)) : __fdiv_rn(acc, (float)G);
             spos[j] = rpos[k];
             sslot[j] = slot;
           }
@@ -334,12 +361,14 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   }
   __syncthreads();
 
-  // 2. argmin: smaller distance, then larger position, then the newer entry
-  if (warp == 0) {
+  // 2. argmin: smaller distance, then larger position, then the newer entry;
+  // warp w takes decision w (the group's, or head w's with per-head matching)
+  const int nd = PH ? G : 1;
+  if (warp < nd) {
     float bd = INFINITY;
     int bp = 0, bj = -1;
     for (int j = lane; j < occ; j += 32) {
-      const float d = sdist[j];
+      const float d = sdist[warp][j];
       const int pos = spos[j];
       if (pos < p_t && (d < bd || (d == bd && bj >= 0 && (pos > bp || (pos == bp && j < bj))))) {
         bd = d;
@@ -361,20 +390,53 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     }
     if (lane == 0) {
       const int hit = (bj >= 0) && (bd < p.tau);
-      UnitPlan pl;
-      pl.end = len;
-      pl.cut = p_t - p.band > 0 ? p_t - p.band : 0;
-      pl.hit = hit;
-      pl.src_slot = hit ? sslot[bj] : -1;
-      pl.start = hit ? (bp - p.band > 0 ? bp - p.band : 0) : 0;
-      pl.dst_slot = n % Wp1;
-      pl.bad = (len < 1 || len > p.capacity) ? 1 : 0;
-      pl.expected = 0;
-      s_plan = pl;
-      spos[0] = hit ? bp : -1;  // matched position (slot 0 of spos no longer needed)
+      s_dhit[warp] = hit;
+      s_dpos[warp] = hit ? bp : -1;
+      s_dslot[warp] = hit ? sslot[bj] : -1;
+      if (!PH) {
+        UnitPlan pl;
+        pl.end = len;
+        pl.cut = p_t - p.band > 0 ? p_t - p.band : 0;
+        pl.hit = hit;
+        pl.src_slot = hit ? sslot[bj] : -1;
+        pl.start = hit ? (bp - p.band > 0 ? bp - p.band : 0) : 0;
+        pl.dst_slot = n % Wp1;
+        pl.bad = (len < 1 || len > p.capacity) ? 1 : 0;
+        pl.expected = 0;
+        s_plan = pl;
+      }
     }
   }
   __syncthreads();
+  if (PH) {
+    // the unit reads the union of its heads' ranges: from the smallest first
+    // fresh key; its reuse slot is the first reusing head's (-1: none)
+    if (tid == 0) {
+      UnitPlan pl;
+      HeadPlan hp;
+      pl.end = len;
+      pl.cut = p_t - p.band > 0 ? p_t - p.band : 0;
+      pl.dst_slot = n % Wp1;
+      pl.bad = (len < 1 || len > p.capacity) ? 1 : 0;
+      pl.expected = 0;
+      int start = len, hmask = 0, src = -1;
+      for (int d = 0; d < nd; ++d) {
+        if (src < 0) src = s_dslot[d];
+        const int st = s_dhit[d] ? (s_dpos[d] - p.band > 0 ? s_dpos[d] - p.band : 0) : 0;
+        start = st < start ? st : start;
+        hmask |= s_dhit[d] << d;
+        hp.hstart[d] = st;
+        hp.hsrc[d] = s_dslot[d];
+      }
+      pl.start = start;
+      pl.hit = hmask != 0;
+      pl.src_slot = src;
+      hp.hmask = hmask;
+      s_plan = pl;
+      p.hplan[u] = hp;
+    }
+    __syncthreads();
+  }
 
   // paged KV: every page the step reads must be a valid pool page
   if (!s_plan.bad && p.page_size > 0) {
@@ -392,10 +454,12 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     const float qnan = __int_as_float(0x7fc00000);
     for (int i = tid; i < GD; i += kMatchThreads) p.out[((size_t)b * p.Hq + (size_t)kvh * G) * D + i] = qnan;
     if (tid < G) p.lse[(size_t)b * p.Hq + kvh * G + tid] = qnan;
+    if (tid < nd) {
+      if (p.hit_mask) p.hit_mask[u * nd + tid] = 0;
+      if (p.match_pos) p.match_pos[u * nd + tid] = -1;
+    }
     if (tid == 0) {
       atomicOr(p.status, s_plan.bad ? MAC_DEV_BAD_SEQ_LEN : MAC_DEV_BAD_PAGE);
-      if (p.hit_mask) p.hit_mask[u] = 0;
-      if (p.match_pos) p.match_pos[u] = -1;
       UnitPlan pl = s_plan;
       pl.bad = 1;
       pl.hit = 0;
@@ -416,10 +480,12 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     // 5. this step's query enters the ring
     float4* rdst = reinterpret_cast<float4*>(p.ring_q + ((size_t)u * Wp1 + s_plan.dst_slot) * GD);
     for (int i = tid; i < n4; i += kMatchThreads) rdst[i] = reinterpret_cast<const float4*>(sq)[i];
+    if (tid < nd) {
+      if (p.hit_mask) p.hit_mask[u * nd + tid] = (uint8_t)s_dhit[tid];
+      if (p.match_pos) p.match_pos[u * nd + tid] = s_dpos[tid];
+    }
     if (tid == 0) {
       p.steps[u] = n + 1;
-      if (p.hit_mask) p.hit_mask[u] = (uint8_t)s_plan.hit;
-      if (p.match_pos) p.match_pos[u] = spos[0];
       p.plan[u] = s_plan;
     }
   }
@@ -441,16 +507,24 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   if (tid == 0) *p.done = 0;
 }
 
+// Variants as for the attention kernel: exact groups of 4 and 8, run-time
+// groups padded to 4 and 8, and per-head matching (run-time group).
 template <int D>
 void launch_d(const MatchParams& p, int U, cudaStream_t s) {
-  if (p.G == 4)
-    mac_match_kernel<D, 4, 4><<<U, kMatchThreads, 0, s>>>(p);
-  else if (p.G == 8)
-    mac_match_kernel<D, 8, 8><<<U, kMatchThreads, 0, s>>>(p);
-  else if (p.G < 4)
-    mac_match_kernel<D, 4, 0><<<U, kMatchThreads, 0, s>>>(p);
-  else
-    mac_match_kernel<D, 8, 0><<<U, kMatchThreads, 0, s>>>(p);
+  if (p.per_head) {
+    if (p.G <= 4)
+      mac_match_kernel<D, 4, 0, true><<<U, kMatchThreads, 0, s>>>(p);
+    else
+      mac_match_kernel<D, 8, 0, true><<<U, kMatchThreads, 0, s>>>(p);
+  } else if (p.G == 4) {
+    mac_match_kernel<D, 4, 4, false><<<U, kMatchThreads, 0, s>>>(p);
+  } else if (p.G == 8) {
+    mac_match_kernel<D, 8, 8, false><<<U, kMatchThreads, 0, s>>>(p);
+  } else if (p.G < 4) {
+    mac_match_kernel<D, 4, 0, false><<<U, kMatchThreads, 0, s>>>(p);
+  } else {
+    mac_match_kernel<D, 8, 0, false><<<U, kMatchThreads, 0, s>>>(p);
+  }
 }
 
 }  // namespace

@@ -174,6 +174,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.inv_freq = reinterpret_cast<const double*>(base + kOffInv);
   mp.qrot = reinterpret_cast<float*>(base + kOffQrot);
   mp.plan = reinterpret_cast<UnitPlan*>(base + kOffPlan);
+  mp.hplan = nullptr;  // no per-head matching here
   mp.seg = reinterpret_cast<Segment*>(base + kOffSeg);
   mp.hdr = reinterpret_cast<PlanHeader*>(base + kOffHdr);
   mp.first_seg = reinterpret_cast<int*>(base + kOffFirst);
@@ -186,6 +187,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.Hq = num_q_heads;
   mp.Hkv = num_kv_heads;
   mp.G = num_q_heads / num_kv_heads;
+  mp.per_head = 0;
   mp.W = 0;
   mp.band = 1 << 30;
   mp.page_size = page_size;
@@ -210,6 +212,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.block_table = page_size > 0 ? block_table : nullptr;
   ap.qrot = mp.qrot;
   ap.plan = mp.plan;
+  ap.hplan = nullptr;
   ap.seg = mp.seg;
   ap.hdr = mp.hdr;
   ap.first_seg = mp.first_seg;
@@ -229,6 +232,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.Hq = num_q_heads;
   ap.Hkv = num_kv_heads;
   ap.G = num_q_heads / num_kv_heads;
+  ap.per_head = 0;
   ap.W = 0;
   ap.page_size = page_size;
   ap.max_pages = max_pages_per_seq;

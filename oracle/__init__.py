@@ -38,7 +38,7 @@ class _Cfg(C.Structure):
     _fields_ = [("B", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("D", C.c_int),
                 ("W", C.c_int), ("band", C.c_int), ("tau", C.c_double), ("rope_theta", C.c_double),
                 ("page_size", C.c_int), ("max_seq", C.c_int), ("max_pages_per_seq", C.c_int),
-                ("cut_mode", C.c_int)]
+                ("cut_mode", C.c_int), ("per_head", C.c_int)]
 
 
 def _load():
@@ -122,22 +122,23 @@ class Oracle:
     """Stateful fp64 MAC decode oracle: one instance per layer of KV heads."""
 
     def __init__(self, B, Hq, Hkv, D, W, band, tau, rope_theta, page_size=0, max_seq=0,
-                 max_pages_per_seq=0, cut_mode=0):
+                 max_pages_per_seq=0, cut_mode=0, per_head=0):
         self.lib = _load()
         self.cfg = _Cfg(B, Hq, Hkv, D, W, band, float(tau), float(rope_theta), page_size, max_seq,
-                        max_pages_per_seq, cut_mode)
+                        max_pages_per_seq, cut_mode, per_head)
         self.h = self.lib.oracle_create(C.byref(self.cfg))
         if not self.h:
             raise ValueError("invalid oracle configuration")
         self.B, self.Hq, self.Hkv, self.D, self.W = B, Hq, Hkv, D, W
         self.G = Hq // Hkv
+        self.nd = Hkv * (self.G if per_head else 1)  # match decisions per sequence
 
     @classmethod
-    def for_workload(cls, wl, cache, tau=None, band=None, W=None, cut_mode=0):
+    def for_workload(cls, wl, cache, tau=None, band=None, W=None, cut_mode=0, per_head=0):
         return cls(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W if W is None else W, wl.band if band is None else band,
                    wl.tau if tau is None else tau, wl.rope_theta, wl.page_size,
                    cache.max_seq if not cache.paged else 0,
-                   cache.block_table.shape[1] if cache.paged else 0, cut_mode)
+                   cache.block_table.shape[1] if cache.paged else 0, cut_mode, per_head)
 
     def __del__(self):
         try:
@@ -156,7 +157,7 @@ class Oracle:
         seq_lens = np.ascontiguousarray(seq_lens, np.int32)
         assert K.dtype == np.uint16 and K.flags.c_contiguous and V.flags.c_contiguous
         bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
-        U = self.B * self.Hkv
+        U = self.B * self.nd
         out = np.empty((self.B, self.Hq, self.D), np.float64)
         lse = np.empty((self.B, self.Hq), np.float64)
         hit = np.empty(U, np.uint8)
@@ -168,14 +169,15 @@ class Oracle:
                                   _p(out), _p(lse), _p(hit), _p(mpos), _p(db), _p(ds), C.byref(kr))
         if rc != 0:
             raise ValueError("oracle_step rejected its inputs (rc=%d)" % rc)
-        return StepResult(out, lse, hit.reshape(self.B, self.Hkv), mpos.reshape(self.B, self.Hkv),
-                          db.reshape(self.B, self.Hkv), ds.reshape(self.B, self.Hkv), kr.value)
+        sh = (self.B, self.nd)
+        return StepResult(out, lse, hit.reshape(sh), mpos.reshape(sh), db.reshape(sh), ds.reshape(sh), kr.value)
 
     def match_step(self, q_pre, seq_lens):
-        """Match stage only (no attention): (hit, match_pos, d_best, d_second)."""
+        """Match stage only (no attention): (hit, match_pos, d_best, d_second), each
+        [B][Hkv] ([B][Hq] with per-head matching)."""
         q_pre = np.ascontiguousarray(q_pre, np.float32)
         seq_lens = np.ascontiguousarray(seq_lens, np.int32)
-        U = self.B * self.Hkv
+        U = self.B * self.nd
         hit = np.empty(U, np.uint8)
         mpos = np.empty(U, np.int32)
         db = np.empty(U, np.float64)
@@ -183,7 +185,7 @@ class Oracle:
         rc = self.lib.oracle_match_step(self.h, _p(q_pre), _p(seq_lens), _p(hit), _p(mpos), _p(db), _p(ds))
         if rc != 0:
             raise ValueError("oracle_match_step rejected its inputs (rc=%d)" % rc)
-        sh = (self.B, self.Hkv)
+        sh = (self.B, self.nd)
         return hit.reshape(sh), mpos.reshape(sh), db.reshape(sh), ds.reshape(sh)
 
     def warm_start(self, q_pre, rope_pos, K, V, block_table, seq_lens) -> None:

@@ -21,6 +21,11 @@
  * reading is named where it is used:
  *   [mean-dist]   distance = mean over the G query heads of a KV head of the
  *                 per-head squared L2 distance of the pre-RoPE queries;
+ *   [per-head]    with per-head matching every query head decides alone: its
+ *                 distance is its own squared L2 distance (the mean over a
+ *                 group of one), its own nearest entry, its own reuse
+ *                 boundary; the keys a KV head serves are the union of its
+ *                 query heads' ranges;
  *   [strict]      hit iff the smallest distance is < tau (strict), ties to the
  *                 more recent entry, NaN distances never match;
  *   [window]      the window is the W most recent previous decode steps of the
@@ -61,6 +66,7 @@ typedef struct {
     int max_seq;           /* rows per sequence (contiguous) */
     int max_pages_per_seq; /* block table row length (paged: K/V [P][page][Hkv][D]) */
     int cut_mode;          /* [cut]: 0 or 1 */
+    int per_head;          /* 0: one decision per KV head ([mean-dist]); 1: per query head ([per-head]) */
 } ocfg_t;
 
 typedef struct {
@@ -197,7 +203,8 @@ void oracle_merge(const double *o1, double m1, double l1, const double *o2, doub
 
 ostate_t *oracle_create(const ocfg_t *cfg) {
     if (!cfg || cfg->Hkv <= 0 || cfg->Hq % cfg->Hkv != 0 || cfg->D <= 0 || (cfg->D & 1) || cfg->W < 0 ||
-        cfg->band < 0 || cfg->B <= 0 || cfg->cut_mode < 0 || cfg->cut_mode > 1)
+        cfg->band < 0 || cfg->B <= 0 || cfg->cut_mode < 0 || cfg->cut_mode > 1 || cfg->per_head < 0 ||
+        cfg->per_head > 1)
         return NULL;
     ostate_t *s = (ostate_t *)calloc(1, sizeof(ostate_t));
     s->c = *cfg;
@@ -244,12 +251,16 @@ int oracle_window(const ostate_t *s, int u, float *q, double *o, double *m, doub
 
 /* ----------------------------------------------------------------- match */
 
-/* Match (page 1): nearest entry of the window to the current pre-RoPE query.
- * [mean-dist] dist = (1/G) sum_h sum_i (q[h][i] - q_e[h][i])^2.
+/* Match (page 1): nearest entry of the window to the current pre-RoPE query
+ * heads h0 .. h0 + nh - 1 of unit u's group (all G heads, or one head with
+ * [per-head] matching).
+ * [mean-dist] dist = (1/nh) sum_h sum_i (q[h][i] - q_e[h][i])^2.
  * [window] only entries whose position precedes p_t are candidates.
  * [strict] returns the index of the smallest distance, ties to the larger
- * position, then to the more recent entry; *best/*second receive the two smallest distances (+inf if absent). */
-static int match_unit(const ostate_t *s, int u, const float *qg, int p_t, double *best, double *second) {
+ * position, then to the more recent entry; best and second receive the two
+ * smallest distances (+inf if absent). */
+static int match_unit(const ostate_t *s, int u, const float *qg, int h0, int nh, int p_t, double *best,
+                      double *second) {
     int G = s->G, D = s->c.D, W = s->c.W > 0 ? s->c.W : 1;
     int n = s->n[u];
     int arg = -1;
@@ -259,12 +270,12 @@ static int match_unit(const ostate_t *s, int u, const float *qg, int p_t, double
         if (pos >= p_t) continue;
         const float *qe = s->wq + (((size_t)u * W + e) * G) * D;
         double acc = 0.0;
-        for (int h = 0; h < G; ++h)
+        for (int h = h0; h < h0 + nh; ++h)
             for (int i = 0; i < D; ++i) {
                 double dlt = (double)qg[h * D + i] - (double)qe[h * D + i];
                 acc += dlt * dlt;
             }
-        double dist = acc / (double)G;
+        double dist = acc / (double)nh;
         if (isnan(dist)) continue;
         /* entries run oldest to newest, so on an exact tie of distance and
          * position the later (more recent) entry wins */
@@ -315,8 +326,9 @@ static void push_entry(ostate_t *s, int u, const float *qg, const double *sn, co
  *   seq_lens  [B] keys visible (the step's own row included); p_t = len - 1
  * Outputs: out [B][Hq][D], lse [B][Hq] (natural log), hit [B*Hkv],
  * match_pos [B*Hkv] (position of the matched entry or -1), best/second
- * distances [B*Hkv] and keys_read (keys attended freshly, summed over units).
- * Returns 0, or -1 on an invalid sequence length. */
+ * distances [B*Hkv] -- [B*Hq] with [per-head] matching -- and keys_read
+ * (keys a unit attends freshly, the union over its heads' ranges, summed
+ * over units).  Returns 0, or -1 on an invalid sequence length. */
 int oracle_step(ostate_t *s, const float *q_pre, const int *rope_pos, const uint16_t *K,
                 const uint16_t *V, const int *block_table, const int *seq_lens, double *out,
                 double *lse, uint8_t *hit, int *match_pos, double *d_best, double *d_second,
@@ -332,17 +344,27 @@ int oracle_step(ostate_t *s, const float *q_pre, const int *rope_pos, const uint
         int p_t = seq_lens[b] - 1;
         const float *qg = q_pre + ((size_t)b * c->Hq + (size_t)kvh * G) * D;
 
-        /* Match. */
-        double best, second;
-        int e = match_unit(s, u, qg, p_t, &best, &second);
-        int is_hit = (e >= 0) && (best < c->tau);
-        int p_s = is_hit ? s->wpos[(size_t)u * W + e] : -1;
-
-        /* [cut] prefix boundaries. */
+        /* Match: one decision for the group, or one per head ([per-head]). */
+        const int nd = c->per_head ? G : 1, hpd = G / nd;
+        int *ent = (int *)malloc(sizeof(int) * (size_t)nd);
         const long shift = c->cut_mode;
+        long first_fresh = (long)p_t + 1;
+        for (int d = 0; d < nd; ++d) {
+            double best, second;
+            int e = match_unit(s, u, qg, d * hpd, hpd, p_t, &best, &second);
+            int is_hit = (e >= 0) && (best < c->tau);
+            ent[d] = is_hit ? e : -1;
+            int p_s = is_hit ? s->wpos[(size_t)u * W + e] : -1;
+            hit[(size_t)u * nd + d] = (uint8_t)is_hit;
+            match_pos[(size_t)u * nd + d] = p_s;
+            if (d_best) d_best[(size_t)u * nd + d] = best;
+            if (d_second) d_second[(size_t)u * nd + d] = second;
+            /* [cut] the reuse boundary c_s of this decision */
+            long c_s = is_hit ? (p_s - c->band + shift > 0 ? (long)(p_s - c->band + shift) : 0) : 0;
+            if (c_s < first_fresh) first_fresh = c_s;
+        }
+        /* [cut] the prefix boundary of this step */
         long c_t = p_t - c->band + shift > 0 ? (long)(p_t - c->band + shift) : 0;
-        long c_s = is_hit ? (p_s - c->band + shift > 0 ? (long)(p_s - c->band + shift) : 0) : 0;
-        long first_fresh = is_hit ? c_s : 0;
         total_keys += (long)p_t + 1 - first_fresh;
 
         double *qr = (double *)malloc(sizeof(double) * (size_t)D);
@@ -353,10 +375,13 @@ int oracle_step(ostate_t *s, const float *q_pre, const int *rope_pos, const uint
         double *snl = (double *)malloc(sizeof(double) * (size_t)G);
         for (int h = 0; h < G; ++h) {
             int hq = kvh * G + h;
+            const int e = ent[h / hpd], is_hit = e >= 0;
             oracle_rope(qg + (size_t)h * D, D, rope_pos[b], c->rope_theta, qr);
-            double ma, la, mb, lb;
+            double ma, la;
             double *o_new = sn + (size_t)h * D;
             if (is_hit) {
+                long p_s = s->wpos[(size_t)u * W + e];
+                long c_s = p_s - c->band + shift > 0 ? p_s - c->band + shift : 0;
                 /* Amend: reuse the matched entry's prefix state over [0, c_s)
                  * and recompute [c_s, c_t) with the current query. */
                 const double *ro = s->wo + (((size_t)u * W + e) * G + h) * D;
@@ -375,14 +400,10 @@ int oracle_step(ostate_t *s, const float *q_pre, const int *rope_pos, const uint
             memcpy(out + ((size_t)b * c->Hq + hq) * D, ob, sizeof(double) * (size_t)D);
             lse[(size_t)b * c->Hq + hq] = mo + log(lo);
         }
-        hit[u] = (uint8_t)is_hit;
-        match_pos[u] = p_s;
-        if (d_best) d_best[u] = best;
-        if (d_second) d_second[u] = second;
 
         /* Store (pre-RoPE query, prefix state, position) as the newest entry. */
         push_entry(s, u, qg, sn, snm, snl, p_t);
-        free(qr); free(oa); free(ob); free(sn); free(snm); free(snl);
+        free(qr); free(oa); free(ob); free(sn); free(snm); free(snl); free(ent);
     }
     if (keys_read) *keys_read = total_keys;
     return 0;
@@ -402,13 +423,16 @@ int oracle_match_step(ostate_t *s, const float *q_pre, const int *seq_lens, uint
         int b = u / c->Hkv, kvh = u % c->Hkv;
         int p_t = seq_lens[b] - 1;
         const float *qg = q_pre + ((size_t)b * c->Hq + (size_t)kvh * G) * D;
-        double best, second;
-        int e = match_unit(s, u, qg, p_t, &best, &second);
-        int is_hit = (e >= 0) && (best < c->tau);
-        hit[u] = (uint8_t)is_hit;
-        match_pos[u] = is_hit ? s->wpos[(size_t)u * W + e] : -1;
-        if (d_best) d_best[u] = best;
-        if (d_second) d_second[u] = second;
+        const int nd = c->per_head ? G : 1, hpd = G / nd;
+        for (int d = 0; d < nd; ++d) {
+            double best, second;
+            int e = match_unit(s, u, qg, d * hpd, hpd, p_t, &best, &second);
+            int is_hit = (e >= 0) && (best < c->tau);
+            hit[(size_t)u * nd + d] = (uint8_t)is_hit;
+            match_pos[(size_t)u * nd + d] = is_hit ? s->wpos[(size_t)u * W + e] : -1;
+            if (d_best) d_best[(size_t)u * nd + d] = best;
+            if (d_second) d_second[(size_t)u * nd + d] = second;
+        }
         double *sn = (double *)malloc(sizeof(double) * (size_t)G * (D + 2));
         for (size_t i = 0; i < (size_t)G * (D + 2); ++i) sn[i] = NAN;
         push_entry(s, u, qg, sn, sn + (size_t)G * D, sn + (size_t)G * D + G, p_t);

@@ -21,6 +21,10 @@ Recipe (all draws from numpy PCG64 streams keyed by (seed, tag, chunk)):
     window is still empty falls back to fresh.
   * Labels: iid Bernoulli, a per-sequence Bernoulli rate, or a two-state
     Markov chain, depending on the workload.
+  * With head_labels, the label and the source step are drawn per query head
+    (each head repeats its own earlier query or draws fresh on its own), so
+    the heads of one KV head's group disagree; otherwise all Hq heads of a
+    sequence share them.
 The distance margins that keep match decisions away from ties are a property
 of these distributions (sigma small against 1); the tests check them with the
 oracle rather than here.
@@ -66,6 +70,7 @@ class Workload:
     hit_model: Tuple       # ("iid", p) | ("per_seq", lo, hi) | ("markov", stay_hit, stay_miss)
     seed: int
     append: bool = False   # the step's own K/V row arrives through an append call
+    head_labels: bool = False  # repeat labels and sources drawn per query head
 
     @property
     def G(self) -> int:
@@ -130,8 +135,8 @@ def all_miss(wl: Workload) -> Workload:
 @dataclasses.dataclass
 class QueryStream:
     q: np.ndarray        # [T, B, Hq, D] float32, pre-RoPE
-    label: np.ndarray    # [T, B] bool: the step was drawn as a repeat
-    src: np.ndarray      # [T, B] int: step index it repeats, -1 if fresh
+    label: np.ndarray    # [T, B] bool ([T, B, Hq] with head_labels): drawn as a repeat
+    src: np.ndarray      # [T, B] int ([T, B, Hq] with head_labels): step index it repeats, -1 if fresh
     rope_pos: np.ndarray  # [T, B] int32, position of the step's token
     seq_lens: np.ndarray  # [T, B] int32, keys visible at the step
 
@@ -140,6 +145,8 @@ def queries(wl: Workload, steps: Optional[int] = None, sigma: Optional[float] = 
     """Draw the pre-RoPE query stream of a workload (deterministic in wl.seed)."""
     T = wl.steps if steps is None else steps
     sig = wl.sigma if sigma is None else sigma
+    if wl.head_labels:
+        return _queries_per_head(wl, T, sig)
     rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(wl.seed, spawn_key=(_TAG_Q, 0))))
     B, Hq, D, W = wl.B, wl.Hq, wl.D, wl.W
     q = np.empty((T, B, Hq, D), dtype=np.float32)
@@ -172,6 +179,42 @@ def queries(wl: Workload, steps: Optional[int] = None, sigma: Optional[float] = 
             else:
                 q[t, b] = rng.standard_normal((Hq, D)).astype(np.float32)
             prev_hit[b] = label[t, b] if kind == "markov" else prev_hit[b]
+    lens = np.stack([wl.seq_lens(t) for t in range(T)]) if T else np.zeros((0, B), np.int32)
+    return QueryStream(q=q, label=label, src=src, rope_pos=(lens - 1).astype(np.int32), seq_lens=lens)
+
+
+def _queries_per_head(wl: Workload, T: int, sig: float) -> QueryStream:
+    """Query stream whose repeat labels and sources are drawn per query head."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(wl.seed, spawn_key=(_TAG_Q, 1))))
+    B, Hq, D, W = wl.B, wl.Hq, wl.D, wl.W
+    q = np.empty((T, B, Hq, D), dtype=np.float32)
+    label = np.zeros((T, B, Hq), dtype=bool)
+    src = np.full((T, B, Hq), -1, dtype=np.int64)
+    kind = wl.hit_model[0]
+    rate = rng.uniform(wl.hit_model[1], wl.hit_model[2], size=B) if kind == "per_seq" else None
+    prev_hit = np.zeros((B, Hq), dtype=bool)
+    for t in range(T):
+        for b in range(B):
+            for h in range(Hq):
+                u = rng.random()
+                if kind == "iid":
+                    want = u < wl.hit_model[1]
+                elif kind == "per_seq":
+                    want = u < rate[b]
+                elif kind == "markov":
+                    want = (u < wl.hit_model[1]) if prev_hit[b, h] else (u >= wl.hit_model[2])
+                else:
+                    raise ValueError(kind)
+                occupied = min(t, W)
+                if want and occupied > 0:
+                    s = t - 1 - int(rng.integers(0, occupied))
+                    noise = rng.standard_normal(D)
+                    q[t, b, h] = (q[s, b, h].astype(np.float64) + sig * noise).astype(np.float32)
+                    label[t, b, h] = True
+                    src[t, b, h] = s
+                else:
+                    q[t, b, h] = rng.standard_normal(D).astype(np.float32)
+                prev_hit[b, h] = label[t, b, h]
     lens = np.stack([wl.seq_lens(t) for t in range(T)]) if T else np.zeros((0, B), np.int32)
     return QueryStream(q=q, label=label, src=src, rope_pos=(lens - 1).astype(np.int32), seq_lens=lens)
 

@@ -19,7 +19,8 @@ def torch_dev():
 class GpuRun:
     """One MacState plus device copies of a workload's cache."""
 
-    def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None, tune=None, cut_mode=0):
+    def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None, tune=None, cut_mode=0,
+                 per_head=0):
         import kv_cache_reuse_b200 as mac
         torch, dev = torch_dev()
         self.torch, self.dev, self.wl, self.cache = torch, dev, wl, cache
@@ -29,10 +30,10 @@ class GpuRun:
         if cache.paged:
             self.st = mac.MacState.for_workload(wl, max_pages_per_seq=cache.block_table.shape[1],
                                                 num_pages=cache.num_pages, tau=tau, band=band, window=window,
-                                                cut_mode=cut_mode)
+                                                cut_mode=cut_mode, match_per_head=per_head)
         else:
             self.st = mac.MacState.for_workload(wl, capacity=cache.max_seq, tau=tau, band=band, window=window,
-                                                cut_mode=cut_mode)
+                                                cut_mode=cut_mode, match_per_head=per_head)
         for name, val in (tune or {}).items():  # work-split knobs: min_keys_per_cta, piece_cost, whole_unit_keys
             getattr(mac, "mac_set_" + name)(self.st, val)
         B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
@@ -42,8 +43,9 @@ class GpuRun:
         self.lens = torch.empty(B, dtype=i32, device=dev)
         self.out = torch.empty((B, Hq, D), dtype=f32, device=dev)
         self.lse = torch.empty((B, Hq), dtype=f32, device=dev)
-        self.hit = torch.empty((B, Hkv), dtype=torch.uint8, device=dev)
-        self.mpos = torch.empty((B, Hkv), dtype=i32, device=dev)
+        nd = Hq if per_head else Hkv  # match decisions per sequence
+        self.hit = torch.empty((B, nd), dtype=torch.uint8, device=dev)
+        self.mpos = torch.empty((B, nd), dtype=i32, device=dev)
 
     def step(self, q, rope_pos, seq_lens):
         torch = self.torch
@@ -57,11 +59,13 @@ class GpuRun:
 
 
 def compare_stream(wl, stream, cache, steps=None, tau=None, band=None, window=None, gpu=None, orc=None,
-                   rope_zero=False, tune=None, cut_mode=0, start=0):
+                   rope_zero=False, tune=None, cut_mode=0, start=0, per_head=0):
     """Run both sides over the stream; assert parity at every step.  Returns stats."""
     T = stream.q.shape[0] if steps is None else steps
-    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune, cut_mode=cut_mode)
-    orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window, cut_mode=cut_mode)
+    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune, cut_mode=cut_mode,
+                        per_head=per_head)
+    orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window, cut_mode=cut_mode,
+                                            per_head=per_head)
     worst_o = worst_l = 0.0
     hits = 0
     for t in range(start, T):

@@ -66,6 +66,7 @@ def test_init_rejects_bad_config_before_touching_the_device(lib):
     is refused without a GPU."""
     import kv_cache_reuse_b200 as mac
     for kw, code in ((dict(cut_mode=2), mac.MAC_ERR_ARG), (dict(cut_mode=-1), mac.MAC_ERR_ARG),
+                     (dict(match_per_head=2), mac.MAC_ERR_ARG),
                      (dict(band=-1), mac.MAC_ERR_ARG), (dict(num_q_heads=20), mac.MAC_ERR_SHAPE),
                      (dict(num_q_heads=72), mac.MAC_ERR_SHAPE),  # 9 query heads per KV head
                      (dict(head_dim=96), mac.MAC_ERR_SHAPE)):

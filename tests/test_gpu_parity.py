@@ -317,6 +317,56 @@ def test_group_sizes_all_miss_large(Hq, Hkv):
     assert r["hits"] == 0
 
 
+@pytest.mark.parametrize("case", ["g4_d64", "g4_d128", "g4_split", "g3_paged", "g8_split", "g1", "g6_cut1"])
+def test_per_head_matching(case):
+    """Per-head matching on streams whose heads repeat on their own: every
+    head's decision bit-exact, ragged reuse boundaries inside a group (each
+    head masked to its own range of the amend band), each head's state from
+    its own ring slot, whole and split units."""
+    tiny, llama, paged = synth.WORKLOADS["tiny"], synth.WORKLOADS["llama8b_32k"], synth.WORKLOADS["paged_mixed"]
+    tune, cut = None, 0
+    if case == "g4_d64":
+        wl = tiny.with_(head_labels=True, steps=48)
+    elif case == "g4_d128":
+        wl = llama.with_(head_labels=True, L0=(6000,), steps=32)
+    elif case == "g4_split":
+        wl, tune = tiny.with_(head_labels=True, steps=40), _SPLIT
+    elif case == "g3_paged":
+        wl = paged.with_(B=3, Hq=12, Hkv=4, L0=(2500, 900, 4100), steps=16, head_labels=True)
+    elif case == "g8_split":
+        wl, tune = llama.with_(B=2, Hq=16, Hkv=2, L0=(6000, 2000), steps=16, head_labels=True), _SPLIT
+    elif case == "g1":
+        wl = tiny.with_(Hq=2, Hkv=2, head_labels=True, steps=32)
+    else:
+        wl, cut = llama.with_(B=2, Hq=12, Hkv=2, L0=(3000, 5000), steps=16, head_labels=True), 1
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tune=tune, cut_mode=cut, per_head=1)
+    hits = r["hits"]
+    assert 0 < hits < wl.steps * wl.B * wl.Hq
+
+
+def test_per_head_host_entry_matches_device_entry():
+    """The host entry returns [B][Hq] decisions with per-head matching."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(steps=20, head_labels=True)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    a = GpuRun(wl, cache, per_head=1)
+    b = GpuRun(wl, cache, per_head=1)
+    torch = a.torch
+    out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32).pin_memory()
+    lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+    hit_h = torch.empty((wl.B, wl.Hq), dtype=torch.uint8).pin_memory()
+    mp_h = torch.empty((wl.B, wl.Hq), dtype=torch.int32).pin_memory()
+    for t in range(wl.steps):
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        q_h = torch.from_numpy(stream.q[t]).pin_memory()
+        p_h = torch.from_numpy(stream.rope_pos[t]).pin_memory()
+        l_h = torch.from_numpy(stream.seq_lens[t]).pin_memory()
+        rc = mac.mac_decode_step_host(b.st, q_h, p_h, l_h, None, None, b.K, b.V, None, out_h, lse_h, hit_h, mp_h)
+        assert rc == mac.MAC_OK
+        for u, v in zip(x, (out_h.numpy(), lse_h.numpy(), hit_h.numpy(), mp_h.numpy())):
+            np.testing.assert_array_equal(u, v)
+
+
 @pytest.mark.parametrize("case", ["tiny", "split", "band0", "llama_paged"])
 def test_cut_mode_band_ends_at_position(case):
     """cut_mode 1: the stored prefix ends at max(0, p + 1 - band) on both sides."""

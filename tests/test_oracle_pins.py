@@ -399,3 +399,133 @@ def test_generator_labels_recovered_with_margin(name, steps):
                 assert not hit[b].any(), (t, b)
                 if t > 0:
                     assert (db[b] > 1.01 * wl.tau).all()
+
+
+# ------------------------------------------------------- per-head matching pins
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (8, 1)])
+def test_per_head_match_equals_brute_force(Hq, Hkv):
+    """Per-head matching: every query head takes its own nearest entry over the
+    window of its own earlier queries (numpy brute force, mean over one head)."""
+    rng = np.random.default_rng(16)
+    B, D, W = 2, 8, 4
+    G = Hq // Hkv
+    orc = oracle.Oracle(B, Hq, Hkv, D, W, 2, 0.5, 1e4, 0, 1 << 10, 0, per_head=1)
+    hist = [[[] for _ in range(Hq)] for _ in range(B)]
+    pool = []
+    K = np.zeros((B, 1 << 10, Hkv, D), np.uint16)
+    nhit = 0
+    for t in range(40):
+        q = np.empty((B, Hq, D), np.float32)
+        for b in range(B):
+            for h in range(Hq):  # each head repeats or draws fresh on its own
+                r = rng.random()
+                if pool and r < 0.3:
+                    q[b, h] = pool[int(rng.integers(0, len(pool)))][b, h]
+                elif pool and r < 0.6:
+                    q[b, h] = pool[-1][b, h] + rng.normal(0, 0.1, D).astype(np.float32)
+                else:
+                    q[b, h] = rng.standard_normal(D).astype(np.float32)
+        if t == 17:
+            q[1, 0, 0] = np.nan
+        pool.append(q.copy())
+        pool = pool[-3:]
+        lens = np.array([t + 5, 2 * t + 9], np.int32)
+        r = orc.step(q, lens - 1, K, K, None, lens)
+        assert r.hit.shape == (B, Hq)
+        for b in range(B):
+            for h in range(Hq):
+                want_hit, want_pos = _brute_match(hist[b][h][-W:], q[b, h:h + 1], 0.5, 1)
+                assert bool(r.hit[b, h]) == want_hit, (t, b, h)
+                assert int(r.match_pos[b, h]) == want_pos, (t, b, h)
+                nhit += int(want_hit)
+                hist[b][h].append((q[b, h:h + 1].copy(), int(lens[b]) - 1))
+    # the heads of a group disagree on some steps, or the test shows nothing
+    assert 0 < nhit < 40 * B * Hq
+
+
+def _heads(**kw):
+    return _tiny(head_labels=True, **kw)
+
+
+def test_per_head_forced_miss_equals_dense():
+    wl = _heads(steps=8, Hq=4, Hkv=2)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=0.0, per_head=1)
+    for t in range(wl.steps):
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        assert not r.hit.any()
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("cut_mode", [0, 1])
+def test_per_head_band_covering_hits_equal_dense(cut_mode):
+    """Band covering the context: every head's reuse boundary is 0, so each
+    head's reused state must be its own exact state, whichever entry it took."""
+    wl = _heads(L0=(40,), steps=16, band=200, Hq=8, Hkv=2)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache, cut_mode=cut_mode, per_head=1)
+    mixed = 0
+    for t in range(wl.steps):
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        grp = r.hit.reshape(wl.B, wl.Hkv, wl.G)
+        mixed += int((grp.any(-1) & ~grp.all(-1)).sum())
+        o, l = dense_step(wl, cache, stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        np.testing.assert_allclose(r.out, o, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
+    assert mixed >= 4  # groups whose heads disagreed
+
+
+def test_per_head_with_single_head_groups_equals_group_matching():
+    """With one query head per KV head the two matching modes coincide."""
+    wl = _heads(steps=24, Hq=2, Hkv=2)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    a = oracle.Oracle.for_workload(wl, cache, per_head=0)
+    b = oracle.Oracle.for_workload(wl, cache, per_head=1)
+    for t in range(wl.steps):
+        ra = a.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        rb = b.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        for x, y in ((ra.out, rb.out), (ra.lse, rb.lse), (ra.hit, rb.hit), (ra.match_pos, rb.match_pos)):
+            np.testing.assert_array_equal(x, y)
+        assert ra.keys_read == rb.keys_read
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(4, 1, 64), (32, 8, 128)])
+def test_per_head_generator_labels_recovered_with_margin(Hq, Hkv, D):
+    """Per-head labels: each repeated head hits its own source, fresh heads miss,
+    with >= 1% margins on the threshold and between the two nearest entries."""
+    base = synth.WORKLOADS["tiny"] if D == 64 else synth.WORKLOADS["llama8b_32k"]
+    wl = base.with_(Hq=Hq, Hkv=Hkv, head_labels=True, steps=64)
+    stream = synth.queries(wl)
+    orc = oracle.Oracle(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W, wl.band, wl.tau, wl.rope_theta, per_head=1)
+    for t in range(wl.steps):
+        hit, mpos, db, ds = orc.match_step(stream.q[t], stream.seq_lens[t])
+        lab = stream.label[t]
+        assert (hit.astype(bool) == lab).all(), t
+        src_pos = np.where(lab, stream.rope_pos[np.maximum(stream.src[t], 0), 0], -1)
+        assert (mpos == src_pos).all(), t
+        assert (db[lab] < 0.99 * wl.tau).all() and (ds[lab] >= 1.01 * db[lab]).all()
+        if t > 0:
+            assert (db[~lab] > 1.01 * wl.tau).all()
+
+
+def test_per_head_keys_read_is_the_union_of_head_ranges():
+    """A KV head's keys are read once for its group: the keys attended freshly
+    are p_t + 1 minus the smallest reuse boundary over its heads (0 on a miss)."""
+    wl = _heads(steps=24, Hq=8, Hkv=2)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache, per_head=1)
+    for t in range(wl.steps):
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        p_t = int(stream.seq_lens[t][0]) - 1
+        want = 0
+        for kvh in range(wl.Hkv):
+            mp = r.match_pos[0, kvh * wl.G:(kvh + 1) * wl.G]
+            first = min(max(0, int(m) - wl.band) if m >= 0 else 0 for m in mp)
+            want += p_t + 1 - first
+        assert r.keys_read == want, t
