@@ -96,6 +96,10 @@ typedef struct MacConfig {
                             * the union of its heads' key ranges once; hit_mask and match_pos
                             * become [B][Hq].  Other values MAC_ERR_ARG.  (Page 1: the method
                             * composes with MQA/GQA; the page does not fix the granularity.) */
+    int q_bf16;            /* 0 (default): q_pre is fp32; 1: q_pre holds bf16 bit patterns (uint16) */
+    int ring_bf16;         /* 0 (default): the window keeps fp32 queries and outputs; 1: it keeps
+                            * them as bf16 (round to nearest even from fp32; m and l stay fp32),
+                            * halving the window scan and state bytes of a hit */
 } MacConfig;
 
 typedef struct MacState MacState; /* opaque; owns device memory on the device current at init */
@@ -116,7 +120,8 @@ int mac_reset_seq(MacState *st, int b, void *stream);
 
 /* One MAC decode step of every sequence and KV head (page 1: match, then
  * amend and complete on a hit, split-KV attention on a miss, stable merge).
- *   q_pre       device fp32 [B][Hq][D], pre-RoPE queries, 16-byte aligned.
+ *   q_pre       device [B][Hq][D] pre-RoPE queries, fp32 (bf16 bits with
+ *               q_bf16), 16-byte aligned.
  *   rope_pos    device int32 [B], position used to rotate the queries.
  *   K, V        device bf16 bit patterns (uint16), 16-byte aligned:
  *               contiguous [B][max_seq][Hkv][D] or paged [P][page_size][Hkv][D].
@@ -133,7 +138,7 @@ int mac_reset_seq(MacState *st, int b, void *stream);
  * nothing else (no allocation, no host synchronisation), so the call can be
  * recorded into a CUDA graph -- e.g. one graph per token over all layers'
  * states -- and replayed; the recording holds the K/V addresses it saw. */
-int mac_decode_step(MacState *st, const float *q_pre, const int *rope_pos, const uint16_t *K,
+int mac_decode_step(MacState *st, const void *q_pre, const int *rope_pos, const uint16_t *K,
                     const uint16_t *V, const int *block_table, const int *seq_lens, float *out,
                     float *lse, uint8_t *hit_mask, int *match_pos, void *stream);
 
@@ -143,7 +148,7 @@ int mac_decode_step(MacState *st, const float *q_pre, const int *rope_pos, const
  * ranges; mac_attend runs amend, complete (or the miss path) and the merge
  * using the plan of the preceding mac_match on the same state.  Arguments as
  * in mac_decode_step; mac_match writes NaN to out/lse of invalid units. */
-int mac_match(MacState *st, const float *q_pre, const int *rope_pos, const int *block_table,
+int mac_match(MacState *st, const void *q_pre, const int *rope_pos, const int *block_table,
               const int *seq_lens, float *out, float *lse, uint8_t *hit_mask, int *match_pos,
               void *stream);
 int mac_attend(MacState *st, const uint16_t *K, const uint16_t *V, const int *block_table,
@@ -168,7 +173,8 @@ int mac_append_kv(MacState *st, uint16_t *K, uint16_t *V, const int *block_table
  * the query rotated at rope_pos (the window of recent queries on the
  * MAC-Attention page, filled before decoding instead of by the first W
  * decode steps).  Cost: n dense passes over each prefix.
- *   q_pre     device fp32 [n][B][Hq][D] pre-RoPE queries of the positions.
+ *   q_pre     device [n][B][Hq][D] pre-RoPE queries of the positions (fp32, or
+ *             bf16 bits with q_bf16).
  *   rope_pos  device int32 [n][B].
  *   K, V, block_table  the cache, as in mac_decode_step; keys [0, p] of every
  *             position must be in it.
@@ -176,7 +182,7 @@ int mac_append_kv(MacState *st, uint16_t *K, uint16_t *V, const int *block_table
  * Enqueued on stream; uses the state's scratch (do not overlap with
  * mac_decode_step_host on the same state).  MAC_ERR_ARG for n outside
  * [0, window] or missing pointers. */
-int mac_warm_start(MacState *st, int n, const float *q_pre, const int *rope_pos, const uint16_t *K,
+int mac_warm_start(MacState *st, int n, const void *q_pre, const int *rope_pos, const uint16_t *K,
                    const uint16_t *V, const int *block_table, const int *seq_lens, void *stream);
 
 /* mac_append_kv (when k_new_h is not NULL) and mac_decode_step with the
@@ -191,7 +197,7 @@ int mac_warm_start(MacState *st, int n, const float *q_pre, const int *rope_pos,
  * (K, V, block_table, append or not) and replayed on `stream` by later calls
  * (the work-split setters drop the recording).  Not thread-safe on one
  * state; do not call it while `stream` is being captured. */
-int mac_decode_step_host(MacState *st, const float *q_pre_h, const int *rope_pos_h,
+int mac_decode_step_host(MacState *st, const void *q_pre_h, const int *rope_pos_h,
                          const int *seq_lens_h, const uint16_t *k_new_h, const uint16_t *v_new_h,
                          uint16_t *K, uint16_t *V, const int *block_table, float *out_h,
                          float *lse_h, uint8_t *hit_h, int *match_pos_h, void *stream);
@@ -201,9 +207,10 @@ int mac_decode_step_host(MacState *st, const float *q_pre_h, const int *rope_pos
 int mac_get_status(MacState *st, int *device_status);
 
 /* Ring state export/import (checkpoint / resume).  The byte layout is:
- * int32 header[8] = {magic 0x4D414331, B*Hkv, W+1, G, D, 0, 0, 0}, then
- * fp32 q[U][W+1][G][D], fp32 o[U][W+1][G][D] (normalised output of each
- * stored prefix state), fp32 m[U][W+1][G] (max score, natural-log units),
+ * int32 header[8] = {magic 0x4D414331, B*Hkv, W+1, G, D, ring_bf16, 0, 0},
+ * then q[U][W+1][G][D] and o[U][W+1][G][D] (fp32, or bf16 bits when
+ * ring_bf16; o is the normalised output of each stored prefix state),
+ * fp32 m[U][W+1][G] (max score, natural-log units),
  * fp32 l[U][W+1][G] (sum of exp(score - m)), int32 pos[U][W+1],
  * int32 steps[U] (decode steps since reset; entry of step n sits in slot
  * n mod (W+1)).  Both calls synchronise the device.  host_buf must hold

@@ -53,10 +53,11 @@ class MacState:
     """Owns one C MacState (ring buffers + scratch of one attention layer)."""
 
     def __init__(self, batch, num_q_heads, num_kv_heads, head_dim, window, band, tau, rope_theta,
-                 page_size=0, max_seq=0, max_pages_per_seq=0, num_pages=0, cut_mode=0, match_per_head=0):
+                 page_size=0, max_seq=0, max_pages_per_seq=0, num_pages=0, cut_mode=0, match_per_head=0,
+                 q_bf16=0, ring_bf16=0):
         self.cfg = MacConfig(batch, num_q_heads, num_kv_heads, head_dim, window, band, float(tau),
                              float(rope_theta), page_size, max_seq, max_pages_per_seq, num_pages, cut_mode,
-                             match_per_head)
+                             match_per_head, q_bf16, ring_bf16)
         self.lib = load()
         h = C.c_void_p()
         check("mac_init_state", self.lib.mac_init_state(C.byref(self.cfg), C.byref(h)))
@@ -64,11 +65,12 @@ class MacState:
 
     @classmethod
     def for_workload(cls, wl, capacity=None, max_pages_per_seq=0, num_pages=0, tau=None, band=None, window=None,
-                     cut_mode=0, match_per_head=0):
+                     cut_mode=0, match_per_head=0, q_bf16=0, ring_bf16=0):
         """State sized for a synth.Workload (contiguous capacity or paged pool)."""
         return cls(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W if window is None else window,
                    wl.band if band is None else band, wl.tau if tau is None else tau, wl.rope_theta,
-                   wl.page_size, capacity or 0, max_pages_per_seq, num_pages, cut_mode, match_per_head)
+                   wl.page_size, capacity or 0, max_pages_per_seq, num_pages, cut_mode, match_per_head, q_bf16,
+                   ring_bf16)
 
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:
@@ -227,19 +229,21 @@ def mac_error_string(code: int) -> str:
 
 
 def parse_state(buf, W: int, G: int, D: int):
-    """Split an exported state buffer into named numpy arrays (layout of include/mac.h)."""
+    """Split an exported state buffer into named numpy arrays (layout of include/mac.h);
+    a bf16 window's q and o come back as their bf16 bit patterns (uint16)."""
     import numpy as np
     hdr = np.frombuffer(buf[:32].tobytes(), np.int32)
     U, W1 = int(hdr[1]), int(hdr[2])
+    qt = np.uint16 if int(hdr[5]) else np.float32
     off = 32
     out = {}
-    for name, n, dt, shape in (("q", U * W1 * G * D, np.float32, (U, W1, G, D)),
-                               ("o", U * W1 * G * D, np.float32, (U, W1, G, D)),
+    for name, n, dt, shape in (("q", U * W1 * G * D, qt, (U, W1, G, D)),
+                               ("o", U * W1 * G * D, qt, (U, W1, G, D)),
                                ("m", U * W1 * G, np.float32, (U, W1, G)),
                                ("l", U * W1 * G, np.float32, (U, W1, G)),
                                ("pos", U * W1, np.int32, (U, W1)),
                                ("steps", U, np.int32, (U,))):
-        nb = n * 4
+        nb = n * np.dtype(dt).itemsize
         out[name] = np.frombuffer(buf[off:off + nb].tobytes(), dt).reshape(shape)
         off += nb
     return out

@@ -51,6 +51,8 @@ class MacConfig(C.Structure):
         ("num_pages", C.c_int),
         ("cut_mode", C.c_int),
         ("match_per_head", C.c_int),
+        ("q_bf16", C.c_int),
+        ("ring_bf16", C.c_int),
     ]
 
 

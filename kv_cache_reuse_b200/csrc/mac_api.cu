@@ -20,10 +20,11 @@ struct MacState {
   MacConfig cfg;
   int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, unit_max, capacity;
   int ND;  // match decisions per unit: 1, or G with per-head matching
+  int QES, RES;  // bytes of a query element (input) and of a window q / o element
   size_t max_parts;
   // ring (library-owned state)
-  float* ring_q = nullptr;
-  float* ring_o = nullptr;
+  unsigned char* ring_q = nullptr;  // fp32 or bf16 (ring_bf16) elements
+  unsigned char* ring_o = nullptr;
   float* ring_m = nullptr;
   float* ring_l = nullptr;
   int* ring_pos = nullptr;
@@ -120,6 +121,7 @@ int check_config(const MacConfig* c) {
   if (c->window < 1 || c->window > kMaxWindow) return MAC_ERR_SHAPE;
   if (c->band < 0 || c->cut_mode < 0 || c->cut_mode > 1) return MAC_ERR_ARG;
   if (c->match_per_head < 0 || c->match_per_head > 1) return MAC_ERR_ARG;
+  if (c->q_bf16 < 0 || c->q_bf16 > 1 || c->ring_bf16 < 0 || c->ring_bf16 > 1) return MAC_ERR_ARG;
   if (!(c->rope_theta > 0.0) || isnan(c->tau)) return MAC_ERR_ARG;
   if (c->page_size == 0) {
     if (c->max_seq < 1) return MAC_ERR_ARG;
@@ -218,6 +220,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   s->cfg = *cfg;
   s->G = cfg->num_q_heads / cfg->num_kv_heads;
   s->ND = cfg->match_per_head ? s->G : 1;
+  s->QES = cfg->q_bf16 ? 2 : 4;
+  s->RES = cfg->ring_bf16 ? 2 : 4;
   s->U = cfg->batch * cfg->num_kv_heads;
   s->D = cfg->head_dim;
   s->W = cfg->window;
@@ -238,8 +242,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   auto A = [&](cudaError_t r) {
     if (e == cudaSuccess) e = r;
   };
-  A(alloc(&s->ring_q, U * W1 * G * D));
-  A(alloc(&s->ring_o, U * W1 * G * D));
+  A(alloc(&s->ring_q, U * W1 * G * D * s->RES));
+  A(alloc(&s->ring_o, U * W1 * G * D * s->RES));
   A(alloc(&s->ring_m, U * W1 * G));
   A(alloc(&s->ring_l, U * W1 * G));
   A(alloc(&s->ring_pos, U * W1));
@@ -259,7 +263,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->done, 1));
   A(alloc(&s->inv_freq, D / 2));
   s->off_q = 0;
-  s->off_pos = up256(s->off_q + B * Hq * D * sizeof(float));
+  s->off_pos = up256(s->off_q + B * Hq * D * s->QES);
   s->off_lens = up256(s->off_pos + B * sizeof(int));
   s->off_knew = up256(s->off_lens + B * sizeof(int));
   s->in_bytes_noappend = s->off_knew;
@@ -282,8 +286,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
     delete s;
     return e == cudaErrorMemoryAllocation ? MAC_ERR_OOM : MAC_ERR_CUDA;
   }
-  A(cudaMemset(s->ring_q, 0, U * W1 * G * D * sizeof(float)));
-  A(cudaMemset(s->ring_o, 0, U * W1 * G * D * sizeof(float)));
+  A(cudaMemset(s->ring_q, 0, U * W1 * G * D * s->RES));
+  A(cudaMemset(s->ring_o, 0, U * W1 * G * D * s->RES));
   A(cudaMemset(s->ring_m, 0, U * W1 * G * sizeof(float)));
   A(cudaMemset(s->ring_l, 0, U * W1 * G * sizeof(float)));
   A(cudaMemset(s->ring_pos, 0, U * W1 * sizeof(int)));
@@ -352,22 +356,24 @@ int mac_set_whole_unit_keys(MacState* s, int keys) {
 
 int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
 
-static int match_impl(MacState* s, float tau, const float* q_pre, const int* rope_pos, const int* block_table,
+static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope_pos, const int* block_table,
                       const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream);
 
-int mac_match(MacState* s, const float* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
+int mac_match(MacState* s, const void* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
               float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
   if (!s) return MAC_ERR_ARG;
   return match_impl(s, s->cfg.tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream);
 }
 
-static int match_impl(MacState* s, float tau, const float* q_pre, const int* rope_pos, const int* block_table,
+static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope_pos, const int* block_table,
                       const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
   if (!s || !q_pre || !rope_pos || !seq_lens || !out || !lse) return MAC_ERR_ARG;
   if (!aligned16(q_pre)) return MAC_ERR_ARG;
   if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
   MatchParams p;
   p.q_pre = q_pre;
+  p.q_bf16 = s->cfg.q_bf16;
+  p.ring_bf16 = s->cfg.ring_bf16;
   p.rope_pos = rope_pos;
   p.seq_lens = seq_lens;
   p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
@@ -397,6 +403,7 @@ static int match_impl(MacState* s, float tau, const float* q_pre, const int* rop
   p.W = s->W;
   p.band = s->cfg.band - s->cfg.cut_mode;  // c = max(0, p - band + cut_mode)
   p.per_head = s->cfg.match_per_head;
+  p.ring_bf16 = s->cfg.ring_bf16;
   p.page_size = s->cfg.page_size;
   p.max_pages = s->cfg.max_pages_per_seq;
   p.num_pages = s->cfg.num_pages;
@@ -456,10 +463,11 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.nseg = 2 * s->U;
   p.grid = s->grid;
   p.per_head = s->cfg.match_per_head;
+  p.ring_bf16 = s->cfg.ring_bf16;
   return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
-int mac_decode_step(MacState* s, const float* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
+int mac_decode_step(MacState* s, const void* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
                     const int* block_table, const int* seq_lens, float* out, float* lse, uint8_t* hit_mask,
                     int* match_pos, void* stream) {
   if (!s || !K || !V) return MAC_ERR_ARG;
@@ -492,7 +500,7 @@ int mac_append_kv(MacState* s, uint16_t* K, uint16_t* V, const int* block_table,
   return launch_append(p, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
-int mac_warm_start(MacState* s, int n, const float* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
+int mac_warm_start(MacState* s, int n, const void* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
                    const int* block_table, const int* seq_lens, void* stream) {
   if (!s || n < 0 || n > s->W) return MAC_ERR_ARG;
   if (n > 0 && (!q_pre || !rope_pos || !seq_lens || !K || !V)) return MAC_ERR_ARG;
@@ -505,7 +513,7 @@ int mac_warm_start(MacState* s, int n, const float* q_pre, const int* rope_pos, 
   float* out = reinterpret_cast<float*>(s->dev_out + s->off_out);  // outputs of these steps are not kept
   float* lse = reinterpret_cast<float*>(s->dev_out + s->off_lse);
   for (int j = 0; j < n; ++j) {
-    int rc = match_impl(s, 0.f, q_pre + (size_t)j * B * Hq * D, rope_pos + (size_t)j * B, block_table,
+    int rc = match_impl(s, 0.f, static_cast<const unsigned char*>(q_pre) + (size_t)j * B * Hq * D * s->QES, rope_pos + (size_t)j * B, block_table,
                         seq_lens + (size_t)j * B, out, lse, nullptr, nullptr, stream);
     if (rc != MAC_OK) return rc;
     rc = mac_attend(s, K, V, block_table, out, lse, stream);
@@ -530,7 +538,7 @@ static int enqueue_host_step(MacState* s, uint16_t* K, uint16_t* V, const int* b
                        reinterpret_cast<const uint16_t*>(di + s->off_vnew), st);
     if (rc != MAC_OK) return rc;
   }
-  rc = mac_decode_step(s, reinterpret_cast<const float*>(di + s->off_q), reinterpret_cast<const int*>(di + s->off_pos),
+  rc = mac_decode_step(s, di + s->off_q, reinterpret_cast<const int*>(di + s->off_pos),
                        K, V, block_table, lens, reinterpret_cast<float*>(dout + s->off_out),
                        reinterpret_cast<float*>(dout + s->off_lse), dout + s->off_hit,
                        reinterpret_cast<int*>(dout + s->off_mpos), st);
@@ -539,7 +547,7 @@ static int enqueue_host_step(MacState* s, uint16_t* K, uint16_t* V, const int* b
                                                                                                       : MAC_ERR_CUDA;
 }
 
-int mac_decode_step_host(MacState* s, const float* q_pre_h, const int* rope_pos_h, const int* seq_lens_h,
+int mac_decode_step_host(MacState* s, const void* q_pre_h, const int* rope_pos_h, const int* seq_lens_h,
                          const uint16_t* k_new_h, const uint16_t* v_new_h, uint16_t* K, uint16_t* V,
                          const int* block_table, float* out_h, float* lse_h, uint8_t* hit_h, int* match_pos_h,
                          void* stream) {
@@ -551,7 +559,7 @@ int mac_decode_step_host(MacState* s, const float* q_pre_h, const int* rope_pos_
   const size_t B = s->cfg.batch, Hq = s->cfg.num_q_heads, Hkv = s->cfg.num_kv_heads, D = s->D, U = s->U;
   const bool append = k_new_h != nullptr;
   // inputs into the pinned block (the graph copies the whole block in)
-  memcpy(s->host_in + s->off_q, q_pre_h, B * Hq * D * sizeof(float));
+  memcpy(s->host_in + s->off_q, q_pre_h, B * Hq * D * s->QES);
   memcpy(s->host_in + s->off_pos, rope_pos_h, B * sizeof(int));
   memcpy(s->host_in + s->off_lens, seq_lens_h, B * sizeof(int));
   if (append) {
@@ -607,14 +615,14 @@ int mac_get_status(MacState* s, int* device_status) {
 size_t mac_state_bytes(const MacState* s) {
   if (!s) return 0;
   const size_t U = s->U, W1 = s->W + 1, G = s->G, D = s->D;
-  return 8 * sizeof(int) + 2 * U * W1 * G * D * sizeof(float) + 2 * U * W1 * G * sizeof(float) +
+  return 8 * sizeof(int) + 2 * U * W1 * G * D * s->RES + 2 * U * W1 * G * sizeof(float) +
          U * W1 * sizeof(int) + U * sizeof(int);
 }
 
 static int copy_state(MacState* s, void* host, size_t bytes, bool to_host) {
   if (!s || !host || bytes < mac_state_bytes(s)) return MAC_ERR_ARG;
   const size_t U = s->U, W1 = s->W + 1, G = s->G, D = s->D;
-  int hdr[8] = {0x4D414331, (int)U, (int)W1, (int)G, (int)D, 0, 0, 0};
+  int hdr[8] = {0x4D414331, (int)U, (int)W1, (int)G, (int)D, s->cfg.ring_bf16, 0, 0};
   unsigned char* h = static_cast<unsigned char*>(host);
   if (to_host) {
     memcpy(h, hdr, sizeof hdr);
@@ -622,10 +630,11 @@ static int copy_state(MacState* s, void* host, size_t bytes, bool to_host) {
     if (memcmp(h, hdr, sizeof hdr) != 0) return MAC_ERR_SHAPE;
   }
   h += sizeof hdr;
+  const size_t es = s->RES;
   struct Part {
     void* dev;
     size_t bytes;
-  } parts[] = {{s->ring_q, U * W1 * G * D * 4}, {s->ring_o, U * W1 * G * D * 4}, {s->ring_m, U * W1 * G * 4},
+  } parts[] = {{s->ring_q, U * W1 * G * D * es}, {s->ring_o, U * W1 * G * D * es}, {s->ring_m, U * W1 * G * 4},
                {s->ring_l, U * W1 * G * 4},     {s->ring_pos, U * W1 * 4},      {s->steps, U * 4}};
   if (cudaDeviceSynchronize() != cudaSuccess) return MAC_ERR_CUDA;
   for (const Part& p : parts) {

@@ -220,6 +220,21 @@ __device__ __forceinline__ int group_of(const AttendParams& p) {
 template <int GF>
 constexpr bool kBulkML = GF > 0 && GF % 4 == 0;
 
+// Stored outputs o of the window: fp32, or bf16 (rb) rounded to nearest even.
+__device__ __forceinline__ float ring_o_at(const void* base, size_t i, bool rb) {
+  return rb ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(base)[i] << 16)
+            : reinterpret_cast<const float*>(base)[i];
+}
+__device__ __forceinline__ void ring_o_put(void* base, size_t i, float v, bool rb) {
+  if (rb)
+    reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(base)[i] = v;
+}
+__device__ __forceinline__ const unsigned char* ring_o_row(const void* base, size_t i, bool rb) {
+  return reinterpret_cast<const unsigned char*>(base) + i * (rb ? 2 : 4);  // address of element i
+}
+
 // ------------------------------------------------------------ consumer state
 // Per warp, in mma fragment layout (lane = 4*gid + tig): the query columns
 // as B fragments, O^T as C fragments (dims 16*dt + gid and + 8, columns
@@ -452,7 +467,14 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
       float o[FPL];
 #pragma unroll
       for (int f = 0; f < F4; ++f) {
-        const float4 t = __ldcg(reinterpret_cast<const float4*>(p.ring_o + rs * GD + fo) + f);
+        float4 t;
+        if (p.ring_bf16) {
+          const uint2 w = __ldcg(reinterpret_cast<const uint2*>(ring_o_row(p.ring_o, rs * GD + fo, true)) + f);
+          t = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+        } else {
+          t = __ldcg(reinterpret_cast<const float4*>(ring_o_row(p.ring_o, rs * GD + fo, false)) + f);
+        }
         o[4 * f] = t.x * rl;
         o[4 * f + 1] = t.y * rl;
         o[4 * f + 2] = t.z * rl;
@@ -515,7 +537,7 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
     for (int j = 0; j < VEC; ++j) {
       const int idx = threadIdx.x * VEC + j, h = h0 + idx / D, d = idx - (idx / D) * D;
       if (h >= G) continue;
-      p.ring_o[ds * GD + (size_t)h * D + d] = PL[j] > 0.f ? PO[j] / PL[j] : 0.f;
+      ring_o_put(p.ring_o, ds * GD + (size_t)h * D + d, PL[j] > 0.f ? PO[j] / PL[j] : 0.f, p.ring_bf16);
       const float M2 = fmaxf(PM[j], QM[j]);
       const float M2u = M2 == -INFINITY ? 0.f : M2;
       const float a0 = ex2(PM[j] - M2u), a1 = ex2(QM[j] - M2u);
@@ -684,10 +706,10 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D,
     if (hh) {
       const float a = ex2(rm - Mu), rl = sm.ring[GDP + GP + h];
       L += rl * a;
-      O += sm.ring[idx] * rl * a;
+      O += ring_o_at(sm.ring, idx, p.ring_bf16) * rl * a;
     }
     const size_t ds = (size_t)u * Wp1 + dst;
-    p.ring_o[ds * GD + idx] = L > 0.f ? O / L : 0.f;
+    ring_o_put(p.ring_o, ds * GD + idx, L > 0.f ? O / L : 0.f, p.ring_bf16);
     if (d == 0) {
       p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
       p.ring_l[ds * G + h] = L;
@@ -992,11 +1014,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       // per-head matching: each reusing head's state comes from its own slot
       const size_t ub = (size_t)cp.unit * (p.W + 1);
       if (warp == 0) {
-        if (lane == 0) mbar_arrive_expect_tx(&sm.rfull, __popc(hmask) * D * 4);
+        const uint32_t ob = D * (p.ring_bf16 ? 2 : 4);  // bytes of one head's o
+        if (lane == 0) mbar_arrive_expect_tx(&sm.rfull, __popc(hmask) * ob);
         __syncwarp();
         if (lane < G && ((hmask >> lane) & 1)) {
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          bulk_load(sm.ring + lane * D, p.ring_o + ((ub + p.hplan[cp.unit].hsrc[lane]) * G + lane) * D, D * 4,
+          bulk_load(reinterpret_cast<unsigned char*>(sm.ring) + lane * ob,
+                    ring_o_row(p.ring_o, ((ub + p.hplan[cp.unit].hsrc[lane]) * G + lane) * D, p.ring_bf16), ob,
                     &sm.rfull);
         }
       }
@@ -1014,8 +1038,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       const size_t rs = (size_t)cp.unit * (p.W + 1) + cp.src;
       if (tid == 0) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(&sm.rfull, (kBulkML<GF> ? GD + 2 * G : GD) * 4);
-        bulk_load(sm.ring, p.ring_o + rs * GD, GD * 4, &sm.rfull);
+        const uint32_t ob = GD * (p.ring_bf16 ? 2 : 4);  // bytes of the group's o
+        mbar_arrive_expect_tx(&sm.rfull, ob + (kBulkML<GF> ? 2 * G * 4 : 0));
+        bulk_load(sm.ring, ring_o_row(p.ring_o, rs * GD, p.ring_bf16), ob, &sm.rfull);
         if constexpr (kBulkML<GF>) {
           bulk_load(sm.ring + C::GD, p.ring_m + rs * G, G * 4, &sm.rfull);
           bulk_load(sm.ring + C::GD + GP, p.ring_l + rs * G, G * 4, &sm.rfull);

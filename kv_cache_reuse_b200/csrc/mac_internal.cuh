@@ -87,7 +87,7 @@ __host__ __device__ inline int group4(int G) { return (G + 3) & ~3; }
 __host__ __device__ inline size_t partial_floats(int G, int D) { return (size_t)G * D + 2 * (size_t)group4(G); }
 
 struct MatchParams {
-  const float* q_pre;      // [B][Hq][D]
+  const void* q_pre;       // [B][Hq][D] fp32, or bf16 bits (q_bf16)
   const int* rope_pos;     // [B]
   const int* seq_lens;     // [B]
   const int* block_table;  // [B][max_pages] or null
@@ -95,7 +95,7 @@ struct MatchParams {
   float* lse;              // [B][Hq]
   uint8_t* hit_mask;       // [U] ([U][G] with per-head matching) or null
   int* match_pos;          // [U] ([U][G] with per-head matching) or null
-  float* ring_q;           // [U][W+1][G][D]
+  void* ring_q;            // [U][W+1][G][D] fp32, or bf16 bits (ring_bf16)
   const int* ring_pos;     // [U][W+1]
   int* steps;              // [U]
   const double* inv_freq;  // [D/2]
@@ -112,6 +112,8 @@ struct MatchParams {
   unsigned* status;
   int B, Hq, Hkv, G, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
   int per_head;   // 1: one match decision per query head
+  int q_bf16;     // 1: q_pre holds bf16
+  int ring_bf16;  // 1: window queries are stored in bf16
   float tau;
   int grid;       // CTAs of the attention kernel
   int min_keys;   // minimum cost-space units per attention CTA
@@ -135,7 +137,7 @@ struct AttendParams {
   double* cw;        // [grid + 1] cumulative range shares (written by CTA 0)
   float* part;       // [max_parts][partial_floats(G, D)]
   int* unit_cnt;     // [U]
-  float* ring_o;     // [U][W+1][G][D]
+  void* ring_o;      // [U][W+1][G][D] fp32, or bf16 bits (ring_bf16)
   float* ring_m;     // [U][W+1][G]
   float* ring_l;     // [U][W+1][G]
   int* ring_pos;     // [U][W+1]
@@ -144,6 +146,7 @@ struct AttendParams {
   unsigned* status;
   int Hq, Hkv, G, W, page_size, max_pages, nseg, grid;
   int per_head;      // 1: heads of a unit reuse states on their own (plan hmask, hstart, hsrc)
+  int ring_bf16;     // 1: stored outputs o are bf16
 };
 
 struct AppendParams {

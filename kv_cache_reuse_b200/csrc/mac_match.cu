@@ -29,6 +29,10 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <type_traits>
+
+#include <cuda_bf16.h>
+
 #include "mac_internal.cuh"
 
 #include "../../include/mac.h"
@@ -40,6 +44,19 @@ constexpr double kLog2e = 1.4426950408889634;
 constexpr double kInvTwoPi = 0.15915494309189535;
 constexpr double kTwoPiHi = 6.2831853069365025;    // 2*pi with the low 21 mantissa bits cleared
 constexpr double kTwoPiLo = 2.430840202602477e-10;   // 2*pi - kTwoPiHi
+
+// Four window elements: fp32 as they are, bf16 (two per 32-bit word, the
+// first in the low half) widened exactly.
+__device__ __forceinline__ float4 widen4(const float4& v) { return v; }
+__device__ __forceinline__ float4 widen4(const uint2& v) {
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
+                     __uint_as_float(v.y & 0xffff0000u));
+}
+// Four fp32 values rounded to bf16 (nearest even), packed as widen4 reads them.
+__device__ __forceinline__ uint2 narrow4(const float4& v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -235,9 +252,11 @@ __device__ void build_segments(const MatchParams& p, int U, double cw_c) {
 // GP: the query group padded to 4 or 8 heads (register and shared-memory
 // shapes); the real group G <= GP sets every global layout.  GF = G for the
 // variants built for one group size (4, 8), 0 for a run-time G (p.G).
-// PH: one decision per query head (per-head matching).
-template <int D, int GP, int GF, bool PH>
+// PH: one decision per query head (per-head matching).  RB: the window's
+// queries are stored in bf16.
+template <int D, int GP, int GF, bool PH, bool RB>
 __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchParams p) {
+  using RT = std::conditional_t<RB, uint2, float4>;  // four window elements
   const int G = GF > 0 ? GF : p.G;
   const int GD = G * D;
   __shared__ __align__(16) float sq[GP * D];
@@ -264,15 +283,15 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   constexpr int NW = kMatchThreads / 32;
   constexpr int BS = GP == 4 ? 5 : 3;  // slots per warp per batch of loads (8 warps x 5 >= W+1 for W <= 39)
   constexpr int F4 = GP * D / 4 / 32;  // float4 per lane per slot, at most
-  const int n4 = GD / 4;               // float4 of one slot
-  float4 r[BS][F4];
+  const int n4 = GD / 4;               // groups of four elements of one slot
+  RT r[BS][F4];
   int rpos[BS];
   auto load_batch = [&](int s0) {
 #pragma unroll
     for (int k = 0; k < BS; ++k) {
       const int slot = s0 + k * NW;
       if (slot < Wp1) {
-        const float4* rq = reinterpret_cast<const float4*>(p.ring_q + ((size_t)u * Wp1 + slot) * GD);
+        const RT* rq = reinterpret_cast<const RT*>(p.ring_q) + ((size_t)u * Wp1 + slot) * n4;
 #pragma unroll
         for (int f = 0; f < F4; ++f)
           if (lane + 32 * f < n4) r[k][f] = rq[lane + 32 * f];
@@ -281,8 +300,14 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
     }
   };
   load_batch(warp);
-  const float4* qsrc = reinterpret_cast<const float4*>(p.q_pre + ((size_t)b * p.Hq + (size_t)kvh * G) * D);
-  for (int i = tid; i < n4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = qsrc[i];
+  const size_t q0 = ((size_t)b * p.Hq + (size_t)kvh * G) * D / 4;  // first group of four of the query
+  if (p.q_bf16) {
+    const uint2* qsrc = reinterpret_cast<const uint2*>(p.q_pre) + q0;
+    for (int i = tid; i < n4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = widen4(qsrc[i]);
+  } else {
+    const float4* qsrc = reinterpret_cast<const float4*>(p.q_pre) + q0;
+    for (int i = tid; i < n4; i += kMatchThreads) reinterpret_cast<float4*>(sq)[i] = qsrc[i];
+  }
   const int len = p.seq_lens[b];
   const int p_t = len - 1;
   const int n = p.steps[u];
@@ -321,8 +346,8 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
             const int i4 = lane + 32 * f;
             float a = 0.f;
             if (i4 < n4) {
-              const float4 q = reinterpret_cast<const float4*>(sq)[i4];
-              const float dx = q.x - r[k][f].x, dy = q.y - r[k][f].y, dz = q.z - r[k][f].z, dw = q.w - r[k][f].w;
+              const float4 q = reinterpret_cast<const float4*>(sq)[i4], e = widen4(r[k][f]);
+              const float dx = q.x - e.x, dy = q.y - e.y, dz = q.z - e.z, dw = q.w - e.w;
               a = fmaf(dx, dx, a);
               a = fmaf(dy, dy, a);
               a = fmaf(dz, dz, a);
@@ -341,8 +366,8 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
 #pragma unroll
           for (int f = 0; f < F4; ++f) {
             if (lane + 32 * f >= n4) break;
-            const float4 q = reinterpret_cast<const float4*>(sq)[lane + 32 * f];
-            const float dx = q.x - r[k][f].x, dy = q.y - r[k][f].y, dz = q.z - r[k][f].z, dw = q.w - r[k][f].w;
+            const float4 q = reinterpret_cast<const float4*>(sq)[lane + 32 * f], e = widen4(r[k][f]);
+            const float dx = q.x - e.x, dy = q.y - e.y, dz = q.z - e.z, dw = q.w - e.w;
             acc = fmaf(dx, dx, acc);
             acc = fmaf(dy, dy, acc);
             acc = fmaf(dz, dz, acc);
@@ -477,9 +502,15 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
         dst[i + D / 2] = (float)((y * cs + x * sn) * scale);
       }
     }
-    // 5. this step's query enters the ring
-    float4* rdst = reinterpret_cast<float4*>(p.ring_q + ((size_t)u * Wp1 + s_plan.dst_slot) * GD);
-    for (int i = tid; i < n4; i += kMatchThreads) rdst[i] = reinterpret_cast<const float4*>(sq)[i];
+    // 5. this step's query enters the ring (bf16: rounded to nearest even)
+    RT* rdst = reinterpret_cast<RT*>(p.ring_q) + ((size_t)u * Wp1 + s_plan.dst_slot) * n4;
+    for (int i = tid; i < n4; i += kMatchThreads) {
+      const float4 v = reinterpret_cast<const float4*>(sq)[i];
+      if constexpr (RB)
+        rdst[i] = narrow4(v);
+      else
+        rdst[i] = v;
+    }
     if (tid < nd) {
       if (p.hit_mask) p.hit_mask[u * nd + tid] = (uint8_t)s_dhit[tid];
       if (p.match_pos) p.match_pos[u * nd + tid] = s_dpos[tid];
@@ -509,22 +540,29 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
 
 // Variants as for the attention kernel: exact groups of 4 and 8, run-time
 // groups padded to 4 and 8, and per-head matching (run-time group).
-template <int D>
-void launch_d(const MatchParams& p, int U, cudaStream_t s) {
+template <int D, bool RB>
+void launch_dr(const MatchParams& p, int U, cudaStream_t s) {
   if (p.per_head) {
     if (p.G <= 4)
-      mac_match_kernel<D, 4, 0, true><<<U, kMatchThreads, 0, s>>>(p);
+      mac_match_kernel<D, 4, 0, true, RB><<<U, kMatchThreads, 0, s>>>(p);
     else
-      mac_match_kernel<D, 8, 0, true><<<U, kMatchThreads, 0, s>>>(p);
+      mac_match_kernel<D, 8, 0, true, RB><<<U, kMatchThreads, 0, s>>>(p);
   } else if (p.G == 4) {
-    mac_match_kernel<D, 4, 4, false><<<U, kMatchThreads, 0, s>>>(p);
+    mac_match_kernel<D, 4, 4, false, RB><<<U, kMatchThreads, 0, s>>>(p);
   } else if (p.G == 8) {
-    mac_match_kernel<D, 8, 8, false><<<U, kMatchThreads, 0, s>>>(p);
+    mac_match_kernel<D, 8, 8, false, RB><<<U, kMatchThreads, 0, s>>>(p);
   } else if (p.G < 4) {
-    mac_match_kernel<D, 4, 0, false><<<U, kMatchThreads, 0, s>>>(p);
+    mac_match_kernel<D, 4, 0, false, RB><<<U, kMatchThreads, 0, s>>>(p);
   } else {
-    mac_match_kernel<D, 8, 0, false><<<U, kMatchThreads, 0, s>>>(p);
+    mac_match_kernel<D, 8, 0, false, RB><<<U, kMatchThreads, 0, s>>>(p);
   }
+}
+template <int D>
+void launch_d(const MatchParams& p, int U, cudaStream_t s) {
+  if (p.ring_bf16)
+    launch_dr<D, true>(p, U, s);
+  else
+    launch_dr<D, false>(p, U, s);
 }
 
 }  // namespace

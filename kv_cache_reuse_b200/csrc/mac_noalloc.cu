@@ -168,7 +168,9 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.lse = lse;
   mp.hit_mask = nullptr;
   mp.match_pos = nullptr;
-  mp.ring_q = reinterpret_cast<float*>(base + kOffRingQ);
+  mp.ring_q = base + kOffRingQ;
+  mp.q_bf16 = 0;
+  mp.ring_bf16 = 0;
   mp.ring_pos = reinterpret_cast<const int*>(base + kOffRingPos);
   mp.steps = cnt + kMaxUnits + 2;
   mp.inv_freq = reinterpret_cast<const double*>(base + kOffInv);
@@ -222,7 +224,8 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.cw = nullptr;
   ap.part = reinterpret_cast<float*>(base + kOffPart);
   ap.unit_cnt = cnt;
-  ap.ring_o = reinterpret_cast<float*>(base + kOffRingO);
+  ap.ring_o = base + kOffRingO;
+  ap.ring_bf16 = 0;
   ap.ring_m = reinterpret_cast<float*>(base + kOffRingM);
   ap.ring_l = reinterpret_cast<float*>(base + kOffRingL);
   ap.ring_pos = reinterpret_cast<int*>(base + kOffRingPos);

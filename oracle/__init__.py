@@ -38,7 +38,7 @@ class _Cfg(C.Structure):
     _fields_ = [("B", C.c_int), ("Hq", C.c_int), ("Hkv", C.c_int), ("D", C.c_int),
                 ("W", C.c_int), ("band", C.c_int), ("tau", C.c_double), ("rope_theta", C.c_double),
                 ("page_size", C.c_int), ("max_seq", C.c_int), ("max_pages_per_seq", C.c_int),
-                ("cut_mode", C.c_int), ("per_head", C.c_int)]
+                ("cut_mode", C.c_int), ("per_head", C.c_int), ("ring_bf16", C.c_int)]
 
 
 def _load():
@@ -122,10 +122,10 @@ class Oracle:
     """Stateful fp64 MAC decode oracle: one instance per layer of KV heads."""
 
     def __init__(self, B, Hq, Hkv, D, W, band, tau, rope_theta, page_size=0, max_seq=0,
-                 max_pages_per_seq=0, cut_mode=0, per_head=0):
+                 max_pages_per_seq=0, cut_mode=0, per_head=0, ring_bf16=0):
         self.lib = _load()
         self.cfg = _Cfg(B, Hq, Hkv, D, W, band, float(tau), float(rope_theta), page_size, max_seq,
-                        max_pages_per_seq, cut_mode, per_head)
+                        max_pages_per_seq, cut_mode, per_head, ring_bf16)
         self.h = self.lib.oracle_create(C.byref(self.cfg))
         if not self.h:
             raise ValueError("invalid oracle configuration")
@@ -134,11 +134,11 @@ class Oracle:
         self.nd = Hkv * (self.G if per_head else 1)  # match decisions per sequence
 
     @classmethod
-    def for_workload(cls, wl, cache, tau=None, band=None, W=None, cut_mode=0, per_head=0):
+    def for_workload(cls, wl, cache, tau=None, band=None, W=None, cut_mode=0, per_head=0, ring_bf16=0):
         return cls(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W if W is None else W, wl.band if band is None else band,
                    wl.tau if tau is None else tau, wl.rope_theta, wl.page_size,
                    cache.max_seq if not cache.paged else 0,
-                   cache.block_table.shape[1] if cache.paged else 0, cut_mode, per_head)
+                   cache.block_table.shape[1] if cache.paged else 0, cut_mode, per_head, ring_bf16)
 
     def __del__(self):
         try:

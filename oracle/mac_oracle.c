@@ -40,6 +40,11 @@
  *                 with rotate-half pairs (i, i + D/2), inv_freq_i =
  *                 theta^(-2i/D), angle in fp64;
  *   [scale]       scores are q.k / sqrt(D), natural-log units;
+ *   [bf16-ring]   with a bf16 window, an entry keeps its pre-RoPE query and the
+ *                 normalised output o of its prefix state rounded to bf16
+ *                 (round to nearest even, o first rounded to fp32, the
+ *                 precision the output is computed in); m and l keep their
+ *                 precision;
  *   [warm]        a window seeded from prefill holds, for each of the last n
  *                 prefill positions, its pre-RoPE query and its prefix state
  *                 over [0, c) with the query rotated at that position -- the
@@ -67,6 +72,7 @@ typedef struct {
     int max_pages_per_seq; /* block table row length (paged: K/V [P][page][Hkv][D]) */
     int cut_mode;          /* [cut]: 0 or 1 */
     int per_head;          /* 0: one decision per KV head ([mean-dist]); 1: per query head ([per-head]) */
+    int ring_bf16;         /* 1: entries keep q and o rounded to bf16 ([bf16-ring]) */
 } ocfg_t;
 
 typedef struct {
@@ -87,6 +93,19 @@ static double bf16_to_f64(uint16_t h) {
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* [bf16-ring] The bf16 value nearest to x (ties to the even bf16), as a
+ * float: keep the top 16 bits of the fp32 pattern after adding half a unit
+ * of the 17th bit, plus one when the kept part is odd.  NaN stays NaN. */
+static float round_bf16(float x) {
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu)) return x;
+    u = (u + 0x7fffu + ((u >> 16) & 1u)) & 0xffff0000u;
+    float r;
+    memcpy(&r, &u, sizeof r);
+    return r;
 }
 
 /* Row of key (or value) position k of sequence b, KV head kvh. */
@@ -204,7 +223,7 @@ void oracle_merge(const double *o1, double m1, double l1, const double *o2, doub
 ostate_t *oracle_create(const ocfg_t *cfg) {
     if (!cfg || cfg->Hkv <= 0 || cfg->Hq % cfg->Hkv != 0 || cfg->D <= 0 || (cfg->D & 1) || cfg->W < 0 ||
         cfg->band < 0 || cfg->B <= 0 || cfg->cut_mode < 0 || cfg->cut_mode > 1 || cfg->per_head < 0 ||
-        cfg->per_head > 1)
+        cfg->per_head > 1 || cfg->ring_bf16 < 0 || cfg->ring_bf16 > 1)
         return NULL;
     ostate_t *s = (ostate_t *)calloc(1, sizeof(ostate_t));
     s->c = *cfg;
@@ -310,6 +329,14 @@ static void push_entry(ostate_t *s, int u, const float *qg, const double *sn, co
     int slot = s->n[u];
     memcpy(s->wq + ((size_t)u * W + slot) * gd, qg, sizeof(float) * gd);
     memcpy(s->wo + ((size_t)u * W + slot) * gd, sn, sizeof(double) * gd);
+    if (s->c.ring_bf16) {
+        float *q = s->wq + ((size_t)u * W + slot) * gd;
+        double *o = s->wo + ((size_t)u * W + slot) * gd;
+        for (size_t i = 0; i < gd; ++i) {
+            q[i] = round_bf16(q[i]);
+            o[i] = (double)round_bf16((float)o[i]);
+        }
+    }
     memcpy(s->wm + ((size_t)u * W + slot) * G, snm, sizeof(double) * (size_t)G);
     memcpy(s->wl + ((size_t)u * W + slot) * G, snl, sizeof(double) * (size_t)G);
     s->wpos[(size_t)u * W + slot] = p_t;

@@ -367,6 +367,55 @@ def test_per_head_host_entry_matches_device_entry():
             np.testing.assert_array_equal(u, v)
 
 
+@pytest.mark.parametrize("case", ["tiny", "llama", "split", "g3_paged", "g8", "per_head", "q_only", "q_and_ring",
+                                  "q_paged_per_head"])
+def test_bf16_window_and_queries(case):
+    """bf16 window (queries and stored outputs rounded to bf16, as the oracle
+    does) and bf16 query input, alone and together, over the kernel variants."""
+    tiny, llama, paged = synth.WORKLOADS["tiny"], synth.WORKLOADS["llama8b_32k"], synth.WORKLOADS["paged_mixed"]
+    tune, ph, qb, rb = None, 0, 0, 1
+    if case == "tiny":
+        wl = tiny.with_(steps=48)
+    elif case == "llama":
+        wl = llama.with_(L0=(6000,), steps=48)
+    elif case == "split":
+        wl, tune = tiny.with_(steps=40), _SPLIT
+    elif case == "g3_paged":
+        wl = paged.with_(B=3, Hq=12, Hkv=4, L0=(2500, 900, 4100), steps=16)
+    elif case == "g8":
+        wl = llama.with_(B=2, Hq=64, Hkv=8, L0=(9000, 4000), steps=16)
+    elif case == "per_head":
+        wl, ph = tiny.with_(head_labels=True, steps=40), 1
+    elif case == "q_only":
+        wl, qb, rb = llama.with_(L0=(6000,), steps=32), 1, 0
+    elif case == "q_and_ring":
+        wl, qb = tiny.with_(steps=40), 1
+    else:
+        wl, qb, ph = paged.with_(B=3, Hq=8, Hkv=2, L0=(2500, 900, 4100), steps=16, head_labels=True), 1, 1
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tune=tune, per_head=ph, q_bf16=qb, ring_bf16=rb)
+    assert r["hits"] > 0
+
+
+def test_bf16_window_export_matches_oracle_window():
+    """The exported bf16 window: queries bit-equal to the rounded inputs; the
+    stored outputs (bf16 bits) within the output tolerance of the oracle's
+    rounded ones, as for the fp32 window (rounding to neighbouring bf16 values
+    can carry along chains of hits)."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(steps=24)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    r = compare_stream(wl, stream, cache, ring_bf16=1)
+    st = mac.parse_state(r["gpu"].st.export_state(), wl.W, wl.G, wl.D)
+    assert st["q"].dtype == np.uint16 and st["o"].dtype == np.uint16
+    q, o, m, l, pos = r["oracle"].window(0)
+    n = len(pos)
+    W1 = wl.W + 1
+    slots = [(wl.steps - n + i) % W1 for i in range(n)]  # entry of step k sits in slot k mod (W+1)
+    np.testing.assert_array_equal(st["q"][0, slots], synth.f32_to_bf16_bits(q))
+    np.testing.assert_allclose(synth.bf16_bits_to_f32(st["o"][0, slots]), o, rtol=0, atol=OUT_TOL)
+    np.testing.assert_array_equal(st["pos"][0, slots], pos)
+
+
 @pytest.mark.parametrize("case", ["tiny", "split", "band0", "llama_paged"])
 def test_cut_mode_band_ends_at_position(case):
     """cut_mode 1: the stored prefix ends at max(0, p + 1 - band) on both sides."""

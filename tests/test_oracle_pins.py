@@ -529,3 +529,97 @@ def test_per_head_keys_read_is_the_union_of_head_ranges():
             first = min(max(0, int(m) - wl.band) if m >= 0 else 0 for m in mp)
             want += p_t + 1 - first
         assert r.keys_read == want, t
+
+
+# ------------------------------------------------------------ bf16 ring pins
+def _torch_bf16(x):
+    """fp32 -> bf16 -> fp32 through torch's own conversion (round to nearest even)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def test_bf16_ring_window_holds_rounded_queries_and_states():
+    """With a bf16 window every entry keeps bf16(q) and bf16(fp32(o)) of its
+    prefix state (a forced-miss step's prefix state is dense attention over
+    [0, c)), and m, l unrounded."""
+    wl = _tiny(steps=6, L0=(300,))
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=0.0, ring_bf16=1)
+    ref = oracle.Oracle.for_workload(wl, cache, tau=0.0)
+    for t in range(wl.steps):
+        orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        ref.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+    q, o, m, l, pos = orc.window(0)
+    rq, ro, rm, rl, rpos = ref.window(0)
+    np.testing.assert_array_equal(q, _torch_bf16(stream.q[:wl.steps, 0]))
+    np.testing.assert_array_equal(pos, rpos)
+    np.testing.assert_array_equal(m, rm)
+    np.testing.assert_array_equal(l, rl)
+    # o against numpy dense attention over the stored prefix [0, c), rounded the same way
+    for e in range(wl.steps):
+        p = int(pos[e])
+        cut = max(0, p - wl.band)
+        Kd = decode(cache.K[0, :cut, 0])
+        Vd = decode(cache.V[0, :cut, 0])
+        qr = np.stack([rope_complex(stream.q[e, 0, h], p, wl.rope_theta) for h in range(wl.G)])
+        od, _ = dense_attention(qr, Kd, Vd)
+        np.testing.assert_array_equal(o[e], _torch_bf16(od.astype(np.float32)))
+    assert (o != ro).any()  # the rounding is really applied
+
+
+def test_bf16_ring_forced_miss_equals_dense():
+    wl = _tiny(steps=8)
+    stream, cache, res = _run(wl, tau=0.0)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=0.0, ring_bf16=1)
+    for t in range(wl.steps):
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        np.testing.assert_array_equal(r.out, res[t].out)
+        np.testing.assert_array_equal(r.lse, res[t].lse)
+
+
+def test_bf16_ring_first_hit_reuses_the_rounded_state():
+    """The first hit of a stream (no earlier reuse, so both windows hold the
+    same states up to rounding) equals the fp32-window computation with only
+    the reused o replaced by bf16(o): reused state (+) amend band, (+) tail."""
+    wl = _tiny(steps=40)
+    stream = synth.queries(wl)
+    cache = synth.kv_cache(wl)
+    a = oracle.Oracle.for_workload(wl, cache)
+    b = oracle.Oracle.for_workload(wl, cache, ring_bf16=1)
+    K2, V2 = cache.K[0, :, 0], cache.V[0, :, 0]
+    for t in range(wl.steps):
+        _, wo, wm, wl_, wpos = a.window(0)  # the fp32 window before this step
+        ra = a.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        rb = b.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, None, stream.seq_lens[t])
+        np.testing.assert_array_equal(ra.hit, rb.hit)
+        if not ra.hit.any():
+            np.testing.assert_array_equal(ra.out, rb.out)
+            continue
+        p_s, p_t = int(ra.match_pos[0, 0]), int(stream.seq_lens[t][0]) - 1
+        e = int(np.nonzero(wpos == p_s)[0][-1])
+        c_s, c_t = max(0, p_s - wl.band), max(0, p_t - wl.band)
+        for h in range(wl.G):
+            qr = oracle.rope(stream.q[t, 0, h], int(stream.rope_pos[t][0]), wl.rope_theta)
+            reused = (_torch_bf16(wo[e, h].astype(np.float32)).astype(np.float64), wm[e, h], wl_[e, h])
+            S = oracle.merge(reused, oracle.partial(qr, K2, V2, c_s, c_t))
+            o, m, l = oracle.merge(S, oracle.partial(qr, K2, V2, c_t, p_t + 1))
+            np.testing.assert_allclose(rb.out[0, h], o, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(rb.lse[0, h], m + np.log(l), rtol=0, atol=1e-12)
+        assert float(np.abs(ra.out - rb.out).max()) > 0.0  # the rounding reached the output
+        return
+    raise AssertionError("the stream has no hit")
+
+
+def test_bf16_ring_keeps_decisions_on_the_workload_margins():
+    """Rounding the stored queries moves distances far less than the
+    generator's margins: every decision of the stream is unchanged."""
+    wl = synth.WORKLOADS["llama8b_32k"]
+    stream = synth.queries(wl)
+    a = oracle.Oracle(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W, wl.band, wl.tau, wl.rope_theta)
+    b = oracle.Oracle(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W, wl.band, wl.tau, wl.rope_theta, ring_bf16=1)
+    for t in range(wl.steps):
+        ha, pa, _, _ = a.match_step(stream.q[t], stream.seq_lens[t])
+        hb, pb, _, _ = b.match_step(stream.q[t], stream.seq_lens[t])
+        np.testing.assert_array_equal(ha, hb)
+        np.testing.assert_array_equal(pa, pb)
