@@ -122,25 +122,31 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
-def step_bytes(wl, hit, mpos, seq_lens, occ):
+def step_bytes(wl, hit, mpos, seq_lens, occ, qes=4, res=4):
     """Algorithmic HBM bytes of one step: (match kernel, attention kernel, K/V only).
 
-    Match: query G*D*4 per unit, window scan occ*G*D*4, ring-q write and rotated
-    query write G*D*4 each.  Attention: K+V of every key attended fresh
-    (2*D*2 per key), rotated query G*D*4, reused state G*(D+2)*4 on a hit, new
-    state G*(D+2)*4 + position, out and lse G*(D+1)*4.
+    hit, mpos: [B][Hkv] decisions, or [B][Hq] with per-head matching.  qes, res:
+    bytes of a query element and of a window element (q and stored o).
+    Match: query G*D*qes per unit, window scan occ*G*D*res, ring-q write
+    G*D*res, rotated query write G*D*4.  Attention: K+V of every key attended
+    fresh -- the union of the unit's heads' ranges -- (2*D*2 per key), rotated
+    query G*D*4, reused state (D*res + 8) per reusing head, new state
+    G*(D*res + 8) + position, out and lse G*(D+1)*4.
     """
     G, D, band = wl.G, wl.D, wl.band
-    gd4 = G * D * 4
+    hpd = G * wl.Hkv // hit.shape[1]  # heads per decision
+    gd = G * D
     kv = att = mt = 0
     for b in range(wl.B):
         p_t = int(seq_lens[b]) - 1
         for h in range(wl.Hkv):
-            start = max(0, int(mpos[b, h]) - band) if hit[b, h] else 0
+            dec = range(h * G // hpd, (h + 1) * G // hpd)
+            start = min(max(0, int(mpos[b, d]) - band) if hit[b, d] else 0 for d in dec)
+            reusing = sum(hpd for d in dec if hit[b, d])
             keys = p_t + 1 - start
             kv += keys * 2 * D * 2
-            att += gd4 + (G * (D + 2) * 4 if hit[b, h] else 0) + G * (D + 2) * 4 + 4 + G * (D + 1) * 4
-            mt += gd4 + occ * gd4 + 2 * gd4
+            att += gd * 4 + reusing * (D * res + 8) + G * (D * res + 8) + 4 + G * (D + 1) * 4
+            mt += gd * qes + occ * gd * res + gd * res + gd * 4
     return mt, att + kv, kv
 
 
@@ -186,8 +192,8 @@ def run_mac(args, rank, world, local_rank):
     lens_all = torch.from_numpy(stream.seq_lens).to(dev)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
     lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-    hit_all = torch.zeros((T, B, Hkv), dtype=torch.uint8, device=dev)
-    mpos_all = torch.zeros((T, B, Hkv), dtype=torch.int32, device=dev)
+    hit_all = torch.zeros((T, B, Hq), dtype=torch.uint8, device=dev)  # [B][Hkv] used unless per-head
+    mpos_all = torch.zeros((T, B, Hq), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     s = torch.cuda.current_stream(dev)
     peak, peak_kind = _peaks()
@@ -201,14 +207,16 @@ def run_mac(args, rank, world, local_rank):
         return (qsrc[0][t].data_ptr(), pos_all[t].data_ptr(), lens_all[t].data_ptr(), hit_all[t].data_ptr(),
                 mpos_all[t].data_ptr())
 
-    def timed_run(tau, nwarm, nsteps, split):
+    def timed_run(tau, nwarm, nsteps, split, cfg=None, bytes_stream=None):
         """Warm-up, then nsteps timed steps.  split=False: one mac_decode_step per
         step (match and attend back to back, programmatic launch), events around
         the step.  split=True: events also between the two kernels, for the
         per-kernel roofline.  The timed steps are queued behind a GPU sleep so the
         host stays ahead of the device and no host latency enters the events."""
-        st = mac.MacState.for_workload(wl, tau=tau, **kw)
+        cfg = cfg or {}
+        st = mac.MacState.for_workload(wl, tau=tau, **kw, **cfg)
         h = st.handle
+        nd = Hq if cfg.get("match_per_head") else Hkv  # decisions per sequence
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
         Kp, Vp, btp, outp, lsep = K.data_ptr(), V.data_ptr(), (bt.data_ptr() if bt is not None else None), \
@@ -246,13 +254,16 @@ def run_mac(args, rank, world, local_rank):
         step_ms = [a.elapsed_time(c) for a, b_, c in ev]
         att_ms = [b_.elapsed_time(c) for a, b_, c in ev] if split else [0.0] * nsteps
         match_ms = [a.elapsed_time(b_) for a, b_, c in ev] if split else [0.0] * nsteps
-        hits = hit_all[nwarm:nwarm + nsteps].cpu().numpy()
-        mpos = mpos_all[nwarm:nwarm + nsteps].cpu().numpy()
+        # decisions of a step: the first nd entries of each step's buffer, [B][nd]
+        hits = hit_all.view(T, -1)[nwarm:nwarm + nsteps, :B * nd].reshape(nsteps, B, nd).cpu().numpy()
+        mpos = mpos_all.view(T, -1)[nwarm:nwarm + nsteps, :B * nd].reshape(nsteps, B, nd).cpu().numpy()
+        qes = 2 if cfg.get("q_bf16") else 4
+        res_ = 2 if cfg.get("ring_bf16") else 4
         mt_b = at_b = kv_b = dense_b = 0
         for i in range(nsteps):
             t = nwarm + i
             occ = min(t, wl.W)
-            a, b_, c = step_bytes(wl, hits[i], mpos[i], stream.seq_lens[t], occ)
+            a, b_, c = step_bytes(wl, hits[i], mpos[i], stream.seq_lens[t], occ, qes, res_)
             mt_b += a
             at_b += b_
             kv_b += c
@@ -286,6 +297,23 @@ def run_mac(args, rank, world, local_rank):
                 "frac": wbytes / (wms * 1e-3) / 1e9 / peak, "device_status": st.get_status()}
         st.close()
     layers = run_layers(args, wl, stream, cache, K, V, bt, kw, dev, peak) if args.layers > 0 else None
+    bf16 = None
+    if not args.no_bf16:
+        # bf16 queries and bf16 window: the same stream with its queries rounded to bf16
+        qsrc[0] = torch.from_numpy(synth.f32_to_bf16_bits(stream.q).view(np.int16)).to(dev)
+        cfg = {"q_bf16": 1, "ring_bf16": 1}
+        bf16 = (timed_run(wl.tau, args.warmup, args.steps, split=False, cfg=cfg),
+                timed_run(wl.tau, args.warmup, args.steps, split=True, cfg=cfg))
+        qsrc[0] = q_all
+    perhead = None
+    if not args.no_per_head:
+        # per-head matching on a stream whose query heads repeat on their own
+        wh = wl.with_(head_labels=True)
+        qsrc[0] = torch.from_numpy(synth.queries(wh, T).q).to(dev)
+        cfg = {"match_per_head": 1}
+        perhead = (timed_run(wl.tau, args.warmup, args.steps, split=False, cfg=cfg),
+                   timed_run(wl.tau, args.warmup, args.steps, split=True, cfg=cfg))
+        qsrc[0] = q_all
     hitrun = None
     if args.hit_steps > 0:
         # the hit path alone: the same shape with every labelled step a near-repeat
@@ -352,6 +380,22 @@ def run_mac(args, rank, world, local_rank):
                            "attend_bytes_per_step": hitrun["att_bytes"] / n, "attend_gbs": h_gbs,
                            "attend_frac": h_gbs / peak, "clocks": hitrun["clocks"],
                            "note": "latency-bound: a few MB per launch"}
+    for name, pair, what in (("bf16_window", bf16, {"q": "bf16", "window_q_and_o": "bf16"}),
+                             ("per_head", perhead, {"matching": "per query head",
+                                                    "stream": "each query head repeats a recent query of its own "
+                                                              "(rate as the workload) or draws fresh"})):
+        if not pair:
+            continue
+        run, kr = pair
+        a_gbs = kr["att_bytes"] / (kr["att_ms"] * 1e-3) / 1e9
+        res[name] = dict(what, **{
+            "steps_per_s": K_ / (run["total_ms"] * 1e-3), "ms_per_step": run["total_ms"] / K_,
+            "vs_headline": (K_ / (run["total_ms"] * 1e-3)) / (world * K_ / (tot * 1e-3)),
+            "hit_fraction": run["hit_frac"], "match_ms_per_step": kr["match_ms"] / K_,
+            "attend_ms_per_step": kr["att_ms"] / K_, "match_bytes_per_step": kr["match_bytes"] / K_,
+            "attend_bytes_per_step": kr["att_bytes"] / K_, "attend_gbs": a_gbs, "attend_frac": a_gbs / peak,
+            "match_gbs": kr["match_bytes"] / (kr["match_ms"] * 1e-3) / 1e9,
+            "clocks": run["clocks"], "device_status": run["status"]})
     if warm:
         res["warm_start"] = warm
     if layers:
@@ -539,6 +583,8 @@ def main():
     ap.add_argument("--warm-start", action="store_true", help="also time seeding the windows from W positions")
     ap.add_argument("--layers", type=int, default=0,
                     help="also time a stack of this many layers per token, one CUDA graph per token")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 query / window run")
+    ap.add_argument("--no-per-head", action="store_true", help="skip the per-head matching run")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
