@@ -431,13 +431,14 @@ __device__ __forceinline__ void fold_state(float& M, float& L, float (&O)[N], fl
 // stored in the ring; that state and segment B's partials give the output.
 // Four heads at a time: the 8 warps share the partials (warp w folds
 // partials w, w + 8, ..., each lane FPL consecutive floats of one head), with
-// up to 48 partials' loads in flight at once; the warps' states then meet in
+// up to 16 partials' loads in flight at once; the warps' states then meet in
 // shared memory.
 template <int D, int GP, int GF, bool PH>
 __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
   constexpr int QD = 4 * D;                    // floats of four heads
   constexpr int FPL = QD / 32, F4 = FPL / 4;   // floats and float4 of those per lane
-  constexpr int BP = 6;                        // partials per warp per round of loads
+  constexpr int BP = 2;                        // partials per warp per round of loads (the code runs cold
+                                               // once per step: a short loop beats more loads in flight)
   constexpr int VEC = QD / (kConsumerWarps * 32);
   static_assert(VEC * kConsumerWarps * 32 == QD && F4 * 4 * 32 == QD, "merge layout");
   const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
@@ -511,7 +512,7 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
     // the warps' sets meet in shared memory ([4][D], m [4], l [4]): set A
     // (prefix), then set B (tail)
     float PM[VEC], PL[VEC], PO[VEC], QM[VEC], QL[VEC], QO[VEC];
-#pragma unroll
+#pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
       for (int j = 0; j < FPL; ++j) wb[f0 + j] = pass == 0 ? OA[j] : OB[j];
@@ -641,6 +642,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D
   warp_combine_store<D, GP>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   float* dst = p.part + (size_t)pidx * (GD + 2 * G4);
+#pragma unroll 1
   for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
     const int h = idx / D;
     float MA, LA, OA, M, L, O;
@@ -689,7 +691,8 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D,
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   // the reused o was copied on chip at the start of the piece
   if (hit && !mbar_wait(&sm.rfull, ring_phase, &sm.abort_flag, p.status)) return false;
-#pragma unroll
+  // cold code once per piece: a rolled loop fetches fewer instruction lines
+#pragma unroll 1
   for (int k = 0; k < PER; ++k) {
     const int idx = threadIdx.x + k * kConsumerWarps * 32;
     if (idx >= GD) break;
