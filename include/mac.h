@@ -274,6 +274,17 @@ int mac_dense_decode_static(const float *q_pre, const int *rope_pos, const uint1
                             int page_size, int max_seq, int max_pages_per_seq, int num_pages,
                             void *stream);
 
+/* Self-test of the device-side failure path.  Every wait inside the
+ * library's kernels is bounded (2 s of %globaltimer); when one gives up, the
+ * kernel sets MAC_DEV_TIMEOUT in its status word, lets its own copies land
+ * and returns, so the context stays usable and the host learns of it from
+ * the status.  This call enqueues one small kernel that waits, through the
+ * same bounded wait, on a barrier nothing arrives on: after about 2 s it
+ * ORs MAC_DEV_TIMEOUT into *device_status (device uint32, caller-owned) and
+ * exits.  No fault, trap or hang is involved.  Returns MAC_ERR_ARG for a
+ * NULL status, MAC_ERR_CUDA if the launch fails. */
+int mac_selftest_wait_timeout(unsigned *device_status, void *stream);
+
 /* Static description of a return code. */
 const char *mac_error_string(int code);
 

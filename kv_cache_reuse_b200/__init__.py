@@ -20,6 +20,7 @@ __all__ = [
     "MacConfig", "MacError", "MacState", "mac_init_state", "mac_destroy", "mac_reset_seq", "mac_decode_step",
     "mac_match", "mac_attend", "mac_append_kv", "mac_decode_step_host", "mac_get_status", "mac_state_bytes",
     "mac_export_state", "mac_import_state", "mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_set_whole_unit_keys", "mac_warm_start", "mac_attend_grid", "mac_error_string", "mac_dense_decode_static",
+    "mac_selftest_wait_timeout",
     "MAC_OK", "MAC_ERR_ARG", "MAC_ERR_SHAPE", "MAC_ERR_CUDA", "MAC_ERR_OOM", "MAC_ERR_DEVICE",
     "MAC_DEV_BAD_SEQ_LEN", "MAC_DEV_BAD_PAGE", "MAC_DEV_TIMEOUT", "LIB_PATH",
 ]
@@ -222,6 +223,12 @@ def mac_dense_decode_static(q_pre, rope_pos, K, V, block_table, seq_lens, out, l
         _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
         _ptr(device_status), int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim), float(rope_theta),
         int(page_size), int(max_seq), int(max_pages_per_seq), int(num_pages), _stream(stream)))
+
+
+def mac_selftest_wait_timeout(device_status, stream=None) -> None:
+    """Enqueue the failure-path self-test: a kernel whose bounded wait runs out
+    (about 2 s) and ORs MAC_DEV_TIMEOUT into device_status."""
+    check("mac_selftest_wait_timeout", load().mac_selftest_wait_timeout(_ptr(device_status), _stream(stream)))
 
 
 def mac_error_string(code: int) -> str:

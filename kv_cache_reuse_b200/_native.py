@@ -31,6 +31,7 @@ SIGNATURES = {
     "mac_warm_start": (C.c_int, [_P, C.c_int, _P, _P, _P, _P, _P, _P, _P]),
     "mac_attend_grid": (C.c_int, [_P]),
     "mac_error_string": (C.c_char_p, [C.c_int]),
+    "mac_selftest_wait_timeout": (C.c_int, [_P, _P]),
     "mac_dense_decode_static": (C.c_int, [_P] * 9 + [C.c_int] * 4 + [C.c_double] + [C.c_int] * 4 + [_P]),
 }
 

@@ -602,6 +602,11 @@ int mac_decode_step_host(MacState* s, const void* q_pre_h, const int* rope_pos_h
   return status ? MAC_ERR_DEVICE : MAC_OK;
 }
 
+int mac_selftest_wait_timeout(unsigned* device_status, void* stream) {
+  if (!device_status) return MAC_ERR_ARG;
+  return launch_wait_selftest(device_status, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+}
+
 int mac_get_status(MacState* s, int* device_status) {
   if (!s) return MAC_ERR_ARG;
   unsigned v = 0;

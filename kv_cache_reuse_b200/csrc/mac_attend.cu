@@ -1120,7 +1120,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   }
 }
 
+// Failure-path self-test: one warp waits, through the kernels' bounded wait,
+// on an mbarrier that nothing arrives on.  After the limit the wait sets
+// MAC_DEV_TIMEOUT in the status word and the kernel returns.
+__global__ void mac_wait_selftest_kernel(unsigned* status) {
+  __shared__ unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, &abort_flag, status);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(unsigned* status, cudaStream_t s) {
+  mac_wait_selftest_kernel<<<1, 32, 0, s>>>(status);
+  return cudaGetLastError();
+}
 
 size_t attend_smem_bytes(int D, int G) {
   const bool g4 = group_pad(G) == 4;

@@ -165,6 +165,7 @@ cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s);
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t attend_prepare(int D, int G);
+cudaError_t launch_wait_selftest(unsigned* status, cudaStream_t s);
 size_t attend_smem_bytes(int D, int G);
 
 }  // namespace mac

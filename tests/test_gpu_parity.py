@@ -518,6 +518,25 @@ def test_work_split_settings_keep_parity(tune):
     compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tune=tune)
 
 
+def test_bounded_wait_times_out_and_context_stays_usable():
+    """A wait that nothing satisfies gives up after its limit: the status word
+    says MAC_DEV_TIMEOUT, the launch ends on its own, and the next steps on the
+    same context match the oracle."""
+    import time
+    import kv_cache_reuse_b200 as mac
+    torch, dev = torch_dev()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    t0 = time.time()
+    mac.mac_selftest_wait_timeout(status)
+    torch.cuda.synchronize()
+    dt = time.time() - t0
+    assert int(status.item()) == mac.MAC_DEV_TIMEOUT
+    assert 1.5 < dt < 30.0
+    wl = synth.WORKLOADS["tiny"].with_(steps=8)
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl))
+    assert r["hits"] > 0
+
+
 def test_nan_query_misses_and_stays_local():
     wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, L0=(700, 900), steps=6)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
