@@ -158,6 +158,8 @@ def rank_workload(args, rank):
         base = base.with_(B=args.batch, L0=base.L0[:1] * args.batch)
     if args.tau is not None:
         base = base.with_(tau=args.tau)
+    if args.q_heads or args.kv_heads:
+        base = base.with_(Hq=args.q_heads or base.Hq, Hkv=args.kv_heads or base.Hkv)
     return base, base.with_(seed=base.seed + 1000 * rank)
 
 
@@ -590,6 +592,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling of smaller cases)")
     ap.add_argument("--tau", type=float, default=None, help="override the match threshold (0 = every step misses)")
+    ap.add_argument("--q-heads", type=int, default=0, help="override the query heads (other group sizes)")
+    ap.add_argument("--kv-heads", type=int, default=0, help="override the KV heads (other group sizes)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
