@@ -240,7 +240,8 @@ def test_host_entry_append_recapture():
     assert a.st.get_status() == 0 and b.st.get_status() == 0
 
 
-@pytest.mark.parametrize("case", ["one_key", "band0", "window1", "ragged", "full_capacity", "band_covers", "d128_short"])
+@pytest.mark.parametrize("case", ["one_key", "band0", "window1", "ragged", "full_capacity", "band_covers", "d128_short",
+                                  "window_max", "many_units", "page64"])
 def test_edge_cases(case):
     base = synth.WORKLOADS["tiny"]
     kw = {}
@@ -259,6 +260,13 @@ def test_edge_cases(case):
     elif case == "d128_short":
         base = synth.WORKLOADS["llama8b_32k"]
         kw = dict(L0=(37,), steps=40, W=8)
+    elif case == "window_max":  # the largest window: the match kernel scans its slots in several batches
+        kw = dict(L0=(60,), steps=280, W=256, band=16)
+    elif case == "many_units":  # 160 units: 320 work items, more than one pass of the plan build
+        kw = dict(B=40, Hq=16, Hkv=4, L0=tuple(200 + 37 * i for i in range(40)), steps=6)
+    elif case == "page64":  # 64-key pages: several boxes per page, block table over a shuffled pool
+        base = synth.WORKLOADS["paged_mixed"]
+        kw = dict(B=3, L0=(3000, 700, 2100), steps=12, page_size=64)
     wl = base.with_(**kw)
     stream = synth.queries(wl)
     cache = synth.kv_cache(wl)  # capacity = L0 + steps exactly: the last step fills it
