@@ -179,15 +179,19 @@ __device__ void build_segments(const MatchParams& p, int U, double cw_c) {
   }
   if (p.claim != nullptr)
     for (int c = tid; c < p.grid; c += kMatchThreads) p.claim[c] = 0;
-  // CTA holding offset x: the largest c with start(c) <= x (weighted: from
-  // the even split's guess, walked to the exact range; the weights are near 1)
+  // CTA holding offset x: the largest c with start(c) <= x (weighted: a
+  // binary search of the range starts, at most 8 steps for 148 ranges)
   auto owner = [&](long long x) -> int {
     if (!weighted) return cta_of(x, T, N, rT);
-    int c = (int)((double)x * N * rT);
-    c = c < 0 ? 0 : (c > N - 1 ? N - 1 : c);
-    while (c > 0 && sbound[c] > x) --c;
-    while (c < N - 1 && sbound[c + 1] <= x) ++c;
-    return c;
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sbound[mid] <= x)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    return lo;
   };
   // first CTA whose range starts at or after x
   auto first_from = [&](long long x) -> long long {
