@@ -158,8 +158,9 @@ def rank_workload(args, rank):
         base = base.with_(B=args.batch, L0=base.L0[:1] * args.batch)
     if args.tau is not None:
         base = base.with_(tau=args.tau)
-    if args.q_heads or args.kv_heads:
-        base = base.with_(Hq=args.q_heads or base.Hq, Hkv=args.kv_heads or base.Hkv)
+    hq, hkv = getattr(args, "q_heads", 0), getattr(args, "kv_heads", 0)
+    if hq or hkv:
+        base = base.with_(Hq=hq or base.Hq, Hkv=hkv or base.Hkv)
     return base, base.with_(seed=base.seed + 1000 * rank)
 
 
