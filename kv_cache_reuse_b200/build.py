@@ -7,6 +7,7 @@ from __future__ import annotations
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
@@ -32,19 +33,23 @@ def _stale(target: str, deps) -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu for sm_100a and link the shared library; returns its path."""
+    """Compile every .cu for sm_100a (the files in parallel) and link the shared
+    library; returns its path."""
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     nvcc = _nvcc()
     for src in SOURCES:
         s = os.path.join(CSRC, src)
         o = os.path.join(BUILD, src.replace(".cu", ".o"))
         objs.append(o)
         if force or _stale(o, [s] + HEADERS):
-            cmd = [nvcc] + ARCH + FLAGS + ["-c", s, "-o", o]
-            if verbose:
-                print(" ".join(cmd))
-            subprocess.check_call(cmd)
+            cmds.append([nvcc] + ARCH + FLAGS + ["-c", s, "-o", o])
+    for cmd in cmds:
+        if verbose:
+            print(" ".join(cmd))
+    with ThreadPoolExecutor(max_workers=max(1, len(cmds))) as ex:
+        for f in [ex.submit(subprocess.check_call, cmd) for cmd in cmds]:
+            f.result()
     if force or _stale(LIB, objs):
         tmp = LIB + ".tmp%d" % os.getpid()
         cmd = [nvcc] + ARCH + ["-shared", "-o", tmp] + objs
