@@ -7,12 +7,18 @@
 // attention computed on the KV tail through a numerically stable merge"; on
 // a miss the step is split-KV decode attention over every key.  All three are
 // the same computation -- attention of the current query group over a key
-// range -- so one persistent kernel runs them over a flattened list of key
-// segments built by the match kernel:
-//   segment 2u   = [start, c_t)  -> folded into the unit's new prefix state
-//   segment 2u+1 = [c_t, p_t]    -> folded into the output only
-// The flattened keys are split evenly over the CTAs, so a mix of hits (a few
-// hundred keys) and misses (the whole context) keeps every SM equally busy.
+// range -- so one persistent kernel runs them over a flattened list of work
+// items built by the match kernel.  A unit (sequence, KV head) with few fresh
+// keys (every hit) is one whole item, done end to end by one CTA; a longer
+// one is two split items,
+//   [start, c_t)  -> folded into the unit's new prefix state
+//   [c_t, p_t]    -> folded into the output only,
+// cut wherever the CTAs' ranges cut them.  The items are laid end to end in a
+// cost space (keys plus a fixed cost per item) split over the CTAs evenly, or
+// on large steps in proportion to each SM's learned streaming rate, so a mix
+// of hits (a few hundred keys) and misses (the whole context) keeps every SM
+// equally busy.  With per-head matching each head masks the keys of the
+// amend range below its own reuse boundary.
 //
 // Per CTA: eight warps; warp w owns boxes w, w+8, w+16, ... of every piece,
 // where a box is 16 keys (it never crosses a page).  Each warp streams its
@@ -39,10 +45,11 @@
 // per head of shared memory per warp.
 //
 // Softmax runs in exp2 units (the query is pre-scaled by log2(e)/sqrt(D)).
-// Every piece a CTA processes ends in a partial (o unnormalised, m, l).  The
-// CTA that delivers a unit's last partial (atomic counter, no waiting) merges
-// the reused ring state, the band and the tail partials, writes the new ring
-// entry, out and lse.
+// A whole item ends in the CTA: reused ring state (+) amend -> new ring
+// entry, (+) tail -> out, lse.  A split piece ends in a partial (o
+// unnormalised, m, l); the CTA that delivers a unit's last partial (atomic
+// counter, no waiting) merges the reused state and the partials the same
+// way.  The window's stored outputs are fp32 or bf16.
 //
 // Every wait is bounded (2 s on %globaltimer): on expiry the kernel sets
 // MAC_DEV_TIMEOUT in the status word and leaves without hanging the GPU.

@@ -10,7 +10,9 @@
 //      fp32 as sum((a - b)^2) -- the expanded |a|^2 + |b|^2 - 2ab form would
 //      cancel catastrophically for near-repeats;
 //   2. argmin with ties to the more recent entry, hit iff the minimum is
-//      strictly below tau; NaN distances never win;
+//      strictly below tau; NaN distances never win (with per-head matching,
+//      steps 1-3 run per query head: its own distance, entry and c_s, the
+//      unit's fresh range starting at the smallest c_s);
 //   3. key ranges: the reused prefix ends at c_s = max(0, p_s - band) (the
 //      amend band starts there), the stored prefix of this step ends at
 //      c_t = max(0, p_t - band), and the tail runs to p_t (band here is the
@@ -19,13 +21,15 @@
 //   4. RoPE of the query to rope_pos (fp64 angle), pre-scaled by
 //      log2(e)/sqrt(D) so the attention kernel works in exp2 units;
 //   5. the query enters the ring slot n mod (W+1) (W+1 slots: the slot
-//      written is never one the window can read this step).
-// The last CTA to finish lays every unit's two key segments end to end in a
-// cost space (each non-empty segment weighs its keys plus a fixed per-piece
-// cost) and splits that space evenly over the attention kernel's CTAs, so a
-// batch mixing short hit ranges with whole-context misses is balanced by
-// time rather than by keys.  No CTA waits for another: the last arrival
-// does the work.
+//      written is never one the window can read this step), in fp32 or
+//      rounded to bf16.
+// The last CTA to finish lays every unit's work items (one whole item, or
+// two split key segments) end to end in a cost space (each non-empty item
+// weighs its keys plus a fixed per-piece cost) and splits that space over
+// the attention kernel's CTAs -- evenly, or on large steps in proportion to
+// each SM's learned streaming rate -- so a batch mixing short hit ranges
+// with whole-context misses is balanced by time rather than by keys.  No CTA
+// waits for another: the last arrival does the work.
 #include <math.h>
 #include <stdint.h>
 
