@@ -204,10 +204,13 @@ def run_mac(args, rank, world, local_rank):
     sptr = s.cuda_stream
     hsz = (B, Hkv)
 
-    qsrc = [q_all]  # the query stream the timed steps read (the hit-path run swaps it)
+    # the stream the timed steps read (the bf16, per-head, hit-path and context runs swap it)
+    cur = {"q": q_all, "pos": pos_all, "lens": lens_all, "stream": stream}
+    qsrc = [q_all]
 
     def ptrs(t):
-        return (qsrc[0][t].data_ptr(), pos_all[t].data_ptr(), lens_all[t].data_ptr(), hit_all[t].data_ptr(),
+        q = qsrc[0] if cur["q"] is q_all else cur["q"]
+        return (q[t].data_ptr(), cur["pos"][t].data_ptr(), cur["lens"][t].data_ptr(), hit_all[t].data_ptr(),
                 mpos_all[t].data_ptr())
 
     def timed_run(tau, nwarm, nsteps, split, cfg=None, bytes_stream=None):
@@ -266,11 +269,11 @@ def run_mac(args, rank, world, local_rank):
         for i in range(nsteps):
             t = nwarm + i
             occ = min(t, wl.W)
-            a, b_, c = step_bytes(wl, hits[i], mpos[i], stream.seq_lens[t], occ, qes, res_)
+            a, b_, c = step_bytes(wl, hits[i], mpos[i], cur["stream"].seq_lens[t], occ, qes, res_)
             mt_b += a
             at_b += b_
             kv_b += c
-            dense_b += synth.dense_equiv_kv_bytes(wl, stream.seq_lens[t])
+            dense_b += synth.dense_equiv_kv_bytes(wl, cur["stream"].seq_lens[t])
         tot_ms = float(np.sum(step_ms))
         return dict(total_ms=tot_ms, step_ms=step_ms, att_ms=float(np.sum(att_ms)), match_ms=float(np.sum(match_ms)),
                     att_bytes=at_b, match_bytes=mt_b, kv_bytes=kv_b, dense_bytes=dense_b,
@@ -318,12 +321,24 @@ def run_mac(args, rank, world, local_rank):
                    timed_run(wl.tau, args.warmup, args.steps, split=True, cfg=cfg))
         qsrc[0] = q_all
     hitrun = None
+    hitctx = []
     if args.hit_steps > 0:
         # the hit path alone: the same shape with every labelled step a near-repeat
         qh = synth.queries(wl.with_(hit_model=("iid", 1.0)), T).q
         qsrc[0] = torch.from_numpy(qh).to(dev)
         hitrun = timed_run(wl.tau, 3, min(args.hit_steps, T - 3), split=True)
         qsrc[0] = q_all
+        if not cache.paged:
+            # the same hit stream at shorter contexts, on the same cache: a hit's
+            # cost should not depend on the context length
+            for L in (8192, 32768):
+                sc = synth.queries(wl.with_(hit_model=("iid", 1.0), L0=(L,) * B), T)
+                cur.update(q=torch.from_numpy(sc.q).to(dev), pos=torch.from_numpy(sc.rope_pos).to(dev),
+                           lens=torch.from_numpy(sc.seq_lens).to(dev), stream=sc)
+                r = timed_run(wl.tau, 3, min(args.hit_steps, T - 3), split=True)
+                hitctx.append((L, r))
+            cur.update(q=q_all, pos=pos_all, lens=lens_all, stream=stream)
+            hitctx.append((int(wl.L0[0]), hitrun))
 
     # max over ranks of the timed duration
     tot = max_over_ranks(main["total_ms"], world, dev)
@@ -383,6 +398,11 @@ def run_mac(args, rank, world, local_rank):
                            "attend_bytes_per_step": hitrun["att_bytes"] / n, "attend_gbs": h_gbs,
                            "attend_frac": h_gbs / peak, "clocks": hitrun["clocks"],
                            "note": "latency-bound: a few MB per launch"}
+        if hitctx:
+            res["hit_path"]["vs_context"] = [
+                {"context": L, "steps_per_s": len(r["step_ms"]) / (r["total_ms"] * 1e-3),
+                 "ms_per_step": r["total_ms"] / len(r["step_ms"]), "hit_fraction": r["hit_frac"],
+                 "attend_bytes_per_step": r["att_bytes"] / len(r["step_ms"])} for L, r in hitctx]
     for name, pair, what in (("bf16_window", bf16, {"q": "bf16", "window_q_and_o": "bf16"}),
                              ("per_head", perhead, {"matching": "per query head",
                                                     "stream": "each query head repeats a recent query of its own "
