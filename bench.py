@@ -340,6 +340,14 @@ def run_mac(args, rank, world, local_rank):
             cur.update(q=q_all, pos=pos_all, lens=lens_all, stream=stream)
             hitctx.append((int(wl.L0[0]), hitrun))
 
+    quality = None
+    if not args.no_quality:
+        quality = run_quality(args, wl, stream, K, V, bt, kw, dev)
+        quality["identity_rope"] = run_quality(args, wl, stream, K, V, bt, kw, dev, identity_rope=True)
+        quality["note"] = ("a hit reuses prefix attention computed with the matched query rotated to its own "
+                           "position; on structure-free random queries and keys every RoPE frequency weighs the "
+                           "same, so the position shift alone decorrelates the reused scores (compare identity_rope)")
+
     # max over ranks of the timed duration
     tot = max_over_ranks(main["total_ms"], world, dev)
 
@@ -419,6 +427,8 @@ def run_mac(args, rank, world, local_rank):
             "attend_bytes_per_step": kr["att_bytes"] / K_, "attend_gbs": a_gbs, "attend_frac": a_gbs / peak,
             "match_gbs": kr["match_bytes"] / (kr["match_ms"] * 1e-3) / 1e9,
             "clocks": run["clocks"], "device_status": run["status"]})
+    if quality:
+        res["approximation_vs_dense"] = quality
     if warm:
         res["warm_start"] = warm
     if layers:
@@ -428,6 +438,50 @@ def run_mac(args, rank, world, local_rank):
     if cpu:
         res["cpu_baseline"] = cpu
     return res
+
+
+def run_quality(args, wl, stream, K, V, bt, kw, dev, identity_rope=False):
+    """Approximation error of MAC against dense attention on the same stream
+    (untimed): one state with the workload's threshold, one with threshold 0
+    (every step a miss: dense attention), step by step; per query head the
+    relative L2 error of out and the lse difference.  identity_rope rotates
+    every query by angle 0 (position 0), which isolates the error of reusing
+    a state computed with a query rotated to another position."""
+    import torch
+    import kv_cache_reuse_b200 as mac
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    T = min(args.warmup + args.steps, stream.q.shape[0])
+    sm_, sd = mac.MacState.for_workload(wl, **kw), mac.MacState.for_workload(wl, tau=0.0, **kw)
+    q = torch.from_numpy(stream.q[:T]).to(dev)
+    pos = torch.from_numpy(np.zeros_like(stream.rope_pos[:T]) if identity_rope else stream.rope_pos[:T]).to(dev)
+    lens = torch.from_numpy(stream.seq_lens[:T]).to(dev)
+    om, od = torch.empty((B, Hq, D), device=dev), torch.empty((B, Hq, D), device=dev)
+    lm, ld = torch.empty((B, Hq), device=dev), torch.empty((B, Hq), device=dev)
+    hit = torch.empty((B, Hkv), dtype=torch.uint8, device=dev)
+    rel_all, rel_hit, dl_hit = [], [], []
+    for t in range(T):
+        mac.mac_decode_step(sm_, q[t], pos[t], K, V, bt, lens[t], om, lm, hit, None)
+        mac.mac_decode_step(sd, q[t], pos[t], K, V, bt, lens[t], od, ld, None, None)
+        if t < args.warmup:
+            continue
+        rel = (torch.linalg.vector_norm(om - od, dim=-1) / torch.linalg.vector_norm(od, dim=-1)).cpu().numpy()
+        dl = (lm - ld).abs().cpu().numpy()
+        hh = np.repeat(hit.cpu().numpy().astype(bool), Hq // Hkv, axis=1)  # [B][Hq]
+        rel_all.append(rel.ravel())
+        rel_hit.append(rel[hh])
+        dl_hit.append(dl[hh])
+    torch.cuda.synchronize(dev)
+    status = (sm_.get_status(), sd.get_status())
+    sm_.close()
+    sd.close()
+    ra, rh, dh = np.concatenate(rel_all), np.concatenate(rel_hit), np.concatenate(dl_hit)
+    return {"steps": T - args.warmup, "heads_on_hits": int(rh.size),
+            "rel_l2_out_mean": float(ra.mean()), "rel_l2_out_on_hits_mean": float(rh.mean()) if rh.size else None,
+            "rel_l2_out_on_hits_p99": float(np.percentile(rh, 99)) if rh.size else None,
+            "rel_l2_out_on_hits_max": float(rh.max()) if rh.size else None,
+            "lse_abs_diff_on_hits_max": float(dh.max()) if dh.size else None,
+            "reference": "the same kernels with threshold 0 (dense attention, parity-tested against the fp64 oracle)",
+            "device_status": status}
 
 
 def run_layers(args, wl, stream, cache, K, V, bt, kw, dev, peak):
@@ -608,6 +662,7 @@ def main():
                     help="also time a stack of this many layers per token, one CUDA graph per token")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 query / window run")
     ap.add_argument("--no-per-head", action="store_true", help="skip the per-head matching run")
+    ap.add_argument("--no-quality", action="store_true", help="skip the approximation-error pass")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
