@@ -206,11 +206,9 @@ def run_mac(args, rank, world, local_rank):
 
     # the stream the timed steps read (the bf16, per-head, hit-path and context runs swap it)
     cur = {"q": q_all, "pos": pos_all, "lens": lens_all, "stream": stream}
-    qsrc = [q_all]
 
     def ptrs(t):
-        q = qsrc[0] if cur["q"] is q_all else cur["q"]
-        return (q[t].data_ptr(), cur["pos"][t].data_ptr(), cur["lens"][t].data_ptr(), hit_all[t].data_ptr(),
+        return (cur["q"][t].data_ptr(), cur["pos"][t].data_ptr(), cur["lens"][t].data_ptr(), hit_all[t].data_ptr(),
                 mpos_all[t].data_ptr())
 
     def timed_run(tau, nwarm, nsteps, split, cfg=None, bytes_stream=None):
@@ -306,28 +304,28 @@ def run_mac(args, rank, world, local_rank):
     bf16 = None
     if not args.no_bf16:
         # bf16 queries and bf16 window: the same stream with its queries rounded to bf16
-        qsrc[0] = torch.from_numpy(synth.f32_to_bf16_bits(stream.q).view(np.int16)).to(dev)
+        cur["q"] = torch.from_numpy(synth.f32_to_bf16_bits(stream.q).view(np.int16)).to(dev)
         cfg = {"q_bf16": 1, "ring_bf16": 1}
         bf16 = (timed_run(wl.tau, args.warmup, args.steps, split=False, cfg=cfg),
                 timed_run(wl.tau, args.warmup, args.steps, split=True, cfg=cfg))
-        qsrc[0] = q_all
+        cur["q"] = q_all
     perhead = None
     if not args.no_per_head:
         # per-head matching on a stream whose query heads repeat on their own
         wh = wl.with_(head_labels=True)
-        qsrc[0] = torch.from_numpy(synth.queries(wh, T).q).to(dev)
+        cur["q"] = torch.from_numpy(synth.queries(wh, T).q).to(dev)
         cfg = {"match_per_head": 1}
         perhead = (timed_run(wl.tau, args.warmup, args.steps, split=False, cfg=cfg),
                    timed_run(wl.tau, args.warmup, args.steps, split=True, cfg=cfg))
-        qsrc[0] = q_all
+        cur["q"] = q_all
     hitrun = None
     hitctx = []
     if args.hit_steps > 0:
         # the hit path alone: the same shape with every labelled step a near-repeat
         qh = synth.queries(wl.with_(hit_model=("iid", 1.0)), T).q
-        qsrc[0] = torch.from_numpy(qh).to(dev)
+        cur["q"] = torch.from_numpy(qh).to(dev)
         hitrun = timed_run(wl.tau, 3, min(args.hit_steps, T - 3), split=True)
-        qsrc[0] = q_all
+        cur["q"] = q_all
         if not cache.paged:
             # the same hit stream at shorter contexts, on the same cache: a hit's
             # cost should not depend on the context length
