@@ -352,6 +352,33 @@ def test_per_head_matching(case):
     assert 0 < hits < wl.steps * wl.B * wl.Hq
 
 
+def test_bf16_host_entry_matches_device_entry():
+    """The host entry with bf16 queries (its input block carries 2 bytes per
+    query element) and a bf16 window, against the device entry, bit for bit."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(steps=20)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    a = GpuRun(wl, cache, q_bf16=1, ring_bf16=1)
+    b = GpuRun(wl, cache, q_bf16=1, ring_bf16=1)
+    torch = a.torch
+    out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32).pin_memory()
+    lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+    hit_h = torch.empty((wl.B, wl.Hkv), dtype=torch.uint8).pin_memory()
+    mp_h = torch.empty((wl.B, wl.Hkv), dtype=torch.int32).pin_memory()
+    hits = 0
+    for t in range(wl.steps):
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        q_h = torch.from_numpy(synth.f32_to_bf16_bits(stream.q[t]).view(np.int16)).pin_memory()
+        p_h = torch.from_numpy(stream.rope_pos[t]).pin_memory()
+        l_h = torch.from_numpy(stream.seq_lens[t]).pin_memory()
+        rc = mac.mac_decode_step_host(b.st, q_h, p_h, l_h, None, None, b.K, b.V, None, out_h, lse_h, hit_h, mp_h)
+        assert rc == mac.MAC_OK
+        for u, v in zip(x, (out_h.numpy(), lse_h.numpy(), hit_h.numpy(), mp_h.numpy())):
+            np.testing.assert_array_equal(u, v)
+        hits += int(x[2].sum())
+    assert hits > 0
+
+
 def test_per_head_host_entry_matches_device_entry():
     """The host entry returns [B][Hq] decisions with per-head matching."""
     import kv_cache_reuse_b200 as mac
@@ -440,21 +467,29 @@ def test_cut_mode_band_ends_at_position(case):
     assert r["hits"] > 0
 
 
-@pytest.mark.parametrize("case", ["tiny", "paged"])
+@pytest.mark.parametrize("case", ["tiny", "paged", "per_head_bf16"])
 def test_warm_start_from_prefill_then_decode(case):
     """Windows seeded from the first n positions of the stream (as prefill
     positions), then decoding: decisions bit-exact and outputs within tolerance
     of the oracle doing the same, and the seeded ring equal to its window."""
     import kv_cache_reuse_b200 as mac
+    ph = qb = rb = 0
     if case == "tiny":
         wl, n = synth.WORKLOADS["tiny"].with_(steps=40), 16
-    else:
+    elif case == "paged":
         wl, n = synth.WORKLOADS["paged_mixed"].with_(B=3, L0=(3000, 900, 5000), steps=20), 8
+    else:  # per-head matching, bf16 queries and bf16 window
+        wl, n = synth.WORKLOADS["tiny"].with_(steps=40, head_labels=True), 16
+        ph = qb = rb = 1
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    gpu = GpuRun(wl, cache)
-    orc = oracle.Oracle.for_workload(wl, cache)
+    if qb:  # the queries as bf16 values: the library reads their bits, the oracle their values
+        stream = synth.QueryStream(q=synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(stream.q)), label=stream.label,
+                                   src=stream.src, rope_pos=stream.rope_pos, seq_lens=stream.seq_lens)
+    gpu = GpuRun(wl, cache, per_head=ph, q_bf16=qb, ring_bf16=rb)
+    orc = oracle.Oracle.for_workload(wl, cache, per_head=ph, ring_bf16=rb)
     torch = gpu.torch
-    qn = torch.from_numpy(np.ascontiguousarray(stream.q[:n])).to(gpu.dev)
+    qh = synth.f32_to_bf16_bits(stream.q[:n]).view(np.int16) if qb else np.ascontiguousarray(stream.q[:n])
+    qn = torch.from_numpy(np.ascontiguousarray(qh)).to(gpu.dev)
     pn = torch.from_numpy(np.ascontiguousarray(stream.rope_pos[:n])).to(gpu.dev)
     ln = torch.from_numpy(np.ascontiguousarray(stream.seq_lens[:n])).to(gpu.dev)
     mac.mac_warm_start(gpu.st, n, qn, pn, gpu.K, gpu.V, gpu.bt, ln)
@@ -468,24 +503,30 @@ def test_warm_start_from_prefill_then_decode(case):
         for j in range(n):
             slot = j % W1
             assert st["pos"][u, slot] == pos_o[j]
-            np.testing.assert_array_equal(st["q"][u, slot], q_o[j])
-            np.testing.assert_allclose(st["o"][u, slot], o_o[j], atol=OUT_TOL)
-    r = compare_stream(wl, stream, cache, gpu=gpu, orc=orc, start=n)
+            if rb:  # the window holds bf16 bits
+                np.testing.assert_array_equal(st["q"][u, slot], synth.f32_to_bf16_bits(q_o[j]))
+                np.testing.assert_allclose(synth.bf16_bits_to_f32(st["o"][u, slot]), o_o[j], atol=OUT_TOL)
+            else:
+                np.testing.assert_array_equal(st["q"][u, slot], q_o[j])
+                np.testing.assert_allclose(st["o"][u, slot], o_o[j], atol=OUT_TOL)
+    r = compare_stream(wl, stream, cache, gpu=gpu, orc=orc, start=n, q_bf16=qb)
     assert r["hits"] > 0
 
 
-def test_graph_captured_multilayer_loop():
+@pytest.mark.parametrize("opts", [{}, {"per_head": 1, "ring_bf16": 1}])
+def test_graph_captured_multilayer_loop(opts):
     """Several layers' steps recorded once as one CUDA graph and replayed for
     every token (inputs copied into fixed buffers before each replay) give
-    the same bits as the same steps run eagerly."""
+    the same bits as the same steps run eagerly (also with per-head matching
+    and a bf16 window)."""
     import kv_cache_reuse_b200 as mac
     torch, dev = torch_dev()
     L = 3
-    wls = [synth.WORKLOADS["tiny"].with_(steps=24, seed=10 + l) for l in range(L)]
+    wls = [synth.WORKLOADS["tiny"].with_(steps=24, seed=10 + l, head_labels=bool(opts)) for l in range(L)]
     streams = [synth.queries(w) for w in wls]
     caches = [synth.kv_cache(w) for w in wls]
-    eager = [GpuRun(w, c) for w, c in zip(wls, caches)]
-    graph = [GpuRun(w, c) for w, c in zip(wls, caches)]
+    eager = [GpuRun(w, c, **opts) for w, c in zip(wls, caches)]
+    graph = [GpuRun(w, c, **opts) for w, c in zip(wls, caches)]
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()

@@ -36,11 +36,12 @@ def test_rejects_shapes_beyond_the_static_scratch():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("paged", [False, True])
-def test_static_scratch_matches_regular_entry_on_two_calls(paged):
+@pytest.mark.parametrize("paged,Hq", [(False, 32), (True, 32), (False, 8), (True, 64)])
+def test_static_scratch_matches_regular_entry_on_two_calls(paged, Hq):
+    """Groups of 4, 1 (8 query heads over 8 KV heads) and 8 (64 over 8)."""
     import kv_cache_reuse_b200 as mac
     base = synth.WORKLOADS["paged_mixed" if paged else "llama8b_32k"]
-    wl = base.with_(B=3, L0=(5000, 3210, 777), steps=2)
+    wl = base.with_(B=3, L0=(5000, 3210, 777), steps=2, Hq=Hq)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
     ref = GpuRun(wl, cache, tau=0.0)  # regular entry point, never hits: dense attention
     torch = ref.torch
