@@ -436,18 +436,17 @@ __device__ __forceinline__ void fold_state(float& M, float& L, float (&O)[N], fl
 // Last arriver of a split unit: merge its partials.  Segment A's partials
 // (with the reused state on a hit) give the new prefix state over [0, c_t),
 // stored in the ring; that state and segment B's partials give the output.
-// Four heads at a time: the 8 warps share the partials (warp w folds
-// partials w, w + 8, ..., each lane FPL consecutive floats of one head), with
-// up to 16 partials' loads in flight at once; the warps' states then meet in
-// shared memory.
+// Every thread owns a slice of VEC consecutive elements of one head (four
+// heads at a time) and folds all of the unit's partials for its slice, BC
+// partials' loads in flight per round: no exchange between warps, no barrier.
 template <int D, int GP, int GF, bool PH>
 __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
-  constexpr int QD = 4 * D;                    // floats of four heads
-  constexpr int FPL = QD / 32, F4 = FPL / 4;   // floats and float4 of those per lane
-  constexpr int BP = 2;                        // partials per warp per round of loads (the code runs cold
-                                               // once per step: a short loop beats more loads in flight)
-  constexpr int VEC = QD / (kConsumerWarps * 32);
-  static_assert(VEC * kConsumerWarps * 32 == QD && F4 * 4 * 32 == QD, "merge layout");
+  constexpr int QD = 4 * D;                         // elements of four heads
+  constexpr int VEC = QD / (kConsumerWarps * 32);  // elements per thread: 2 (D = 128) or 1 (D = 64)
+  constexpr int BC = 4;  // partials per round of loads (cold code: 4 measured best of 2, 4, 8, 16, 24)
+  static_assert(VEC * kConsumerWarps * 32 == QD && (VEC == 1 || VEC == 2), "merge layout");
+  (void)sm;
+  (void)sync_phase;
   const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
   const UnitPlan* const pp = p.plan + u;
   const HeadPlan* const hp = p.hplan + u;
@@ -457,106 +456,69 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
   const int nA = sA.npieces, n = nA + sB.npieces;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t ds = (size_t)u * Wp1 + dst_slot;
-  float* wb = sm.wbuf[warp];
+  const int e0 = threadIdx.x * VEC;  // this thread's first element in a quad [4][D]
+  const int hq = e0 / D, d0 = e0 - hq * D;
 
   for (int h0 = 0; h0 < G; h0 += 4) {
-    const int f0 = lane * FPL, hq = f0 / D, hl = h0 + hq;  // this lane's head
-    const bool live = hl < G;
-    const int fo = h0 * D + f0;                         // its first float in a partial's o
-    float MA = -INFINITY, LA = 0.f, OA[FPL], MB = -INFINITY, LB = 0.f, OB[FPL];
+    const int h = h0 + hq;
+    if (h >= G) break;  // no barriers below: a thread past the group leaves
+    const size_t oo = (size_t)h * D + d0;  // the slice's offset in an o [G][D]
+    float MA = -INFINITY, LA = 0.f, OA[VEC], MB = -INFINITY, LB = 0.f, OB[VEC];
 #pragma unroll
-    for (int j = 0; j < FPL; ++j) OA[j] = OB[j] = 0.f;
-    const bool reuse = PH ? live && ((hmask >> hl) & 1) : hit && live;
-    if (warp == 0 && reuse) {  // the reused state joins set A (its o is normalised)
-      const size_t rs = (size_t)u * Wp1 + (PH ? hp->hsrc[hl] : src_slot);
-      const float rl = __ldcg(p.ring_l + rs * G + hl), rm = __ldcg(p.ring_m + rs * G + hl) * kLog2e;
-      float o[FPL];
+    for (int j = 0; j < VEC; ++j) OA[j] = OB[j] = 0.f;
+    if (PH ? ((hmask >> h) & 1) : hit) {  // the reused state joins set A (its o is normalised)
+      const size_t rs = (size_t)u * Wp1 + (PH ? hp->hsrc[h] : src_slot);
+      const float rl = __ldcg(p.ring_l + rs * G + h), rm = __ldcg(p.ring_m + rs * G + h) * kLog2e;
+      float o[VEC];
 #pragma unroll
-      for (int f = 0; f < F4; ++f) {
-        float4 t;
-        if (p.ring_bf16) {
-          const uint2 w = __ldcg(reinterpret_cast<const uint2*>(ring_o_row(p.ring_o, rs * GD + fo, true)) + f);
-          t = make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
-                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
-        } else {
-          t = __ldcg(reinterpret_cast<const float4*>(ring_o_row(p.ring_o, rs * GD + fo, false)) + f);
-        }
-        o[4 * f] = t.x * rl;
-        o[4 * f + 1] = t.y * rl;
-        o[4 * f + 2] = t.z * rl;
-        o[4 * f + 3] = t.w * rl;
-      }
-      fold_state<FPL>(MA, LA, OA, rm, rl, o);
+      for (int j = 0; j < VEC; ++j) o[j] = ring_o_at(p.ring_o, rs * GD + oo + j, p.ring_bf16) * rl;
+      fold_state<VEC>(MA, LA, OA, rm, rl, o);
     }
-    for (int i0 = warp; i0 < n && live; i0 += kConsumerWarps * BP) {
-      float4 v[BP][F4];
-      float mv[BP], lv[BP];
+    for (int i0 = 0; i0 < n; i0 += BC) {
+      float ov[BC][VEC], mv[BC], lv[BC];
 #pragma unroll
-      for (int k = 0; k < BP; ++k) {
-        const int i = i0 + k * kConsumerWarps;
+      for (int k = 0; k < BC; ++k) {
+        const int i = i0 + k;
         if (i < n) {
-          const float* pp = p.part + (size_t)(i < nA ? sA.pbase + i : sB.pbase + (i - nA)) * PF;
-#pragma unroll
-          for (int f = 0; f < F4; ++f) v[k][f] = __ldcg(reinterpret_cast<const float4*>(pp + fo) + f);
-          mv[k] = __ldcg(pp + GD + hl);
-          lv[k] = __ldcg(pp + GD + G4 + hl);
+          const float* q = p.part + (size_t)(i < nA ? sA.pbase + i : sB.pbase + (i - nA)) * PF;
+          if constexpr (VEC == 2) {
+            const float2 t = __ldcg(reinterpret_cast<const float2*>(q + oo));
+            ov[k][0] = t.x;
+            ov[k][VEC - 1] = t.y;
+          } else {
+            ov[k][0] = __ldcg(q + oo);
+          }
+          mv[k] = __ldcg(q + GD + h);
+          lv[k] = __ldcg(q + GD + G4 + h);
         }
       }
 #pragma unroll
-      for (int k = 0; k < BP; ++k) {
-        const int i = i0 + k * kConsumerWarps;
+      for (int k = 0; k < BC; ++k) {
+        const int i = i0 + k;
         if (i < n) {
-          const float* o = reinterpret_cast<const float*>(v[k]);
           if (i < nA)
-            fold_state<FPL>(MA, LA, OA, mv[k], lv[k], o);
+            fold_state<VEC>(MA, LA, OA, mv[k], lv[k], ov[k]);
           else
-            fold_state<FPL>(MB, LB, OB, mv[k], lv[k], o);
+            fold_state<VEC>(MB, LB, OB, mv[k], lv[k], ov[k]);
         }
       }
     }
-    // the warps' sets meet in shared memory ([4][D], m [4], l [4]): set A
-    // (prefix), then set B (tail)
-    float PM[VEC], PL[VEC], PO[VEC], QM[VEC], QL[VEC], QO[VEC];
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll
-      for (int j = 0; j < FPL; ++j) wb[f0 + j] = pass == 0 ? OA[j] : OB[j];
-      if (f0 - hq * D == 0) {
-        wb[QD + hq] = pass == 0 ? MA : MB;
-        wb[QD + 4 + hq] = pass == 0 ? LA : LB;
-      }
-      if (!consumer_sync(sm, sync_phase, p.status)) return false;
-#pragma unroll
-      for (int j = 0; j < VEC; ++j) {
-        const int idx = threadIdx.x * VEC + j;
-        float m_, l_, o_, xm, xl, xo;
-        combine_warps2<D, GP, 4>(sm, kConsumerWarps, idx, idx / D, m_, l_, o_, xm, xl, xo);
-        if (pass == 0) {
-          PM[j] = m_, PL[j] = l_, PO[j] = o_;
-        } else {
-          QM[j] = m_, QL[j] = l_, QO[j] = o_;
-        }
-      }
-      if (!consumer_sync(sm, sync_phase, p.status)) return false;
-    }
+    // new prefix state = set A (normalised) into the ring; output = A (+) B
+    const float M2 = fmaxf(MA, MB);
+    const float M2u = M2 == -INFINITY ? 0.f : M2;
+    const float a0 = ex2(MA - M2u), a1 = ex2(MB - M2u);
+    const float L2 = LA * a0 + LB * a1;
+    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
 #pragma unroll
     for (int j = 0; j < VEC; ++j) {
-      const int idx = threadIdx.x * VEC + j, h = h0 + idx / D, d = idx - (idx / D) * D;
-      if (h >= G) continue;
-      ring_o_put(p.ring_o, ds * GD + (size_t)h * D + d, PL[j] > 0.f ? PO[j] / PL[j] : 0.f, p.ring_bf16);
-      const float M2 = fmaxf(PM[j], QM[j]);
-      const float M2u = M2 == -INFINITY ? 0.f : M2;
-      const float a0 = ex2(PM[j] - M2u), a1 = ex2(QM[j] - M2u);
-      const float L2 = PL[j] * a0 + QL[j] * a1;
-      const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
-      p.out[orow * D + d] = (PO[j] * a0 + QO[j] * a1) / L2;
-      if (d == 0) {
-        p.ring_m[ds * G + h] = PL[j] > 0.f ? PM[j] * kLn2 : -INFINITY;
-        p.ring_l[ds * G + h] = PL[j];
-        p.lse[orow] = (M2 + log2f(L2)) * kLn2;
-      }
+      ring_o_put(p.ring_o, ds * GD + oo + j, LA > 0.f ? OA[j] / LA : 0.f, p.ring_bf16);
+      p.out[orow * D + d0 + j] = (OA[j] * a0 + OB[j] * a1) / L2;
+    }
+    if (d0 == 0) {
+      p.ring_m[ds * G + h] = LA > 0.f ? MA * kLn2 : -INFINITY;
+      p.ring_l[ds * G + h] = LA;
+      p.lse[orow] = (M2 + log2f(L2)) * kLn2;
     }
   }
   if (threadIdx.x == 0) {
