@@ -541,7 +541,9 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
+  // no fence needed: every CTA's plan store precedes its ticket (a release),
+  // the last ticket's acquire makes them visible to thread 0, and the block
+  // barrier above orders this CTA's other threads after that acquire
   build_segments(p, (int)gridDim.x, cw_c);
   if (tid == 0) *p.done = 0;
 }
