@@ -596,19 +596,31 @@ def run_e2e(args, wl, stream, cache, K, V, bt, kw, dev, world):
 
 def run_cpu_baseline(wl, stream, cache, seconds):
     """The fp64 oracle on the host cores, on the first steps of the same stream
-    (bounded to about `seconds` of CPU work)."""
+    (bounded to about `seconds` of CPU work): steps/s overall and split by
+    step kind (every unit hit / some unit missed), and GB/s of bf16 K/V read."""
     import oracle
     orc = oracle.Oracle.for_workload(wl, cache)
     t0 = time.perf_counter()
     n = nh = 0
+    kv = 0
+    kind_s = {"all_hit": [0, 0.0], "with_miss": [0, 0.0]}
     while n < stream.q.shape[0]:
+        ts = time.perf_counter()
         r = orc.step(stream.q[n], stream.rope_pos[n], cache.K, cache.V, cache.block_table, stream.seq_lens[n])
+        te = time.perf_counter()
         nh += int(r.hit.sum())
+        kv += int(r.keys_read) * 2 * wl.D * 2  # K and V rows of every key a unit read
+        k = kind_s["all_hit" if r.hit.all() else "with_miss"]
+        k[0] += 1
+        k[1] += te - ts
         n += 1
-        if time.perf_counter() - t0 > seconds:
+        if te - t0 > seconds:
             break
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "kv_gbs": kv / dt / 1e9,
+            "steps_per_s_by_kind": {k: (v[0] / v[1] if v[1] > 0 else None) for k, v in kind_s.items()},
+            "steps_by_kind": {k: v[0] for k, v in kind_s.items()},
             "sample": "first %d decode steps of %s from an empty window (%d of %d unit decisions hit), %.1f s" % (
                 n, wl.name, nh, n * wl.B * wl.Hkv, dt)}
 
