@@ -379,6 +379,15 @@ def test_bf16_host_entry_matches_device_entry():
     assert hits > 0
 
 
+def test_per_head_weighted_split():
+    """Per-head matching on large steps (most units have a head that misses, so
+    they read every key): the rate-weighted split with per-head key bounds."""
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=4, L0=(32768, 30000, 31000, 29000), steps=6, head_labels=True,
+                                              hit_model=("iid", 0.5))
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), per_head=1)
+    assert 0 < r["hits"] < wl.steps * wl.B * wl.Hq
+
+
 def test_per_head_host_entry_matches_device_entry():
     """The host entry returns [B][Hq] decisions with per-head matching."""
     import kv_cache_reuse_b200 as mac
