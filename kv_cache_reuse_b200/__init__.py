@@ -41,6 +41,78 @@ def _ptr(t) -> Optional[int]:
     raise TypeError("unsupported argument type %r" % type(t))
 
 
+class _Kinds(dict):
+    """Accepted element types, named by suffix ("float32" matches torch.float32
+    and numpy float32); each dtype object seen is decided once and remembered."""
+
+    def __init__(self, *names):
+        super().__init__()
+        self.names = names
+
+    def __missing__(self, dtype):
+        ok = self[dtype] = any(str(dtype).endswith(k) for k in self.names)
+        return ok
+
+
+_F32, _I32, _U8 = _Kinds("float32"), _Kinds("int32"), _Kinds("uint8", "bool")
+_BF16 = _Kinds("int16", "uint16", "bfloat16")  # bf16 bit patterns
+
+
+def _expect(t, name, shape, kinds, where=None):
+    """Check a tensor or array argument against the state's configuration:
+    shape (or element count when shape is an int), element type, and device
+    ("cuda" or "cpu") -- a mismatch would make the kernels read or write
+    outside the caller's buffer.  Raw integer pointers and None are not
+    checked (the caller vouches for them)."""
+    if t is None or t.__class__ is int:
+        return
+    if not kinds[t.dtype]:
+        raise ValueError("%s: element type %s, expected one of %s" % (name, t.dtype, "/".join(kinds.names)))
+    if shape.__class__ is int:
+        n = t.numel() if hasattr(t, "numel") else t.size
+        if n < shape:
+            raise ValueError("%s: %d elements, the configuration needs %d" % (name, n, shape))
+    elif t.shape != shape:
+        raise ValueError("%s: shape %s, expected %s" % (name, tuple(t.shape), shape))
+    if where is not None and getattr(t, "is_cuda", False) != (where == "cuda"):
+        raise ValueError("%s: expected a %s buffer" % (name, "device" if where == "cuda" else "host"))
+
+
+def _spec(st):
+    """Expected shapes and element types of a state's buffers (computed once)."""
+    sp = st.__dict__.get("_spec_cache")
+    if sp is None:
+        c = st.cfg
+        B, Hq, Hkv, D = c.batch, c.num_q_heads, c.num_kv_heads, c.head_dim
+        nd = Hq if c.match_per_head else Hkv
+        rows = c.max_seq * B if c.page_size == 0 else c.num_pages * c.page_size
+        sp = dict(B=B, Hq=Hq, Hkv=Hkv, D=D, q=(B, Hq, D), qk=_BF16 if c.q_bf16 else _F32, b=(B,), o=(B, Hq, D),
+                  l=(B, Hq), d=(B, nd), kv=rows * Hkv * D, paged=c.page_size > 0, bt=(B, c.max_pages_per_seq),
+                  row=(B, Hkv, D))
+        st.__dict__["_spec_cache"] = sp
+    return sp
+
+
+def _check_step_args(st, q_pre=None, rope_pos=None, seq_lens=None, out=None, lse=None, hit=None, mpos=None,
+                     K=None, V=None, block_table=None, where="cuda", n=None):
+    """Validate the tensors of a step against a MacState's configuration."""
+    if not isinstance(st, MacState):
+        return
+    sp = _spec(st)
+    lead = () if n is None else (n,)
+    _expect(q_pre, "q_pre", lead + sp["q"], sp["qk"], where)
+    _expect(rope_pos, "rope_pos", lead + sp["b"], _I32, where)
+    _expect(seq_lens, "seq_lens", lead + sp["b"], _I32, where)
+    _expect(out, "out", sp["o"], _F32, where)
+    _expect(lse, "lse", sp["l"], _F32, where)
+    _expect(hit, "hit_mask", sp["d"], _U8, where)
+    _expect(mpos, "match_pos", sp["d"], _I32, where)
+    _expect(K, "K", sp["kv"], _BF16, "cuda")
+    _expect(V, "V", sp["kv"], _BF16, "cuda")
+    if sp["paged"]:
+        _expect(block_table, "block_table", sp["bt"], _I32, "cuda")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -135,6 +207,7 @@ def mac_reset_seq(st, b: int, stream=None) -> None:
 
 def mac_decode_step(st, q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
                     stream=None) -> None:
+    _check_step_args(st, q_pre, rope_pos, seq_lens, out, lse, hit_mask, match_pos, K, V, block_table)
     check("mac_decode_step", load().mac_decode_step(
         _h(st), _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens), _ptr(out),
         _ptr(lse), _ptr(hit_mask), _ptr(match_pos), _stream(stream)))
@@ -142,17 +215,23 @@ def mac_decode_step(st, q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, 
 
 def mac_match(st, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
               stream=None) -> None:
+    _check_step_args(st, q_pre, rope_pos, seq_lens, out, lse, hit_mask, match_pos, block_table=block_table)
     check("mac_match", load().mac_match(
         _h(st), _ptr(q_pre), _ptr(rope_pos), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
         _ptr(hit_mask), _ptr(match_pos), _stream(stream)))
 
 
 def mac_attend(st, K, V, block_table, out, lse, stream=None) -> None:
+    _check_step_args(st, out=out, lse=lse, K=K, V=V, block_table=block_table)
     check("mac_attend", load().mac_attend(_h(st), _ptr(K), _ptr(V), _ptr(block_table), _ptr(out), _ptr(lse),
                                           _stream(stream)))
 
 
 def mac_append_kv(st, K, V, block_table, seq_lens, k_new, v_new, stream=None) -> None:
+    _check_step_args(st, seq_lens=seq_lens, K=K, V=V, block_table=block_table)
+    if isinstance(st, MacState):
+        _expect(k_new, "k_new", _spec(st)["row"], _BF16, "cuda")
+        _expect(v_new, "v_new", _spec(st)["row"], _BF16, "cuda")
     check("mac_append_kv", load().mac_append_kv(_h(st), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens),
                                                 _ptr(k_new), _ptr(v_new), _stream(stream)))
 
@@ -160,6 +239,11 @@ def mac_append_kv(st, K, V, block_table, seq_lens, k_new, v_new, stream=None) ->
 def mac_decode_step_host(st, q_pre_h, rope_pos_h, seq_lens_h, k_new_h, v_new_h, K, V, block_table, out_h, lse_h,
                          hit_h=None, match_pos_h=None, stream=None) -> int:
     """Host-buffer step; returns MAC_OK or MAC_ERR_DEVICE (status word set)."""
+    _check_step_args(st, q_pre_h, rope_pos_h, seq_lens_h, out_h, lse_h, hit_h, match_pos_h, K, V, block_table,
+                     where="cpu")
+    if isinstance(st, MacState):
+        _expect(k_new_h, "k_new_h", _spec(st)["row"], _BF16, "cpu")
+        _expect(v_new_h, "v_new_h", _spec(st)["row"], _BF16, "cpu")
     rc = load().mac_decode_step_host(
         _h(st), _ptr(q_pre_h), _ptr(rope_pos_h), _ptr(seq_lens_h), _ptr(k_new_h), _ptr(v_new_h), _ptr(K), _ptr(V),
         _ptr(block_table), _ptr(out_h), _ptr(lse_h), _ptr(hit_h), _ptr(match_pos_h), _stream(stream))
@@ -202,6 +286,8 @@ def mac_set_piece_cost(st, keys: int) -> None:
 
 
 def mac_warm_start(st, n: int, q_pre, rope_pos, K, V, block_table, seq_lens, stream=None) -> None:
+    if n > 0:
+        _check_step_args(st, q_pre, rope_pos, seq_lens, K=K, V=V, block_table=block_table, n=n)
     check("mac_warm_start", load().mac_warm_start(_h(st), int(n), _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V),
                                                  _ptr(block_table), _ptr(seq_lens), _stream(stream)))
 

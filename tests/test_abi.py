@@ -83,3 +83,29 @@ def test_warm_start_rejects_bad_arguments(lib):
     with pytest.raises(mac.MacError) as e:
         mac.mac_warm_start(None, 1, 16, 16, 16, 16, None, 16, stream=0)
     assert e.value.code == mac.MAC_ERR_ARG
+
+
+def test_binding_rejects_buffers_that_do_not_fit_the_state(lib):
+    """A tensor whose shape, element type or device does not match the state's
+    configuration is refused in the binding, before anything reaches a kernel
+    (the kernels would read or write outside it)."""
+    import torch
+    import kv_cache_reuse_b200 as mac
+    st = mac.MacState.__new__(mac.MacState)  # configuration only, no device state
+    st.cfg = mac.MacConfig(2, 8, 2, 64, 4, 8, 0.1, 1e4, 0, 100, 0, 0, 0, 0, 0, 0)
+    st.handle = None
+    B, Hq, Hkv, D = 2, 8, 2, 64
+    ok = dict(q_pre=torch.zeros(B, Hq, D), rope_pos=torch.zeros(B, dtype=torch.int32),
+              seq_lens=torch.zeros(B, dtype=torch.int32), out=torch.zeros(B, Hq, D), lse=torch.zeros(B, Hq))
+    for name, bad in (("q_pre", torch.zeros(B, Hkv, D)), ("q_pre", torch.zeros(B, Hq, D, dtype=torch.float64)),
+                      ("out", torch.zeros(B, Hq, D - 1)), ("lse", torch.zeros(B, Hq, dtype=torch.int32)),
+                      ("seq_lens", torch.zeros(B + 1, dtype=torch.int32))):
+        args = dict(ok, **{name: bad})
+        with pytest.raises(ValueError):
+            mac.mac_match(st, args["q_pre"], args["rope_pos"], None, args["seq_lens"], args["out"], args["lse"])
+    # host buffers are refused where device buffers are expected
+    with pytest.raises(ValueError, match="device"):
+        mac.mac_match(st, ok["q_pre"], ok["rope_pos"], None, ok["seq_lens"], ok["out"], ok["lse"])
+    # a cache smaller than the configured capacity
+    with pytest.raises(ValueError, match="elements"):
+        mac.mac_attend(st, torch.zeros(B * 99 * Hkv * D, dtype=torch.int16), 16, None, 16, 16)
