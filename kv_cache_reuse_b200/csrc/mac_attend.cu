@@ -88,6 +88,7 @@ struct Cfg {
   static constexpr int PB = kSubKeys * GP;        // floats of one weights exchange buffer
   static constexpr int WB = SF > 2 * PB ? SF : 2 * PB;  // per-warp scratch floats
   static constexpr int QW = GP == 4 ? 2 : 4;      // query B-fragment registers per k-step
+  static_assert(WB % 4 == 0 && (NQ * GD) % 4 == 0, "warp slots hold 16-byte aligned runs");
 };
 
 template <int D, int GP>
@@ -433,101 +434,6 @@ __device__ __forceinline__ void fold_state(float& M, float& L, float (&O)[N], fl
   M = Mn;
 }
 
-// Last arriver of a split unit: merge its partials.  Segment A's partials
-// (with the reused state on a hit) give the new prefix state over [0, c_t),
-// stored in the ring; that state and segment B's partials give the output.
-// Every thread owns a slice of VEC consecutive elements of one head (four
-// heads at a time) and folds all of the unit's partials for its slice, BC
-// partials' loads in flight per round: no exchange between warps, no barrier.
-template <int D, int GP, int GF, bool PH>
-__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
-  constexpr int QD = 4 * D;                         // elements of four heads
-  constexpr int VEC = QD / (kConsumerWarps * 32);  // elements per thread: 2 (D = 128) or 1 (D = 64)
-  constexpr int BC = 4;  // partials per round of loads (cold code: 4 measured best of 2, 4, 8, 16, 24)
-  static_assert(VEC * kConsumerWarps * 32 == QD && (VEC == 1 || VEC == 2), "merge layout");
-  (void)sm;
-  (void)sync_phase;
-  const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
-  const UnitPlan* const pp = p.plan + u;
-  const HeadPlan* const hp = p.hplan + u;
-  const int hit = pp->hit, hmask = PH ? hp->hmask : 0, src_slot = pp->src_slot, dst_slot = pp->dst_slot;
-  const int end = pp->end;
-  const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
-  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
-  const int Wp1 = p.W + 1;
-  const int nA = sA.npieces, n = nA + sB.npieces;
-  const size_t ds = (size_t)u * Wp1 + dst_slot;
-  const int e0 = threadIdx.x * VEC;  // this thread's first element in a quad [4][D]
-  const int hq = e0 / D, d0 = e0 - hq * D;
-
-  for (int h0 = 0; h0 < G; h0 += 4) {
-    const int h = h0 + hq;
-    if (h >= G) break;  // no barriers below: a thread past the group leaves
-    const size_t oo = (size_t)h * D + d0;  // the slice's offset in an o [G][D]
-    float MA = -INFINITY, LA = 0.f, OA[VEC], MB = -INFINITY, LB = 0.f, OB[VEC];
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) OA[j] = OB[j] = 0.f;
-    if (PH ? ((hmask >> h) & 1) : hit) {  // the reused state joins set A (its o is normalised)
-      const size_t rs = (size_t)u * Wp1 + (PH ? hp->hsrc[h] : src_slot);
-      const float rl = __ldcg(p.ring_l + rs * G + h), rm = __ldcg(p.ring_m + rs * G + h) * kLog2e;
-      float o[VEC];
-#pragma unroll
-      for (int j = 0; j < VEC; ++j) o[j] = ring_o_at(p.ring_o, rs * GD + oo + j, p.ring_bf16) * rl;
-      fold_state<VEC>(MA, LA, OA, rm, rl, o);
-    }
-    for (int i0 = 0; i0 < n; i0 += BC) {
-      float ov[BC][VEC], mv[BC], lv[BC];
-#pragma unroll
-      for (int k = 0; k < BC; ++k) {
-        const int i = i0 + k;
-        if (i < n) {
-          const float* q = p.part + (size_t)(i < nA ? sA.pbase + i : sB.pbase + (i - nA)) * PF;
-          if constexpr (VEC == 2) {
-            const float2 t = __ldcg(reinterpret_cast<const float2*>(q + oo));
-            ov[k][0] = t.x;
-            ov[k][VEC - 1] = t.y;
-          } else {
-            ov[k][0] = __ldcg(q + oo);
-          }
-          mv[k] = __ldcg(q + GD + h);
-          lv[k] = __ldcg(q + GD + G4 + h);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < BC; ++k) {
-        const int i = i0 + k;
-        if (i < n) {
-          if (i < nA)
-            fold_state<VEC>(MA, LA, OA, mv[k], lv[k], ov[k]);
-          else
-            fold_state<VEC>(MB, LB, OB, mv[k], lv[k], ov[k]);
-        }
-      }
-    }
-    // new prefix state = set A (normalised) into the ring; output = A (+) B
-    const float M2 = fmaxf(MA, MB);
-    const float M2u = M2 == -INFINITY ? 0.f : M2;
-    const float a0 = ex2(MA - M2u), a1 = ex2(MB - M2u);
-    const float L2 = LA * a0 + LB * a1;
-    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-      ring_o_put(p.ring_o, ds * GD + oo + j, LA > 0.f ? OA[j] / LA : 0.f, p.ring_bf16);
-      p.out[orow * D + d0 + j] = (OA[j] * a0 + OB[j] * a1) / L2;
-    }
-    if (d0 == 0) {
-      p.ring_m[ds * G + h] = LA > 0.f ? MA * kLn2 : -INFINITY;
-      p.ring_l[ds * G + h] = LA;
-      p.lse[orow] = (M2 + log2f(L2)) * kLn2;
-    }
-  }
-  if (threadIdx.x == 0) {
-    p.ring_pos[(size_t)u * Wp1 + dst_slot] = end - 1;
-    p.unit_cnt[u] = 0;
-  }
-  return true;
-}
-
 // Store the warp's state in its shared-memory slot: o [GP][D] unnormalised,
 // then m [GP] and l [GP].  GP = 4: lanes tig and tig ^ 2 hold the high and
 // residual columns of the same heads.  Lanes of one tig hold different key
@@ -602,6 +508,156 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA
   }
 }
 
+// Finish of a unit from the eight warps' states in their shared-memory
+// slots: warps [0, wA) hold set A (the amend range, or segment A's
+// partials), warps [wA, 8) set B (the tail).  With a reused state (heads in
+// hmask; o, m and l on chip in sm.ring) S = reused + A, else S = A; S is the
+// unit's new ring entry in slot dst and S + B its output.
+template <int D, int GP, int GF>
+__device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D, GP>& sm, int u, int wA, int hit,
+                                              int hmask, int dst, int end) {
+  constexpr int GDP = Cfg<D, GP>::GD;
+  const int G = group_of<GF>(p), GD = G * D;
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
+  const int Wp1 = p.W + 1;
+  constexpr int PER = (GDP + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
+  // cold code once per piece: a rolled loop fetches fewer instruction lines
+#pragma unroll 1
+  for (int k = 0; k < PER; ++k) {
+    const int idx = threadIdx.x + k * kConsumerWarps * 32;
+    if (idx >= GD) break;
+    const int h = idx / D, d = idx - h * D;
+    float MA, LA, OA, MB, LB, OB;
+    combine_warps2<D, GP, GP>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
+    // new prefix state S = reused (hit) + amend
+    const bool hh = hit && ((hmask >> h) & 1);
+    const float rm = hh ? sm.ring[GDP + h] * kLog2e : -INFINITY;
+    float M = fmaxf(MA, rm);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    const float aA = ex2(MA - Mu);
+    float L = LA * aA, O = OA * aA;
+    if (hh) {
+      const float a = ex2(rm - Mu), rl = sm.ring[GDP + GP + h];
+      L += rl * a;
+      O += ring_o_at(sm.ring, idx, p.ring_bf16) * rl * a;
+    }
+    const size_t ds = (size_t)u * Wp1 + dst;
+    ring_o_put(p.ring_o, ds * GD + idx, L > 0.f ? O / L : 0.f, p.ring_bf16);
+    if (d == 0) {
+      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
+      p.ring_l[ds * G + h] = L;
+    }
+    // output = S + tail
+    const float M2 = fmaxf(M, MB);
+    const float M2u = M2 == -INFINITY ? 0.f : M2;
+    const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
+    const float L2 = L * a0 + LB * aB, O2 = O * a0 + OB * aB;
+    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    p.out[orow * D + d] = O2 / L2;
+    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+  }
+  if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
+}
+
+// Last arriver of a split unit: merge its partials.  Segment A's partials
+// (with the reused state on a hit) give the new prefix state over [0, c_t),
+// stored in the ring; that state and segment B's partials give the output.
+// The warps share the partials out -- A's over warps [0, wA), B's over the
+// rest, in proportion to their counts -- and each folds its own into one
+// state (lane: four consecutive elements of every 128, KB partials per round
+// of loads); the finish of a whole unit then combines the eight states.
+template <int D, int GP, int GF, bool PH>
+__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
+  using C = Cfg<D, GP>;
+  constexpr int NCH = C::GD / 128;                // 128-element runs of a padded group: 2, 4 or 8
+  constexpr int KB = NCH <= 2 ? 8 : 16 / NCH;     // partials per round of loads
+  const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const UnitPlan* const pp = p.plan + u;
+  const int src_slot = pp->src_slot, dst_slot = pp->dst_slot, end = pp->end;
+  const int hmask = PH ? p.hplan[u].hmask : (pp->hit ? (1 << G) - 1 : 0);  // heads with a reused state
+  const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
+  const int nA = sA.npieces, nB = sB.npieces, n = nA + nB;
+  int wA = kConsumerWarps;
+  if (nB > 0) {
+    wA = nA > 0 ? (kConsumerWarps * nA + n / 2) / n : 0;
+    if (nA > 0) wA = wA < 1 ? 1 : (wA > kConsumerWarps - 1 ? kConsumerWarps - 1 : wA);
+  }
+  const bool onA = warp < wA;
+  const int cnt = onA ? nA : nB, stride = onA ? wA : kConsumerWarps - wA, first = onA ? warp : warp - wA;
+  const float* const part = p.part + (size_t)(onA ? sA.pbase : sB.pbase) * PF;
+  // the reused state on chip, in the layout of a whole unit's copy: each
+  // head's o row (fp32 or bf16 as stored), then m at GP*D and l at GP*D + GP
+  if (hmask != 0) {
+    const size_t ub = (size_t)u * (p.W + 1);
+    const int es = p.ring_bf16 ? 2 : 4, cph = D * es / 16;  // 16-byte chunks of one head's o
+    const int h = tid / cph, c = tid - h * cph;
+    if (h < G && ((hmask >> h) & 1)) {
+      const int slot = PH ? p.hplan[u].hsrc[h] : src_slot;
+      const uint4* src = reinterpret_cast<const uint4*>(ring_o_row(p.ring_o, ((ub + slot) * G + h) * D, p.ring_bf16));
+      reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.ring) + (size_t)h * D * es)[c] = __ldcg(src + c);
+    }
+    if (tid < 2 * G) {
+      const int hh = tid < G ? tid : tid - G;
+      if ((hmask >> hh) & 1) {
+        const size_t e = (ub + (PH ? p.hplan[u].hsrc[hh] : src_slot)) * G + hh;
+        sm.ring[C::GD + (tid < G ? hh : GP + hh)] = __ldcg(tid < G ? p.ring_m + e : p.ring_l + e);
+      }
+    }
+  }
+  float M[NCH], L[NCH], O[NCH][4];
+#pragma unroll
+  for (int j = 0; j < NCH; ++j) {
+    M[j] = -INFINITY;
+    L[j] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) O[j][c] = 0.f;
+  }
+#pragma unroll 1
+  for (int i0 = first; i0 < cnt; i0 += KB * stride) {
+    float4 ov[KB][NCH];
+    float mv[KB][NCH], lv[KB][NCH];
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int i = i0 + k * stride;
+      const float* q = part + (size_t)i * PF;
+#pragma unroll
+      for (int j = 0; j < NCH; ++j) {
+        const int e = j * 128 + lane * 4, h = e / D;
+        if (i < cnt && e < GD) {
+          ov[k][j] = __ldcg(reinterpret_cast<const float4*>(q + e));
+          mv[k][j] = __ldcg(q + GD + h);
+          lv[k][j] = __ldcg(q + GD + G4 + h);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < KB; ++k)
+#pragma unroll
+      for (int j = 0; j < NCH; ++j)
+        if (i0 + k * stride < cnt && j * 128 + lane * 4 < GD)
+          fold_state<4>(M[j], L[j], O[j], mv[k][j], lv[k][j], &ov[k][j].x);
+  }
+  // this warp's state into its slot: o [GP][D], m [GP], l [GP]
+  float* const wb = sm.wbuf[warp];
+#pragma unroll
+  for (int j = 0; j < NCH; ++j) {
+    const int e = j * 128 + lane * 4, h = e / D;
+    if (e < GD) {
+      *reinterpret_cast<float4*>(wb + e) = make_float4(O[j][0], O[j][1], O[j][2], O[j][3]);
+      if (e - h * D == 0) {
+        wb[C::GD + h] = M[j];
+        wb[C::GD + GP + h] = L[j];
+      }
+    }
+  }
+  if (!consumer_sync(sm, sync_phase, p.status)) return false;
+  unit_epilogue<D, GP, GF>(p, sm, u, wA, hmask != 0, hmask, dst_slot, end);
+  if (tid == 0) p.unit_cnt[u] = 0;
+  // the warps' slots and the ring buffer are reused by the next piece
+  return consumer_sync(sm, sync_phase, p.status);
+}
+
 // End of a split piece: combine the 8 warps, write the partial, count it
 // and, if it was the unit's last, merge the unit.
 template <int D, int GP, int GF, bool PH>
@@ -649,10 +705,7 @@ template <int D, int GP, int GF>
 __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D, GP>& A, int u, int wA, int hit,
                               int hmask, int dst, int end, float rml, uint32_t ring_phase, uint32_t& sync_phase) {
   constexpr int GDP = Cfg<D, GP>::GD;
-  const int G = group_of<GF>(p), GD = G * D;
-  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
-  const int Wp1 = p.W + 1;
-  constexpr int PER = (GDP + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
+  const int G = group_of<GF>(p);
   warp_combine_store<D, GP>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!kBulkML<GF> && hit && (int)threadIdx.x < 2 * G &&
       ((hmask >> ((int)threadIdx.x < G ? (int)threadIdx.x : (int)threadIdx.x - G)) & 1))
@@ -660,42 +713,7 @@ __device__ bool finalize_unit(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D,
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   // the reused o was copied on chip at the start of the piece
   if (hit && !mbar_wait(&sm.rfull, ring_phase, &sm.abort_flag, p.status)) return false;
-  // cold code once per piece: a rolled loop fetches fewer instruction lines
-#pragma unroll 1
-  for (int k = 0; k < PER; ++k) {
-    const int idx = threadIdx.x + k * kConsumerWarps * 32;
-    if (idx >= GD) break;
-    const int h = idx / D, d = idx - h * D;
-    float MA, LA, OA, MB, LB, OB;
-    combine_warps2<D, GP, GP>(sm, wA, idx, h, MA, LA, OA, MB, LB, OB);
-    // new prefix state S = reused (hit) + amend
-    const bool hh = hit && ((hmask >> h) & 1);
-    const float rm = hh ? sm.ring[GDP + h] * kLog2e : -INFINITY;
-    float M = fmaxf(MA, rm);
-    const float Mu = M == -INFINITY ? 0.f : M;
-    const float aA = ex2(MA - Mu);
-    float L = LA * aA, O = OA * aA;
-    if (hh) {
-      const float a = ex2(rm - Mu), rl = sm.ring[GDP + GP + h];
-      L += rl * a;
-      O += ring_o_at(sm.ring, idx, p.ring_bf16) * rl * a;
-    }
-    const size_t ds = (size_t)u * Wp1 + dst;
-    ring_o_put(p.ring_o, ds * GD + idx, L > 0.f ? O / L : 0.f, p.ring_bf16);
-    if (d == 0) {
-      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
-      p.ring_l[ds * G + h] = L;
-    }
-    // output = S + tail
-    const float M2 = fmaxf(M, MB);
-    const float M2u = M2 == -INFINITY ? 0.f : M2;
-    const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
-    const float L2 = L * a0 + LB * aB, O2 = O * a0 + OB * aB;
-    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
-    p.out[orow * D + d] = O2 / L2;
-    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
-  }
-  if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
+  unit_epilogue<D, GP, GF>(p, sm, u, wA, hit, hmask, dst, end);
   // the warps' slots are reused by the next piece
   return consumer_sync(sm, sync_phase, p.status);
 }
