@@ -542,7 +542,7 @@ __device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D,
       O += ring_o_at(sm.ring, idx, p.ring_bf16) * rl * a;
     }
     const size_t ds = (size_t)u * Wp1 + dst;
-    ring_o_put(p.ring_o, ds * GD + idx, L > 0.f ? O / L : 0.f, p.ring_bf16);
+    ring_o_put(p.ring_o, ds * GD + idx, L > 0.f ? __fdividef(O, L) : 0.f, p.ring_bf16);
     if (d == 0) {
       p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
       p.ring_l[ds * G + h] = L;
@@ -553,8 +553,8 @@ __device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D,
     const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
     const float L2 = L * a0 + LB * aB, O2 = O * a0 + OB * aB;
     const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
-    p.out[orow * D + d] = O2 / L2;
-    if (d == 0) p.lse[orow] = (M2 + log2f(L2)) * kLn2;
+    p.out[orow * D + d] = __fdividef(O2, L2);  // L2 >= 1: every unit attends at least one key
+    if (d == 0) p.lse[orow] = (M2 + __log2f(L2)) * kLn2;
   }
   if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
 }
