@@ -325,6 +325,26 @@ def test_group_sizes_all_miss_large(Hq, Hkv):
     assert r["hits"] == 0
 
 
+@pytest.mark.parametrize("case", ["g4_d128", "g8_d128", "g3_d64", "g8_d128_hits"])
+def test_one_unit_over_every_cta(case):
+    """A single (sequence, KV head) whose keys are cut over all 148 CTAs: the
+    merge folds ~150 partials, several rounds of loads per warp, with the
+    group padded (3 of 4) or exact (4, 8), on misses and on hits (the reused
+    state joins segment A, the amend band and tail are the fresh range)."""
+    tiny, llama = synth.WORKLOADS["tiny"], synth.WORKLOADS["llama8b_32k"]
+    tau = 0.0
+    if case == "g4_d128":
+        wl = llama.with_(B=1, Hq=4, Hkv=1, L0=(40000,), steps=3)
+    elif case == "g8_d128":
+        wl = llama.with_(B=1, Hq=8, Hkv=1, L0=(24000,), steps=3)
+    elif case == "g3_d64":
+        wl = tiny.with_(B=1, Hq=3, Hkv=1, L0=(30000,), steps=3)
+    else:
+        wl, tau = llama.with_(B=1, Hq=8, Hkv=1, L0=(24000,), steps=12), None
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=tau, tune={"whole_unit_keys": 0})
+    assert r["hits"] == 0 if tau == 0.0 else r["hits"] > 0
+
+
 @pytest.mark.parametrize("case", ["g4_d64", "g4_d128", "g4_split", "g3_paged", "g8_split", "g1", "g6_cut1"])
 def test_per_head_matching(case):
     """Per-head matching on streams whose heads repeat on their own: every
