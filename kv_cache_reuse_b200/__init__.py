@@ -58,14 +58,21 @@ _F32, _I32, _U8 = _Kinds("float32"), _Kinds("int32"), _Kinds("uint8", "bool")
 _BF16 = _Kinds("int16", "uint16", "bfloat16")  # bf16 bit patterns
 
 
-def _expect(t, name, shape, kinds, where=None):
-    """Check a tensor or array argument against the state's configuration:
-    shape (or element count when shape is an int), element type, and device
-    ("cuda" or "cpu") -- a mismatch would make the kernels read or write
-    outside the caller's buffer.  Raw integer pointers and None are not
-    checked (the caller vouches for them)."""
-    if t is None or t.__class__ is int:
-        return
+_tensor_cls = None  # torch.Tensor, once one has been seen (keeps torch a lazy import)
+
+
+def _arg(t, name, shape, kinds, where=None):
+    """Address of a tensor or array argument after checking it against the
+    state's configuration: shape (or element count when shape is an int),
+    element type, device ("cuda" or "cpu") and contiguity -- a mismatch would
+    make the kernels read or write outside the caller's buffer.  None stays
+    None; a raw integer address passes unchecked (the caller vouches for it)."""
+    global _tensor_cls
+    if t is None:
+        return None
+    c = t.__class__
+    if c is int:
+        return t
     if not kinds[t.dtype]:
         raise ValueError("%s: element type %s, expected one of %s" % (name, t.dtype, "/".join(kinds.names)))
     if shape.__class__ is int:
@@ -74,8 +81,18 @@ def _expect(t, name, shape, kinds, where=None):
             raise ValueError("%s: %d elements, the configuration needs %d" % (name, n, shape))
     elif t.shape != shape:
         raise ValueError("%s: shape %s, expected %s" % (name, tuple(t.shape), shape))
-    if where is not None and getattr(t, "is_cuda", False) != (where == "cuda"):
-        raise ValueError("%s: expected a %s buffer" % (name, "device" if where == "cuda" else "host"))
+    if c is _tensor_cls or hasattr(t, "data_ptr"):
+        _tensor_cls = c
+        if where is not None and t.is_cuda != (where == "cuda"):
+            raise ValueError("%s: expected a %s buffer" % (name, "device" if where == "cuda" else "host"))
+        if not t.is_contiguous():
+            raise ValueError("%s: tensor arguments must be contiguous" % name)
+        return t.data_ptr()
+    if where == "cuda":
+        raise ValueError("%s: expected a device buffer" % name)
+    if not t.flags.c_contiguous:
+        raise ValueError("%s: arrays must be C-contiguous" % name)
+    return t.ctypes.data
 
 
 def _spec(st):
@@ -93,24 +110,31 @@ def _spec(st):
     return sp
 
 
-def _check_step_args(st, q_pre=None, rope_pos=None, seq_lens=None, out=None, lse=None, hit=None, mpos=None,
-                     K=None, V=None, block_table=None, where="cuda", n=None):
-    """Validate the tensors of a step against a MacState's configuration."""
+def _args(st, where, q_pre=None, rope_pos=None, seq_lens=None, out=None, lse=None, hit=None, mpos=None, K=None,
+          V=None, block_table=None, k_new=None, v_new=None, n=None):
+    """Addresses of a step's arguments, in this order: q_pre, rope_pos,
+    seq_lens, out, lse, hit_mask, match_pos, K, V, block_table, k_new, v_new.
+    With a MacState each is checked against its configuration (the step's
+    own buffers on `where`, the cache always on the device; n: leading
+    dimension of q_pre, rope_pos and seq_lens for a warm start); a raw
+    handle gets the addresses unchecked."""
     if not isinstance(st, MacState):
-        return
+        return (_ptr(q_pre), _ptr(rope_pos), _ptr(seq_lens), _ptr(out), _ptr(lse), _ptr(hit), _ptr(mpos), _ptr(K),
+                _ptr(V), _ptr(block_table), _ptr(k_new), _ptr(v_new))
     sp = _spec(st)
-    lead = () if n is None else (n,)
-    _expect(q_pre, "q_pre", lead + sp["q"], sp["qk"], where)
-    _expect(rope_pos, "rope_pos", lead + sp["b"], _I32, where)
-    _expect(seq_lens, "seq_lens", lead + sp["b"], _I32, where)
-    _expect(out, "out", sp["o"], _F32, where)
-    _expect(lse, "lse", sp["l"], _F32, where)
-    _expect(hit, "hit_mask", sp["d"], _U8, where)
-    _expect(mpos, "match_pos", sp["d"], _I32, where)
-    _expect(K, "K", sp["kv"], _BF16, "cuda")
-    _expect(V, "V", sp["kv"], _BF16, "cuda")
-    if sp["paged"]:
-        _expect(block_table, "block_table", sp["bt"], _I32, "cuda")
+    q, b = (sp["q"], sp["b"]) if n is None else ((n,) + sp["q"], (n,) + sp["b"])
+    return (_arg(q_pre, "q_pre", q, sp["qk"], where),
+            _arg(rope_pos, "rope_pos", b, _I32, where),
+            _arg(seq_lens, "seq_lens", b, _I32, where),
+            _arg(out, "out", sp["o"], _F32, where),
+            _arg(lse, "lse", sp["l"], _F32, where),
+            _arg(hit, "hit_mask", sp["d"], _U8, where),
+            _arg(mpos, "match_pos", sp["d"], _I32, where),
+            _arg(K, "K", sp["kv"], _BF16, "cuda"),
+            _arg(V, "V", sp["kv"], _BF16, "cuda"),
+            _arg(block_table, "block_table", sp["bt"], _I32, "cuda") if sp["paged"] else _ptr(block_table),
+            _arg(k_new, "k_new", sp["row"], _BF16, where),
+            _arg(v_new, "v_new", sp["row"], _BF16, where))
 
 
 def _stream(stream) -> Optional[int]:
@@ -207,46 +231,35 @@ def mac_reset_seq(st, b: int, stream=None) -> None:
 
 def mac_decode_step(st, q_pre, rope_pos, K, V, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
                     stream=None) -> None:
-    _check_step_args(st, q_pre, rope_pos, seq_lens, out, lse, hit_mask, match_pos, K, V, block_table)
-    check("mac_decode_step", load().mac_decode_step(
-        _h(st), _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens), _ptr(out),
-        _ptr(lse), _ptr(hit_mask), _ptr(match_pos), _stream(stream)))
+    q, pz, ln, o, l, hm, mp, k, v, bt, _, _ = _args(st, "cuda", q_pre, rope_pos, seq_lens, out, lse, hit_mask,
+                                                   match_pos, K, V, block_table)
+    check("mac_decode_step", load().mac_decode_step(_h(st), q, pz, k, v, bt, ln, o, l, hm, mp, _stream(stream)))
 
 
 def mac_match(st, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask=None, match_pos=None,
               stream=None) -> None:
-    _check_step_args(st, q_pre, rope_pos, seq_lens, out, lse, hit_mask, match_pos, block_table=block_table)
-    check("mac_match", load().mac_match(
-        _h(st), _ptr(q_pre), _ptr(rope_pos), _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse),
-        _ptr(hit_mask), _ptr(match_pos), _stream(stream)))
+    q, pz, ln, o, l, hm, mp, _, _, bt, _, _ = _args(st, "cuda", q_pre, rope_pos, seq_lens, out, lse, hit_mask,
+                                                   match_pos, block_table=block_table)
+    check("mac_match", load().mac_match(_h(st), q, pz, bt, ln, o, l, hm, mp, _stream(stream)))
 
 
 def mac_attend(st, K, V, block_table, out, lse, stream=None) -> None:
-    _check_step_args(st, out=out, lse=lse, K=K, V=V, block_table=block_table)
-    check("mac_attend", load().mac_attend(_h(st), _ptr(K), _ptr(V), _ptr(block_table), _ptr(out), _ptr(lse),
-                                          _stream(stream)))
+    _, _, _, o, l, _, _, k, v, bt, _, _ = _args(st, "cuda", out=out, lse=lse, K=K, V=V, block_table=block_table)
+    check("mac_attend", load().mac_attend(_h(st), k, v, bt, o, l, _stream(stream)))
 
 
 def mac_append_kv(st, K, V, block_table, seq_lens, k_new, v_new, stream=None) -> None:
-    _check_step_args(st, seq_lens=seq_lens, K=K, V=V, block_table=block_table)
-    if isinstance(st, MacState):
-        _expect(k_new, "k_new", _spec(st)["row"], _BF16, "cuda")
-        _expect(v_new, "v_new", _spec(st)["row"], _BF16, "cuda")
-    check("mac_append_kv", load().mac_append_kv(_h(st), _ptr(K), _ptr(V), _ptr(block_table), _ptr(seq_lens),
-                                                _ptr(k_new), _ptr(v_new), _stream(stream)))
+    _, _, ln, _, _, _, _, k, v, bt, kn, vn = _args(st, "cuda", seq_lens=seq_lens, K=K, V=V, block_table=block_table,
+                                                  k_new=k_new, v_new=v_new)
+    check("mac_append_kv", load().mac_append_kv(_h(st), k, v, bt, ln, kn, vn, _stream(stream)))
 
 
 def mac_decode_step_host(st, q_pre_h, rope_pos_h, seq_lens_h, k_new_h, v_new_h, K, V, block_table, out_h, lse_h,
                          hit_h=None, match_pos_h=None, stream=None) -> int:
     """Host-buffer step; returns MAC_OK or MAC_ERR_DEVICE (status word set)."""
-    _check_step_args(st, q_pre_h, rope_pos_h, seq_lens_h, out_h, lse_h, hit_h, match_pos_h, K, V, block_table,
-                     where="cpu")
-    if isinstance(st, MacState):
-        _expect(k_new_h, "k_new_h", _spec(st)["row"], _BF16, "cpu")
-        _expect(v_new_h, "v_new_h", _spec(st)["row"], _BF16, "cpu")
-    rc = load().mac_decode_step_host(
-        _h(st), _ptr(q_pre_h), _ptr(rope_pos_h), _ptr(seq_lens_h), _ptr(k_new_h), _ptr(v_new_h), _ptr(K), _ptr(V),
-        _ptr(block_table), _ptr(out_h), _ptr(lse_h), _ptr(hit_h), _ptr(match_pos_h), _stream(stream))
+    q, pz, ln, o, l, hm, mp, k, v, bt, kn, vn = _args(st, "cpu", q_pre_h, rope_pos_h, seq_lens_h, out_h, lse_h, hit_h,
+                                                     match_pos_h, K, V, block_table, k_new_h, v_new_h)
+    rc = load().mac_decode_step_host(_h(st), q, pz, ln, kn, vn, k, v, bt, o, l, hm, mp, _stream(stream))
     if rc not in (MAC_OK, MAC_ERR_DEVICE):
         check("mac_decode_step_host", rc)
     return rc
@@ -287,9 +300,11 @@ def mac_set_piece_cost(st, keys: int) -> None:
 
 def mac_warm_start(st, n: int, q_pre, rope_pos, K, V, block_table, seq_lens, stream=None) -> None:
     if n > 0:
-        _check_step_args(st, q_pre, rope_pos, seq_lens, K=K, V=V, block_table=block_table, n=n)
-    check("mac_warm_start", load().mac_warm_start(_h(st), int(n), _ptr(q_pre), _ptr(rope_pos), _ptr(K), _ptr(V),
-                                                 _ptr(block_table), _ptr(seq_lens), _stream(stream)))
+        q, pz, ln, _, _, _, _, k, v, bt, _, _ = _args(st, "cuda", q_pre, rope_pos, seq_lens, K=K, V=V,
+                                                     block_table=block_table, n=n)
+    else:
+        q, pz, ln, k, v, bt = _ptr(q_pre), _ptr(rope_pos), _ptr(seq_lens), _ptr(K), _ptr(V), _ptr(block_table)
+    check("mac_warm_start", load().mac_warm_start(_h(st), int(n), q, pz, k, v, bt, ln, _stream(stream)))
 
 
 def mac_set_whole_unit_keys(st, keys: int) -> None:
