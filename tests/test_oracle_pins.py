@@ -127,6 +127,44 @@ def _run(wl, steps=None, stream=None, cache=None, tau=None, band=None, rope_zero
     return stream, cache, res
 
 
+@pytest.mark.parametrize("G", [1, 4])
+def test_distance_equal_to_threshold_is_a_miss(G):
+    """The match test is strict: an entry at distance exactly tau misses, and
+    one ulp more of tau makes it a hit.  The queries are multiples of 1/8 and
+    differ by 0.5 in one element per head, so the mean over heads of the
+    squared L2 distance is exactly 0.25 in any precision."""
+    wl = _tiny(Hq=G, Hkv=1, steps=3)
+    cache = synth.kv_cache(wl)
+    stream = synth.queries(wl)
+    q0 = ((np.arange(G * wl.D).reshape(1, G, wl.D) % 16 - 8) / 8).astype(np.float32)
+    q1 = q0.copy()
+    q1[0, :, 3] += np.float32(0.5)
+    for tau, hit in ((0.25, False), (np.nextafter(0.25, 1.0), True)):
+        orc = oracle.Oracle.for_workload(wl, cache, tau=tau)
+        orc.step(q0, stream.rope_pos[0], cache.K, cache.V, cache.block_table, stream.seq_lens[0])
+        r = orc.step(q1, stream.rope_pos[1], cache.K, cache.V, cache.block_table, stream.seq_lens[1])
+        assert bool(r.hit[0, 0]) is hit
+        assert r.d_best[0, 0] == 0.25
+        if hit:
+            assert r.match_pos[0, 0] == stream.seq_lens[0][0] - 1  # the first step's position
+
+
+def test_equal_distances_pick_the_most_recent_entry():
+    """Two window entries at the same distance: the match is the more recent
+    one (its reused prefix is longer and its tail shorter)."""
+    wl = _tiny(steps=5)
+    cache = synth.kv_cache(wl)
+    stream = synth.queries(wl)
+    q = stream.q[0].copy()
+    far = (q + np.float32(3.0)).astype(np.float32)
+    orc = oracle.Oracle.for_workload(wl, cache, tau=1.0)
+    seq = [q, far, q, q]  # steps 0 and 2 hold the same query; step 3 repeats it
+    for t, qt in enumerate(seq):
+        r = orc.step(qt, stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+    assert r.hit[0, 0] and r.d_best[0, 0] == 0.0 and r.d_second[0, 0] == 0.0
+    assert r.match_pos[0, 0] == stream.seq_lens[2][0] - 1
+
+
 @pytest.mark.parametrize("cut_mode", [0, 1])
 def test_forced_miss_equals_dense(cut_mode):
     """Threshold 0 (strict test) makes every step a miss, i.e. dense attention,
