@@ -325,6 +325,35 @@ def test_group_sizes_all_miss_large(Hq, Hkv):
     assert r["hits"] == 0
 
 
+@pytest.mark.parametrize("G", [1, 4])
+def test_threshold_is_strict_and_ties_pick_the_most_recent(G):
+    """Decisions at the edges the generator's margins stay away from: a
+    distance exactly at the threshold misses and one ulp more of threshold
+    hits (the queries make the distance exactly 0.25 in fp32 and fp64), and
+    equal distances pick the most recent entry -- the kernels decide as the
+    oracle does."""
+    wl = synth.WORKLOADS["tiny"].with_(Hq=G, Hkv=1, steps=6)
+    cache, stream = synth.kv_cache(wl), synth.queries(wl)
+    q0 = ((np.arange(G * wl.D).reshape(1, G, wl.D) % 16 - 8) / 8).astype(np.float32)
+    q1 = q0.copy()
+    q1[0, :, 3] += np.float32(0.5)
+    far = (q0 + np.float32(3.0)).astype(np.float32)
+    for tau, hit1 in ((0.25, 0), (float(np.nextafter(np.float32(0.25), np.float32(1.0))), 1)):
+        gpu = GpuRun(wl, cache, tau=tau)
+        orc = oracle.Oracle.for_workload(wl, cache, tau=tau)
+        for t, qt in enumerate([q0, q1, far, q0, q0]):
+            r = orc.step(qt, stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+            out, lse, hit, mpos = gpu.step(qt, stream.rope_pos[t], stream.seq_lens[t])
+            np.testing.assert_array_equal(hit, r.hit, err_msg="tau %r step %d" % (tau, t))
+            np.testing.assert_array_equal(mpos, r.match_pos, err_msg="tau %r step %d" % (tau, t))
+            assert float(np.abs(out - r.out).max()) <= OUT_TOL and float(np.abs(lse - r.lse).max()) <= LSE_TOL
+            if t == 1:
+                assert int(hit[0, 0]) == hit1
+            if t == 4:  # steps 0 and 3 hold the same query: the later one is reused
+                assert hit[0, 0] == 1 and mpos[0, 0] == stream.seq_lens[3][0] - 1
+        assert gpu.st.get_status() == 0
+
+
 @pytest.mark.parametrize("case", ["g4_d128", "g8_d128", "g3_d64", "g8_d128_hits"])
 def test_one_unit_over_every_cta(case):
     """A single (sequence, KV head) whose keys are cut over all 148 CTAs: the
