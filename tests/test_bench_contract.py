@@ -49,3 +49,20 @@ def test_reference_arm_under_torchrun_prints_on_rank_zero_only():
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
     _check_line(lines[0], 2)
+
+
+def test_clock_records_that_disqualify_a_timed_region():
+    """Hardware or thermal slowdown, or SM clocks stuck well below their
+    maximum with no reason reported, send the main timed run round once more;
+    a power cap alone does not."""
+    import sys
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+    ok = {"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": []}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected({"sm_mhz": 1320.0, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]})
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected({"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": [r]})
+    assert bench.clocks_rejected({"sm_mhz": 1100.0, "sm_max_mhz": 1965, "reasons": []})  # a leftover clock lock
+    assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": []})  # no NVML: nothing to judge
