@@ -109,3 +109,64 @@ def test_binding_rejects_buffers_that_do_not_fit_the_state(lib):
     # a cache smaller than the configured capacity
     with pytest.raises(ValueError, match="elements"):
         mac.mac_attend(st, torch.zeros(B * 99 * Hkv * D, dtype=torch.int16), 16, None, 16, 16)
+
+
+def _state_of(**kw):
+    """A MacState carrying only a configuration (no device state), for the binding's checks."""
+    import kv_cache_reuse_b200 as mac
+    f = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=64, window=4, band=8, tau=0.1, rope_theta=1e4,
+             page_size=0, max_seq=100, max_pages_per_seq=0, num_pages=0, cut_mode=0, match_per_head=0, q_bf16=0,
+             ring_bf16=0)
+    f.update(kw)
+    st = mac.MacState.__new__(mac.MacState)
+    st.cfg = mac.MacConfig(*[f[name] for name, _ in mac.MacConfig._fields_])
+    st.handle = None
+    return st
+
+
+def test_binding_checks_follow_the_configuration(lib):
+    """The expected shapes and element types follow the state: per-head
+    matching reports a decision per query head, a bf16 query is bf16 bits, a
+    paged cache needs its block table, a warm start has a leading position
+    dimension; host arrays are accepted where host buffers are expected, raw
+    integer addresses pass unchecked, non-contiguous tensors are refused."""
+    import numpy as np
+    import torch
+    from kv_cache_reuse_b200 import _args
+    B, Hq, Hkv, D = 2, 8, 2, 64
+    q, p = torch.zeros(B, Hq, D), torch.zeros(B, dtype=torch.int32)
+    o, l = torch.zeros(B, Hq, D), torch.zeros(B, Hq)
+    # per-head matching: hit mask and match positions are [B][Hq]
+    ph = _state_of(match_per_head=1)
+    a = _args(ph, "cpu", q, p, p, o, l, torch.zeros(B, Hq, dtype=torch.uint8), torch.zeros(B, Hq, dtype=torch.int32))
+    assert all(isinstance(x, int) for x in a[:7])
+    with pytest.raises(ValueError, match="hit_mask"):
+        _args(ph, "cpu", q, p, p, o, l, torch.zeros(B, Hkv, dtype=torch.uint8))
+    # bf16 query input: bf16 bits (int16 / uint16 / bfloat16), not fp32
+    qb = _state_of(q_bf16=1)
+    for dt in (torch.int16, torch.bfloat16):
+        assert _args(qb, "cpu", torch.zeros(B, Hq, D, dtype=dt))[0]
+    with pytest.raises(ValueError, match="q_pre"):
+        _args(qb, "cpu", q)
+    # paged cache: the block table is [B][max_pages] int32 on the device
+    pg = _state_of(page_size=16, max_seq=0, max_pages_per_seq=5, num_pages=20)
+    with pytest.raises(ValueError, match="block_table: shape"):
+        _args(pg, "cuda", block_table=torch.zeros(B, 4, dtype=torch.int32))
+    with pytest.raises(ValueError, match="block_table: expected a device"):
+        _args(pg, "cuda", block_table=torch.zeros(B, 5, dtype=torch.int32))
+    with pytest.raises(ValueError, match="K: .*elements"):
+        _args(pg, "cuda", K=torch.zeros(20 * 16 * Hkv * D - 1, dtype=torch.int16))
+    # warm start: [n][B][Hq][D] queries, [n][B] positions and lengths
+    st = _state_of()
+    assert _args(st, "cpu", torch.zeros(3, B, Hq, D), torch.zeros(3, B, dtype=torch.int32), n=3)[0]
+    with pytest.raises(ValueError, match="q_pre"):
+        _args(st, "cpu", q, n=3)
+    # host arrays, raw addresses, contiguity
+    assert _args(st, "cpu", np.zeros((B, Hq, D), np.float32))[0]
+    with pytest.raises(ValueError, match="element type"):
+        _args(st, "cpu", np.zeros((B, Hq, D), np.float64))
+    with pytest.raises(ValueError, match="device buffer"):
+        _args(st, "cuda", np.zeros((B, Hq, D), np.float32))
+    assert _args(st, "cuda", 12345)[0] == 12345
+    with pytest.raises(ValueError, match="contiguous"):
+        _args(st, "cpu", torch.zeros(B, D, Hq).transpose(1, 2))
