@@ -16,7 +16,7 @@ def torch_dev():
     return torch, torch.device("cuda:0")
 
 
-class GpuRun:
+class DeviceRun:
     """One MacState plus device copies of a workload's cache."""
 
     def __init__(self, wl, cache, tau=None, band=None, window=None, K_dev=None, V_dev=None, tune=None, cut_mode=0,
@@ -70,7 +70,7 @@ def compare_stream(wl, stream, cache, steps=None, tau=None, band=None, window=No
     With q_bf16 the queries are rounded to bf16 first: the library reads the
     bits, the oracle their exact values."""
     T = stream.q.shape[0] if steps is None else steps
-    gpu = gpu or GpuRun(wl, cache, tau=tau, band=band, window=window, tune=tune, cut_mode=cut_mode,
+    gpu = gpu or DeviceRun(wl, cache, tau=tau, band=band, window=window, tune=tune, cut_mode=cut_mode,
                         per_head=per_head, q_bf16=q_bf16, ring_bf16=ring_bf16)
     orc = orc or oracle.Oracle.for_workload(wl, cache, tau=tau, band=band, W=window, cut_mode=cut_mode,
                                             per_head=per_head, ring_bf16=ring_bf16)

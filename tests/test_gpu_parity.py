@@ -9,7 +9,7 @@ import pytest
 import oracle
 import synth
 from tests.dense_ref import load_hand_example
-from tests.gpu_harness import LSE_TOL, OUT_TOL, GpuRun, compare_stream, torch_dev
+from tests.gpu_harness import LSE_TOL, OUT_TOL, DeviceRun, compare_stream, torch_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +21,7 @@ def test_hand_worked_example_on_gpu():
                         band=sh["band"], tau=sh["tau"], sigma=0.0, rope_theta=sh["rope_theta"], page_size=0,
                         hit_model=("iid", 0.0), seed=0)
     cache = synth.KVCache(K, V, None, sh["max_seq"], 0)
-    gpu = GpuRun(wl, cache)
+    gpu = DeviceRun(wl, cache)
     for st, q in zip(g["steps"], qs):
         out, lse, hit, mpos = gpu.step(q, np.array([st["rope_pos"]], np.int32), np.array([st["seq_len"]], np.int32))
         assert int(hit[0, 0]) == st["hit"] and int(mpos[0, 0]) == st["match_pos"]
@@ -85,8 +85,8 @@ def test_paged_equals_contiguous_bitwise():
         Vc[b, :n * ps] = paged.V[pages].reshape(n * ps, wl.Hkv, wl.D)
     contig = synth.KVCache(Kc, Vc, None, cap, 0)
     wc = wl.with_(page_size=0)
-    g1 = GpuRun(wl, paged)
-    g2 = GpuRun(wc, contig)
+    g1 = DeviceRun(wl, paged)
+    g2 = DeviceRun(wc, contig)
     for t in range(wl.steps):
         a = g1.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
         b = g2.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
@@ -111,7 +111,7 @@ def test_continuous_append_stream():
             pg = int(cache.block_table[b, pos // ps])
             Kd[pg, pos % ps] = 0x7FC0
             Vd[pg, pos % ps] = 0x7FC0
-    gpu = GpuRun(wl, cache, K_dev=Kd, V_dev=Vd)
+    gpu = DeviceRun(wl, cache, K_dev=Kd, V_dev=Vd)
     orc = oracle.Oracle.for_workload(wl, cache)
     knew = torch.empty((wl.B, wl.Hkv, wl.D), dtype=torch.int16, device=dev)
     vnew = torch.empty_like(knew)
@@ -155,11 +155,11 @@ def test_export_import_resumes_identically():
     import kv_cache_reuse_b200 as mac
     wl = synth.WORKLOADS["tiny"].with_(steps=30)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    a = GpuRun(wl, cache)
+    a = DeviceRun(wl, cache)
     for t in range(15):
         a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
     buf = a.st.export_state()
-    b = GpuRun(wl, cache)
+    b = DeviceRun(wl, cache)
     b.st.import_state(buf)
     for t in range(15, 30):
         x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
@@ -172,8 +172,8 @@ def test_host_entry_matches_device_entry():
     import kv_cache_reuse_b200 as mac
     wl = synth.WORKLOADS["tiny"].with_(steps=20)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    a = GpuRun(wl, cache)
-    b = GpuRun(wl, cache)
+    a = DeviceRun(wl, cache)
+    b = DeviceRun(wl, cache)
     torch = a.torch
     out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32).pin_memory()
     lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
@@ -201,8 +201,8 @@ def test_host_entry_append_recapture():
     cache = synth.kv_cache(wl, steps)
     torch, dev = torch_dev()
     pool = [torch.from_numpy(x.view(np.int16)).to(dev) for x in (cache.K, cache.V)]
-    a = GpuRun(wl, cache, K_dev=pool[0].clone(), V_dev=pool[1].clone())
-    b = GpuRun(wl, cache, K_dev=pool[0].clone(), V_dev=pool[1].clone())
+    a = DeviceRun(wl, cache, K_dev=pool[0].clone(), V_dev=pool[1].clone())
+    b = DeviceRun(wl, cache, K_dev=pool[0].clone(), V_dev=pool[1].clone())
     Kb2, Vb2 = b.K.clone(), b.V.clone()
     knew = torch.empty((wl.B, wl.Hkv, wl.D), dtype=torch.int16, device=dev)
     vnew = torch.empty_like(knew)
@@ -339,7 +339,7 @@ def test_threshold_is_strict_and_ties_pick_the_most_recent(G):
     q1[0, :, 3] += np.float32(0.5)
     far = (q0 + np.float32(3.0)).astype(np.float32)
     for tau, hit1 in ((0.25, 0), (float(np.nextafter(np.float32(0.25), np.float32(1.0))), 1)):
-        gpu = GpuRun(wl, cache, tau=tau)
+        gpu = DeviceRun(wl, cache, tau=tau)
         orc = oracle.Oracle.for_workload(wl, cache, tau=tau)
         for t, qt in enumerate([q0, q1, far, q0, q0]):
             r = orc.step(qt, stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
@@ -407,8 +407,8 @@ def test_bf16_host_entry_matches_device_entry():
     import kv_cache_reuse_b200 as mac
     wl = synth.WORKLOADS["tiny"].with_(steps=20)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    a = GpuRun(wl, cache, q_bf16=1, ring_bf16=1)
-    b = GpuRun(wl, cache, q_bf16=1, ring_bf16=1)
+    a = DeviceRun(wl, cache, q_bf16=1, ring_bf16=1)
+    b = DeviceRun(wl, cache, q_bf16=1, ring_bf16=1)
     torch = a.torch
     out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32).pin_memory()
     lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
@@ -442,8 +442,8 @@ def test_per_head_host_entry_matches_device_entry():
     import kv_cache_reuse_b200 as mac
     wl = synth.WORKLOADS["tiny"].with_(steps=20, head_labels=True)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    a = GpuRun(wl, cache, per_head=1)
-    b = GpuRun(wl, cache, per_head=1)
+    a = DeviceRun(wl, cache, per_head=1)
+    b = DeviceRun(wl, cache, per_head=1)
     torch = a.torch
     out_h = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.float32).pin_memory()
     lse_h = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
@@ -543,7 +543,7 @@ def test_warm_start_from_prefill_then_decode(case):
     if qb:  # the queries as bf16 values: the library reads their bits, the oracle their values
         stream = synth.QueryStream(q=synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(stream.q)), label=stream.label,
                                    src=stream.src, rope_pos=stream.rope_pos, seq_lens=stream.seq_lens)
-    gpu = GpuRun(wl, cache, per_head=ph, q_bf16=qb, ring_bf16=rb)
+    gpu = DeviceRun(wl, cache, per_head=ph, q_bf16=qb, ring_bf16=rb)
     orc = oracle.Oracle.for_workload(wl, cache, per_head=ph, ring_bf16=rb)
     torch = gpu.torch
     qh = synth.f32_to_bf16_bits(stream.q[:n]).view(np.int16) if qb else np.ascontiguousarray(stream.q[:n])
@@ -583,8 +583,8 @@ def test_graph_captured_multilayer_loop(opts):
     wls = [synth.WORKLOADS["tiny"].with_(steps=24, seed=10 + l, head_labels=bool(opts)) for l in range(L)]
     streams = [synth.queries(w) for w in wls]
     caches = [synth.kv_cache(w) for w in wls]
-    eager = [GpuRun(w, c, **opts) for w, c in zip(wls, caches)]
-    graph = [GpuRun(w, c, **opts) for w, c in zip(wls, caches)]
+    eager = [DeviceRun(w, c, **opts) for w, c in zip(wls, caches)]
+    graph = [DeviceRun(w, c, **opts) for w, c in zip(wls, caches)]
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
@@ -647,7 +647,7 @@ def test_bounded_wait_times_out_and_context_stays_usable():
 def test_nan_query_misses_and_stays_local():
     wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, L0=(700, 900), steps=6)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    gpu = GpuRun(wl, cache)
+    gpu = DeviceRun(wl, cache)
     for t in range(wl.steps):
         q = stream.q[t].copy()
         if t == 4:
@@ -669,7 +669,7 @@ def test_bad_page_and_seq_len_flagged():
     bt = cache.block_table.copy()
     bt[1, 2] = cache.num_pages + 5  # sequence 1 reads its page 2 at every step
     bad = synth.KVCache(cache.K, cache.V, bt, cache.max_seq, cache.num_pages)
-    gpu = GpuRun(wl, bad)
+    gpu = DeviceRun(wl, bad)
     out, lse, hit, mpos = gpu.step(stream.q[0], stream.rope_pos[0], stream.seq_lens[0])
     assert np.isnan(out[1]).all() and np.isnan(lse[1]).all()
     assert np.isfinite(out[0]).all() and np.isfinite(out[2]).all()

@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 
 import synth
-from tests.gpu_harness import LSE_TOL, OUT_TOL, GpuRun
+from tests.gpu_harness import LSE_TOL, OUT_TOL, DeviceRun
 
 
 def test_rejects_shapes_beyond_the_static_scratch():
@@ -43,7 +43,7 @@ def test_static_scratch_matches_regular_entry_on_two_calls(paged, Hq):
     base = synth.WORKLOADS["paged_mixed" if paged else "llama8b_32k"]
     wl = base.with_(B=3, L0=(5000, 3210, 777), steps=2, Hq=Hq)
     stream, cache = synth.queries(wl), synth.kv_cache(wl)
-    ref = GpuRun(wl, cache, tau=0.0)  # regular entry point, never hits: dense attention
+    ref = DeviceRun(wl, cache, tau=0.0)  # regular entry point, never hits: dense attention
     torch = ref.torch
     out = torch.empty_like(ref.out)
     lse = torch.empty_like(ref.lse)
