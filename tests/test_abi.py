@@ -170,3 +170,20 @@ def test_binding_checks_follow_the_configuration(lib):
     assert _args(st, "cuda", 12345)[0] == 12345
     with pytest.raises(ValueError, match="contiguous"):
         _args(st, "cpu", torch.zeros(B, D, Hq).transpose(1, 2))
+
+
+def test_config_struct_layout_matches_the_header(tmp_path):
+    """The binding's MacConfig has the C header's size and field offsets: a C
+    program built here from include/mac.h prints them (gcc, no GPU)."""
+    import ctypes
+    import subprocess
+    from kv_cache_reuse_b200._native import MacConfig
+    names = [n for n, _ in MacConfig._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include "mac.h"\nint main(void) {\n  printf("%zu\\n", sizeof(MacConfig));\n'
+                   + "".join('  printf("%%zu\\n", offsetof(MacConfig, %s));\n' % n for n in names) + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    vals = [int(x) for x in subprocess.check_output([str(exe)]).decode().split()]
+    assert vals[0] == ctypes.sizeof(MacConfig)
+    assert vals[1:] == [getattr(MacConfig, n).offset for n in names]
