@@ -187,3 +187,26 @@ def test_config_struct_layout_matches_the_header(tmp_path):
     vals = [int(x) for x in subprocess.check_output([str(exe)]).decode().split()]
     assert vals[0] == ctypes.sizeof(MacConfig)
     assert vals[1:] == [getattr(MacConfig, n).offset for n in names]
+
+
+def test_every_entry_point_is_documented_in_the_header():
+    """Each function include/mac.h declares comes with a comment (its own, or
+    the one heading the group of declarations it belongs to)."""
+    src = open(os.path.join(ROOT, "include", "mac.h")).read()
+    code = re.sub(r"/\*.*?\*/", lambda m: "\0" * len(m.group(0)), src, flags=re.S)  # keep offsets
+    decl = re.compile(r"^[A-Za-z_][\w \t\*]*\b(mac_[a-z_]+)\s*\(", re.M)
+    documented = {}
+    prev_end, prev_name = 0, None
+    for m in decl.finditer(code):
+        between = src[prev_end:m.start()]
+        has_comment = "*/" in between
+        blank_line = "\n\n" in between.replace("\0", "")
+        if has_comment:
+            documented[m.group(1)] = True
+        elif prev_name is not None and not blank_line:
+            documented[m.group(1)] = documented[prev_name]  # same group as the declaration above
+        else:
+            documented[m.group(1)] = False
+        prev_end, prev_name = code.index(";", m.end()) + 1, m.group(1)
+    assert len(documented) >= 15
+    assert all(documented.values()), sorted(n for n, ok in documented.items() if not ok)
