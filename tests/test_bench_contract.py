@@ -7,6 +7,8 @@ import socket
 import subprocess
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 ARGS = ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3", "--workload", "tiny"]
 
@@ -66,3 +68,27 @@ def test_clock_records_that_disqualify_a_timed_region():
         assert bench.clocks_rejected({"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": [r]})
     assert bench.clocks_rejected({"sm_mhz": 1100.0, "sm_max_mhz": 1965, "reasons": []})  # a leftover clock lock
     assert not bench.clocks_rejected({"sm_mhz": None, "sm_max_mhz": None, "reasons": []})  # no NVML: nothing to judge
+
+
+
+@pytest.mark.parametrize("per_head", [0, 1])
+def test_roofline_key_bytes_agree_with_the_oracles_key_count(per_head):
+    """The K/V bytes the roofline counts per step (2 x D x 2 bytes per key of
+    the union of each unit's fresh ranges, from the step's decisions) equal
+    the keys the oracle actually reads, on a stream with hits and misses."""
+    import sys
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+    import oracle
+    import synth
+    wl = synth.WORKLOADS["tiny"].with_(steps=40, head_labels=bool(per_head))
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    orc = oracle.Oracle.for_workload(wl, cache, per_head=per_head)
+    hits = 0
+    for t in range(wl.steps):
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+        _, _, kv = bench.step_bytes(wl, r.hit, r.match_pos, stream.seq_lens[t], min(t, wl.W))
+        assert kv == r.keys_read * 2 * wl.D * 2, t
+        hits += int(r.hit.sum())
+    assert 0 < hits < wl.steps * r.hit.size
