@@ -1,6 +1,8 @@
-"""The benchmark's reference arm -- the fp64 oracle timed on the host cores --
-keeps the one-JSON-line contract, alone and under torchrun (rank 0 alone runs
-and prints; the other ranks exit 0 without work).  Both run on CPU."""
+"""The benchmark's host-side logic, on CPU: the reference arm -- the fp64
+oracle timed on the host cores -- keeps the one-JSON-line contract, alone and
+under torchrun (rank 0 alone runs and prints; the other ranks exit 0 without
+work); the rule that sends a timed run round again on a bad clock record; and
+the roofline's byte accounting against the keys the oracle reads."""
 import json
 import os
 import socket
