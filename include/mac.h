@@ -15,7 +15,7 @@
  *
  * Conventions used by every entry point
  *   - Group: each KV head serves G = num_q_heads / num_kv_heads query heads
- *     (GQA, page 1 "composes with ... MQA/GQA"); G may be 1 (multi-head
+ *     (GQA; page 1 states that the method works with MQA and GQA); G may be 1 (multi-head
  *     attention) up to 8.  Larger groups (MQA with more than 8 query heads
  *     per KV head) return MAC_ERR_SHAPE.  One match decision is taken per
  *     (sequence, KV head) over its G heads.

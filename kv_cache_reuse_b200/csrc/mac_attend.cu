@@ -2,10 +2,10 @@
 //
 // "MAC-Attention: a Match-Amend-Complete Scheme for Fast and Accurate
 // Attention Computation", page 1 (abstract): on a hit the amend stage
-// "rectifies the reused attention by recomputing a small band near the match
-// boundary" and the complete stage "fuses the rectified results with fresh
-// attention computed on the KV tail through a numerically stable merge"; on
-// a miss the step is split-KV decode attention over every key.  All three are
+// corrects the reused attention by recomputing a small band of keys next to
+// the match boundary, and the complete stage combines that result with fresh
+// attention over the KV tail in a numerically stable merge; on a miss the
+// step is split-KV decode attention over every key.  All three are
 // the same computation -- attention of the current query group over a key
 // range -- so one persistent kernel runs them over a flattened list of work
 // items built by the match kernel.  A unit (sequence, KV head) with few fresh

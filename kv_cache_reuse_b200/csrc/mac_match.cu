@@ -1,9 +1,9 @@
 // mac_match.cu -- Match stage of MAC-Attention and the step's work plan.
 //
 // "MAC-Attention: a Match-Amend-Complete Scheme for Fast and Accurate
-// Attention Computation", page 1 (abstract): the match stage "performs
-// pre-RoPE L2 matching over a short local window" of recent queries whose
-// attention results can be reused.  One CTA handles one (sequence, KV head)
+// Attention Computation", page 1 (abstract): the match stage compares the
+// current query, before RoPE, by L2 distance with a short window of recent
+// queries whose attention results can be reused.  One CTA handles one (sequence, KV head)
 // unit:
 //   1. distance of the current pre-RoPE query group (G heads) to every
 //      window entry: mean over heads of the squared L2 distance, summed in

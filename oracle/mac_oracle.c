@@ -9,12 +9,13 @@
  * Source: "MAC-Attention: a Match-Amend-Complete Scheme for Fast and Accurate
  * Attention Computation", page 1 (the abstract).  The abstract names three
  * stages and every function below cites the part it follows:
- *   Match    -- "pre-RoPE L2 matching over a short local window" of recent
- *               queries, whose prior attention computations are reused;
- *   Amend    -- the reused attention is rectified by recomputing "a small
- *               band near the match boundary";
- *   Complete -- fresh attention over the KV tail is fused with the rectified
- *               result "through a numerically stable merge".
+ *   Match    -- the current query is compared, before RoPE, by L2 distance
+ *               with a short window of recent queries whose attention results
+ *               can be reused;
+ *   Amend    -- the reused attention is corrected by recomputing a small band
+ *               of keys just before the match boundary;
+ *   Complete -- fresh attention over the KV tail is combined with the
+ *               corrected result by a numerically stable merge.
  * On a miss the step is plain decode attention over every key.
  *
  * Where the abstract is silent this file takes the plainest reading; each
@@ -126,7 +127,7 @@ static const uint16_t *kv_row(const ocfg_t *c, const uint16_t *base, const int *
 
 /* [rope] Rotate a pre-RoPE query to position pos.  Pair i couples element i
  * with element i + D/2 and turns by pos * theta^(-2i/D) radians.  The match
- * stage uses the unrotated query ("pre-RoPE L2 matching", page 1); attention
+ * stage uses the unrotated query (page 1: the match compares queries before RoPE); attention
  * uses the rotated one, since the cache holds rotated keys. */
 void oracle_rope(const float *q, int D, long pos, double theta, double *out) {
     int half = D / 2;
@@ -188,7 +189,7 @@ void oracle_partial(const double *qrot, const uint16_t *K, const uint16_t *V, in
     partial_view(&c, K, V, NULL, 0, 0, qrot, x, y, o, m, l);
 }
 
-/* "numerically stable merge" (page 1, complete stage): combine two states of
+/* Stable merge (page 1, complete stage): combine two states of
  * disjoint key ranges.  Each side's weight is l_i * exp(m_i - M) with M the
  * larger max, so no exponent is positive.  The empty state is the identity. */
 void oracle_merge(const double *o1, double m1, double l1, const double *o2, double m2, double l2,
