@@ -177,6 +177,14 @@ def rank_workload(args, rank):
     return base, base.with_(seed=base.seed + 1000 * rank)
 
 
+def bench_config(wl, paged: bool, world: int) -> dict:
+    """The workload description both arms print (same keys, same values)."""
+    return {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.D,
+            "context": int(wl.L0[0]), "window": wl.W, "band": wl.band, "tau": wl.tau,
+            "hit_label_rate": wl.hit_model[1], "kv": "bf16 %s" % ("paged" if paged else "contiguous"),
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas" if world > 1 else "1 GPU"}
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """Largest value of x over the ranks (the job's time is its slowest rank's)."""
     if world <= 1:
@@ -342,7 +350,8 @@ def run_mac(args, rank, world, local_rank):
         # the hit path alone: the same shape with every labelled step a near-repeat
         qh = synth.queries(wl.with_(hit_model=("iid", 1.0)), T).q
         cur["q"] = torch.from_numpy(qh).to(dev)
-        hitrun = timed_run(wl.tau, 3, min(args.hit_steps, T - 3), split=True)
+        # the windows filled first (W untimed steps), so every timed step scans a full window
+        hitrun = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=True)
         cur["q"] = q_all
         if not cache.paged:
             # the same hit stream at shorter contexts, on the same cache: a hit's
@@ -351,7 +360,7 @@ def run_mac(args, rank, world, local_rank):
                 sc = synth.queries(wl.with_(hit_model=("iid", 1.0), L0=(L,) * B), T)
                 cur.update(q=torch.from_numpy(sc.q).to(dev), pos=torch.from_numpy(sc.rope_pos).to(dev),
                            lens=torch.from_numpy(sc.seq_lens).to(dev), stream=sc)
-                r = timed_run(wl.tau, 3, min(args.hit_steps, T - 3), split=True)
+                r = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=True)
                 hitctx.append((L, r))
             cur.update(q=q_all, pos=pos_all, lens=lens_all, stream=stream)
             hitctx.append((int(wl.L0[0]), hitrun))
@@ -375,6 +384,10 @@ def run_mac(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(wl, stream, cache, args.cpu_seconds)
 
+    hitshapes = []
+    if args.hit_steps > 0 and args.hit_shapes:
+        hitshapes = [run_hit_shape(n, args.hit_steps, dev, peak, world) for n in args.hit_shapes.split(",") if n]
+
     if rank != 0:
         return None
     K_ = args.steps
@@ -382,51 +395,70 @@ def run_mac(args, rank, world, local_rank):
     ratio = _profiled_traffic()
     # traffic per launch: the profiled DRAM/algorithmic ratio scaled to this run's launches
     traffic = ratio * kern["att_bytes"] / K_ if ratio else None
+    occ = [min(t, wl.W) for t in range(args.warmup, args.warmup + K_)]
+    roof = {"bound": "hbm", "kernel": "mac_attend_kernel", "achieved": att_gbs, "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": att_gbs / peak, "traffic": traffic,
+            "bytes_per_launch": kern["att_bytes"] / K_, "us_per_launch": kern["att_ms"] * 1e3 / K_}
+    detail = {}
+    if allmiss:
+        n = len(allmiss["step_ms"])
+        a_gbs = allmiss["att_bytes"] / (allmiss["att_ms"] * 1e-3) / 1e9
+        roof["miss"] = {"kernel": "mac_attend_kernel", "workload": "%s, threshold 0 (every unit misses)" % wl.name,
+                        "achieved": a_gbs, "frac": a_gbs / peak, "mb_per_launch": allmiss["att_bytes"] / n / 1e6,
+                        "us_per_launch": allmiss["att_ms"] * 1e3 / n, "steps_per_s": n / (allmiss["total_ms"] * 1e-3)}
+        detail["all_miss"] = {"steps": n, "ms_per_step": allmiss["total_ms"] / n,
+                              "speedup_of_mac": (world * K_ / (tot * 1e-3)) / (n / (allmiss["total_ms"] * 1e-3)),
+                              "clocks": allmiss["clocks"]}
+    if hitrun:
+        n = len(hitrun["step_ms"])
+        h_gbs = hitrun["att_bytes"] / (hitrun["att_ms"] * 1e-3) / 1e9
+        m_gbs = hitrun["match_bytes"] / (hitrun["match_ms"] * 1e-3) / 1e9
+        roof["hit"] = {
+            "kernel": "mac_attend_kernel", "workload": "%s, every step a repeat" % wl.name,
+            "achieved": h_gbs, "frac": h_gbs / peak, "mb_per_launch": hitrun["att_bytes"] / n / 1e6,
+            "us_per_launch": hitrun["att_ms"] * 1e3 / n,
+            "match": {"kernel": "mac_match_kernel", "achieved": m_gbs, "frac": m_gbs / peak,
+                      "mb_per_launch": hitrun["match_bytes"] / n / 1e6, "us_per_launch": hitrun["match_ms"] * 1e3 / n},
+            "step_us": hitrun["total_ms"] * 1e3 / n, "hit_fraction": hitrun["hit_frac"],
+            "larger": [{"workload": h["workload"], "attend_frac": h["attend"]["frac"],
+                        "attend_us": h["attend"]["us_per_launch"], "attend_mb": h["attend"]["mb_per_launch"],
+                        "match_frac": h["match"]["frac"], "match_us": h["match"]["us_per_launch"],
+                        "step_us": h["step"]["us"], "step_frac": h["step"]["frac"]} for h in hitshapes]}
+        detail["hit_path"] = {"steps": n, "clocks": hitrun["clocks"], "shapes": hitshapes}
+        if hitctx:
+            roof["hit"]["vs_context"] = [
+                {"context": L, "step_us": r["total_ms"] * 1e3 / len(r["step_ms"]),
+                 "attend_mb": r["att_bytes"] / len(r["step_ms"]) / 1e6} for L, r in hitctx]
     res = {
         "metric": METRIC, "value": world * K_ / (tot * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K_,
         "warmup": args.warmup, "ms_per_step": tot / K_, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.D,
-                   "context": int(wl.L0[0]), "window": wl.W, "band": wl.band, "tau": wl.tau,
-                   "hit_label_rate": wl.hit_model[1], "kv": "bf16 %s" % ("paged" if cache.paged else "contiguous"),
-                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas" if world > 1 else "1 GPU"},
-        "roofline": {"bound": "hbm", "kernel": "mac_attend_kernel", "achieved": att_gbs, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": att_gbs / peak,
-                     "traffic": traffic},
+        "config": bench_config(wl, cache.paged, world),
+        "roofline": roof,
         "hit_fraction": main["hit_frac"],
+        "window_occupancy": {"mean": float(np.mean(occ)), "min": int(min(occ)), "max": int(max(occ)),
+                             "window": wl.W},
+        "gpu_launches": 2 * K_ * world,
+        "clocks": main["clocks"],
+        "device_status": main["status"],
+    }
+    if layers:
+        res["layer_stack"] = {k: layers[k] for k in ("layers", "us_per_layer", "tokens_per_s", "hit_fraction",
+                                                    "device_status")}
+        detail["layer_stack"] = layers
+    if e2e:
+        res["e2e"] = e2e
+    if cpu:
+        res["cpu_baseline"] = cpu
+    detail.update({
         "match_kernel_gbs": kern["match_bytes"] / (kern["match_ms"] * 1e-3) / 1e9,
         "kernel_ms_per_step": {"match": kern["match_ms"] / K_, "attend": kern["att_ms"] / K_,
                                "timed_separately": kern["total_ms"] / K_},
         "step_gbs": (main["att_bytes"] + main["match_bytes"]) / (main["total_ms"] * 1e-3) / 1e9,
         "effective_kv_gbs": main["dense_bytes"] / (main["total_ms"] * 1e-3) / 1e9,
         "kv_bytes_per_step": main["kv_bytes"] / K_, "dense_kv_bytes_per_step": main["dense_bytes"] / K_,
-        "gpu_launches": 2 * K_ * world,
         "timing": "CUDA events around each step on the launching stream; steps queued behind a GPU sleep so host "
-                  "latency is excluded; roofline from a second timed pass with events between the two kernels",
-        "clocks": main["clocks"],
-        "device_status": main["status"],
-    }
-    if allmiss:
-        n = len(allmiss["step_ms"])
-        a_gbs = allmiss["att_bytes"] / (allmiss["att_ms"] * 1e-3) / 1e9
-        res["all_miss"] = {"steps": n, "steps_per_s": n / (allmiss["total_ms"] * 1e-3),
-                           "ms_per_step": allmiss["total_ms"] / n, "attend_gbs": a_gbs, "attend_frac": a_gbs / peak,
-                           "speedup_of_mac": (world * K_ / (tot * 1e-3)) / (n / (allmiss["total_ms"] * 1e-3)),
-                           "clocks": allmiss["clocks"]}
-    if hitrun:
-        n = len(hitrun["step_ms"])
-        h_gbs = hitrun["att_bytes"] / (hitrun["att_ms"] * 1e-3) / 1e9
-        res["hit_path"] = {"steps": n, "hit_fraction": hitrun["hit_frac"],
-                           "steps_per_s": n / (hitrun["total_ms"] * 1e-3), "ms_per_step": hitrun["total_ms"] / n,
-                           "match_ms_per_step": hitrun["match_ms"] / n, "attend_ms_per_step": hitrun["att_ms"] / n,
-                           "attend_bytes_per_step": hitrun["att_bytes"] / n, "attend_gbs": h_gbs,
-                           "attend_frac": h_gbs / peak, "clocks": hitrun["clocks"],
-                           "note": "latency-bound: a few MB per launch"}
-        if hitctx:
-            res["hit_path"]["vs_context"] = [
-                {"context": L, "steps_per_s": len(r["step_ms"]) / (r["total_ms"] * 1e-3),
-                 "ms_per_step": r["total_ms"] / len(r["step_ms"]), "hit_fraction": r["hit_frac"],
-                 "attend_bytes_per_step": r["att_bytes"] / len(r["step_ms"])} for L, r in hitctx]
+                  "latency is excluded; roofline from a second timed pass with events between the two kernels"})
     for name, pair, what in (("bf16_window", bf16, {"q": "bf16", "window_q_and_o": "bf16"}),
                              ("per_head", perhead, {"matching": "per query head",
                                                     "stream": "each query head repeats a recent query of its own "
@@ -435,7 +467,7 @@ def run_mac(args, rank, world, local_rank):
             continue
         run, kr = pair
         a_gbs = kr["att_bytes"] / (kr["att_ms"] * 1e-3) / 1e9
-        res[name] = dict(what, **{
+        detail[name] = dict(what, **{
             "steps_per_s": K_ / (run["total_ms"] * 1e-3), "ms_per_step": run["total_ms"] / K_,
             "vs_headline": (K_ / (run["total_ms"] * 1e-3)) / (world * K_ / (tot * 1e-3)),
             "hit_fraction": run["hit_frac"], "match_ms_per_step": kr["match_ms"] / K_,
@@ -444,16 +476,83 @@ def run_mac(args, rank, world, local_rank):
             "match_gbs": kr["match_bytes"] / (kr["match_ms"] * 1e-3) / 1e9,
             "clocks": run["clocks"], "device_status": run["status"]})
     if quality:
-        res["approximation_vs_dense"] = quality
+        detail["approximation_vs_dense"] = quality
     if warm:
-        res["warm_start"] = warm
-    if layers:
-        res["layer_stack"] = layers
-    if e2e:
-        res["e2e"] = e2e
-    if cpu:
-        res["cpu_baseline"] = cpu
-    return res
+        detail["warm_start"] = warm
+    res["detail"] = "full record on stderr (one JSON line)"
+    return res, detail
+
+
+def run_hit_shape(name, nsteps, dev, peak, world):
+    """The hit path alone on another workload's shape (every labelled step a
+    near-repeat of a recent query), with the windows filled first: the window
+    length of untimed steps, then nsteps steps timed with events before, between
+    and after the two kernels.  K/V values do not change the work of a step,
+    so the cache is drawn on the device (seeded N(0, 1), bf16) in the
+    workload's layout instead of on the host."""
+    import torch
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS[name].with_(hit_model=("iid", 1.0))
+    nwarm = wl.W
+    T = nwarm + nsteps
+    stream = synth.queries(wl, T)
+    bt_h, max_seq, P = synth.kv_layout(wl, T)
+    shape = (wl.B, max_seq, wl.Hkv, wl.D) if bt_h is None else (P, wl.page_size, wl.Hkv, wl.D)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    K = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16).view(torch.int16)
+    V = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16).view(torch.int16)
+    bt = None if bt_h is None else torch.from_numpy(bt_h).to(dev)
+    kw = dict(capacity=max_seq) if bt_h is None else dict(max_pages_per_seq=bt_h.shape[1], num_pages=P)
+    st = mac.MacState.for_workload(wl, **kw)
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    q = torch.from_numpy(stream.q).to(dev)
+    pos = torch.from_numpy(stream.rope_pos).to(dev)
+    lens = torch.from_numpy(stream.seq_lens).to(dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    hit = torch.zeros((T, B, Hkv), dtype=torch.uint8, device=dev)
+    mpos = torch.zeros((T, B, Hkv), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    s = torch.cuda.current_stream(dev)
+    for t in range(nwarm):
+        st.decode_step(q[t], pos[t], K, V, bt, lens[t], out, lse, hit[t], mpos[t])
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
+    h, sp = st.handle, s.cuda_stream
+    btp = bt.data_ptr() if bt is not None else None
+    torch.cuda._sleep(int(2e6 + 4e5 * nsteps))
+    for i in range(nsteps):
+        t = nwarm + i
+        ev[i][0].record(s)
+        mac.mac_match(h, q[t].data_ptr(), pos[t].data_ptr(), btp, lens[t].data_ptr(), out.data_ptr(),
+                      lse.data_ptr(), hit[t].data_ptr(), mpos[t].data_ptr(), sp)
+        ev[i][1].record(s)
+        mac.mac_attend(h, K.data_ptr(), V.data_ptr(), btp, out.data_ptr(), lse.data_ptr(), sp)
+        ev[i][2].record(s)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    status = st.get_status()
+    st.close()
+    hits = hit.cpu().numpy()[nwarm:]
+    mps = mpos.cpu().numpy()[nwarm:]
+    mt = at = kv = 0
+    for i in range(nsteps):
+        a, b_, c = step_bytes(wl, hits[i], mps[i], stream.seq_lens[nwarm + i], min(nwarm + i, wl.W))
+        mt, at, kv = mt + a, at + b_, kv + c
+    m_ms = float(sum(e[0].elapsed_time(e[1]) for e in ev))
+    a_ms = float(sum(e[1].elapsed_time(e[2]) for e in ev))
+    step_ms = float(sum(e[0].elapsed_time(e[2]) for e in ev))
+    return {"workload": "%s shape, every step a repeat" % name, "batch": B, "window": wl.W, "band": wl.band,
+            "paged": bt_h is not None, "steps": nsteps, "hit_fraction": float(hits.mean()),
+            "attend": {"mb_per_launch": at / nsteps / 1e6, "us_per_launch": a_ms * 1e3 / nsteps,
+                       "achieved": at / (a_ms * 1e-3) / 1e9, "frac": at / (a_ms * 1e-3) / 1e9 / peak},
+            "match": {"mb_per_launch": mt / nsteps / 1e6, "us_per_launch": m_ms * 1e3 / nsteps,
+                      "achieved": mt / (m_ms * 1e-3) / 1e9, "frac": mt / (m_ms * 1e-3) / 1e9 / peak},
+            "step": {"us": step_ms * 1e3 / nsteps, "mb": (mt + at) / nsteps / 1e6,
+                     "frac": (mt + at) / (step_ms * 1e-3) / 1e9 / peak},
+            "device_status": status}
 
 
 def run_quality(args, wl, stream, K, V, bt, kw, dev, identity_rope=False):
@@ -669,8 +768,7 @@ def run_reference(args, rank, world):
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": n,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / n, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.D,
-                       "context": int(wl.L0[0]), "window": wl.W, "band": wl.band},
+            "config": bench_config(wl, cache.paged, world),
             "cpu_baseline": {"value": v, "unit": UNIT, "kind": "oracle", "cores": oracle.num_threads(),
                              "sample": sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -686,8 +784,10 @@ def main():
     ap.add_argument("--miss-steps", type=int, default=16, help="timed steps of the all-miss run (0 = skip)")
     ap.add_argument("--hit-steps", type=int, default=16, help="timed steps of the all-hit run (0 = skip)")
     ap.add_argument("--warm-start", action="store_true", help="also time seeding the windows from W positions")
-    ap.add_argument("--layers", type=int, default=0,
-                    help="also time a stack of this many layers per token, one CUDA graph per token")
+    ap.add_argument("--layers", type=int, default=4,
+                    help="also time a stack of this many layers per token, one CUDA graph per token (0 = skip)")
+    ap.add_argument("--hit-shapes", default="paged_mixed,continuous_16k",
+                    help="workloads whose shapes also get an all-hit run (comma-separated, empty = none)")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 query / window run")
     ap.add_argument("--no-per-head", action="store_true", help="skip the per-head matching run")
     ap.add_argument("--no-quality", action="store_true", help="skip the approximation-error pass")
@@ -718,6 +818,9 @@ def main():
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
     if res is not None:
+        if isinstance(res, tuple):
+            res, detail = res
+            print(json.dumps(dict(detail, metric=res["metric"], value=res["value"])), file=sys.stderr, flush=True)
         print(json.dumps(res), flush=True)
 
 

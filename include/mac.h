@@ -137,7 +137,13 @@ int mac_reset_seq(MacState *st, int b, void *stream);
  * The window of every unit advances by one entry.  Enqueues two kernels and
  * nothing else (no allocation, no host synchronisation), so the call can be
  * recorded into a CUDA graph -- e.g. one graph per token over all layers'
- * states -- and replayed; the recording holds the K/V addresses it saw. */
+ * states -- and replayed; the recording holds the K/V addresses it saw.
+ * Reproducibility: hit/miss decisions never depend on the work split, but
+ * on large steps (at least 4096 keys of work per SM) the split learns each
+ * SM's streaming rate from earlier steps by default, so the order in which
+ * partial results are merged -- and with it the last bits of out and lse --
+ * depends on the state's history and on the GPU.  mac_set_reproducible
+ * turns the learning off: the same inputs then give the same bits. */
 int mac_decode_step(MacState *st, const void *q_pre, const int *rope_pos, const uint16_t *K,
                     const uint16_t *V, const int *block_table, const int *seq_lens, float *out,
                     float *lse, uint8_t *hit_mask, int *match_pos, void *stream);
@@ -235,6 +241,14 @@ int mac_set_piece_cost(MacState *st, int keys);
  * range. */
 int mac_set_whole_unit_keys(MacState *st, int keys);
 
+/* Reproducible work split.  on = 1: every step splits the key ranges evenly
+ * over the CTAs and no streaming rate is learned or used, so a step's out and
+ * lse depend only on its inputs and the window (bit for bit, on any B200);
+ * on = 0 (default): large steps size each SM's range by its learned rate
+ * (faster all-miss steps, history-dependent rounding).  MAC_ERR_ARG for a
+ * NULL state or another value. */
+int mac_set_reproducible(MacState *st, int on);
+
 /* Persistent grid size of the attention kernel (CTAs). */
 int mac_attend_grid(const MacState *st);
 
@@ -252,7 +266,8 @@ int mac_attend_grid(const MacState *st);
  *       mac_decode_step (device pointers, caller-owned, 16-byte aligned
  *       q_pre, K, V).
  *   device_status: device uint32 receiving MAC_DEV_* bits (OR-ed in, not
- *       cleared), or NULL to use a word inside the static scratch.
+ *       cleared); required (NULL returns MAC_ERR_ARG), since it is the only
+ *       way a bad sequence length or page id reaches the caller.
  *   batch .. num_pages: shapes as in MacConfig.
  * Limits: batch * num_kv_heads <= 64, batch * num_q_heads <= 256, head_dim
  * 64 or 128, Hq / Hkv an integer from 1 to 8; other shapes return
@@ -262,7 +277,9 @@ int mac_attend_grid(const MacState *st);
  * device looks up the array's device address and sets kernel attributes
  * (make that first call before any stream capture); a call whose
  * rope_theta or head_dim differs from the previous call's uploads 512 bytes
- * of inverse frequencies from host memory.  Every call shares the one array
+ * of inverse frequencies from host memory, which cannot happen inside a
+ * stream capture: such a call on a capturing stream returns MAC_ERR_ARG
+ * (make the first call with new frequencies outside the capture).  Every call shares the one array
  * and finds it as the previous call left it; the call clears the counters
  * that must start at zero.  Two calls whose kernels overlap on the GPU (on
  * different streams, or on the same device from different threads without

@@ -311,6 +311,10 @@ def mac_set_whole_unit_keys(st, keys: int) -> None:
     check("mac_set_whole_unit_keys", load().mac_set_whole_unit_keys(_h(st), int(keys)))
 
 
+def mac_set_reproducible(st, on: int) -> None:
+    check("mac_set_reproducible", load().mac_set_reproducible(_h(st), int(on)))
+
+
 def mac_attend_grid(st) -> int:
     return int(load().mac_attend_grid(_h(st)))
 

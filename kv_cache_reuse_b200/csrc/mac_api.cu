@@ -20,6 +20,7 @@ struct MacState {
   MacConfig cfg;
   int G, U, D, W, device, num_sms, grid, min_keys, piece_cost, unit_max, capacity;
   int ND;  // match decisions per unit: 1, or G with per-head matching
+  int reproducible = 0;  // 1: even split on every step, no learned rates
   int QES, RES;  // bytes of a query element (input) and of a window q / o element
   size_t max_parts;
   // ring (library-owned state)
@@ -354,6 +355,13 @@ int mac_set_whole_unit_keys(MacState* s, int keys) {
   return MAC_OK;
 }
 
+int mac_set_reproducible(MacState* s, int on) {
+  if (!s || on < 0 || on > 1) return MAC_ERR_ARG;
+  s->reproducible = on;
+  drop_graph(s);
+  return MAC_OK;
+}
+
 int mac_attend_grid(const MacState* s) { return s ? s->grid : 0; }
 
 static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope_pos, const int* block_table,
@@ -391,7 +399,7 @@ static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope
   p.seg = s->seg;
   p.hdr = s->hdr;
   p.first_seg = s->first_seg;
-  p.cw = s->cw;
+  p.cw = s->reproducible ? nullptr : s->cw;  // null: the even split on every step
   p.bounds = s->bounds;
   p.claim = s->claim;
   p.done = s->done;
@@ -443,8 +451,8 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.first_seg = s->first_seg;
   p.bounds = s->bounds;
   p.claim = s->claim;
-  p.rate = s->rate;
-  p.cw = s->cw;
+  p.rate = s->reproducible ? nullptr : s->rate;  // null: no rate is learned
+  p.cw = s->reproducible ? nullptr : s->cw;
   p.part = s->part;
   p.unit_cnt = s->unit_cnt;
   p.ring_o = s->ring_o;

@@ -46,7 +46,7 @@ constexpr size_t kOffHdr = align256(kOffSeg + 2 * kMaxUnits * sizeof(Segment));
 constexpr size_t kOffFirst = align256(kOffHdr + sizeof(PlanHeader));
 constexpr size_t kOffPart = align256(kOffFirst + kMaxCtas * 4);
 constexpr size_t kOffCnt = align256(kOffPart + (size_t)(kMaxCtas + 2 * kMaxUnits) * kPartFloats * 4);
-// counters block, cleared on every call: unit_cnt[kMaxUnits], done, status, steps[kMaxUnits]
+// counters block, cleared on every call: unit_cnt[kMaxUnits], done, (unused), steps[kMaxUnits]
 constexpr size_t kCntBytes = (2 * kMaxUnits + 2) * 4;
 constexpr size_t kOffInv = align256(kOffCnt + kCntBytes);
 constexpr size_t kOffRingQ = align256(kOffInv + (kMaxD / 2) * 8);
@@ -74,16 +74,13 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// cuTensorMapEncodeTiled, looked up once under g_mutex (by the first call's
+// per-device set-up) and only read afterwards.
+EncodeTiledFn g_encode = nullptr;
+
 int encode_map(CUtensorMap* map, const void* base, int D, int Hkv, int rows, int outer) {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return MAC_ERR_CUDA;
-    fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+  const EncodeTiledFn fn = g_encode;
+  if (!fn) return MAC_ERR_CUDA;
   const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows, (cuuint64_t)outer};
   const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2, (cuuint64_t)rows * Hkv * D * 2};
   const cuuint32_t box[4] = {64u, 1u, (cuuint32_t)kSubKeys, 1u};
@@ -104,7 +101,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
                                        int num_kv_heads, int head_dim, double rope_theta, int page_size,
                                        int max_seq, int max_pages_per_seq, int num_pages, void* stream) {
   // --- host-side checks: nothing is enqueued on failure
-  if (!q_pre || !rope_pos || !K || !V || !seq_lens || !out || !lse) return MAC_ERR_ARG;
+  if (!q_pre || !rope_pos || !K || !V || !seq_lens || !out || !lse || !device_status) return MAC_ERR_ARG;
   if (!aligned16(q_pre) || !aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
   if (batch < 1 || num_kv_heads < 1 || num_q_heads < 1 || !(rope_theta > 0.0)) return MAC_ERR_ARG;
   if (num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads > kMaxGroup) return MAC_ERR_SHAPE;
@@ -127,6 +124,14 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!ds->ready) {
+      if (!g_encode) {
+        void* fp = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fp)
+          return MAC_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fp);
+      }
       void* ptr = nullptr;
       if (cudaGetSymbolAddress(&ptr, g_mac_static_scratch) != cudaSuccess || !ptr) return MAC_ERR_CUDA;
       int sms = 0;
@@ -140,6 +145,11 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
       ds->ready = true;
     }
     if (ds->inv_D != head_dim || ds->inv_theta != rope_theta) {
+      // the upload reads a host array on this stack: it cannot be recorded
+      // into a stream capture, so a change of frequencies during one is refused
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return MAC_ERR_CUDA;
+      if (cs != cudaStreamCaptureStatusNone) return MAC_ERR_ARG;
       double inv[kMaxD / 2];
       for (int i = 0; i < head_dim / 2; ++i) inv[i] = pow(rope_theta, -2.0 * (double)i / (double)head_dim);
       // pageable source: the copy is complete when the call returns
@@ -154,7 +164,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   const int U = batch * num_kv_heads;
   const int grid = ds->num_sms < kMaxCtas ? ds->num_sms : kMaxCtas;
   int* cnt = reinterpret_cast<int*>(base + kOffCnt);
-  unsigned* status = device_status ? device_status : reinterpret_cast<unsigned*>(cnt + kMaxUnits + 1);
+  unsigned* status = device_status;
   // counters start at zero on every call (the previous call's values persist)
   if (cudaMemsetAsync(cnt, 0, kCntBytes, st) != cudaSuccess) return MAC_ERR_CUDA;
 

@@ -274,15 +274,22 @@ def kv_cache(wl: Workload, steps: Optional[int] = None) -> KVCache:
     owns ceil((L0_b + steps) / page) pages, assigned from a shared pool by a
     random permutation.
     """
+    bt, max_seq, P = kv_layout(wl, steps)
+    shape = (wl.B, max_seq, wl.Hkv, wl.D) if bt is None else (P, wl.page_size, wl.Hkv, wl.D)
+    K = np.empty(shape, np.uint16)
+    V = np.empty(shape, np.uint16)
+    _fill_normal_bf16(K, wl.seed, _TAG_K)
+    _fill_normal_bf16(V, wl.seed, _TAG_V)
+    return KVCache(K, V, bt, max_seq, P)
+
+
+def kv_layout(wl: Workload, steps: Optional[int] = None):
+    """The cache's layout alone: (block_table or None, per-sequence capacity,
+    pages in the pool (0 when contiguous)), as kv_cache lays it out."""
     T = wl.steps if steps is None else steps
     cap = wl.capacity(T)
     if wl.page_size == 0:
-        shape = (wl.B, cap, wl.Hkv, wl.D)
-        K = np.empty(shape, np.uint16)
-        V = np.empty(shape, np.uint16)
-        _fill_normal_bf16(K, wl.seed, _TAG_K)
-        _fill_normal_bf16(V, wl.seed, _TAG_V)
-        return KVCache(K, V, None, cap, 0)
+        return None, cap, 0
     ps = wl.page_size
     npages = [-(-(l0 + T) // ps) for l0 in wl.L0]
     P = int(sum(npages))
@@ -294,12 +301,7 @@ def kv_cache(wl: Workload, steps: Optional[int] = None) -> KVCache:
     for b, n in enumerate(npages):
         bt[b, :n] = perm[off:off + n]
         off += n
-    shape = (P, ps, wl.Hkv, wl.D)
-    K = np.empty(shape, np.uint16)
-    V = np.empty(shape, np.uint16)
-    _fill_normal_bf16(K, wl.seed, _TAG_K)
-    _fill_normal_bf16(V, wl.seed, _TAG_V)
-    return KVCache(K, V, bt, maxp * ps, P)
+    return bt, maxp * ps, P
 
 
 def kv_row(cache: KVCache, b: int, pos: int) -> Tuple[np.ndarray, np.ndarray]:

@@ -55,7 +55,8 @@ def test_missing_library_fails_loudly(tmp_path):
 def test_tuning_setters_reject_bad_handles(lib):
     """Every setter validates its arguments on the host (NULL state -> MAC_ERR_ARG)."""
     import kv_cache_reuse_b200 as mac
-    for name in ("mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_set_whole_unit_keys"):
+    for name in ("mac_set_min_keys_per_cta", "mac_set_piece_cost", "mac_set_whole_unit_keys",
+                 "mac_set_reproducible"):
         with pytest.raises(mac.MacError) as e:
             getattr(mac, name)(None, 4)
         assert e.value.code == mac.MAC_ERR_ARG

@@ -12,6 +12,8 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
 ARGS = ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3", "--workload", "tiny"]
 
 
@@ -27,6 +29,10 @@ def _check_line(d, n_gpus):
     assert d["n_gpus"] == n_gpus and d["steps"] == 2 and d["warmup"] == 3
     assert d["higher_is_better"] is True and d["vs_baseline"] is None
     assert d["config"]["workload"] == "tiny"
+    # the same config dict the GPU arm prints (the driver compares them key by key)
+    import synth
+    import bench
+    assert d["config"] == bench.bench_config(synth.WORKLOADS["tiny"], False, n_gpus)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     e2e = d["e2e"]

@@ -63,10 +63,14 @@ def test_long_128k_all_miss_steps():
     compare_stream(wl, synth.queries(wl, 4), synth.kv_cache(wl, 4), tau=0.0)
 
 
-def test_paged_mixed_stream():
+@pytest.mark.slow
+def test_paged_mixed_stream_full():
+    """The paged workload at its stated size: 16 sequences of 8K-64K keys on a
+    shuffled pool of 16-key pages, all 64 steps, every step against the oracle."""
     wl = synth.WORKLOADS["paged_mixed"]
-    steps = 24
-    compare_stream(wl, synth.queries(wl, steps), synth.kv_cache(wl, steps))
+    assert wl.steps == 64
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl))
+    assert 0 < r["hits"] < wl.steps * wl.B * wl.Hkv
 
 
 def test_paged_equals_contiguous_bitwise():
@@ -94,27 +98,28 @@ def test_paged_equals_contiguous_bitwise():
             np.testing.assert_array_equal(x, y)
 
 
-def test_continuous_append_stream():
-    """Paged cache filled one row per step through mac_append_kv, ring updated every step."""
+def _continuous_append_stream(wl, steps):
+    """Paged cache filled one row per step through mac_append_kv (every decode
+    row poisoned with NaN until its append), the window updated every step;
+    every step against the oracle.  Returns the number of hits."""
     import kv_cache_reuse_b200 as mac
-    wl = synth.WORKLOADS["continuous_16k"]
-    steps = 96
     stream = synth.queries(wl, steps)
     cache = synth.kv_cache(wl, steps)
     torch, dev = torch_dev()
-    # device pool with every decode-step row poisoned (NaN) until appended
     Kd = torch.from_numpy(cache.K.view(np.int16)).to(dev)
     Vd = torch.from_numpy(cache.V.view(np.int16)).to(dev)
     ps = wl.page_size
-    for b in range(wl.B):
-        for pos in range(wl.L0[b], wl.L0[b] + steps):
-            pg = int(cache.block_table[b, pos // ps])
-            Kd[pg, pos % ps] = 0x7FC0
-            Vd[pg, pos % ps] = 0x7FC0
+    pos = np.concatenate([np.arange(wl.L0[b], wl.L0[b] + steps) for b in range(wl.B)])
+    seq = np.repeat(np.arange(wl.B), steps)
+    pg = torch.from_numpy(cache.block_table[seq, pos // ps].astype(np.int64)).to(dev)
+    row = torch.from_numpy((pos % ps).astype(np.int64)).to(dev)
+    Kd[pg, row] = 0x7FC0
+    Vd[pg, row] = 0x7FC0
     gpu = DeviceRun(wl, cache, K_dev=Kd, V_dev=Vd)
     orc = oracle.Oracle.for_workload(wl, cache)
     knew = torch.empty((wl.B, wl.Hkv, wl.D), dtype=torch.int16, device=dev)
     vnew = torch.empty_like(knew)
+    hits = 0
     for t in range(steps):
         kr, vr = synth.step_rows(cache, stream.seq_lens[t])
         knew.copy_(torch.from_numpy(kr.view(np.int16)))
@@ -123,11 +128,30 @@ def test_continuous_append_stream():
         mac.mac_append_kv(gpu.st, Kd, Vd, gpu.bt, gpu.lens, knew, vnew)
         r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
         out, lse, hit, mpos = gpu.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
-        np.testing.assert_array_equal(hit, r.hit)
-        np.testing.assert_array_equal(mpos, r.match_pos)
-        assert np.abs(out - r.out).max() <= OUT_TOL
-        assert np.abs(lse - r.lse).max() <= LSE_TOL
+        np.testing.assert_array_equal(hit, r.hit, err_msg="hit mask, step %d" % t)
+        np.testing.assert_array_equal(mpos, r.match_pos, err_msg="match position, step %d" % t)
+        assert np.abs(out - r.out).max() <= OUT_TOL, "out, step %d" % t
+        assert np.abs(lse - r.lse).max() <= LSE_TOL, "lse, step %d" % t
+        hits += int(hit.sum())
     assert gpu.st.get_status() == 0
+    return hits
+
+
+def test_continuous_append_stream():
+    """The first 96 steps of the continuous workload."""
+    wl = synth.WORKLOADS["continuous_16k"]
+    assert _continuous_append_stream(wl, 96) > 0
+
+
+@pytest.mark.slow
+def test_continuous_append_stream_full():
+    """The continuous workload at its stated size: 8 sequences, 16K prefix,
+    all 4096 decode steps with an append each step, hits from the two-state
+    Markov chain -- the ring, the hit chains and the append path over a long run."""
+    wl = synth.WORKLOADS["continuous_16k"]
+    assert wl.steps == 4096
+    hits = _continuous_append_stream(wl, wl.steps)
+    assert 0.6 * wl.steps * wl.B * wl.Hkv < hits < wl.steps * wl.B * wl.Hkv
 
 
 def test_ring_state_matches_oracle_window():
@@ -280,6 +304,34 @@ def test_weighted_split_all_miss():
     wl = synth.WORKLOADS["llama8b_32k"].with_(B=4, L0=(32768, 30000, 31000, 29000), steps=5)
     r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=0.0)
     assert r["hits"] == 0
+
+
+def test_reproducible_split_gives_identical_bits():
+    """mac_set_reproducible: on large steps (above the rate-weighted split's
+    threshold) two states with different histories -- one first ran steps of
+    another stream, which would have taught it per-SM rates -- give the same
+    bits on the same inputs, and match the oracle."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=4, L0=(32768, 30000, 31000, 29000), steps=6)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    a = DeviceRun(wl, cache, tune={"reproducible": 1})
+    b = DeviceRun(wl, cache, tune={"reproducible": 1})
+    other = synth.queries(wl.with_(seed=wl.seed + 99))
+    for t in range(4):
+        b.step(other.q[t], other.rope_pos[t], other.seq_lens[t])
+    for s_ in range(wl.B):
+        mac.mac_reset_seq(b.st, s_)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    for t in range(wl.steps):
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        y = b.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        for u, v in zip(x, y):
+            np.testing.assert_array_equal(u, v, err_msg="step %d" % t)
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+        np.testing.assert_array_equal(x[2], r.hit)
+        np.testing.assert_array_equal(x[3], r.match_pos)
+        assert float(np.abs(x[0] - r.out).max()) <= OUT_TOL and float(np.abs(x[1] - r.lse).max()) <= LSE_TOL
+    assert a.st.get_status() == 0 and b.st.get_status() == 0
 
 
 _SPLIT = {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 64}
@@ -574,15 +626,18 @@ def test_warm_start_from_prefill_then_decode(case):
 @pytest.mark.parametrize("opts", [{}, {"per_head": 1, "ring_bf16": 1}])
 def test_graph_captured_multilayer_loop(opts):
     """Several layers' steps recorded once as one CUDA graph and replayed for
-    every token (inputs copied into fixed buffers before each replay) give
-    the same bits as the same steps run eagerly (also with per-head matching
-    and a bf16 window)."""
+    every token (inputs copied into fixed buffers before each replay): each
+    layer's decisions bit-exact and its out / lse within tolerance of its own
+    fp64 oracle at every token (also with per-head matching and a bf16 window),
+    and the replayed bits equal to the same steps run eagerly."""
     import kv_cache_reuse_b200 as mac
     torch, dev = torch_dev()
     L = 3
     wls = [synth.WORKLOADS["tiny"].with_(steps=24, seed=10 + l, head_labels=bool(opts)) for l in range(L)]
     streams = [synth.queries(w) for w in wls]
     caches = [synth.kv_cache(w) for w in wls]
+    oracles = [oracle.Oracle.for_workload(w, c, per_head=opts.get("per_head", 0), ring_bf16=opts.get("ring_bf16", 0))
+               for w, c in zip(wls, caches)]
     eager = [DeviceRun(w, c, **opts) for w, c in zip(wls, caches)]
     graph = [DeviceRun(w, c, **opts) for w, c in zip(wls, caches)]
     s = torch.cuda.Stream()
@@ -602,13 +657,18 @@ def test_graph_captured_multilayer_loop(opts):
         g.replay()
         torch.cuda.synchronize()
         for l in range(L):
-            st = streams[l]
-            x = eager[l].step(st.q[t], st.rope_pos[t], st.seq_lens[t])
+            st, c = streams[l], caches[l]
             y = (graph[l].out.cpu().numpy(), graph[l].lse.cpu().numpy(), graph[l].hit.cpu().numpy(),
                  graph[l].mpos.cpu().numpy())
+            ref = oracles[l].step(st.q[t], st.rope_pos[t], c.K, c.V, c.block_table, st.seq_lens[t])
+            np.testing.assert_array_equal(y[2], ref.hit, err_msg="hit mask, layer %d step %d" % (l, t))
+            np.testing.assert_array_equal(y[3], ref.match_pos, err_msg="match position, layer %d step %d" % (l, t))
+            assert float(np.abs(y[0] - ref.out).max()) <= OUT_TOL, "out, layer %d step %d" % (l, t)
+            assert float(np.abs(y[1] - ref.lse).max()) <= LSE_TOL, "lse, layer %d step %d" % (l, t)
+            x = eager[l].step(st.q[t], st.rope_pos[t], st.seq_lens[t])
             for u, v in zip(x, y):
-                np.testing.assert_array_equal(u, v, err_msg="layer %d step %d" % (l, t))
-            hits += int(x[2].sum())
+                np.testing.assert_array_equal(u, v, err_msg="graph vs eager, layer %d step %d" % (l, t))
+            hits += int(ref.hit.sum())
     assert hits > 0
     assert all(r.st.get_status() == 0 for r in graph)
 
