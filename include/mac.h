@@ -15,10 +15,14 @@
  *
  * Conventions used by every entry point
  *   - Group: each KV head serves G = num_q_heads / num_kv_heads query heads
- *     (GQA; page 1 states that the method works with MQA and GQA); G may be 1 (multi-head
- *     attention) up to 8.  Larger groups (MQA with more than 8 query heads
- *     per KV head) return MAC_ERR_SHAPE.  One match decision is taken per
- *     (sequence, KV head) over its G heads.
+ *     (page 1 states that the method works with MQA and GQA): G from 1
+ *     (multi-head attention) to 8, or 16, 32 or 64 (multi-query attention
+ *     sized groups, e.g. 32 query heads over one KV head); other sizes return
+ *     MAC_ERR_SHAPE.  One match decision is taken per (sequence, KV head)
+ *     over its G heads.  Groups of 16-64 heads are processed as chunks of 8
+ *     that read each K/V row from memory once for the whole group; they take
+ *     no per-head matching, and every key range runs through partial
+ *     results (the whole-unit setting does not apply to them).
  *   - Distance: mean over the G heads of the squared L2 distance between the
  *     pre-RoPE queries.  Hit iff the smallest distance over the window is
  *     strictly below tau; ties go to the more recent entry; NaN never hits.
@@ -77,7 +81,7 @@ enum {
 typedef struct MacConfig {
     int batch;             /* B >= 1 */
     int num_q_heads;       /* Hq */
-    int num_kv_heads;      /* Hkv; Hq must be a multiple of it, Hq / Hkv <= 8 */
+    int num_kv_heads;      /* Hkv; Hq must be a multiple of it, Hq / Hkv in 1..8, 16, 32 or 64 */
     int head_dim;          /* D: 64 or 128 */
     int window;            /* W: entries kept per (sequence, KV head), 1..256 */
     int band;              /* b >= 0: keys before the match position that are recomputed */
@@ -94,8 +98,9 @@ typedef struct MacConfig {
                             * query heads; 1: one decision per query head (its own squared L2
                             * distance, nearest entry and reuse boundary), the KV head then reads
                             * the union of its heads' key ranges once; hit_mask and match_pos
-                            * become [B][Hq].  Other values MAC_ERR_ARG.  (Page 1: the method
-                            * composes with MQA/GQA; the page does not fix the granularity.) */
+                            * become [B][Hq].  Other values MAC_ERR_ARG; groups of more than 8
+                            * heads MAC_ERR_SHAPE.  (Page 1: the method composes with MQA/GQA;
+                            * the page does not fix the granularity.) */
     int q_bf16;            /* 0 (default): q_pre is fp32; 1: q_pre holds bf16 bit patterns (uint16) */
     int ring_bf16;         /* 0 (default): the window keeps fp32 queries and outputs; 1: it keeps
                             * them as bf16 (round to nearest even from fp32; m and l stay fp32),

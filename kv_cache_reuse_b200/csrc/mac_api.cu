@@ -44,6 +44,8 @@ struct MacState {
   float* part = nullptr;
   int* unit_cnt = nullptr;
   int* done = nullptr;
+  float* dpart = nullptr;  // groups of 16-64 heads: each chunk's part of every entry's distance
+  int* ucnt = nullptr;     // groups of 16-64 heads: chunk CTAs of a unit that arrived
   unsigned* status = nullptr;
   double* inv_freq = nullptr;
   // staging of mac_decode_step_host: one packed block each way, on the
@@ -103,7 +105,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,   s->hplan,
-                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done,  s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done, s->dpart, s->ucnt, s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -117,11 +119,13 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 int check_config(const MacConfig* c) {
   if (!c) return MAC_ERR_ARG;
   if (c->batch < 1 || c->num_kv_heads < 1 || c->num_q_heads < 1) return MAC_ERR_ARG;
-  if (c->num_q_heads % c->num_kv_heads != 0 || c->num_q_heads / c->num_kv_heads > kMaxGroup) return MAC_ERR_SHAPE;
+  if (c->num_q_heads % c->num_kv_heads != 0 || !group_ok(c->num_q_heads / c->num_kv_heads)) return MAC_ERR_SHAPE;
   if (c->head_dim != 64 && c->head_dim != 128) return MAC_ERR_SHAPE;
   if (c->window < 1 || c->window > kMaxWindow) return MAC_ERR_SHAPE;
   if (c->band < 0 || c->cut_mode < 0 || c->cut_mode > 1) return MAC_ERR_ARG;
   if (c->match_per_head < 0 || c->match_per_head > 1) return MAC_ERR_ARG;
+  // per-head matching holds a group in one tile: groups of up to 8 heads
+  if (c->match_per_head && c->num_q_heads / c->num_kv_heads > kMaxGroup) return MAC_ERR_SHAPE;
   if (c->q_bf16 < 0 || c->q_bf16 > 1 || c->ring_bf16 < 0 || c->ring_bf16 > 1) return MAC_ERR_ARG;
   if (!(c->rope_theta > 0.0) || isnan(c->tau)) return MAC_ERR_ARG;
   if (c->page_size == 0) {
@@ -262,6 +266,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->part, s->max_parts * partial_floats((int)G, (int)D)));
   A(alloc(&s->unit_cnt, U));
   A(alloc(&s->done, 1));
+  A(alloc(&s->dpart, U * W1 * (size_t)group_chunks((int)G)));
+  A(alloc(&s->ucnt, U));
   A(alloc(&s->inv_freq, D / 2));
   s->off_q = 0;
   s->off_pos = up256(s->off_q + B * Hq * D * s->QES);
@@ -295,6 +301,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->steps, 0, U * sizeof(int)));
   A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
   A(cudaMemset(s->done, 0, sizeof(int)));
+  A(cudaMemset(s->ucnt, 0, U * sizeof(int)));
   A(cudaMemset(s->rate, 0, s->grid * sizeof(float)));
   A(cudaMemset(s->claim, 0, s->grid * sizeof(int)));
   {  // even shares until the first rates are measured
@@ -403,6 +410,8 @@ static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope
   p.bounds = s->bounds;
   p.claim = s->claim;
   p.done = s->done;
+  p.dpart = s->dpart;
+  p.ucnt = s->ucnt;
   p.status = s->status;
   p.B = s->cfg.batch;
   p.Hq = s->cfg.num_q_heads;
@@ -420,7 +429,7 @@ static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope
   p.grid = s->grid;
   p.min_keys = s->min_keys;
   p.piece_cost = s->piece_cost;
-  p.unit_max = s->unit_max;
+  p.unit_max = s->G > kMaxGroup ? 0 : s->unit_max;  // groups of 16-64 heads run split items only
   return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 

@@ -99,6 +99,7 @@ struct __align__(1024) AttnSmem {
   float q[C::NQ][C::GD];              // queries of the upcoming pieces (heads >= G unused)
   float wbuf[kConsumerWarps][C::WB];  // weights exchange / piece combine
   unsigned long long full[kConsumerWarps][C::NST];
+  unsigned long long empty[kConsumerWarps][C::NST];  // chunked groups: a box slot's C readers are done
   unsigned long long qfull[C::NQ];
   unsigned long long csync;
   unsigned long long rfull;          // reused ring state of the current whole-unit piece landed
@@ -513,11 +514,16 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA
 // partials), warps [wA, 8) set B (the tail).  With a reused state (heads in
 // hmask; o, m and l on chip in sm.ring) S = reused + A, else S = A; S is the
 // unit's new ring entry in slot dst and S + B its output.
-template <int D, int GP, int GF>
+//
+// Chunked groups (NC > 1, G = 8 NC heads per KV head): the call finishes the
+// 8 heads of chunk ch, whose states the warps' slots and sm.ring hold; the
+// global layouts are those of the whole group.
+template <int D, int GP, int GF, int NC = 1>
 __device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D, GP>& sm, int u, int wA, int hit,
-                                              int hmask, int dst, int end) {
+                                              int hmask, int dst, int end, int ch = 0) {
   constexpr int GDP = Cfg<D, GP>::GD;
-  const int G = group_of<GF>(p), GD = G * D;
+  const int G = NC > 1 ? GP : group_of<GF>(p), GD = G * D;  // heads of this call, and their elements
+  const int Gt = NC > 1 ? GF : G, h0 = NC > 1 ? ch * GP : 0;  // heads of the unit; first head of the call
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int Wp1 = p.W + 1;
   constexpr int PER = (GDP + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32);
@@ -542,21 +548,21 @@ __device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D,
       O += ring_o_at(sm.ring, idx, p.ring_bf16) * rl * a;
     }
     const size_t ds = (size_t)u * Wp1 + dst;
-    ring_o_put(p.ring_o, ds * GD + idx, L > 0.f ? __fdividef(O, L) : 0.f, p.ring_bf16);
+    ring_o_put(p.ring_o, (ds * Gt + h0) * D + idx, L > 0.f ? __fdividef(O, L) : 0.f, p.ring_bf16);
     if (d == 0) {
-      p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
-      p.ring_l[ds * G + h] = L;
+      p.ring_m[ds * Gt + h0 + h] = L > 0.f ? M * kLn2 : -INFINITY;
+      p.ring_l[ds * Gt + h0 + h] = L;
     }
     // output = S + tail
     const float M2 = fmaxf(M, MB);
     const float M2u = M2 == -INFINITY ? 0.f : M2;
     const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
     const float L2 = L * a0 + LB * aB, O2 = O * a0 + OB * aB;
-    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+    const size_t orow = (size_t)b * p.Hq + (size_t)kvh * Gt + h0 + h;
     p.out[orow * D + d] = __fdividef(O2, L2);  // L2 >= 1: every unit attends at least one key
     if (d == 0) p.lse[orow] = (M2 + __log2f(L2)) * kLn2;
   }
-  if (threadIdx.x == 0) p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
+  if (threadIdx.x == 0 && ch == 0) p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
 }
 
 // Last arriver of a split unit: merge its partials.  Segment A's partials
@@ -566,12 +572,16 @@ __device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D,
 // rest, in proportion to their counts -- and each folds its own into one
 // state (lane: four consecutive elements of every 128, KB partials per round
 // of loads); the finish of a whole unit then combines the eight states.
-template <int D, int GP, int GF, bool PH>
+template <int D, int GP, int GF, bool PH, int NC = 1>
 __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
   using C = Cfg<D, GP>;
   constexpr int NCH = C::GD / 128;                // 128-element runs of a padded group: 2, 4 or 8
   constexpr int KB = NCH <= 2 ? 8 : 16 / NCH;     // partials per round of loads
-  const int G = group_of<GF>(p), GD = G * D, G4 = group4(G), PF = GD + 2 * G4;
+  // chunked groups (NC > 1): the unit's 8 NC heads are merged 8 at a time;
+  // chunk ch of a partial is a run of partial_floats(8, D) floats at ch times that
+  const int G = NC > 1 ? GP : group_of<GF>(p), GD = G * D, G4 = group4(G);  // heads of one chunk
+  const int Gt = NC > 1 ? GF : G;                                           // heads of the unit
+  const int PF = NC > 1 ? (int)partial_floats(Gt, D) : GD + 2 * G4;         // floats of one partial
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const UnitPlan* const pp = p.plan + u;
   const int src_slot = pp->src_slot, dst_slot = pp->dst_slot, end = pp->end;
@@ -585,97 +595,147 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
   }
   const bool onA = warp < wA;
   const int cnt = onA ? nA : nB, stride = onA ? wA : kConsumerWarps - wA, first = onA ? warp : warp - wA;
-  const float* const part = p.part + (size_t)(onA ? sA.pbase : sB.pbase) * PF;
-  // the reused state on chip, in the layout of a whole unit's copy: each
-  // head's o row (fp32 or bf16 as stored), then m at GP*D and l at GP*D + GP
-  if (hmask != 0) {
-    const size_t ub = (size_t)u * (p.W + 1);
-    const int es = p.ring_bf16 ? 2 : 4, cph = D * es / 16;  // 16-byte chunks of one head's o
-    const int h = tid / cph, c = tid - h * cph;
-    if (h < G && ((hmask >> h) & 1)) {
-      const int slot = PH ? p.hplan[u].hsrc[h] : src_slot;
-      const uint4* src = reinterpret_cast<const uint4*>(ring_o_row(p.ring_o, ((ub + slot) * G + h) * D, p.ring_bf16));
-      reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.ring) + (size_t)h * D * es)[c] = __ldcg(src + c);
-    }
-    if (tid < 2 * G) {
-      const int hh = tid < G ? tid : tid - G;
-      if ((hmask >> hh) & 1) {
-        const size_t e = (ub + (PH ? p.hplan[u].hsrc[hh] : src_slot)) * G + hh;
-        sm.ring[C::GD + (tid < G ? hh : GP + hh)] = __ldcg(tid < G ? p.ring_m + e : p.ring_l + e);
-      }
-    }
-  }
-  float M[NCH], L[NCH], O[NCH][4];
-#pragma unroll
-  for (int j = 0; j < NCH; ++j) {
-    M[j] = -INFINITY;
-    L[j] = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) O[j][c] = 0.f;
-  }
 #pragma unroll 1
-  for (int i0 = first; i0 < cnt; i0 += KB * stride) {
-    float4 ov[KB][NCH];
-    float mv[KB][NCH], lv[KB][NCH];
-#pragma unroll
-    for (int k = 0; k < KB; ++k) {
-      const int i = i0 + k * stride;
-      const float* q = part + (size_t)i * PF;
-#pragma unroll
-      for (int j = 0; j < NCH; ++j) {
-        const int e = j * 128 + lane * 4, h = e / D;
-        if (i < cnt && e < GD) {
-          ov[k][j] = __ldcg(reinterpret_cast<const float4*>(q + e));
-          mv[k][j] = __ldcg(q + GD + h);
-          lv[k][j] = __ldcg(q + GD + G4 + h);
+  for (int ch = 0; ch < NC; ++ch) {
+    const int h0 = ch * G;  // first head of this chunk in the unit
+    const float* const part = p.part + (size_t)(onA ? sA.pbase : sB.pbase) * PF + (size_t)ch * (GD + 2 * G4);
+    // the reused state on chip, in the layout of a whole unit's copy: each
+    // head's o row (fp32 or bf16 as stored), then m at GP*D and l at GP*D + GP
+    if (hmask != 0) {
+      const size_t ub = (size_t)u * (p.W + 1);
+      const int es = p.ring_bf16 ? 2 : 4, cph = D * es / 16;  // 16-byte chunks of one head's o
+      const int h = tid / cph, c = tid - h * cph;
+      if (h < G && ((hmask >> h) & 1)) {
+        const int slot = PH ? p.hplan[u].hsrc[h] : src_slot;
+        const uint4* src = reinterpret_cast<const uint4*>(
+            ring_o_row(p.ring_o, ((ub + slot) * Gt + h0 + h) * D, p.ring_bf16));
+        reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.ring) + (size_t)h * D * es)[c] = __ldcg(src + c);
+      }
+      if (tid < 2 * G) {
+        const int hh = tid < G ? tid : tid - G;
+        if ((hmask >> hh) & 1) {
+          const size_t e = (ub + (PH ? p.hplan[u].hsrc[hh] : src_slot)) * Gt + h0 + hh;
+          sm.ring[C::GD + (tid < G ? hh : GP + hh)] = __ldcg(tid < G ? p.ring_m + e : p.ring_l + e);
         }
       }
     }
+    float M[NCH], L[NCH], O[NCH][4];
 #pragma unroll
-    for (int k = 0; k < KB; ++k)
+    for (int j = 0; j < NCH; ++j) {
+      M[j] = -INFINITY;
+      L[j] = 0.f;
 #pragma unroll
-      for (int j = 0; j < NCH; ++j)
-        if (i0 + k * stride < cnt && j * 128 + lane * 4 < GD)
-          fold_state<4>(M[j], L[j], O[j], mv[k][j], lv[k][j], &ov[k][j].x);
-  }
-  // this warp's state into its slot: o [GP][D], m [GP], l [GP]
-  float* const wb = sm.wbuf[warp];
+      for (int c = 0; c < 4; ++c) O[j][c] = 0.f;
+    }
+#pragma unroll 1
+    for (int i0 = first; i0 < cnt; i0 += KB * stride) {
+      float4 ov[KB][NCH];
+      float mv[KB][NCH], lv[KB][NCH];
 #pragma unroll
-  for (int j = 0; j < NCH; ++j) {
-    const int e = j * 128 + lane * 4, h = e / D;
-    if (e < GD) {
-      *reinterpret_cast<float4*>(wb + e) = make_float4(O[j][0], O[j][1], O[j][2], O[j][3]);
-      if (e - h * D == 0) {
-        wb[C::GD + h] = M[j];
-        wb[C::GD + GP + h] = L[j];
+      for (int k = 0; k < KB; ++k) {
+        const int i = i0 + k * stride;
+        const float* q = part + (size_t)i * PF;
+#pragma unroll
+        for (int j = 0; j < NCH; ++j) {
+          const int e = j * 128 + lane * 4, h = e / D;
+          if (i < cnt && e < GD) {
+            ov[k][j] = __ldcg(reinterpret_cast<const float4*>(q + e));
+            mv[k][j] = __ldcg(q + GD + h);
+            lv[k][j] = __ldcg(q + GD + G4 + h);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+#pragma unroll
+        for (int j = 0; j < NCH; ++j)
+          if (i0 + k * stride < cnt && j * 128 + lane * 4 < GD)
+            fold_state<4>(M[j], L[j], O[j], mv[k][j], lv[k][j], &ov[k][j].x);
+    }
+    // this warp's state into its slot: o [GP][D], m [GP], l [GP]
+    float* const wb = sm.wbuf[warp];
+#pragma unroll
+    for (int j = 0; j < NCH; ++j) {
+      const int e = j * 128 + lane * 4, h = e / D;
+      if (e < GD) {
+        *reinterpret_cast<float4*>(wb + e) = make_float4(O[j][0], O[j][1], O[j][2], O[j][3]);
+        if (e - h * D == 0) {
+          wb[C::GD + h] = M[j];
+          wb[C::GD + GP + h] = L[j];
+        }
       }
     }
+    if (!consumer_sync(sm, sync_phase, p.status)) return false;
+    unit_epilogue<D, GP, GF, NC>(p, sm, u, wA, hmask != 0, hmask, dst_slot, end, ch);
+    // the warps' slots and the ring buffer are reused by the next chunk or piece
+    if (!consumer_sync(sm, sync_phase, p.status)) return false;
   }
-  if (!consumer_sync(sm, sync_phase, p.status)) return false;
-  unit_epilogue<D, GP, GF>(p, sm, u, wA, hmask != 0, hmask, dst_slot, end);
   if (tid == 0) p.unit_cnt[u] = 0;
-  // the warps' slots and the ring buffer are reused by the next piece
-  return consumer_sync(sm, sync_phase, p.status);
+  return true;
 }
 
 // End of a split piece: combine the 8 warps, write the partial, count it
 // and, if it was the unit's last, merge the unit.
-template <int D, int GP, int GF, bool PH>
+// Chunked groups: merge element e (head h) of chunk ch from the slots of the
+// warps that hold that chunk (warps ch, ch + NC, ...), sums relative to 2^M.
+template <int D, int GP, int NC>
+__device__ __forceinline__ void combine_team(const AttnSmem<D, GP>& sm, int ch, int e, int h, float& M, float& L,
+                                             float& O) {
+  constexpr int NKL = kConsumerWarps / NC, GD = Cfg<D, GP>::GD;
+  float m[NKL], l[NKL], o[NKL];
+#pragma unroll
+  for (int k = 0; k < NKL; ++k) {
+    const int w = ch + NC * k;
+    m[k] = sm.wbuf[w][GD + h];
+    l[k] = sm.wbuf[w][GD + GP + h];
+    o[k] = sm.wbuf[w][e];
+  }
+  M = m[0];
+#pragma unroll
+  for (int k = 1; k < NKL; ++k) M = fmaxf(M, m[k]);
+  const float Mu = M == -INFINITY ? 0.f : M;
+  L = O = 0.f;
+#pragma unroll
+  for (int k = 0; k < NKL; ++k) {
+    const float a = ex2(m[k] - Mu);
+    L += l[k] * a;
+    O += o[k] * a;
+  }
+}
+
+template <int D, int GP, int GF, bool PH, int NC = 1>
 __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D, GP>& A, int unit, int pidx,
                                uint32_t& sync_phase) {
   const int G = group_of<GF>(p), GD = G * D, G4 = group4(G);
   warp_combine_store<D, GP>(A, sm.wbuf[threadIdx.x >> 5]);
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   float* dst = p.part + (size_t)pidx * (GD + 2 * G4);
+  if constexpr (NC > 1) {
+    // chunk ch of the partial: o [8][D], m [8], l [8] (the layout of an 8-head partial)
+    constexpr int GDc = GP * D, PFc = GDc + 2 * GP;
 #pragma unroll 1
-  for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
-    const int h = idx / D;
-    float MA, LA, OA, M, L, O;
-    combine_warps2<D, GP, GP>(sm, 0, idx, h, MA, LA, OA, M, L, O);
-    dst[idx] = O;
-    if (idx - h * D == 0) {
-      dst[GD + h] = M;
-      dst[GD + G4 + h] = L;
+    for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
+      const int ch = idx / GDc, e = idx - ch * GDc, h = e / D;
+      float M, L, O;
+      combine_team<D, GP, NC>(sm, ch, e, h, M, L, O);
+      float* dc = dst + (size_t)ch * PFc;
+      dc[e] = O;
+      if (e - h * D == 0) {
+        dc[GDc + h] = M;
+        dc[GDc + GP + h] = L;
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int idx = threadIdx.x; idx < GD; idx += kConsumerWarps * 32) {
+      const int h = idx / D;
+      float MA, LA, OA, M, L, O;
+      combine_warps2<D, GP, GP>(sm, 0, idx, h, MA, LA, OA, M, L, O);
+      dst[idx] = O;
+      if (idx - h * D == 0) {
+        dst[GD + h] = M;
+        dst[GD + G4 + h] = L;
+      }
     }
   }
   // every thread's partial stores happen-before thread 0's fence through the
@@ -689,7 +749,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
-    return merge_unit<D, GP, GF, PH>(p, sm, unit, sync_phase);
+    return merge_unit<D, GP, GF, PH, NC>(p, sm, unit, sync_phase);
   }
   return true;
 }
@@ -750,6 +810,17 @@ __device__ __forceinline__ WarpRange warp_range(const Piece& pc, int warp) {
     r.first = warp - base;
     r.stride = kConsumerWarps - base;
   }
+  return r;
+}
+// Chunked groups: the boxes of a split piece taken by key-lane kl of nkl.
+__device__ __forceinline__ WarpRange team_range(const Piece& pc, int kl, int nkl) {
+  WarpRange r;
+  r.kb0 = pc.kb0;
+  r.k0 = pc.k0;
+  r.k1 = pc.k1;
+  r.nbox = pc.nbox;
+  r.first = kl;
+  r.stride = nkl;
   return r;
 }
 __device__ __forceinline__ int box_count(int k0, int k1) {
@@ -855,10 +926,19 @@ __device__ __noinline__ void rate_shares(const AttendParams& p) {
   if (tid == 0) p.cw[G] = 1.0;
 }
 
-template <int D, int GP, int GF, bool PH>
+// NC: chunks of 8 heads per KV head (1 for groups of up to 8).  With NC > 1
+// (G = 8 NC) warp w holds the heads [8 (w % NC), 8 (w % NC) + 8) over the
+// boxes of key-lane w / NC: the NC warps of a key-lane read the same boxes
+// from one ring of NST * NC slots, filled by the key-lane's first warp after
+// every reader of the slot has released it (an mbarrier with NC arrivals), so
+// each K/V byte crosses from HBM once for all 8 NC heads.  Such groups run
+// split items only.
+template <int D, int GP, int GF, bool PH, int NC = 1>
 __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
   using C = Cfg<D, GP>;
   constexpr int NST = C::NST, NQ = C::NQ;
+  constexpr int NKL = kConsumerWarps / NC, NSTT = NST * NC;  // key-lanes; box slots of one key-lane
+  static_assert(NC == 1 || (GP == 8 && GF == 8 * NC && kConsumerWarps % NC == 0), "chunked groups of 8 heads");
   constexpr uint32_t kBoxBytes = kSubKeys * D * 2;
   extern __shared__ __align__(128) unsigned char smem_raw[];
   // the swizzled TMA boxes need 1024-byte alignment of the shared window
@@ -866,6 +946,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       *reinterpret_cast<AttnSmem<D, GP>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = group_of<GF>(p), GD = G * D;  // real group: global layouts
+  const int ch = warp % NC, kl = warp / NC;   // chunk of heads, key-lane (NC = 1: 0 and the warp)
+  const bool issuer = ch == 0;                // fills the key-lane's box slots
+  // box slot st of this key-lane: K box, V box (+ kSubKeys * D), its barriers
+  auto kv_slot = [&](int st) -> uint16_t* {
+    const int f = kl * NSTT + st;
+    return sm.kv[f / NST][f % NST][0];
+  };
+  auto full_bar = [&](int st) -> unsigned long long* {
+    const int f = kl * NSTT + st;
+    return &sm.full[f / NST][f % NST];
+  };
+  auto empty_bar = [&](int st) -> unsigned long long* {
+    const int f = kl * NSTT + st;
+    return &sm.empty[f / NST][f % NST];
+  };
 
   const int cta = blockIdx.x;
   if (tid == 32) {  // bring both TMA descriptors on chip while the match kernel runs
@@ -874,7 +969,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   }
   if (tid == 0) {
     for (int w = 0; w < kConsumerWarps; ++w)
-      for (int s = 0; s < NST; ++s) mbar_init(&sm.full[w][s], 1);
+      for (int s = 0; s < NST; ++s) {
+        mbar_init(&sm.full[w][s], 1);
+        if (NC > 1) mbar_init(&sm.empty[w][s], NC);
+      }
     for (int s = 0; s < NQ; ++s) mbar_init(&sm.qfull[s], 1);
     mbar_init(&sm.csync, kConsumerWarps);
     mbar_init(&sm.rfull, 1);
@@ -921,18 +1019,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   __syncthreads();
   const uint64_t pol = evict_first_policy();
 
-  // issue cursor: this warp's boxes of every piece, NST ahead
+  // issue cursor: this warp's (NC > 1: this key-lane's) boxes of every piece, NSTT ahead
+  auto range_of = [&](const Piece& pc) { return NC == 1 ? warp_range(pc, warp) : team_range(pc, kl, NKL); };
   Walker wi{first_seg, lo, hi, sm.items, first_seg};
   Piece ip;
   WarpRange ir;
-  bool ivalid = wi.next(p, slot, ip);
-  if (ivalid) ir = warp_range(ip, warp);
+  bool ivalid = issuer && wi.next(p, slot, ip);
+  if (ivalid) ir = range_of(ip);
   int ib = ivalid ? ir.first : 0, ipn = 0, nissued = 0, nq_issued = 0;
   auto issue_advance = [&]() {
     while (ivalid && ib >= ir.nbox) {
       ivalid = wi.next(p, slot, ip);
       if (ivalid) {
-        ir = warp_range(ip, warp);
+        ir = range_of(ip);
         ib = ir.first;
       }
       ++ipn;
@@ -940,7 +1039,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   };
   auto issue_box = [&](int st) {
     // warp 0 always owns box 0 of its range in every piece: it brings the query
-    const bool qfirst = warp == 0 && ib == 0;
+    // (chunked groups read their query straight from global memory instead)
+    const bool qfirst = NC == 1 && warp == 0 && ib == 0;
     if (lane == 0) {
       if (qfirst) {
         const int qs = ipn % NQ;
@@ -957,11 +1057,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
         c2 = key;
         c3 = b;
       }
-      mbar_arrive_expect_tx(&sm.full[warp][st], 2 * kBoxBytes);
+      unsigned long long* fb = full_bar(st);
+      uint16_t* kbuf = kv_slot(st);
+      mbar_arrive_expect_tx(fb, 2 * kBoxBytes);
 #pragma unroll
       for (int hf = 0; hf < C::HALVES; ++hf) {
-        tma_load_4d(sm.kv[warp][st][0] + hf * kSubKeys * 64, &p.tmK, &sm.full[warp][st], 64 * hf, kvh, c2, c3, pol);
-        tma_load_4d(sm.kv[warp][st][1] + hf * kSubKeys * 64, &p.tmV, &sm.full[warp][st], 64 * hf, kvh, c2, c3, pol);
+        tma_load_4d(kbuf + hf * kSubKeys * 64, &p.tmK, fb, 64 * hf, kvh, c2, c3, pol);
+        tma_load_4d(kbuf + kSubKeys * D + hf * kSubKeys * 64, &p.tmV, fb, 64 * hf, kvh, c2, c3, pol);
       }
     }
     if (qfirst) ++nq_issued;
@@ -970,7 +1072,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     issue_advance();
   };
   issue_advance();
-  for (int k = 0; k < NST && ivalid; ++k) issue_box(k);
+  for (int k = 0; k < NSTT && ivalid; ++k) issue_box(k);
 
   // consume cursor
   Acc<D, GP> A;
@@ -982,9 +1084,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   bool ok = true;
   unsigned long long t_first = 0, t_last = 0;  // thread 0: first and last box consumed
   while (ok && wc.next(p, slot, cp)) {
-    const int qs = cpn % NQ;
-    if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
-    load_query<D, GP>(A, sm.q[qs], G);
+    if constexpr (NC == 1) {
+      const int qs = cpn % NQ;
+      if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
+      load_query<D, GP>(A, sm.q[qs], G);
+    } else {
+      // this warp's 8 heads of the unit's rotated query (written by the match kernel)
+      load_query<D, GP>(A, p.qrot + ((size_t)cp.unit * GF + ch * GP) * D, GP);
+    }
     const bool ring_copy = cp.whole && cp.hit;
     ring_pending = ring_copy;
     float rml = 0.f;  // m (thread t < G) or l (G <= t < 2G) of the reused state
@@ -1039,21 +1146,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       if (!kBulkML<GF> && tid < 2 * G)
         rml = __ldcg(tid < G ? p.ring_m + rs * G + tid : p.ring_l + rs * G + (tid - G));
     }
-    const WarpRange cr = warp_range(cp, warp);
+    const WarpRange cr = range_of(cp);
     for (int bj = cr.first; bj < cr.nbox; bj += cr.stride) {
-      const int st = cons % NST;
-      if (!mbar_wait(&sm.full[warp][st], (uint32_t)(cons / NST) & 1u, &sm.abort_flag, p.status)) {
+      const int st = cons % NSTT;
+      const uint32_t ph = (uint32_t)(cons / NSTT) & 1u;
+      if (!mbar_wait(full_bar(st), ph, &sm.abort_flag, p.status)) {
         ok = false;
         break;
       }
       if (tid == 0 && cons == 0) t_first = globaltimer();
       const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * C::PB;
-      process_box<D, GP, PH>(A, sm.kv[warp][st][0], sm.kv[warp][st][1], pbuf, key_box, cr.k0, cr.k1,
+      uint16_t* kbuf = kv_slot(st);
+      process_box<D, GP, PH>(A, kbuf, kbuf + kSubKeys * D, pbuf, key_box, cr.k0, cr.k1,
                              key_box < cr.k0 || key_box + kSubKeys > cr.k1, lo0, lo1);
       par ^= 1;
       ++cons;
-      __syncwarp();
+      if constexpr (NC > 1) {
+        // release the slot: this warp's reads (and its zeroing of rows outside
+        // the range, identical in every reader) are done before the next copy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(st));
+        __syncwarp();
+        if (ivalid && !mbar_wait(empty_bar(st), ph, &sm.abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+      } else {
+        __syncwarp();
+      }
       if (ivalid) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         issue_box(st);
@@ -1061,9 +1183,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     }
     if (!ok) break;
     if (tid == 0) t_last = globaltimer();
-    const bool fin = cp.whole ? finalize_unit<D, GP, GF>(p, sm, A, cp.unit, cp.wA, cp.hit, hmask, cp.dst, cp.k1,
-                                                         rml, ring_phase, sync_phase)
-                              : finalize_piece<D, GP, GF, PH>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    bool fin;
+    if constexpr (NC > 1)
+      fin = finalize_piece<D, GP, GF, PH, NC>(p, sm, A, cp.unit, cp.pidx, sync_phase);
+    else
+      fin = cp.whole ? finalize_unit<D, GP, GF>(p, sm, A, cp.unit, cp.wA, cp.hit, hmask, cp.dst, cp.k1, rml,
+                                                ring_phase, sync_phase)
+                     : finalize_piece<D, GP, GF, PH>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (ring_copy) ring_phase ^= 1u;
     ring_pending = false;
     if (!fin) break;
@@ -1072,7 +1198,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   if (weighted && p.rate != nullptr) {
     // fold this SM's streaming rate (boxes per microsecond) into its record;
     // only CTAs that mostly streamed (at least kRateMinBoxes boxes) measure it
-    if (lane == 0) atomicAdd(&sm.box_total, cons);
+    if (lane == 0 && issuer) atomicAdd(&sm.box_total, cons);  // each box once, by the warp that filled it
     __syncthreads();
     const int boxes = sm.box_total;
     if (ok && tid == 0 && (int)smid < p.grid && boxes >= kRateMinBoxes && t_last > t_first + 2000) {
@@ -1087,8 +1213,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     if (lane == 0) {
       for (int k = cons; k < nissued; ++k) {
         const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(&sm.full[warp][k % NST], (uint32_t)(k / NST) & 1u) &&
-               globaltimer() - t0 < 100000000ull) {
+        while (!mbar_try_wait(full_bar(k % NSTT), (uint32_t)(k / NSTT) & 1u) && globaltimer() - t0 < 100000000ull) {
         }
       }
       if (warp == 0) {
@@ -1138,9 +1263,9 @@ size_t attend_smem_bytes(int D, int G) {
 namespace {
 // Kernel variants: exact groups of 4 and 8 (compile-time G), groups of 1-3
 // and 5-7 padded to 4 and 8 (run-time G), and per-head matching (run-time G).
-template <int D, int GP, int GF, bool PH>
+template <int D, int GP, int GF, bool PH, int NC = 1>
 cudaError_t set_smem() {
-  return cudaFuncSetAttribute(mac_attend_kernel<D, GP, GF, PH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(mac_attend_kernel<D, GP, GF, PH, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)attend_smem_bytes(D, GP));
 }
 template <int D>
@@ -1151,6 +1276,9 @@ cudaError_t set_smem_all() {
   if (e == cudaSuccess) e = set_smem<D, 8, 0, false>();
   if (e == cudaSuccess) e = set_smem<D, 4, 0, true>();
   if (e == cudaSuccess) e = set_smem<D, 8, 0, true>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 16, false, 2>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 32, false, 4>();
+  if (e == cudaSuccess) e = set_smem<D, 8, 64, false, 8>();
   return e;
 }
 // Per-head matching runs the run-time-group variants with per-head bounds.
@@ -1162,6 +1290,9 @@ cudaError_t launch_d(cudaLaunchConfig_t& cfg, const AttendParams& p) {
     if (G <= 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 0, true>, p);
     return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 0, true>, p);
   }
+  if (G == 16) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 16, false, 2>, p);
+  if (G == 32) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 32, false, 4>, p);
+  if (G == 64) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 64, false, 8>, p);
   if (G == 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 4, false>, p);
   if (G == 8) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 8, false>, p);
   if (G < 4) return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 4, 0, false>, p);
@@ -1170,12 +1301,12 @@ cudaError_t launch_d(cudaLaunchConfig_t& cfg, const AttendParams& p) {
 }  // namespace
 
 cudaError_t attend_prepare(int D, int G) {
-  if ((D != 64 && D != 128) || G < 1 || G > kMaxGroup) return cudaErrorInvalidValue;
+  if ((D != 64 && D != 128) || !group_ok(G)) return cudaErrorInvalidValue;
   return D == 128 ? set_smem_all<128>() : set_smem_all<64>();
 }
 
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s) {
-  if ((D != 64 && D != 128) || p.G < 1 || p.G > kMaxGroup) return cudaErrorInvalidValue;
+  if ((D != 64 && D != 128) || !group_ok(p.G) || (p.G > kMaxGroup && p.per_head)) return cudaErrorInvalidValue;
   // Programmatic stream serialization: the kernel may be scheduled while the
   // preceding match kernel drains; it calls griddepcontrol.wait before it
   // reads anything that kernel wrote.

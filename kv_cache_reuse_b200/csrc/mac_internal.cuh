@@ -8,7 +8,8 @@
 
 namespace mac {
 
-constexpr int kMaxGroup = 8;          // query heads per KV head (G) the kernels handle: 1..8
+constexpr int kMaxGroup = 8;          // query heads per KV head held in one tensor-core tile: 1..8
+constexpr int kMaxWideGroup = 64;     // larger groups: 16, 32 or 64 heads, as 2, 4 or 8 chunks of 8
 constexpr int kSubKeys = 16;          // keys per TMA box (one box never crosses a page)
 constexpr int kConsumerWarps = 8;     // attention warps that compute
 constexpr int kKeysPerStage = 128;    // keys in flight per round of boxes (kConsumerWarps * 16)
@@ -77,6 +78,14 @@ struct PlanHeader {
 // split uses (cw[c] = share of ranges 0..c-1, cw[grid] = 1).
 constexpr long long kWeightMinCost = 4096;
 
+// Group sizes the kernels take: 1 to 8 heads per KV head in one tile, or
+// 16, 32, 64 heads (multi-query attention sized groups) in chunks of 8.
+__host__ __device__ inline bool group_ok(int G) {
+  return (G >= 1 && G <= kMaxGroup) || G == 16 || G == 32 || G == 64;
+}
+// Chunks of 8 heads a group is processed in (1 for groups of up to 8).
+__host__ __device__ inline int group_chunks(int G) { return G > kMaxGroup ? G / kMaxGroup : 1; }
+
 // The kernels hold a query group padded to GP = 4 or 8 heads (the columns of
 // their tensor-core tiles); heads G..GP-1 are zero and never stored.
 __host__ __device__ inline int group_pad(int G) { return G <= 4 ? 4 : 8; }
@@ -109,6 +118,8 @@ struct MatchParams {
   long long* bounds;       // [grid + 1] range starts of a weighted split
   int* claim;              // [grid] ranges taken by the attention CTAs (reset here)
   int* done;               // arrival counter of the match CTAs (reset by the last)
+  float* dpart;            // chunked groups: [U][W+1][NC] each chunk's part of an entry's distance
+  int* ucnt;               // chunked groups: [U] arrivals of a unit's chunk CTAs (reset by the last)
   unsigned* status;
   int B, Hq, Hkv, G, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
   int per_head;   // 1: one match decision per query head

@@ -70,6 +70,9 @@ def test_init_rejects_bad_config_before_touching_the_device(lib):
                      (dict(match_per_head=2), mac.MAC_ERR_ARG),
                      (dict(band=-1), mac.MAC_ERR_ARG), (dict(num_q_heads=20), mac.MAC_ERR_SHAPE),
                      (dict(num_q_heads=72), mac.MAC_ERR_SHAPE),  # 9 query heads per KV head
+                     (dict(num_q_heads=96), mac.MAC_ERR_SHAPE),  # 12: larger groups are 16, 32 or 64
+                     (dict(num_q_heads=1024), mac.MAC_ERR_SHAPE),  # 128 per KV head
+                     (dict(num_q_heads=128, match_per_head=1), mac.MAC_ERR_SHAPE),  # per-head: up to 8
                      (dict(head_dim=96), mac.MAC_ERR_SHAPE)):
         args = dict(batch=1, num_q_heads=32, num_kv_heads=8, head_dim=128, window=8, band=16, tau=0.1,
                     rope_theta=1e4, max_seq=64)

@@ -368,6 +368,66 @@ def test_group_sizes(case):
     assert r["hits"] > 0
 
 
+@pytest.mark.parametrize("case", ["g16_d128", "g32_mqa", "g64_mqa", "g16_d64", "g64_d64", "g32_paged", "g64_bf16",
+                                  "g32_cut1", "g16_band_covers", "g32_window_max"])
+def test_mqa_groups(case):
+    """Groups of 16, 32 and 64 query heads per KV head (multi-query attention,
+    which page 1 says the method composes with): the heads run in chunks of 8
+    over the same K/V boxes, the window scan over G/8 CTAs per unit; decisions
+    bit-exact, outputs within tolerance, every step, hits and misses."""
+    tiny, llama, paged = synth.WORKLOADS["tiny"], synth.WORKLOADS["llama8b_32k"], synth.WORKLOADS["paged_mixed"]
+    cut, qb, rb = 0, 0, 0
+    if case == "g16_d128":
+        wl = llama.with_(B=2, Hq=32, Hkv=2, L0=(5000, 3100), steps=16)
+    elif case == "g32_mqa":
+        wl = llama.with_(B=2, Hq=32, Hkv=1, L0=(9000, 4000), steps=24)
+    elif case == "g64_mqa":
+        wl = llama.with_(B=1, Hq=64, Hkv=1, L0=(12000,), steps=24)
+    elif case == "g16_d64":
+        wl = tiny.with_(Hq=16, Hkv=1, steps=40)
+    elif case == "g64_d64":
+        wl = tiny.with_(B=2, Hq=64, Hkv=1, L0=(1500, 700), steps=24)
+    elif case == "g32_paged":
+        wl = paged.with_(B=3, Hq=32, Hkv=1, L0=(3000, 1200, 6000), steps=16)
+    elif case == "g64_bf16":  # bf16 queries and window
+        wl, qb, rb = llama.with_(B=2, Hq=64, Hkv=1, L0=(6000, 2500), steps=16), 1, 1
+    elif case == "g32_cut1":
+        wl, cut = llama.with_(B=2, Hq=32, Hkv=1, L0=(3000, 5000), steps=16), 1
+    elif case == "g16_band_covers":  # the band reaches key 0: every reused prefix is empty
+        wl = tiny.with_(Hq=16, Hkv=1, L0=(40,), band=500, steps=24)
+    else:  # the largest window: the chunk CTAs scan their slots in several batches
+        wl = tiny.with_(Hq=32, Hkv=1, L0=(60,), steps=280, W=256, band=16)
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), cut_mode=cut, q_bf16=qb, ring_bf16=rb)
+    assert 0 < r["hits"] < wl.steps * wl.B * wl.Hkv
+
+
+@pytest.mark.parametrize("Hq,Hkv,L0", [(32, 1, (32768, 20000)), (64, 1, (24000, 30000)), (64, 4, (32768, 9000))])
+def test_mqa_all_miss_large(Hq, Hkv, L0):
+    """Large all-miss steps of multi-query groups: the rate-weighted split, a
+    single KV head's keys cut over every CTA (more than 100 partials per unit,
+    merged chunk by chunk)."""
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, Hq=Hq, Hkv=Hkv, L0=L0, steps=3)
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=0.0)
+    assert r["hits"] == 0
+
+
+def test_mqa_export_matches_oracle_window():
+    """The window of a 32-head group after a stream: positions and queries
+    equal to the oracle's, stored states within tolerance."""
+    import kv_cache_reuse_b200 as mac
+    wl = synth.WORKLOADS["tiny"].with_(Hq=32, Hkv=1, steps=30)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    r = compare_stream(wl, stream, cache)
+    st = mac.parse_state(r["gpu"].st.export_state(), wl.W, wl.G, wl.D)
+    q, o, m, l, pos = r["oracle"].window(0)
+    n = len(pos)
+    slots = [(wl.steps - n + i) % (wl.W + 1) for i in range(n)]
+    np.testing.assert_array_equal(st["pos"][0, slots], pos)
+    np.testing.assert_array_equal(st["q"][0, slots], q)
+    np.testing.assert_allclose(st["o"][0, slots], o, atol=OUT_TOL)
+    np.testing.assert_allclose(st["m"][0, slots] + np.log(st["l"][0, slots]), m + np.log(l), atol=LSE_TOL)
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (24, 8), (64, 8)])
 def test_group_sizes_all_miss_large(Hq, Hkv):
     """Large all-miss steps (weighted split, many partials per unit) for
@@ -377,7 +437,7 @@ def test_group_sizes_all_miss_large(Hq, Hkv):
     assert r["hits"] == 0
 
 
-@pytest.mark.parametrize("G", [1, 4])
+@pytest.mark.parametrize("G", [1, 4, 16, 64])
 def test_threshold_is_strict_and_ties_pick_the_most_recent(G):
     """Decisions at the edges the generator's margins stay away from: a
     distance exactly at the threshold misses and one ulp more of threshold

@@ -127,7 +127,7 @@ def _run(wl, steps=None, stream=None, cache=None, tau=None, band=None, rope_zero
     return stream, cache, res
 
 
-@pytest.mark.parametrize("G", [1, 4])
+@pytest.mark.parametrize("G", [1, 4, 16])
 def test_distance_equal_to_threshold_is_a_miss(G):
     """The match test is strict: an entry at distance exactly tau misses, and
     one ulp more of tau makes it a hit.  The queries are multiples of 1/8 and
@@ -202,10 +202,11 @@ def test_exact_repeats_without_rotation_equal_dense():
     assert nhit >= 6
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (6, 2), (8, 1)])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (6, 2), (8, 1), (32, 2), (32, 1), (64, 1)])
 def test_group_sizes_forced_miss_equals_dense(Hq, Hkv):
-    """Groups of 1 (multi-head), 3 and 8 query heads per KV head: a forced
-    miss is dense attention of every query head over its KV head."""
+    """Groups of 1 (multi-head), 3, 8, 16, 32 and 64 (multi-query) query heads
+    per KV head: a forced miss is dense attention of every query head over its
+    KV head."""
     wl = _tiny(steps=8, Hq=Hq, Hkv=Hkv)
     stream, cache, res = _run(wl, tau=0.0)
     for t, r in enumerate(res):
@@ -215,7 +216,7 @@ def test_group_sizes_forced_miss_equals_dense(Hq, Hkv):
         np.testing.assert_allclose(r.lse, l, rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(3, 3), (10, 2), (8, 1)])
+@pytest.mark.parametrize("Hq,Hkv", [(3, 3), (10, 2), (8, 1), (16, 1), (64, 1)])
 def test_group_sizes_band_covering_hits_equal_dense(Hq, Hkv):
     """With the band covering the context, hits reuse an empty prefix: the
     stored and reused states of every head in the group must come out exact."""
@@ -380,7 +381,7 @@ def _brute_match(window, q, tau, G):
     return False, -1
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (2, 2), (9, 3), (16, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (2, 2), (9, 3), (16, 2), (32, 1), (64, 2)])
 def test_match_equals_brute_force(Hq, Hkv):
     rng = np.random.default_rng(15)
     B, D, W = 2, 8, 4
@@ -433,6 +434,26 @@ def test_generator_labels_recovered_with_margin(name, steps):
                 assert (mpos[b] == stream.rope_pos[stream.src[t, b], b]).all(), (t, b)
                 assert (db[b] < 0.99 * wl.tau).all()
                 assert (ds[b] >= 1.01 * db[b]).all()
+            else:
+                assert not hit[b].any(), (t, b)
+                if t > 0:
+                    assert (db[b] > 1.01 * wl.tau).all()
+
+
+@pytest.mark.parametrize("Hq,Hkv,name", [(32, 1, "llama8b_32k"), (64, 1, "tiny"), (16, 1, "paged_mixed")])
+def test_mqa_generator_labels_recovered_with_margin(Hq, Hkv, name):
+    """Multi-query shapes (16 to 64 query heads over one KV head): repeats hit
+    their source step, fresh queries miss, with >= 1% distance margins."""
+    wl = synth.WORKLOADS[name].with_(Hq=Hq, Hkv=Hkv, B=min(synth.WORKLOADS[name].B, 4),
+                                     L0=synth.WORKLOADS[name].L0[:4])
+    stream = synth.queries(wl, 96)
+    orc = oracle.Oracle(wl.B, wl.Hq, wl.Hkv, wl.D, wl.W, wl.band, wl.tau, wl.rope_theta)
+    for t in range(stream.q.shape[0]):
+        hit, mpos, db, ds = orc.match_step(stream.q[t], stream.seq_lens[t])
+        for b in range(wl.B):
+            if stream.label[t, b]:
+                assert hit[b].all() and (mpos[b] == stream.rope_pos[stream.src[t, b], b]).all(), (t, b)
+                assert (db[b] < 0.99 * wl.tau).all() and (ds[b] >= 1.01 * db[b]).all()
             else:
                 assert not hit[b].any(), (t, b)
                 if t > 0:
