@@ -384,6 +384,14 @@ def run_mac(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = run_cpu_baseline(wl, stream, cache, args.cpu_seconds)
 
+    mqa = None
+    if args.mqa_steps > 0:
+        # multi-query groups: the workload's shape with 32 query heads over one KV
+        # head, every step a miss (the dense-decode bandwidth of the chunked
+        # kernel) and the workload's own repeat stream
+        wq = wl.with_(Hq=32, Hkv=1)
+        mqa = {"all_miss": run_shape(wq.with_(tau=0.0), args.mqa_steps, dev, peak, nwarm=3),
+               "mixed": run_shape(wq, args.mqa_steps, dev, peak)}
     hitshapes = []
     if args.hit_steps > 0 and args.hit_shapes:
         hitshapes = [run_hit_shape(n, args.hit_steps, dev, peak, world) for n in args.hit_shapes.split(",") if n]
@@ -429,6 +437,11 @@ def run_mac(args, rank, world, local_rank):
             roof["hit"]["vs_context"] = [
                 {"context": L, "step_us": r["total_ms"] * 1e3 / len(r["step_ms"]),
                  "attend_mb": r["att_bytes"] / len(r["step_ms"]) / 1e6} for L, r in hitctx]
+    if mqa:
+        a = mqa["all_miss"]["attend"]
+        roof.setdefault("miss", {})["mqa_32_1"] = {"frac": a["frac"], "achieved": a["achieved"], "mb_per_launch": a["mb_per_launch"],
+                                    "us_per_launch": a["us_per_launch"]}
+        detail["mqa_32_1"] = mqa
     res = {
         "metric": METRIC, "value": world * K_ / (tot * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K_,
         "warmup": args.warmup, "ms_per_step": tot / K_, "higher_is_better": True, "scaling": "weak",
@@ -484,16 +497,23 @@ def run_mac(args, rank, world, local_rank):
 
 
 def run_hit_shape(name, nsteps, dev, peak, world):
-    """The hit path alone on another workload's shape (every labelled step a
-    near-repeat of a recent query), with the windows filled first: the window
-    length of untimed steps, then nsteps steps timed with events before, between
-    and after the two kernels.  K/V values do not change the work of a step,
-    so the cache is drawn on the device (seeded N(0, 1), bf16) in the
-    workload's layout instead of on the host."""
+    """The hit path alone on another workload's shape: every labelled step a
+    near-repeat of a recent query."""
+    r = run_shape(synth.WORKLOADS[name].with_(hit_model=("iid", 1.0)), nsteps, dev, peak)
+    r["workload"] = "%s shape, every step a repeat" % name
+    return r
+
+
+def run_shape(wl, nsteps, dev, peak, nwarm=None):
+    """Steps of another workload shape, with the windows filled first (the
+    window length of untimed steps unless nwarm says otherwise), then nsteps
+    steps timed with events before, between and after the two kernels.  K/V
+    values do not change the work of a step, so the cache is drawn on the
+    device (seeded N(0, 1), bf16) in the workload's layout instead of on the
+    host."""
     import torch
     import kv_cache_reuse_b200 as mac
-    wl = synth.WORKLOADS[name].with_(hit_model=("iid", 1.0))
-    nwarm = wl.W
+    nwarm = wl.W if nwarm is None else nwarm
     T = nwarm + nsteps
     stream = synth.queries(wl, T)
     bt_h, max_seq, P = synth.kv_layout(wl, T)
@@ -544,7 +564,7 @@ def run_hit_shape(name, nsteps, dev, peak, world):
     m_ms = float(sum(e[0].elapsed_time(e[1]) for e in ev))
     a_ms = float(sum(e[1].elapsed_time(e[2]) for e in ev))
     step_ms = float(sum(e[0].elapsed_time(e[2]) for e in ev))
-    return {"workload": "%s shape, every step a repeat" % name, "batch": B, "window": wl.W, "band": wl.band,
+    return {"workload": wl.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "window": wl.W, "band": wl.band,
             "paged": bt_h is not None, "steps": nsteps, "hit_fraction": float(hits.mean()),
             "attend": {"mb_per_launch": at / nsteps / 1e6, "us_per_launch": a_ms * 1e3 / nsteps,
                        "achieved": at / (a_ms * 1e-3) / 1e9, "frac": at / (a_ms * 1e-3) / 1e9 / peak},
@@ -786,6 +806,8 @@ def main():
     ap.add_argument("--warm-start", action="store_true", help="also time seeding the windows from W positions")
     ap.add_argument("--layers", type=int, default=4,
                     help="also time a stack of this many layers per token, one CUDA graph per token (0 = skip)")
+    ap.add_argument("--mqa-steps", type=int, default=8,
+                    help="timed steps of the 32-query-heads-over-one-KV-head runs (0 = skip)")
     ap.add_argument("--hit-shapes", default="paged_mixed,continuous_16k",
                     help="workloads whose shapes also get an all-hit run (comma-separated, empty = none)")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16 query / window run")
