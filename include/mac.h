@@ -139,10 +139,11 @@ int mac_reset_seq(MacState *st, int b, void *stream);
  *               the match hit; may be NULL.
  *   match_pos   device int32 [B][Hkv] ([B][Hq] with match_per_head), position
  *               of the matched entry or -1; may be NULL.
- * The window of every unit advances by one entry.  Enqueues two kernels and
- * nothing else (no allocation, no host synchronisation), so the call can be
- * recorded into a CUDA graph -- e.g. one graph per token over all layers'
- * states -- and replayed; the recording holds the K/V addresses it saw.
+ * The window of every unit advances by one entry.  Enqueues one kernel (the
+ * one-launch step, see mac_set_one_launch) or two, and nothing else (no
+ * allocation, no host synchronisation), so the call can be recorded into a
+ * CUDA graph -- e.g. one graph per token over all layers' states -- and
+ * replayed; the recording holds the K/V addresses it saw.
  * Reproducibility: hit/miss decisions never depend on the work split, but
  * on large steps (at least 4096 keys of work per SM) the split learns each
  * SM's streaming rate from earlier steps by default, so the order in which
@@ -245,6 +246,23 @@ int mac_set_piece_cost(MacState *st, int keys);
  * cut over several CTAs and merged by the last of them.  0 cuts every
  * range. */
 int mac_set_whole_unit_keys(MacState *st, int keys);
+
+/* One-launch step.  For groups of up to 8 query heads per KV head with one
+ * decision per KV head (no per-head matching), and at most two units per SM,
+ * mac_decode_step runs the whole step as one cooperative launch of one CTA
+ * per SM: each CTA matches its own units and finishes every unit with at
+ * most whole_unit_keys fresh keys (every hit) on the spot; the last CTA to
+ * finish matching lays out the longer ranges (the misses) over all SMs, each
+ * SM's range shortened by the whole units it already carries, and the CTAs
+ * then stream them.  A hit step then costs one launch and no serial layout.
+ * on = 1 (default): use it where the configuration allows; 0: two launches
+ * (mac_match, then mac_attend), as every other configuration runs.  Both
+ * give the same decisions; outputs agree within rounding.  MAC_ERR_ARG for
+ * a NULL state or another value. */
+int mac_set_one_launch(MacState *st, int on);
+
+/* 1 if mac_decode_step on this state runs as one launch, else 0. */
+int mac_one_launch(const MacState *st);
 
 /* Reproducible work split.  on = 1: every step splits the key ranges evenly
  * over the CTAs and no streaming rate is learned or used, so a step's out and

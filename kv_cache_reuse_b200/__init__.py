@@ -315,6 +315,14 @@ def mac_set_reproducible(st, on: int) -> None:
     check("mac_set_reproducible", load().mac_set_reproducible(_h(st), int(on)))
 
 
+def mac_set_one_launch(st, on: int) -> None:
+    check("mac_set_one_launch", load().mac_set_one_launch(_h(st), int(on)))
+
+
+def mac_one_launch(st) -> int:
+    return int(load().mac_one_launch(_h(st)))
+
+
 def mac_attend_grid(st) -> int:
     return int(load().mac_attend_grid(_h(st)))
 

@@ -30,6 +30,8 @@ SIGNATURES = {
     "mac_set_whole_unit_keys": (C.c_int, [_P, C.c_int]),
     "mac_warm_start": (C.c_int, [_P, C.c_int, _P, _P, _P, _P, _P, _P, _P]),
     "mac_set_reproducible": (C.c_int, [_P, C.c_int]),
+    "mac_set_one_launch": (C.c_int, [_P, C.c_int]),
+    "mac_one_launch": (C.c_int, [_P]),
     "mac_attend_grid": (C.c_int, [_P]),
     "mac_error_string": (C.c_char_p, [C.c_int]),
     "mac_selftest_wait_timeout": (C.c_int, [_P, _P]),

@@ -46,6 +46,12 @@ struct MacState {
   int* done = nullptr;
   float* dpart = nullptr;  // groups of 16-64 heads: each chunk's part of every entry's distance
   int* ucnt = nullptr;     // groups of 16-64 heads: chunk CTAs of a unit that arrived
+  // the one-launch step
+  int* smid_of = nullptr;  // [grid] SM of each CTA
+  int* rank_of = nullptr;  // [grid] range of each split slot
+  int* fsync = nullptr;    // {ticket, epoch}
+  int one_launch_ok = 0;   // the configuration can run the step as one launch
+  int one_launch = 1;      // ... and it does (mac_set_one_launch)
   unsigned* status = nullptr;
   double* inv_freq = nullptr;
   // staging of mac_decode_step_host: one packed block each way, on the
@@ -105,7 +111,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,   s->hplan,
-                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done, s->dpart, s->ucnt, s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done, s->dpart, s->ucnt, s->smid_of, s->rank_of, s->fsync, s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -268,6 +274,9 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->done, 1));
   A(alloc(&s->dpart, U * W1 * (size_t)group_chunks((int)G)));
   A(alloc(&s->ucnt, U));
+  A(alloc(&s->smid_of, (size_t)s->grid));
+  A(alloc(&s->rank_of, (size_t)s->grid));
+  A(alloc(&s->fsync, 2));
   A(alloc(&s->inv_freq, D / 2));
   s->off_q = 0;
   s->off_pos = up256(s->off_q + B * Hq * D * s->QES);
@@ -302,6 +311,7 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->unit_cnt, 0, U * sizeof(int)));
   A(cudaMemset(s->done, 0, sizeof(int)));
   A(cudaMemset(s->ucnt, 0, U * sizeof(int)));
+  A(cudaMemset(s->fsync, 0, 2 * sizeof(int)));
   A(cudaMemset(s->rate, 0, s->grid * sizeof(float)));
   A(cudaMemset(s->claim, 0, s->grid * sizeof(int)));
   {  // even shares until the first rates are measured
@@ -317,6 +327,16 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemcpy(s->inv_freq, inv, sizeof(double) * (D / 2), cudaMemcpyHostToDevice));
   free(inv);
   A(attend_prepare((int)D, (int)G));
+  // the one-launch step: groups of up to 8 heads, one decision per KV head,
+  // every CTA resident at once (a cooperative launch of one CTA per SM) and
+  // each CTA's whole units within its item cache
+  if (e == cudaSuccess && G <= (size_t)kMaxGroup && !cfg->match_per_head && U <= 2 * (size_t)s->grid) {
+    int coop = 0, nb = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, s->device) == cudaSuccess && coop &&
+        step_prepare((int)D, (int)G, &nb) == cudaSuccess && nb >= 1)
+      s->one_launch_ok = 1;
+    cudaGetLastError();
+  }
   A(cudaDeviceSynchronize());
   if (e != cudaSuccess) {
     free_all(s);
@@ -362,6 +382,15 @@ int mac_set_whole_unit_keys(MacState* s, int keys) {
   return MAC_OK;
 }
 
+int mac_set_one_launch(MacState* s, int on) {
+  if (!s || on < 0 || on > 1) return MAC_ERR_ARG;
+  s->one_launch = on;
+  drop_graph(s);
+  return MAC_OK;
+}
+
+int mac_one_launch(const MacState* s) { return s && s->one_launch && s->one_launch_ok ? 1 : 0; }
+
 int mac_set_reproducible(MacState* s, int on) {
   if (!s || on < 0 || on > 1) return MAC_ERR_ARG;
   s->reproducible = on;
@@ -380,12 +409,12 @@ int mac_match(MacState* s, const void* q_pre, const int* rope_pos, const int* bl
   return match_impl(s, s->cfg.tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream);
 }
 
-static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope_pos, const int* block_table,
-                      const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
+static int fill_match(MacState* s, float tau, const void* q_pre, const int* rope_pos, const int* block_table,
+                      const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos,
+                      MatchParams& p) {
   if (!s || !q_pre || !rope_pos || !seq_lens || !out || !lse) return MAC_ERR_ARG;
   if (!aligned16(q_pre)) return MAC_ERR_ARG;
   if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
-  MatchParams p;
   p.q_pre = q_pre;
   p.q_bf16 = s->cfg.q_bf16;
   p.ring_bf16 = s->cfg.ring_bf16;
@@ -430,11 +459,19 @@ static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope
   p.min_keys = s->min_keys;
   p.piece_cost = s->piece_cost;
   p.unit_max = s->G > kMaxGroup ? 0 : s->unit_max;  // groups of 16-64 heads run split items only
+  return MAC_OK;
+}
+
+static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope_pos, const int* block_table,
+                      const int* seq_lens, float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
+  MatchParams p;
+  const int rc = fill_match(s, tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, p);
+  if (rc != MAC_OK) return rc;
   return launch_match(p, s->D, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
-int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* block_table, float* out, float* lse,
-               void* stream) {
+static int fill_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* block_table, float* out,
+                       float* lse, AttendParams& p) {
   if (!s || !K || !V || !out || !lse) return MAC_ERR_ARG;
   if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
   if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
@@ -448,7 +485,6 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
     if (rc != MAC_OK) return rc;
     s->tm_v_ptr = V;
   }
-  AttendParams p;
   p.tmK = s->tmK;
   p.tmV = s->tmV;
   p.block_table = s->cfg.page_size > 0 ? block_table : nullptr;
@@ -481,6 +517,17 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
   p.grid = s->grid;
   p.per_head = s->cfg.match_per_head;
   p.ring_bf16 = s->cfg.ring_bf16;
+  p.smid_of = s->smid_of;
+  p.rank_of = s->rank_of;
+  p.fsync = s->fsync;
+  return MAC_OK;
+}
+
+int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* block_table, float* out, float* lse,
+               void* stream) {
+  AttendParams p;
+  const int rc = fill_attend(s, K, V, block_table, out, lse, p);
+  if (rc != MAC_OK) return rc;
   return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
 
@@ -489,6 +536,15 @@ int mac_decode_step(MacState* s, const void* q_pre, const int* rope_pos, const u
                     int* match_pos, void* stream) {
   if (!s || !K || !V) return MAC_ERR_ARG;
   if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
+  if (s->one_launch && s->one_launch_ok) {
+    // match, every whole unit and the split ranges in one cooperative launch
+    MatchParams mp;
+    AttendParams ap;
+    int rc = fill_match(s, s->cfg.tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, mp);
+    if (rc == MAC_OK) rc = fill_attend(s, K, V, block_table, out, lse, ap);
+    if (rc != MAC_OK) return rc;
+    return launch_step(ap, mp, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
+  }
   int rc = mac_match(s, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream);
   if (rc != MAC_OK) return rc;
   return mac_attend(s, K, V, block_table, out, lse, stream);

@@ -60,6 +60,7 @@
 #include <cuda_bf16.h>
 
 #include "mac_internal.cuh"
+#include "mac_match_dev.cuh"
 
 #include "../../include/mac.h"
 
@@ -107,6 +108,7 @@ struct __align__(1024) AttnSmem {
   int last_flag;
   int box_total;                     // boxes consumed by all warps (rate record)
   Segment items[kItemCache];         // the CTA's work items, from its first one on
+  int nlocal;                        // one-launch step: whole units this CTA matched (in items)
   alignas(16) float ring[C::SF];     // that ring state: o [G][D], then m at GD, l at GD + GP
 };
 
@@ -172,6 +174,24 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                    smem_u32(dst)),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_u32(const int* ptr) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(int* ptr, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+// A work item read through L2 (the one-launch step's items are written by
+// another CTA of the same launch, so no SM may serve an old copy from L1).
+static_assert(sizeof(Segment) == 32, "a work item is two 16-byte loads");
+__device__ __forceinline__ Segment load_segment(const Segment* src) {
+  const int4 a = __ldcg(reinterpret_cast<const int4*>(src)), b = __ldcg(reinterpret_cast<const int4*>(src) + 1);
+  Segment sg;
+  memcpy(reinterpret_cast<int4*>(&sg), &a, 16);
+  memcpy(reinterpret_cast<int4*>(&sg) + 1, &b, 16);
+  return sg;
 }
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;
@@ -583,10 +603,11 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
   const int Gt = NC > 1 ? GF : G;                                           // heads of the unit
   const int PF = NC > 1 ? (int)partial_floats(Gt, D) : GD + 2 * G4;         // floats of one partial
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // plan and items may come from other CTAs of the same launch: read through L2
   const UnitPlan* const pp = p.plan + u;
-  const int src_slot = pp->src_slot, dst_slot = pp->dst_slot, end = pp->end;
-  const int hmask = PH ? p.hplan[u].hmask : (pp->hit ? (1 << G) - 1 : 0);  // heads with a reused state
-  const Segment sA = p.seg[2 * u], sB = p.seg[2 * u + 1];
+  const int src_slot = __ldcg(&pp->src_slot), dst_slot = __ldcg(&pp->dst_slot), end = __ldcg(&pp->end);
+  const int hmask = PH ? p.hplan[u].hmask : (__ldcg(&pp->hit) ? (1 << G) - 1 : 0);  // heads with a reused state
+  const Segment sA = load_segment(p.seg + 2 * u), sB = load_segment(p.seg + 2 * u + 1);
   const int nA = sA.npieces, nB = sB.npieces, n = nA + nB;
   int wA = kConsumerWarps;
   if (nB > 0) {
@@ -744,7 +765,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D
   if (threadIdx.x == 0) {
     __threadfence();
     const int old = atomicAdd(p.unit_cnt + unit, 1);
-    sm.last_flag = (old == p.plan[unit].expected - 1);
+    sm.last_flag = (old == __ldcg(&p.plan[unit].expected) - 1);
   }
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
@@ -832,16 +853,19 @@ struct Walker {
   long long lo, hi;
   const Segment* cache;  // shared-memory copy of items [base, base + kItemCache)
   int base;
-  __device__ __forceinline__ bool next(const AttendParams& p, int cta, Piece& pc) {
-    while (s < p.nseg) {
-      const Segment sg = (s - base < kItemCache) ? cache[s - base] : p.seg[s];
+  const Segment* table;  // the items
+  int nseg;
+  bool local;            // a CTA's own whole units: flat holds the unit (else item 2u, 2u+1 is unit u)
+  __device__ __forceinline__ bool next(int cta, Piece& pc) {
+    while (s < nseg) {
+      const Segment sg = (local || s - base < kItemCache) ? cache[s - base] : load_segment(table + s);
       const int cur = s++;
       if (sg.kind < 0) continue;
-      if (sg.flat >= hi) {  // this and every later item start past the range
-        s = p.nseg;
+      if (!local && sg.flat >= hi) {  // this and every later item start past the range
+        s = nseg;
         return false;
       }
-      pc.unit = cur >> 1;
+      pc.unit = local ? (int)sg.flat : cur >> 1;
       if (sg.kind == kItemWhole) {
         if (sg.first_cta != cta) continue;  // owned by the CTA whose range holds its start
         const int start = sg.key0, cut = sg.pbase, end = sg.key0 + sg.len;
@@ -933,8 +957,16 @@ __device__ __noinline__ void rate_shares(const AttendParams& p) {
 // every reader of the slot has released it (an mbarrier with NC arrivals), so
 // each K/V byte crosses from HBM once for all 8 NC heads.  Such groups run
 // split items only.
-template <int D, int GP, int GF, bool PH, int NC = 1>
-__global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
+//
+// FUSED (the one-launch step, mac_step.cu): the CTAs first run the match
+// stage of their own units (unit u on CTA u mod grid), do every whole unit
+// they matched on the spot (no other CTA is involved), then take the range
+// of the step's split items that the last CTA to finish matching laid out
+// (build_split_table) and stream it as the attention kernel does.  Needs all
+// CTAs resident at once (a cooperative launch): a CTA waits, bounded, for
+// the layout.
+template <int D, int GP, int GF, bool PH, int NC, bool FUSED, bool RB>
+__device__ __forceinline__ void attend_body(const AttendParams& p, const MatchParams& mp) {
   using C = Cfg<D, GP>;
   constexpr int NST = C::NST, NQ = C::NQ;
   constexpr int NKL = kConsumerWarps / NC, NSTT = NST * NC;  // key-lanes; box slots of one key-lane
@@ -982,54 +1014,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  // launched with programmatic stream serialization: everything above
-  // overlaps the match kernel; its results are visible after this wait
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // one round of loads: the split, then the CTA's items into shared memory
   unsigned smid;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-  const int n_cta = p.hdr->n_cta, weighted = p.hdr->weighted;
-  const long long T = p.hdr->total;
-  int first_seg = p.first_seg[cta];
-  // a weighted split: take the range of this SM (claimed in the same round
-  // of loads), else the first free one
-  int mine = 0;
-  if (tid == 0 && p.claim != nullptr && (int)smid < p.grid) mine = atomicCAS(p.claim + smid, 0, 1) == 0;
-  int slot = cta;
-  long long lo, hi;
-  if (weighted) {
-    if (tid == 0) {
-      int c = mine ? (int)smid : -1;
-      for (int k = 0; c < 0 && k < n_cta; ++k)
-        if (atomicCAS(p.claim + k, 0, 1) == 0) c = k;
-      sm.last_flag = c;
-    }
-    __syncthreads();
-    slot = sm.last_flag;
-    if (slot < 0) return;  // never: n_cta = grid ranges for grid CTAs
-    lo = p.bounds[slot];
-    hi = p.bounds[slot + 1];
-    first_seg = p.first_seg[slot];
-  } else {
-    if (cta >= n_cta) return;
-    lo = (long long)cta * T / n_cta;
-    hi = (long long)(cta + 1) * T / n_cta;
-  }
-  if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = p.seg[first_seg + tid];
-  __syncthreads();
   const uint64_t pol = evict_first_policy();
 
-  // issue cursor: this warp's (NC > 1: this key-lane's) boxes of every piece, NSTT ahead
+  // cursors, counters and barrier phases of this CTA; they carry over from
+  // one walk to the next (the box slots' phases follow the box counts)
+  int ipn = 0, nissued = 0, nq_issued = 0;    // issue side: pieces passed, boxes and queries issued
+  Acc<D, GP> A;
+  int cpn = 0, cons = 0, par = 0;             // consume side: pieces and boxes done
+  uint32_t sync_phase = 0, ring_phase = 0;
+  bool ring_pending = false;  // a reused-state copy was issued and not yet waited for
+  bool ok = true;
+  unsigned long long t_first = 0, t_last = 0;  // thread 0: first and last box of the timed walk
+  int cons0 = 0;                               // boxes consumed before the timed walk
   auto range_of = [&](const Piece& pc) { return NC == 1 ? warp_range(pc, warp) : team_range(pc, kl, NKL); };
-  Walker wi{first_seg, lo, hi, sm.items, first_seg};
+
+  // One walk over the items of `table` from first_seg on whose cost range
+  // meets [lo, hi), as range `slot` of the table's split.
+  auto walk = [&](const Segment* table, int nseg, int first_seg, long long lo, long long hi, int slot,
+                  bool timed, bool local) {
+  // issue cursor: this warp's (NC > 1: this key-lane's) boxes of every piece, NSTT ahead
+  Walker wi{first_seg, lo, hi, sm.items, first_seg, table, nseg, local};
   Piece ip;
   WarpRange ir;
-  bool ivalid = issuer && wi.next(p, slot, ip);
+  bool ivalid = issuer && wi.next(slot, ip);
   if (ivalid) ir = range_of(ip);
-  int ib = ivalid ? ir.first : 0, ipn = 0, nissued = 0, nq_issued = 0;
+  int ib = ivalid ? ir.first : 0;
   auto issue_advance = [&]() {
     while (ivalid && ib >= ir.nbox) {
-      ivalid = wi.next(p, slot, ip);
+      ivalid = wi.next(slot, ip);
       if (ivalid) {
         ir = range_of(ip);
         ib = ir.first;
@@ -1075,15 +1089,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
   for (int k = 0; k < NSTT && ivalid; ++k) issue_box(k);
 
   // consume cursor
-  Acc<D, GP> A;
-  Walker wc{first_seg, lo, hi, sm.items, first_seg};
+  Walker wc{first_seg, lo, hi, sm.items, first_seg, table, nseg, local};
   Piece cp;
-  int cpn = 0, cons = 0, par = 0;
-  uint32_t sync_phase = 0, ring_phase = 0;
-  bool ring_pending = false;  // a reused-state copy was issued and not yet waited for
-  bool ok = true;
-  unsigned long long t_first = 0, t_last = 0;  // thread 0: first and last box consumed
-  while (ok && wc.next(p, slot, cp)) {
+  if (timed) cons0 = cons;
+  while (ok && wc.next(slot, cp)) {
     if constexpr (NC == 1) {
       const int qs = cpn % NQ;
       if (!mbar_wait(&sm.qfull[qs], (uint32_t)(cpn / NQ) & 1u, &sm.abort_flag, p.status)) break;
@@ -1154,7 +1163,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
         ok = false;
         break;
       }
-      if (tid == 0 && cons == 0) t_first = globaltimer();
+      if (timed && tid == 0 && cons == cons0) t_first = globaltimer();
       const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * C::PB;
       uint16_t* kbuf = kv_slot(st);
@@ -1182,7 +1191,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
       }
     }
     if (!ok) break;
-    if (tid == 0) t_last = globaltimer();
+    if (timed && tid == 0) t_last = globaltimer();
     bool fin;
     if constexpr (NC > 1)
       fin = finalize_piece<D, GP, GF, PH, NC>(p, sm, A, cp.unit, cp.pidx, sync_phase);
@@ -1192,13 +1201,146 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
                      : finalize_piece<D, GP, GF, PH>(p, sm, A, cp.unit, cp.pidx, sync_phase);
     if (ring_copy) ring_phase ^= 1u;
     ring_pending = false;
-    if (!fin) break;
+    if (!fin) {
+      ok = false;
+      break;
+    }
     ++cpn;
+  }
+  };  // walk
+
+  int weighted = 0;
+  int first_seg = 0, slot = cta;
+  long long lo = 0, hi = 0;
+  if constexpr (FUSED) {
+    // ---- the one-launch step: match, whole units on the spot, then the split range
+    const int U = mp.B * mp.Hkv;
+    using MS = MatchSmem<D, GP, false>;
+    static_assert(sizeof(MS) <= sizeof(sm.kv), "match scratch lives in the box slots");
+    MS& ms = *reinterpret_cast<MS*>(&sm.kv[0][0][0][0]);
+    if (tid == 0) {
+      sm.nlocal = 0;
+      sm.last_flag = (int)ld_acquire_u32(p.fsync + 1);  // this launch's epoch, before its ticket
+    }
+    __syncthreads();
+    // match stage of this CTA's units; whole units become local items
+#pragma unroll 1
+    for (int u = cta; u < U; u += gridDim.x) {
+      match_body<D, GP, GF, false, RB>(mp, u, ms);
+      __syncthreads();
+      if (tid == 0) {
+        const UnitPlan pl = ms.s_plan;
+        if (!(pl.bad || ms.s_bad_page) && pl.end - pl.start <= mp.unit_max && sm.nlocal < kItemCache) {
+          Segment sg;
+          sg.kind = kItemWhole;
+          sg.flat = u;  // a local item carries its unit
+          sg.len = pl.end - pl.start;
+          sg.key0 = pl.start;
+          sg.first_cta = cta;
+          sg.pbase = pl.cut;
+          sg.npieces = (pl.hit ? 1 : 0) | ((pl.hit && pl.src_slot >= 0 ? pl.src_slot & 0x7ff : 0) << 1) |
+                       ((pl.dst_slot & 0x7ff) << 12);
+          sm.items[sm.nlocal++] = sg;
+        }
+      }
+    }
+    const unsigned epoch = (unsigned)sm.last_flag;
+    // the box slots held the match scratch, and the bulk copies of this launch
+    // read the rotated queries just written: order those generic writes (shared
+    // and global) before any copy, then publish them device-wide
+    asm volatile("fence.proxy.async;" ::: "memory");
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      p.smid_of[cta] = (int)smid;
+      int ticket;
+      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(p.fsync) : "memory");
+      sm.last_flag = (ticket == (int)gridDim.x - 1);
+    }
+    __syncthreads();
+    if (sm.last_flag) {
+      // every CTA's plans and SM id precede its ticket: lay out the split items
+      __threadfence();
+      static_assert(sizeof(SplitScratch) <= sizeof(sm.kv), "split scratch lives in the box slots");
+      build_split_table(mp, U, (int)gridDim.x, p.smid_of, p.rank_of,
+                        *reinterpret_cast<SplitScratch*>(&sm.kv[0][0][0][0]));
+      asm volatile("fence.proxy.async;" ::: "memory");  // the scratch in the box slots, before copies
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        p.fsync[0] = 0;
+        st_release_u32(p.fsync + 1, epoch + 1u);
+      }
+    }
+    __syncthreads();
+    // this CTA's whole units
+    const int nlocal = sm.nlocal;
+    if (nlocal > 0) walk(sm.items, nlocal, 0, 0, LLONG_MAX, cta, false, true);
+    // the step's split table (bounded wait for the last CTA's layout)
+    if (tid == 0 && ok) {
+      const unsigned long long t0 = globaltimer();
+      while (ld_acquire_u32(p.fsync + 1) != epoch + 1u) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          atomicOr(p.status, MAC_DEV_TIMEOUT);
+          sm.abort_flag = 1;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    // (written by another CTA of this launch: read through L2)
+    if (ok && !sm.abort_flag && __ldcg(&p.hdr->total) > 0) {
+      weighted = __ldcg(&p.hdr->weighted);
+      const int rank = __ldcg(p.rank_of + (weighted ? (int)smid : cta));
+      if (rank >= 0) {
+        slot = rank;
+        lo = __ldcg(p.bounds + rank);
+        hi = __ldcg(p.bounds + rank + 1);
+        first_seg = __ldcg(p.first_seg + rank);
+      }
+    }
+    ok = ok && !sm.abort_flag;
+  } else {
+    // launched with programmatic stream serialization: everything above
+    // overlaps the match kernel; its results are visible after this wait
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // one round of loads: the split, then the CTA's items into shared memory
+    const int n_cta = p.hdr->n_cta;
+    weighted = p.hdr->weighted;
+    const long long T = p.hdr->total;
+    first_seg = p.first_seg[cta];
+    // a weighted split: take the range of this SM (claimed in the same round
+    // of loads), else the first free one
+    int mine = 0;
+    if (tid == 0 && p.claim != nullptr && (int)smid < p.grid) mine = atomicCAS(p.claim + smid, 0, 1) == 0;
+    if (weighted) {
+      if (tid == 0) {
+        int c = mine ? (int)smid : -1;
+        for (int k = 0; c < 0 && k < n_cta; ++k)
+          if (atomicCAS(p.claim + k, 0, 1) == 0) c = k;
+        sm.last_flag = c;
+      }
+      __syncthreads();
+      slot = sm.last_flag;
+      if (slot < 0) return;  // never: n_cta = grid ranges for grid CTAs
+      lo = p.bounds[slot];
+      hi = p.bounds[slot + 1];
+      first_seg = p.first_seg[slot];
+    } else {
+      if (cta >= n_cta) return;
+      lo = (long long)cta * T / n_cta;
+      hi = (long long)(cta + 1) * T / n_cta;
+    }
+  }
+  if (ok && lo < hi) {
+    if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = load_segment(p.seg + first_seg + tid);
+    __syncthreads();
+    walk(p.seg, p.nseg, first_seg, lo, hi, slot, true, false);
   }
   if (weighted && p.rate != nullptr) {
     // fold this SM's streaming rate (boxes per microsecond) into its record;
     // only CTAs that mostly streamed (at least kRateMinBoxes boxes) measure it
-    if (lane == 0 && issuer) atomicAdd(&sm.box_total, cons);  // each box once, by the warp that filled it
+    if (lane == 0 && issuer) atomicAdd(&sm.box_total, cons - cons0);  // each box once, by the warp that filled it
     __syncthreads();
     const int boxes = sm.box_total;
     if (ok && tid == 0 && (int)smid < p.grid && boxes >= kRateMinBoxes && t_last > t_first + 2000) {
@@ -1230,6 +1372,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __gri
     }
     __syncwarp();
   }
+}
+
+template <int D, int GP, int GF, bool PH, int NC = 1>
+__global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_kernel(const __grid_constant__ AttendParams p) {
+  attend_body<D, GP, GF, PH, NC, false, false>(p, MatchParams{});
+}
+
+// The whole decode step in one cooperative launch (groups of up to 8 heads,
+// one decision per KV head): match, every whole unit by the CTA that matched
+// it, then the split ranges.  RB: the window's queries are stored in bf16.
+template <int D, int GP, int GF, bool RB>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    mac_step_kernel(const __grid_constant__ AttendParams p, const __grid_constant__ MatchParams mp) {
+  attend_body<D, GP, GF, false, 1, true, RB>(p, mp);
 }
 
 // Failure-path self-test: one warp waits, through the kernels' bounded wait,
@@ -1299,6 +1455,94 @@ cudaError_t launch_d(cudaLaunchConfig_t& cfg, const AttendParams& p) {
   return cudaLaunchKernelEx(&cfg, mac_attend_kernel<D, 8, 0, false>, p);
 }
 }  // namespace
+
+namespace {
+template <int D, bool RB>
+const void* step_kernel(int G) {
+  if (G == 4) return reinterpret_cast<const void*>(mac_step_kernel<D, 4, 4, RB>);
+  if (G == 8) return reinterpret_cast<const void*>(mac_step_kernel<D, 8, 8, RB>);
+  if (G < 4) return reinterpret_cast<const void*>(mac_step_kernel<D, 4, 0, RB>);
+  return reinterpret_cast<const void*>(mac_step_kernel<D, 8, 0, RB>);
+}
+template <int D, bool RB>
+cudaError_t step_launch_d(cudaLaunchConfig_t& cfg, const AttendParams& p, const MatchParams& mp) {
+  const int G = p.G;
+  if (G == 4) return cudaLaunchKernelEx(&cfg, mac_step_kernel<D, 4, 4, RB>, p, mp);
+  if (G == 8) return cudaLaunchKernelEx(&cfg, mac_step_kernel<D, 8, 8, RB>, p, mp);
+  if (G < 4) return cudaLaunchKernelEx(&cfg, mac_step_kernel<D, 4, 0, RB>, p, mp);
+  return cudaLaunchKernelEx(&cfg, mac_step_kernel<D, 8, 0, RB>, p, mp);
+}
+}  // namespace
+
+// Shared memory of one CTA of the one-launch step: the attention layout, but
+// more than half of an SM, so that no SM ever holds two of its CTAs (the
+// split's ranges are keyed by SM on large steps).
+size_t step_smem_bytes(int D, int G) {
+  static int half = -1;
+  if (half < 0) {
+    int dev = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess)
+      half = per_sm / 2 + 1024;
+    else
+      half = 0;
+  }
+  const size_t need = attend_smem_bytes(D, G);
+  return need > (size_t)half ? need : (size_t)half;
+}
+
+namespace {
+template <int D, int GP, int GF, bool RB>
+cudaError_t step_smem_set(size_t bytes) {
+  return cudaFuncSetAttribute(mac_step_kernel<D, GP, GF, RB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)bytes);
+}
+template <int D, bool RB>
+cudaError_t step_smem_set_all(size_t b4, size_t b8) {
+  cudaError_t e = step_smem_set<D, 4, 4, RB>(b4);
+  if (e == cudaSuccess) e = step_smem_set<D, 4, 0, RB>(b4);
+  if (e == cudaSuccess) e = step_smem_set<D, 8, 8, RB>(b8);
+  if (e == cudaSuccess) e = step_smem_set<D, 8, 0, RB>(b8);
+  return e;
+}
+}  // namespace
+
+cudaError_t step_prepare(int D, int G, int* blocks_per_sm) {
+  *blocks_per_sm = 0;
+  if ((D != 64 && D != 128) || G < 1 || G > kMaxGroup) return cudaErrorInvalidValue;
+  const size_t b4 = step_smem_bytes(D, 4), b8 = step_smem_bytes(D, 8);
+  cudaError_t e = D == 128 ? step_smem_set_all<128, false>(b4, b8) : step_smem_set_all<64, false>(b4, b8);
+  if (e == cudaSuccess) e = D == 128 ? step_smem_set_all<128, true>(b4, b8) : step_smem_set_all<64, true>(b4, b8);
+  if (e != cudaSuccess) return e;
+  // the launch needs every CTA resident at once: one per SM
+  int nb = 0, nb2 = 0;
+  const size_t smem = step_smem_bytes(D, G);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, D == 128 ? step_kernel<128, false>(G) : step_kernel<64, false>(G),
+                                                    kAttnThreads, smem);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb2, D == 128 ? step_kernel<128, true>(G)
+                                                                      : step_kernel<64, true>(G),
+                                                      kAttnThreads, smem);
+  *blocks_per_sm = nb < nb2 ? nb : nb2;
+  return e;
+}
+
+cudaError_t launch_step(const AttendParams& p, const MatchParams& mp, int D, int grid, cudaStream_t s) {
+  if ((D != 64 && D != 128) || p.G < 1 || p.G > kMaxGroup || p.per_head || mp.per_head)
+    return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: they wait for the split table
+  attr[0].val.cooperative = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kAttnThreads);
+  cfg.dynamicSmemBytes = step_smem_bytes(D, p.G);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) return mp.ring_bf16 ? step_launch_d<128, true>(cfg, p, mp) : step_launch_d<128, false>(cfg, p, mp);
+  return mp.ring_bf16 ? step_launch_d<64, true>(cfg, p, mp) : step_launch_d<64, false>(cfg, p, mp);
+}
 
 cudaError_t attend_prepare(int D, int G) {
   if ((D != 64 && D != 128) || !group_ok(G)) return cudaErrorInvalidValue;

@@ -148,6 +148,9 @@ struct AttendParams {
   double* cw;        // [grid + 1] cumulative range shares (written by CTA 0)
   float* part;       // [max_parts][partial_floats(G, D)]
   int* unit_cnt;     // [U]
+  int* smid_of;      // one-launch step: [grid] SM of each CTA
+  int* rank_of;      // one-launch step: [grid] range of each split slot (-1: none)
+  int* fsync;        // one-launch step: {CTAs that finished matching, epoch of the published split}
   void* ring_o;      // [U][W+1][G][D] fp32, or bf16 bits (ring_bf16)
   float* ring_m;     // [U][W+1][G]
   float* ring_l;     // [U][W+1][G]
@@ -176,6 +179,10 @@ cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s);
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t attend_prepare(int D, int G);
+// The one-launch step (groups of up to 8 heads, one decision per KV head):
+// prepare sets its kernels' attributes and reports how many CTAs fit on an SM.
+cudaError_t step_prepare(int D, int G, int* blocks_per_sm);
+cudaError_t launch_step(const AttendParams& p, const MatchParams& mp, int D, int grid, cudaStream_t s);
 cudaError_t launch_wait_selftest(unsigned* status, cudaStream_t s);
 size_t attend_smem_bytes(int D, int G);
 

@@ -334,6 +334,42 @@ def test_reproducible_split_gives_identical_bits():
     assert a.st.get_status() == 0 and b.st.get_status() == 0
 
 
+def test_one_launch_is_used_where_it_applies():
+    """Groups of up to 8 heads with one decision per KV head run the step as
+    one launch by default; per-head matching, groups of 16-64 heads and the
+    switch mac_set_one_launch(0) run two."""
+    import kv_cache_reuse_b200 as mac
+    tiny = synth.WORKLOADS["tiny"]
+    cache = synth.kv_cache(tiny.with_(steps=2))
+    assert mac.mac_one_launch(DeviceRun(tiny, cache).st) == 1
+    assert mac.mac_one_launch(DeviceRun(tiny, cache, tune={"one_launch": 0}).st) == 0
+    assert mac.mac_one_launch(DeviceRun(tiny, cache, per_head=1).st) == 0
+    assert mac.mac_one_launch(DeviceRun(tiny.with_(Hq=32), cache).st) == 0
+
+
+@pytest.mark.parametrize("case", ["tiny", "llama", "paged", "weighted_all_miss", "many_units", "bf16"])
+def test_two_launch_path(case):
+    """mac_decode_step with the one-launch step switched off: the match kernel
+    (which lays out every unit's items) and the attention kernel launched one
+    after the other, against the oracle."""
+    tiny, llama, paged = synth.WORKLOADS["tiny"], synth.WORKLOADS["llama8b_32k"], synth.WORKLOADS["paged_mixed"]
+    tau, rb = None, 0
+    if case == "tiny":
+        wl = tiny.with_(steps=40)
+    elif case == "llama":
+        wl = llama.with_(L0=(9000,), steps=40)
+    elif case == "paged":
+        wl = paged.with_(B=4, L0=(9000, 1500, 300, 4100), steps=16)
+    elif case == "weighted_all_miss":
+        wl, tau = llama.with_(B=4, L0=(32768, 30000, 31000, 29000), steps=4), 0.0
+    elif case == "many_units":
+        wl = tiny.with_(B=40, Hq=16, Hkv=4, L0=tuple(200 + 37 * i for i in range(40)), steps=6)
+    else:
+        wl, rb = llama.with_(L0=(6000,), steps=24), 1
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl), tau=tau, ring_bf16=rb, tune={"one_launch": 0})
+    assert r["gpu"].st is not None
+
+
 _SPLIT = {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 64}
 
 
