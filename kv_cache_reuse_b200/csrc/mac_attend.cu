@@ -1086,7 +1086,9 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     issue_advance();
   };
   issue_advance();
-  for (int k = 0; k < NSTT && ivalid; ++k) issue_box(k);
+  // the first boxes of the walk go to the slots after the previous walk's last
+  // (the consume side reads box n from slot n mod NSTT)
+  for (int k = 0; k < NSTT && ivalid; ++k) issue_box(nissued % NSTT);
 
   // consume cursor
   Walker wc{first_seg, lo, hi, sm.items, first_seg, table, nseg, local};
@@ -1288,6 +1290,9 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       }
     }
     __syncthreads();
+    // the split pieces' queries were written by other CTAs of this launch and
+    // are read by bulk copies: order the acquire before those copies
+    asm volatile("fence.proxy.async.global;" ::: "memory");
     // (written by another CTA of this launch: read through L2)
     if (ok && !sm.abort_flag && __ldcg(&p.hdr->total) > 0) {
       weighted = __ldcg(&p.hdr->weighted);
