@@ -275,6 +275,7 @@ def run_mac(args, rank, world, local_rank):
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
         status = st.get_status()
+        one = mac.mac_one_launch(st) if not split else 0
         st.close()
         step_ms = [a.elapsed_time(c) for a, b_, c in ev]
         att_ms = [b_.elapsed_time(c) for a, b_, c in ev] if split else [0.0] * nsteps
@@ -295,6 +296,7 @@ def run_mac(args, rank, world, local_rank):
             dense_b += synth.dense_equiv_kv_bytes(wl, cur["stream"].seq_lens[t])
         tot_ms = float(np.sum(step_ms))
         return dict(total_ms=tot_ms, step_ms=step_ms, att_ms=float(np.sum(att_ms)), match_ms=float(np.sum(match_ms)),
+                    one_launch=one,
                     att_bytes=at_b, match_bytes=mt_b, kv_bytes=kv_b, dense_bytes=dense_b,
                     hit_frac=float(hits.mean()), status=status, clocks=clocks.summary())
 
@@ -305,7 +307,11 @@ def run_mac(args, rank, world, local_rank):
         main = timed_run(wl.tau, args.warmup, args.steps, split=False)
     main["clocks"]["remeasured"] = remeasured
     kern = timed_run(wl.tau, args.warmup, args.steps, split=True)
-    allmiss = timed_run(0.0, 3, min(args.miss_steps, T - 3), split=True) if args.miss_steps > 0 else None
+    allmiss = allmiss2 = None
+    if args.miss_steps > 0:
+        nm = min(args.miss_steps, T - 3)
+        allmiss = timed_run(0.0, 3, nm, split=False)   # the step as it runs (one launch where it applies)
+        allmiss2 = timed_run(0.0, 3, nm, split=True)   # the two kernels timed apart
     warm = None
     if args.warm_start:
         # seed the windows from the first W positions of the stream (as prefill
@@ -344,14 +350,15 @@ def run_mac(args, rank, world, local_rank):
         perhead = (timed_run(wl.tau, args.warmup, args.steps, split=False, cfg=cfg),
                    timed_run(wl.tau, args.warmup, args.steps, split=True, cfg=cfg))
         cur["q"] = q_all
-    hitrun = None
+    hitrun = hitrun2 = None
     hitctx = []
     if args.hit_steps > 0:
         # the hit path alone: the same shape with every labelled step a near-repeat
         qh = synth.queries(wl.with_(hit_model=("iid", 1.0)), T).q
         cur["q"] = torch.from_numpy(qh).to(dev)
         # the windows filled first (W untimed steps), so every timed step scans a full window
-        hitrun = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=True)
+        hitrun = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=False)
+        hitrun2 = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=True)
         cur["q"] = q_all
         if not cache.paged:
             # the same hit stream at shorter contexts, on the same cache: a hit's
@@ -360,7 +367,7 @@ def run_mac(args, rank, world, local_rank):
                 sc = synth.queries(wl.with_(hit_model=("iid", 1.0), L0=(L,) * B), T)
                 cur.update(q=torch.from_numpy(sc.q).to(dev), pos=torch.from_numpy(sc.rope_pos).to(dev),
                            lens=torch.from_numpy(sc.seq_lens).to(dev), stream=sc)
-                r = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=True)
+                r = timed_run(wl.tau, wl.W, min(args.hit_steps, T - wl.W), split=False)
                 hitctx.append((L, r))
             cur.update(q=q_all, pos=pos_all, lens=lens_all, stream=stream)
             hitctx.append((int(wl.L0[0]), hitrun))
@@ -399,44 +406,57 @@ def run_mac(args, rank, world, local_rank):
     if rank != 0:
         return None
     K_ = args.steps
-    att_gbs = kern["att_bytes"] / (kern["att_ms"] * 1e-3) / 1e9
-    ratio = _profiled_traffic()
-    # traffic per launch: the profiled DRAM/algorithmic ratio scaled to this run's launches
-    traffic = ratio * kern["att_bytes"] / K_ if ratio else None
+    gbs = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9
+
+    def two_launch(r, n):
+        """The same steps with the match and attention kernels launched (and timed) apart."""
+        a, m = gbs(r["att_bytes"], r["att_ms"]), gbs(r["match_bytes"], r["match_ms"])
+        return {"attend": {"kernel": "mac_attend_kernel", "achieved": a, "frac": a / peak,
+                           "mb_per_launch": r["att_bytes"] / n / 1e6, "us_per_launch": r["att_ms"] * 1e3 / n},
+                "match": {"kernel": "mac_match_kernel", "achieved": m, "frac": m / peak,
+                          "mb_per_launch": r["match_bytes"] / n / 1e6, "us_per_launch": r["match_ms"] * 1e3 / n},
+                "step_us": r["total_ms"] * 1e3 / n}
+
+    def step_roof(r, n):
+        """The step as it runs: one launch (match, whole units, split ranges) or two."""
+        nbytes = r["att_bytes"] + r["match_bytes"]
+        a = gbs(nbytes, r["total_ms"])
+        return {"kernel": "mac_step_kernel" if r["one_launch"] else "mac_match_kernel + mac_attend_kernel",
+                "achieved": a, "frac": a / peak, "mb_per_launch": nbytes / n / 1e6,
+                "us_per_launch": r["total_ms"] * 1e3 / n}
+
     occ = [min(t, wl.W) for t in range(args.warmup, args.warmup + K_)]
-    roof = {"bound": "hbm", "kernel": "mac_attend_kernel", "achieved": att_gbs, "peak": peak,
-            "peak_kind": peak_kind, "unit": "GB/s", "frac": att_gbs / peak, "traffic": traffic,
-            "bytes_per_launch": kern["att_bytes"] / K_, "us_per_launch": kern["att_ms"] * 1e3 / K_}
+    main_roof = step_roof(main, K_)
+    roof = {"bound": "hbm", "kernel": main_roof["kernel"], "achieved": main_roof["achieved"], "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": main_roof["frac"],
+            # traffic of the step kernel from the committed ncu capture, when it matches this source
+            "traffic": (_profiled_traffic() * (main["att_bytes"] + main["match_bytes"]) / K_)
+            if _profiled_traffic() else None,
+            "bytes_per_launch": (main["att_bytes"] + main["match_bytes"]) / K_,
+            "us_per_launch": main["total_ms"] * 1e3 / K_,
+            "two_launch": two_launch(kern, K_)}
     detail = {}
     if allmiss:
         n = len(allmiss["step_ms"])
-        a_gbs = allmiss["att_bytes"] / (allmiss["att_ms"] * 1e-3) / 1e9
-        roof["miss"] = {"kernel": "mac_attend_kernel", "workload": "%s, threshold 0 (every unit misses)" % wl.name,
-                        "achieved": a_gbs, "frac": a_gbs / peak, "mb_per_launch": allmiss["att_bytes"] / n / 1e6,
-                        "us_per_launch": allmiss["att_ms"] * 1e3 / n, "steps_per_s": n / (allmiss["total_ms"] * 1e-3)}
+        roof["miss"] = dict(step_roof(allmiss, n),
+                            workload="%s, threshold 0 (every unit misses)" % wl.name,
+                            steps_per_s=n / (allmiss["total_ms"] * 1e-3),
+                            two_launch=two_launch(allmiss2, n))
         detail["all_miss"] = {"steps": n, "ms_per_step": allmiss["total_ms"] / n,
                               "speedup_of_mac": (world * K_ / (tot * 1e-3)) / (n / (allmiss["total_ms"] * 1e-3)),
                               "clocks": allmiss["clocks"]}
     if hitrun:
         n = len(hitrun["step_ms"])
-        h_gbs = hitrun["att_bytes"] / (hitrun["att_ms"] * 1e-3) / 1e9
-        m_gbs = hitrun["match_bytes"] / (hitrun["match_ms"] * 1e-3) / 1e9
-        roof["hit"] = {
-            "kernel": "mac_attend_kernel", "workload": "%s, every step a repeat" % wl.name,
-            "achieved": h_gbs, "frac": h_gbs / peak, "mb_per_launch": hitrun["att_bytes"] / n / 1e6,
-            "us_per_launch": hitrun["att_ms"] * 1e3 / n,
-            "match": {"kernel": "mac_match_kernel", "achieved": m_gbs, "frac": m_gbs / peak,
-                      "mb_per_launch": hitrun["match_bytes"] / n / 1e6, "us_per_launch": hitrun["match_ms"] * 1e3 / n},
-            "step_us": hitrun["total_ms"] * 1e3 / n, "hit_fraction": hitrun["hit_frac"],
-            "larger": [{"workload": h["workload"], "attend_frac": h["attend"]["frac"],
-                        "attend_us": h["attend"]["us_per_launch"], "attend_mb": h["attend"]["mb_per_launch"],
-                        "match_frac": h["match"]["frac"], "match_us": h["match"]["us_per_launch"],
-                        "step_us": h["step"]["us"], "step_frac": h["step"]["frac"]} for h in hitshapes]}
+        roof["hit"] = dict(step_roof(hitrun, n), workload="%s, every step a repeat" % wl.name,
+                           hit_fraction=hitrun["hit_frac"], two_launch=two_launch(hitrun2, n),
+                           larger=[{"workload": h["workload"], "step_us": h["step"]["us"], "step_mb": h["step"]["mb"],
+                                    "step_frac": h["step"]["frac"], "kernel": h["step"]["kernel"]}
+                                   for h in hitshapes])
         detail["hit_path"] = {"steps": n, "clocks": hitrun["clocks"], "shapes": hitshapes}
         if hitctx:
             roof["hit"]["vs_context"] = [
                 {"context": L, "step_us": r["total_ms"] * 1e3 / len(r["step_ms"]),
-                 "attend_mb": r["att_bytes"] / len(r["step_ms"]) / 1e6} for L, r in hitctx]
+                 "step_mb": (r["att_bytes"] + r["match_bytes"]) / len(r["step_ms"]) / 1e6} for L, r in hitctx]
     if mqa:
         a = mqa["all_miss"]["attend"]
         roof.setdefault("miss", {})["mqa_32_1"] = {"frac": a["frac"], "achieved": a["achieved"], "mb_per_launch": a["mb_per_launch"],
@@ -451,7 +471,7 @@ def run_mac(args, rank, world, local_rank):
         "hit_fraction": main["hit_frac"],
         "window_occupancy": {"mean": float(np.mean(occ)), "min": int(min(occ)), "max": int(max(occ)),
                              "window": wl.W},
-        "gpu_launches": 2 * K_ * world,
+        "gpu_launches": (1 if main["one_launch"] else 2) * K_ * world,
         "clocks": main["clocks"],
         "device_status": main["status"],
     }
@@ -464,9 +484,8 @@ def run_mac(args, rank, world, local_rank):
     if cpu:
         res["cpu_baseline"] = cpu
     detail.update({
-        "match_kernel_gbs": kern["match_bytes"] / (kern["match_ms"] * 1e-3) / 1e9,
-        "kernel_ms_per_step": {"match": kern["match_ms"] / K_, "attend": kern["att_ms"] / K_,
-                               "timed_separately": kern["total_ms"] / K_},
+        "kernel_ms_per_step_two_launch": {"match": kern["match_ms"] / K_, "attend": kern["att_ms"] / K_,
+                                          "timed_separately": kern["total_ms"] / K_},
         "step_gbs": (main["att_bytes"] + main["match_bytes"]) / (main["total_ms"] * 1e-3) / 1e9,
         "effective_kv_gbs": main["dense_bytes"] / (main["total_ms"] * 1e-3) / 1e9,
         "kv_bytes_per_step": main["kv_bytes"] / K_, "dense_kv_bytes_per_step": main["dense_bytes"] / K_,
@@ -507,10 +526,11 @@ def run_hit_shape(name, nsteps, dev, peak, world):
 def run_shape(wl, nsteps, dev, peak, nwarm=None):
     """Steps of another workload shape, with the windows filled first (the
     window length of untimed steps unless nwarm says otherwise), then nsteps
-    steps timed with events before, between and after the two kernels.  K/V
-    values do not change the work of a step, so the cache is drawn on the
-    device (seeded N(0, 1), bf16) in the workload's layout instead of on the
-    host."""
+    timed steps: once as the step runs (mac_decode_step, one launch where it
+    applies; events around each step) and once with the match and attention
+    kernels launched and timed apart.  K/V values do not change the work of a
+    step, so the cache is drawn on the device (seeded N(0, 1), bf16) in the
+    workload's layout instead of on the host."""
     import torch
     import kv_cache_reuse_b200 as mac
     nwarm = wl.W if nwarm is None else nwarm
@@ -524,7 +544,6 @@ def run_shape(wl, nsteps, dev, peak, nwarm=None):
     V = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16).view(torch.int16)
     bt = None if bt_h is None else torch.from_numpy(bt_h).to(dev)
     kw = dict(capacity=max_seq) if bt_h is None else dict(max_pages_per_seq=bt_h.shape[1], num_pages=P)
-    st = mac.MacState.for_workload(wl, **kw)
     B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
     q = torch.from_numpy(stream.q).to(dev)
     pos = torch.from_numpy(stream.rope_pos).to(dev)
@@ -535,44 +554,61 @@ def run_shape(wl, nsteps, dev, peak, nwarm=None):
     mpos = torch.zeros((T, B, Hkv), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     s = torch.cuda.current_stream(dev)
-    for t in range(nwarm):
-        st.decode_step(q[t], pos[t], K, V, bt, lens[t], out, lse, hit[t], mpos[t])
-        flush.zero_()
-    torch.cuda.synchronize(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
-    h, sp = st.handle, s.cuda_stream
     btp = bt.data_ptr() if bt is not None else None
-    torch.cuda._sleep(int(2e6 + 4e5 * nsteps))
-    for i in range(nsteps):
-        t = nwarm + i
-        ev[i][0].record(s)
-        mac.mac_match(h, q[t].data_ptr(), pos[t].data_ptr(), btp, lens[t].data_ptr(), out.data_ptr(),
-                      lse.data_ptr(), hit[t].data_ptr(), mpos[t].data_ptr(), sp)
-        ev[i][1].record(s)
-        mac.mac_attend(h, K.data_ptr(), V.data_ptr(), btp, out.data_ptr(), lse.data_ptr(), sp)
-        ev[i][2].record(s)
-        flush.zero_()
-    torch.cuda.synchronize(dev)
-    status = st.get_status()
-    st.close()
-    hits = hit.cpu().numpy()[nwarm:]
-    mps = mpos.cpu().numpy()[nwarm:]
-    mt = at = kv = 0
-    for i in range(nsteps):
-        a, b_, c = step_bytes(wl, hits[i], mps[i], stream.seq_lens[nwarm + i], min(nwarm + i, wl.W))
-        mt, at, kv = mt + a, at + b_, kv + c
-    m_ms = float(sum(e[0].elapsed_time(e[1]) for e in ev))
-    a_ms = float(sum(e[1].elapsed_time(e[2]) for e in ev))
-    step_ms = float(sum(e[0].elapsed_time(e[2]) for e in ev))
+
+    def one_pass(split):
+        st = mac.MacState.for_workload(wl, **kw)
+        for t in range(nwarm):
+            st.decode_step(q[t], pos[t], K, V, bt, lens[t], out, lse, hit[t], mpos[t])
+            flush.zero_()
+        torch.cuda.synchronize(dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
+        h, sp = st.handle, s.cuda_stream
+        torch.cuda._sleep(int(2e6 + 4e5 * nsteps))
+        for i in range(nsteps):
+            t = nwarm + i
+            ev[i][0].record(s)
+            if split:
+                mac.mac_match(h, q[t].data_ptr(), pos[t].data_ptr(), btp, lens[t].data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), hit[t].data_ptr(), mpos[t].data_ptr(), sp)
+                ev[i][1].record(s)
+                mac.mac_attend(h, K.data_ptr(), V.data_ptr(), btp, out.data_ptr(), lse.data_ptr(), sp)
+            else:
+                mac.mac_decode_step(h, q[t].data_ptr(), pos[t].data_ptr(), K.data_ptr(), V.data_ptr(), btp,
+                                    lens[t].data_ptr(), out.data_ptr(), lse.data_ptr(), hit[t].data_ptr(),
+                                    mpos[t].data_ptr(), sp)
+                ev[i][1].record(s)
+            ev[i][2].record(s)
+            flush.zero_()
+        torch.cuda.synchronize(dev)
+        one = mac.mac_one_launch(st)
+        status = st.get_status()
+        st.close()
+        hits = hit.cpu().numpy()[nwarm:]
+        mps = mpos.cpu().numpy()[nwarm:]
+        mt = at = 0
+        for i in range(nsteps):
+            a, b_, _ = step_bytes(wl, hits[i], mps[i], stream.seq_lens[nwarm + i], min(nwarm + i, wl.W))
+            mt, at = mt + a, at + b_
+        m_ms = float(sum(e[0].elapsed_time(e[1]) for e in ev))
+        a_ms = float(sum(e[1].elapsed_time(e[2]) for e in ev))
+        step_ms = float(sum(e[0].elapsed_time(e[2]) for e in ev))
+        return dict(mt=mt, at=at, m_ms=m_ms, a_ms=a_ms, step_ms=step_ms, one=one, status=status,
+                    hit_frac=float(hits.mean()))
+
+    r1, r2 = one_pass(False), one_pass(True)
+    frac = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9 / peak
     return {"workload": wl.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "window": wl.W, "band": wl.band,
-            "paged": bt_h is not None, "steps": nsteps, "hit_fraction": float(hits.mean()),
-            "attend": {"mb_per_launch": at / nsteps / 1e6, "us_per_launch": a_ms * 1e3 / nsteps,
-                       "achieved": at / (a_ms * 1e-3) / 1e9, "frac": at / (a_ms * 1e-3) / 1e9 / peak},
-            "match": {"mb_per_launch": mt / nsteps / 1e6, "us_per_launch": m_ms * 1e3 / nsteps,
-                      "achieved": mt / (m_ms * 1e-3) / 1e9, "frac": mt / (m_ms * 1e-3) / 1e9 / peak},
-            "step": {"us": step_ms * 1e3 / nsteps, "mb": (mt + at) / nsteps / 1e6,
-                     "frac": (mt + at) / (step_ms * 1e-3) / 1e9 / peak},
-            "device_status": status}
+            "paged": bt_h is not None, "steps": nsteps, "hit_fraction": r1["hit_frac"],
+            "step": {"kernel": "mac_step_kernel" if r1["one"] else "mac_match_kernel + mac_attend_kernel",
+                     "us": r1["step_ms"] * 1e3 / nsteps, "mb": (r1["mt"] + r1["at"]) / nsteps / 1e6,
+                     "frac": frac(r1["mt"] + r1["at"], r1["step_ms"])},
+            "attend": {"mb_per_launch": r2["at"] / nsteps / 1e6, "us_per_launch": r2["a_ms"] * 1e3 / nsteps,
+                       "achieved": r2["at"] / (r2["a_ms"] * 1e-3) / 1e9, "frac": frac(r2["at"], r2["a_ms"])},
+            "match": {"mb_per_launch": r2["mt"] / nsteps / 1e6, "us_per_launch": r2["m_ms"] * 1e3 / nsteps,
+                      "achieved": r2["mt"] / (r2["m_ms"] * 1e-3) / 1e9, "frac": frac(r2["mt"], r2["m_ms"])},
+            "two_launch_step_us": r2["step_ms"] * 1e3 / nsteps,
+            "device_status": max(r1["status"], r2["status"])}
 
 
 def run_quality(args, wl, stream, K, V, bt, kw, dev, identity_rope=False):
