@@ -399,6 +399,13 @@ def run_mac(args, rank, world, local_rank):
         wq = wl.with_(Hq=32, Hkv=1)
         mqa = {"all_miss": run_shape(wq.with_(tau=0.0), args.mqa_steps, dev, peak, nwarm=3),
                "mixed": run_shape(wq, args.mqa_steps, dev, peak)}
+    traces = None
+    if args.trace_steps > 0:
+        # the phase breakdown of hit steps (and of steps with misses) from the device trace
+        traces = {"long_128k_all_hit": run_trace(wl.with_(hit_model=("iid", 1.0)), args.trace_steps, dev, peak),
+                  "long_128k_mixed": run_trace(wl, args.trace_steps, dev, peak),
+                  "paged_mixed_all_hit": run_trace(synth.WORKLOADS["paged_mixed"].with_(hit_model=("iid", 1.0)),
+                                                   args.trace_steps, dev, peak)}
     hitshapes = []
     if args.hit_steps > 0 and args.hit_shapes:
         hitshapes = [run_hit_shape(n, args.hit_steps, dev, peak, world) for n in args.hit_shapes.split(",") if n]
@@ -509,6 +516,8 @@ def run_mac(args, rank, world, local_rank):
             "clocks": run["clocks"], "device_status": run["status"]})
     if quality:
         detail["approximation_vs_dense"] = quality
+    if traces:
+        detail["phase_trace"] = traces
     if warm:
         detail["warm_start"] = warm
     res["detail"] = "full record on stderr (one JSON line)"
@@ -609,6 +618,64 @@ def run_shape(wl, nsteps, dev, peak, nwarm=None):
                       "achieved": r2["mt"] / (r2["m_ms"] * 1e-3) / 1e9, "frac": frac(r2["mt"], r2["m_ms"])},
             "two_launch_step_us": r2["step_ms"] * 1e3 / nsteps,
             "device_status": max(r1["status"], r2["status"])}
+
+
+TRACE_PHASES = ("start", "matched", "published", "whole_done", "table_seen", "range_done", "table_built", "end")
+
+
+def run_trace(wl, nsteps, dev, peak):
+    """Where the time of a step goes: steps of a workload shape (every labelled
+    step a repeat when the workload's stream says so) with the device trace on
+    (mac_set_trace), windows filled first.  Per step, each phase's time is
+    taken from the first CTA's start, for the median CTA and the last CTA to
+    pass it; reported as the median over the steps (microseconds)."""
+    import torch
+    import kv_cache_reuse_b200 as mac
+    nwarm = wl.W
+    T = nwarm + nsteps
+    stream = synth.queries(wl, T)
+    bt_h, max_seq, P = synth.kv_layout(wl, T)
+    shape = (wl.B, max_seq, wl.Hkv, wl.D) if bt_h is None else (P, wl.page_size, wl.Hkv, wl.D)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    K = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16).view(torch.int16)
+    V = torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16).view(torch.int16)
+    bt = None if bt_h is None else torch.from_numpy(bt_h).to(dev)
+    kw = dict(capacity=max_seq) if bt_h is None else dict(max_pages_per_seq=bt_h.shape[1], num_pages=P)
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    q = torch.from_numpy(stream.q).to(dev)
+    pos = torch.from_numpy(stream.rope_pos).to(dev)
+    lens = torch.from_numpy(stream.seq_lens).to(dev)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    hit = torch.zeros((B, Hkv), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    st = mac.MacState.for_workload(wl, **kw)
+    mac.mac_set_trace(st, 1)
+    med, last, keys = [], [], []
+    for t in range(T):
+        flush.zero_()
+        st.decode_step(q[t], pos[t], K, V, bt, lens[t], out, lse, hit)
+        stamps, counters = mac.mac_get_trace(st)
+        if t < nwarm:
+            continue
+        s_ = stamps.astype(np.float64)
+        t0 = s_[:, 0][s_[:, 0] > 0].min()
+        rel = np.where(s_ > 0, (s_ - t0) * 1e-3, np.nan)
+        with np.errstate(all="ignore"):
+            med.append(np.nanmedian(rel, axis=0))
+            last.append(np.nanmax(rel, axis=0))
+        keys.append(int(counters[0]))
+    one = mac.mac_one_launch(st)
+    st.close()
+    with np.errstate(all="ignore"):
+        m, l_ = np.nanmedian(np.array(med), axis=0), np.nanmedian(np.array(last), axis=0)
+    clean = lambda x: None if not np.isfinite(x) else round(float(x), 2)
+    return {"workload": wl.name, "kernel": "mac_step_kernel" if one else "mac_match_kernel + mac_attend_kernel",
+            "steps": nsteps, "keys_per_step": float(np.median(keys)),
+            "median_cta_us": {n: clean(x) for n, x in zip(TRACE_PHASES, m)},
+            "last_cta_us": {n: clean(x) for n, x in zip(TRACE_PHASES, l_)},
+            "note": "times from the first CTA's start (%globaltimer), median over steps"}
 
 
 def run_quality(args, wl, stream, K, V, bt, kw, dev, identity_rope=False):
@@ -842,6 +909,8 @@ def main():
     ap.add_argument("--warm-start", action="store_true", help="also time seeding the windows from W positions")
     ap.add_argument("--layers", type=int, default=4,
                     help="also time a stack of this many layers per token, one CUDA graph per token (0 = skip)")
+    ap.add_argument("--trace-steps", type=int, default=12,
+                    help="steps of the device phase trace runs (0 = skip)")
     ap.add_argument("--mqa-steps", type=int, default=8,
                     help="timed steps of the 32-query-heads-over-one-KV-head runs (0 = skip)")
     ap.add_argument("--hit-shapes", default="paged_mixed,continuous_16k",

@@ -264,6 +264,27 @@ int mac_set_one_launch(MacState *st, int on);
 /* 1 if mac_decode_step on this state runs as one launch, else 0. */
 int mac_one_launch(const MacState *st);
 
+/* Observability.  With on = 1 every step records, for each CTA of its
+ * launch, the %globaltimer time (ns) at which the CTA passed each phase:
+ * 0 kernel start, 1 its units matched, 2 its plans published, 3 its whole
+ * units done, 4 the split table seen, 5 its split range done, 6 the table
+ * published (the laying-out CTA of the one-launch step), 7 end; and adds to
+ * four counters: 0 keys attended with the current query (the fresh keys of
+ * every unit), 1 pieces walked, 2 units done whole, 3 split units merged.
+ * The keys counter checks on the device that a hit reads only its band and
+ * tail whatever the context length (page 1: the cost of a hit does not grow
+ * with the context).  Costs one small memset per step and a few atomics per
+ * piece; 0 (default) turns it off.  MAC_ERR_ARG for a NULL state or another
+ * value. */
+int mac_set_trace(MacState *st, int on);
+
+/* Copy the last traced step's phase times to stamps ([mac_attend_grid(st)][8]
+ * unsigned 64-bit ns; a phase a CTA did not reach is 0; may be NULL, else
+ * n_stamps must be at least grid * 8) and the counters accumulated since the
+ * last call to counters ([4]; may be NULL), then clear the counters.
+ * Synchronises the device. */
+int mac_get_trace(MacState *st, unsigned long long *stamps, size_t n_stamps, unsigned long long *counters);
+
 /* Reproducible work split.  on = 1: every step splits the key ranges evenly
  * over the CTAs and no streaming rate is learned or used, so a step's out and
  * lse depend only on its inputs and the window (bit for bit, on any B200);

@@ -323,6 +323,21 @@ def mac_one_launch(st) -> int:
     return int(load().mac_one_launch(_h(st)))
 
 
+def mac_set_trace(st, on: int) -> None:
+    check("mac_set_trace", load().mac_set_trace(_h(st), int(on)))
+
+
+def mac_get_trace(st):
+    """(stamps [grid][8] uint64 ns of the last traced step's phases, counters [4]
+    uint64 since the last call: keys attended fresh, pieces, whole units, merges)."""
+    import numpy as np
+    g = mac_attend_grid(st)
+    stamps = np.zeros((g, 8), np.uint64)
+    counters = np.zeros(4, np.uint64)
+    check("mac_get_trace", load().mac_get_trace(_h(st), stamps.ctypes.data, stamps.size, counters.ctypes.data))
+    return stamps, counters
+
+
 def mac_attend_grid(st) -> int:
     return int(load().mac_attend_grid(_h(st)))
 

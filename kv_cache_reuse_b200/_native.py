@@ -32,6 +32,8 @@ SIGNATURES = {
     "mac_set_reproducible": (C.c_int, [_P, C.c_int]),
     "mac_set_one_launch": (C.c_int, [_P, C.c_int]),
     "mac_one_launch": (C.c_int, [_P]),
+    "mac_set_trace": (C.c_int, [_P, C.c_int]),
+    "mac_get_trace": (C.c_int, [_P, _P, C.c_size_t, _P]),
     "mac_attend_grid": (C.c_int, [_P]),
     "mac_error_string": (C.c_char_p, [C.c_int]),
     "mac_selftest_wait_timeout": (C.c_int, [_P, _P]),

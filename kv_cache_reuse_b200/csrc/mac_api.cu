@@ -52,6 +52,10 @@ struct MacState {
   int* fsync = nullptr;    // {ticket, epoch}
   int one_launch_ok = 0;   // the configuration can run the step as one launch
   int one_launch = 1;      // ... and it does (mac_set_one_launch)
+  // observability (mac_set_trace)
+  unsigned long long* trace = nullptr;     // [grid][kTracePoints]
+  unsigned long long* counters = nullptr;  // [kCounters]
+  int tracing = 0;
   unsigned* status = nullptr;
   double* inv_freq = nullptr;
   // staging of mac_decode_step_host: one packed block each way, on the
@@ -111,7 +115,7 @@ void drop_graph(MacState* s) {
 void free_all(MacState* s) {
   drop_graph(s);
   void* ptrs[] = {s->ring_q, s->ring_o, s->ring_m, s->ring_l, s->ring_pos, s->steps, s->qrot,     s->plan,   s->hplan,
-                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done, s->dpart, s->ucnt, s->smid_of, s->rank_of, s->fsync, s->inv_freq, s->dev_in,
+                  s->seg,    s->hdr,    s->first_seg, s->rate, s->cw, s->bounds, s->claim, s->part, s->unit_cnt, s->done, s->dpart, s->ucnt, s->smid_of, s->rank_of, s->fsync, s->trace, s->counters, s->inv_freq, s->dev_in,
                   s->dev_out};
   for (void* p : ptrs)
     if (p) cudaFree(p);
@@ -277,6 +281,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(alloc(&s->smid_of, (size_t)s->grid));
   A(alloc(&s->rank_of, (size_t)s->grid));
   A(alloc(&s->fsync, 2));
+  A(alloc(&s->trace, (size_t)s->grid * kTracePoints));
+  A(alloc(&s->counters, (size_t)kCounters));
   A(alloc(&s->inv_freq, D / 2));
   s->off_q = 0;
   s->off_pos = up256(s->off_q + B * Hq * D * s->QES);
@@ -312,6 +318,8 @@ int mac_init_state(const MacConfig* cfg, MacState** out) {
   A(cudaMemset(s->done, 0, sizeof(int)));
   A(cudaMemset(s->ucnt, 0, U * sizeof(int)));
   A(cudaMemset(s->fsync, 0, 2 * sizeof(int)));
+  A(cudaMemset(s->trace, 0, (size_t)s->grid * kTracePoints * sizeof(unsigned long long)));
+  A(cudaMemset(s->counters, 0, kCounters * sizeof(unsigned long long)));
   A(cudaMemset(s->rate, 0, s->grid * sizeof(float)));
   A(cudaMemset(s->claim, 0, s->grid * sizeof(int)));
   {  // even shares until the first rates are measured
@@ -390,6 +398,29 @@ int mac_set_one_launch(MacState* s, int on) {
 }
 
 int mac_one_launch(const MacState* s) { return s && s->one_launch && s->one_launch_ok ? 1 : 0; }
+
+int mac_set_trace(MacState* s, int on) {
+  if (!s || on < 0 || on > 1) return MAC_ERR_ARG;
+  s->tracing = on;
+  drop_graph(s);
+  return MAC_OK;
+}
+
+int mac_get_trace(MacState* s, unsigned long long* stamps, size_t n_stamps, unsigned long long* counters) {
+  if (!s) return MAC_ERR_ARG;
+  const size_t n = (size_t)s->grid * kTracePoints;
+  if (stamps && n_stamps < n) return MAC_ERR_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MAC_ERR_CUDA;
+  if (stamps && cudaMemcpy(stamps, s->trace, n * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MAC_ERR_CUDA;
+  if (counters) {
+    if (cudaMemcpy(counters, s->counters, kCounters * sizeof(unsigned long long), cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      return MAC_ERR_CUDA;
+  }
+  if (cudaMemset(s->counters, 0, kCounters * sizeof(unsigned long long)) != cudaSuccess) return MAC_ERR_CUDA;
+  return MAC_OK;
+}
 
 int mac_set_reproducible(MacState* s, int on) {
   if (!s || on < 0 || on > 1) return MAC_ERR_ARG;
@@ -520,13 +551,26 @@ static int fill_attend(MacState* s, const uint16_t* K, const uint16_t* V, const 
   p.smid_of = s->smid_of;
   p.rank_of = s->rank_of;
   p.fsync = s->fsync;
+  p.trace = s->tracing ? s->trace : nullptr;
+  p.counters = s->tracing ? s->counters : nullptr;
   return MAC_OK;
+}
+
+// With tracing on, a step's phase times start from zero (a phase a CTA does
+// not reach stays 0).
+static int clear_trace(MacState* s, cudaStream_t st) {
+  if (!s->tracing) return MAC_OK;
+  return cudaMemsetAsync(s->trace, 0, (size_t)s->grid * kTracePoints * sizeof(unsigned long long), st) ==
+                 cudaSuccess
+             ? MAC_OK
+             : MAC_ERR_CUDA;
 }
 
 int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* block_table, float* out, float* lse,
                void* stream) {
   AttendParams p;
-  const int rc = fill_attend(s, K, V, block_table, out, lse, p);
+  int rc = fill_attend(s, K, V, block_table, out, lse, p);
+  if (rc == MAC_OK) rc = clear_trace(s, (cudaStream_t)stream);
   if (rc != MAC_OK) return rc;
   return launch_attend(p, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
 }
@@ -542,6 +586,7 @@ int mac_decode_step(MacState* s, const void* q_pre, const int* rope_pos, const u
     AttendParams ap;
     int rc = fill_match(s, s->cfg.tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, mp);
     if (rc == MAC_OK) rc = fill_attend(s, K, V, block_table, out, lse, ap);
+    if (rc == MAC_OK) rc = clear_trace(s, (cudaStream_t)stream);
     if (rc != MAC_OK) return rc;
     return launch_step(ap, mp, s->D, s->grid, (cudaStream_t)stream) == cudaSuccess ? MAC_OK : MAC_ERR_CUDA;
   }

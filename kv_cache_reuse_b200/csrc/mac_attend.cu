@@ -180,6 +180,11 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const int* ptr) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
   return v;
 }
+__device__ __forceinline__ unsigned ld_relaxed_u32(const int* ptr) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_release_u32(int* ptr, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
@@ -770,6 +775,7 @@ __device__ bool finalize_piece(const AttendParams& p, AttnSmem<D, GP>& sm, Acc<D
   if (!consumer_sync(sm, sync_phase, p.status)) return false;
   if (sm.last_flag) {
     __threadfence();
+    if (p.counters != nullptr && threadIdx.x == 0) atomicAdd(p.counters + kCountMerged, 1ull);
     return merge_unit<D, GP, GF, PH, NC>(p, sm, unit, sync_phase);
   }
   return true;
@@ -1017,6 +1023,10 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   unsigned smid;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
   const uint64_t pol = evict_first_policy();
+  auto stamp = [&](int k) {
+    if (p.trace != nullptr && tid == 0) p.trace[cta * kTracePoints + k] = globaltimer();
+  };
+  stamp(kTraceStart);
 
   // cursors, counters and barrier phases of this CTA; they carry over from
   // one walk to the next (the box slots' phases follow the box counts)
@@ -1207,6 +1217,11 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       ok = false;
       break;
     }
+    if (p.counters != nullptr && tid == 0) {
+      atomicAdd(p.counters + kCountKeys, (unsigned long long)(cp.k1 - cp.k0 + (cp.whole ? cp.a1 - cp.a0 : 0)));
+      atomicAdd(p.counters + kCountPieces, 1ull);
+      if (cp.whole) atomicAdd(p.counters + kCountWhole, 1ull);
+    }
     ++cpn;
   }
   };  // walk
@@ -1220,10 +1235,10 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     using MS = MatchSmem<D, GP, false>;
     static_assert(sizeof(MS) <= sizeof(sm.kv), "match scratch lives in the box slots");
     MS& ms = *reinterpret_cast<MS*>(&sm.kv[0][0][0][0]);
-    if (tid == 0) {
-      sm.nlocal = 0;
-      sm.last_flag = (int)ld_acquire_u32(p.fsync + 1);  // this launch's epoch, before its ticket
-    }
+    // this launch's epoch: read before the ticket (the layout advances it only
+    // after every ticket), consumed after the match stage
+    const unsigned epoch = tid == 0 ? ld_relaxed_u32(p.fsync + 1) : 0u;
+    if (tid == 0) sm.nlocal = 0;
     __syncthreads();
     // match stage of this CTA's units; whole units become local items
 #pragma unroll 1
@@ -1246,22 +1261,36 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
         }
       }
     }
-    const unsigned epoch = (unsigned)sm.last_flag;
+    stamp(kTraceMatched);
     // the box slots held the match scratch, and the bulk copies of this launch
     // read the rotated queries just written: order those generic writes (shared
     // and global) before any copy, then publish them device-wide
     asm volatile("fence.proxy.async;" ::: "memory");
     __threadfence();
     __syncthreads();
+    // the last CTA lays out the split items once every other CTA has published
+    // its plans (it holds a unit only when there are as many units as CTAs, so
+    // the layout seldom waits behind a match or delays a whole unit)
+    const int builder = (int)gridDim.x - 1;
     if (tid == 0) {
       p.smid_of[cta] = (int)smid;
-      int ticket;
-      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(p.fsync) : "memory");
-      sm.last_flag = (ticket == (int)gridDim.x - 1);
+      if (cta != builder) {
+        asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.fsync) : "memory");
+      } else {
+        const unsigned long long t0 = globaltimer();
+        while ((int)ld_acquire_u32(p.fsync) != builder) {
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicOr(p.status, MAC_DEV_TIMEOUT);
+            sm.abort_flag = 1;
+            break;
+          }
+        }
+      }
+      if (p.trace) p.trace[cta * kTracePoints + kTraceTicket] = globaltimer();
     }
     __syncthreads();
-    if (sm.last_flag) {
-      // every CTA's plans and SM id precede its ticket: lay out the split items
+    if (cta == builder) {
+      // every other CTA's plans and SM id precede its arrival: lay out the split items
       __threadfence();
       static_assert(sizeof(SplitScratch) <= sizeof(sm.kv), "split scratch lives in the box slots");
       build_split_table(mp, U, (int)gridDim.x, p.smid_of, p.rank_of,
@@ -1272,12 +1301,14 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       if (tid == 0) {
         p.fsync[0] = 0;
         st_release_u32(p.fsync + 1, epoch + 1u);
+        if (p.trace) p.trace[cta * kTracePoints + kTraceBuilt] = globaltimer();
       }
     }
     __syncthreads();
     // this CTA's whole units
     const int nlocal = sm.nlocal;
     if (nlocal > 0) walk(sm.items, nlocal, 0, 0, LLONG_MAX, cta, false, true);
+    stamp(kTraceLocal);
     // the step's split table (bounded wait for the last CTA's layout)
     if (tid == 0 && ok) {
       const unsigned long long t0 = globaltimer();
@@ -1293,6 +1324,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     // the split pieces' queries were written by other CTAs of this launch and
     // are read by bulk copies: order the acquire before those copies
     asm volatile("fence.proxy.async.global;" ::: "memory");
+    stamp(kTraceTable);
     // (written by another CTA of this launch: read through L2)
     if (ok && !sm.abort_flag && __ldcg(&p.hdr->total) > 0) {
       weighted = __ldcg(&p.hdr->weighted);
@@ -1336,11 +1368,13 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       lo = (long long)cta * T / n_cta;
       hi = (long long)(cta + 1) * T / n_cta;
     }
+    stamp(kTraceTable);
   }
   if (ok && lo < hi) {
     if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = load_segment(p.seg + first_seg + tid);
     __syncthreads();
     walk(p.seg, p.nseg, first_seg, lo, hi, slot, true, false);
+    stamp(kTraceRange);
   }
   if (weighted && p.rate != nullptr) {
     // fold this SM's streaming rate (boxes per microsecond) into its record;
@@ -1377,6 +1411,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     }
     __syncwarp();
   }
+  stamp(kTraceEnd);
 }
 
 template <int D, int GP, int GF, bool PH, int NC = 1>

@@ -151,6 +151,8 @@ struct AttendParams {
   int* smid_of;      // one-launch step: [grid] SM of each CTA
   int* rank_of;      // one-launch step: [grid] range of each split slot (-1: none)
   int* fsync;        // one-launch step: {CTAs that finished matching, epoch of the published split}
+  unsigned long long* trace;     // [grid][kTracePoints] %globaltimer at each phase of the last step, or null
+  unsigned long long* counters;  // [kCounters] step counters (added to), or null
   void* ring_o;      // [U][W+1][G][D] fp32, or bf16 bits (ring_bf16)
   float* ring_m;     // [U][W+1][G]
   float* ring_l;     // [U][W+1][G]
@@ -173,6 +175,24 @@ struct AppendParams {
   unsigned* status;
   int B, Hkv, D, page_size, max_pages, num_pages, capacity;
 };
+
+// Observability.  Phases a CTA stamps (ns of %globaltimer) when tracing is
+// on; a phase the CTA does not go through keeps 0.
+enum {
+  kTraceStart = 0,      // barriers initialised
+  kTraceMatched = 1,    // one-launch step: this CTA's units matched
+  kTraceTicket = 2,     // one-launch step: this CTA's plans published
+  kTraceLocal = 3,      // one-launch step: this CTA's whole units done
+  kTraceTable = 4,      // the split table seen (after the wait for it)
+  kTraceRange = 5,      // this CTA's range of split items done
+  kTraceBuilt = 6,      // one-launch step, the laying-out CTA: split table published
+  kTraceEnd = 7,        // about to leave
+  kTracePoints = 8
+};
+// Counters the kernels add to when they are on: keys attended with the
+// current query (fresh keys), pieces walked, units done whole, split units
+// merged.
+enum { kCountKeys = 0, kCountPieces = 1, kCountWhole = 2, kCountMerged = 3, kCounters = 4 };
 
 // Launchers (defined in the .cu files).
 cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s);

@@ -239,6 +239,8 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   ap.smid_of = nullptr;  // two launches here, never the one-launch step
   ap.rank_of = nullptr;
   ap.fsync = nullptr;
+  ap.trace = nullptr;
+  ap.counters = nullptr;
   ap.ring_o = base + kOffRingO;
   ap.ring_bf16 = 0;
   ap.ring_m = reinterpret_cast<float*>(base + kOffRingM);

@@ -370,6 +370,44 @@ def test_two_launch_path(case):
     assert r["gpu"].st is not None
 
 
+@pytest.mark.parametrize("one_launch", [1, 0])
+def test_trace_counts_keys_and_orders_phases(one_launch):
+    """mac_set_trace: the device's count of keys attended with the current
+    query equals the keys the oracle reads at every step, and on steps where
+    every unit hits it is the same at 8K and 32K keys of context (page 1: the
+    cost of a hit does not grow with the context); each CTA's phase times come
+    in order."""
+    import kv_cache_reuse_b200 as mac
+    per_ctx = {}
+    for L in (8192, 32768):
+        wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, L0=(L, L), steps=10, hit_model=("iid", 1.0))
+        stream, cache = synth.queries(wl), synth.kv_cache(wl)
+        gpu = DeviceRun(wl, cache, tune={"trace": 1, "one_launch": one_launch})
+        orc = oracle.Oracle.for_workload(wl, cache)
+        keys = []
+        for t in range(wl.steps):
+            r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+            out, lse, hit, mpos = gpu.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+            np.testing.assert_array_equal(hit, r.hit)
+            assert float(np.abs(out - r.out).max()) <= OUT_TOL
+            stamps, counters = mac.mac_get_trace(gpu.st)
+            assert int(counters[0]) == r.keys_read, "step %d" % t
+            assert int(counters[1]) >= 1 and int(counters[2]) + int(counters[3]) >= 1
+            keys.append((int(r.hit.all()), int(counters[0])))
+            for row in stamps.astype(np.int64):
+                seen = [row[k] for k in (0, 1, 2, 3, 4, 5, 7) if row[k] > 0]
+                assert seen == sorted(seen), row
+                if row[6] > 0:  # the laying-out CTA published the table after its ticket
+                    assert row[2] <= row[6] and (row[4] == 0 or row[6] <= row[4])
+            assert (stamps[:, 0] > 0).any()
+        per_ctx[L] = keys
+        assert gpu.st.get_status() == 0
+    hit_steps = [t for t in range(1, 10) if per_ctx[8192][t][0] and per_ctx[32768][t][0]]
+    assert len(hit_steps) >= 5
+    for t in hit_steps:
+        assert per_ctx[8192][t][1] == per_ctx[32768][t][1], t
+
+
 _SPLIT = {"whole_unit_keys": 0, "piece_cost": 0, "min_keys_per_cta": 64}
 
 
