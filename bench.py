@@ -620,7 +620,8 @@ def run_shape(wl, nsteps, dev, peak, nwarm=None):
             "device_status": max(r1["status"], r2["status"])}
 
 
-TRACE_PHASES = ("start", "matched", "published", "whole_done", "table_seen", "range_done", "table_built", "end")
+TRACE_PHASES = ("start", "loaded", "decided", "matched", "published", "first_box", "boxes_done", "whole_done",
+                "table_built", "table_seen", "range_done", "end")
 
 
 def run_trace(wl, nsteps, dev, peak):

@@ -266,9 +266,12 @@ int mac_one_launch(const MacState *st);
 
 /* Observability.  With on = 1 every step records, for each CTA of its
  * launch, the %globaltimer time (ns) at which the CTA passed each phase:
- * 0 kernel start, 1 its units matched, 2 its plans published, 3 its whole
- * units done, 4 the split table seen, 5 its split range done, 6 the table
- * published (the laying-out CTA of the one-launch step), 7 end; and adds to
+ * 0 kernel start, 1 its first unit's query and window loaded, 2 that unit's
+ * decision taken, 3 its units matched, 4 its plans published, 5 its first
+ * K/V box on chip, 6 the last box of its whole units consumed, 7 its whole
+ * units done, 8 the split table published (the laying-out CTA of the
+ * one-launch step), 9 the split table seen, 10 its split range done, 11 end
+ * (phases 1-2 also in the match kernel of two launches); and adds to
  * four counters: 0 keys attended with the current query (the fresh keys of
  * every unit), 1 pieces walked, 2 units done whole, 3 split units merged.
  * The keys counter checks on the device that a hit reads only its band and
@@ -278,9 +281,9 @@ int mac_one_launch(const MacState *st);
  * value. */
 int mac_set_trace(MacState *st, int on);
 
-/* Copy the last traced step's phase times to stamps ([mac_attend_grid(st)][8]
+/* Copy the last traced step's phase times to stamps ([mac_attend_grid(st)][12]
  * unsigned 64-bit ns; a phase a CTA did not reach is 0; may be NULL, else
- * n_stamps must be at least grid * 8) and the counters accumulated since the
+ * n_stamps must be at least grid * 12) and the counters accumulated since the
  * last call to counters ([4]; may be NULL), then clear the counters.
  * Synchronises the device. */
 int mac_get_trace(MacState *st, unsigned long long *stamps, size_t n_stamps, unsigned long long *counters);

@@ -328,11 +328,11 @@ def mac_set_trace(st, on: int) -> None:
 
 
 def mac_get_trace(st):
-    """(stamps [grid][8] uint64 ns of the last traced step's phases, counters [4]
+    """(stamps [grid][12] uint64 ns of the last traced step's phases, counters [4]
     uint64 since the last call: keys attended fresh, pieces, whole units, merges)."""
     import numpy as np
     g = mac_attend_grid(st)
-    stamps = np.zeros((g, 8), np.uint64)
+    stamps = np.zeros((g, 12), np.uint64)
     counters = np.zeros(4, np.uint64)
     check("mac_get_trace", load().mac_get_trace(_h(st), stamps.ctypes.data, stamps.size, counters.ctypes.data))
     return stamps, counters

@@ -472,6 +472,7 @@ static int fill_match(MacState* s, float tau, const void* q_pre, const int* rope
   p.done = s->done;
   p.dpart = s->dpart;
   p.ucnt = s->ucnt;
+  p.trace = s->tracing ? s->trace : nullptr;
   p.status = s->status;
   p.B = s->cfg.batch;
   p.Hq = s->cfg.num_q_heads;

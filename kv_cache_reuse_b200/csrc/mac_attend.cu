@@ -1176,6 +1176,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
         break;
       }
       if (timed && tid == 0 && cons == cons0) t_first = globaltimer();
+      if (tid == 0 && cons == 0) stamp(kTraceFirstBox);
       const int key_box = cr.kb0 + bj * kSubKeys;
       float* pbuf = sm.wbuf[warp] + par * C::PB;
       uint16_t* kbuf = kv_slot(st);
@@ -1204,6 +1205,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     }
     if (!ok) break;
     if (timed && tid == 0) t_last = globaltimer();
+    if (local) stamp(kTraceBoxesDone);
     bool fin;
     if constexpr (NC > 1)
       fin = finalize_piece<D, GP, GF, PH, NC>(p, sm, A, cp.unit, cp.pidx, sync_phase);
@@ -1266,7 +1268,6 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     // read the rotated queries just written: order those generic writes (shared
     // and global) before any copy, then publish them device-wide
     asm volatile("fence.proxy.async;" ::: "memory");
-    __threadfence();
     __syncthreads();
     // the last CTA lays out the split items once every other CTA has published
     // its plans (it holds a unit only when there are as many units as CTAs, so
@@ -1275,6 +1276,9 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     if (tid == 0) {
       p.smid_of[cta] = (int)smid;
       if (cta != builder) {
+        // the block barrier above orders every thread's writes before this
+        // thread's device-scope fence; the arrival then publishes them
+        __threadfence();
         asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.fsync) : "memory");
       } else {
         const unsigned long long t0 = globaltimer();
@@ -1296,10 +1300,10 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       build_split_table(mp, U, (int)gridDim.x, p.smid_of, p.rank_of,
                         *reinterpret_cast<SplitScratch*>(&sm.kv[0][0][0][0]));
       asm volatile("fence.proxy.async;" ::: "memory");  // the scratch in the box slots, before copies
-      __threadfence();
       __syncthreads();
       if (tid == 0) {
         p.fsync[0] = 0;
+        __threadfence();  // every thread's table writes, ordered by the barrier, before the epoch
         st_release_u32(p.fsync + 1, epoch + 1u);
         if (p.trace) p.trace[cta * kTracePoints + kTraceBuilt] = globaltimer();
       }

@@ -120,6 +120,7 @@ struct MatchParams {
   int* done;               // arrival counter of the match CTAs (reset by the last)
   float* dpart;            // chunked groups: [U][W+1][NC] each chunk's part of an entry's distance
   int* ucnt;               // chunked groups: [U] arrivals of a unit's chunk CTAs (reset by the last)
+  unsigned long long* trace;  // [grid][kTracePoints] phase times (one-launch step), or null
   unsigned* status;
   int B, Hq, Hkv, G, W, band, page_size, max_pages, num_pages, capacity;  // band: b - cut_mode
   int per_head;   // 1: one match decision per query head
@@ -179,15 +180,19 @@ struct AppendParams {
 // Observability.  Phases a CTA stamps (ns of %globaltimer) when tracing is
 // on; a phase the CTA does not go through keeps 0.
 enum {
-  kTraceStart = 0,      // barriers initialised
-  kTraceMatched = 1,    // one-launch step: this CTA's units matched
-  kTraceTicket = 2,     // one-launch step: this CTA's plans published
-  kTraceLocal = 3,      // one-launch step: this CTA's whole units done
-  kTraceTable = 4,      // the split table seen (after the wait for it)
-  kTraceRange = 5,      // this CTA's range of split items done
-  kTraceBuilt = 6,      // one-launch step, the laying-out CTA: split table published
-  kTraceEnd = 7,        // about to leave
-  kTracePoints = 8
+  kTraceStart = 0,       // barriers initialised
+  kTraceLoaded = 1,      // match: the first unit's query and window in registers
+  kTraceDecided = 2,     // match: the first unit's decision taken
+  kTraceMatched = 3,     // one-launch step: this CTA's units matched and recorded
+  kTraceTicket = 4,      // one-launch step: this CTA's plans published
+  kTraceFirstBox = 5,    // the CTA's first K/V box on chip
+  kTraceBoxesDone = 6,   // one-launch step: the last box of this CTA's whole units consumed
+  kTraceLocal = 7,       // one-launch step: this CTA's whole units done
+  kTraceBuilt = 8,       // one-launch step, the laying-out CTA: split table published
+  kTraceTable = 9,       // the split table seen (after the wait for it)
+  kTraceRange = 10,      // this CTA's range of split items done
+  kTraceEnd = 11,        // about to leave
+  kTracePoints = 12
 };
 // Counters the kernels add to when they are on: keys attended with the
 // current query (fresh keys), pieces walked, units done whole, split units

@@ -64,6 +64,12 @@ __device__ __forceinline__ uint2 narrow4(const float4& v) {
   return make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
 }
 
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -572,6 +578,9 @@ __device__ __forceinline__ void match_body(const MatchParams& p, int u, MatchSme
   if (tid < D / 2) rope_sincos(p.rope_pos[b], p.inv_freq[tid], &rot_sn, &rot_cs);
   if (tid == 0) s_bad_page = 0;
   __syncthreads();
+  const bool traced = p.trace != nullptr && tid == 0 && (int)blockIdx.x < p.grid;
+  if (traced && p.trace[blockIdx.x * kTracePoints + kTraceLoaded] == 0)
+    p.trace[blockIdx.x * kTracePoints + kTraceLoaded] = globaltimer_ns();
 
   // 1. distances: mean over the G heads of sum((q - q_s)^2), for the slots
   // holding the occ most recent entries (age j = 0 is step n - 1, in slot
@@ -707,6 +716,8 @@ __device__ __forceinline__ void match_body(const MatchParams& p, int u, MatchSme
     __syncthreads();
   }
 
+  if (traced && p.trace[blockIdx.x * kTracePoints + kTraceDecided] == 0)
+    p.trace[blockIdx.x * kTracePoints + kTraceDecided] = globaltimer_ns();
   // paged KV: every page the step reads must be a valid pool page
   if (!s_plan.bad && p.page_size > 0) {
     const int pg0 = s_plan.start / p.page_size, pg1 = (s_plan.end - 1) / p.page_size;

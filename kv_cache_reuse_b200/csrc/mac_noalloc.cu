@@ -196,6 +196,7 @@ extern "C" int mac_dense_decode_static(const float* q_pre, const int* rope_pos, 
   mp.done = cnt + kMaxUnits;
   mp.dpart = nullptr;  // groups of up to 8 heads only: one match CTA per unit
   mp.ucnt = nullptr;
+  mp.trace = nullptr;
   mp.status = status;
   mp.B = batch;
   mp.Hq = num_q_heads;

@@ -395,10 +395,10 @@ def test_trace_counts_keys_and_orders_phases(one_launch):
             assert int(counters[1]) >= 1 and int(counters[2]) + int(counters[3]) >= 1
             keys.append((int(r.hit.all()), int(counters[0])))
             for row in stamps.astype(np.int64):
-                seen = [row[k] for k in (0, 1, 2, 3, 4, 5, 7) if row[k] > 0]
+                seen = [row[k] for k in (0, 1, 2, 3, 4, 7, 9, 10, 11) if row[k] > 0]
                 assert seen == sorted(seen), row
-                if row[6] > 0:  # the laying-out CTA published the table after its ticket
-                    assert row[2] <= row[6] and (row[4] == 0 or row[6] <= row[4])
+                if row[8] > 0:  # the laying-out CTA published the table after its ticket
+                    assert row[4] <= row[8] and (row[9] == 0 or row[8] <= row[9])
             assert (stamps[:, 0] > 0).any()
         per_ctx[L] = keys
         assert gpu.st.get_status() == 0
