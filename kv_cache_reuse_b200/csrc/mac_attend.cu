@@ -1023,7 +1023,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   unsigned smid;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
   const uint64_t pol = evict_first_policy();
-  auto stamp = [&](int k) {
+  auto stamp = [&](int k) __attribute__((always_inline)) {
     if (p.trace != nullptr && tid == 0) p.trace[cta * kTracePoints + k] = globaltimer();
   };
   stamp(kTraceStart);
@@ -1038,12 +1038,13 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   bool ok = true;
   unsigned long long t_first = 0, t_last = 0;  // thread 0: first and last box of the timed walk
   int cons0 = 0;                               // boxes consumed before the timed walk
-  auto range_of = [&](const Piece& pc) { return NC == 1 ? warp_range(pc, warp) : team_range(pc, kl, NKL); };
+  auto range_of = [&](const Piece& pc) __attribute__((always_inline)) { return NC == 1 ? warp_range(pc, warp) : team_range(pc, kl, NKL); };
 
   // One walk over the items of `table` from first_seg on whose cost range
   // meets [lo, hi), as range `slot` of the table's split.
+  // (forced inline: called twice, it must keep the accumulators in registers)
   auto walk = [&](const Segment* table, int nseg, int first_seg, long long lo, long long hi, int slot,
-                  bool timed, bool local) {
+                  bool timed, bool local) __attribute__((always_inline)) {
   // issue cursor: this warp's (NC > 1: this key-lane's) boxes of every piece, NSTT ahead
   Walker wi{first_seg, lo, hi, sm.items, first_seg, table, nseg, local};
   Piece ip;
@@ -1051,7 +1052,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   bool ivalid = issuer && wi.next(slot, ip);
   if (ivalid) ir = range_of(ip);
   int ib = ivalid ? ir.first : 0;
-  auto issue_advance = [&]() {
+  auto issue_advance = [&]() __attribute__((always_inline)) {
     while (ivalid && ib >= ir.nbox) {
       ivalid = wi.next(slot, ip);
       if (ivalid) {
@@ -1061,7 +1062,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       ++ipn;
     }
   };
-  auto issue_box = [&](int st) {
+  auto issue_box = [&](int st) __attribute__((always_inline)) {
     // warp 0 always owns box 0 of its range in every piece: it brings the query
     // (chunked groups read their query straight from global memory instead)
     const bool qfirst = NC == 1 && warp == 0 && ib == 0;
