@@ -328,13 +328,21 @@ __device__ void build_split_table(const MatchParams& p, int U, int grid, const i
   const int tid = threadIdx.x;
   const int nseg = 2 * U;
   const long long cost = p.piece_cost;
+  // the SM map and (when the items fit one pass) the plans in one round of loads
+  const int sm_ = tid < grid ? __ldcg(smid_of + tid) : -1;
+  UnitPlan pre;
+  pre.bad = 1;
+  if (nseg <= kMatchThreads && tid < nseg) {
+    const UnitPlan* pl = p.plan + (tid >> 1);
+    pre.bad = __ldcg(&pl->bad);
+    pre.start = __ldcg(&pl->start);
+    pre.cut = __ldcg(&pl->cut);
+    pre.end = __ldcg(&pl->end);
+  }
   wsum[tid] = 0;
   cta_on[tid] = -1;
   __syncthreads();
-  if (tid < grid) {
-    const int sm_ = __ldcg(smid_of + tid);
-    if (sm_ >= 0 && sm_ < grid) cta_on[sm_] = tid;
-  }
+  if (sm_ >= 0 && sm_ < grid) cta_on[sm_] = tid;
   __syncthreads();
   // ranges can be keyed by SM only if the CTAs sit on grid distinct SMs
   // with ids below grid (otherwise every slot is a CTA)
@@ -348,9 +356,18 @@ __device__ void build_split_table(const MatchParams& p, int U, int grid, const i
     int len = 0, key0 = 0, kind = kItemEmpty, cut = 0;
     long long wlen = 0;
     if (s < nseg) {
-      const UnitPlan* pl = p.plan + (s >> 1);
-      if (!__ldcg(&pl->bad)) {
-        const int start = __ldcg(&pl->start), c = __ldcg(&pl->cut), end = __ldcg(&pl->end);
+      UnitPlan pl;
+      if (nseg <= kMatchThreads) {
+        pl = pre;
+      } else {
+        const UnitPlan* pp = p.plan + (s >> 1);
+        pl.bad = __ldcg(&pp->bad);
+        pl.start = __ldcg(&pp->start);
+        pl.cut = __ldcg(&pp->cut);
+        pl.end = __ldcg(&pp->end);
+      }
+      if (!pl.bad) {
+        const int start = pl.start, c = pl.cut, end = pl.end;
         if (end - start <= p.unit_max) {
           if ((s & 1) == 0) atomicAdd(&wsum[(s >> 1) % grid], (unsigned long long)(end - start + cost));
         } else {
@@ -416,7 +433,10 @@ __device__ void build_split_table(const MatchParams& p, int U, int grid, const i
     const double sh = block_sum_d(in ? h : 0.0, dbuf);
     const double so = block_sum_d(in ? om : 0.0, dbuf);
     t = so > 0.0 ? ((double)S + sh) / so : 0.0;
-    in = active && om * t > h;
+    const bool next = active && om * t > h;
+    const int changed = __syncthreads_or(next != in);  // the same answer in every thread
+    in = next;
+    if (!changed) break;
   }
   const long long ri = active ? (long long)fmax(0.0, om * t - h) : 0;
   long long tot_r;
@@ -520,8 +540,14 @@ struct MatchSmem {
 // decision, the unit's plan, the rotated query and the window's new query.
 // Afterwards ms.s_plan holds the plan and ms.s_bad_page whether a page id
 // was invalid.
-template <int D, int GP, int GF, bool PH, bool RB>
-__device__ __forceinline__ void match_body(const MatchParams& p, int u, MatchSmem<D, GP, PH>& ms) {
+// A hook that does nothing (the match kernels).
+struct NoHook {
+  __device__ __forceinline__ void operator()(int, int) const {}
+};
+
+template <int D, int GP, int GF, bool PH, bool RB, typename Hook = NoHook>
+__device__ __forceinline__ void match_body(const MatchParams& p, int u, MatchSmem<D, GP, PH>& ms,
+                                           const Hook& hook = Hook()) {
   using RT = std::conditional_t<RB, uint2, float4>;  // four window elements
   const int G = GF > 0 ? GF : p.G;
   const int GD = G * D;
@@ -576,6 +602,9 @@ __device__ __forceinline__ void match_body(const MatchParams& p, int u, MatchSme
   // RoPE angle of pair i = tid (D/2 <= 64 threads)
   double rot_sn = 0.0, rot_cs = 1.0;
   if (tid < D / 2) rope_sincos(p.rope_pos[b], p.inv_freq[tid], &rot_sn, &rot_cs);
+  // the caller's work that needs the sequence length, issued while this
+  // unit's loads are in flight (the one-launch step prefetches the K/V tail)
+  hook(b, len);
   if (tid == 0) s_bad_page = 0;
   __syncthreads();
   const bool traced = p.trace != nullptr && tid == 0 && (int)blockIdx.x < p.grid;
