@@ -1110,8 +1110,9 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   // the first boxes of the walk go to the slots after the previous walk's last
   // (the consume side reads box n from slot n mod NSTT)
   for (int k = 0; k < NSTT && ivalid; ++k) issue_box(nissued % NSTT);
-  if (publish && tid == 0) {
-    // one-launch step: this CTA's plans go out while its first boxes are in flight
+  if (publish && tid == 1) {
+    // one-launch step: this CTA's plans go out while its first boxes are in
+    // flight (a lane that issued no copy, so its fence waits for no copy)
     __threadfence();
     asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.fsync) : "memory");
     if (p.trace != nullptr) p.trace[cta * kTracePoints + kTraceTicket] = globaltimer();
@@ -1259,33 +1260,31 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     const unsigned epoch = tid == 0 ? ld_relaxed_u32(p.fsync + 1) : 0u;
     if (tid == 0) sm.nlocal = 0;
     __syncthreads();
-    // Everything a unit's attention reads whatever its decision goes to L2
-    // while the match runs: the window's stored states (o, m, l of every
-    // slot: a hit reuses one of them) now, and the K/V tail [c_t, p_t] (read
-    // on a hit and on a miss alike) once the sequence length has arrived.
+    // While the match's own loads are in flight, everything the unit's
+    // attention may read goes to L2: the window's stored states (o, m, l of
+    // every slot: a hit reuses one of them) and the keys [p_t - W - band, p_t]
+    // (the tail, read on a hit and on a miss alike, and every amend band a
+    // hit on one of the last W positions can have).
     const int Wp1 = mp.W + 1;
-#pragma unroll 1
-    for (int u = cta; u < U; u += gridDim.x) {
-      const size_t ob = (size_t)Wp1 * G * D * (mp.ring_bf16 ? 2 : 4), mlb = (size_t)Wp1 * G * 4;
-      const unsigned char* ro = static_cast<const unsigned char*>(p.ring_o) + (size_t)u * ob;
-      for (size_t off = (size_t)tid * 128; off < ob; off += (size_t)kAttnThreads * 128) prefetch_l2(ro + off);
-      if ((size_t)tid * 128 < mlb) {
-        prefetch_l2(reinterpret_cast<const unsigned char*>(p.ring_m + (size_t)u * Wp1 * G) + tid * 128);
-        prefetch_l2(reinterpret_cast<const unsigned char*>(p.ring_l + (size_t)u * Wp1 * G) + tid * 128);
-      }
-    }
     // match stage of this CTA's units; whole units become local items
 #pragma unroll 1
     for (int u = cta; u < U; u += gridDim.x) {
       const int kvh_u = u % mp.Hkv;
       match_body<D, GP, GF, false, RB>(mp, u, ms, [&](int b, int len) __attribute__((always_inline)) {
+        const size_t ob = (size_t)Wp1 * G * D * (mp.ring_bf16 ? 2 : 4), mlb = (size_t)Wp1 * G * 4;
+        const unsigned char* ro = static_cast<const unsigned char*>(p.ring_o) + (size_t)u * ob;
+        for (size_t off = (size_t)tid * 128; off < ob; off += (size_t)kAttnThreads * 128) prefetch_l2(ro + off);
+        if ((size_t)tid * 128 < mlb) {
+          prefetch_l2(reinterpret_cast<const unsigned char*>(p.ring_m + (size_t)u * Wp1 * G) + tid * 128);
+          prefetch_l2(reinterpret_cast<const unsigned char*>(p.ring_l + (size_t)u * Wp1 * G) + tid * 128);
+        }
         if (len < 1 || len > mp.capacity) return;
         const int p_t = len - 1;
-        const int c = p_t - mp.band > 0 ? p_t - mp.band : 0;
+        const int c = p_t - mp.band - mp.W > 0 ? p_t - mp.band - mp.W : 0;
         const int kb0 = c & ~(kSubKeys - 1), nbox = (p_t - kb0) / kSubKeys + 1;
         if (mp.page_size > 0) {
-          // paged: the tail's block-table entries (a page id must arrive before
-          // its rows can be named, so the rows themselves are left to the walk)
+          // paged: the block-table entries (a page id must arrive before its
+          // rows can be named, so the rows themselves are left to the walk)
           const int* row = mp.block_table + (size_t)b * mp.max_pages;
           const int pg0 = kb0 / mp.page_size, pg1 = p_t / mp.page_size;
           for (int pg = pg0 + tid * 32; pg <= pg1; pg += kAttnThreads * 32) prefetch_l2(row + pg);
