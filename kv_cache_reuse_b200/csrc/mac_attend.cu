@@ -169,16 +169,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
-// Bring one TMA box into L2 (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-               : "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void* ptr) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, unsigned long long* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
@@ -1054,7 +1044,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   // meets [lo, hi), as range `slot` of the table's split.
   // (forced inline: called twice, it must keep the accumulators in registers)
   auto walk = [&](const Segment* table, int nseg, int first_seg, long long lo, long long hi, int slot,
-                  bool timed, bool local, bool publish) __attribute__((always_inline)) {
+                  bool timed, bool local) __attribute__((always_inline)) {
   // issue cursor: this warp's (NC > 1: this key-lane's) boxes of every piece, NSTT ahead
   Walker wi{first_seg, lo, hi, sm.items, first_seg, table, nseg, local};
   Piece ip;
@@ -1110,13 +1100,6 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   // the first boxes of the walk go to the slots after the previous walk's last
   // (the consume side reads box n from slot n mod NSTT)
   for (int k = 0; k < NSTT && ivalid; ++k) issue_box(nissued % NSTT);
-  if (publish && tid == 1) {
-    // one-launch step: this CTA's plans go out while its first boxes are in
-    // flight (a lane that issued no copy, so its fence waits for no copy)
-    __threadfence();
-    asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.fsync) : "memory");
-    if (p.trace != nullptr) p.trace[cta * kTracePoints + kTraceTicket] = globaltimer();
-  }
 
   // consume cursor
   Walker wc{first_seg, lo, hi, sm.items, first_seg, table, nseg, local};
@@ -1260,42 +1243,10 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     const unsigned epoch = tid == 0 ? ld_relaxed_u32(p.fsync + 1) : 0u;
     if (tid == 0) sm.nlocal = 0;
     __syncthreads();
-    // While the match's own loads are in flight, everything the unit's
-    // attention may read goes to L2: the window's stored states (o, m, l of
-    // every slot: a hit reuses one of them) and the keys [p_t - W - band, p_t]
-    // (the tail, read on a hit and on a miss alike, and every amend band a
-    // hit on one of the last W positions can have).
-    const int Wp1 = mp.W + 1;
     // match stage of this CTA's units; whole units become local items
 #pragma unroll 1
     for (int u = cta; u < U; u += gridDim.x) {
-      const int kvh_u = u % mp.Hkv;
-      match_body<D, GP, GF, false, RB>(mp, u, ms, [&](int b, int len) __attribute__((always_inline)) {
-        const size_t ob = (size_t)Wp1 * G * D * (mp.ring_bf16 ? 2 : 4), mlb = (size_t)Wp1 * G * 4;
-        const unsigned char* ro = static_cast<const unsigned char*>(p.ring_o) + (size_t)u * ob;
-        for (size_t off = (size_t)tid * 128; off < ob; off += (size_t)kAttnThreads * 128) prefetch_l2(ro + off);
-        if ((size_t)tid * 128 < mlb) {
-          prefetch_l2(reinterpret_cast<const unsigned char*>(p.ring_m + (size_t)u * Wp1 * G) + tid * 128);
-          prefetch_l2(reinterpret_cast<const unsigned char*>(p.ring_l + (size_t)u * Wp1 * G) + tid * 128);
-        }
-        if (len < 1 || len > mp.capacity) return;
-        const int p_t = len - 1;
-        const int c = p_t - mp.band - mp.W > 0 ? p_t - mp.band - mp.W : 0;
-        const int kb0 = c & ~(kSubKeys - 1), nbox = (p_t - kb0) / kSubKeys + 1;
-        if (mp.page_size > 0) {
-          // paged: the block-table entries (a page id must arrive before its
-          // rows can be named, so the rows themselves are left to the walk)
-          const int* row = mp.block_table + (size_t)b * mp.max_pages;
-          const int pg0 = kb0 / mp.page_size, pg1 = p_t / mp.page_size;
-          for (int pg = pg0 + tid * 32; pg <= pg1; pg += kAttnThreads * 32) prefetch_l2(row + pg);
-          return;
-        }
-        constexpr int H = Cfg<D, GP>::HALVES;
-        for (int i = tid; i < nbox * 2 * H; i += kAttnThreads) {
-          const int box = i / (2 * H), kv = (i / H) & 1, hf = i % H;
-          tma_prefetch_4d(kv ? &p.tmV : &p.tmK, 64 * hf, kvh_u, kb0 + box * kSubKeys, b);
-        }
-      });
+      match_body<D, GP, GF, false, RB>(mp, u, ms);
       __syncthreads();
       if (tid == 0) {
         const UnitPlan pl = ms.s_plan;
@@ -1323,18 +1274,14 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     // its plans (it holds a unit only when there are as many units as CTAs, so
     // the layout seldom waits behind a match or delays a whole unit)
     const int builder = (int)gridDim.x - 1;
-    // a CTA with whole units arrives once its first boxes are in flight (in
-    // its walk below), the others now
-    const bool late_arrival = cta != builder && sm.nlocal > 0;
     if (tid == 0) {
       p.smid_of[cta] = (int)smid;
-      if (cta != builder && !late_arrival) {
+      if (cta != builder) {
         // the block barrier above orders every thread's writes before this
         // thread's device-scope fence; the arrival then publishes them
         __threadfence();
         asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.fsync) : "memory");
-        if (p.trace) p.trace[cta * kTracePoints + kTraceTicket] = globaltimer();
-      } else if (cta == builder) {
+      } else {
         const unsigned long long t0 = globaltimer();
         while ((int)ld_acquire_u32(p.fsync) != builder) {
           if (globaltimer() - t0 > kWaitLimitNs) {
@@ -1343,13 +1290,13 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
             break;
           }
         }
-        if (p.trace) p.trace[cta * kTracePoints + kTraceTicket] = globaltimer();
       }
+      if (p.trace) p.trace[cta * kTracePoints + kTraceTicket] = globaltimer();
     }
     __syncthreads();
     if (cta == builder) {
-      // every other CTA's plans and SM id precede its arrival (acquired by
-      // thread 0, ordered for the others by the barrier): lay out the split items
+      // every other CTA's plans and SM id precede its arrival: lay out the split items
+      __threadfence();
       static_assert(sizeof(SplitScratch) <= sizeof(sm.kv), "split scratch lives in the box slots");
       build_split_table(mp, U, (int)gridDim.x, p.smid_of, p.rank_of,
                         *reinterpret_cast<SplitScratch*>(&sm.kv[0][0][0][0]));
@@ -1357,7 +1304,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       __syncthreads();
       if (tid == 0) {
         p.fsync[0] = 0;
-        // every thread's table writes, ordered by the barrier, go out with the epoch
+        __threadfence();  // every thread's table writes, ordered by the barrier, before the epoch
         st_release_u32(p.fsync + 1, epoch + 1u);
         if (p.trace) p.trace[cta * kTracePoints + kTraceBuilt] = globaltimer();
       }
@@ -1365,7 +1312,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
     __syncthreads();
     // this CTA's whole units
     const int nlocal = sm.nlocal;
-    if (nlocal > 0) walk(sm.items, nlocal, 0, 0, LLONG_MAX, cta, false, true, late_arrival);
+    if (nlocal > 0) walk(sm.items, nlocal, 0, 0, LLONG_MAX, cta, false, true);
     stamp(kTraceLocal);
     // the step's split table (bounded wait for the last CTA's layout)
     if (tid == 0 && ok) {
@@ -1431,7 +1378,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
   if (ok && lo < hi) {
     if (tid < kItemCache && first_seg + tid < p.nseg) sm.items[tid] = load_segment(p.seg + first_seg + tid);
     __syncthreads();
-    walk(p.seg, p.nseg, first_seg, lo, hi, slot, true, false, false);
+    walk(p.seg, p.nseg, first_seg, lo, hi, slot, true, false);
     stamp(kTraceRange);
   }
   if (weighted && p.rate != nullptr) {
