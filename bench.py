@@ -47,10 +47,11 @@ def _peaks():
 
 
 def _kernel_hash() -> str:
-    """Hash of the attention kernel's source code (comments and blank space
-    removed, so that a comment edit does not orphan a profile)."""
+    """Hash of the step kernel's source code (the attention file, the match
+    stage it includes and the shared layout; comments and blank space removed,
+    so that a comment edit does not orphan a profile)."""
     h = hashlib.sha256()
-    for f in ("mac_attend.cu", "mac_internal.cuh"):
+    for f in ("mac_attend.cu", "mac_internal.cuh", "mac_match_dev.cuh"):
         with open(os.path.join(ROOT, "kv_cache_reuse_b200", "csrc", f)) as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -60,9 +61,9 @@ def _kernel_hash() -> str:
 
 
 def _profiled_traffic():
-    """Ratio of DRAM bytes to algorithmic bytes of the attention kernel from the
+    """Ratio of DRAM bytes to algorithmic bytes of the step kernel from the
     committed ncu summary, if it was taken on the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "mac_attend_long_128k_traffic.txt")
+    p = os.path.join(ROOT, "profiles", "mac_step_long_128k_traffic.txt")
     try:
         txt = open(p).read()
     except OSError:
@@ -406,6 +407,13 @@ def run_mac(args, rank, world, local_rank):
                   "long_128k_mixed": run_trace(wl, args.trace_steps, dev, peak),
                   "paged_mixed_all_hit": run_trace(synth.WORKLOADS["paged_mixed"].with_(hit_model=("iid", 1.0)),
                                                    args.trace_steps, dev, peak)}
+    paged_gap = None
+    if args.miss_steps > 0 and args.paged_gap:
+        # paged against contiguous K/V at the same size, every step a miss: the
+        # paged_mixed shape (16 sequences of 8K-64K keys) in both layouts
+        wp = synth.WORKLOADS["paged_mixed"].with_(tau=0.0)
+        paged_gap = {"paged": run_shape(wp, 4, dev, peak, nwarm=3),
+                     "contiguous": run_shape(wp.with_(page_size=0), 4, dev, peak, nwarm=3)}
     hitshapes = []
     if args.hit_steps > 0 and args.hit_shapes:
         hitshapes = [run_hit_shape(n, args.hit_steps, dev, peak, world) for n in args.hit_shapes.split(",") if n]
@@ -464,6 +472,13 @@ def run_mac(args, rank, world, local_rank):
             roof["hit"]["vs_context"] = [
                 {"context": L, "step_us": r["total_ms"] * 1e3 / len(r["step_ms"]),
                  "step_mb": (r["att_bytes"] + r["match_bytes"]) / len(r["step_ms"]) / 1e6} for L, r in hitctx]
+    if paged_gap:
+        roof.setdefault("miss", {})["paged_vs_contiguous"] = {
+            "workload": "paged_mixed shape, threshold 0 (every unit misses)",
+            "paged_frac": paged_gap["paged"]["step"]["frac"], "contiguous_frac": paged_gap["contiguous"]["step"]["frac"],
+            "paged_attend_frac": paged_gap["paged"]["attend"]["frac"],
+            "contiguous_attend_frac": paged_gap["contiguous"]["attend"]["frac"]}
+        detail["paged_vs_contiguous"] = paged_gap
     if mqa:
         a = mqa["all_miss"]["attend"]
         roof.setdefault("miss", {})["mqa_32_1"] = {"frac": a["frac"], "achieved": a["achieved"], "mb_per_launch": a["mb_per_launch"],
@@ -912,6 +927,8 @@ def main():
                     help="also time a stack of this many layers per token, one CUDA graph per token (0 = skip)")
     ap.add_argument("--trace-steps", type=int, default=12,
                     help="steps of the device phase trace runs (0 = skip)")
+    ap.add_argument("--no-paged-gap", dest="paged_gap", action="store_false",
+                    help="skip the paged-against-contiguous all-miss runs")
     ap.add_argument("--mqa-steps", type=int, default=8,
                     help="timed steps of the 32-query-heads-over-one-KV-head runs (0 = skip)")
     ap.add_argument("--hit-shapes", default="paged_mixed,continuous_16k",
