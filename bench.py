@@ -239,8 +239,10 @@ def run_mac(args, rank, world, local_rank):
         the step.  split=True: events also between the two kernels, for the
         per-kernel roofline.  The timed steps are queued behind a GPU sleep so the
         host stays ahead of the device and no host latency enters the events."""
-        cfg = cfg or {}
+        cfg = dict(cfg or {})
+        one_launch = cfg.pop("one_launch", 1)
         st = mac.MacState.for_workload(wl, tau=tau, **kw, **cfg)
+        mac.mac_set_one_launch(st, one_launch)
         h = st.handle
         nd = Hq if cfg.get("match_per_head") else Hkv  # decisions per sequence
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -308,6 +310,9 @@ def run_mac(args, rank, world, local_rank):
         main = timed_run(wl.tau, args.warmup, args.steps, split=False)
     main["clocks"]["remeasured"] = remeasured
     kern = timed_run(wl.tau, args.warmup, args.steps, split=True)
+    # the same steps as two launches (match kernel, then attention kernel with
+    # programmatic dependent launch), timed as the main run is
+    main2 = timed_run(wl.tau, args.warmup, args.steps, split=False, cfg={"one_launch": 0})
     allmiss = allmiss2 = None
     if args.miss_steps > 0:
         nm = min(args.miss_steps, T - 3)
@@ -449,7 +454,8 @@ def run_mac(args, rank, world, local_rank):
             if _profiled_traffic() else None,
             "bytes_per_launch": (main["att_bytes"] + main["match_bytes"]) / K_,
             "us_per_launch": main["total_ms"] * 1e3 / K_,
-            "two_launch": two_launch(kern, K_)}
+            "two_launch": dict(two_launch(kern, K_), steps_per_s=K_ / (main2["total_ms"] * 1e-3),
+                               step_us_back_to_back=main2["total_ms"] * 1e3 / K_)}
     detail = {}
     if allmiss:
         n = len(allmiss["step_ms"])
