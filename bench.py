@@ -298,8 +298,13 @@ def run_mac(args, rank, world, local_rank):
             kv_b += c
             dense_b += synth.dense_equiv_kv_bytes(wl, cur["stream"].seq_lens[t])
         tot_ms = float(np.sum(step_ms))
+        allhit = [bool(hits[i].all()) for i in range(nsteps)]
+        by_class = {k: (float(np.mean([step_ms[i] for i in range(nsteps) if allhit[i] == v])) * 1e3
+                        if any(allhit[i] == v for i in range(nsteps)) else None)
+                    for k, v in (("all_hit_us", True), ("with_miss_us", False))}
+        by_class["with_miss_steps"] = int(nsteps - sum(allhit))
         return dict(total_ms=tot_ms, step_ms=step_ms, att_ms=float(np.sum(att_ms)), match_ms=float(np.sum(match_ms)),
-                    one_launch=one,
+                    one_launch=one, by_class=by_class,
                     att_bytes=at_b, match_bytes=mt_b, kv_bytes=kv_b, dense_bytes=dense_b,
                     hit_frac=float(hits.mean()), status=status, clocks=clocks.summary())
 
@@ -411,7 +416,8 @@ def run_mac(args, rank, world, local_rank):
         traces = {"long_128k_all_hit": run_trace(wl.with_(hit_model=("iid", 1.0)), args.trace_steps, dev, peak),
                   "long_128k_mixed": run_trace(wl, args.trace_steps, dev, peak),
                   "paged_mixed_all_hit": run_trace(synth.WORKLOADS["paged_mixed"].with_(hit_model=("iid", 1.0)),
-                                                   args.trace_steps, dev, peak)}
+                                                   args.trace_steps, dev, peak),
+                  "mqa_32_1_all_miss": run_trace(wl.with_(Hq=32, Hkv=1, tau=0.0), 4, dev, peak)}
     paged_gap = None
     if args.miss_steps > 0 and args.paged_gap:
         # paged against contiguous K/V at the same size, every step a miss: the
@@ -454,8 +460,9 @@ def run_mac(args, rank, world, local_rank):
             if _profiled_traffic() else None,
             "bytes_per_launch": (main["att_bytes"] + main["match_bytes"]) / K_,
             "us_per_launch": main["total_ms"] * 1e3 / K_,
+            "by_class": main["by_class"],
             "two_launch": dict(two_launch(kern, K_), steps_per_s=K_ / (main2["total_ms"] * 1e-3),
-                               step_us_back_to_back=main2["total_ms"] * 1e3 / K_)}
+                               step_us_back_to_back=main2["total_ms"] * 1e3 / K_, by_class=main2["by_class"])}
     detail = {}
     if allmiss:
         n = len(allmiss["step_ms"])
