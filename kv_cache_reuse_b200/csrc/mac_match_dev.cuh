@@ -302,8 +302,9 @@ __device__ double block_sum_d(double v, double* sbuf) {
 // its keys plus the fixed piece cost.  The space is cut into one range per
 // slot -- per SM on large steps (each SM's range sized by its learned
 // streaming rate), per CTA otherwise -- such that each slot's whole-unit work
-// plus its range comes out proportional to its weight: with weights w_r and
-// whole work h_r, range r holds max(0, w_r t - h_r) cost units, t chosen so
+// (its keys plus an eighth of the piece cost) plus its range comes out
+// proportional to its weight: with weights w_r and whole work h_r, range r
+// holds max(0, w_r t - h_r) cost units, t chosen so
 // the ranges add up to the split work (water filling).  Small steps use
 // only the last ceil(S / min_keys) CTAs.  Empty ranges are dropped and the
 // rest numbered in slot order (their rank): the items' first range and
@@ -369,7 +370,10 @@ __device__ void build_split_table(const MatchParams& p, int U, int grid, const i
       if (!pl.bad) {
         const int start = pl.start, c = pl.cut, end = pl.end;
         if (end - start <= p.unit_max) {
-          if ((s & 1) == 0) atomicAdd(&wsum[(s >> 1) % grid], (unsigned long long)(end - start + cost));
+          // a whole unit delays its CTA's range by about its keys plus an eighth
+          // of a piece's fixed cost (traced: a hit unit of ~270 keys holds its
+          // CTA ~5 us, the time to stream ~430 keys on one SM)
+          if ((s & 1) == 0) atomicAdd(&wsum[(s >> 1) % grid], (unsigned long long)(end - start + cost / 8));
         } else {
           len = (s & 1) ? end - c : c - start;
           key0 = (s & 1) ? c : start;
