@@ -143,6 +143,19 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t 
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of phase `parity` (a polling loop over several barriers
+// uses it: try_wait may hold the thread for a while on one of them).
+__device__ __forceinline__ bool mbar_test(unsigned long long* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait on phase `parity` of an mbarrier.  Returns false if the CTA
 // is aborting or the wait exceeded kWaitLimitNs (then it flags the abort).
 __device__ bool mbar_wait(unsigned long long* bar, uint32_t parity, volatile int* abort_flag,
@@ -434,8 +447,8 @@ __device__ __forceinline__ void process_box(Acc<D, GP>& A, const uint16_t* kbox,
 }
 
 // Bounded barrier of the 8 consumer warps (mbarrier with one arrival per warp).
-template <int D, int GP>
-__device__ __forceinline__ bool consumer_sync(AttnSmem<D, GP>& sm, uint32_t& phase, unsigned* status) {
+template <typename SM>
+__device__ __forceinline__ bool consumer_sync(SM& sm, uint32_t& phase, unsigned* status) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.csync);
   const bool ok = mbar_wait(&sm.csync, phase, &sm.abort_flag, status);
@@ -444,8 +457,8 @@ __device__ __forceinline__ bool consumer_sync(AttnSmem<D, GP>& sm, uint32_t& pha
   return ok;
 }
 
-template <int D, int GP, int NH>
-__device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA, int idx, int h, float& MA,
+template <int D, int GP, int NH, typename SM>
+__device__ __forceinline__ void combine_warps2(const SM& sm, int wA, int idx, int h, float& MA,
                                                float& LA, float& OA, float& MB, float& LB, float& OB);
 
 // Fold one state (max m, sum l, outputs o relative to 2^m) into (M, L, O).
@@ -503,8 +516,8 @@ __device__ __forceinline__ void warp_combine_store(Acc<D, GP>& A, float* wb) {
 // Merge the warps' states for element idx of head h, from slots laid out as
 // o [NH][D], m [NH], l [NH]: warps below wA into (MA, LA, OA), the others
 // into (MB, LB, OB); sums relative to 2^M.
-template <int D, int GP, int NH>
-__device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA, int idx, int h, float& MA,
+template <int D, int GP, int NH, typename SM>
+__device__ __forceinline__ void combine_warps2(const SM& sm, int wA, int idx, int h, float& MA,
                                                float& LA, float& OA, float& MB, float& LB, float& OB) {
   float m[kConsumerWarps], l[kConsumerWarps], o[kConsumerWarps];
 #pragma unroll
@@ -543,8 +556,8 @@ __device__ __forceinline__ void combine_warps2(const AttnSmem<D, GP>& sm, int wA
 // Chunked groups (NC > 1, G = 8 NC heads per KV head): the call finishes the
 // 8 heads of chunk ch, whose states the warps' slots and sm.ring hold; the
 // global layouts are those of the whole group.
-template <int D, int GP, int GF, int NC = 1>
-__device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D, GP>& sm, int u, int wA, int hit,
+template <int D, int GP, int GF, int NC = 1, typename SM>
+__device__ __forceinline__ void unit_epilogue(const AttendParams& p, SM& sm, int u, int wA, int hit,
                                               int hmask, int dst, int end, int ch = 0) {
   constexpr int GDP = Cfg<D, GP>::GD;
   const int G = NC > 1 ? GP : group_of<GF>(p), GD = G * D;  // heads of this call, and their elements
@@ -597,11 +610,16 @@ __device__ __forceinline__ void unit_epilogue(const AttendParams& p, AttnSmem<D,
 // rest, in proportion to their counts -- and each folds its own into one
 // state (lane: four consecutive elements of every 128, KB partials per round
 // of loads); the finish of a whole unit then combines the eight states.
-template <int D, int GP, int GF, bool PH, int NC = 1>
-__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
+// (SM: the attention kernel's shared memory, or the merge kernel's, which
+// has the same warp slots, ring buffer and barrier.  Chunked groups: chunks
+// [ch0, ch1) of the unit; KBO: partials per warp and round of loads, 0 for
+// the attention kernel's register budget.)
+template <int D, int GP, int GF, bool PH, int NC = 1, int KBO = 0, typename SM>
+__device__ __noinline__ bool merge_unit(const AttendParams& p, SM& sm, int u, uint32_t& sync_phase, int ch0 = 0,
+                                        int ch1 = NC) {
   using C = Cfg<D, GP>;
-  constexpr int NCH = C::GD / 128;                // 128-element runs of a padded group: 2, 4 or 8
-  constexpr int KB = NCH <= 2 ? 8 : 16 / NCH;     // partials per round of loads
+  constexpr int NCH = C::GD / 128;                                   // 128-element runs of a padded group: 2, 4 or 8
+  constexpr int KB = KBO > 0 ? KBO : (NCH <= 2 ? 8 : 16 / NCH);     // partials per round of loads
   // chunked groups (NC > 1): the unit's 8 NC heads are merged 8 at a time;
   // chunk ch of a partial is a run of partial_floats(8, D) floats at ch times that
   const int G = NC > 1 ? GP : group_of<GF>(p), GD = G * D, G4 = group4(G);  // heads of one chunk
@@ -622,7 +640,7 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& 
   const bool onA = warp < wA;
   const int cnt = onA ? nA : nB, stride = onA ? wA : kConsumerWarps - wA, first = onA ? warp : warp - wA;
 #pragma unroll 1
-  for (int ch = 0; ch < NC; ++ch) {
+  for (int ch = ch0; ch < ch1; ++ch) {
     const int h0 = ch * G;  // first head of this chunk in the unit
     const float* const part = p.part + (size_t)(onA ? sA.pbase : sB.pbase) * PF + (size_t)ch * (GD + 2 * G4);
     // the reused state on chip, in the layout of a whole unit's copy: each
@@ -1433,6 +1451,642 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   attend_body<D, GP, GF, false, 1, true, RB>(p, mp);
 }
 
+// ============================================================ tcgen05 path
+// Groups of 16, 32 or 64 query heads per KV head at head_dim 128: here the
+// group is a real dense tile, so both products run on the fifth-generation
+// tensor cores (tcgen05.mma, operands in shared memory, accumulators in
+// tensor memory).  Per tile of 128 keys of one unit:
+//   S^T [128 keys x N] = K [128 x D] . [Q_hi; Q_res]^T
+//   O^T [D x N]       += V^T [D x 128 keys] . [P_hi | P_res]   (V read as stored,
+//                                                               the MN-major operand)
+// The query and the weights are split into a bf16 high part and a bf16
+// residual (~16 mantissa bits, as in the box kernel), stacked along N: the
+// columns of S and O are the G heads' high parts, then their residuals
+// (padded to N = 64), and a head's value is the sum of its two columns.
+// Warp 0 streams the K tiles and warp 2 the V tiles (16-key TMA boxes, each
+// ring with its own barriers, so a K buffer returns to the stream as soon as
+// its product is done), one thread of warp 1 issues the MMAs as their inputs
+// arrive (S double-buffered in TMEM, O in TMEM), warps 4-7 run the softmax:
+// thread k owns key k of the tile (TMEM lane k) and keeps its keys' running
+// sums per head in registers; O is rescaled only when some head's maximum
+// grows by more than 2^8 (weights stay below 256).  Every piece (a unit's keys
+// in this CTA's range) ends in a partial in the chunk-major layout, and a
+// second kernel merges each unit's partials with its reused state
+// (merge_unit).
+namespace tc {
+constexpr int kKeys = 128;     // keys per tile: M of QK, K of PV
+constexpr int kSoftWarp0 = 4;  // softmax warps 4..7 (TMEM lanes 32 (w % 4) ..)
+// Columns of S and of O: high parts and residuals of the G heads, at least 64.
+__host__ __device__ constexpr int ncols(int G) { return 2 * G < 64 ? 64 : 2 * G; }
+// Tiles in flight per ring and buffers of the weights P^T (shared memory:
+// 2 + 3 tiles of K and V beside a 64-column query and two 64-column weight
+// tiles; 2 + 3 beside 128-column ones and one weight tile).
+__host__ __device__ constexpr int stages_k(int G) { return 2; }
+__host__ __device__ constexpr int stages_v(int G) { return 3; }
+__host__ __device__ constexpr int p_bufs(int G) { return G <= 32 ? 2 : 1; }
+// Tensor memory: S[2] and O, N columns each, rounded to a power of two.
+__host__ __device__ constexpr uint32_t tmem_cols(int G) { return 3 * ncols(G) <= 256 ? 256u : 512u; }
+}  // namespace tc
+
+// Shared memory of the tcgen05 kernel: the 128-byte-swizzled tiles first (each
+// a multiple of 1 KB from a 1 KB-aligned base), then the small fields.
+template <int G>
+struct TcSmem {
+  static constexpr int N = tc::ncols(G), SK = tc::stages_k(G), SV = tc::stages_v(G), NPB = tc::p_bufs(G);
+  uint16_t k[SK][2][tc::kKeys * 64];  // [stage][half of D][128 keys][64 dims]
+  uint16_t v[SV][2][tc::kKeys * 64];
+  uint16_t q[2][N * 64];              // [half of D][N rows: Q_hi, Q_res, zero][64 dims]
+  uint16_t pw[NPB][N / 64][tc::kKeys * 64];  // P^T: [buffer][64-column block][128 keys][64 columns]
+  float m[G];                         // running maximum per head (log2 units)
+  float red[4][G];                    // cross-warp reductions of the softmax warps
+  unsigned long long full_k[SK], empty_k[SK], full_v[SV], empty_v[SV], s_full[2], s_empty[2];
+  unsigned long long p_full[NPB], p_empty[NPB], q_full, drain;
+  uint32_t tmem;
+  int abort_flag;
+  int last_flag;
+};
+
+template <int D>
+struct MergeSmem {
+  float wbuf[kConsumerWarps][Cfg<D, 8>::WB];
+  alignas(16) float ring[Cfg<D, 8>::SF];
+  unsigned long long csync;
+  int abort_flag;
+};
+
+// Byte offset of element (row, col) of a [rows][64] bf16 tile with the
+// 128-byte swizzle (16-byte chunk c of row r at c ^ (r & 7)).
+__device__ __forceinline__ uint32_t sw128_off(int row, int col64) {
+  return (uint32_t)(row * 128 + ((((col64 >> 3) & 7) ^ (row & 7)) << 4) + (col64 & 7) * 2);
+}
+// Shared-memory matrix descriptor (tcgen05): start, leading and stride byte
+// offsets, descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr & 0x3FFFF) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, the
+// operands' majorness, N and M.
+__host__ __device__ constexpr uint32_t umma_idesc(int a_mn, int b_mn, int N, int M) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred pa;\n\tsetp.ne.u32 pa, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, pa;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(unsigned long long* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// 32 consecutive fp32 columns into this warp's 32 TMEM lanes (thread i: lane i).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// Named barrier of the four softmax warps, with an OR of one flag.
+__device__ __forceinline__ int softmax_sync_or(int flag) {
+  int out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 128, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"(flag)
+      : "memory");
+  return out;
+}
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// A CTA role's walk over its pieces, tile by tile.
+struct TileCursor {
+  Walker w;
+  Piece pc;
+  int ntile, i, np;  // tiles of the piece, next tile in it, index of the piece
+  bool live;
+  __device__ __forceinline__ void open(int slot) {
+    live = w.next(slot, pc);
+    ntile = live ? (pc.k1 - pc.kb0 + tc::kKeys - 1) / tc::kKeys : 0;
+    i = 0;
+  }
+  __device__ __forceinline__ void step(int slot) {
+    if (++i >= ntile) {
+      ++np;
+      open(slot);
+    }
+  }
+};
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes, issued without
+// waiting; tmem_ld_wait() completes every load issued so far and ties the
+// registers to that point.
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+template <int NR>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < NR; ++j) asm volatile("" : "+r"(r[j]));
+}
+// Heads [h0, h0 + HC) of this thread's TMEM lane at accumulator column base
+// `base`: the high-part column plus the residual column (HC = 16 for groups of
+// 16, whose 32 columns come in one load; else 32).
+template <int G>
+__device__ __forceinline__ void tmem_heads(uint32_t base, int h0, float* v) {
+  if constexpr (G == 16) {
+    uint32_t a[32];
+    tmem_ld32_issue(base, a);
+    tmem_ld_wait<32>(a);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(a[j]) + __uint_as_float(a[16 + j]);
+  } else {
+    uint32_t a[64];
+    tmem_ld32_issue(base + h0, a);
+    tmem_ld32_issue(base + G + h0, a + 32);
+    tmem_ld_wait<64>(a);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) + __uint_as_float(a[32 + j]);
+  }
+}
+
+// One ring of K or V tiles: boxes of 16 keys x 64 dims (two per key row of
+// 128 dims) into stage t % S, never across a page; a tile's boxes past the
+// piece's last key are not loaded.  Leaves once its copies have landed.
+template <int S>
+__device__ __forceinline__ void tc_stream(const AttendParams& p, const CUtensorMap* map, uint16_t (*ring)[2][tc::kKeys * 64],
+                                          unsigned long long* full, unsigned long long* empty, TileCursor c, int slot,
+                                          volatile int* abort_flag, uint64_t pol, unsigned long long* counters) {
+  constexpr uint32_t kBox = 16 * 64 * 2;
+  unsigned long long nkeys = 0, npieces = 0;
+  int t = 0;
+  while (c.live) {
+    const int b = c.pc.unit / p.Hkv, kvh = c.pc.unit - b * p.Hkv;
+    const int key0 = c.pc.kb0 + c.i * tc::kKeys, st = t % S;
+    if (c.i == 0) {
+      nkeys += (unsigned long long)(c.pc.k1 - c.pc.k0);
+      ++npieces;
+    }
+    if (t >= S && !mbar_wait(&empty[st], (uint32_t)((t / S) - 1) & 1u, abort_flag, p.status)) break;
+    const int left = (c.pc.k1 - key0 + kSubKeys - 1) / kSubKeys;
+    const int nb = left < tc::kKeys / kSubKeys ? left : tc::kKeys / kSubKeys;
+    mbar_arrive_expect_tx(&full[st], (uint32_t)nb * 2u * kBox);
+    for (int j = 0; j < nb; ++j) {
+      const int key = key0 + kSubKeys * j;
+      int c2, c3;
+      if (p.page_size > 0) {
+        c3 = p.block_table[(size_t)b * p.max_pages + key / p.page_size];
+        c2 = key % p.page_size;
+      } else {
+        c2 = key;
+        c3 = b;
+      }
+      tma_load_4d(ring[st][0] + j * kSubKeys * 64, map, &full[st], 0, kvh, c2, c3, pol);
+      tma_load_4d(ring[st][1] + j * kSubKeys * 64, map, &full[st], 64, kvh, c2, c3, pol);
+    }
+    ++t;
+    c.step(slot);
+  }
+  // every copy issued has landed before the CTA leaves (bounded)
+  for (int tt = t - S < 0 ? 0 : t - S; tt < t; ++tt) {
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(&full[tt % S], (uint32_t)(tt / S) & 1u) && globaltimer() - t0 < kWaitLimitNs) {
+    }
+  }
+  if (counters != nullptr && npieces > 0) {
+    atomicAdd(counters + kCountKeys, nkeys);
+    atomicAdd(counters + kCountPieces, npieces);
+  }
+}
+
+template <int GF>
+__global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __grid_constant__ AttendParams p) {
+  constexpr int D = 128, G = GF, N = tc::ncols(G), SK = TcSmem<G>::SK, SV = TcSmem<G>::SV, NPB = TcSmem<G>::NPB;
+  static_assert(G == 16 || G == 32 || G == 64, "groups of 16, 32 or 64 heads");
+  constexpr int HC = G == 16 ? 16 : 32;  // heads per pass over the accumulator columns
+  constexpr int GDc = 8 * D, PFc = GDc + 16;  // one 8-head chunk of a partial: o [8][D], m [8], l [8]
+  constexpr uint32_t kCols = tc::tmem_cols(G), kColO = 2 * N;  // S[0] at 0, S[1] at N, O at 2N
+  constexpr uint32_t idesc_qk = umma_idesc(0, 0, N, tc::kKeys);
+  constexpr uint32_t idesc_pv = umma_idesc(1, 1, N, tc::kKeys);
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  TcSmem<G>& sm = *reinterpret_cast<TcSmem<G>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cta = blockIdx.x;
+  if (tid == 32) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmK)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmV)) : "memory");
+  }
+  if (tid == 0) {
+    for (int s_ = 0; s_ < SK; ++s_) {
+      mbar_init(&sm.full_k[s_], 1);
+      mbar_init(&sm.empty_k[s_], 1);
+    }
+    for (int s_ = 0; s_ < SV; ++s_) {
+      mbar_init(&sm.full_v[s_], 1);
+      mbar_init(&sm.empty_v[s_], 1);
+    }
+    for (int s_ = 0; s_ < 2; ++s_) {
+      mbar_init(&sm.s_full[s_], 1);
+      mbar_init(&sm.s_empty[s_], 4);
+    }
+    for (int s_ = 0; s_ < NPB; ++s_) {
+      mbar_init(&sm.p_full[s_], 4);
+      mbar_init(&sm.p_empty[s_], 1);
+    }
+    mbar_init(&sm.q_full, 4);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (p.trace != nullptr) p.trace[cta * kTracePoints + kTraceStart] = globaltimer();
+  }
+  __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the CTA's range of the cost space (as in the attention kernel)
+  unsigned smid;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+  const int n_cta = p.hdr->n_cta, weighted = p.hdr->weighted;
+  const long long T = p.hdr->total;
+  int first_seg = p.first_seg[cta];
+  int slot = cta;
+  long long lo, hi;
+  if (weighted) {
+    if (tid == 0) {
+      int c = (p.claim != nullptr && (int)smid < p.grid && atomicCAS(p.claim + smid, 0, 1) == 0) ? (int)smid : -1;
+      for (int k = 0; c < 0 && k < n_cta; ++k)
+        if (atomicCAS(p.claim + k, 0, 1) == 0) c = k;
+      sm.last_flag = c;
+    }
+    __syncthreads();
+    slot = sm.last_flag;
+    if (slot < 0) return;
+    lo = p.bounds[slot];
+    hi = p.bounds[slot + 1];
+    first_seg = p.first_seg[slot];
+  } else {
+    if (cta >= n_cta) return;
+    lo = (long long)cta * T / n_cta;
+    hi = (long long)(cta + 1) * T / n_cta;
+  }
+  // tensor memory for S[2] and O
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
+                 "r"(kCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  volatile int* abort_flag = &sm.abort_flag;
+  // every role walks the items from global memory (no shared copy: the base
+  // puts them all past the cache)
+  TileCursor cur;
+  cur.w = Walker{first_seg, lo, hi, nullptr, first_seg - kItemCache, p.seg, p.nseg, false};
+  cur.np = 0;
+  cur.open(slot);
+
+  if (warp == 0 || warp == 2) {
+    // ---- the K stream (warp 0) and the V stream (warp 2)
+    if (lane == 0) {
+      const uint64_t pol = evict_first_policy();
+      if (warp == 0)
+        tc_stream<SK>(p, &p.tmK, sm.k, sm.full_k, sm.empty_k, cur, slot, abort_flag, pol, p.counters);
+      else
+        tc_stream<SV>(p, &p.tmV, sm.v, sm.full_v, sm.empty_v, cur, slot, abort_flag, pol, nullptr);
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer: QK of tile tq and PV of tile tp, whichever has its inputs
+    if (lane == 0) {
+      TileCursor cq = cur, cv = cur;
+      int tq = 0, tp = 0;
+      bool idle = false;
+      unsigned long long idle0 = 0;
+      while (cv.live) {
+        bool prog = false;
+        if (cq.live) {
+          const int sb = tq & 1, st = tq % SK;
+          if ((cq.i != 0 || mbar_test(&sm.q_full, (uint32_t)cq.np & 1u)) &&
+              mbar_test(&sm.full_k[st], (uint32_t)(tq / SK) & 1u) &&
+              (tq < 2 || mbar_test(&sm.s_empty[sb], (uint32_t)((tq >> 1) - 1) & 1u))) {
+            tc_fence_after();
+            if (tq == 0 && p.trace != nullptr) p.trace[cta * kTracePoints + kTraceFirstBox] = globaltimer();
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const int half = ks >> 2, kin = ks & 3;
+              const uint64_t a = umma_desc(smem_u32(sm.k[st][half]) + kin * 32, 16, 1024);
+              const uint64_t b = umma_desc(smem_u32(sm.q[half]) + kin * 32, 16, 1024);
+              umma(tmem + (uint32_t)(N * sb), a, b, idesc_qk, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[sb]);
+            umma_commit(&sm.empty_k[st]);
+            ++tq;
+            cq.step(slot);
+            prog = true;
+          }
+        }
+        if (tp < tq) {
+          const int st = tp % SV, pb = tp % NPB;
+          if (mbar_test(&sm.p_full[pb], (uint32_t)(tp / NPB) & 1u) &&
+              mbar_test(&sm.full_v[st], (uint32_t)(tp / SV) & 1u)) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < tc::kKeys / 16; ++kk) {
+              const uint64_t a = umma_desc(smem_u32(sm.v[st][0]) + kk * 2048, tc::kKeys * 128, 1024);
+              const uint64_t b = umma_desc(smem_u32(sm.pw[pb][0]) + kk * 2048, tc::kKeys * 128, 1024);
+              umma(tmem + kColO, a, b, idesc_pv, (cv.i > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&sm.empty_v[st]);
+            umma_commit(&sm.p_empty[pb]);
+            ++tp;
+            cv.step(slot);
+            prog = true;
+          }
+        }
+        if (prog) {
+          idle = false;
+        } else {
+          if (*abort_flag) break;
+          const unsigned long long now = globaltimer();
+          if (!idle) {
+            idle = true;
+            idle0 = now;
+          } else if (now - idle0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(p.status, MAC_DEV_TIMEOUT);
+            break;
+          }
+        }
+      }
+      // every MMA issued has completed before the tensor memory is released
+      umma_commit(&sm.drain);
+      const unsigned long long t0 = globaltimer();
+      while (!mbar_try_wait(&sm.drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else if (warp >= tc::kSoftWarp0) {
+    // ---- softmax warps: thread k owns key k of the tile (TMEM lane k)
+    const int k = tid - tc::kSoftWarp0 * 32, wq = warp - tc::kSoftWarp0;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * wq) << 16);
+    if constexpr (2 * G < N) {
+      // padding: columns 2G..N-1 of P^T and rows 2G..N-1 of the query stay zero
+#pragma unroll
+      for (int pb = 0; pb < NPB; ++pb)
+#pragma unroll
+        for (int c = 2 * G / 8; c < 8; ++c)
+          *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.pw[pb][0]) + sw128_off(k, c * 8)) =
+              make_uint4(0u, 0u, 0u, 0u);
+      for (int idx = k; idx < 2 * (N - 2 * G); idx += 128) {
+        const int row = 2 * G + (idx >> 1), half = idx & 1;
+        unsigned char* qd = reinterpret_cast<unsigned char*>(sm.q[half]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(qd + sw128_off(row, c * 8)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    // A failed wait flags the CTA's abort (every later wait then returns at
+    // once) but the softmax warps still go through every tile and barrier of
+    // their walk, so the named barriers always see all 128 threads.
+    bool ok = true;
+    float lsum[G];
+    int t = 0;
+    for (; cur.live; cur.i = cur.ntile - 1, cur.step(slot)) {
+      const Piece& pc = cur.pc;
+      // the piece's query: rows [0, G) high parts, [G, 2G) residuals; the
+      // previous piece's products are done (every S and O of it was read)
+      for (int idx = k; idx < 4 * G; idx += 128) {
+        const int row = idx >> 1, half = idx & 1, h = row < G ? row : row - G;
+        const float* qsrc = p.qrot + ((size_t)pc.unit * G + h) * D + half * 64;
+        unsigned char* qd = reinterpret_cast<unsigned char*>(sm.q[half]);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float4 a = *reinterpret_cast<const float4*>(qsrc + c * 8);
+          const float4 b4 = *reinterpret_cast<const float4*>(qsrc + c * 8 + 4);
+          uint4 vh;
+          vh.x = pack_bf16(a.x, a.y);
+          vh.y = pack_bf16(a.z, a.w);
+          vh.z = pack_bf16(b4.x, b4.y);
+          vh.w = pack_bf16(b4.z, b4.w);
+          if (row >= G) {
+            vh.x = pack_bf16_residual(a.x, a.y, vh.x);
+            vh.y = pack_bf16_residual(a.z, a.w, vh.y);
+            vh.z = pack_bf16_residual(b4.x, b4.y, vh.z);
+            vh.w = pack_bf16_residual(b4.z, b4.w, vh.w);
+          }
+          *reinterpret_cast<uint4*>(qd + sw128_off(row, c * 8)) = vh;
+        }
+      }
+      if (k < G) sm.m[k] = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < G; ++h) lsum[h] = 0.f;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full);
+      softmax_sync();
+      for (int i = 0; i < cur.ntile; ++i, ++t) {
+        const int sb = t & 1, st = t % SV;
+        const int key = pc.kb0 + i * tc::kKeys + k;
+        const bool valid = key >= pc.k0 && key < pc.k1;
+        const uint32_t sbase = lane_base + (uint32_t)(N * sb);
+        unsigned char* const pw0 = reinterpret_cast<unsigned char*>(sm.pw[t % NPB][0]);
+        ok &= mbar_wait(&sm.s_full[sb], (uint32_t)(t >> 1) & 1u, abort_flag, p.status);
+        __syncwarp();
+        tc_fence_after();
+        int grow = 0;
+#pragma unroll
+        for (int h0 = 0; h0 < G; h0 += HC) {
+          float v[HC];
+          tmem_heads<G>(sbase, h0, v);
+#pragma unroll
+          for (int j = 0; j < HC; ++j) grow |= (valid && v[j] > sm.m[h0 + j] + 8.f) ? 1 : 0;
+        }
+        if (softmax_sync_or(grow)) {
+          // some head's maximum grew: new maxima, O and the sums rescaled
+#pragma unroll
+          for (int h0 = 0; h0 < G; h0 += HC) {
+            float v[HC];
+            tmem_heads<G>(sbase, h0, v);
+#pragma unroll
+            for (int j = 0; j < HC; ++j) {
+              float x = valid ? v[j] : -INFINITY;
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+              if (lane == 0) sm.red[wq][h0 + j] = x;
+            }
+          }
+          softmax_sync();
+          if (k < G) {
+            const float mo = sm.m[k];
+            const float mn = fmaxf(mo, fmaxf(fmaxf(sm.red[0][k], sm.red[1][k]), fmaxf(sm.red[2][k], sm.red[3][k])));
+            sm.red[0][k] = mo == -INFINITY ? 0.f : ex2(mo - mn);  // scale of the old sums
+            sm.m[k] = mn;
+          }
+          softmax_sync();
+          if (i > 0) {
+            // O holds the previous tile's product once that is done
+            ok &= mbar_wait(&sm.p_empty[(t - 1) % NPB], (uint32_t)((t - 1) / NPB) & 1u, abort_flag, p.status);
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < 2 * G; c0 += 32) {
+              uint32_t r[32];
+              float ov[32];
+              tmem_ld32_issue(lane_base + kColO + c0, r);
+              tmem_ld_wait<32>(r);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int col = c0 + j, h = col < G ? col : col - G;
+                ov[j] = __uint_as_float(r[j]) * sm.red[0][h];
+              }
+              tmem_st32(lane_base + kColO + c0, ov);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) lsum[h] *= sm.red[0][h];
+          softmax_sync();
+        }
+        // this key's weights into row k of P^T buffer t % NPB (free once the
+        // product of tile t - NPB is done): high parts at column h, residuals
+        // at column G + h
+        if (t >= NPB) ok &= mbar_wait(&sm.p_empty[t % NPB], (uint32_t)((t / NPB) - 1) & 1u, abort_flag, p.status);
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int h0 = 0; h0 < G; h0 += HC) {
+          float v[HC];
+          tmem_heads<G>(sbase, h0, v);
+#pragma unroll
+          for (int c = 0; c < HC / 8; ++c) {
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int h = h0 + c * 8 + j;
+              x[j] = valid ? ex2(v[c * 8 + j] - sm.m[h]) : 0.f;
+              lsum[h] += x[j];
+            }
+            uint4 vh, vr;
+            vh.x = pack_bf16(x[0], x[1]);
+            vh.y = pack_bf16(x[2], x[3]);
+            vh.z = pack_bf16(x[4], x[5]);
+            vh.w = pack_bf16(x[6], x[7]);
+            vr.x = pack_bf16_residual(x[0], x[1], vh.x);
+            vr.y = pack_bf16_residual(x[2], x[3], vh.y);
+            vr.z = pack_bf16_residual(x[4], x[5], vh.z);
+            vr.w = pack_bf16_residual(x[6], x[7], vh.w);
+            const int ch = h0 + c * 8, cr = G + ch;
+            *reinterpret_cast<uint4*>(pw0 + (ch >> 6) * (tc::kKeys * 128) + sw128_off(k, ch & 63)) = vh;
+            *reinterpret_cast<uint4*>(pw0 + (cr >> 6) * (tc::kKeys * 128) + sw128_off(k, cr & 63)) = vr;
+          }
+        }
+        // S is consumed: its buffer takes the product of tile t + 2
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
+        if (!valid) {
+          // rows outside the piece: zero V (they may hold anything, NaN included)
+          ok &= mbar_wait(&sm.full_v[st], (uint32_t)(t / SV) & 1u, abort_flag, p.status);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint4* vrow = reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.v[st][hf]) + k * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[t % NPB]);
+      }
+      // the piece's partial: O (after its last product), running maxima, sums
+      ok &= mbar_wait(&sm.p_empty[(t - 1) % NPB], (uint32_t)((t - 1) / NPB) & 1u, abort_flag, p.status);
+      __syncwarp();
+      tc_fence_after();
+      float* dst = p.part + (size_t)pc.pidx * partial_floats(G, D);
+#pragma unroll
+      for (int h0 = 0; h0 < G; h0 += HC) {
+        float v[HC];
+        tmem_heads<G>(lane_base + kColO, h0, v);
+#pragma unroll
+        for (int j = 0; j < HC; ++j) {
+          const int h = h0 + j;  // element (h, d = k)
+          dst[(h >> 3) * PFc + (h & 7) * D + k] = v[j];
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float v = lsum[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+        if (lane == 0) sm.red[wq][h] = v;
+      }
+      softmax_sync();
+      if (k < G) {
+        float* dc = dst + (k >> 3) * PFc;
+        dc[GDc + (k & 7)] = sm.m[k];
+        dc[GDc + 8 + (k & 7)] = sm.red[0][k] + sm.red[1][k] + sm.red[2][k] + sm.red[3][k];
+      }
+      tc_fence_before();
+      softmax_sync();
+    }
+    (void)ok;
+  }
+  // everyone is done with the tensor memory (the issuer drained its MMAs)
+  // and the streams' copies have landed
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0 && p.trace != nullptr) {
+    const unsigned long long now = globaltimer();
+    p.trace[cta * kTracePoints + kTraceRange] = now;
+    p.trace[cta * kTracePoints + kTraceEnd] = now;
+  }
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kCols) : "memory");
+  }
+}
+
+// Merge of the partials of the tcgen05 path: one CTA per unit (blockIdx.x)
+// and 8-head chunk (blockIdx.y), four partials per warp in flight.
+template <int D, int GF>
+__global__ void __launch_bounds__(kAttnThreads, 1) mac_merge_kernel(const __grid_constant__ AttendParams p) {
+  __shared__ MergeSmem<D> sm;
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.csync, kConsumerWarps);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int u = blockIdx.x, ch = blockIdx.y;
+  if (__ldcg(&p.plan[u].bad)) return;
+  if (p.counters != nullptr && threadIdx.x == 0 && ch == 0) atomicAdd(p.counters + kCountMerged, 1ull);
+  uint32_t phase = 0;
+  merge_unit<D, 8, GF, false, GF / 8, 4>(p, sm, u, phase, ch, ch + 1);
+}
+
 // Failure-path self-test: one warp waits, through the kernels' bounded wait,
 // on an mbarrier that nothing arrives on.  After the limit the wait sets
 // MAC_DEV_TIMEOUT in the status word and the kernel returns.
@@ -1589,8 +2243,34 @@ cudaError_t launch_step(const AttendParams& p, const MatchParams& mp, int D, int
   return mp.ring_bf16 ? step_launch_d<64, true>(cfg, p, mp) : step_launch_d<64, false>(cfg, p, mp);
 }
 
+namespace {
+template <int GF>
+constexpr size_t tc_smem_bytes() { return sizeof(TcSmem<GF>) + 1024; }  // + alignment of the tiles to 1 KB
+static_assert(tc_smem_bytes<16>() <= 232448 && tc_smem_bytes<32>() <= 232448 && tc_smem_bytes<64>() <= 232448,
+              "the tcgen05 kernel's shared memory fits one CTA");
+template <int GF>
+cudaError_t tc_prepare() {
+  return cudaFuncSetAttribute(mac_attend_tc_kernel<GF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)tc_smem_bytes<GF>());
+}
+template <int GF>
+cudaError_t tc_launch(cudaLaunchConfig_t& cfg, const AttendParams& p, int U, cudaStream_t s) {
+  cfg.dynamicSmemBytes = tc_smem_bytes<GF>();
+  cudaError_t e = cudaLaunchKernelEx(&cfg, mac_attend_tc_kernel<GF>, p);
+  if (e != cudaSuccess) return e;
+  // the merge may start while the products drain (it waits on them first)
+  cfg.gridDim = dim3(U, GF / 8);
+  cfg.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&cfg, mac_merge_kernel<128, GF>, p);
+}
+}  // namespace
+
 cudaError_t attend_prepare(int D, int G) {
   if ((D != 64 && D != 128) || !group_ok(G)) return cudaErrorInvalidValue;
+  if (D == 128 && G > kMaxGroup) {  // the tcgen05 path for groups of 16-64 heads
+    cudaError_t e = G == 16 ? tc_prepare<16>() : (G == 32 ? tc_prepare<32>() : tc_prepare<64>());
+    if (e != cudaSuccess) return e;
+  }
   return D == 128 ? set_smem_all<128>() : set_smem_all<64>();
 }
 
@@ -1608,6 +2288,11 @@ cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (D == 128 && p.G > kMaxGroup && !p.per_head) {
+    // groups of 16-64 heads at head_dim 128: tcgen05 products, then the merge
+    const int U = p.nseg / 2;
+    return p.G == 16 ? tc_launch<16>(cfg, p, U, s) : (p.G == 32 ? tc_launch<32>(cfg, p, U, s) : tc_launch<64>(cfg, p, U, s));
+  }
   return D == 128 ? launch_d<128>(cfg, p) : launch_d<64>(cfg, p);
 }
 
