@@ -610,16 +610,11 @@ __device__ __forceinline__ void unit_epilogue(const AttendParams& p, SM& sm, int
 // rest, in proportion to their counts -- and each folds its own into one
 // state (lane: four consecutive elements of every 128, KB partials per round
 // of loads); the finish of a whole unit then combines the eight states.
-// (SM: the attention kernel's shared memory, or the merge kernel's, which
-// has the same warp slots, ring buffer and barrier.  Chunked groups: chunks
-// [ch0, ch1) of the unit; KBO: partials per warp and round of loads, 0 for
-// the attention kernel's register budget.)
-template <int D, int GP, int GF, bool PH, int NC = 1, int KBO = 0, typename SM>
-__device__ __noinline__ bool merge_unit(const AttendParams& p, SM& sm, int u, uint32_t& sync_phase, int ch0 = 0,
-                                        int ch1 = NC) {
+template <int D, int GP, int GF, bool PH, int NC = 1>
+__device__ __noinline__ bool merge_unit(const AttendParams& p, AttnSmem<D, GP>& sm, int u, uint32_t& sync_phase) {
   using C = Cfg<D, GP>;
-  constexpr int NCH = C::GD / 128;                                   // 128-element runs of a padded group: 2, 4 or 8
-  constexpr int KB = KBO > 0 ? KBO : (NCH <= 2 ? 8 : 16 / NCH);     // partials per round of loads
+  constexpr int NCH = C::GD / 128;                // 128-element runs of a padded group: 2, 4 or 8
+  constexpr int KB = NCH <= 2 ? 8 : 16 / NCH;     // partials per round of loads
   // chunked groups (NC > 1): the unit's 8 NC heads are merged 8 at a time;
   // chunk ch of a partial is a run of partial_floats(8, D) floats at ch times that
   const int G = NC > 1 ? GP : group_of<GF>(p), GD = G * D, G4 = group4(G);  // heads of one chunk
@@ -640,7 +635,7 @@ __device__ __noinline__ bool merge_unit(const AttendParams& p, SM& sm, int u, ui
   const bool onA = warp < wA;
   const int cnt = onA ? nA : nB, stride = onA ? wA : kConsumerWarps - wA, first = onA ? warp : warp - wA;
 #pragma unroll 1
-  for (int ch = ch0; ch < ch1; ++ch) {
+  for (int ch = 0; ch < NC; ++ch) {
     const int h0 = ch * G;  // first head of this chunk in the unit
     const float* const part = p.part + (size_t)(onA ? sA.pbase : sB.pbase) * PF + (size_t)ch * (GD + 2 * G4);
     // the reused state on chip, in the layout of a whole unit's copy: each
@@ -1475,7 +1470,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // (merge_unit).
 namespace tc {
 constexpr int kKeys = 128;     // keys per tile: M of QK, K of PV
-constexpr int kSoftWarp0 = 4;  // softmax warps 4..7 (TMEM lanes 32 (w % 4) ..)
+constexpr int kSoftWarp0 = 4;  // softmax warps 4..11: warp w reads TMEM lanes 32 (w % 4) ..
+constexpr int kThreads = 12 * 32;
 // Columns of S and of O: high parts and residuals of the G heads, at least 64.
 __host__ __device__ constexpr int ncols(int G) { return 2 * G < 64 ? 64 : 2 * G; }
 // Tiles in flight per ring and buffers of the weights P^T (shared memory:
@@ -1504,14 +1500,6 @@ struct TcSmem {
   uint32_t tmem;
   int abort_flag;
   int last_flag;
-};
-
-template <int D>
-struct MergeSmem {
-  float wbuf[kConsumerWarps][Cfg<D, 8>::WB];
-  alignas(16) float ring[Cfg<D, 8>::SF];
-  unsigned long long csync;
-  int abort_flag;
 };
 
 // Byte offset of element (row, col) of a [rows][64] bf16 tile with the
@@ -1544,36 +1532,18 @@ __device__ __forceinline__ void umma_commit(unsigned long long* bar) {
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// 32 consecutive fp32 columns into this warp's 32 TMEM lanes (thread i: lane i).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// Named barrier of the four softmax warps, with an OR of one flag.
+// Named barrier of the eight softmax warps, with an OR of one flag.
 __device__ __forceinline__ int softmax_sync_or(int flag) {
   int out;
   asm volatile(
-      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 128, pi;\n\t"
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 256, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(out)
       : "r"(flag)
       : "memory");
   return out;
 }
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // A CTA role's walk over its pieces, tile by tile.
 struct TileCursor {
@@ -1594,43 +1564,75 @@ struct TileCursor {
   }
 };
 
-// 32 consecutive fp32 columns of this warp's 32 TMEM lanes, issued without
-// waiting; tmem_ld_wait() completes every load issued so far and ties the
-// registers to that point.
-__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
+// n consecutive fp32 columns (n = 8, 16, 32) of this warp's 32 TMEM lanes,
+// issued without waiting (tmem_ld_wait completes them), and stored back.
+template <int NCOL>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t* r);
+template <int NCOL>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t* r);
+template <>
+__device__ __forceinline__ void tmem_ldn<8>(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
 }
+template <>
+__device__ __forceinline__ void tmem_stn<8>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ldn<16>(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_stn<16>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ldn<32>(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_stn<32>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+// Completes every TMEM load issued so far and ties the registers to that
+// point.
 template <int NR>
 __device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int j = 0; j < NR; ++j) asm volatile("" : "+r"(r[j]));
 }
-// Heads [h0, h0 + HC) of this thread's TMEM lane at accumulator column base
-// `base`: the high-part column plus the residual column (HC = 16 for groups of
-// 16, whose 32 columns come in one load; else 32).
-template <int G>
-__device__ __forceinline__ void tmem_heads(uint32_t base, int h0, float* v) {
-  if constexpr (G == 16) {
-    uint32_t a[32];
-    tmem_ld32_issue(base, a);
-    tmem_ld_wait<32>(a);
+// Values of GH heads of this thread's TMEM lane: the high-part columns at
+// `hi` plus the residual columns at `res` (32 heads: one half after the
+// other, to bound the registers in flight).
+template <int GH>
+__device__ __forceinline__ void tmem_heads(uint32_t hi, uint32_t res, float* v) {
+  if constexpr (GH <= 16) {
+    uint32_t r[2 * GH];
+    tmem_ldn<GH>(hi, r);
+    tmem_ldn<GH>(res, r + GH);
+    tmem_ld_wait<2 * GH>(r);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(a[j]) + __uint_as_float(a[16 + j]);
+    for (int j = 0; j < GH; ++j) v[j] = __uint_as_float(r[j]) + __uint_as_float(r[GH + j]);
   } else {
-    uint32_t a[64];
-    tmem_ld32_issue(base + h0, a);
-    tmem_ld32_issue(base + G + h0, a + 32);
-    tmem_ld_wait<64>(a);
+    uint32_t r[GH];
+    tmem_ldn<GH>(hi, r);
+    tmem_ld_wait<GH>(r);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(a[j]) + __uint_as_float(a[32 + j]);
+    for (int j = 0; j < GH; ++j) v[j] = __uint_as_float(r[j]);
+    tmem_ldn<GH>(res, r);
+    tmem_ld_wait<GH>(r);
+#pragma unroll
+    for (int j = 0; j < GH; ++j) v[j] += __uint_as_float(r[j]);
   }
 }
 
@@ -1684,10 +1686,9 @@ __device__ __forceinline__ void tc_stream(const AttendParams& p, const CUtensorM
 }
 
 template <int GF>
-__global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __grid_constant__ AttendParams p) {
+__global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __grid_constant__ AttendParams p) {
   constexpr int D = 128, G = GF, N = tc::ncols(G), SK = TcSmem<G>::SK, SV = TcSmem<G>::SV, NPB = TcSmem<G>::NPB;
   static_assert(G == 16 || G == 32 || G == 64, "groups of 16, 32 or 64 heads");
-  constexpr int HC = G == 16 ? 16 : 32;  // heads per pass over the accumulator columns
   constexpr int GDc = 8 * D, PFc = GDc + 16;  // one 8-head chunk of a partial: o [8][D], m [8], l [8]
   constexpr uint32_t kCols = tc::tmem_cols(G), kColO = 2 * N;  // S[0] at 0, S[1] at N, O at 2N
   constexpr uint32_t idesc_qk = umma_idesc(0, 0, N, tc::kKeys);
@@ -1710,13 +1711,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
     }
     for (int s_ = 0; s_ < 2; ++s_) {
       mbar_init(&sm.s_full[s_], 1);
-      mbar_init(&sm.s_empty[s_], 4);
+      mbar_init(&sm.s_empty[s_], 8);
     }
     for (int s_ = 0; s_ < NPB; ++s_) {
-      mbar_init(&sm.p_full[s_], 4);
+      mbar_init(&sm.p_full[s_], 8);
       mbar_init(&sm.p_empty[s_], 1);
     }
-    mbar_init(&sm.q_full, 4);
+    mbar_init(&sm.q_full, 8);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1848,18 +1849,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
       }
     }
   } else if (warp >= tc::kSoftWarp0) {
-    // ---- softmax warps: thread k owns key k of the tile (TMEM lane k)
-    const int k = tid - tc::kSoftWarp0 * 32, wq = warp - tc::kSoftWarp0;
+    // ---- softmax warps: warp 4 + 4 hh + wq owns TMEM lanes 32 wq .. 32 wq + 31
+    // (the tile's keys) and heads [hh GH, hh GH + GH)
+    constexpr int GH = G / 2;
+    const int sw = warp - tc::kSoftWarp0, wq = sw & 3, hh = sw >> 2;
+    const int ts = tid - tc::kSoftWarp0 * 32;  // 0 .. 255
+    const int k = 32 * wq + lane, hb = hh * GH;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * wq) << 16);
     if constexpr (2 * G < N) {
       // padding: columns 2G..N-1 of P^T and rows 2G..N-1 of the query stay zero
+      if (hh == 0) {
 #pragma unroll
-      for (int pb = 0; pb < NPB; ++pb)
+        for (int pb = 0; pb < NPB; ++pb)
 #pragma unroll
-        for (int c = 2 * G / 8; c < 8; ++c)
-          *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.pw[pb][0]) + sw128_off(k, c * 8)) =
-              make_uint4(0u, 0u, 0u, 0u);
-      for (int idx = k; idx < 2 * (N - 2 * G); idx += 128) {
+          for (int c = 2 * G / 8; c < 8; ++c)
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.pw[pb][0]) + sw128_off(k, c * 8)) =
+                make_uint4(0u, 0u, 0u, 0u);
+      }
+      for (int idx = ts; idx < 2 * (N - 2 * G); idx += 2 * 128) {
         const int row = 2 * G + (idx >> 1), half = idx & 1;
         unsigned char* qd = reinterpret_cast<unsigned char*>(sm.q[half]);
 #pragma unroll
@@ -1868,15 +1875,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
     }
     // A failed wait flags the CTA's abort (every later wait then returns at
     // once) but the softmax warps still go through every tile and barrier of
-    // their walk, so the named barriers always see all 128 threads.
+    // their walk, so the named barriers always see all 256 threads.
     bool ok = true;
-    float lsum[G];
+    // per head of this warp: key sums, this key's scores and (up to 16 heads)
+    // the running maxima; 32 heads read the maxima from shared memory
+    constexpr bool kMaxInRegs = GH <= 16;
+    float lsum[GH], sv[GH], mr[kMaxInRegs ? GH : 1];
+#pragma unroll
+    for (int j = 0; j < (kMaxInRegs ? GH : 1); ++j) mr[j] = -INFINITY;
+    auto mget = [&](int j) __attribute__((always_inline)) {
+      if constexpr (kMaxInRegs) return mr[j];
+      else return sm.m[hb + j];
+    };
     int t = 0;
     for (; cur.live; cur.i = cur.ntile - 1, cur.step(slot)) {
       const Piece& pc = cur.pc;
       // the piece's query: rows [0, G) high parts, [G, 2G) residuals; the
       // previous piece's products are done (every S and O of it was read)
-      for (int idx = k; idx < 4 * G; idx += 128) {
+      for (int idx = ts; idx < 4 * G; idx += 2 * 128) {
         const int row = idx >> 1, half = idx & 1, h = row < G ? row : row - G;
         const float* qsrc = p.qrot + ((size_t)pc.unit * G + h) * D + half * 64;
         unsigned char* qd = reinterpret_cast<unsigned char*>(sm.q[half]);
@@ -1898,50 +1914,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
           *reinterpret_cast<uint4*>(qd + sw128_off(row, c * 8)) = vh;
         }
       }
-      if (k < G) sm.m[k] = -INFINITY;
+      if (ts < G) sm.m[ts] = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < G; ++h) lsum[h] = 0.f;
+      for (int j = 0; j < GH; ++j) lsum[j] = 0.f;
+#pragma unroll
+      for (int j = 0; j < (kMaxInRegs ? GH : 1); ++j) mr[j] = -INFINITY;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.q_full);
-      softmax_sync();
       for (int i = 0; i < cur.ntile; ++i, ++t) {
         const int sb = t & 1, st = t % SV;
         const int key = pc.kb0 + i * tc::kKeys + k;
         const bool valid = key >= pc.k0 && key < pc.k1;
-        const uint32_t sbase = lane_base + (uint32_t)(N * sb);
-        unsigned char* const pw0 = reinterpret_cast<unsigned char*>(sm.pw[t % NPB][0]);
         ok &= mbar_wait(&sm.s_full[sb], (uint32_t)(t >> 1) & 1u, abort_flag, p.status);
         __syncwarp();
         tc_fence_after();
+        // this key's scores for the warp's heads: high-part plus residual column
+        tmem_heads<GH>(lane_base + (uint32_t)(N * sb + hb), lane_base + (uint32_t)(N * sb + G + hb), sv);
+#pragma unroll
+        for (int j = 0; j < GH; ++j) sv[j] = valid ? sv[j] : -INFINITY;
+        // S is in registers: its buffer takes the product of tile t + 2
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
         int grow = 0;
 #pragma unroll
-        for (int h0 = 0; h0 < G; h0 += HC) {
-          float v[HC];
-          tmem_heads<G>(sbase, h0, v);
-#pragma unroll
-          for (int j = 0; j < HC; ++j) grow |= (valid && v[j] > sm.m[h0 + j] + 8.f) ? 1 : 0;
-        }
+        for (int j = 0; j < GH; ++j) grow |= sv[j] > mget(j) + 8.f ? 1 : 0;
         if (softmax_sync_or(grow)) {
           // some head's maximum grew: new maxima, O and the sums rescaled
 #pragma unroll
-          for (int h0 = 0; h0 < G; h0 += HC) {
-            float v[HC];
-            tmem_heads<G>(sbase, h0, v);
+          for (int j = 0; j < GH; ++j) {
+            float x = sv[j];
 #pragma unroll
-            for (int j = 0; j < HC; ++j) {
-              float x = valid ? v[j] : -INFINITY;
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
-              if (lane == 0) sm.red[wq][h0 + j] = x;
-            }
+            for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+            if (lane == 0) sm.red[wq][hb + j] = x;
           }
           softmax_sync();
-          if (k < G) {
-            const float mo = sm.m[k];
-            const float mn = fmaxf(mo, fmaxf(fmaxf(sm.red[0][k], sm.red[1][k]), fmaxf(sm.red[2][k], sm.red[3][k])));
-            sm.red[0][k] = mo == -INFINITY ? 0.f : ex2(mo - mn);  // scale of the old sums
-            sm.m[k] = mn;
+          if (ts < G) {
+            const float mo = sm.m[ts];
+            const float mn = fmaxf(mo, fmaxf(fmaxf(sm.red[0][ts], sm.red[1][ts]), fmaxf(sm.red[2][ts], sm.red[3][ts])));
+            sm.red[0][ts] = mo == -INFINITY ? 0.f : ex2(mo - mn);  // scale of the old sums
+            sm.m[ts] = mn;
           }
           softmax_sync();
           if (i > 0) {
@@ -1950,21 +1963,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
             __syncwarp();
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < 2 * G; c0 += 32) {
-              uint32_t r[32];
-              float ov[32];
-              tmem_ld32_issue(lane_base + kColO + c0, r);
-              tmem_ld_wait<32>(r);
+            for (int part = 0; part < 2; ++part) {  // high-part columns, then residual columns
+              const uint32_t ta = lane_base + kColO + (uint32_t)(part * G + hb);
+              uint32_t r[GH];
+              tmem_ldn<GH>(ta, r);
+              tmem_ld_wait<GH>(r);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int col = c0 + j, h = col < G ? col : col - G;
-                ov[j] = __uint_as_float(r[j]) * sm.red[0][h];
-              }
-              tmem_st32(lane_base + kColO + c0, ov);
+              for (int j = 0; j < GH; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * sm.red[0][hb + j]);
+              tmem_stn<GH>(ta, r);
+              asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             }
           }
 #pragma unroll
-          for (int h = 0; h < G; ++h) lsum[h] *= sm.red[0][h];
+          for (int j = 0; j < GH; ++j) lsum[j] *= sm.red[0][hb + j];
+#pragma unroll
+          for (int j = 0; j < (kMaxInRegs ? GH : 1); ++j) mr[j] = sm.m[hb + j];
           softmax_sync();
         }
         // this key's weights into row k of P^T buffer t % NPB (free once the
@@ -1973,38 +1986,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
         if (t >= NPB) ok &= mbar_wait(&sm.p_empty[t % NPB], (uint32_t)((t / NPB) - 1) & 1u, abort_flag, p.status);
         __syncwarp();
         tc_fence_after();
+        unsigned char* const pw0 = reinterpret_cast<unsigned char*>(sm.pw[t % NPB][0]);
 #pragma unroll
-        for (int h0 = 0; h0 < G; h0 += HC) {
-          float v[HC];
-          tmem_heads<G>(sbase, h0, v);
+        for (int c = 0; c < GH / 8; ++c) {
+          float x[8];
 #pragma unroll
-          for (int c = 0; c < HC / 8; ++c) {
-            float x[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int h = h0 + c * 8 + j;
-              x[j] = valid ? ex2(v[c * 8 + j] - sm.m[h]) : 0.f;
-              lsum[h] += x[j];
-            }
-            uint4 vh, vr;
-            vh.x = pack_bf16(x[0], x[1]);
-            vh.y = pack_bf16(x[2], x[3]);
-            vh.z = pack_bf16(x[4], x[5]);
-            vh.w = pack_bf16(x[6], x[7]);
-            vr.x = pack_bf16_residual(x[0], x[1], vh.x);
-            vr.y = pack_bf16_residual(x[2], x[3], vh.y);
-            vr.z = pack_bf16_residual(x[4], x[5], vh.z);
-            vr.w = pack_bf16_residual(x[6], x[7], vh.w);
-            const int ch = h0 + c * 8, cr = G + ch;
-            *reinterpret_cast<uint4*>(pw0 + (ch >> 6) * (tc::kKeys * 128) + sw128_off(k, ch & 63)) = vh;
-            *reinterpret_cast<uint4*>(pw0 + (cr >> 6) * (tc::kKeys * 128) + sw128_off(k, cr & 63)) = vr;
+          for (int j = 0; j < 8; ++j) {
+            x[j] = valid ? ex2(sv[c * 8 + j] - mget(c * 8 + j)) : 0.f;
+            lsum[c * 8 + j] += x[j];
           }
+          uint4 vh, vr;
+          vh.x = pack_bf16(x[0], x[1]);
+          vh.y = pack_bf16(x[2], x[3]);
+          vh.z = pack_bf16(x[4], x[5]);
+          vh.w = pack_bf16(x[6], x[7]);
+          vr.x = pack_bf16_residual(x[0], x[1], vh.x);
+          vr.y = pack_bf16_residual(x[2], x[3], vh.y);
+          vr.z = pack_bf16_residual(x[4], x[5], vh.z);
+          vr.w = pack_bf16_residual(x[6], x[7], vh.w);
+          const int ch = hb + c * 8, cr = G + ch;
+          *reinterpret_cast<uint4*>(pw0 + (ch >> 6) * (tc::kKeys * 128) + sw128_off(k, ch & 63)) = vh;
+          *reinterpret_cast<uint4*>(pw0 + (cr >> 6) * (tc::kKeys * 128) + sw128_off(k, cr & 63)) = vr;
         }
-        // S is consumed: its buffer takes the product of tile t + 2
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_empty[sb]);
-        if (!valid) {
+        if (!valid && hh == 0) {
           // rows outside the piece: zero V (they may hold anything, NaN included)
           ok &= mbar_wait(&sm.full_v[st], (uint32_t)(t / SV) & 1u, abort_flag, p.status);
 #pragma unroll
@@ -2024,28 +2028,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
       __syncwarp();
       tc_fence_after();
       float* dst = p.part + (size_t)pc.pidx * partial_floats(G, D);
+      tmem_heads<GH>(lane_base + kColO + hb, lane_base + kColO + G + hb, sv);
 #pragma unroll
-      for (int h0 = 0; h0 < G; h0 += HC) {
-        float v[HC];
-        tmem_heads<G>(lane_base + kColO, h0, v);
-#pragma unroll
-        for (int j = 0; j < HC; ++j) {
-          const int h = h0 + j;  // element (h, d = k)
-          dst[(h >> 3) * PFc + (h & 7) * D + k] = v[j];
-        }
+      for (int j = 0; j < GH; ++j) {
+        const int h = hb + j;  // element (h, d = k)
+        dst[(h >> 3) * PFc + (h & 7) * D + k] = sv[j];
       }
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float v = lsum[h];
+      for (int j = 0; j < GH; ++j) {
+        float v = lsum[j];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-        if (lane == 0) sm.red[wq][h] = v;
+        if (lane == 0) sm.red[wq][hb + j] = v;
       }
       softmax_sync();
-      if (k < G) {
-        float* dc = dst + (k >> 3) * PFc;
-        dc[GDc + (k & 7)] = sm.m[k];
-        dc[GDc + 8 + (k & 7)] = sm.red[0][k] + sm.red[1][k] + sm.red[2][k] + sm.red[3][k];
+      if (ts < G) {
+        float* dc = dst + (ts >> 3) * PFc;
+        dc[GDc + (ts & 7)] = sm.m[ts];
+        dc[GDc + 8 + (ts & 7)] = sm.red[0][ts] + sm.red[1][ts] + sm.red[2][ts] + sm.red[3][ts];
       }
       tc_fence_before();
       softmax_sync();
@@ -2068,23 +2068,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1) mac_attend_tc_kernel(const __
   }
 }
 
-// Merge of the partials of the tcgen05 path: one CTA per unit (blockIdx.x)
-// and 8-head chunk (blockIdx.y), four partials per warp in flight.
-template <int D, int GF>
-__global__ void __launch_bounds__(kAttnThreads, 1) mac_merge_kernel(const __grid_constant__ AttendParams p) {
-  __shared__ MergeSmem<D> sm;
-  if (threadIdx.x == 0) {
-    mbar_init(&sm.csync, kConsumerWarps);
-    sm.abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
+// Merge of the tcgen05 path's partials, one CTA per unit (blockIdx.x) and
+// 8-head chunk (blockIdx.y): warp w takes head w of the chunk and lane l its
+// elements 4l .. 4l + 3, and each warp folds every partial of its head with
+// KB of them in flight per lane.  Segment A's partials with the reused state
+// (on a hit) give the new prefix state over [0, c_t), stored in ring slot
+// dst; that state and segment B's partials give the output.
+template <int GF>
+__global__ void __launch_bounds__(kAttnThreads) mac_tc_merge_kernel(const __grid_constant__ AttendParams p) {
+  constexpr int D = 128, G = GF, PFc = 8 * D + 16, KB = 16;
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int u = blockIdx.x, ch = blockIdx.y;
-  if (__ldcg(&p.plan[u].bad)) return;
-  if (p.counters != nullptr && threadIdx.x == 0 && ch == 0) atomicAdd(p.counters + kCountMerged, 1ull);
-  uint32_t phase = 0;
-  merge_unit<D, 8, GF, false, GF / 8, 4>(p, sm, u, phase, ch, ch + 1);
+  const int u = blockIdx.x, ch = blockIdx.y, hl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const UnitPlan* const pp = p.plan + u;
+  if (__ldcg(&pp->bad)) return;
+  const int hit = __ldcg(&pp->hit), src = __ldcg(&pp->src_slot), dst = __ldcg(&pp->dst_slot), end = __ldcg(&pp->end);
+  const Segment sA = load_segment(p.seg + 2 * u), sB = load_segment(p.seg + 2 * u + 1);
+  const size_t PF = partial_floats(G, D);
+  const int h = ch * 8 + hl, d0 = lane * 4;
+  auto fold = [&](const Segment& sg, float& M, float& L, float (&O)[4]) __attribute__((always_inline)) {
+    const int n = sg.kind < 0 ? 0 : sg.npieces;
+    const float* base = p.part + (size_t)sg.pbase * PF + (size_t)ch * PFc;
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += KB) {
+      float4 ov[KB];
+      float mv[KB], lv[KB];
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+        if (i0 + k < n) {
+          const float* q = base + (size_t)(i0 + k) * PF;
+          ov[k] = __ldcg(reinterpret_cast<const float4*>(q + hl * D + d0));
+          mv[k] = __ldcg(q + 8 * D + hl);
+          lv[k] = __ldcg(q + 8 * D + 8 + hl);
+        }
+#pragma unroll
+      for (int k = 0; k < KB; ++k)
+        if (i0 + k < n) fold_state<4>(M, L, O, mv[k], lv[k], &ov[k].x);
+    }
+  };
+  // new prefix state: segment A, plus the reused state on a hit
+  float M = -INFINITY, L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
+  fold(sA, M, L, O);
+  const size_t Wp1 = (size_t)p.W + 1;
+  if (hit) {
+    const size_t e = ((size_t)u * Wp1 + src) * G + h;
+    const float rm = __ldcg(p.ring_m + e) * kLog2e, rl = __ldcg(p.ring_l + e);
+    const float Mn = fmaxf(M, rm), Mu = Mn == -INFINITY ? 0.f : Mn;
+    const float a = ex2(M - Mu), c = ex2(rm - Mu);
+    L = L * a + rl * c;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) O[j] = O[j] * a + ring_o_at(p.ring_o, e * D + d0 + j, p.ring_bf16) * rl * c;
+    M = Mn;
+  }
+  const size_t ds = (size_t)u * Wp1 + dst;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    ring_o_put(p.ring_o, (ds * G + h) * D + d0 + j, L > 0.f ? __fdividef(O[j], L) : 0.f, p.ring_bf16);
+  if (lane == 0) {
+    p.ring_m[ds * G + h] = L > 0.f ? M * kLn2 : -INFINITY;
+    p.ring_l[ds * G + h] = L;
+  }
+  // output: the prefix state and segment B (the tail)
+  float MB = -INFINITY, LB = 0.f, OB[4] = {0.f, 0.f, 0.f, 0.f};
+  fold(sB, MB, LB, OB);
+  const float M2 = fmaxf(M, MB), M2u = M2 == -INFINITY ? 0.f : M2;
+  const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
+  const float L2 = L * a0 + LB * aB;  // >= 1: every unit attends at least one key
+  const int b = u / p.Hkv, kvh = u - b * p.Hkv;
+  const size_t orow = (size_t)b * p.Hq + (size_t)kvh * G + h;
+  float4 o4;
+  o4.x = __fdividef(O[0] * a0 + OB[0] * aB, L2);
+  o4.y = __fdividef(O[1] * a0 + OB[1] * aB, L2);
+  o4.z = __fdividef(O[2] * a0 + OB[2] * aB, L2);
+  o4.w = __fdividef(O[3] * a0 + OB[3] * aB, L2);
+  *reinterpret_cast<float4*>(p.out + orow * D + d0) = o4;
+  if (lane == 0) p.lse[orow] = (M2 + __log2f(L2)) * kLn2;
+  if (ch == 0 && threadIdx.x == 0) {
+    p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
+    if (p.counters != nullptr) atomicAdd(p.counters + kCountMerged, 1ull);
+  }
 }
 
 // Failure-path self-test: one warp waits, through the kernels' bounded wait,
@@ -2256,12 +2317,14 @@ cudaError_t tc_prepare() {
 template <int GF>
 cudaError_t tc_launch(cudaLaunchConfig_t& cfg, const AttendParams& p, int U, cudaStream_t s) {
   cfg.dynamicSmemBytes = tc_smem_bytes<GF>();
+  cfg.blockDim = dim3(tc::kThreads);
   cudaError_t e = cudaLaunchKernelEx(&cfg, mac_attend_tc_kernel<GF>, p);
+  cfg.blockDim = dim3(kAttnThreads);
   if (e != cudaSuccess) return e;
   // the merge may start while the products drain (it waits on them first)
   cfg.gridDim = dim3(U, GF / 8);
   cfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&cfg, mac_merge_kernel<128, GF>, p);
+  return cudaLaunchKernelEx(&cfg, mac_tc_merge_kernel<GF>, p);
 }
 }  // namespace
 
