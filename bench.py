@@ -48,10 +48,10 @@ def _peaks():
 
 def _kernel_hash() -> str:
     """Hash of the step kernel's source code (the attention file, the match
-    stage it includes and the shared layout; comments and blank space removed,
-    so that a comment edit does not orphan a profile)."""
+    stage and device helpers it includes and the shared layout; comments and
+    blank space removed, so that a comment edit does not orphan a profile)."""
     h = hashlib.sha256()
-    for f in ("mac_attend.cu", "mac_internal.cuh", "mac_match_dev.cuh"):
+    for f in ("mac_attend.cu", "mac_attend_dev.cuh", "mac_internal.cuh", "mac_match_dev.cuh"):
         with open(os.path.join(ROOT, "kv_cache_reuse_b200", "csrc", f)) as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)

@@ -14,8 +14,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmac_b200.so")
-SOURCES = ["mac_api.cu", "mac_match.cu", "mac_attend.cu", "mac_noalloc.cu"]
+SOURCES = ["mac_api.cu", "mac_match.cu", "mac_attend.cu", "mac_attend_tc.cu", "mac_noalloc.cu"]
 HEADERS = [os.path.join(CSRC, "mac_internal.cuh"), os.path.join(CSRC, "mac_match_dev.cuh"),
+           os.path.join(CSRC, "mac_attend_dev.cuh"),
            os.path.join(ROOT, "include", "mac.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2"]

@@ -204,6 +204,10 @@ cudaError_t launch_match(const MatchParams& p, int D, cudaStream_t s);
 cudaError_t launch_attend(const AttendParams& p, int D, int grid, cudaStream_t s);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 cudaError_t attend_prepare(int D, int G);
+// The tcgen05 path (mac_attend_tc.cu): groups of 16, 32 or 64 heads at head
+// dim 128, one decision per KV head; products then merge, two launches.
+cudaError_t attend_tc_prepare(int G);
+cudaError_t launch_attend_tc(const AttendParams& p, int grid, cudaStream_t s);
 // The one-launch step (groups of up to 8 heads, one decision per KV head):
 // prepare sets its kernels' attributes and reports how many CTAs fit on an SM.
 cudaError_t step_prepare(int D, int G, int* blocks_per_sm);
