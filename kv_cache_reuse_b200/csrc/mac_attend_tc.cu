@@ -643,13 +643,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
 
 // Merge of the tcgen05 path's partials, one CTA per unit (blockIdx.x) and
 // 8-head chunk (blockIdx.y): warp w takes head w of the chunk and lane l its
-// elements 4l .. 4l + 3, and each warp folds every partial of its head with
-// KB of them in flight per lane.  Segment A's partials with the reused state
-// (on a hit) give the new prefix state over [0, c_t), stored in ring slot
-// dst; that state and segment B's partials give the output.
+// elements 4l .. 4l + 3, and each warp folds every partial of its head --
+// segment A's and B's in one sequence, KB of them in flight per lane.
+// Segment A's partials with the reused state (on a hit) give the new prefix
+// state over [0, c_t), stored in ring slot dst; that state and segment B's
+// partials give the output.
 template <int GF>
 __global__ void __launch_bounds__(kAttnThreads) mac_tc_merge_kernel(const __grid_constant__ AttendParams p) {
-  constexpr int D = 128, G = GF, PFc = 8 * D + 16, KB = 16;
+  constexpr int D = 128, G = GF, PFc = 8 * D + 16, KB = 20;
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int u = blockIdx.x, ch = blockIdx.y, hl = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const UnitPlan* const pp = p.plan + u;
@@ -658,29 +659,36 @@ __global__ void __launch_bounds__(kAttnThreads) mac_tc_merge_kernel(const __grid
   const Segment sA = load_segment(p.seg + 2 * u), sB = load_segment(p.seg + 2 * u + 1);
   const size_t PF = partial_floats(G, D);
   const int h = ch * 8 + hl, d0 = lane * 4;
-  auto fold = [&](const Segment& sg, float& M, float& L, float (&O)[4]) __attribute__((always_inline)) {
-    const int n = sg.kind < 0 ? 0 : sg.npieces;
-    const float* base = p.part + (size_t)sg.pbase * PF + (size_t)ch * PFc;
-#pragma unroll 1
-    for (int i0 = 0; i0 < n; i0 += KB) {
-      float4 ov[KB];
-      float mv[KB], lv[KB];
-#pragma unroll
-      for (int k = 0; k < KB; ++k)
-        if (i0 + k < n) {
-          const float* q = base + (size_t)(i0 + k) * PF;
-          ov[k] = __ldcg(reinterpret_cast<const float4*>(q + hl * D + d0));
-          mv[k] = __ldcg(q + 8 * D + hl);
-          lv[k] = __ldcg(q + 8 * D + 8 + hl);
-        }
-#pragma unroll
-      for (int k = 0; k < KB; ++k)
-        if (i0 + k < n) fold_state<4>(M, L, O, mv[k], lv[k], &ov[k].x);
-    }
-  };
-  // new prefix state: segment A, plus the reused state on a hit
+  const int nA = sA.kind < 0 ? 0 : sA.npieces, nB = sB.kind < 0 ? 0 : sB.npieces;
+  const float* const baseA = p.part + (size_t)sA.pbase * PF + (size_t)ch * PFc + hl * D + d0;
+  const float* const baseB = p.part + (size_t)sB.pbase * PF + (size_t)ch * PFc + hl * D + d0;
+  // segment A folds into (M, L, O), segment B into (MB, LB, OB)
   float M = -INFINITY, L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
-  fold(sA, M, L, O);
+  float MB = -INFINITY, LB = 0.f, OB[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+  for (int i0 = 0; i0 < nA + nB; i0 += KB) {
+    float4 ov[KB];
+    float mv[KB], lv[KB];
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int i = i0 + k;
+      if (i < nA + nB) {
+        const float* q = i < nA ? baseA + (size_t)i * PF : baseB + (size_t)(i - nA) * PF;
+        ov[k] = __ldcg(reinterpret_cast<const float4*>(q));
+        mv[k] = __ldcg(q - hl * D - d0 + 8 * D + hl);
+        lv[k] = __ldcg(q - hl * D - d0 + 8 * D + 8 + hl);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int i = i0 + k;
+      if (i < nA)
+        fold_state<4>(M, L, O, mv[k], lv[k], &ov[k].x);
+      else if (i < nA + nB)
+        fold_state<4>(MB, LB, OB, mv[k], lv[k], &ov[k].x);
+    }
+  }
+  // new prefix state: segment A, plus the reused state on a hit
   const size_t Wp1 = (size_t)p.W + 1;
   if (hit) {
     const size_t e = ((size_t)u * Wp1 + src) * G + h;
@@ -701,8 +709,6 @@ __global__ void __launch_bounds__(kAttnThreads) mac_tc_merge_kernel(const __grid
     p.ring_l[ds * G + h] = L;
   }
   // output: the prefix state and segment B (the tail)
-  float MB = -INFINITY, LB = 0.f, OB[4] = {0.f, 0.f, 0.f, 0.f};
-  fold(sB, MB, LB, OB);
   const float M2 = fmaxf(M, MB), M2u = M2 == -INFINITY ? 0.f : M2;
   const float a0 = ex2(M - M2u), aB = ex2(MB - M2u);
   const float L2 = L * a0 + LB * aB;  // >= 1: every unit attends at least one key
