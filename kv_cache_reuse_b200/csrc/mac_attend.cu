@@ -1070,8 +1070,8 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       p.smid_of[cta] = (int)smid;
       if (cta != builder) {
         // the block barrier above orders every thread's writes before this
-        // thread's device-scope fence; the arrival then publishes them
-        __threadfence();
+        // thread's arrival, and a release is cumulative: the arrival publishes
+        // them device-wide
         asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(p.fsync) : "memory");
       } else {
         const unsigned long long t0 = globaltimer();
@@ -1096,7 +1096,7 @@ __device__ __forceinline__ void attend_body(const AttendParams& p, const MatchPa
       __syncthreads();
       if (tid == 0) {
         p.fsync[0] = 0;
-        __threadfence();  // every thread's table writes, ordered by the barrier, before the epoch
+        // every thread's table writes, ordered by the barrier, are published by the release
         st_release_u32(p.fsync + 1, epoch + 1u);
         if (p.trace) p.trace[cta * kTracePoints + kTraceBuilt] = globaltimer();
       }
