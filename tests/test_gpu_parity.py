@@ -502,6 +502,28 @@ def test_mqa_export_matches_oracle_window():
     np.testing.assert_allclose(st["m"][0, slots] + np.log(st["l"][0, slots]), m + np.log(l), atol=LSE_TOL)
 
 
+def test_mqa_steps_repeat_bit_for_bit():
+    """The tensor-memory path of a 32-head group on large all-miss steps (a
+    single KV head's keys cut over every CTA) and on the repeats after them:
+    two states fed the same stream give the same bits (each partial comes from
+    one range of the split whichever CTA runs it, and the merge folds them in a
+    fixed order), and both match the oracle."""
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=2, Hq=32, Hkv=1, L0=(32768, 20000), steps=5)
+    stream, cache = synth.queries(wl), synth.kv_cache(wl)
+    a, b = DeviceRun(wl, cache), DeviceRun(wl, cache)
+    orc = oracle.Oracle.for_workload(wl, cache)
+    for t in range(wl.steps):
+        x = a.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        y = b.step(stream.q[t], stream.rope_pos[t], stream.seq_lens[t])
+        for u, v in zip(x, y):
+            np.testing.assert_array_equal(u, v, err_msg="step %d" % t)
+        r = orc.step(stream.q[t], stream.rope_pos[t], cache.K, cache.V, cache.block_table, stream.seq_lens[t])
+        np.testing.assert_array_equal(x[2], r.hit)
+        np.testing.assert_array_equal(x[3], r.match_pos)
+        assert float(np.abs(x[0] - r.out).max()) <= OUT_TOL and float(np.abs(x[1] - r.lse).max()) <= LSE_TOL
+    assert a.st.get_status() == 0 and b.st.get_status() == 0
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (24, 8), (64, 8)])
 def test_group_sizes_all_miss_large(Hq, Hkv):
     """Large all-miss steps (weighted split, many partials per unit) for
@@ -755,6 +777,53 @@ def test_warm_start_from_prefill_then_decode(case):
                 np.testing.assert_allclose(st["o"][u, slot], o_o[j], atol=OUT_TOL)
     r = compare_stream(wl, stream, cache, gpu=gpu, orc=orc, start=n, q_bf16=qb)
     assert r["hits"] > 0
+
+
+def test_graph_captured_mqa_loop():
+    """Two layers of 32 query heads over one KV head (head_dim 128: the
+    tensor-memory products and their merge, two launches with programmatic
+    dependent launch) recorded as one CUDA graph and replayed for every token:
+    each layer against its own fp64 oracle and bit-equal to eager steps."""
+    import kv_cache_reuse_b200 as mac
+    torch, dev = torch_dev()
+    llama = synth.WORKLOADS["llama8b_32k"]
+    wls = [llama.with_(B=2, Hq=32, Hkv=1, L0=(3000, 1200), steps=12, seed=20 + l) for l in range(2)]
+    streams = [synth.queries(w) for w in wls]
+    caches = [synth.kv_cache(w) for w in wls]
+    oracles = [oracle.Oracle.for_workload(w, c) for w, c in zip(wls, caches)]
+    eager = [DeviceRun(w, c) for w, c in zip(wls, caches)]
+    graph = [DeviceRun(w, c) for w, c in zip(wls, caches)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for r in graph:
+            mac.mac_decode_step(r.st, r.q, r.pos, r.K, r.V, None, r.lens, r.out, r.lse, r.hit, r.mpos)
+    hits = 0
+    for t in range(wls[0].steps):
+        for l, r in enumerate(graph):
+            st = streams[l]
+            r.q.copy_(torch.from_numpy(np.ascontiguousarray(st.q[t])))
+            r.pos.copy_(torch.from_numpy(st.rope_pos[t]))
+            r.lens.copy_(torch.from_numpy(st.seq_lens[t]))
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        for l in range(len(graph)):
+            st, c = streams[l], caches[l]
+            y = (graph[l].out.cpu().numpy(), graph[l].lse.cpu().numpy(), graph[l].hit.cpu().numpy(),
+                 graph[l].mpos.cpu().numpy())
+            ref = oracles[l].step(st.q[t], st.rope_pos[t], c.K, c.V, c.block_table, st.seq_lens[t])
+            np.testing.assert_array_equal(y[2], ref.hit, err_msg="hit mask, layer %d step %d" % (l, t))
+            np.testing.assert_array_equal(y[3], ref.match_pos, err_msg="match position, layer %d step %d" % (l, t))
+            assert float(np.abs(y[0] - ref.out).max()) <= OUT_TOL, "out, layer %d step %d" % (l, t)
+            assert float(np.abs(y[1] - ref.lse).max()) <= LSE_TOL, "lse, layer %d step %d" % (l, t)
+            x = eager[l].step(st.q[t], st.rope_pos[t], st.seq_lens[t])
+            for u, v in zip(x, y):
+                np.testing.assert_array_equal(u, v, err_msg="graph vs eager, layer %d step %d" % (l, t))
+            hits += int(ref.hit.sum())
+    assert hits > 0
+    assert all(r.st.get_status() == 0 for r in graph + eager)
 
 
 @pytest.mark.parametrize("opts", [{}, {"per_head": 1, "ring_bf16": 1}])
