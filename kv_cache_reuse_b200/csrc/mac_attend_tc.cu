@@ -43,8 +43,11 @@ namespace {
 // (merge_unit).
 namespace tc {
 constexpr int kKeys = 128;     // keys per tile: M of QK, K of PV
-constexpr int kSoftWarp0 = 4;  // softmax warps 4..11: warp w reads TMEM lanes 32 (w % 4) ..
-constexpr int kThreads = 12 * 32;
+constexpr int kSoftWarp0 = 4;  // softmax warps from 4 on: warp w reads TMEM lanes 32 (w % 4) ..
+// Softmax warps: four per TMEM lane quadrant for groups of 64 heads (16 heads
+// each), two for smaller groups.
+__host__ __device__ constexpr int soft_warps(int G) { return G >= 64 ? 16 : 8; }
+__host__ __device__ constexpr int threads(int G) { return (kSoftWarp0 + soft_warps(G)) * 32; }
 // Columns of S and of O: high parts and residuals of the G heads, at least 64.
 __host__ __device__ constexpr int ncols(int G) { return 2 * G < 64 ? 64 : 2 * G; }
 // Tiles in flight per ring and buffers of the weights P^T (shared memory:
@@ -105,18 +108,20 @@ __device__ __forceinline__ void umma_commit(unsigned long long* bar) {
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// Named barrier of the eight softmax warps, with an OR of one flag.
+// Named barrier of the NT softmax threads, with an OR of one flag.
+template <int NT>
 __device__ __forceinline__ int softmax_sync_or(int flag) {
   int out;
   asm volatile(
-      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, 256, pi;\n\t"
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.or.pred po, 1, %2, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(out)
-      : "r"(flag)
+      : "r"(flag), "n"(NT)
       : "memory");
   return out;
 }
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+template <int NT>
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); }
 
 // A CTA role's walk over its pieces, tile by tile.
 struct TileCursor {
@@ -259,8 +264,9 @@ __device__ __forceinline__ void tc_stream(const AttendParams& p, const CUtensorM
 }
 
 template <int GF>
-__global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __grid_constant__ AttendParams p) {
+__global__ void __launch_bounds__(tc::threads(GF), 1) mac_attend_tc_kernel(const __grid_constant__ AttendParams p) {
   constexpr int D = 128, G = GF, N = tc::ncols(G), SK = TcSmem<G>::SK, SV = TcSmem<G>::SV, NPB = TcSmem<G>::NPB;
+  constexpr int SW = tc::soft_warps(G), NT = SW * 32;  // softmax warps and threads
   static_assert(G == 16 || G == 32 || G == 64, "groups of 16, 32 or 64 heads");
   constexpr int GDc = 8 * D, PFc = GDc + 16;  // one 8-head chunk of a partial: o [8][D], m [8], l [8]
   constexpr uint32_t kCols = tc::tmem_cols(G), kColO = 2 * N;  // S[0] at 0, S[1] at N, O at 2N
@@ -284,13 +290,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
     }
     for (int s_ = 0; s_ < 2; ++s_) {
       mbar_init(&sm.s_full[s_], 1);
-      mbar_init(&sm.s_empty[s_], 8);
+      mbar_init(&sm.s_empty[s_], SW);
     }
     for (int s_ = 0; s_ < NPB; ++s_) {
-      mbar_init(&sm.p_full[s_], 8);
+      mbar_init(&sm.p_full[s_], SW);
       mbar_init(&sm.p_empty[s_], 1);
     }
-    mbar_init(&sm.q_full, 8);
+    mbar_init(&sm.q_full, SW);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -424,9 +430,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
   } else if (warp >= tc::kSoftWarp0) {
     // ---- softmax warps: warp 4 + 4 hh + wq owns TMEM lanes 32 wq .. 32 wq + 31
     // (the tile's keys) and heads [hh GH, hh GH + GH)
-    constexpr int GH = G / 2;
+    constexpr int GH = G / (SW / 4);
     const int sw = warp - tc::kSoftWarp0, wq = sw & 3, hh = sw >> 2;
-    const int ts = tid - tc::kSoftWarp0 * 32;  // 0 .. 255
+    const int ts = tid - tc::kSoftWarp0 * 32;  // 0 .. NT - 1
     const int k = 32 * wq + lane, hb = hh * GH;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * wq) << 16);
     if constexpr (2 * G < N) {
@@ -439,7 +445,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
             *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(sm.pw[pb][0]) + sw128_off(k, c * 8)) =
                 make_uint4(0u, 0u, 0u, 0u);
       }
-      for (int idx = ts; idx < 2 * (N - 2 * G); idx += 2 * 128) {
+      for (int idx = ts; idx < 2 * (N - 2 * G); idx += NT) {
         const int row = 2 * G + (idx >> 1), half = idx & 1;
         unsigned char* qd = reinterpret_cast<unsigned char*>(sm.q[half]);
 #pragma unroll
@@ -448,11 +454,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
     }
     // A failed wait flags the CTA's abort (every later wait then returns at
     // once) but the softmax warps still go through every tile and barrier of
-    // their walk, so the named barriers always see all 256 threads.
+    // their walk, so the named barriers always see all NT threads.
     bool ok = true;
-    // per head of this warp: key sums, this key's scores and (up to 16 heads)
-    // the running maxima; 32 heads read the maxima from shared memory
-    constexpr bool kMaxInRegs = GH <= 16;
+    // per head of this warp: key sums, this key's scores and (16 heads at most,
+    // 168 registers a thread) the running maxima; otherwise the maxima are read
+    // from shared memory
+    constexpr bool kMaxInRegs = GH <= 16 && SW == 8;
     float lsum[GH], sv[GH], mr[kMaxInRegs ? GH : 1];
 #pragma unroll
     for (int j = 0; j < (kMaxInRegs ? GH : 1); ++j) mr[j] = -INFINITY;
@@ -465,7 +472,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
       const Piece& pc = cur.pc;
       // the piece's query: rows [0, G) high parts, [G, 2G) residuals; the
       // previous piece's products are done (every S and O of it was read)
-      for (int idx = ts; idx < 4 * G; idx += 2 * 128) {
+      for (int idx = ts; idx < 4 * G; idx += NT) {
         const int row = idx >> 1, half = idx & 1, h = row < G ? row : row - G;
         const float* qsrc = p.qrot + ((size_t)pc.unit * G + h) * D + half * 64;
         unsigned char* qd = reinterpret_cast<unsigned char*>(sm.q[half]);
@@ -513,7 +520,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
         int grow = 0;
 #pragma unroll
         for (int j = 0; j < GH; ++j) grow |= sv[j] > mget(j) + 8.f ? 1 : 0;
-        if (softmax_sync_or(grow)) {
+        if (softmax_sync_or<NT>(grow)) {
           // some head's maximum grew: new maxima, O and the sums rescaled
 #pragma unroll
           for (int j = 0; j < GH; ++j) {
@@ -522,14 +529,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
             for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
             if (lane == 0) sm.red[wq][hb + j] = x;
           }
-          softmax_sync();
+          softmax_sync<NT>();
           if (ts < G) {
             const float mo = sm.m[ts];
             const float mn = fmaxf(mo, fmaxf(fmaxf(sm.red[0][ts], sm.red[1][ts]), fmaxf(sm.red[2][ts], sm.red[3][ts])));
             sm.red[0][ts] = mo == -INFINITY ? 0.f : ex2(mo - mn);  // scale of the old sums
             sm.m[ts] = mn;
           }
-          softmax_sync();
+          softmax_sync<NT>();
           if (i > 0) {
             // O holds the previous tile's product once that is done
             ok &= mbar_wait(&sm.p_empty[(t - 1) % NPB], (uint32_t)((t - 1) / NPB) & 1u, abort_flag, p.status);
@@ -551,7 +558,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
           for (int j = 0; j < GH; ++j) lsum[j] *= sm.red[0][hb + j];
 #pragma unroll
           for (int j = 0; j < (kMaxInRegs ? GH : 1); ++j) mr[j] = sm.m[hb + j];
-          softmax_sync();
+          softmax_sync<NT>();
         }
         // this key's weights into row k of P^T buffer t % NPB (free once the
         // product of tile t - NPB is done): high parts at column h, residuals
@@ -614,14 +621,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
         if (lane == 0) sm.red[wq][hb + j] = v;
       }
-      softmax_sync();
+      softmax_sync<NT>();
       if (ts < G) {
         float* dc = dst + (ts >> 3) * PFc;
         dc[GDc + (ts & 7)] = sm.m[ts];
         dc[GDc + 8 + (ts & 7)] = sm.red[0][ts] + sm.red[1][ts] + sm.red[2][ts] + sm.red[3][ts];
       }
       tc_fence_before();
-      softmax_sync();
+      softmax_sync<NT>();
     }
     (void)ok;
   }
@@ -642,52 +649,72 @@ __global__ void __launch_bounds__(tc::kThreads, 1) mac_attend_tc_kernel(const __
 }
 
 // Merge of the tcgen05 path's partials, one CTA per unit (blockIdx.x) and
-// 8-head chunk (blockIdx.y): warp w takes head w of the chunk and lane l its
-// elements 4l .. 4l + 3, and each warp folds every partial of its head --
-// segment A's and B's in one sequence, KB of them in flight per lane.
-// Segment A's partials with the reused state (on a hit) give the new prefix
-// state over [0, c_t), stored in ring slot dst; that state and segment B's
-// partials give the output.
+// pair of heads (blockIdx.y): warp w takes head w & 1 of the pair and every
+// fourth partial from w >> 1 on (segment A's and B's in one sequence, KB in
+// flight per lane), lane l the elements 4l .. 4l + 3; the four warps of a
+// head then combine their states through shared memory.  Segment A's
+// partials with the reused state (on a hit) give the new prefix state over
+// [0, c_t), stored in ring slot dst; that state and segment B's partials give
+// the output.
 template <int GF>
 __global__ void __launch_bounds__(kAttnThreads) mac_tc_merge_kernel(const __grid_constant__ AttendParams p) {
-  constexpr int D = 128, G = GF, PFc = 8 * D + 16, KB = 20;
+  constexpr int D = 128, G = GF, PFc = 8 * D + 16, KB = 10, NS = kAttnThreads / 64;  // NS warps per head
+  __shared__ float4 so[2][NS][2][32];  // [head][warp][A|B][lane]: o
+  __shared__ float sml[2][NS][2][2];   // [head][warp][A|B]: m, l
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int u = blockIdx.x, ch = blockIdx.y, hl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int u = blockIdx.x, hp = threadIdx.x >> 5 & 1, part = threadIdx.x >> 6, lane = threadIdx.x & 31;
   const UnitPlan* const pp = p.plan + u;
   if (__ldcg(&pp->bad)) return;
-  const int hit = __ldcg(&pp->hit), src = __ldcg(&pp->src_slot), dst = __ldcg(&pp->dst_slot), end = __ldcg(&pp->end);
   const Segment sA = load_segment(p.seg + 2 * u), sB = load_segment(p.seg + 2 * u + 1);
   const size_t PF = partial_floats(G, D);
-  const int h = ch * 8 + hl, d0 = lane * 4;
+  const int h = blockIdx.y * 2 + hp, ch = h >> 3, hl = h & 7, d0 = lane * 4;
   const int nA = sA.kind < 0 ? 0 : sA.npieces, nB = sB.kind < 0 ? 0 : sB.npieces;
-  const float* const baseA = p.part + (size_t)sA.pbase * PF + (size_t)ch * PFc + hl * D + d0;
-  const float* const baseB = p.part + (size_t)sB.pbase * PF + (size_t)ch * PFc + hl * D + d0;
+  const float* const baseA = p.part + (size_t)sA.pbase * PF + (size_t)ch * PFc;
+  const float* const baseB = p.part + (size_t)sB.pbase * PF + (size_t)ch * PFc;
   // segment A folds into (M, L, O), segment B into (MB, LB, OB)
   float M = -INFINITY, L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
   float MB = -INFINITY, LB = 0.f, OB[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-  for (int i0 = 0; i0 < nA + nB; i0 += KB) {
+  for (int i0 = part; i0 < nA + nB; i0 += KB * NS) {
     float4 ov[KB];
     float mv[KB], lv[KB];
 #pragma unroll
     for (int k = 0; k < KB; ++k) {
-      const int i = i0 + k;
+      const int i = i0 + k * NS;
       if (i < nA + nB) {
         const float* q = i < nA ? baseA + (size_t)i * PF : baseB + (size_t)(i - nA) * PF;
-        ov[k] = __ldcg(reinterpret_cast<const float4*>(q));
-        mv[k] = __ldcg(q - hl * D - d0 + 8 * D + hl);
-        lv[k] = __ldcg(q - hl * D - d0 + 8 * D + 8 + hl);
+        ov[k] = __ldcg(reinterpret_cast<const float4*>(q + hl * D + d0));
+        mv[k] = __ldcg(q + 8 * D + hl);
+        lv[k] = __ldcg(q + 8 * D + 8 + hl);
       }
     }
 #pragma unroll
     for (int k = 0; k < KB; ++k) {
-      const int i = i0 + k;
+      const int i = i0 + k * NS;
       if (i < nA)
         fold_state<4>(M, L, O, mv[k], lv[k], &ov[k].x);
       else if (i < nA + nB)
         fold_state<4>(MB, LB, OB, mv[k], lv[k], &ov[k].x);
     }
   }
+  so[hp][part][0][lane] = make_float4(O[0], O[1], O[2], O[3]);
+  so[hp][part][1][lane] = make_float4(OB[0], OB[1], OB[2], OB[3]);
+  if (lane == 0) {
+    sml[hp][part][0][0] = M;
+    sml[hp][part][0][1] = L;
+    sml[hp][part][1][0] = MB;
+    sml[hp][part][1][1] = LB;
+  }
+  __syncthreads();
+  if (part != 0) return;
+  // warps 0 and 1: the head's four states, in warp order
+#pragma unroll
+  for (int w = 1; w < NS; ++w) {
+    float4 a = so[hp][w][0][lane], c = so[hp][w][1][lane];
+    fold_state<4>(M, L, O, sml[hp][w][0][0], sml[hp][w][0][1], &a.x);
+    fold_state<4>(MB, LB, OB, sml[hp][w][1][0], sml[hp][w][1][1], &c.x);
+  }
+  const int hit = __ldcg(&pp->hit), src = __ldcg(&pp->src_slot), dst = __ldcg(&pp->dst_slot), end = __ldcg(&pp->end);
   // new prefix state: segment A, plus the reused state on a hit
   const size_t Wp1 = (size_t)p.W + 1;
   if (hit) {
@@ -721,7 +748,7 @@ __global__ void __launch_bounds__(kAttnThreads) mac_tc_merge_kernel(const __grid
   o4.w = __fdividef(O[3] * a0 + OB[3] * aB, L2);
   *reinterpret_cast<float4*>(p.out + orow * D + d0) = o4;
   if (lane == 0) p.lse[orow] = (M2 + __log2f(L2)) * kLn2;
-  if (ch == 0 && threadIdx.x == 0) {
+  if (blockIdx.y == 0 && threadIdx.x == 0) {
     p.ring_pos[(size_t)u * Wp1 + dst] = end - 1;
     if (p.counters != nullptr) atomicAdd(p.counters + kCountMerged, 1ull);
   }
@@ -742,12 +769,12 @@ cudaError_t tc_prepare() {
 template <int GF>
 cudaError_t tc_launch(cudaLaunchConfig_t& cfg, const AttendParams& p, int U, cudaStream_t s) {
   cfg.dynamicSmemBytes = tc_smem_bytes<GF>();
-  cfg.blockDim = dim3(tc::kThreads);
+  cfg.blockDim = dim3(tc::threads(GF));
   cudaError_t e = cudaLaunchKernelEx(&cfg, mac_attend_tc_kernel<GF>, p);
   cfg.blockDim = dim3(kAttnThreads);
   if (e != cudaSuccess) return e;
   // the merge may start while the products drain (it waits on them first)
-  cfg.gridDim = dim3(U, GF / 8);
+  cfg.gridDim = dim3(U, GF / 2);
   cfg.dynamicSmemBytes = 0;
   return cudaLaunchKernelEx(&cfg, mac_tc_merge_kernel<GF>, p);
 }
