@@ -41,13 +41,22 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_kernel(const MatchPar
 }
 
 
+// Groups of window slots each chunk's scan is split into (16-64-head groups):
+// as many as the SMs allow, up to 4, with `ctas` = units x chunks.
+__host__ __device__ inline int wide_slot_groups(int ctas, int grid) {
+  const int s = ctas > 0 ? grid / ctas : 1;
+  return s < 1 ? 1 : (s > 4 ? 4 : s);
+}
+
 // Groups of 16, 32 or 64 query heads per KV head (multi-query attention):
-// NC = G / 8 CTAs per unit, CTA (u, c) holding the heads [8c, 8c + 8).  Each
-// sums, for every window entry, the squared L2 distance of its heads to the
-// entry's (the window scan is spread over NC SMs instead of one), stores the
-// part in dpart, rotates its heads' queries and writes them to the step's
-// ring slot.  The last of the unit's NC CTAs to arrive (atomic ticket, nobody
-// waits) adds the NC parts of each entry in chunk order -- the mean over the
+// NC = G / 8 chunks per unit, each split into S groups of window slots when
+// the SMs allow (wide_slot_groups), CTA (u, c, g) holding the heads
+// [8c, 8c + 8) and the slots of group g.  Each sums, for every window entry
+// of its group, the squared L2 distance of its heads to the entry's (the
+// window scan is spread over NC S SMs instead of one) and stores the part in
+// dpart; group 0 rotates the chunk's queries and writes them to the step's
+// ring slot.  The last of the unit's NC S CTAs to arrive (atomic ticket,
+// nobody waits) adds the NC parts of each entry in chunk order -- the mean over the
 // G heads -- and takes the decision exactly as the 8-head kernel does
 // (argmin, ties to the larger position, then the newer entry; strict
 // threshold; NaN never hits), then writes the plan; the last unit decided
@@ -66,8 +75,8 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_wide_kernel(const Mat
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const double cw_c = (p.cw != nullptr && (int)threadIdx.x <= p.grid) ? __ldcg(p.cw + threadIdx.x) : 0.0;
-  const int G = p.G, NC = G / GP;
-  const int u = blockIdx.x / NC, c = blockIdx.x - u * NC;
+  const int G = p.G, NC = G / GP, S = wide_slot_groups(p.B * p.Hkv * NC, p.grid);
+  const int u = blockIdx.x / (NC * S), cs = blockIdx.x - u * NC * S, c = cs / S, sg = cs - c * S;
   const int b = u / p.Hkv, kvh = u - b * p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Wp1 = p.W + 1;
@@ -75,19 +84,21 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_wide_kernel(const Mat
   constexpr int BS = 3;                 // slots per warp per batch of loads
   constexpr int F4 = GDc / 4 / 32;      // float4 per lane per slot
   constexpr int n4 = GDc / 4;
+  // this CTA's slots: group sg of S
+  const int per = (Wp1 + S - 1) / S, sl0 = sg * per, sl1 = sl0 + per < Wp1 ? sl0 + per : Wp1;
   RT r[BS][F4];
   auto load_batch = [&](int s0) {
 #pragma unroll
     for (int k = 0; k < BS; ++k) {
       const int slot = s0 + k * NW;
-      if (slot < Wp1) {
+      if (slot < sl1) {
         const RT* rq = reinterpret_cast<const RT*>(p.ring_q) + (((size_t)u * Wp1 + slot) * G + (size_t)c * GP) * D / 4;
 #pragma unroll
         for (int f = 0; f < F4; ++f) r[k][f] = rq[lane + 32 * f];
       }
     }
   };
-  load_batch(warp);
+  load_batch(sl0 + warp);
   const size_t q0 = ((size_t)b * p.Hq + (size_t)kvh * G + (size_t)c * GP) * D / 4;  // this chunk's heads
   if (p.q_bf16) {
     const uint2* qsrc = reinterpret_cast<const uint2*>(p.q_pre) + q0;
@@ -107,12 +118,12 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_wide_kernel(const Mat
 
   // 1. this chunk's part of every occupied entry's distance: sum over its 8
   // heads of sum((q - q_s)^2), in fp32 (the difference form)
-  for (int s0 = warp; s0 < Wp1; s0 += BS * NW) {
-    if (s0 != warp) load_batch(s0);
+  for (int s0 = sl0 + warp; s0 < sl1; s0 += BS * NW) {
+    if (s0 != sl0 + warp) load_batch(s0);
 #pragma unroll
     for (int k = 0; k < BS; ++k) {
       const int slot = s0 + k * NW;
-      if (slot < Wp1) {
+      if (slot < sl1) {
         const int j = (((n - 1 - slot) % Wp1) + Wp1) % Wp1;
         if (j < occ) {
           float acc = 0.f;
@@ -132,8 +143,9 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_wide_kernel(const Mat
     }
   }
   // 2. rotate this chunk's heads (pair i = tid) and record them in the step's
-  // ring slot (outside the window this step; skipped for an invalid length)
-  {
+  // ring slot (outside the window this step; skipped for an invalid length);
+  // the chunk's first slot group does it
+  if (sg == 0) {
     const double scale = kLog2eD / sqrt((double)D);
     for (int i = tid; i < D / 2; i += kMatchThreads) {
       for (int h = 0; h < GP; ++h) {
@@ -160,7 +172,7 @@ __global__ void __launch_bounds__(kMatchThreads) mac_match_wide_kernel(const Mat
   if (tid == 0) {
     int ticket;
     asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(p.ucnt + u) : "memory");
-    s_decider = (ticket == NC - 1);
+    s_decider = (ticket == NC * S - 1);
     if (s_decider) p.ucnt[u] = 0;
     s_bad_page = 0;
   }
@@ -283,7 +295,7 @@ void launch_dr(const MatchParams& p, int U, cudaStream_t s) {
 template <int D>
 void launch_d(const MatchParams& p, int U, cudaStream_t s) {
   if (p.G > kMaxGroup) {  // 16, 32 or 64 heads: G / 8 CTAs per unit
-    const int grid = U * group_chunks(p.G);
+    const int NC = group_chunks(p.G), grid = U * NC * wide_slot_groups(U * NC, p.grid);
     if (p.ring_bf16)
       mac_match_wide_kernel<D, true><<<grid, kMatchThreads, 0, s>>>(p);
     else
