@@ -142,7 +142,7 @@ struct TileCursor {
   }
 };
 
-// n consecutive fp32 columns (n = 8, 16, 32) of this warp's 32 TMEM lanes,
+// n consecutive fp32 columns (n = 8, 16) of this warp's 32 TMEM lanes,
 // issued without waiting (tmem_ld_wait completes them), and stored back.
 template <int NCOL>
 __device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t* r);
@@ -170,48 +170,23 @@ __device__ __forceinline__ void tmem_stn<16>(uint32_t taddr, const uint32_t* r) 
   asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
                : "memory");
 }
-template <>
-__device__ __forceinline__ void tmem_ldn<32>(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-               : "r"(taddr));
-}
-template <>
-__device__ __forceinline__ void tmem_stn<32>(uint32_t taddr, const uint32_t* r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-               : "memory");
-}
-// Completes every TMEM load issued so far and ties the registers to that
-// point.
 template <int NR>
 __device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int j = 0; j < NR; ++j) asm volatile("" : "+r"(r[j]));
 }
-// Values of GH heads of this thread's TMEM lane: the high-part columns at
-// `hi` plus the residual columns at `res` (32 heads: one half after the
-// other, to bound the registers in flight).
+// Values of GH heads (8 or 16) of this thread's TMEM lane: the high-part
+// columns at `hi` plus the residual columns at `res`.
 template <int GH>
 __device__ __forceinline__ void tmem_heads(uint32_t hi, uint32_t res, float* v) {
-  if constexpr (GH <= 16) {
-    uint32_t r[2 * GH];
-    tmem_ldn<GH>(hi, r);
-    tmem_ldn<GH>(res, r + GH);
-    tmem_ld_wait<2 * GH>(r);
+  static_assert(GH == 8 || GH == 16, "a softmax warp owns 8 or 16 heads");
+  uint32_t r[2 * GH];
+  tmem_ldn<GH>(hi, r);
+  tmem_ldn<GH>(res, r + GH);
+  tmem_ld_wait<2 * GH>(r);
 #pragma unroll
-    for (int j = 0; j < GH; ++j) v[j] = __uint_as_float(r[j]) + __uint_as_float(r[GH + j]);
-  } else {
-    uint32_t r[GH];
-    tmem_ldn<GH>(hi, r);
-    tmem_ld_wait<GH>(r);
-#pragma unroll
-    for (int j = 0; j < GH; ++j) v[j] = __uint_as_float(r[j]);
-    tmem_ldn<GH>(res, r);
-    tmem_ld_wait<GH>(r);
-#pragma unroll
-    for (int j = 0; j < GH; ++j) v[j] += __uint_as_float(r[j]);
-  }
+  for (int j = 0; j < GH; ++j) v[j] = __uint_as_float(r[j]) + __uint_as_float(r[GH + j]);
 }
 
 // One ring of K or V tiles: boxes of 16 keys x 64 dims (two per key row of
