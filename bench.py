@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import re
 import sys
@@ -443,6 +444,11 @@ def run_mac(args, rank, world, local_rank):
                           "mb_per_launch": r["match_bytes"] / n / 1e6, "us_per_launch": r["match_ms"] * 1e3 / n},
                 "step_us": r["total_ms"] * 1e3 / n}
 
+    def brief(t):
+        """A two-launch record as it goes on the one JSON line (the full one on stderr)."""
+        return {"attend_frac": t["attend"]["frac"], "attend_us": t["attend"]["us_per_launch"],
+                "match_us": t["match"]["us_per_launch"], "step_us": t["step_us"]}
+
     def step_roof(r, n):
         """The step as it runs: one launch (match, whole units, split ranges) or two."""
         nbytes = r["att_bytes"] + r["match_bytes"]
@@ -461,41 +467,41 @@ def run_mac(args, rank, world, local_rank):
             "bytes_per_launch": (main["att_bytes"] + main["match_bytes"]) / K_,
             "us_per_launch": main["total_ms"] * 1e3 / K_,
             "by_class": main["by_class"],
-            "two_launch": dict(two_launch(kern, K_), steps_per_s=K_ / (main2["total_ms"] * 1e-3),
+            "two_launch": dict(brief(two_launch(kern, K_)), steps_per_s=K_ / (main2["total_ms"] * 1e-3),
                                step_us_back_to_back=main2["total_ms"] * 1e3 / K_, by_class=main2["by_class"])}
-    detail = {}
+    detail = {"two_launch": two_launch(kern, K_)}
     if allmiss:
         n = len(allmiss["step_ms"])
         roof["miss"] = dict(step_roof(allmiss, n),
                             workload="%s, threshold 0 (every unit misses)" % wl.name,
                             steps_per_s=n / (allmiss["total_ms"] * 1e-3),
-                            two_launch=two_launch(allmiss2, n))
-        detail["all_miss"] = {"steps": n, "ms_per_step": allmiss["total_ms"] / n,
+                            two_launch=brief(two_launch(allmiss2, n)))
+        detail["all_miss"] = {"steps": n, "ms_per_step": allmiss["total_ms"] / n, "two_launch": two_launch(allmiss2, n),
                               "speedup_of_mac": (world * K_ / (tot * 1e-3)) / (n / (allmiss["total_ms"] * 1e-3)),
                               "clocks": allmiss["clocks"]}
     if hitrun:
         n = len(hitrun["step_ms"])
         roof["hit"] = dict(step_roof(hitrun, n), workload="%s, every step a repeat" % wl.name,
-                           hit_fraction=hitrun["hit_frac"], two_launch=two_launch(hitrun2, n),
-                           larger=[{"workload": h["workload"], "step_us": h["step"]["us"], "step_mb": h["step"]["mb"],
-                                    "step_frac": h["step"]["frac"], "kernel": h["step"]["kernel"]}
-                                   for h in hitshapes])
-        detail["hit_path"] = {"steps": n, "clocks": hitrun["clocks"], "shapes": hitshapes}
+                           hit_fraction=hitrun["hit_frac"], two_launch=brief(two_launch(hitrun2, n)),
+                           larger={h["workload"].split(" ")[0]: {"step_us": h["step"]["us"], "step_frac": h["step"]["frac"]}
+                                   for h in hitshapes})
+        detail["hit_path"] = {"steps": n, "clocks": hitrun["clocks"], "shapes": hitshapes,
+                              "two_launch": two_launch(hitrun2, n)}
         if hitctx:
-            roof["hit"]["vs_context"] = [
+            # step time of the same all-hit stream against the context length (the same MB per step)
+            roof["hit"]["us_vs_context"] = {str(L): r["total_ms"] * 1e3 / len(r["step_ms"]) for L, r in hitctx}
+            detail["hit_path"]["vs_context"] = [
                 {"context": L, "step_us": r["total_ms"] * 1e3 / len(r["step_ms"]),
                  "step_mb": (r["att_bytes"] + r["match_bytes"]) / len(r["step_ms"]) / 1e6} for L, r in hitctx]
     if paged_gap:
-        roof.setdefault("miss", {})["paged_vs_contiguous"] = {
-            "workload": "paged_mixed shape, threshold 0 (every unit misses)",
+        roof.setdefault("miss", {})["paged_vs_contiguous"] = {  # the paged_mixed shape, every unit missing
             "paged_frac": paged_gap["paged"]["step"]["frac"], "contiguous_frac": paged_gap["contiguous"]["step"]["frac"],
             "paged_attend_frac": paged_gap["paged"]["attend"]["frac"],
             "contiguous_attend_frac": paged_gap["contiguous"]["attend"]["frac"]}
         detail["paged_vs_contiguous"] = paged_gap
     if mqa:
         a = mqa["all_miss"]["attend"]
-        roof.setdefault("miss", {})["mqa_32_1"] = {"frac": a["frac"], "achieved": a["achieved"], "mb_per_launch": a["mb_per_launch"],
-                                    "us_per_launch": a["us_per_launch"]}
+        roof.setdefault("miss", {})["mqa_32_1"] = {"frac": a["frac"], "us_per_launch": a["us_per_launch"]}
         detail["mqa_32_1"] = mqa
     res = {
         "metric": METRIC, "value": world * K_ / (tot * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K_,
@@ -979,7 +985,19 @@ def main():
         if isinstance(res, tuple):
             res, detail = res
             print(json.dumps(dict(detail, metric=res["metric"], value=res["value"])), file=sys.stderr, flush=True)
-        print(json.dumps(res), flush=True)
+        print(json.dumps(_compact(res)), flush=True)
+
+
+def _compact(x, digits=5):
+    """The result with every float rounded to `digits` significant digits
+    (keeps the one JSON line short; the full-precision record is on stderr)."""
+    if isinstance(x, float):
+        return float("%.*g" % (digits, x)) if math.isfinite(x) else x
+    if isinstance(x, dict):
+        return {k: _compact(v, digits) for k, v in x.items()}
+    if isinstance(x, (list, tuple)):
+        return [_compact(v, digits) for v in x]
+    return x
 
 
 if __name__ == "__main__":
