@@ -279,6 +279,9 @@ __global__ void __launch_bounds__(tc::threads(GF), 1) mac_attend_tc_kernel(const
   }
   __syncthreads();
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the merge may be scheduled now: its CTAs take SMs as these CTAs leave,
+  // and wait for this grid to complete before they read any partial
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // the CTA's range of the cost space (as in the attention kernel)
   unsigned smid;
   asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
