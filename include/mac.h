@@ -19,8 +19,10 @@
  *     (multi-head attention) to 8, or 16, 32 or 64 (multi-query attention
  *     sized groups, e.g. 32 query heads over one KV head); other sizes return
  *     MAC_ERR_SHAPE.  One match decision is taken per (sequence, KV head)
- *     over its G heads.  Groups of 16-64 heads are processed as chunks of 8
- *     that read each K/V row from memory once for the whole group; they take
+ *     over its G heads.  Groups of 16-64 heads read each K/V row from memory
+ *     once for the whole group: at head_dim 128 the group is one tensor-core
+ *     tile (tcgen05 products with tensor-memory accumulators, then a merge
+ *     launch), at head_dim 64 chunks of 8 heads share every box.  They take
  *     no per-head matching, and every key range runs through partial
  *     results (the whole-unit setting does not apply to them).
  *   - Distance: mean over the G heads of the squared L2 distance between the
