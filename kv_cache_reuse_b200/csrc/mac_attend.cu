@@ -23,7 +23,7 @@
 // Per CTA: eight warps; warp w owns boxes w, w+8, w+16, ... of every piece,
 // where a box is 16 keys (it never crosses a page).  Each warp streams its
 // own boxes through its own ring of shared-memory slots with TMA
-// (cp.async.bulk.tensor, 128-byte swizzle, no multicast), keeping NST boxes
+// (cp.async.bulk.tensor, 128-byte swizzle, each CTA its own copies), keeping NST boxes
 // in flight, so the warps never wait on one another inside a piece.
 //
 // A box is a small dense product on the tensor cores (mma.sync m16n8k16,
