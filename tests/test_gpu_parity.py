@@ -502,6 +502,17 @@ def test_mqa_export_matches_oracle_window():
     np.testing.assert_allclose(st["m"][0, slots] + np.log(st["l"][0, slots]), m + np.log(l), atol=LSE_TOL)
 
 
+@pytest.mark.parametrize("G,B,L0,band", [(16, 3, (40, 130, 300), 64), (64, 2, (100, 700), 600), (32, 2, (127, 129), 16)])
+def test_mqa_tensor_memory_edges(G, B, L0, band):
+    """The tensor-memory path (head dim 128) at its edges: sequences shorter
+    than one 128-key tile or just across it, bands that reach key 0 (empty
+    reused prefix, empty amend range), pieces that start and end inside a
+    tile -- decisions bit-exact and outputs within tolerance at every step."""
+    wl = synth.WORKLOADS["llama8b_32k"].with_(B=B, Hq=G, Hkv=1, L0=L0, band=band, steps=20)
+    r = compare_stream(wl, synth.queries(wl), synth.kv_cache(wl))
+    assert r["hits"] > 0
+
+
 def test_mqa_steps_repeat_bit_for_bit():
     """The tensor-memory path of a 32-head group on large all-miss steps (a
     single KV head's keys cut over every CTA) and on the repeats after them:
