@@ -34,13 +34,14 @@ namespace {
 // Warp 0 streams the K tiles and warp 2 the V tiles (16-key TMA boxes, each
 // ring with its own barriers, so a K buffer returns to the stream as soon as
 // its product is done), one thread of warp 1 issues the MMAs as their inputs
-// arrive (S double-buffered in TMEM, O in TMEM), warps 4-7 run the softmax:
-// thread k owns key k of the tile (TMEM lane k) and keeps its keys' running
-// sums per head in registers; O is rescaled only when some head's maximum
-// grows by more than 2^8 (weights stay below 256).  Every piece (a unit's keys
-// in this CTA's range) ends in a partial in the chunk-major layout, and a
-// second kernel merges each unit's partials with its reused state
-// (merge_unit).
+// arrive (S double-buffered in TMEM, O in TMEM), and the softmax warps from 4
+// on (two per TMEM lane quadrant, four for groups of 64) each own a share of
+// the heads for the 32 keys of their lanes: a thread holds one key's scores
+// and its keys' running sums per head in registers; O is rescaled only when
+// some head's maximum grows by more than 2^8 (weights stay below 256).  Every
+// piece (a unit's keys in this CTA's range) ends in a partial in the
+// chunk-major layout, and a second kernel (mac_tc_merge_kernel) merges each
+// unit's partials with its reused state.
 namespace tc {
 constexpr int kKeys = 128;     // keys per tile: M of QK, K of PV
 constexpr int kSoftWarp0 = 4;  // softmax warps from 4 on: warp w reads TMEM lanes 32 (w % 4) ..
