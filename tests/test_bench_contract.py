@@ -100,3 +100,15 @@ def test_roofline_key_bytes_agree_with_the_oracles_key_count(per_head):
         assert kv == r.keys_read * 2 * wl.D * 2, t
         hits += int(r.hit.sum())
     assert 0 < hits < wl.steps * r.hit.size
+
+
+def test_compact_line_keeps_five_significant_digits():
+    """The one JSON line rounds floats to five significant digits (the full
+    record goes to stderr) and leaves every other value as it is."""
+    import bench
+    rec = {"value": 14396.609269749571, "frac": 0.6022880969335624, "n": 20, "ok": True, "none": None,
+           "nested": {"us": [20.285333041101694, 143.22400093078613], "name": "x"}, "inf": float("inf")}
+    out = bench._compact(rec)
+    assert out["value"] == 14397.0 and out["frac"] == 0.60229 and out["n"] == 20 and out["ok"] is True
+    assert out["none"] is None and out["nested"]["name"] == "x" and out["inf"] == float("inf")
+    assert out["nested"]["us"] == [20.285, 143.22]
