@@ -10,6 +10,8 @@
 
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "mac_internal.cuh"
 
 #include "../../include/mac.h"
@@ -82,6 +84,15 @@ struct MacState {
 };
 
 namespace {
+
+// A profiler range (NVTX) over an entry point or a host-side stage of one;
+// without a profiler attached the calls do nothing.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -436,6 +447,7 @@ static int match_impl(MacState* s, float tau, const void* q_pre, const int* rope
 
 int mac_match(MacState* s, const void* q_pre, const int* rope_pos, const int* block_table, const int* seq_lens,
               float* out, float* lse, uint8_t* hit_mask, int* match_pos, void* stream) {
+  Range r("mac_match");
   if (!s) return MAC_ERR_ARG;
   return match_impl(s, s->cfg.tau, q_pre, rope_pos, block_table, seq_lens, out, lse, hit_mask, match_pos, stream);
 }
@@ -569,6 +581,7 @@ static int clear_trace(MacState* s, cudaStream_t st) {
 
 int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* block_table, float* out, float* lse,
                void* stream) {
+  Range r("mac_attend");
   AttendParams p;
   int rc = fill_attend(s, K, V, block_table, out, lse, p);
   if (rc == MAC_OK) rc = clear_trace(s, (cudaStream_t)stream);
@@ -579,6 +592,7 @@ int mac_attend(MacState* s, const uint16_t* K, const uint16_t* V, const int* blo
 int mac_decode_step(MacState* s, const void* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
                     const int* block_table, const int* seq_lens, float* out, float* lse, uint8_t* hit_mask,
                     int* match_pos, void* stream) {
+  Range r("mac_decode_step");
   if (!s || !K || !V) return MAC_ERR_ARG;
   if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
   if (s->one_launch && s->one_launch_ok) {
@@ -598,6 +612,7 @@ int mac_decode_step(MacState* s, const void* q_pre, const int* rope_pos, const u
 
 int mac_append_kv(MacState* s, uint16_t* K, uint16_t* V, const int* block_table, const int* seq_lens,
                   const uint16_t* k_new, const uint16_t* v_new, void* stream) {
+  Range r("mac_append_kv");
   if (!s || !K || !V || !seq_lens || !k_new || !v_new) return MAC_ERR_ARG;
   if (!aligned16(K) || !aligned16(V) || !aligned16(k_new) || !aligned16(v_new)) return MAC_ERR_ARG;
   if (s->cfg.page_size > 0 && !block_table) return MAC_ERR_ARG;
@@ -621,6 +636,7 @@ int mac_append_kv(MacState* s, uint16_t* K, uint16_t* V, const int* block_table,
 
 int mac_warm_start(MacState* s, int n, const void* q_pre, const int* rope_pos, const uint16_t* K, const uint16_t* V,
                    const int* block_table, const int* seq_lens, void* stream) {
+  Range r("mac_warm_start");
   if (!s || n < 0 || n > s->W) return MAC_ERR_ARG;
   if (n > 0 && (!q_pre || !rope_pos || !seq_lens || !K || !V)) return MAC_ERR_ARG;
   if (n > 0 && (!aligned16(q_pre) || !aligned16(K) || !aligned16(V))) return MAC_ERR_ARG;
@@ -670,6 +686,7 @@ int mac_decode_step_host(MacState* s, const void* q_pre_h, const int* rope_pos_h
                          const uint16_t* k_new_h, const uint16_t* v_new_h, uint16_t* K, uint16_t* V,
                          const int* block_table, float* out_h, float* lse_h, uint8_t* hit_h, int* match_pos_h,
                          void* stream) {
+  Range r("mac_decode_step_host");
   if (!s || !q_pre_h || !rope_pos_h || !seq_lens_h || !K || !V) return MAC_ERR_ARG;
   if ((k_new_h == nullptr) != (v_new_h == nullptr)) return MAC_ERR_ARG;
   if (!aligned16(K) || !aligned16(V)) return MAC_ERR_ARG;
@@ -711,7 +728,10 @@ int mac_decode_step_host(MacState* s, const void* q_pre_h, const int* rope_pos_h
     const int rc = enqueue_host_step(s, K, V, bt, append, st);  // no graph: the same work, launched directly
     if (rc != MAC_OK) return rc;
   }
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MAC_ERR_CUDA;
+  {
+    Range w("wait for the step");
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MAC_ERR_CUDA;
+  }
   if (out_h) memcpy(out_h, s->host_out + s->off_out, B * Hq * D * sizeof(float));
   if (lse_h) memcpy(lse_h, s->host_out + s->off_lse, B * Hq * sizeof(float));
   if (hit_h) memcpy(hit_h, s->host_out + s->off_hit, U * s->ND);
